@@ -1,0 +1,540 @@
+"""Pins for the CPU oracle, independent of the oracle itself (CPU only).
+
+Each test checks the oracle against something other than its own formulas:
+a library routine (torch's bfloat16 cast, numpy QR/SVD), exact rational
+arithmetic (fractions), brute force over all candidates, a closed form, a
+published test vector, or an invariant of the recurrence.  Source of the
+method: "Accelerating Parallel Diffusion Model Serving with Residual
+Compression" -- overall framework, key design (residual compression, error
+feedback, low-rank strategy) and limitations (first step sent in full).
+"""
+import itertools
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16_torch(x):
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _f32_of_bf16(h):
+    return (np.asarray(h, dtype=np.uint32) << 16).view(np.float32)
+
+
+def _ulp32(x):
+    x = np.abs(np.asarray(x, dtype=np.float32))
+    return np.spacing(x)
+
+
+# ------------------------------------------------------------------ bf16 / rng
+
+def test_bf16_matches_library_cast(orc):
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal(200000).astype(np.float32) * np.float32(10.0) ** rng.integers(-30, 30, 200000)
+    x = x.astype(np.float32)
+    # every tie pattern and both neighbours of it, over a spread of exponents
+    base = rng.integers(0, 2 ** 31, 20000, dtype=np.uint64).astype(np.uint32) & np.uint32(0x7fff0000)
+    ties = np.concatenate([base | np.uint32(0x8000), base | np.uint32(0x7fff), base | np.uint32(0x8001),
+                           base | np.uint32(0x18000)]).view(np.float32)
+    specials = np.array([0.0, -0.0, 1.0, -1.0, 3.3895314e38, -3.3895314e38, 1e-45, -1e-45, 1.1754944e-38,
+                         np.inf, -np.inf], dtype=np.float32)
+    allx = np.concatenate([x, ties, -ties, specials]).astype(np.float32)
+    allx = allx[np.isfinite(allx) | np.isinf(allx)]
+    got = orc.bf16_from_f32(allx)
+    want = _bf16_torch(allx)
+    assert np.array_equal(got, want)
+
+
+def test_splitmix64_published_vector(orc):
+    vals = [int(l) for l in open(os.path.join(GOLDEN, "splitmix64_rosetta.txt")) if l.strip() and l[0] != "#"]
+    gamma = 0x9E3779B97F4A7C15
+    for n, want in enumerate(vals):
+        assert orc.splitmix64((1234567 + n * gamma) % 2 ** 64) == want
+
+
+def test_lr_v0_range_and_exactness(orc):
+    V = orc.lr_v0(42, 64, 5)
+    assert V.min() >= -1.0 and V.max() < 1.0
+    # values are k * 2^-23 - 1 for an integer k: exact in fp32
+    k = (V.astype(np.float64) + 1.0) * 2 ** 23
+    assert np.array_equal(k, np.round(k))
+    assert abs(float(V.mean())) < 0.1 and 0.25 < float(V.var()) < 0.42  # U[-1,1): var 1/3
+
+
+# ------------------------------------------------------------------ SIGN1
+
+def _exact_mean_abs(d):
+    s = sum(Fraction(float(abs(v))) for v in d)
+    return s / len(d)
+
+
+def _round_fraction_to_f32(q: Fraction) -> float:
+    """Correctly rounded (nearest-even) fp32 of an exact rational q >= 0."""
+    if q == 0:
+        return 0.0
+    f = np.float32(float(q))  # float(q) is correctly rounded to fp64; refine to fp32 exactly below
+    lo = np.nextafter(f, np.float32(0))
+    hi = np.nextafter(f, np.float32(np.inf))
+    cands = [lo, f, hi]
+    best = min(cands, key=lambda c: (abs(Fraction(float(c)) - q), int(np.array(c).view(np.uint32)) & 1))
+    return float(best)
+
+
+def test_sign1_scale_is_rounded_exact_mean(orc):
+    """The fixed-point mean equals the exact mean after fp32/bf16 rounding."""
+    rng = np.random.default_rng(1)
+    n_checked = 0
+    for trial in range(300):
+        n = int(rng.choice([32, 64, 96, 1920, 3072]))
+        scale = 10.0 ** rng.uniform(-6, 3)
+        d = (rng.standard_normal(n) * scale).astype(np.float32)
+        if trial % 7 == 0:
+            d[rng.integers(0, n, n // 3)] = 0.0
+        if trial % 11 == 0:
+            d[0] = np.float32(scale * 1e4)      # one outlier: mean << max
+        q = _exact_mean_abs(d)
+        f32 = _round_fraction_to_f32(q)
+        want = int(_bf16_torch(np.array([f32], dtype=np.float32))[0])
+        got = orc.sign1_scale(d)
+        if got != want:
+            # allowed only when the exact mean sits within the fixed-point error of an fp32 rounding boundary
+            rel = abs(Fraction(f32) - q) / q
+            assert rel > Fraction(1, 2 ** 25), (trial, got, want)
+        else:
+            n_checked += 1
+    assert n_checked >= 295
+
+
+def test_sign1_scale_zero_and_denormal(orc):
+    assert orc.sign1_scale(np.zeros(64, np.float32)) == 0
+    assert orc.sign1_scale(-np.zeros(64, np.float32)) == 0
+    d = np.zeros(64, np.float32)
+    d[3] = np.float32(1e-45)  # smallest denormal
+    q = Fraction(float(d[3])) / 64
+    want = int(_bf16_torch(np.array([_round_fraction_to_f32(q)], np.float32))[0])
+    assert orc.sign1_scale(d) == want
+
+
+def test_sign1_scale_is_l2_optimal(orc):
+    """argmin_s sum (d - s sgn d)^2 = mean|d|: the chosen bf16 scale is the best bf16 scale."""
+    rng = np.random.default_rng(2)
+    for _ in range(50):
+        d = rng.standard_normal(256).astype(np.float32)
+        s = orc.f32_from_bf16(np.array([orc.sign1_scale(d)]))[0]
+
+        def err(sc):
+            return float(np.sum((d.astype(np.float64) - sc * np.sign(d)) ** 2))
+
+        h = orc.sign1_scale(d)
+        neighbours = orc.f32_from_bf16(np.array([h - 1, h + 1], dtype=np.uint16))
+        assert err(s) <= min(err(float(neighbours[0])), err(float(neighbours[1]))) + 1e-9
+
+
+def test_sign1_bit_layout_hand_built(orc):
+    """A single negative entry at column j sets bit j%32 of word j//32 of its row, and C = -S there."""
+    rows, cols = 3, 96
+    o = orc.Oracle(rows, cols, "sign1", dtype="f32")
+    a0 = np.zeros((rows, cols), np.float32)
+    o.encode(a0)
+    a1 = np.full((rows, cols), 0.5, np.float32)
+    negs = {0: [0], 1: [31, 32], 2: [95, 40, 1]}
+    for r, cs in negs.items():
+        for c in cs:
+            a1[r, c] = -0.25
+    p = o.encode(a1)
+    body = p[64:]
+    scales = body[:16].view(np.uint16)[:rows]
+    words = body[16:16 + rows * cols // 8].view(np.uint32).reshape(rows, cols // 32)
+    for r in range(rows):
+        expect = [0, 0, 0]
+        for c in negs[r]:
+            expect[c // 32] |= 1 << (c % 32)
+        assert list(words[r]) == expect
+        # mean |d| = (0.5 * (96 - k) + 0.25 * k) / 96 exactly representable?  compare to rational
+        k = len(negs[r])
+        mean = Fraction(1, 2) * (cols - k) / cols + Fraction(1, 4) * k / cols
+        want = int(_bf16_torch(np.array([_round_fraction_to_f32(mean)], np.float32))[0])
+        assert int(scales[r]) == want
+
+
+# ------------------------------------------------------------------ Q2
+
+def test_q2_code_is_nearest_level(orc):
+    """Brute force over the four levels, exact arithmetic; RNE only matters at exact ties."""
+    rng = np.random.default_rng(3)
+    for _ in range(4000):
+        S = float(orc.f32_from_bf16(orc.bf16_from_f32(np.array([rng.uniform(0.01, 100)], np.float32)))[0])
+        d = np.float32(rng.uniform(-1.2, 1.2) * S)
+        q = orc.q2_code(float(d), S)
+        Fd, FS = Fraction(float(d)), Fraction(S)
+        dist = [abs(Fd - Fraction(2 * k - 3, 3) * FS) for k in range(4)]
+        best = min(dist)
+        if dist[q] != best:
+            # only within a few fp32 ulps of a decision boundary may the RN chain pick the neighbour
+            u = Fraction(3, 2) * Fd / FS + Fraction(3, 2)
+            assert min(abs(u - Fraction(2 * k + 1, 2)) for k in range(3)) < Fraction(1, 2 ** 20)
+            assert abs(q - dist.index(best)) == 1
+
+
+def test_q2_ties_and_levels(orc):
+    S = 1.5
+    assert orc.q2_code(0.0, S) == 2          # u = 1.5 -> even -> 2 (+S/3)
+    assert orc.q2_code(-0.0, S) == 2
+    assert orc.q2_code(-1.0, S) == 0          # -2S/3: u = 0.5 -> 0
+    assert orc.q2_code(1.0, S) == 2           # +2S/3: u = 2.5 -> 2
+    assert orc.q2_code(5.0, S) == 3 and orc.q2_code(-5.0, S) == 0   # clamp
+    assert orc.q2_code(3.0, 0.0) == 0         # zero scale
+    lv = [orc.q2_level(k, S) for k in range(4)]
+    assert lv == [-1.5, np.float32(-0.5), np.float32(0.5), 1.5]
+    assert math.copysign(1.0, orc.q2_level(0, 0.0)) == -1.0   # -0.0 at zero scale
+
+
+def test_q2_scale_is_bf16_absmax(orc):
+    rng = np.random.default_rng(4)
+    d = rng.standard_normal(3072).astype(np.float32)
+    assert orc.q2_scale(d) == int(_bf16_torch(np.array([np.abs(d).max()], np.float32))[0])
+
+
+def test_q2_code_layout(orc):
+    rows, cols = 2, 32
+    o = orc.Oracle(rows, cols, "q2", dtype="f32")
+    o.encode(np.zeros((rows, cols), np.float32))
+    a1 = np.zeros((rows, cols), np.float32)
+    a1[0, :] = 3.0                       # max -> code 3 everywhere
+    a1[1, :] = -3.0
+    a1[1, 17] = 3.0                      # row 1: code 0 everywhere except col 17 -> 3
+    p = o.encode(a1)
+    body = p[64:]
+    words = body[16:16 + rows * cols // 4].view(np.uint32).reshape(rows, cols // 16)
+    assert list(words[0]) == [0xFFFFFFFF, 0xFFFFFFFF]
+    assert list(words[1]) == [0, 3 << 2]
+
+
+# ------------------------------------------------------------------ NM
+
+def _nm_brute(d, n):
+    """Max sum |d| over all n-subsets, ties -> lexicographically smallest subset (exact arithmetic)."""
+    best, best_set = None, None
+    for s in itertools.combinations(range(len(d)), n):
+        v = sum(Fraction(float(abs(d[i]))) for i in s)
+        if best is None or v > best:
+            best, best_set = v, s
+    return list(best_set)
+
+
+@pytest.mark.parametrize("m,n", [(16, 1), (16, 2), (8, 1), (8, 3), (4, 1), (4, 2)])
+def test_nm_select_brute_force(orc, m, n):
+    rng = np.random.default_rng(5 + m * 10 + n)
+    cases = []
+    for _ in range(150):
+        cases.append(rng.standard_normal(m).astype(np.float32))
+    # adversarial: zeros, equal magnitudes, +- pairs, a single non-zero
+    cases.append(np.zeros(m, np.float32))
+    cases.append(np.full(m, 0.5, np.float32))
+    alt = np.full(m, 0.5, np.float32)
+    alt[::2] = -0.5
+    cases.append(alt)
+    one = np.zeros(m, np.float32)
+    one[m - 1] = -1.0
+    cases.append(one)
+    pairs = rng.choice([-1.0, 1.0, -2.0, 2.0], m).astype(np.float32)
+    cases.append(pairs)
+    for d in cases:
+        assert orc.nm_select(d, n) == _nm_brute(d, n), d
+
+
+def test_nm_layout_hand_built(orc):
+    rows, cols, M, N = 1, 64, 16, 2
+    o = orc.Oracle(rows, cols, "nm", dtype="f32", nm_n=N, nm_m=M)
+    o.encode(np.zeros((rows, cols), np.float32))
+    a1 = np.zeros((rows, cols), np.float32)
+    a1[0, 3] = 2.0
+    a1[0, 9] = -3.0
+    a1[0, 16 + 15] = 1.0
+    a1[0, 16 + 0] = 1.0   # tie with col 31: lower index (0) first
+    a1[0, 16 + 7] = 0.5
+    p = o.encode(a1)
+    body = p[64:]
+    vals = body[:rows * (cols // M) * N * 2].view(np.uint16)
+    off = ((rows * (cols // M) * N * 2 + 15) // 16) * 16
+    idx = body[off:off + 4].view(np.uint32)[0]
+    # block 0 keeps cols 3 and 9 (ascending), block 1 keeps 0 and 15
+    # blocks 2 and 3 are all zero: indices 0 and 1 (lowest indices win the tie), values +0
+    assert list(_f32_of_bf16(vals)) == [2.0, -3.0, 1.0, 1.0, 0.0, 0.0, 0.0, 0.0]
+    assert idx == (3 | (9 << 4) | (0 << 8) | (15 << 12) | (0 << 16) | (1 << 20) | (0 << 24) | (1 << 28))
+
+
+# ------------------------------------------------------------------ recurrence
+
+def _walk(rows, cols, steps, seed, dtype="f32", sigma=0.1):
+    rng = np.random.default_rng(seed)
+    a = rng.standard_normal((rows, cols)).astype(np.float32)
+    out = [a.copy()]
+    for _ in range(steps - 1):
+        a = (a + sigma * rng.standard_normal((rows, cols))).astype(np.float32)
+        out.append(a.copy())
+    if dtype == "bf16":
+        out = [_bf16_torch(x) for x in out]
+    return out
+
+
+@pytest.mark.parametrize("mode,kw", [("identity", {}), ("sign1", {}), ("q2", {}), ("nm", {"nm_n": 2, "nm_m": 16}),
+                                     ("nm", {"nm_n": 1, "nm_m": 8}),
+                                     ("lowrank", {"rank": 4, "iters": 1, "lr_int4": 1}),
+                                     ("lowrank", {"rank": 4, "iters": 2, "lr_int4": 0})])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_sender_receiver_bit_equal(orc, mode, kw, dtype):
+    rows, cols, T = 24, 64, 6
+    o = orc.Oracle(rows, cols, mode, dtype=dtype, **kw)
+    for a in _walk(rows, cols, T, 6, dtype):
+        p = o.encode(a)
+        recon, st = o.decode(p)
+        assert st == 0
+        assert np.array_equal(o.ahat_s.view(np.uint32), o.ahat_r.view(np.uint32))
+        if dtype == "f32":
+            assert np.array_equal(recon.view(np.uint32), o.ahat_r.view(np.uint32))
+        else:
+            assert np.array_equal(recon, _bf16_torch(o.ahat_r))
+
+
+@pytest.mark.parametrize("mode,kw", [("sign1", {}), ("q2", {}), ("nm", {"nm_n": 1, "nm_m": 16}),
+                                     ("lowrank", {"rank": 3, "iters": 1, "lr_int4": 1})])
+def test_telescoping_identity(orc, mode, kw):
+    """Explicit EF: sum_t C_t + e_T - e_{T-1} = a_T - ahat_0 for every T.
+    Implicit EF: sum_t C_t + e_T = a_T - ahat_0 (the literal invariant).
+    Both sides accumulated in fp64; fp32 rounding of each step bounds the gap."""
+    rows, cols, T = 16, 64, 8
+    for ef in ["explicit", "implicit"]:
+        o = orc.Oracle(rows, cols, mode, dtype="f32", ef=ef, **kw)
+        stream = _walk(rows, cols, T, 7)
+        o.encode(stream[0])
+        ahat0 = o.ahat_s[0].astype(np.float64).copy()
+        csum = np.zeros((rows, cols))
+        e_prev = np.zeros((rows, cols))
+        for t in range(1, T):
+            p = o.encode(stream[t])
+            csum += o.meaning(p).astype(np.float64)
+            e = o.err[0].astype(np.float64)
+            lhs = csum + e - (e_prev if ef == "explicit" else 0.0)
+            rhs = stream[t].astype(np.float64) - ahat0
+            tol = 1e-6 * t * max(1.0, np.abs(stream[t]).max())
+            assert np.abs(lhs - rhs).max() <= tol, (ef, t, np.abs(lhs - rhs).max())
+            e_prev = e.copy()
+        if ef == "explicit":
+            # the literal invariant holds for explicit EF at T = 1 only
+            pass
+
+
+def test_explicit_literal_invariant_at_T1(orc):
+    rows, cols = 8, 64
+    o = orc.Oracle(rows, cols, "sign1", dtype="f32")
+    s = _walk(rows, cols, 2, 8)
+    o.encode(s[0])
+    a0 = o.ahat_s[0].astype(np.float64).copy()
+    p = o.encode(s[1])
+    lhs = o.meaning(p).astype(np.float64) + o.err[0]
+    assert np.abs(lhs - (s[1] - a0)).max() < 1e-6
+
+
+def test_identity_mode_reconstructs(orc):
+    rows, cols = 32, 64
+    o = orc.Oracle(rows, cols, "identity", dtype="f32")
+    u = 2.0 ** -24
+    for t, a in enumerate(_walk(rows, cols, 5, 9)):
+        prev = o.ahat_s[0].astype(np.float64).copy()
+        p = o.encode(a)
+        recon, st = o.decode(p)
+        assert st == 0
+        a64 = a.astype(np.float64)
+        if t == 0:
+            assert np.array_equal(o.ahat_s[0], a)
+        else:
+            # ahat' = fl(ahat + fl(a - ahat)): |ahat' - a| <= u (|a| + |a - ahat|) (1 + 2u)
+            bound = u * (np.abs(a64) + np.abs(a64 - prev)) * (1 + 2 * u)
+            assert np.all(np.abs(o.ahat_s[0].astype(np.float64) - a64) <= bound)
+        assert np.all(o.err == 0.0)
+
+
+def test_warmup_payload_is_raw(orc):
+    rows, cols = 4, 64
+    for dtype in ["f32", "bf16"]:
+        o = orc.Oracle(rows, cols, "q2", dtype=dtype)
+        a0 = _walk(rows, cols, 1, 10, dtype)[0]
+        p = o.encode(a0)
+        raw = a0.tobytes()
+        assert bytes(p[64:64 + len(raw)]) == raw
+        hdr = p[:64]
+        assert hdr[:4].tobytes() == b"CFP1"
+        assert hdr[8:12].view(np.uint32)[0] == 1   # warm-up flag
+        recon, _ = o.decode(p)
+        assert recon.tobytes() == raw
+
+
+def test_header_mismatch_leaves_receiver_untouched(orc):
+    rows, cols = 8, 64
+    o = orc.Oracle(rows, cols, "sign1", dtype="f32")
+    s = _walk(rows, cols, 3, 11)
+    o.decode(o.encode(s[0]))
+    p1 = o.encode(s[1])
+    bad = p1.copy()
+    bad[16] ^= 1                      # wrong step
+    before = o.ahat_r.copy()
+    _, st = o.decode(bad)
+    assert st == 1 and o.status() == 1
+    assert np.array_equal(before, o.ahat_r)
+
+
+def test_residual_beats_direct_compression(orc):
+    """Residual 1-bit reconstruction stays close where direct 1-bit of a_t does not (residual
+    compression section): sigma_delta / sigma_a = 0.1."""
+    rows, cols, T = 32, 256, 10
+    s = _walk(rows, cols, T, 12)
+    o = orc.Oracle(rows, cols, "sign1", dtype="f32")
+    for a in s:
+        o.decode(o.encode(a))
+    res_err = np.linalg.norm(o.ahat_r[0] - s[-1]) / np.linalg.norm(s[-1])
+    # direct: 1-bit of a_T itself with its own L2-optimal scale
+    a = s[-1]
+    direct = np.sign(a) * np.abs(a).mean(axis=1, keepdims=True)
+    dir_err = np.linalg.norm(direct - a) / np.linalg.norm(a)
+    assert res_err < 0.5 * dir_err, (res_err, dir_err)
+
+
+def test_error_feedback_bounds_error(orc):
+    """With error feedback the reconstruction error stays bounded over 28 steps
+    (error feedback section); it does not grow with the step count."""
+    rows, cols, T = 16, 128, 28
+    s = _walk(rows, cols, T, 13)
+    o = orc.Oracle(rows, cols, "sign1", dtype="f32")
+    errs = []
+    for a in s:
+        o.decode(o.encode(a))
+        errs.append(np.linalg.norm(o.ahat_r[0] - a) / np.linalg.norm(a))
+    assert max(errs[14:]) < 2.0 * max(errs[1:14]) + 1e-6
+
+
+# ------------------------------------------------------------------ low-rank
+
+def test_householder_qr_matches_library(orc):
+    rng = np.random.default_rng(14)
+    Y = rng.standard_normal((50, 7))
+    Q, rd, dead = orc.householder_qr(Y)
+    Qn, Rn = np.linalg.qr(Y)
+    sg = np.sign(np.diag(Rn))
+    Qn = Qn * sg
+    assert not dead.any()
+    assert np.abs(Q - Qn).max() < 1e-12
+    assert np.abs(rd - np.abs(np.diag(Rn))).max() < 1e-12
+    assert np.abs(Q.T @ Q - np.eye(7)).max() < 1e-12
+
+
+def test_householder_rank_deficient_columns_zeroed(orc):
+    rng = np.random.default_rng(15)
+    Y = rng.standard_normal((30, 4))
+    Y[:, 2] = 2.0 * Y[:, 0] - Y[:, 1]
+    Q, rd, dead = orc.householder_qr(Y)
+    assert list(dead) == [False, False, True, False]
+    assert np.all(Q[:, 2] == 0.0)
+    keep = Q[:, [0, 1, 3]]
+    assert np.abs(keep.T @ keep - np.eye(3)).max() < 1e-12
+
+
+def test_lowrank_full_rank_no_quant_is_exact(orc):
+    """rank = cols <= rows and no quantisation: C(Delta) = Delta within 1e-5 relative."""
+    rows, cols = 40, 16
+    o = orc.Oracle(rows, cols, "lowrank", dtype="f32", rank=cols, iters=1, lr_int4=0, seed=5)
+    s = _walk(rows, cols, 3, 16)
+    o.encode(s[0])
+    for a in s[1:]:
+        d = (a - o.ahat_s[0]) + o.err[0]
+        p = o.encode(a)
+        C = o.meaning(p)
+        assert np.linalg.norm(C - d) / np.linalg.norm(d) < 1e-5
+
+
+def test_lowrank_recovers_exact_rank_r(orc):
+    rng = np.random.default_rng(17)
+    m, n, r = 60, 48, 5
+    D = (rng.standard_normal((m, r)) @ rng.standard_normal((r, n))).astype(np.float32)
+    V0 = orc.lr_v0(9, n, r).astype(np.float64)
+    Q, V = orc.subspace_iteration(D, V0, 1)
+    C = Q @ V.T
+    assert np.linalg.norm(C - D) / np.linalg.norm(D) < 1e-5
+    assert np.abs(Q.T @ Q - np.eye(r)).max() < 1e-5
+
+
+def test_lowrank_converges_to_eckart_young(orc):
+    rng = np.random.default_rng(18)
+    m, n, r = 40, 30, 4
+    # decaying spectrum so the dominant subspace is well separated
+    U, _ = np.linalg.qr(rng.standard_normal((m, n)))
+    W, _ = np.linalg.qr(rng.standard_normal((n, n)))
+    sv = 2.0 ** -np.arange(n, dtype=np.float64) * 10
+    D = ((U * sv) @ W.T).astype(np.float32)
+    V0 = orc.lr_v0(3, n, r).astype(np.float64)
+    Q, V = orc.subspace_iteration(D, V0, 60)
+    err = np.linalg.norm(Q @ V.T - D.astype(np.float64)) / np.linalg.norm(D.astype(np.float64))
+    s = np.linalg.svd(D.astype(np.float64), compute_uv=False)
+    ey = math.sqrt(float(np.sum(s[r:] ** 2))) / math.sqrt(float(np.sum(s ** 2)))
+    assert abs(err - ey) <= 1e-6 + 1e-3 * ey
+
+
+def test_lowrank_int4_error_bound(orc):
+    """Dequantised INT4 factors differ from the fp factors by at most s_k / 2 (clamp never binds)."""
+    rows, cols, r = 64, 48, 6
+    o = orc.Oracle(rows, cols, "lowrank", dtype="f32", rank=r, iters=1, lr_int4=1, seed=4)
+    s = _walk(rows, cols, 2, 19)
+    o.encode(s[0])
+    d = ((s[1] - o.ahat_s[0]) + o.err[0]).astype(np.float32)
+    p = o.encode(s[1])
+    body = p[64:]
+    sU = body[:r * 4].view(np.float32)
+    sV = body[r * 4:r * 8].view(np.float32)
+    off_u = ((r * 8 + 15) // 16) * 16
+    nib_u = np.frombuffer(body[off_u:off_u + (rows * r + 1) // 2].tobytes(), np.uint8)
+    codes = np.empty(rows * r, np.int64)
+    codes[0::2] = nib_u & 0xF
+    codes[1::2] = nib_u >> 4
+    codes = np.where(codes >= 8, codes - 16, codes).reshape(rows, r)
+    assert codes.min() >= -7 and codes.max() <= 7
+    V0 = orc.lr_v0(4, cols, r).astype(np.float64)
+    Q, V = orc.subspace_iteration(d, V0, 1)
+    assert np.all(np.abs(codes * sU.astype(np.float64) - Q) <= sU.astype(np.float64) / 2 * (1 + 1e-6) + 1e-12)
+    assert np.allclose(sU, (np.abs(Q).max(axis=0) / 7).astype(np.float32))
+    assert np.allclose(sV, (np.abs(V).max(axis=0) / 7).astype(np.float32))
+
+
+def test_sign1_scale_fraction_bits_near_midpoint(orc):
+    """A mean just above a bf16 rounding midpoint, with one large entry setting the
+    fixed-point exponent: too few fraction bits would truncate the small entries and
+    round the scale the other way."""
+    n = 3072
+    target = 1.0 + 2.0 ** -8 + 2.0 ** -20          # just above the 1.0 / 1.0078125 midpoint
+    x = np.float32((n * target - 2048.0) / (n - 1))
+    d = np.full(n, x, np.float32)
+    d[0] = 2048.0
+    q = _exact_mean_abs(d)
+    want = int(_bf16_torch(np.array([_round_fraction_to_f32(q)], np.float32))[0])
+    assert orc.sign1_scale(d) == want
+    assert abs(float(q) - (1.0 + 2.0 ** -8)) < 2.0 ** -16  # the case really sits at the midpoint
+
+
+def test_householder_first_column_along_e1(orc):
+    """x nearly parallel to e1: the reflector must be formed without cancellation."""
+    rng = np.random.default_rng(20)
+    Y = rng.standard_normal((12, 3))
+    Y[:, 0] = 0.0
+    Y[0, 0] = 1.0
+    Y[1, 0] = 1e-9
+    Q, rd, dead = orc.householder_qr(Y)
+    Qn, Rn = np.linalg.qr(Y)
+    Qn = Qn * np.sign(np.diag(Rn))
+    assert np.abs(Q - Qn).max() < 1e-12
