@@ -1,0 +1,87 @@
+"""The C-ABI library loads and exports every entry point include/cf.h declares;
+host-side validation answers without a GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "cf.h")).read()
+    return sorted(set(re.findall(r"^CF_API\s+(?:const\s+char\s*\*|int)\s*(cf_\w+)\s*\(", src, re.M)))
+
+
+@pytest.fixture(scope="module")
+def cf():
+    from activation_residual_compression_b200 import build
+    build.build()
+    import activation_residual_compression_b200 as m
+    m._cf.load()
+    return m
+
+
+def test_every_declared_symbol_is_exported(cf):
+    names = _declared()
+    assert len(names) >= 18
+    lib = ctypes.CDLL(cf._cf.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(cf._cf.EXPORTS)
+
+
+def test_strerror_and_version(cf):
+    assert "sm_100a" in cf.cf_version()
+    for code in range(0, -11, -1):
+        assert cf.cf_strerror(code) != "unknown status"
+    assert cf.cf_strerror(-99) == "unknown status"
+
+
+def test_params_defaults(cf):
+    p = cf.cf_params_init()
+    assert (p.dtype, p.role, p.ef, p.nm_n, p.nm_m, p.rank, p.iters, p.lr_int4, p.batch) == \
+        (cf.CF_BF16, cf.CF_SENDER, cf.CF_EF_EXPLICIT, 2, 16, 70, 1, 1, 1)
+
+
+def _ws(cf, rows, cols, mode, **kw):
+    p = cf.cf_params_init(**kw)
+    out = ctypes.c_size_t()
+    rc = cf.raw("cf_workspace_bytes")(rows, cols, mode, ctypes.byref(p), ctypes.byref(out))
+    return rc, out.value
+
+
+def test_shape_rules_rejected_on_host(cf):
+    assert _ws(cf, 4608, 3072, cf.CF_SIGN1)[0] == cf.CF_OK
+    assert _ws(cf, 4608, 3072 + 16, cf.CF_SIGN1)[0] == cf.CF_ERR_SHAPE      # cols % 32
+    assert _ws(cf, 4608, 3072 + 16, cf.CF_Q2)[0] == cf.CF_OK
+    assert _ws(cf, 4608, 3072 + 8, cf.CF_Q2)[0] == cf.CF_ERR_SHAPE          # cols % 16
+    assert _ws(cf, 4608, 3072 + 4, cf.CF_IDENTITY)[0] == cf.CF_ERR_SHAPE    # cols % 8
+    assert _ws(cf, 0, 64, cf.CF_Q2)[0] == cf.CF_ERR_SHAPE
+    assert _ws(cf, 4, 8192 + 32, cf.CF_SIGN1)[0] == cf.CF_ERR_SHAPE         # > max row width
+    assert _ws(cf, 4, 1920, cf.CF_NM, nm_n=1, nm_m=16)[0] == cf.CF_OK
+    assert _ws(cf, 4, 1920 + 64, cf.CF_NM, nm_n=1, nm_m=16)[0] == cf.CF_ERR_SHAPE  # index words
+    assert _ws(cf, 4, 64, cf.CF_NM, nm_n=2, nm_m=8)[0] == cf.CF_ERR_UNSUPPORTED
+    assert _ws(cf, 4, 64, cf.CF_NM, nm_n=3, nm_m=16)[0] == cf.CF_ERR_UNSUPPORTED
+    assert _ws(cf, 4, 64, 7)[0] == cf.CF_ERR_ARG
+    assert _ws(cf, 4, 64, cf.CF_Q2, dtype=5)[0] == cf.CF_ERR_ARG
+    assert _ws(cf, 4, 64, cf.CF_Q2, batch=0)[0] == cf.CF_ERR_ARG
+
+
+def test_workspace_sizes(cf):
+    E = 4608 * 3072
+    rc, s = _ws(cf, 4608, 3072, cf.CF_SIGN1, role=cf.CF_SENDER)
+    assert rc == 0 and s >= 2 * E * 4 and s < 2 * E * 4 + 4096
+    rc, r = _ws(cf, 4608, 3072, cf.CF_SIGN1, role=cf.CF_RECEIVER)
+    assert rc == 0 and r >= E * 4 and r < E * 4 + 4096
+
+
+def test_null_handles_rejected(cf):
+    P = ctypes.c_void_p
+    assert cf.raw("cf_encode")(None, P(16), P(16), None) == cf.CF_ERR_STATE
+    assert cf.raw("cf_decode")(None, P(16), P(16), None) == cf.CF_ERR_STATE
+    assert cf.raw("cf_destroy")(P(12345)) == cf.CF_ERR_STATE
+    assert cf.raw("cf_status")(P(12345), None) == cf.CF_ERR_STATE
+    out = ctypes.c_size_t()
+    assert cf.raw("cf_payload_bytes")(P(12345), 0, ctypes.byref(out)) == cf.CF_ERR_STATE
