@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of the residual codec on B200: activation GB/s and ms/step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {cf,reference}]
+
+Workload: the FLUX.1-dev-shaped activation stream (4608 x 3072 bf16, 1%
+outlier channels x20, random walk with sigma/sigma_a = 0.1) compressed with
+residual compression + explicit error feedback in the 1-bit and the 2-bit
+modes ("Accelerating Parallel Diffusion Model Serving with Residual
+Compression": experiments, main table).  Each mode is a sender/receiver pair
+of its own on its own seeded stream; one step = encode + decode of one
+activation in every mode.  Inputs are pre-generated in HBM (a fresh tensor
+per step; the per-kernel working set exceeds the 126 MB L2).
+
+value  = activation bytes (rows*cols*2 per mode) / device time per step,
+         CUDA events on the launching stream, max over ranks.
+e2e    = the same metric with the activation in pinned host memory: each
+         step copies a_t host->device, encodes, decodes and copies the
+         reconstruction device->host, inside the timed region.
+roofline = the encode kernel of the first mode: algorithmic bytes per launch
+         (read a, ahat, e; write ahat, e, payload) / its mean event-timed
+         duration, against the measured copy bandwidth.
+
+With --gpus N (torchrun) every rank runs an independent replica on its own
+GPU (the method needs no exchange here); value sums all ranks' activation
+bytes over the slowest rank's time.  --impl reference times the CPU oracle
+(rank 0 only) on a row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+ROWS, COLS = 4608, 3072
+MODES = [("sign1", {}), ("q2", {})]
+WORKLOAD = "flux1dev-4608x3072-bf16"
+METRIC = "activation GB/s and ms/step per mode (encode+EF+decode), % of B200 HBM roofline"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _payload_body(mode, rows, cols, kw):
+    pad = lambda b: (b + 15) // 16 * 16  # noqa: E731
+    if mode == "sign1":
+        return pad(rows * 2) + pad(rows * cols // 8)
+    if mode == "q2":
+        return pad(rows * 2) + pad(rows * cols // 4)
+    if mode == "nm":
+        n, m = kw["nm_n"], kw["nm_m"]
+        return pad(rows * cols // m * n * 2) + pad(rows * (cols // m * n * (m.bit_length() - 1) // 32) * 4)
+    if mode == "identity":
+        return rows * cols * 4
+    raise ValueError(mode)
+
+
+def encode_bytes(mode, rows, cols, kw, act_size=2):
+    """Algorithmic bytes of one encode launch: read a, ahat, e; write ahat, e, payload."""
+    E = rows * cols
+    return E * (act_size + 4 + 4 + 4 + 4) + 64 + _payload_body(mode, rows, cols, kw)
+
+
+def decode_bytes(mode, rows, cols, kw, act_size=2):
+    """Algorithmic bytes of one decode launch: read payload, ahat; write ahat, recon."""
+    E = rows * cols
+    return E * (4 + 4 + act_size) + 64 + _payload_body(mode, rows, cols, kw)
+
+
+def _traffic_record():
+    """dram read+write bytes per encode launch from the committed ncu summary,
+    valid only while the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "encode_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "activation_residual_compression_b200", "csrc", "cf_stream.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if d.get("source_sha256") != h:
+        return None
+    return d
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            self.path = f"/tmp/cf_clocks_{os.getpid()}.csv"
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu_index)], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_cf(args, rank, world, device):
+    import torch
+
+    import activation_residual_compression_b200 as cf
+    from activation_residual_compression_b200 import inputs
+
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream()
+    K, W = args.steps, args.warmup
+    n_inputs = min(W + K + 1, args.max_resident)
+    codecs = []
+    for mi, (mode, kw) in enumerate(MODES):
+        s = inputs.flux("cuda", rows=ROWS, cols=COLS, seed=1 + 100 * mi + 1000 * rank)
+        acts = [s.next() for _ in range(n_inputs)]
+        base = dict(dtype=cf.CF_BF16, **kw)
+        S = cf.cf_create(ROWS, COLS, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_SENDER, **base))
+        R = cf.cf_create(ROWS, COLS, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_RECEIVER, **base))
+        pay = torch.empty(max(cf.cf_payload_bytes(S, True), cf.cf_payload_bytes(S, False)), dtype=torch.uint8,
+                          device="cuda")
+        rec = torch.empty(ROWS, COLS, dtype=torch.bfloat16, device="cuda")
+        codecs.append(dict(mode=mode, kw=kw, S=S, R=R, pay=pay, rec=rec, acts=acts))
+    torch.cuda.synchronize()
+
+    def step(i, evs=None):
+        for c in codecs:
+            a = c["acts"][i % n_inputs]
+            if evs is not None:
+                evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
+            cf.cf_encode(c["S"], a, c["pay"], stream)
+            if evs is not None:
+                evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
+            cf.cf_decode(c["R"], c["pay"], c["rec"], stream)
+        if evs is not None:
+            evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            step(i)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(device)
+    clocks.start()
+    time.sleep(0.3)
+    evs = []
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for i in range(W, W + K):
+            step(i, evs)
+        t1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    # per-kernel durations: evs per step = [pre_enc0, pre_dec0/post_enc0, pre_enc1 ..., end]
+    nm = len(codecs)
+    per = {c["mode"]: {"enc": [], "dec": []} for c in codecs}
+    # events per step: for each codec (before encode, before decode), then one at the end
+    stride = 2 * nm + 1
+    for k in range(K):
+        base = k * stride
+        for mi, c in enumerate(codecs):
+            e_enc0 = evs[base + 2 * mi]
+            e_dec0 = evs[base + 2 * mi + 1]
+            e_next = evs[base + 2 * mi + 2]
+            per[c["mode"]]["enc"].append(e_enc0.elapsed_time(e_dec0))
+            per[c["mode"]]["dec"].append(e_dec0.elapsed_time(e_next))
+    for c in codecs:
+        if cf.cf_status(c["R"], stream) != cf.CF_OK:
+            raise RuntimeError(f"receiver of {c['mode']} reported a desync")
+
+    # e2e: pinned host activations in, pinned host reconstruction out
+    e2e = None
+    if args.e2e_steps > 0:
+        host_in = [c["acts"][0].cpu().pin_memory() for c in codecs]
+        host_out = [torch.empty(ROWS, COLS, dtype=torch.bfloat16).pin_memory() for _ in codecs]
+        dev_in = [torch.empty_like(h, device="cuda") for h in host_in]
+        for c in codecs:
+            cf.cf_reset(c["S"]); cf.cf_reset(c["R"])
+
+        def e2e_step():
+            for ci, c in enumerate(codecs):
+                dev_in[ci].copy_(host_in[ci], non_blocking=True)
+                cf.cf_encode(c["S"], dev_in[ci], c["pay"], stream)
+                cf.cf_decode(c["R"], c["pay"], c["rec"], stream)
+                host_out[ci].copy_(c["rec"], non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                e2e_step()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a0.record(stream)
+            for _ in range(args.e2e_steps):
+                e2e_step()
+            a1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a0.elapsed_time(a1) / args.e2e_steps
+        e2e = dict(ms=e2e_ms, h2d=sum(t.numel() * 2 for t in host_in), d2h=sum(t.numel() * 2 for t in host_out))
+
+    for c in codecs:
+        cf.cf_destroy(c["S"]); cf.cf_destroy(c["R"])
+
+    ms_step = total_ms / K
+    stats = dict(ms_step=ms_step, per={m: {k: statistics.mean(v) for k, v in d.items()} for m, d in per.items()},
+                 e2e=e2e, clocks=clk)
+    return stats
+
+
+def cpu_baseline(max_seconds=20.0):
+    """The CPU oracle, as it stands, on the same workload: full 4608 x 3072 bf16
+    FLUX-shaped stream, both modes, compressed steps until max_seconds of oracle
+    time (warm-up step untimed)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from activation_residual_compression_b200 import inputs
+
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    orcs = []
+    for mi, (mode, kw) in enumerate(MODES):
+        s = inputs.flux("cpu", rows=ROWS, cols=COLS, seed=1 + 100 * mi)
+        o = oracle.Oracle(ROWS, COLS, mode, dtype="bf16", **kw)
+        a = s.next().view(torch.int16).numpy().view(np.uint16)
+        o.decode(o.encode(a))
+        orcs.append((s, o))
+    spent, steps = 0.0, 0
+    while spent < max_seconds and steps < 27:
+        ins = [s.next().view(torch.int16).numpy().view(np.uint16) for s, _ in orcs]
+        t = time.perf_counter()
+        for (s, o), a in zip(orcs, ins):
+            o.decode(o.encode(a))
+        spent += time.perf_counter() - t
+        steps += 1
+    act_bytes = steps * len(MODES) * ROWS * COLS * 2
+    return {"value": act_bytes / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{steps} compressed steps of the full {ROWS}x{COLS} bf16 stream, modes "
+                      f"{'+'.join(m for m, _ in MODES)} (encode+decode), {spent:.1f} s of oracle time",
+            "ms_per_step": spent / steps * 1e3}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step = encode+decode in both modes of
+    a 1152-row sample (a quarter of the rows; rows are independent) of the stream."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from activation_residual_compression_b200 import inputs
+
+    rows = 1152
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    orcs = []
+    for mi, (mode, kw) in enumerate(MODES):
+        s = inputs.flux("cpu", rows=rows, cols=COLS, seed=1 + 100 * mi)
+        orcs.append((s, oracle.Oracle(rows, COLS, mode, dtype="bf16", **kw)))
+
+    def one():
+        ins = [s.next().view(torch.int16).numpy().view(np.uint16) for s, _ in orcs]
+        t = time.perf_counter()
+        for (s, o), a in zip(orcs, ins):
+            o.decode(o.encode(a))
+        return time.perf_counter() - t
+
+    one()  # the stream's raw first step
+    for _ in range(args.warmup):
+        one()
+    spent = sum(one() for _ in range(args.steps))
+    ms = spent / args.steps * 1e3
+    val = len(MODES) * rows * COLS * 2 / (ms / 1e3) / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "modes": [m for m, _ in MODES], "sample_rows": rows},
+            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{rows} of {ROWS} rows x {COLS} bf16 per step, both modes"},
+            "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cf", choices=["cf", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--max-resident", type=int, default=400, help="pre-generated inputs per mode (cycled)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    st = run_cf(args, rank, world, local)
+    ms = st["ms_step"]
+    e2e_ms = st["e2e"]["ms"] if st["e2e"] else None
+    if dist:
+        t = torch.tensor([ms, e2e_ms or 0.0], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+    act_bytes = len(MODES) * ROWS * COLS * 2 * world
+    value = act_bytes / (ms / 1e3) / 1e9
+    peak, peak_kind = _peaks()
+    m0, kw0 = MODES[0]
+    enc_ms = st["per"][m0]["enc"]
+    achieved = encode_bytes(m0, ROWS, COLS, kw0) / (enc_ms / 1e3) / 1e9
+    tr = _traffic_record()
+    per_mode = {}
+    for m, kw in MODES:
+        pm = st["per"][m]
+        step_ms = pm["enc"] + pm["dec"]
+        alg = encode_bytes(m, ROWS, COLS, kw) + decode_bytes(m, ROWS, COLS, kw)
+        per_mode[m] = {"ms_per_step": round(step_ms, 5), "encode_ms": round(pm["enc"], 5),
+                       "decode_ms": round(pm["dec"], 5),
+                       "activation_gbs": round(ROWS * COLS * 2 / (step_ms / 1e3) / 1e9, 2),
+                       "hbm_gbs": round(alg / (step_ms / 1e3) / 1e9, 1),
+                       "roofline_frac": round(alg / (step_ms / 1e3) / 1e9 / peak, 4),
+                       "payload_bytes": 64 + _payload_body(m, ROWS, COLS, kw),
+                       "ratio_vs_bf16": round(ROWS * COLS * 2 / (64 + _payload_body(m, ROWS, COLS, kw)), 2)}
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "activation_dtype": "bf16",
+                   "modes": [m for m, _ in MODES], "error_feedback": "explicit",
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2: fresh 28 MB input per step, per-kernel working set 170-230 MB",
+                   "inputs_resident": True},
+        "per_mode": per_mode,
+        "roofline": {"bound": "hbm", "kernel": f"encode_kernel<{m0}, bf16>", "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": (tr["bytes_per_launch"] if tr else None),
+                     "algorithmic_bytes": encode_bytes(m0, ROWS, COLS, kw0), "peak_source": peak_kind},
+        "gpu_launches": 2 * len(MODES) * args.steps,
+        "clocks": st["clocks"],
+    }
+    if e2e_ms:
+        line["e2e"] = {"value": round(act_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+                       "h2d_bytes_per_step": st["e2e"]["h2d"], "d2h_bytes_per_step": st["e2e"]["d2h"],
+                       "ms_per_step": round(e2e_ms, 4)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
