@@ -25,6 +25,7 @@ CF_ERR_DESYNC = -7
 CF_ERR_ALIGN = -8
 CF_ERR_STATE = -9
 CF_ERR_SIZE = -10
+CF_ERR_TIMEOUT = -11
 
 CF_IDENTITY, CF_SIGN1, CF_Q2, CF_NM, CF_LOWRANK = 0, 1, 2, 3, 4
 CF_F32, CF_BF16 = 0, 1
@@ -191,9 +192,9 @@ def cf_decode_batched(state, payload, recon_list, stream=None) -> int:
 
 
 def cf_status(state, stream=None) -> int:
-    """Device status after synchronising the stream: CF_OK or CF_ERR_DESYNC (not raised)."""
+    """Device status after synchronising the stream: CF_OK, CF_ERR_DESYNC or CF_ERR_TIMEOUT (not raised)."""
     rc = load().cf_status(state, _stream(stream))
-    if rc not in (CF_OK, CF_ERR_DESYNC):
+    if rc not in (CF_OK, CF_ERR_DESYNC, CF_ERR_TIMEOUT):
         raise CFError("cf_status", rc)
     return rc
 

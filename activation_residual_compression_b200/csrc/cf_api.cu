@@ -58,12 +58,6 @@ int ilog2(int m) {
   return c;
 }
 
-int ceil_log2(int64_t n) {
-  int c = 0;
-  while (((int64_t)1 << c) < n) c++;
-  return c;
-}
-
 size_t act_size(int dtype) { return dtype == CF_BF16 ? 2u : 4u; }
 
 Layout layout_of(int64_t rows, int64_t cols, int mode, const cf_params &p) {
@@ -206,7 +200,7 @@ EncArgs enc_args(cf_state *s, const void *a, void *payload, bool warm) {
   A.batch = s->p.batch;
   A.ef_explicit = s->p.ef == CF_EF_EXPLICIT;
   A.team_log2 = s->cfg.team_log2;
-  A.fx_F = 62 - ceil_log2(s->cols);
+  A.status = s->status;
   A.hdr = header_of(s, warm, s->step);
   if (!warm) {
     // [end of first section, sec1) and [end of second section, body)
@@ -336,6 +330,7 @@ const char *cf_strerror(int status) {
     case CF_ERR_ALIGN: return "pointer not 16-byte aligned";
     case CF_ERR_STATE: return "not a live state";
     case CF_ERR_SIZE: return "host buffer size mismatch";
+    case CF_ERR_TIMEOUT: return "a kernel's bounded wait for its own asynchronous copy gave up";
   }
   return "unknown status";
 }
@@ -385,7 +380,8 @@ int cf_create(int64_t rows, int64_t cols, int mode, const cf_params *p, cf_state
   }
   if (mode == CF_LOWRANK) lowrank_plan(rows, cols, *p, &s->lr);
   s->lay = layout_of(rows, cols, mode, *p);
-  const int rc = stream_config(mode, p->dtype, p->nm_m, p->nm_n, rows, cols, p->batch, s->sm_count, &s->cfg);
+  const int rc = stream_config(mode, p->dtype, p->nm_m, p->nm_n, rows, cols, p->batch, s->sm_count,
+                               p->ef == CF_EF_EXPLICIT, &s->cfg);
   if (rc != CF_OK) {
     delete s;
     return rc;
@@ -470,7 +466,8 @@ int cf_status(cf_state *s, void *stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return cuda_err(cudaErrorUnknown);
   int h = 0;
   if (cudaMemcpy(&h, s->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_err(cudaErrorUnknown);
-  return h ? CF_ERR_DESYNC : CF_OK;
+  if (h & 2) return CF_ERR_TIMEOUT;
+  return (h & 1) ? CF_ERR_DESYNC : CF_OK;
 }
 
 int cf_tensor(cf_state *s, int which, void **dptr, size_t *bytes) {

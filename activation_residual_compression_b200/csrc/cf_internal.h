@@ -49,9 +49,9 @@ struct EncArgs {
   int batch;
   int ef_explicit;
   int team_log2;          // threads per row = 1 << team_log2 (>= 32)
-  int fx_F;               // SIGN1 fixed-point fraction bits: 62 - ceil(log2 cols)
   int64_t padA_off, padA_len;  // alignment padding inside each body, zeroed by the encoder
   int64_t padB_off, padB_len;
+  int *status;            // sticky device status word of the sender
   Header hdr;
 };
 
@@ -80,7 +80,7 @@ struct StreamCfg {
 
 // ---- streaming kernels (cf_stream.cu) ----
 int stream_config(int mode, int dtype, int nm_m, int nm_n, int64_t rows, int64_t cols, int batch,
-                  int sm_count, StreamCfg *cfg);
+                  int sm_count, int ef_explicit, StreamCfg *cfg);
 cudaError_t launch_encode(int mode, int dtype, int nm_m, int nm_n, const StreamCfg &cfg,
                           const EncArgs &args, const PtrTable *tab, cudaStream_t st);
 cudaError_t launch_decode(int mode, int dtype, int nm_m, int nm_n, const StreamCfg &cfg,

@@ -1,4 +1,5 @@
-// cf_stream.cu -- fused streaming kernels of the residual codec on sm_100a.
+// cf_stream.cu -- launch configuration and dispatch of the streaming
+// kernels (the kernels are in cf_stream_kernels.cuh).
 //
 // Method: "Accelerating Parallel Diffusion Model Serving with Residual
 // Compression" (NeurIPS 2025 paper notes).  One encode launch per step fuses
@@ -30,780 +31,21 @@
 #include <cstdint>
 
 #include "cf_internal.h"
+#include "cf_stream_kernels.cuh"
 
 namespace cfi {
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
-
-// ---------------------------------------------------------------- activations
-
-template <typename T>
-struct Act;
-
-template <>
-struct Act<float> {
-  struct Raw {
-    float4 lo, hi;
-  };
-  static __device__ __forceinline__ Raw load(const float *p) {
-    const float4 *q = reinterpret_cast<const float4 *>(p);
-    return Raw{__ldcs(q), __ldcs(q + 1)};
-  }
-  static __device__ __forceinline__ void to_f32(const Raw &r, float (&x)[8]) {
-    x[0] = r.lo.x; x[1] = r.lo.y; x[2] = r.lo.z; x[3] = r.lo.w;
-    x[4] = r.hi.x; x[5] = r.hi.y; x[6] = r.hi.z; x[7] = r.hi.w;
-  }
-  static __device__ __forceinline__ void store_raw(float *p, const Raw &r) {
-    float4 *q = reinterpret_cast<float4 *>(p);
-    __stcs(q, r.lo);
-    __stcs(q + 1, r.hi);
-  }
-  static __device__ __forceinline__ void store_f32(float *p, const float (&x)[8]) {
-    float4 *q = reinterpret_cast<float4 *>(p);
-    __stcs(q, make_float4(x[0], x[1], x[2], x[3]));
-    __stcs(q + 1, make_float4(x[4], x[5], x[6], x[7]));
-  }
-};
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-  uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-  return a | (b << 16);
-}
-
-template <>
-struct Act<__nv_bfloat16> {
-  using Raw = uint4;
-  static __device__ __forceinline__ Raw load(const __nv_bfloat16 *p) {
-    return __ldcs(reinterpret_cast<const uint4 *>(p));
-  }
-  // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 bits.
-  static __device__ __forceinline__ void to_f32(const Raw &r, float (&x)[8]) {
-    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-    for (int k = 0; k < 4; k++) {
-      x[2 * k] = __uint_as_float(w[k] << 16);
-      x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-    }
-  }
-  static __device__ __forceinline__ void store_raw(__nv_bfloat16 *p, const Raw &r) {
-    __stcs(reinterpret_cast<uint4 *>(p), r);
-  }
-  static __device__ __forceinline__ void store_f32(__nv_bfloat16 *p, const float (&x)[8]) {
-    uint4 r;
-    r.x = pack_bf16x2(x[0], x[1]);
-    r.y = pack_bf16x2(x[2], x[3]);
-    r.z = pack_bf16x2(x[4], x[5]);
-    r.w = pack_bf16x2(x[6], x[7]);
-    __stcs(reinterpret_cast<uint4 *>(p), r);
-  }
-};
-
-__device__ __forceinline__ void load_f32x8(const float *p, float (&x)[8]) {
-  const float4 *q = reinterpret_cast<const float4 *>(p);
-  float4 a = __ldcs(q), b = __ldcs(q + 1);
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-
-__device__ __forceinline__ void store_f32x8(float *p, const float (&x)[8]) {
-  float4 *q = reinterpret_cast<float4 *>(p);
-  __stcs(q, make_float4(x[0], x[1], x[2], x[3]));
-  __stcs(q + 1, make_float4(x[4], x[5], x[6], x[7]));
-}
-
-template <typename T, typename Tab>
-__device__ __forceinline__ const T *act_tensor(const void *base, const Tab &tab, int64_t b, int64_t E);
-template <>
-__device__ __forceinline__ const float *act_tensor<float, NoTable>(const void *base, const NoTable &, int64_t b,
-                                                                    int64_t E) {
-  return static_cast<const float *>(base) + b * E;
-}
-template <>
-__device__ __forceinline__ const __nv_bfloat16 *act_tensor<__nv_bfloat16, NoTable>(const void *base, const NoTable &,
-                                                                                    int64_t b, int64_t E) {
-  return static_cast<const __nv_bfloat16 *>(base) + b * E;
-}
-template <>
-__device__ __forceinline__ const float *act_tensor<float, PtrTable>(const void *, const PtrTable &tab, int64_t b,
-                                                                     int64_t) {
-  return static_cast<const float *>(tab.p[b]);
-}
-template <>
-__device__ __forceinline__ const __nv_bfloat16 *act_tensor<__nv_bfloat16, PtrTable>(const void *, const PtrTable &tab,
-                                                                                     int64_t b, int64_t) {
-  return static_cast<const __nv_bfloat16 *>(tab.p[b]);
-}
-
-// ---------------------------------------------------------------- reductions
-
-// Max over the team (all threads of the block call this together).
-__device__ __forceinline__ float team_max(float x, int team_log2, float *sm) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
-  if (team_log2 > 5) {
-    const int warp = threadIdx.x >> 5, wpt = 1 << (team_log2 - 5);
-    if ((threadIdx.x & 31) == 0) sm[warp] = x;
-    __syncthreads();
-    const int w0 = warp & ~(wpt - 1);
-    x = sm[w0];
-    for (int w = 1; w < wpt; w++) x = fmaxf(x, sm[w0 + w]);
-    __syncthreads();
-  }
-  return x;
-}
-
-__device__ __forceinline__ unsigned long long team_sum_u64(unsigned long long x, int team_log2,
-                                                           unsigned long long *sm) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
-  if (team_log2 > 5) {
-    const int warp = threadIdx.x >> 5, wpt = 1 << (team_log2 - 5);
-    if ((threadIdx.x & 31) == 0) sm[warp] = x;
-    __syncthreads();
-    const int w0 = warp & ~(wpt - 1);
-    x = sm[w0];
-    for (int w = 1; w < wpt; w++) x += sm[w0 + w];
-    __syncthreads();
-  }
-  return x;
-}
-
-// OR over aligned groups of G consecutive lanes (G a power of two <= 32).
-template <int G>
-__device__ __forceinline__ uint32_t group_or(uint32_t x) {
-#pragma unroll
-  for (int o = 1; o < G; o <<= 1) x |= __shfl_xor_sync(kFull, x, o);
-  return x;
-}
-
-// ---------------------------------------------------------------- SIGN1 scale
-
-// floor(ad * 2^sh_base) for a non-negative finite fp32 ad, exactly, from its
-// bits (sh_base = F - E with ad < 2^(E+1), so the result is < 2^63).
-__device__ __forceinline__ unsigned long long fixed_term(float ad, int sh_base) {
-  const uint32_t bits = __float_as_uint(ad);
-  int e = int(bits >> 23);
-  uint32_t mant = bits & 0x7fffffu;
-  if (e) mant |= 0x800000u; else e = 1;
-  const int sh = e - 150 + sh_base;
-  if (sh >= 0) return (unsigned long long)mant << sh;
-  const int rs = -sh;
-  return rs >= 24 ? 0ull : (unsigned long long)(mant >> rs);
-}
-
-// floor(log2 m) for a finite m > 0.
-__device__ __forceinline__ int floor_log2_f32(float m) {
-  const uint32_t bits = __float_as_uint(m);
-  const int e = int(bits >> 23);
-  if (e) return e - 127;
-  return (31 - __clz(bits & 0x7fffffu)) - 149;
-}
-
-// ---------------------------------------------------------------- mode traits
-
-enum { M_ID = CF_IDENTITY, M_S1 = CF_SIGN1, M_Q2 = CF_Q2, M_NM = CF_NM };
-
-// Bits of packed code per 8-element vector, and lanes per payload word.
-template <int MODE, int NM_M, int NM_N>
-struct Pack {
-  static constexpr int bpv = MODE == M_S1 ? 8 : MODE == M_Q2 ? 16 : MODE == M_NM ? (NM_M == 16 ? 2 * NM_N : 4 * NM_N) : 0;
-  static constexpr int G = bpv ? 32 / bpv : 1;
-};
-
-// Top-N (N <= 2) of |x[k]| over k in [k0, k0+cnt), key (|x| desc, index asc).
-template <int N>
-__device__ __forceinline__ void local_topn(const float (&x)[8], int k0, int cnt, float (&bv)[2], int (&bi)[2]) {
-  bv[0] = -1.0f; bv[1] = -1.0f; bi[0] = 0; bi[1] = 0;
-#pragma unroll
-  for (int k = 0; k < cnt; k++) {
-    const float a = fabsf(x[k0 + k]);
-    if (a > bv[0]) {
-      bv[1] = bv[0]; bi[1] = bi[0];
-      bv[0] = a; bi[0] = k;
-    } else if (N == 2 && a > bv[1]) {
-      bv[1] = a; bi[1] = k;
-    }
-  }
-}
-
-__device__ __forceinline__ bool better(float a, int ia, float b, int ib) { return a > b || (a == b && ia < ib); }
-
-// ---------------------------------------------------------------- encode kernel
-
-// The (< 16 byte) alignment padding of every tensor body is written as zero,
-// so the whole payload is defined.  One thread per tensor.
-__device__ __forceinline__ void zero_padding(const EncArgs &A) {
-  const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < A.batch; b += nthr) {
-    uint8_t *body = A.payload + kHdrBytes + b * A.body_bytes;
-    for (int64_t i = 0; i < A.padA_len; i++) body[A.padA_off + i] = 0;
-    for (int64_t i = 0; i < A.padB_len; i++) body[A.padB_off + i] = 0;
-  }
-}
-
-template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename Tab>
-__global__ void __launch_bounds__(kBlock) encode_kernel(const EncArgs A, const __grid_constant__ Tab tab) {
-  using P = Pack<MODE, NM_M, NM_N>;
-  __shared__ float sm_f[kBlock / 32];
-  __shared__ unsigned long long sm_u[kBlock / 32];
-
-  const int tlog = A.team_log2;
-  const int TEAM = 1 << tlog;
-  const int t = threadIdx.x & (TEAM - 1);
-  const int team = threadIdx.x >> tlog;
-  const int tpb = kBlock >> tlog;
-  const int64_t cols = A.cols;
-  const int64_t V = cols >> 3;
-  const int64_t E = A.rows * cols;
-  const int64_t nrows = (int64_t)A.batch * A.rows;
-  const int64_t n_rg = (nrows + tpb - 1) / tpb;
-
-  if (blockIdx.x == 0 && threadIdx.x < 16) reinterpret_cast<uint32_t *>(A.payload)[threadIdx.x] = A.hdr.w[threadIdx.x];
-  zero_padding(A);
-
-  for (int64_t rg = blockIdx.x; rg < n_rg; rg += gridDim.x) {
-    const int64_t gr = rg * tpb + team;
-    const bool row_ok = gr < nrows;
-    const int64_t b = row_ok ? gr / A.rows : 0;
-    const int64_t r = row_ok ? gr - b * A.rows : 0;
-    const T *arow = act_tensor<T, Tab>(A.a, tab, b, E) + r * cols;
-    float *hrow = A.ahat + (row_ok ? gr : 0) * cols;
-    float *erow = A.err + (row_ok ? gr : 0) * cols;
-    uint8_t *body = A.payload + kHdrBytes + b * A.body_bytes;
-
-    // ---- load the row (all loads issued before any use) ----
-    typename Act<T>::Raw ra[VPT];
-    float4 rh[VPT][2], re[VPT][2];
-#pragma unroll
-    for (int j = 0; j < VPT; j++) {
-      const int64_t v = t + ((int64_t)j << tlog);
-      if (row_ok && v < V) {
-        ra[j] = Act<T>::load(arow + v * 8);
-        const float4 *hp = reinterpret_cast<const float4 *>(hrow + v * 8);
-        rh[j][0] = __ldcs(hp);
-        rh[j][1] = __ldcs(hp + 1);
-        if (A.ef_explicit) {
-          const float4 *ep = reinterpret_cast<const float4 *>(erow + v * 8);
-          re[j][0] = __ldcs(ep);
-          re[j][1] = __ldcs(ep + 1);
-        } else {
-          re[j][0] = make_float4(0.f, 0.f, 0.f, 0.f);
-          re[j][1] = re[j][0];
-        }
-      } else {
-        ra[j] = typename Act<T>::Raw{};
-        rh[j][0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        rh[j][1] = rh[j][0];
-        re[j][0] = rh[j][0];
-        re[j][1] = rh[j][0];
-      }
-    }
-
-    // ---- residual with error feedback: D = (a - ahat) + e ----
-    float d[VPT][8], h[VPT][8];
-#pragma unroll
-    for (int j = 0; j < VPT; j++) {
-      float x[8];
-      Act<T>::to_f32(ra[j], x);
-      const float hv[8] = {rh[j][0].x, rh[j][0].y, rh[j][0].z, rh[j][0].w,
-                           rh[j][1].x, rh[j][1].y, rh[j][1].z, rh[j][1].w};
-      const float ev[8] = {re[j][0].x, re[j][0].y, re[j][0].z, re[j][0].w,
-                           re[j][1].x, re[j][1].y, re[j][1].z, re[j][1].w};
-#pragma unroll
-      for (int k = 0; k < 8; k++) {
-        h[j][k] = hv[k];
-        const float tt = __fsub_rn(x[k], hv[k]);
-        d[j][k] = A.ef_explicit ? __fadd_rn(tt, ev[k]) : tt;
-      }
-    }
-
-    // ---- encode; c[j][k] = C(D) from the encoded values ----
-    float c[VPT][8];
-    uint32_t cbits[VPT];
-#pragma unroll
-    for (int j = 0; j < VPT; j++) cbits[j] = 0;
-
-    if constexpr (MODE == M_ID) {
-#pragma unroll
-      for (int j = 0; j < VPT; j++) {
-        const int64_t v = t + ((int64_t)j << tlog);
-#pragma unroll
-        for (int k = 0; k < 8; k++) c[j][k] = d[j][k];
-        if (row_ok && v < V) store_f32x8(reinterpret_cast<float *>(body) + r * cols + v * 8, d[j]);
-      }
-    } else if constexpr (MODE == M_S1) {
-      float m = 0.0f;
-#pragma unroll
-      for (int j = 0; j < VPT; j++)
-#pragma unroll
-        for (int k = 0; k < 8; k++) m = fmaxf(m, fabsf(d[j][k]));
-      m = team_max(m, tlog, sm_f);
-      float S = 0.0f;
-      unsigned long long q = 0;
-      const int Ex = m > 0.0f ? floor_log2_f32(m) : 0;
-      const int shb = A.fx_F - Ex;
-      if (m > 0.0f) {
-#pragma unroll
-        for (int j = 0; j < VPT; j++)
-#pragma unroll
-          for (int k = 0; k < 8; k++) q += fixed_term(fabsf(d[j][k]), shb);
-      }
-      q = team_sum_u64(q, tlog, sm_u);
-      uint16_t sbits = 0;
-      if (m > 0.0f) {
-        // mean = fp64(Q) * 2^(E - F) / cols; the power of two scaling is exact
-        const double p2 = __hiloint2double((Ex - A.fx_F + 1023) << 20, 0);
-        const double mean = __ddiv_rn(__dmul_rn(__ull2double_rn(q), p2), (double)cols);
-        sbits = __bfloat16_as_ushort(__float2bfloat16_rn(__double2float_rn(mean)));
-        S = __uint_as_float((uint32_t)sbits << 16);
-      }
-      if (row_ok && t == 0) reinterpret_cast<uint16_t *>(body)[r] = sbits;
-#pragma unroll
-      for (int j = 0; j < VPT; j++) {
-        uint32_t byte = 0;
-#pragma unroll
-        for (int k = 0; k < 8; k++) {
-          const bool neg = d[j][k] < 0.0f;
-          byte |= (uint32_t)neg << k;
-          c[j][k] = neg ? -S : S;
-        }
-        const int64_t v = t + ((int64_t)j << tlog);
-        cbits[j] = byte << ((v % P::G) * P::bpv);
-      }
-    } else if constexpr (MODE == M_Q2) {
-      float m = 0.0f;
-#pragma unroll
-      for (int j = 0; j < VPT; j++)
-#pragma unroll
-        for (int k = 0; k < 8; k++) m = fmaxf(m, fabsf(d[j][k]));
-      m = team_max(m, tlog, sm_f);
-      const uint16_t sbits = __bfloat16_as_ushort(__float2bfloat16_rn(m));
-      const float S = __uint_as_float((uint32_t)sbits << 16);
-      if (row_ok && t == 0) reinterpret_cast<uint16_t *>(body)[r] = sbits;
-      float L[4];
-#pragma unroll
-      for (int qv = 0; qv < 4; qv++) L[qv] = __fdiv_rn(__fmul_rn((float)(2 * qv - 3), S), 3.0f);
-#pragma unroll
-      for (int j = 0; j < VPT; j++) {
-        uint32_t codes = 0;
-#pragma unroll
-        for (int k = 0; k < 8; k++) {
-          int qv = 0;
-          if (S != 0.0f) {
-            float u = __fmul_rn(__fdiv_rn(d[j][k], S), 1.5f);
-            u = __fadd_rn(u, 1.5f);
-            u = fminf(fmaxf(u, 0.0f), 3.0f);
-            qv = (int)rintf(u);
-          }
-          codes |= (uint32_t)qv << (2 * k);
-          c[j][k] = qv == 0 ? L[0] : qv == 1 ? L[1] : qv == 2 ? L[2] : L[3];
-        }
-        const int64_t v = t + ((int64_t)j << tlog);
-        cbits[j] = codes << ((v % P::G) * P::bpv);
-      }
-    } else {  // M_NM
-      const int64_t nblk_row = cols / NM_M;
-      uint16_t *vals = reinterpret_cast<uint16_t *>(body) + r * nblk_row * NM_N;
-#pragma unroll
-      for (int j = 0; j < VPT; j++) {
-        const int64_t v = t + ((int64_t)j << tlog);
-        const bool ok = row_ok && v < V;
-#pragma unroll
-        for (int k = 0; k < 8; k++) c[j][k] = 0.0f;
-        if constexpr (NM_M == 16) {
-          // a block of 16 columns spans the vector pair (v even, v odd) held by lanes (t, t^1)
-          float bv[2];
-          int bi[2];
-          local_topn<NM_N>(d[j], 0, 8, bv, bi);
-          const int half = int(v & 1);
-          float bd[2] = {d[j][0], d[j][0]};
-#pragma unroll
-          for (int k = 0; k < 8; k++) {
-            if (k == bi[0]) bd[0] = d[j][k];
-            if (k == bi[1]) bd[1] = d[j][k];
-          }
-          int gi[2] = {bi[0] + 8 * half, bi[1] + 8 * half};
-          float pv[2], pd[2];
-          int pi[2];
-#pragma unroll
-          for (int s = 0; s < 2; s++) {
-            pv[s] = __shfl_xor_sync(kFull, bv[s], 1);
-            pd[s] = __shfl_xor_sync(kFull, bd[s], 1);
-            pi[s] = __shfl_xor_sync(kFull, gi[s], 1);
-          }
-          // merge the two sorted candidate lists, keep the first NM_N
-          float kv[2];
-          int ki[2];
-          float kd[2];
-          {
-            int ia = 0, ib = 0;
-#pragma unroll
-            for (int s = 0; s < NM_N; s++) {
-              const float av = ia == 0 ? bv[0] : bv[1];
-              const int ai = ia == 0 ? gi[0] : gi[1];
-              const float ad = ia == 0 ? bd[0] : bd[1];
-              const float bvv = ib == 0 ? pv[0] : pv[1];
-              const int bii = ib == 0 ? pi[0] : pi[1];
-              const float bdd = ib == 0 ? pd[0] : pd[1];
-              if (better(av, ai, bvv, bii)) {
-                kv[s] = av; ki[s] = ai; kd[s] = ad; ia++;
-              } else {
-                kv[s] = bvv; ki[s] = bii; kd[s] = bdd; ib++;
-              }
-            }
-          }
-          (void)kv;
-          if (NM_N == 2 && ki[0] > ki[1]) {
-            const int ti = ki[0]; ki[0] = ki[1]; ki[1] = ti;
-            const float td = kd[0]; kd[0] = kd[1]; kd[1] = td;
-          }
-#pragma unroll
-          for (int k = 0; k < 8; k++) {
-            const int gk = k + 8 * half;
-            bool keep = gk == ki[0];
-            if (NM_N == 2) keep = keep || gk == ki[1];
-            if (keep) c[j][k] = __bfloat162float(__float2bfloat16_rn(d[j][k]));
-          }
-          if (half == 0) {
-            const int64_t blk = v >> 1;
-            uint32_t fields = 0;
-#pragma unroll
-            for (int s = 0; s < NM_N; s++) fields |= (uint32_t)ki[s] << (4 * s);
-            cbits[j] = fields << ((v % P::G) * P::bpv);
-            if (ok) {
-              if (NM_N == 1) {
-                vals[blk] = __bfloat16_as_ushort(__float2bfloat16_rn(kd[0]));
-              } else {
-                reinterpret_cast<uint32_t *>(vals)[blk] = pack_bf16x2(kd[0], kd[1]);
-              }
-            }
-          }
-        } else {  // NM_M == 4: two blocks inside the vector
-          uint32_t fields = 0;
-          uint16_t vb[4];
-#pragma unroll
-          for (int qb = 0; qb < 2; qb++) {
-            float bv[2];
-            int bi[2];
-            local_topn<NM_N>(d[j], 4 * qb, 4, bv, bi);
-            int ki[2] = {bi[0], bi[1]};
-            if (NM_N == 2 && ki[0] > ki[1]) { const int ti = ki[0]; ki[0] = ki[1]; ki[1] = ti; }
-#pragma unroll
-            for (int s = 0; s < NM_N; s++) {
-              float dv = d[j][4 * qb];
-#pragma unroll
-              for (int k = 1; k < 4; k++)
-                if (k == ki[s]) dv = d[j][4 * qb + k];
-              const __nv_bfloat16 bb = __float2bfloat16_rn(dv);
-              vb[qb * NM_N + s] = __bfloat16_as_ushort(bb);
-              fields |= (uint32_t)ki[s] << (2 * (qb * NM_N + s));
-#pragma unroll
-              for (int k = 0; k < 4; k++)
-                if (k == ki[s]) c[j][4 * qb + k] = __bfloat162float(bb);
-            }
-          }
-          cbits[j] = fields << ((v % P::G) * P::bpv);
-          if (ok) {
-            const int64_t blk0 = 2 * v;
-            if (NM_N == 1) {
-              reinterpret_cast<uint32_t *>(vals + blk0)[0] = (uint32_t)vb[0] | ((uint32_t)vb[1] << 16);
-            } else {
-              uint2 w;
-              w.x = (uint32_t)vb[0] | ((uint32_t)vb[1] << 16);
-              w.y = (uint32_t)vb[2] | ((uint32_t)vb[3] << 16);
-              reinterpret_cast<uint2 *>(vals + blk0 * 2)[0] = w;
-            }
-          }
-        }
-      }
-    }
-
-    // ---- packed code words: OR over the G lanes of a word, one store ----
-    if constexpr (P::bpv > 0) {
-      const int64_t W = V / P::G;
-      uint32_t *words = reinterpret_cast<uint32_t *>(body + A.sec1) + r * W;
-#pragma unroll
-      for (int j = 0; j < VPT; j++) {
-        const int64_t v = t + ((int64_t)j << tlog);
-        const uint32_t w = group_or<P::G>(cbits[j]);
-        if (row_ok && v < V && (v % P::G) == 0) words[v / P::G] = w;
-      }
-    }
-
-    // ---- error feedback and sender reconstruction ----
-#pragma unroll
-    for (int j = 0; j < VPT; j++) {
-      const int64_t v = t + ((int64_t)j << tlog);
-      if (row_ok && v < V) {
-        float en[8], hn[8];
-#pragma unroll
-        for (int k = 0; k < 8; k++) {
-          en[k] = __fsub_rn(d[j][k], c[j][k]);
-          hn[k] = __fadd_rn(h[j][k], c[j][k]);
-        }
-        store_f32x8(erow + v * 8, en);
-        store_f32x8(hrow + v * 8, hn);
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------- decode kernel
-
-template <typename Tab>
-__device__ __forceinline__ void *recon_tensor(void *base, const Tab &tab, int64_t b, int64_t bytes);
-template <>
-__device__ __forceinline__ void *recon_tensor<NoTable>(void *base, const NoTable &, int64_t b, int64_t bytes) {
-  return static_cast<uint8_t *>(base) + b * bytes;
-}
-template <>
-__device__ __forceinline__ void *recon_tensor<PtrTable>(void *, const PtrTable &tab, int64_t b, int64_t) {
-  return const_cast<void *>(tab.p[b]);
-}
-
-// Compare the payload header with the expected one; on a mismatch record the
-// status (block 0) and tell the caller to return.
-__device__ __forceinline__ bool header_ok(const DecArgs &A) {
-  __shared__ int bad;
-  if (threadIdx.x == 0) bad = 0;
-  __syncthreads();
-  if (threadIdx.x < 16) {
-    const uint32_t w = reinterpret_cast<const uint32_t *>(A.payload)[threadIdx.x];
-    if (w != A.expect.w[threadIdx.x]) atomicOr(&bad, 1);
-  }
-  __syncthreads();
-  if (bad) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(A.status, 1);
-    return false;
-  }
-  return true;
-}
-
-template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename Tab>
-__global__ void __launch_bounds__(kBlock) decode_kernel(const DecArgs A, const __grid_constant__ Tab tab) {
-  using P = Pack<MODE, NM_M, NM_N>;
-  if (!header_ok(A)) return;
-  const int tlog = A.team_log2;
-  const int TEAM = 1 << tlog;
-  const int t = threadIdx.x & (TEAM - 1);
-  const int team = threadIdx.x >> tlog;
-  const int tpb = kBlock >> tlog;
-  const int64_t cols = A.cols;
-  const int64_t V = cols >> 3;
-  const int64_t E = A.rows * cols;
-  const int64_t nrows = (int64_t)A.batch * A.rows;
-  const int64_t n_rg = (nrows + tpb - 1) / tpb;
-
-  for (int64_t rg = blockIdx.x; rg < n_rg; rg += gridDim.x) {
-    const int64_t gr = rg * tpb + team;
-    if (gr >= nrows) continue;  // no block-wide synchronisation below
-    const int64_t b = gr / A.rows;
-    const int64_t r = gr - b * A.rows;
-    const uint8_t *body = A.payload + kHdrBytes + b * A.body_bytes;
-    T *rrow = static_cast<T *>(recon_tensor<Tab>(A.recon, tab, b, E * (int64_t)sizeof(T))) + r * cols;
-    float *hrow = A.ahat + gr * cols;
-
-    float S = 0.0f, L[4] = {0.f, 0.f, 0.f, 0.f};
-    if constexpr (MODE == M_S1 || MODE == M_Q2) {
-      S = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(body)[r] << 16);
-      if constexpr (MODE == M_Q2) {
-#pragma unroll
-        for (int qv = 0; qv < 4; qv++) L[qv] = __fdiv_rn(__fmul_rn((float)(2 * qv - 3), S), 3.0f);
-      }
-    }
-    const int64_t W = P::bpv ? V / P::G : 0;
-    const uint32_t *words = reinterpret_cast<const uint32_t *>(body + A.sec1) + r * W;
-
-    float4 rh[VPT][2];
-    float c[VPT][8];
-#pragma unroll
-    for (int j = 0; j < VPT; j++) {
-      const int64_t v = t + ((int64_t)j << tlog);
-      if (v < V) {
-        const float4 *hp = reinterpret_cast<const float4 *>(hrow + v * 8);
-        rh[j][0] = __ldcs(hp);
-        rh[j][1] = __ldcs(hp + 1);
-        if constexpr (MODE == M_ID) {
-          load_f32x8(reinterpret_cast<const float *>(body) + r * cols + v * 8, c[j]);
-        } else if constexpr (MODE == M_S1) {
-          const uint32_t byte = (words[v / P::G] >> ((v % P::G) * P::bpv)) & 0xffu;
-#pragma unroll
-          for (int k = 0; k < 8; k++) c[j][k] = ((byte >> k) & 1u) ? -S : S;
-        } else if constexpr (MODE == M_Q2) {
-          const uint32_t codes = (words[v / P::G] >> ((v % P::G) * P::bpv)) & 0xffffu;
-#pragma unroll
-          for (int k = 0; k < 8; k++) {
-            const uint32_t qv = (codes >> (2 * k)) & 3u;
-            c[j][k] = qv == 0 ? L[0] : qv == 1 ? L[1] : qv == 2 ? L[2] : L[3];
-          }
-        } else {  // NM
-          const int64_t nblk_row = cols / NM_M;
-          const uint16_t *vals = reinterpret_cast<const uint16_t *>(body) + r * nblk_row * NM_N;
-#pragma unroll
-          for (int k = 0; k < 8; k++) c[j][k] = 0.0f;
-          if constexpr (NM_M == 16) {
-            const int64_t blk = v >> 1;
-            const int half = int(v & 1);
-            const int64_t v0 = blk * 2;  // even vector of the pair: owner of the fields
-            const uint32_t fields = (words[v0 / P::G] >> ((v0 % P::G) * P::bpv)) & ((1u << (4 * NM_N)) - 1u);
-#pragma unroll
-            for (int s = 0; s < NM_N; s++) {
-              const int idx = int((fields >> (4 * s)) & 15u);
-              const float val = __uint_as_float((uint32_t)vals[blk * NM_N + s] << 16);
-              if ((idx >> 3) == half) {
-#pragma unroll
-                for (int k = 0; k < 8; k++)
-                  if (k == (idx & 7)) c[j][k] = val;
-              }
-            }
-          } else {  // NM_M == 4
-            const uint32_t fields = (words[v / P::G] >> ((v % P::G) * P::bpv)) & ((1u << P::bpv) - 1u);
-#pragma unroll
-            for (int qb = 0; qb < 2; qb++)
-#pragma unroll
-              for (int s = 0; s < NM_N; s++) {
-                const int idx = int((fields >> (2 * (qb * NM_N + s))) & 3u);
-                const float val = __uint_as_float((uint32_t)vals[(2 * v + qb) * NM_N + s] << 16);
-#pragma unroll
-                for (int k = 0; k < 4; k++)
-                  if (k == idx) c[j][4 * qb + k] = val;
-              }
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < VPT; j++) {
-      const int64_t v = t + ((int64_t)j << tlog);
-      if (v < V) {
-        const float hv[8] = {rh[j][0].x, rh[j][0].y, rh[j][0].z, rh[j][0].w,
-                             rh[j][1].x, rh[j][1].y, rh[j][1].z, rh[j][1].w};
-        float hn[8];
-#pragma unroll
-        for (int k = 0; k < 8; k++) hn[k] = __fadd_rn(hv[k], c[j][k]);
-        store_f32x8(hrow + v * 8, hn);
-        Act<T>::store_f32(rrow + v * 8, hn);
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------- warm-up kernels
-
-// Step 0: payload body = raw a; ahat = fp32(a); e = 0.
-template <typename T, int VPT, typename Tab>
-__global__ void __launch_bounds__(kBlock) warm_encode_kernel(const EncArgs A, const __grid_constant__ Tab tab) {
-  const int tlog = A.team_log2;
-  const int TEAM = 1 << tlog;
-  const int t = threadIdx.x & (TEAM - 1);
-  const int team = threadIdx.x >> tlog;
-  const int tpb = kBlock >> tlog;
-  const int64_t cols = A.cols, V = cols >> 3, E = A.rows * cols;
-  const int64_t nrows = (int64_t)A.batch * A.rows;
-  const int64_t n_rg = (nrows + tpb - 1) / tpb;
-  if (blockIdx.x == 0 && threadIdx.x < 16) reinterpret_cast<uint32_t *>(A.payload)[threadIdx.x] = A.hdr.w[threadIdx.x];
-  for (int64_t rg = blockIdx.x; rg < n_rg; rg += gridDim.x) {
-    const int64_t gr = rg * tpb + team;
-    if (gr >= nrows) continue;
-    const int64_t b = gr / A.rows, r = gr - b * A.rows;
-    const T *arow = act_tensor<T, Tab>(A.a, tab, b, E) + r * cols;
-    T *prow = reinterpret_cast<T *>(A.payload + kHdrBytes + b * A.body_bytes) + r * cols;
-#pragma unroll
-    for (int j = 0; j < VPT; j++) {
-      const int64_t v = t + ((int64_t)j << tlog);
-      if (v < V) {
-        const typename Act<T>::Raw raw = Act<T>::load(arow + v * 8);
-        float x[8];
-        Act<T>::to_f32(raw, x);
-        Act<T>::store_raw(prow + v * 8, raw);
-        store_f32x8(A.ahat + gr * cols + v * 8, x);
-        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        store_f32x8(A.err + gr * cols + v * 8, z);
-      }
-    }
-  }
-}
-
-// Step 0 receiver: ahat = fp32(body); recon = body.
-template <typename T, int VPT, typename Tab>
-__global__ void __launch_bounds__(kBlock) warm_decode_kernel(const DecArgs A, const __grid_constant__ Tab tab) {
-  if (!header_ok(A)) return;
-  const int tlog = A.team_log2;
-  const int TEAM = 1 << tlog;
-  const int t = threadIdx.x & (TEAM - 1);
-  const int team = threadIdx.x >> tlog;
-  const int tpb = kBlock >> tlog;
-  const int64_t cols = A.cols, V = cols >> 3, E = A.rows * cols;
-  const int64_t nrows = (int64_t)A.batch * A.rows;
-  const int64_t n_rg = (nrows + tpb - 1) / tpb;
-  for (int64_t rg = blockIdx.x; rg < n_rg; rg += gridDim.x) {
-    const int64_t gr = rg * tpb + team;
-    if (gr >= nrows) continue;
-    const int64_t b = gr / A.rows, r = gr - b * A.rows;
-    const T *prow = reinterpret_cast<const T *>(A.payload + kHdrBytes + b * A.body_bytes) + r * cols;
-    T *rrow = static_cast<T *>(recon_tensor<Tab>(A.recon, tab, b, E * (int64_t)sizeof(T))) + r * cols;
-#pragma unroll
-    for (int j = 0; j < VPT; j++) {
-      const int64_t v = t + ((int64_t)j << tlog);
-      if (v < V) {
-        const typename Act<T>::Raw raw = Act<T>::load(prow + v * 8);
-        float x[8];
-        Act<T>::to_f32(raw, x);
-        store_f32x8(A.ahat + gr * cols + v * 8, x);
-        Act<T>::store_raw(rrow + v * 8, raw);
-      }
-    }
-  }
-}
-
 // ---------------------------------------------------------------- dispatch
 
-template <int MODE, int NM_M, int NM_N, typename T, typename Tab>
-const void *pick_encode(int vpt) {
-  switch (vpt) {
-    case 1: return reinterpret_cast<const void *>(&encode_kernel<MODE, T, 1, NM_M, NM_N, Tab>);
-    case 2: return reinterpret_cast<const void *>(&encode_kernel<MODE, T, 2, NM_M, NM_N, Tab>);
-    case 3: return reinterpret_cast<const void *>(&encode_kernel<MODE, T, 3, NM_M, NM_N, Tab>);
-    case 4: return reinterpret_cast<const void *>(&encode_kernel<MODE, T, 4, NM_M, NM_N, Tab>);
-  }
-  return nullptr;
-}
-
-template <int MODE, int NM_M, int NM_N, typename T, typename Tab>
-const void *pick_decode(int vpt) {
-  switch (vpt) {
-    case 1: return reinterpret_cast<const void *>(&decode_kernel<MODE, T, 1, NM_M, NM_N, Tab>);
-    case 2: return reinterpret_cast<const void *>(&decode_kernel<MODE, T, 2, NM_M, NM_N, Tab>);
-    case 3: return reinterpret_cast<const void *>(&decode_kernel<MODE, T, 3, NM_M, NM_N, Tab>);
-    case 4: return reinterpret_cast<const void *>(&decode_kernel<MODE, T, 4, NM_M, NM_N, Tab>);
-  }
-  return nullptr;
-}
-
-template <typename T, typename Tab>
-const void *kernel_for(bool enc, int mode, int nm_m, int nm_n, int vpt) {
-  switch (mode) {
-    case CF_IDENTITY: return enc ? pick_encode<M_ID, 0, 0, T, Tab>(vpt) : pick_decode<M_ID, 0, 0, T, Tab>(vpt);
-    case CF_SIGN1: return enc ? pick_encode<M_S1, 0, 0, T, Tab>(vpt) : pick_decode<M_S1, 0, 0, T, Tab>(vpt);
-    case CF_Q2: return enc ? pick_encode<M_Q2, 0, 0, T, Tab>(vpt) : pick_decode<M_Q2, 0, 0, T, Tab>(vpt);
-    case CF_NM:
-      if (nm_m == 16 && nm_n == 1) return enc ? pick_encode<M_NM, 16, 1, T, Tab>(vpt) : pick_decode<M_NM, 16, 1, T, Tab>(vpt);
-      if (nm_m == 16 && nm_n == 2) return enc ? pick_encode<M_NM, 16, 2, T, Tab>(vpt) : pick_decode<M_NM, 16, 2, T, Tab>(vpt);
-      if (nm_m == 4 && nm_n == 1) return enc ? pick_encode<M_NM, 4, 1, T, Tab>(vpt) : pick_decode<M_NM, 4, 1, T, Tab>(vpt);
-      if (nm_m == 4 && nm_n == 2) return enc ? pick_encode<M_NM, 4, 2, T, Tab>(vpt) : pick_decode<M_NM, 4, 2, T, Tab>(vpt);
-      return nullptr;
-  }
-  return nullptr;
-}
-
 const void *kernel_any(bool enc, int mode, int dtype, int nm_m, int nm_n, int vpt, bool table) {
-  if (dtype == CF_BF16)
-    return table ? kernel_for<__nv_bfloat16, PtrTable>(enc, mode, nm_m, nm_n, vpt)
-                 : kernel_for<__nv_bfloat16, NoTable>(enc, mode, nm_m, nm_n, vpt);
-  return table ? kernel_for<float, PtrTable>(enc, mode, nm_m, nm_n, vpt)
-               : kernel_for<float, NoTable>(enc, mode, nm_m, nm_n, vpt);
+  switch (mode) {
+    case CF_IDENTITY: return stream_kernel_id(enc, dtype, nm_m, nm_n, vpt, table);
+    case CF_SIGN1: return stream_kernel_s1(enc, dtype, nm_m, nm_n, vpt, table);
+    case CF_Q2: return stream_kernel_q2(enc, dtype, nm_m, nm_n, vpt, table);
+    case CF_NM: return stream_kernel_nm(enc, dtype, nm_m, nm_n, vpt, table);
+  }
+  return nullptr;
 }
 
 template <typename T, typename Tab>
@@ -823,39 +65,49 @@ const void *warm_any(bool enc, int dtype, int vpt, bool table) {
 }
 
 template <typename Args>
-cudaError_t launch(const void *fn, int grid, const Args &args, const PtrTable *tab, cudaStream_t st) {
+cudaError_t launch(const void *fn, int grid, size_t smem, const Args &args, const PtrTable *tab, cudaStream_t st) {
   if (!fn) return cudaErrorInvalidDeviceFunction;
   if (grid < 1) grid = 1;
   NoTable none;
   void *params[2] = {const_cast<Args *>(&args), tab ? const_cast<PtrTable *>(tab) : static_cast<void *>(&none)};
-  return cudaLaunchKernel(fn, dim3(grid), dim3(kBlock), params, 0, st);
+  return cudaLaunchKernel(fn, dim3(grid), dim3(kBlock), params, smem, st);
 }
 
-int occupancy(const void *fn) {
+int occupancy(const void *fn, size_t smem) {
   int n = 0;
-  if (!fn || cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kBlock, 0) != cudaSuccess) return 1;
+  if (!fn || cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kBlock, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 1;
+  }
   return n > 0 ? n : 1;
 }
 
 }  // namespace
 
 // Choose threads per row (a power of two >= 32) and vectors per thread
-// (1..4) so that TEAM * VPT covers cols/8 with the least idle lanes, then
-// size each persistent grid as (resident blocks per SM) x (SM count),
-// capped by the number of row groups.
+// (1..4) so that TEAM * VPT covers cols/8 with the fewest idle lanes (ties:
+// 128 threads per row, then wider teams), then size each persistent grid as
+// (resident blocks per SM) x (SM count), capped by the number of row groups.
 int stream_config(int mode, int dtype, int nm_m, int nm_n, int64_t rows, int64_t cols, int batch, int sm_count,
-                  StreamCfg *cfg) {
+                  int ef_explicit, StreamCfg *cfg) {
+  (void)ef_explicit;
   const int64_t V = cols / 8;
   int best_t = -1, best_v = 0;
-  int64_t best_waste = 0;
+  int64_t best_key[3] = {0, 0, 0};
   for (int vpt = 4; vpt >= 1; vpt--) {
-    int64_t need = (V + vpt - 1) / vpt;
+    const int64_t need = (V + vpt - 1) / vpt;
     int tl = 5;
     while ((1 << tl) < need) tl++;
     if (tl > 8) continue;
-    const int64_t waste = ((int64_t)1 << tl) * vpt - V;
-    if (best_t < 0 || waste < best_waste) {
-      best_t = tl; best_v = vpt; best_waste = waste;
+    const int64_t key[3] = {((int64_t)1 << tl) * vpt - V, tl > 7 ? tl - 7 : 7 - tl, -tl};
+    bool better = best_t < 0;
+    for (int k = 0; !better && k < 3; k++) {
+      if (key[k] < best_key[k]) better = true;
+      if (key[k] != best_key[k]) break;
+    }
+    if (better) {
+      best_t = tl; best_v = vpt;
+      for (int k = 0; k < 3; k++) best_key[k] = key[k];
     }
   }
   if (best_t < 0) return CF_ERR_SHAPE;
@@ -863,38 +115,37 @@ int stream_config(int mode, int dtype, int nm_m, int nm_n, int64_t rows, int64_t
   cfg->vpt = best_v;
   const int64_t tpb = kBlock >> best_t;
   const int64_t n_rg = ((int64_t)batch * rows + tpb - 1) / tpb;
-  auto grid_of = [&](const void *fn) -> int {
-    const int64_t g = (int64_t)occupancy(fn) * sm_count;
-    return (int)(g < n_rg ? g : n_rg);
-  };
+  auto cap = [&](int64_t g) -> int { return (int)(g < n_rg ? g : n_rg); };
+  cfg->enc_grid = cfg->dec_grid = 1;
   if (mode != CF_LOWRANK) {
-    cfg->enc_grid = grid_of(kernel_any(true, mode, dtype, nm_m, nm_n, best_v, false));
-    cfg->dec_grid = grid_of(kernel_any(false, mode, dtype, nm_m, nm_n, best_v, false));
-  } else {
-    cfg->enc_grid = cfg->dec_grid = 1;
+    const void *efn = kernel_any(true, mode, dtype, nm_m, nm_n, best_v, false);
+    const void *dfn = kernel_any(false, mode, dtype, nm_m, nm_n, best_v, false);
+    if (!efn || !dfn) return CF_ERR_UNSUPPORTED;
+    cfg->enc_grid = cap((int64_t)occupancy(efn, 0) * sm_count);
+    cfg->dec_grid = cap((int64_t)occupancy(dfn, 0) * sm_count);
   }
-  cfg->warm_grid = grid_of(warm_any(true, dtype, best_v, false));
+  cfg->warm_grid = cap((int64_t)occupancy(warm_any(true, dtype, best_v, false), 0) * sm_count);
   return CF_OK;
 }
 
 cudaError_t launch_encode(int mode, int dtype, int nm_m, int nm_n, const StreamCfg &cfg, const EncArgs &args,
                           const PtrTable *tab, cudaStream_t st) {
-  return launch(kernel_any(true, mode, dtype, nm_m, nm_n, cfg.vpt, tab != nullptr), cfg.enc_grid, args, tab, st);
+  return launch(kernel_any(true, mode, dtype, nm_m, nm_n, cfg.vpt, tab != nullptr), cfg.enc_grid, 0, args, tab, st);
 }
 
 cudaError_t launch_decode(int mode, int dtype, int nm_m, int nm_n, const StreamCfg &cfg, const DecArgs &args,
                           const PtrTable *tab, cudaStream_t st) {
-  return launch(kernel_any(false, mode, dtype, nm_m, nm_n, cfg.vpt, tab != nullptr), cfg.dec_grid, args, tab, st);
+  return launch(kernel_any(false, mode, dtype, nm_m, nm_n, cfg.vpt, tab != nullptr), cfg.dec_grid, 0, args, tab, st);
 }
 
 cudaError_t launch_warm_encode(int dtype, const StreamCfg &cfg, const EncArgs &args, const PtrTable *tab,
                                cudaStream_t st) {
-  return launch(warm_any(true, dtype, cfg.vpt, tab != nullptr), cfg.warm_grid, args, tab, st);
+  return launch(warm_any(true, dtype, cfg.vpt, tab != nullptr), cfg.warm_grid, 0, args, tab, st);
 }
 
 cudaError_t launch_warm_decode(int dtype, const StreamCfg &cfg, const DecArgs &args, const PtrTable *tab,
                                cudaStream_t st) {
-  return launch(warm_any(false, dtype, cfg.vpt, tab != nullptr), cfg.warm_grid, args, tab, st);
+  return launch(warm_any(false, dtype, cfg.vpt, tab != nullptr), cfg.warm_grid, 0, args, tab, st);
 }
 
 }  // namespace cfi

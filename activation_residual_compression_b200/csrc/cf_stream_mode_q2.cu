@@ -1,0 +1,13 @@
+// cf_stream_mode_q2.cu -- instantiations of the streaming kernels for the
+// 2-bit mode (one translation unit per mode so they compile in parallel).
+#include "cf_stream_kernels.cuh"
+
+namespace cfi {
+
+const void *stream_kernel_q2(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table) {
+  (void)nm_m;
+  (void)nm_n;
+  return pick_any<M_Q2, 0, 0>(enc, dtype, vpt, table);
+}
+
+}  // namespace cfi

@@ -81,6 +81,17 @@ def decode_bytes(mode, rows, cols, kw, act_size=2):
     return E * (4 + 4 + act_size) + 64 + _payload_body(mode, rows, cols, kw)
 
 
+def _kernel_sources_sha256():
+    """Hash of the streaming kernels' sources (the ncu traffic figure is only
+    valid for the kernels it was taken on)."""
+    csrc = os.path.join(ROOT, "activation_residual_compression_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        if f.startswith("cf_stream"):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()
+
+
 def _traffic_record():
     """dram read+write bytes per encode launch from the committed ncu summary,
     valid only while the kernel source is unchanged."""
@@ -89,8 +100,7 @@ def _traffic_record():
         return None
     with open(p) as f:
         d = json.load(f)
-    src = os.path.join(ROOT, "activation_residual_compression_b200", "csrc", "cf_stream.cu")
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    h = _kernel_sources_sha256()
     if d.get("source_sha256") != h:
         return None
     return d

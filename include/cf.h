@@ -54,8 +54,10 @@
  *     CF_IDENTITY: D as fp32 [rows][cols]
  *     CF_SIGN1  : scale bf16 [rows] (pad 16) | bits u32 [rows][cols/32];
  *                 bit (i mod 32) of word i/32 is 1 iff D_i < 0;
- *                 C_i = bit ? -S : +S with S = bf16(mean_i |D_i|), the mean
- *                 taken as an exact fixed-point sum (order independent)
+ *                 C_i = bit ? -S : +S with S = bf16(fp32(mean_i |D_i|)),
+ *                 the mean taken as an exact fixed-point sum (order
+ *                 independent): E = floor(log2 max|D|), q_i =
+ *                 floor(|D_i| 2^(31-E)), mean = fp64(sum q_i) 2^(E-31) / cols
  *     CF_Q2     : scale bf16 [rows] (pad 16) | codes u32 [rows][cols/16];
  *                 code of column i in bits 2(i mod 16).. of word i/16;
  *                 S = bf16(max |D|), u = (D/S)*1.5 + 1.5 clamped to [0,3],
@@ -101,6 +103,7 @@ extern "C" {
 #define CF_ERR_ALIGN (-8)        /* a pointer is not 16-byte aligned */
 #define CF_ERR_STATE (-9)        /* handle is not a live state (destroyed or foreign) */
 #define CF_ERR_SIZE (-10)        /* a host buffer size does not match */
+#define CF_ERR_TIMEOUT (-11)     /* (device) a bounded wait for an asynchronous copy gave up */
 
 /* ---- enumerations ---------------------------------------------------- */
 typedef enum { CF_IDENTITY = 0, CF_SIGN1 = 1, CF_Q2 = 2, CF_NM = 3, CF_LOWRANK = 4 } cf_mode;
@@ -177,7 +180,9 @@ CF_API int cf_encode_batched(cf_state *s, const void *const *a_ptrs, void *paylo
 CF_API int cf_decode_batched(cf_state *s, const void *payload, void *const *recon_ptrs, void *stream);
 
 /* Synchronises `stream`, then returns the state's sticky device status:
- * CF_OK, or CF_ERR_DESYNC after a payload that did not match this receiver.
+ * CF_OK; CF_ERR_DESYNC after a payload that did not match this receiver;
+ * CF_ERR_TIMEOUT if a kernel's bounded wait for one of its own asynchronous
+ * copies gave up (the kernel then returned early; its outputs are not valid).
  * Returns CF_ERR_CUDA if the stream reports an error. */
 CF_API int cf_status(cf_state *s, void *stream);
 

@@ -82,13 +82,6 @@ uint16_t orc_bf16_from_f32(float x)
 
 float orc_f32_from_bf16(uint16_t h) { return u2f((uint32_t)h << 16); }
 
-static int ceil_log2_i64(int64_t n)
-{
-    int c = 0;
-    while (((int64_t)1 << c) < n) c++;
-    return c;
-}
-
 static int ilog2_i(int m)
 {
     int c = 0;
@@ -103,14 +96,17 @@ static size_t pad16(size_t b) { return (b + 15u) & ~(size_t)15u; }
 /* ------------------------------------------------------------------ */
 
 /* SIGN1 scale: bf16(fp32(mean |d_i|)).  The mean is made independent of the
- * summation order by summing exact fixed-point values:
+ * summation order by summing exact fixed-point values with 31 fraction bits
+ * below the row maximum's leading bit:
  *   m = max|d|; if m == 0 the scale is 0
- *   E = floor(log2 m), F = 62 - ceil(log2 n)
+ *   E = floor(log2 m), F = 31
  *   q_i = floor(|d_i| * 2^(F-E))   (exact: a 24-bit significand scaled by a
- *                                   power of two, then floored)
- *   Q = sum q_i in uint64           (q_i < 2^(F+1), so Q < 2^63: no overflow)
- *   mean = fp64(Q) * 2^(E-F) / n    (fp64 round-to-nearest)
+ *                                   power of two, then floored; q_i < 2^32)
+ *   Q = sum q_i in uint64           (exact for n < 2^32)
+ *   mean = fp64(Q) * 2^(E-F) / n    (fp64 round-to-nearest; Q < 2^53 is exact)
+ * The truncation moves the mean by less than 2^(E-F) <= n 2^-31 of itself.
  * The L2-optimal scale for sign codes is mean|d| (argmin_s sum (d - s sgn d)^2). */
+#define ORC_SIGN1_F 31
 uint16_t orc_sign1_scale(const float *d, int64_t n)
 {
     float m = 0.0f;
@@ -122,7 +118,7 @@ uint16_t orc_sign1_scale(const float *d, int64_t n)
     int k;
     frexp((double)m, &k);                 /* m = f * 2^k, f in [0.5, 1) */
     int E = k - 1;
-    int F = 62 - ceil_log2_i64(n);
+    int F = ORC_SIGN1_F;
     uint64_t Q = 0;
     for (int64_t i = 0; i < n; i++) {
         double s = ldexp((double)fabsf(d[i]), F - E);

@@ -65,10 +65,10 @@ def test_tiny_config_bit_exact(mode):
 # ----------------------------------------------------------------------------- shapes / modes
 
 CASES = [
-    ("identity", {}, [64, 200, 3072]),
+    ("identity", {}, [64, 200, 3072, 8192]),
     ("sign1", {}, [32, 96, 640, 1920, 3072, 8192]),
     ("q2", {}, [16, 48, 1920, 3072, 8192]),
-    ("nm", {"nm_n": 1, "nm_m": 16}, [128, 1920, 3072]),
+    ("nm", {"nm_n": 1, "nm_m": 16}, [128, 1920, 3072, 8192]),
     ("nm", {"nm_n": 2, "nm_m": 16}, [64, 1920, 3072]),
     ("nm", {"nm_n": 1, "nm_m": 4}, [64, 640, 3072]),
     ("nm", {"nm_n": 2, "nm_m": 4}, [32, 96, 3072]),
@@ -218,5 +218,37 @@ def test_cogvideox_full_step_sampled_rows():
                 assert np.array_equal(cw_g, cw_o), (t, b)
             del a, parts
         assert pair.guards_ok()
+    finally:
+        pair.close()
+
+
+def test_q2_decision_boundaries_bit_exact():
+    """Residuals at and a few ulps around the 2-bit decision boundaries (-2S/3, 0,
+    +2S/3), where the kernel's fast code path hands over to the exact division
+    chain, must still match the oracle bit for bit."""
+    rows, cols = 24, 256
+    rng = np.random.default_rng(31)
+    a1 = np.zeros((rows, cols), np.float32)
+    for r in range(rows):
+        S = np.float32(rng.choice([1.5, 0.75, 3.0, 1.0, 0.1, 7.0, 2.0 ** -60, 2.0 ** 60]))
+        a1[r, 0] = S                                  # the row maximum: S = bf16(S) = S
+        two3 = np.float32(2.0 * float(S) / 3.0)
+        cand = []
+        for base in (two3, -two3, np.float32(0.0)):
+            x = base
+            for _ in range(6):
+                x = np.nextafter(x, np.float32(-np.inf))
+            for _ in range(13):
+                cand.append(x)
+                x = np.nextafter(x, np.float32(np.inf))
+        cand = np.array(cand, np.float32)
+        a1[r, 1:1 + len(cand)] = cand
+        a1[r, 1 + len(cand):] = (rng.uniform(-1, 1, cols - 1 - len(cand)) * float(S)).astype(np.float32)
+    seq = [np.zeros((rows, cols), np.float32), a1, a1 * np.float32(0.5)]
+    pair = GpuPair(rows, cols, "q2", dtype="f32")
+    orc = oracle.Oracle(rows, cols, "q2", dtype="f32")
+    it = iter(seq)
+    try:
+        _run_and_compare(pair, orc, lambda: torch.from_numpy(next(it)).cuda().unsqueeze(0), len(seq))
     finally:
         pair.close()
