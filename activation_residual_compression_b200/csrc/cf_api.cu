@@ -115,12 +115,14 @@ int validate(int64_t rows, int64_t cols, int mode, const cf_params *p) {
     if (((cols / p->nm_m) * p->nm_n * ilog2(p->nm_m)) % 32) return CF_ERR_SHAPE;
   }
   if (mode == CF_LOWRANK) {
+    if (p->rank < 1 || p->rank > kMaxRank || p->rank > rows || p->rank > cols) return CF_ERR_SHAPE;
+    if (rows % 128 || cols % 128) return CF_ERR_SHAPE;
+    if (p->iters < 1 || p->iters > 2) return CF_ERR_UNSUPPORTED;
+    if (p->lr_int4 != 0 && p->lr_int4 != 1) return CF_ERR_ARG;
+    if (p->batch != 1) return CF_ERR_UNSUPPORTED;
     LowrankPlan plan{};
     lowrank_plan(rows, cols, *p, &plan);
     if (!plan.supported) return CF_ERR_UNSUPPORTED;
-    if (p->rank < 1 || p->rank > kMaxRank || p->rank > rows || p->rank > cols) return CF_ERR_SHAPE;
-    if (p->iters < 1 || p->iters > 2) return CF_ERR_UNSUPPORTED;
-    if (p->lr_int4 != 0 && p->lr_int4 != 1) return CF_ERR_ARG;
   }
   return CF_OK;
 }
@@ -256,7 +258,7 @@ int do_encode(cf_state *s, const void *a, const PtrTable *tab, void *payload, cu
   if (warm) {
     e = launch_warm_encode(s->p.dtype, s->cfg, A, tab, st);
   } else if (s->mode == CF_LOWRANK) {
-    e = lowrank_encode(s->lr, A, tab, s->vprev, s->lr_scratch, s->p.seed, st);
+    e = lowrank_encode(s->lr, A, tab, s->vprev, s->step, s->p.seed, st);
   } else {
     e = launch_encode(s->mode, s->p.dtype, s->p.nm_m, s->p.nm_n, s->cfg, A, tab, st);
   }
@@ -278,7 +280,7 @@ int do_decode(cf_state *s, const void *payload, void *recon, const PtrTable *tab
   if (warm) {
     e = launch_warm_decode(s->p.dtype, s->cfg, A, tab, st);
   } else if (s->mode == CF_LOWRANK) {
-    e = lowrank_decode(s->lr, A, tab, s->lr_scratch, st);
+    e = lowrank_decode(s->lr, A, tab, st);
   } else {
     e = launch_decode(s->mode, s->p.dtype, s->p.nm_m, s->p.nm_n, s->cfg, A, tab, st);
   }
@@ -409,6 +411,14 @@ int cf_create(int64_t rows, int64_t cols, int mode, const cf_params *p, cf_state
   s->err = p->role == CF_SENDER ? reinterpret_cast<float *>(base + c.err) : nullptr;
   s->vprev = (p->role == CF_SENDER && mode == CF_LOWRANK) ? reinterpret_cast<float *>(base + c.vprev) : nullptr;
   s->lr_scratch = mode == CF_LOWRANK ? static_cast<void *>(base + c.lr) : nullptr;
+  if (mode == CF_LOWRANK) {
+    const int rc2 = lowrank_bind(&s->lr, s->lr_scratch);
+    if (rc2 != CF_OK) {
+      if (s->own_slab) cudaFree(s->slab);
+      delete s;
+      return rc2;
+    }
+  }
   if (cudaMemsetAsync(s->slab, 0, c.total, 0) != cudaSuccess || cudaStreamSynchronize(0) != cudaSuccess) {
     (void)cudaGetLastError();
     if (s->own_slab) cudaFree(s->slab);

@@ -1,8 +1,786 @@
-// cf_lowrank.cu -- low-rank mode of libcf (not yet implemented: creation of
-// a CF_LOWRANK state is rejected with CF_ERR_UNSUPPORTED).
+// cf_lowrank.cu -- low-rank mode of libcf on sm_100a.
+//
+// Method: "Accelerating Parallel Diffusion Model Serving with Residual
+// Compression", section "Key design: low-rank strategy for extreme ratios":
+// the residual D (with error feedback) is approximated as U V^T by
+// warm-started subspace iteration instead of an SVD, and U, V are quantised
+// to INT4 so that more rank fits the same bandwidth.  One iteration is
+//     Y = D V;  Q = orth(Y);  V = D^T Q          (U = Q is transmitted)
+// with V warm-started from the previous step's V.  orth is the thin-QR
+// factor with positive diagonal, computed by CholeskyQR2 in fp64 (unique for
+// full column rank, so it agrees with a Householder QR up to rounding);
+// columns with R_kk <= 1e-6 R_00 are rank deficient and set to zero.
+//
+// GEMMs: the two thin products (N = rank padded to a multiple of 16) and the
+// reconstruction C = U V^T run on the 5th-generation tensor cores (tcgen05
+// MMA, operands staged by TMA in 128-byte swizzled K-major tiles, fp32
+// accumulators in tensor memory).  Operands are bf16 pairs x = hi + lo
+// (hi = bf16(x), lo = bf16(x - hi)), and each product sums hi*hi + hi*lo +
+// lo*hi, which keeps about 16 significant bits: enough that the INT4 codes
+// the GPU picks agree with an fp64 computation except near rounding ties.
+// The reconstruction is one deterministic kernel run by both the sender and
+// the receiver on operands dequantised from the payload bytes, so sender and
+// receiver reconstructions are bit-identical.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+
 #include "cf_lowrank.h"
+#include "cf_umma.cuh"
 
 namespace cfi {
+namespace {
+
+constexpr int kTileM = 128;     // UMMA M and TMA box rows of the A operand
+constexpr int kTileK = 64;      // bf16 per 128-byte swizzled row
+constexpr int kReconN = 128;    // N of a reconstruction tile
+constexpr int kGramRows = 64;   // rows per partial Gram block
+constexpr int kStatusDesync = 1;
+constexpr int kStatusTimeout = 2;
+
+size_t pad256(size_t b) { return (b + 255u) & ~(size_t)255u; }
+size_t pad16(size_t b) { return (b + 15u) & ~(size_t)15u; }
+
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bfloat16 &lo) {
+  hi = __float2bfloat16_rn(x);
+  lo = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
+}
+
+// Header check for the receiver's kernels (same rule as the streaming decode).
+__device__ __forceinline__ bool lr_header_ok(const uint8_t *payload, const Header &expect, int *status) {
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  if (threadIdx.x < 16) {
+    const uint32_t w = reinterpret_cast<const uint32_t *>(payload)[threadIdx.x];
+    if (w != expect.w[threadIdx.x]) atomicOr(&bad, 1);
+  }
+  __syncthreads();
+  if (bad) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) atomicOr(status, kStatusDesync);
+    return false;
+  }
+  return true;
+}
+
+// splitmix64 (Steele, Lea, Flood; Vigna's public-domain reference).
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9e3779b97f4a7c15ull;
+  z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ull;
+  z = (z ^ (z >> 27)) * 0x94d049bb133111ebull;
+  return z ^ (z >> 31);
+}
+
+// First step's V (the pages leave it open): 2 * (splitmix64(seed ^ (j r + k)) >> 40) * 2^-24 - 1.
+__device__ __forceinline__ float v0_entry(uint64_t seed, int64_t j, int r, int k) {
+  const uint64_t z = splitmix64(seed ^ (uint64_t)(j * (int64_t)r + k));
+  const double u = (double)(z >> 40) * (1.0 / 16777216.0);
+  return (float)(2.0 * u - 1.0);
+}
+
+// ---------------------------------------------------------------- V preparation
+
+// Vt (split bf16, [rp][cols]) from the warm start: the previous step's V
+// (fp32 [cols][r]), or V0 on the first step and for any all-zero column.
+__global__ void __launch_bounds__(256) lr_vprep_kernel(const float *vprev, int64_t cols, int r, int rp, int first,
+                                                       uint64_t seed, __nv_bfloat16 *vthi, __nv_bfloat16 *vtlo) {
+  const int k = blockIdx.x;
+  __shared__ int nonzero;
+  if (threadIdx.x == 0) nonzero = 0;
+  __syncthreads();
+  if (k < r && !first) {
+    int nz = 0;
+    for (int64_t j = threadIdx.x; j < cols; j += blockDim.x) nz |= vprev[j * r + k] != 0.0f;
+    if (__syncthreads_or(nz) && threadIdx.x == 0) nonzero = 1;
+  }
+  __syncthreads();
+  const bool use_prev = nonzero != 0;
+  for (int64_t j = threadIdx.x; j < cols; j += blockDim.x) {
+    float x = 0.0f;
+    if (k < r) x = use_prev ? vprev[j * r + k] : v0_entry(seed, j, r, k);
+    __nv_bfloat16 hi, lo;
+    split_bf16(x, hi, lo);
+    vthi[(int64_t)k * cols + j] = hi;
+    vtlo[(int64_t)k * cols + j] = lo;
+  }
+}
+
+// ---------------------------------------------------------------- residual pass
+
+// D = (a - ahat) + e for a 64 x 64 tile, written as split bf16 both
+// row-major ([rows][cols], the K-major A operand of Y = D V) and transposed
+// ([cols][rows], the K-major A operand of V = D^T Q).  The fp32 D is not
+// stored: the reconstruction pass recomputes it bit for bit.
+template <typename T>
+__global__ void __launch_bounds__(256) lr_delta_kernel(const T *a, const float *ahat, const float *err, int ef_explicit,
+                                                       int64_t rows, int64_t cols, __nv_bfloat16 *dhi,
+                                                       __nv_bfloat16 *dlo, __nv_bfloat16 *dthi,
+                                                       __nv_bfloat16 *dtlo) {
+  __shared__ __nv_bfloat16 shi[64][72];
+  __shared__ __nv_bfloat16 slo[64][72];
+  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    const int lr = ty + 16 * i;
+    const int64_t off = (r0 + lr) * cols + c0 + 4 * tx;
+    float x[4];
+    if constexpr (sizeof(T) == 2) {
+      const uint2 raw = *reinterpret_cast<const uint2 *>(a + off);
+      x[0] = __uint_as_float(raw.x << 16);
+      x[1] = __uint_as_float(raw.x & 0xffff0000u);
+      x[2] = __uint_as_float(raw.y << 16);
+      x[3] = __uint_as_float(raw.y & 0xffff0000u);
+    } else {
+      const float4 f = *reinterpret_cast<const float4 *>(a + off);
+      x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+    }
+    const float4 h = *reinterpret_cast<const float4 *>(ahat + off);
+    const float4 e = ef_explicit ? *reinterpret_cast<const float4 *>(err + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float hv[4] = {h.x, h.y, h.z, h.w}, ev[4] = {e.x, e.y, e.z, e.w};
+    __nv_bfloat16 hi[4], lo[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const float tt = __fsub_rn(x[k], hv[k]);
+      const float d = ef_explicit ? __fadd_rn(tt, ev[k]) : tt;
+      split_bf16(d, hi[k], lo[k]);
+      shi[lr][4 * tx + k] = hi[k];
+      slo[lr][4 * tx + k] = lo[k];
+    }
+    uint2 ph, pl;
+    ph.x = (uint32_t)__bfloat16_as_ushort(hi[0]) | ((uint32_t)__bfloat16_as_ushort(hi[1]) << 16);
+    ph.y = (uint32_t)__bfloat16_as_ushort(hi[2]) | ((uint32_t)__bfloat16_as_ushort(hi[3]) << 16);
+    pl.x = (uint32_t)__bfloat16_as_ushort(lo[0]) | ((uint32_t)__bfloat16_as_ushort(lo[1]) << 16);
+    pl.y = (uint32_t)__bfloat16_as_ushort(lo[2]) | ((uint32_t)__bfloat16_as_ushort(lo[3]) << 16);
+    *reinterpret_cast<uint2 *>(dhi + off) = ph;
+    *reinterpret_cast<uint2 *>(dlo + off) = pl;
+  }
+  __syncthreads();
+  // transposed: output row c0 + oc holds rows r0 .. r0 + 63 of column oc
+  const int oc = threadIdx.x >> 2, part = threadIdx.x & 3;
+  uint32_t wh[8], wl[8];
+#pragma unroll
+  for (int k = 0; k < 8; k++) {
+    const int rr = part * 16 + 2 * k;
+    wh[k] = (uint32_t)__bfloat16_as_ushort(shi[rr][oc]) | ((uint32_t)__bfloat16_as_ushort(shi[rr + 1][oc]) << 16);
+    wl[k] = (uint32_t)__bfloat16_as_ushort(slo[rr][oc]) | ((uint32_t)__bfloat16_as_ushort(slo[rr + 1][oc]) << 16);
+  }
+  const int64_t toff = (c0 + oc) * rows + r0 + part * 16;
+  uint4 *th = reinterpret_cast<uint4 *>(dthi + toff);
+  uint4 *tl = reinterpret_cast<uint4 *>(dtlo + toff);
+  th[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+  th[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+  tl[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+  tl[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
+}
+
+// ---------------------------------------------------------------- thin GEMM (tcgen05)
+
+struct ThinArgs {
+  float *out;     // [splits][M][n]
+  int64_t M;      // rows of A
+  int n;          // columns of the product (UMMA N, multiple of 16, <= 128)
+  int kblocks;    // K / 64
+  int splits;
+  int stages;
+  int *status;
+};
+
+// out[s] = A[:, K_s] * B[:, K_s]^T for the s-th K range, A = ahi + alo
+// ([M][K] bf16, K-major), B = bhi + blo ([n][K] bf16, K-major), summing the
+// products hi*hi + hi*lo + lo*hi in fp32 tensor memory.  One CTA per
+// (128-row tile, K split); warp 0 lane 0 streams tiles with TMA into a ring
+// of shared-memory stages, warp 1 lane 0 issues the MMAs, all four warps
+// read the accumulator back (one row per thread) and write the partial.
+__global__ void __launch_bounds__(128, 1)
+    lr_thin_gemm_kernel(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
+                        const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
+                        const ThinArgs A) {
+  extern __shared__ __align__(1024) uint8_t dsm[];
+  __shared__ __align__(8) uint64_t full[4], empty[4], accb;
+  __shared__ uint32_t tmem_base;
+  uint8_t *sm = reinterpret_cast<uint8_t *>(((uintptr_t)dsm + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kTileM;
+  const int s = blockIdx.y;
+  const int kb0 = (int)((int64_t)s * A.kblocks / A.splits);
+  const int kb1 = (int)((int64_t)(s + 1) * A.kblocks / A.splits);
+  const int nk = kb1 - kb0;
+  const uint32_t a_bytes = kTileM * kTileK * 2;         // 16 KiB
+  const uint32_t b_bytes = (uint32_t)A.n * kTileK * 2;  // n * 128 B (a multiple of 1024 for n % 8 == 0)
+  const uint32_t stage_bytes = 2 * a_bytes + 2 * b_bytes;
+  const int ST = A.stages;
+
+  if (threadIdx.x == 0) {
+    umma::prefetch_tensormap(&ta_hi);
+    umma::prefetch_tensormap(&ta_lo);
+    umma::prefetch_tensormap(&tb_hi);
+    umma::prefetch_tensormap(&tb_lo);
+    for (int i = 0; i < ST; i++) {
+      umma::mbar_init(&full[i], 1);
+      umma::mbar_init(&empty[i], 1);
+    }
+    umma::mbar_init(&accb, 1);
+    umma::fence_barrier_init();
+  }
+  if (warp == 0) {
+    umma::tmem_alloc(&tmem_base, 128);
+    umma::tmem_relinquish();
+  }
+  umma::fence_before_sync();
+  __syncthreads();
+  umma::fence_after_sync();
+  const uint32_t tmem = tmem_base;
+  int ok = 1;
+
+  if (warp == 0 && lane == 0) {
+    // producer
+    for (int i = 0; i < nk && ok; i++) {
+      const int st = i % ST;
+      if (i >= ST && !umma::mbar_wait(&empty[st], (uint32_t)(((i / ST) - 1) & 1))) { ok = 0; break; }
+      uint8_t *base = sm + (size_t)st * stage_bytes;
+      umma::mbar_arrive_expect_tx(&full[st], stage_bytes);
+      const int kc = (kb0 + i) * kTileK;
+      umma::tma_load_2d(base, &ta_hi, kc, m0, &full[st]);
+      umma::tma_load_2d(base + a_bytes, &ta_lo, kc, m0, &full[st]);
+      umma::tma_load_2d(base + 2 * a_bytes, &tb_hi, kc, 0, &full[st]);
+      umma::tma_load_2d(base + 2 * a_bytes + b_bytes, &tb_lo, kc, 0, &full[st]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer
+    const uint32_t idesc = umma::idesc_bf16_f32(kTileM, A.n);
+    for (int i = 0; i < nk && ok; i++) {
+      const int st = i % ST;
+      if (!umma::mbar_wait(&full[st], (uint32_t)((i / ST) & 1))) { ok = 0; break; }
+      umma::fence_after_sync();
+      const uint32_t base = umma::saddr(sm + (size_t)st * stage_bytes);
+#pragma unroll
+      for (int kk = 0; kk < kTileK / 16; kk++) {
+        const uint64_t ah = umma::desc_kmajor_sw128(base + kk * 32);
+        const uint64_t al = umma::desc_kmajor_sw128(base + a_bytes + kk * 32);
+        const uint64_t bh = umma::desc_kmajor_sw128(base + 2 * a_bytes + kk * 32);
+        const uint64_t bl = umma::desc_kmajor_sw128(base + 2 * a_bytes + b_bytes + kk * 32);
+        umma::mma_bf16(tmem, ah, bh, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        umma::mma_bf16(tmem, ah, bl, idesc, 1u);
+        umma::mma_bf16(tmem, al, bh, idesc, 1u);
+      }
+      umma::mma_commit(&empty[st]);
+    }
+    umma::mma_commit(&accb);
+  }
+  __syncwarp();
+  if (ok) ok = umma::mbar_wait(&accb, 0) ? 1 : 0;
+  if (!__syncthreads_and(ok)) {
+    if (threadIdx.x == 0) atomicOr(A.status, kStatusTimeout);
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) umma::tmem_dealloc(tmem, 128);
+    return;
+  }
+  umma::fence_after_sync();
+  // epilogue: thread = accumulator row m0 + 32 warp + lane
+  const int64_t row = m0 + 32 * warp + lane;
+  float *dst = A.out + ((int64_t)s * A.M + row) * A.n;
+  for (int c = 0; c < A.n; c += 16) {
+    float v[16];
+    umma::tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
+    float4 *d4 = reinterpret_cast<float4 *>(dst + c);
+    d4[0] = make_float4(v[0], v[1], v[2], v[3]);
+    d4[1] = make_float4(v[4], v[5], v[6], v[7]);
+    d4[2] = make_float4(v[8], v[9], v[10], v[11]);
+    d4[3] = make_float4(v[12], v[13], v[14], v[15]);
+  }
+  umma::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) umma::tmem_dealloc(tmem, 128);
+}
+
+// ---------------------------------------------------------------- CholeskyQR2 pieces
+
+// X = sum of the nsrc partial slabs (fixed order), stored fp32 [rows][n], and
+// the partial Gram matrix X^T X (fp64) of this block's kGramRows rows.
+__global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc, int64_t rows, int n, float *x,
+                                                      double *gpart) {
+  extern __shared__ __align__(16) uint8_t gsm[];
+  float *tile = reinterpret_cast<float *>(gsm);  // [kGramRows][n]
+  const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
+  for (int idx = threadIdx.x; idx < kGramRows * n; idx += blockDim.x) {
+    const int64_t off = (r0 + idx / n) * n + idx % n;
+    float acc = src[off];
+    for (int p = 1; p < nsrc; p++) acc = __fadd_rn(acc, src[(int64_t)p * rows * n + off]);
+    tile[idx] = acc;
+    x[off] = acc;
+  }
+  __syncthreads();
+  double *g = gpart + (int64_t)blockIdx.x * n * n;
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+    const int i = e / n, j = e % n;
+    if (j < i) continue;
+    double acc = 0.0;
+    for (int rr = 0; rr < kGramRows; rr++) acc += (double)tile[rr * n + i] * (double)tile[rr * n + j];
+    g[i * n + j] = acc;
+    g[j * n + i] = acc;
+  }
+}
+
+// Sum of the partial Gram matrices (fixed order) and its Cholesky factor L
+// (lower, fp64).  A pivot <= 1e-12 G_00 (R_kk <= 1e-6 R_00) marks column k
+// rank deficient: dead[k] = 1, L[k][k] = 1 and L[i][k] = 0 below it.
+__global__ void __launch_bounds__(256) lr_chol_kernel(const double *gpart, int nblk, int n, double *Lout, int *dead) {
+  extern __shared__ __align__(16) uint8_t csm[];
+  double *G = reinterpret_cast<double *>(csm);  // [n][n]
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+    double acc = 0.0;
+    for (int b = 0; b < nblk; b++) acc += gpart[(int64_t)b * n * n + e];
+    G[e] = acc;
+  }
+  __syncthreads();
+  const double thr = 1e-12 * G[0];
+  for (int k = 0; k < n; k++) {
+    const double piv = G[k * n + k];
+    const bool dk = !(piv > thr);
+    __syncthreads();
+    const double lkk = dk ? 1.0 : sqrt(piv);
+    for (int i = k + threadIdx.x; i < n; i += blockDim.x) {
+      if (i == k) G[k * n + k] = lkk;
+      else G[i * n + k] = dk ? 0.0 : G[i * n + k] / lkk;
+    }
+    if (threadIdx.x == 0) dead[k] = dk ? 1 : 0;
+    __syncthreads();
+    const int m = n - k - 1;
+    for (int e = threadIdx.x; e < m * m; e += blockDim.x) {
+      const int i = k + 1 + e / m, j = k + 1 + e % m;
+      if (j <= i) G[i * n + j] -= G[i * n + k] * G[j * n + k];
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+    const int i = e / n, j = e % n;
+    Lout[e] = j <= i ? G[e] : 0.0;
+  }
+}
+
+// Q = X L^-T row by row (forward substitution in fp64); dead columns are 0.
+// Writes Q fp32 [rows][n] and, when qthi != nullptr, Q^T split in bf16
+// ([n][rows], the K-major B operand of V = D^T Q).
+__global__ void lr_apply_kernel(const float *x, const double *L, const int *dead, int64_t rows, int n, float *q,
+                                __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo) {
+  extern __shared__ __align__(16) uint8_t asm_[];
+  double *Ls = reinterpret_cast<double *>(asm_);  // [n][n]
+  double *qs = Ls + n * n;                        // [n][blockDim]
+  int *ds = reinterpret_cast<int *>(qs + (size_t)n * blockDim.x);
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) Ls[e] = L[e];
+  for (int e = threadIdx.x; e < n; e += blockDim.x) ds[e] = dead[e];
+  __syncthreads();
+  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= rows) return;
+  const int T = blockDim.x;
+  for (int k = 0; k < n; k++) {
+    double acc = (double)x[row * n + k];
+    for (int j = 0; j < k; j++) acc -= Ls[k * n + j] * qs[j * T + threadIdx.x];
+    const double qk = ds[k] ? 0.0 : acc / Ls[k * n + k];
+    qs[k * T + threadIdx.x] = qk;
+  }
+  for (int k = 0; k < n; k++) {
+    const float qf = (float)qs[k * T + threadIdx.x];
+    q[row * n + k] = qf;
+    if (qthi) {
+      __nv_bfloat16 hi, lo;
+      split_bf16(qf, hi, lo);
+      qthi[(int64_t)k * rows + row] = hi;
+      qtlo[(int64_t)k * rows + row] = lo;
+    }
+  }
+}
+
+// V = sum of the partial slabs (fixed order) [cols][n]; V_prev (state,
+// [cols][r]) = V[:, :r]; when vthi != nullptr also V^T split for the next
+// iteration's Y = D V.
+__global__ void __launch_bounds__(256) lr_vsum_kernel(const float *vpart, int nsrc, int64_t cols, int n, int r,
+                                                      float *v, float *vprev, __nv_bfloat16 *vthi,
+                                                      __nv_bfloat16 *vtlo) {
+  const int64_t total = cols * n;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
+    float acc = vpart[idx];
+    for (int p = 1; p < nsrc; p++) acc = __fadd_rn(acc, vpart[(int64_t)p * total + idx]);
+    const int64_t j = idx / n;
+    const int k = (int)(idx % n);
+    v[idx] = acc;
+    if (k < r) vprev[j * r + k] = acc;
+    if (vthi) {
+      __nv_bfloat16 hi, lo;
+      split_bf16(k < r ? acc : 0.0f, hi, lo);
+      vthi[(int64_t)k * cols + j] = hi;
+      vtlo[(int64_t)k * cols + j] = lo;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- INT4 payload
+
+struct PackArgs {
+  uint8_t *payload;  // header + body
+  const float *q;    // [rows][n]
+  const float *v;    // [cols][n]
+  int64_t rows, cols;
+  int r, n, int4;
+  int64_t sec1, sec2, body;
+  Header hdr;
+};
+
+// Per-column scales s_k = fp32(absmax_k / 7) of U (blocks 0..r-1) and V
+// (blocks r..2r-1), into the payload's scale section.
+__global__ void __launch_bounds__(256) lr_scale_kernel(PackArgs P) {
+  const int k = blockIdx.x % P.r;
+  const bool isv = blockIdx.x >= P.r;
+  const float *m = isv ? P.v : P.q;
+  const int64_t len = isv ? P.cols : P.rows;
+  float amax = 0.0f;
+  for (int64_t i = threadIdx.x; i < len; i += blockDim.x) amax = fmaxf(amax, fabsf(m[i * P.n + k]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  __shared__ float wm[8];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); w++) amax = fmaxf(amax, wm[w]);
+    amax = fmaxf(amax, wm[0]);
+    float *sc = reinterpret_cast<float *>(P.payload + kHdrBytes);
+    sc[(isv ? P.r : 0) + k] = (float)((double)amax / 7.0);
+  }
+}
+
+__device__ __forceinline__ uint32_t int4_code(float x, float s) {
+  if (s == 0.0f) return 0;
+  double t = rint((double)x / (double)s);
+  t = t > 7.0 ? 7.0 : (t < -7.0 ? -7.0 : t);
+  return (uint32_t)((int)t & 0xF);
+}
+
+// Nibbles of U and V (element (i,k) is nibble i*r + k, low nibble first) or
+// the fp32 factors, padding bytes zero, and the header.
+__global__ void __launch_bounds__(256) lr_pack_kernel(PackArgs P) {
+  uint8_t *body = P.payload + kHdrBytes;
+  if (blockIdx.x == 0 && threadIdx.x < 16) reinterpret_cast<uint32_t *>(P.payload)[threadIdx.x] = P.hdr.w[threadIdx.x];
+  const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (P.int4) {
+    const float *sc = reinterpret_cast<const float *>(body);
+    // scale section padding
+    for (int64_t b = (int64_t)P.r * 8 + tid; b < P.sec1; b += nthr) body[b] = 0;
+    const int64_t ubytes = P.sec2 - P.sec1, vbytes = P.body - P.sec2;
+    const int64_t un = P.rows * P.r, vn = P.cols * P.r;
+    for (int64_t b = tid; b < ubytes + vbytes; b += nthr) {
+      const bool isv = b >= ubytes;
+      const int64_t bb = isv ? b - ubytes : b;
+      const int64_t nel = isv ? vn : un;
+      const float *m = isv ? P.v : P.q;
+      uint32_t byte = 0;
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const int64_t e = 2 * bb + h;
+        if (e < nel) {
+          const int64_t i = e / P.r;
+          const int k = (int)(e % P.r);
+          byte |= int4_code(m[i * P.n + k], sc[(isv ? P.r : 0) + k]) << (4 * h);
+        }
+      }
+      body[(isv ? P.sec2 : P.sec1) + bb] = (uint8_t)byte;
+    }
+  } else {
+    float *u = reinterpret_cast<float *>(body);
+    float *vv = reinterpret_cast<float *>(body + P.sec2);
+    const int64_t un = P.rows * P.r, vn = P.cols * P.r;
+    for (int64_t e = tid; e < un; e += nthr) u[e] = P.q[(e / P.r) * P.n + e % P.r];
+    for (int64_t e = tid; e < vn; e += nthr) vv[e] = P.v[(e / P.r) * P.n + e % P.r];
+    for (int64_t b = un * 4 + tid; b < P.sec2; b += nthr) body[b] = 0;
+    for (int64_t b = P.sec2 + vn * 4 + tid; b < P.body; b += nthr) body[b] = 0;
+  }
+}
+
+__device__ __forceinline__ int nibble_at(const uint8_t *base, int64_t idx) {
+  const int v = (idx & 1) ? (base[idx >> 1] >> 4) : (base[idx >> 1] & 0xF);
+  return (v & 0x8) ? v - 16 : v;
+}
+
+// Reconstruction operands from the payload alone (both roles): A = U
+// ([rows][kp]; INT4: the integer codes, exact in bf16; fp32 factors: split),
+// B = V scaled ([cols][kp], split; INT4: fp32(qV * sU * sV) per entry).
+struct DequantArgs {
+  const uint8_t *payload;
+  int64_t rows, cols;
+  int r, kp, int4;
+  int64_t sec1, sec2;
+  __nv_bfloat16 *uahi, *ualo, *vbhi, *vblo;
+  int check_header;
+  Header expect;
+  int *status;
+};
+
+__global__ void __launch_bounds__(256) lr_dequant_kernel(DequantArgs D) {
+  if (D.check_header && !lr_header_ok(D.payload, D.expect, D.status)) return;
+  const uint8_t *body = D.payload + kHdrBytes;
+  const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t un = D.rows * D.kp, vn = D.cols * D.kp;
+  const float *sc = reinterpret_cast<const float *>(body);
+  for (int64_t e = tid; e < un + vn; e += nthr) {
+    const bool isv = e >= un;
+    const int64_t ee = isv ? e - un : e;
+    const int64_t i = ee / D.kp;
+    const int k = (int)(ee % D.kp);
+    float x = 0.0f;
+    if (k < D.r) {
+      if (D.int4) {
+        const uint8_t *nb = body + (isv ? D.sec2 : D.sec1);
+        const int q = nibble_at(nb, i * D.r + k);
+        x = isv ? (float)((double)q * (double)sc[k] * (double)sc[D.r + k]) : (float)q;
+      } else {
+        const float *f = reinterpret_cast<const float *>(body + (isv ? D.sec2 : 0));
+        x = f[i * D.r + k];
+      }
+    }
+    __nv_bfloat16 hi, lo;
+    split_bf16(x, hi, lo);
+    if (isv) {
+      D.vbhi[ee] = hi;
+      D.vblo[ee] = lo;
+    } else {
+      D.uahi[ee] = hi;
+      if (D.ualo) D.ualo[ee] = lo;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- reconstruction GEMM (tcgen05)
+
+struct ReconArgs {
+  int64_t rows, cols;
+  int kblocks;        // kp / 64
+  int a_split;        // 1: A carries a lo term (fp32 factors)
+  int role;           // CF_SENDER: e, ahat update; CF_RECEIVER: ahat, recon
+  int ef_explicit;
+  const void *a;      // sender: activations [rows][cols]
+  float *ahat;
+  float *err;
+  void *recon;        // receiver
+  int *status;
+  const uint8_t *payload;
+  int check_header;
+  Header expect;
+};
+
+template <typename T>
+__device__ __forceinline__ void load16_act(const T *p, float (&x)[16]) {
+  if constexpr (sizeof(T) == 2) {
+    const uint4 u0 = reinterpret_cast<const uint4 *>(p)[0], u1 = reinterpret_cast<const uint4 *>(p)[1];
+    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      x[2 * k] = __uint_as_float(w[k] << 16);
+      x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+  } else {
+    const float4 *q = reinterpret_cast<const float4 *>(p);
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const float4 f = q[k];
+      x[4 * k] = f.x; x[4 * k + 1] = f.y; x[4 * k + 2] = f.z; x[4 * k + 3] = f.w;
+    }
+  }
+}
+
+__device__ __forceinline__ void load16_f32(const float *p, float (&x)[16]) {
+  const float4 *q = reinterpret_cast<const float4 *>(p);
+#pragma unroll
+  for (int k = 0; k < 4; k++) {
+    const float4 f = __ldcs(q + k);
+    x[4 * k] = f.x; x[4 * k + 1] = f.y; x[4 * k + 2] = f.z; x[4 * k + 3] = f.w;
+  }
+}
+
+__device__ __forceinline__ void store16_f32(float *p, const float (&x)[16]) {
+  float4 *q = reinterpret_cast<float4 *>(p);
+#pragma unroll
+  for (int k = 0; k < 4; k++) __stcs(q + k, make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]));
+}
+
+template <typename T>
+__device__ __forceinline__ void store16_act(T *p, const float (&x)[16]) {
+  if constexpr (sizeof(T) == 2) {
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      w[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[2 * k])) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[2 * k + 1])) << 16);
+    }
+    uint4 *q = reinterpret_cast<uint4 *>(p);
+    q[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    q[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  } else {
+    store16_f32(reinterpret_cast<float *>(p), x);
+  }
+}
+
+// C tile (128 rows x 128 cols) = A[rows tile] * B[cols tile]^T over K = kp,
+// products hi*hi + hi*lo (+ lo*hi when A is split), then the fused update:
+// sender: D = (a - ahat) + e recomputed bit for bit; e = D - C; ahat = ahat + C;
+// receiver: ahat = ahat + C; recon = cast(ahat).
+template <typename T>
+__global__ void __launch_bounds__(128, 1)
+    lr_recon_kernel(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
+                    const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
+                    const ReconArgs R) {
+  extern __shared__ __align__(1024) uint8_t dsm[];
+  __shared__ __align__(8) uint64_t full, accb;
+  __shared__ uint32_t tmem_base;
+  if (R.check_header && !lr_header_ok(R.payload, R.expect, R.status)) return;
+  uint8_t *sm = reinterpret_cast<uint8_t *>(((uintptr_t)dsm + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m0 = (int64_t)blockIdx.x * kTileM, n0 = (int64_t)blockIdx.y * kReconN;
+  const uint32_t tile = kTileM * kTileK * 2;  // 16 KiB per 128 x 64 tile
+  const int nkb = R.kblocks;
+  // layout: A hi [nkb] | A lo [nkb] (if split) | B hi [nkb] | B lo [nkb]
+  const uint32_t off_al = nkb * tile;
+  const uint32_t off_bh = off_al + (R.a_split ? nkb * tile : 0);
+  const uint32_t off_bl = off_bh + nkb * tile;
+  const uint32_t total = off_bl + nkb * tile;
+
+  if (threadIdx.x == 0) {
+    umma::mbar_init(&full, 1);
+    umma::mbar_init(&accb, 1);
+    umma::fence_barrier_init();
+  }
+  if (warp == 0) {
+    umma::tmem_alloc(&tmem_base, 128);
+    umma::tmem_relinquish();
+  }
+  umma::fence_before_sync();
+  __syncthreads();
+  umma::fence_after_sync();
+  const uint32_t tmem = tmem_base;
+  int ok = 1;
+  if (warp == 0 && lane == 0) {
+    umma::mbar_arrive_expect_tx(&full, total);
+    for (int kb = 0; kb < nkb; kb++) {
+      umma::tma_load_2d(sm + kb * tile, &ta_hi, kb * kTileK, (int)m0, &full);
+      if (R.a_split) umma::tma_load_2d(sm + off_al + kb * tile, &ta_lo, kb * kTileK, (int)m0, &full);
+      umma::tma_load_2d(sm + off_bh + kb * tile, &tb_hi, kb * kTileK, (int)n0, &full);
+      umma::tma_load_2d(sm + off_bl + kb * tile, &tb_lo, kb * kTileK, (int)n0, &full);
+    }
+    if (!umma::mbar_wait(&full, 0)) {
+      ok = 0;
+    } else {
+      umma::fence_after_sync();
+      const uint32_t idesc = umma::idesc_bf16_f32(kTileM, kReconN);
+      const uint32_t base = umma::saddr(sm);
+      for (int kb = 0; kb < nkb; kb++) {
+#pragma unroll
+        for (int kk = 0; kk < kTileK / 16; kk++) {
+          const uint32_t o = kb * tile + kk * 32;
+          const uint64_t ah = umma::desc_kmajor_sw128(base + o);
+          const uint64_t bh = umma::desc_kmajor_sw128(base + off_bh + o);
+          const uint64_t bl = umma::desc_kmajor_sw128(base + off_bl + o);
+          umma::mma_bf16(tmem, ah, bh, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          umma::mma_bf16(tmem, ah, bl, idesc, 1u);
+          if (R.a_split) umma::mma_bf16(tmem, umma::desc_kmajor_sw128(base + off_al + o), bh, idesc, 1u);
+        }
+      }
+      umma::mma_commit(&accb);
+    }
+  }
+  __syncwarp();
+  if (!__syncthreads_and(ok)) {
+    if (threadIdx.x == 0) atomicOr(R.status, kStatusTimeout);
+    __syncthreads();
+    if (warp == 0) umma::tmem_dealloc(tmem, 128);
+    return;
+  }
+  ok = umma::mbar_wait(&accb, 0) ? 1 : 0;
+  if (!__syncthreads_and(ok)) {
+    if (threadIdx.x == 0) atomicOr(R.status, kStatusTimeout);
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) umma::tmem_dealloc(tmem, 128);
+    return;
+  }
+  umma::fence_after_sync();
+  const int64_t row = m0 + 32 * warp + lane;
+  const int64_t base_off = row * R.cols + n0;
+  for (int c = 0; c < kReconN; c += 16) {
+    float cv[16];
+    umma::tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, cv);
+    const int64_t off = base_off + c;
+    float h[16];
+    load16_f32(R.ahat + off, h);
+    if (R.role == CF_SENDER) {
+      float x[16], e[16];
+      load16_act(static_cast<const T *>(R.a) + off, x);
+      if (R.ef_explicit) load16_f32(R.err + off, e);
+      float en[16], hn[16];
+#pragma unroll
+      for (int k = 0; k < 16; k++) {
+        const float tt = __fsub_rn(x[k], h[k]);
+        const float d = R.ef_explicit ? __fadd_rn(tt, e[k]) : tt;
+        en[k] = __fsub_rn(d, cv[k]);
+        hn[k] = __fadd_rn(h[k], cv[k]);
+      }
+      store16_f32(R.err + off, en);
+      store16_f32(R.ahat + off, hn);
+    } else {
+      float hn[16];
+#pragma unroll
+      for (int k = 0; k < 16; k++) hn[k] = __fadd_rn(h[k], cv[k]);
+      store16_f32(R.ahat + off, hn);
+      store16_act(static_cast<T *>(R.recon) + off, hn);
+    }
+  }
+  umma::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) umma::tmem_dealloc(tmem, 128);
+}
+
+// ---------------------------------------------------------------- host
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    (void)cudaGetLastError();
+  }
+  return fn;
+}
+
+// bf16 [outer][inner] row-major, box {64, box_rows}, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kTileK, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+size_t thin_smem(int n, int stages) { return (size_t)stages * (2u * kTileM * kTileK * 2 + 2u * n * kTileK * 2) + 1024; }
+int thin_stages(int n) { return n <= 96 ? 4 : 3; }
+size_t recon_smem(int kblocks, int a_split) { return (size_t)kblocks * kTileM * kTileK * 2 * (3 + a_split) + 1024; }
+size_t apply_smem(int n, int threads) { return (size_t)n * n * 8 + (size_t)n * threads * 8 + (size_t)n * 4; }
+int apply_threads(int n) { return n <= 96 ? 128 : 64; }
+
+}  // namespace
 
 void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *plan) {
   plan->rows = rows;
@@ -11,16 +789,245 @@ void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *p
   plan->iters = p.iters;
   plan->int4 = p.lr_int4;
   plan->batch = p.batch;
-  plan->supported = false;
+  plan->role = p.role;
+  plan->dtype = p.dtype;
+  plan->ef_explicit = p.ef == CF_EF_EXPLICIT;
+  plan->rp = round_up(p.rank < 16 ? 16 : p.rank, 16);
+  plan->kp = round_up(p.rank, kTileK);
+  plan->supported = rows % 128 == 0 && cols % 128 == 0 && rows >= 128 && cols >= 128 && p.batch == 1 &&
+                    p.rank >= 1 && p.rank <= 128 && rows < (1ll << 30) && cols < (1ll << 30);
+  // split-K so that each thin GEMM fills the SMs: (tiles of 128 rows) x splits
+  const int ty = (int)(rows / kTileM), tv = (int)(cols / kTileM);
+  const int kby = (int)(cols / kTileK), kbv = (int)(rows / kTileK);
+  auto splits = [](int tiles, int kblocks) {
+    int s = (144 + tiles - 1) / tiles;
+    if (s > kblocks) s = kblocks;
+    return s < 1 ? 1 : s;
+  };
+  plan->sy = splits(ty, kby);
+  plan->sv = splits(tv, kbv);
+  const int64_t mx = rows > cols ? rows : cols;
+  plan->nblk_gram = (int)(mx / kGramRows);
+  const size_t R = (size_t)rows, C = (size_t)cols, rp = (size_t)plan->rp, kp = (size_t)plan->kp;
+  size_t dec = 0;
+  dec += pad256(R * kp * 2) * 2;  // uahi, ualo
+  dec += pad256(C * kp * 2) * 2;  // vbhi, vblo
+  size_t enc = dec;
+  enc += pad256(R * C * 2) * 4;                               // dhi dlo dthi dtlo
+  enc += pad256(rp * C * 2) * 2 + pad256(rp * R * 2) * 2;     // vt, qt
+  enc += pad256((size_t)plan->sy * R * rp * 4);               // ypart
+  enc += pad256((size_t)plan->sv * C * rp * 4);               // vpart
+  enc += pad256(mx * rp * 4) * 2 + pad256(C * rp * 4);        // xbuf, q, v
+  enc += pad256((size_t)plan->nblk_gram * rp * rp * 8);       // gpart
+  enc += pad256(rp * rp * 8) + pad256(rp * 4);                // L, dead
+  plan->enc_scratch_bytes = enc;
+  plan->dec_scratch_bytes = dec;
 }
 
-cudaError_t lowrank_encode(const LowrankPlan &, const EncArgs &, const PtrTable *, float *, void *, uint64_t,
-                           cudaStream_t) {
-  return cudaErrorNotSupported;
+int lowrank_bind(LowrankPlan *plan, void *scratch) {
+  uint8_t *p = static_cast<uint8_t *>(scratch);
+  const size_t R = (size_t)plan->rows, C = (size_t)plan->cols, rp = (size_t)plan->rp, kp = (size_t)plan->kp;
+  const size_t mx = R > C ? R : C;
+  auto take = [&](size_t bytes) {
+    uint8_t *q = p;
+    p += pad256(bytes);
+    return q;
+  };
+  LowrankBufs &b = plan->b;
+  b.uahi = reinterpret_cast<__nv_bfloat16 *>(take(R * kp * 2));
+  b.ualo = reinterpret_cast<__nv_bfloat16 *>(take(R * kp * 2));
+  b.vbhi = reinterpret_cast<__nv_bfloat16 *>(take(C * kp * 2));
+  b.vblo = reinterpret_cast<__nv_bfloat16 *>(take(C * kp * 2));
+  bool ok = make_map(&plan->tm_uahi, b.uahi, kp, R, kTileM) && make_map(&plan->tm_ualo, b.ualo, kp, R, kTileM) &&
+            make_map(&plan->tm_vbhi, b.vbhi, kp, C, kReconN) && make_map(&plan->tm_vblo, b.vblo, kp, C, kReconN);
+  if (plan->role == CF_SENDER) {
+    b.dhi = reinterpret_cast<__nv_bfloat16 *>(take(R * C * 2));
+    b.dlo = reinterpret_cast<__nv_bfloat16 *>(take(R * C * 2));
+    b.dthi = reinterpret_cast<__nv_bfloat16 *>(take(R * C * 2));
+    b.dtlo = reinterpret_cast<__nv_bfloat16 *>(take(R * C * 2));
+    b.vthi = reinterpret_cast<__nv_bfloat16 *>(take(rp * C * 2));
+    b.vtlo = reinterpret_cast<__nv_bfloat16 *>(take(rp * C * 2));
+    b.qthi = reinterpret_cast<__nv_bfloat16 *>(take(rp * R * 2));
+    b.qtlo = reinterpret_cast<__nv_bfloat16 *>(take(rp * R * 2));
+    b.ypart = reinterpret_cast<float *>(take((size_t)plan->sy * R * rp * 4));
+    b.vpart = reinterpret_cast<float *>(take((size_t)plan->sv * C * rp * 4));
+    b.xbuf = reinterpret_cast<float *>(take(mx * rp * 4));
+    b.q = reinterpret_cast<float *>(take(mx * rp * 4));
+    b.v = reinterpret_cast<float *>(take(C * rp * 4));
+    b.gpart = reinterpret_cast<double *>(take((size_t)plan->nblk_gram * rp * rp * 8));
+    b.L = reinterpret_cast<double *>(take(rp * rp * 8));
+    b.dead = reinterpret_cast<int *>(take(rp * 4));
+    ok = ok && make_map(&plan->tm_dhi, b.dhi, C, R, kTileM) && make_map(&plan->tm_dlo, b.dlo, C, R, kTileM) &&
+         make_map(&plan->tm_vthi, b.vthi, C, rp, (uint32_t)rp) && make_map(&plan->tm_vtlo, b.vtlo, C, rp, (uint32_t)rp) &&
+         make_map(&plan->tm_dthi, b.dthi, R, C, kTileM) && make_map(&plan->tm_dtlo, b.dtlo, R, C, kTileM) &&
+         make_map(&plan->tm_qthi, b.qthi, R, rp, (uint32_t)rp) && make_map(&plan->tm_qtlo, b.qtlo, R, rp, (uint32_t)rp);
+  }
+  if (!ok) return CF_ERR_CUDA;
+  // kernels that need more than 48 KiB of dynamic shared memory
+  const int rpi = plan->rp;
+  if (cudaFuncSetAttribute(lr_thin_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)thin_smem(rpi, thin_stages(rpi))) != cudaSuccess ||
+      cudaFuncSetAttribute(lr_recon_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)recon_smem(plan->kp / kTileK, 1)) != cudaSuccess ||
+      cudaFuncSetAttribute(lr_recon_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)recon_smem(plan->kp / kTileK, 1)) != cudaSuccess ||
+      cudaFuncSetAttribute(lr_chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rpi * rpi * 8) != cudaSuccess ||
+      cudaFuncSetAttribute(lr_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)apply_smem(rpi, apply_threads(rpi))) != cudaSuccess ||
+      cudaFuncSetAttribute(lr_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kGramRows * rpi * 4) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return CF_ERR_CUDA;
+  }
+  return CF_OK;
 }
 
-cudaError_t lowrank_decode(const LowrankPlan &, const DecArgs &, const PtrTable *, void *, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+cudaError_t launch_thin(const LowrankPlan &P, const CUtensorMap &ah, const CUtensorMap &al, const CUtensorMap &bh,
+                        const CUtensorMap &bl, float *out, int64_t M, int64_t K, int splits, int *status,
+                        cudaStream_t st) {
+  ThinArgs A{};
+  A.out = out;
+  A.M = M;
+  A.n = P.rp;
+  A.kblocks = (int)(K / kTileK);
+  A.splits = splits;
+  A.stages = thin_stages(P.rp);
+  A.status = status;
+  lr_thin_gemm_kernel<<<dim3((unsigned)(M / kTileM), (unsigned)splits), 128, thin_smem(P.rp, A.stages), st>>>(
+      ah, al, bh, bl, A);
+  return cudaGetLastError();
+}
+
+cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int64_t rows, bool final_pass,
+                           cudaStream_t st) {
+  const LowrankBufs &b = P.b;
+  const int n = P.rp;
+  const int nblk = (int)(rows / kGramRows);
+  lr_gram_kernel<<<nblk, 256, kGramRows * n * 4, st>>>(src, nsrc, rows, n, b.xbuf, b.gpart);
+  lr_chol_kernel<<<1, 256, (size_t)n * n * 8, st>>>(b.gpart, nblk, n, b.L, b.dead);
+  const int th = apply_threads(n);
+  lr_apply_kernel<<<(unsigned)((rows + th - 1) / th), th, apply_smem(n, th), st>>>(
+      b.xbuf, b.L, b.dead, rows, n, b.q, final_pass ? b.qthi : nullptr, final_pass ? b.qtlo : nullptr);
+  return cudaGetLastError();
+}
+
+PackArgs pack_args(const LowrankPlan &P, uint8_t *payload, const Header &hdr) {
+  PackArgs A{};
+  A.payload = payload;
+  A.q = P.b.q;
+  A.v = P.b.v;
+  A.rows = P.rows;
+  A.cols = P.cols;
+  A.r = P.rank;
+  A.n = P.rp;
+  A.int4 = P.int4;
+  const size_t R = (size_t)P.rows, C = (size_t)P.cols, r = (size_t)P.rank;
+  if (P.int4) {
+    A.sec1 = (int64_t)pad16(r * 8);
+    A.sec2 = A.sec1 + (int64_t)pad16((R * r + 1) / 2);
+    A.body = A.sec2 + (int64_t)pad16((C * r + 1) / 2);
+  } else {
+    A.sec1 = 0;
+    A.sec2 = (int64_t)pad16(R * r * 4);
+    A.body = A.sec2 + (int64_t)pad16(C * r * 4);
+  }
+  A.hdr = hdr;
+  return A;
+}
+
+cudaError_t dequant_and_recon(const LowrankPlan &P, const uint8_t *payload, bool receiver, const Header &expect,
+                              const void *a, float *ahat, float *err, void *recon, int *status, cudaStream_t st) {
+  const PackArgs pa = pack_args(P, nullptr, expect);
+  DequantArgs D{};
+  D.payload = payload;
+  D.rows = P.rows;
+  D.cols = P.cols;
+  D.r = P.rank;
+  D.kp = P.kp;
+  D.int4 = P.int4;
+  D.sec1 = pa.sec1;
+  D.sec2 = pa.sec2;
+  D.uahi = P.b.uahi;
+  D.ualo = P.int4 ? nullptr : P.b.ualo;
+  D.vbhi = P.b.vbhi;
+  D.vblo = P.b.vblo;
+  D.check_header = receiver;
+  D.expect = expect;
+  D.status = status;
+  lr_dequant_kernel<<<1184, 256, 0, st>>>(D);
+  ReconArgs R{};
+  R.rows = P.rows;
+  R.cols = P.cols;
+  R.kblocks = P.kp / kTileK;
+  R.a_split = P.int4 ? 0 : 1;
+  R.role = receiver ? CF_RECEIVER : CF_SENDER;
+  R.ef_explicit = P.ef_explicit;
+  R.a = a;
+  R.ahat = ahat;
+  R.err = err;
+  R.recon = recon;
+  R.status = status;
+  R.payload = payload;
+  R.check_header = receiver;
+  R.expect = expect;
+  const dim3 grid((unsigned)(P.rows / kTileM), (unsigned)(P.cols / kReconN));
+  const size_t smem = recon_smem(R.kblocks, R.a_split);
+  if (P.dtype == CF_BF16)
+    lr_recon_kernel<__nv_bfloat16><<<grid, 128, smem, st>>>(P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
+  else
+    lr_recon_kernel<float><<<grid, 128, smem, st>>>(P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrTable *tab, float *vprev,
+                           uint64_t step, uint64_t seed, cudaStream_t st) {
+  if (tab) return cudaErrorNotSupported;  // batch 1 only
+  const LowrankBufs &b = P.b;
+  const int64_t R = P.rows, C = P.cols;
+  lr_vprep_kernel<<<P.rp, 256, 0, st>>>(vprev, C, P.rank, P.rp, step == 1 ? 1 : 0, seed, b.vthi, b.vtlo);
+  const dim3 dg((unsigned)(C / 64), (unsigned)(R / 64));
+  if (P.dtype == CF_BF16)
+    lr_delta_kernel<__nv_bfloat16><<<dg, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(args.a), args.ahat, args.err,
+                                                        P.ef_explicit, R, C, b.dhi, b.dlo, b.dthi, b.dtlo);
+  else
+    lr_delta_kernel<float><<<dg, 256, 0, st>>>(static_cast<const float *>(args.a), args.ahat, args.err, P.ef_explicit,
+                                               R, C, b.dhi, b.dlo, b.dthi, b.dtlo);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  for (int it = 0; it < P.iters; it++) {
+    // Y = D V
+    if ((e = launch_thin(P, P.tm_dhi, P.tm_dlo, P.tm_vthi, P.tm_vtlo, b.ypart, R, C, P.sy, args.status, st)) !=
+        cudaSuccess)
+      return e;
+    // Q = orth(Y): CholeskyQR2
+    if ((e = orthonormalise(P, b.ypart, P.sy, R, false, st)) != cudaSuccess) return e;
+    if ((e = orthonormalise(P, b.q, 1, R, true, st)) != cudaSuccess) return e;
+    // V = D^T Q
+    if ((e = launch_thin(P, P.tm_dthi, P.tm_dtlo, P.tm_qthi, P.tm_qtlo, b.vpart, C, R, P.sv, args.status, st)) !=
+        cudaSuccess)
+      return e;
+    const bool more = it + 1 < P.iters;
+    lr_vsum_kernel<<<592, 256, 0, st>>>(b.vpart, P.sv, C, P.rp, P.rank, b.v, vprev, more ? b.vthi : nullptr,
+                                        more ? b.vtlo : nullptr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // INT4 (or fp32) factors into the payload
+  const PackArgs pa = pack_args(P, args.payload, args.hdr);
+  if (P.int4) lr_scale_kernel<<<2 * P.rank, 256, 0, st>>>(pa);
+  lr_pack_kernel<<<592, 256, 0, st>>>(pa);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // sender reconstruction from the payload bytes
+  return dequant_and_recon(P, args.payload, false, args.hdr, args.a, args.ahat, args.err, nullptr, args.status, st);
+}
+
+cudaError_t lowrank_decode(const LowrankPlan &P, const DecArgs &args, const PtrTable *tab, cudaStream_t st) {
+  if (tab) return cudaErrorNotSupported;
+  return dequant_and_recon(P, args.payload, true, args.expect, nullptr, args.ahat, nullptr, args.recon, args.status,
+                           st);
 }
 
 }  // namespace cfi

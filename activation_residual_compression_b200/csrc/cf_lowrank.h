@@ -2,6 +2,8 @@
 // factors) of libcf.  Internal.
 #pragma once
 
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "cf.h"
@@ -9,18 +11,45 @@
 
 namespace cfi {
 
+struct LowrankBufs {
+  // sender only
+  __nv_bfloat16 *dhi = nullptr, *dlo = nullptr;    // residual D split in two bf16 terms, [rows][cols]
+  __nv_bfloat16 *dthi = nullptr, *dtlo = nullptr;  // the same, transposed [cols][rows]
+  __nv_bfloat16 *vthi = nullptr, *vtlo = nullptr;  // V^T split, [rp][cols]
+  __nv_bfloat16 *qthi = nullptr, *qtlo = nullptr;  // Q^T split, [rp][rows]
+  float *ypart = nullptr;                          // split-K partial products [sy][rows][rp]
+  float *vpart = nullptr;                          // [sv][cols][rp]
+  float *xbuf = nullptr;                           // matrix being orthonormalised [rows][rp]
+  float *q = nullptr;                              // orthonormal factor [rows][rp]
+  float *v = nullptr;                              // right factor [cols][rp]
+  double *gpart = nullptr;                         // partial Gram matrices [nblk][rp][rp]
+  double *L = nullptr;                             // Cholesky factor [rp][rp]
+  int *dead = nullptr;                             // rank-deficient column flags [rp]
+  // both roles: reconstruction operands dequantised from the payload
+  __nv_bfloat16 *uahi = nullptr, *ualo = nullptr;  // [rows][kp]
+  __nv_bfloat16 *vbhi = nullptr, *vblo = nullptr;  // [cols][kp]
+};
+
 struct LowrankPlan {
   int64_t rows = 0, cols = 0;
-  int rank = 0, rpad = 0, iters = 1, int4 = 1, batch = 1;
+  int rank = 0, rp = 0, kp = 0, iters = 1, int4 = 1, batch = 1;
+  int role = 0, ef_explicit = 1, dtype = CF_BF16;
+  int sy = 1, sv = 1;            // split-K factors of the two thin GEMMs
+  int nblk_gram = 1;             // row blocks of the partial Gram matrices
   size_t enc_scratch_bytes = 0;
   size_t dec_scratch_bytes = 0;
   bool supported = false;
+  LowrankBufs b;
+  CUtensorMap tm_dhi, tm_dlo, tm_vthi, tm_vtlo;    // Y = D V
+  CUtensorMap tm_dthi, tm_dtlo, tm_qthi, tm_qtlo;  // V = D^T Q
+  CUtensorMap tm_uahi, tm_ualo, tm_vbhi, tm_vblo;  // C = U V^T
 };
 
 void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *plan);
+// Carve the scratch buffers out of `scratch` and encode the TMA tensor maps.
+int lowrank_bind(LowrankPlan *plan, void *scratch);
 cudaError_t lowrank_encode(const LowrankPlan &plan, const EncArgs &args, const PtrTable *tab, float *vprev,
-                           void *scratch, uint64_t seed, cudaStream_t st);
-cudaError_t lowrank_decode(const LowrankPlan &plan, const DecArgs &args, const PtrTable *tab, void *scratch,
-                           cudaStream_t st);
+                           uint64_t step, uint64_t seed, cudaStream_t st);
+cudaError_t lowrank_decode(const LowrankPlan &plan, const DecArgs &args, const PtrTable *tab, cudaStream_t st);
 
 }  // namespace cfi

@@ -149,9 +149,11 @@ CF_API int cf_params_init(cf_params *p);
 CF_API int cf_workspace_bytes(int64_t rows, int64_t cols, int mode, const cf_params *p, size_t *out);
 
 /* Create a sender or receiver state on the current CUDA device.  Shape
- * rules: rows >= 1; cols % 8 == 0 and cols <= 8192 (streaming modes);
- * CF_SIGN1 cols % 32 == 0; CF_Q2 cols % 16 == 0; CF_NM cols % M == 0 and
- * (cols/M) N log2(M) % 32 == 0.  The state owns its tensors (in `workspace`
+ * rules: rows >= 1; cols % 8 == 0 and cols <= 8192; CF_SIGN1 cols % 32 == 0;
+ * CF_Q2 cols % 16 == 0; CF_NM cols % M == 0 and (cols/M) N log2(M) % 32 == 0;
+ * CF_LOWRANK rows % 128 == 0, cols % 128 == 0, rank <= min(rows, cols, 128),
+ * batch 1 (the low-rank state also holds its factor scratch: about
+ * 8 rows*cols bytes for a sender).  The state owns its tensors (in `workspace`
  * when given, else in memory it allocates with cudaMalloc) and starts at
  * step 0 (the warm-up step).  Blocks until its memory is initialised. */
 CF_API int cf_create(int64_t rows, int64_t cols, int mode, const cf_params *p, cf_state **out);

@@ -66,8 +66,9 @@ class GpuPair:
         cf.cf_state_export(st, buf)
         return buf
 
-    def state(self, which="S"):
-        """(ahat, err or None) as float32 arrays of shape (batch, rows, cols)."""
+    def state(self, which="S", with_vprev=False):
+        """(ahat, err or None) as float32 arrays of shape (batch, rows, cols); with
+        with_vprev the sender's low-rank warm start (batch, cols, rank) is appended."""
         buf = self.export(which)
         tb = int(buf[80:88].view(np.uint64)[0])
         ten = buf[len(buf) - tb:]
@@ -76,6 +77,9 @@ class GpuPair:
         err = None
         if which == "S":
             err = ten[4 * n:8 * n].view(np.float32).reshape(self.batch, self.rows, self.cols)
+        if with_vprev:
+            vp = ten[8 * n:].view(np.float32).reshape(self.batch, self.cols, -1)
+            return ahat, err, vp
         return ahat, err
 
     def guards_ok(self) -> bool:
