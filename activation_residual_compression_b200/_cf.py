@@ -26,6 +26,7 @@ CF_ERR_ALIGN = -8
 CF_ERR_STATE = -9
 CF_ERR_SIZE = -10
 CF_ERR_TIMEOUT = -11
+CF_ERR_TOO_LARGE = -12
 
 CF_IDENTITY, CF_SIGN1, CF_Q2, CF_NM, CF_LOWRANK = 0, 1, 2, 3, 4
 CF_F32, CF_BF16 = 0, 1
@@ -63,7 +64,8 @@ _lib = None
 
 EXPORTS = ["cf_version", "cf_strerror", "cf_params_init", "cf_workspace_bytes", "cf_create", "cf_payload_bytes",
            "cf_encode", "cf_decode", "cf_encode_batched", "cf_decode_batched", "cf_status", "cf_tensor",
-           "cf_step", "cf_reset", "cf_state_bytes", "cf_state_export", "cf_state_import", "cf_destroy"]
+           "cf_step", "cf_reset", "cf_state_bytes", "cf_state_export", "cf_state_import", "cf_destroy",
+           "cf_lowrank_decode_noalloc"]
 
 
 def load(path: str = LIB_PATH):
@@ -98,6 +100,7 @@ def load(path: str = LIB_PATH):
     L.cf_state_export.argtypes = [P, P, c.c_size_t, P]
     L.cf_state_import.argtypes = [P, P, c.c_size_t, P]
     L.cf_destroy.argtypes = [P]
+    L.cf_lowrank_decode_noalloc.argtypes = [c.c_int64, c.c_int64, c.POINTER(cf_params), c.c_uint64, P, P, P, P, P]
     for name in EXPORTS:
         if name not in ("cf_version", "cf_strerror"):
             getattr(L, name).restype = c.c_int
@@ -237,6 +240,14 @@ def cf_state_import(state, host_buf, stream=None) -> int:
 
 def cf_destroy(state) -> int:
     return _check("cf_destroy", load().cf_destroy(state))
+
+
+def cf_lowrank_decode_noalloc(rows: int, cols: int, params: cf_params, step: int, payload, ahat, recon, status,
+                              stream=None) -> int:
+    """Allocation-free low-rank decode (see include/cf.h); all tensors caller-owned."""
+    return _check("cf_lowrank_decode_noalloc", load().cf_lowrank_decode_noalloc(
+        rows, cols, ctypes.byref(params), step, _ptr(payload), _ptr(ahat), _ptr(recon), _ptr(status),
+        _stream(stream)))
 
 
 def raw(name: str):

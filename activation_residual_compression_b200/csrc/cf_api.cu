@@ -333,6 +333,7 @@ const char *cf_strerror(int status) {
     case CF_ERR_STATE: return "not a live state";
     case CF_ERR_SIZE: return "host buffer size mismatch";
     case CF_ERR_TIMEOUT: return "a kernel's bounded wait for its own asynchronous copy gave up";
+    case CF_ERR_TOO_LARGE: return "problem larger than the allocation-free entry point's fixed scratch";
   }
   return "unknown status";
 }

@@ -28,6 +28,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "cf_lowrank.h"
 #include "cf_umma.cuh"
@@ -1031,3 +1032,114 @@ cudaError_t lowrank_decode(const LowrankPlan &P, const DecArgs &args, const PtrT
 }
 
 }  // namespace cfi
+
+// ---------------------------------------------------------------- allocation-free decode
+
+namespace cfi {
+namespace {
+
+// Fixed scratch of cf_lowrank_decode_noalloc: the dequantised reconstruction
+// operands.  Host code must not use the symbol as an address: the device
+// address comes from cudaGetSymbolAddress, once per device.
+constexpr size_t kNoAllocBytes = 8u << 20;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch for the current device (set-up on first use).
+int noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return CF_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+      (void)cudaGetLastError();
+      return CF_ERR_CUDA;
+    }
+    const int smem = (int)recon_smem(2, 1);
+    if (cudaFuncSetAttribute(lr_recon_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(lr_recon_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess) {
+      (void)cudaGetLastError();
+      return CF_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return CF_OK;
+}
+
+}  // namespace
+}  // namespace cfi
+
+extern "C" int cf_lowrank_decode_noalloc(int64_t rows, int64_t cols, const cf_params *p, uint64_t step,
+                                         const void *payload, float *ahat, void *recon, int *status, void *stream) {
+  using namespace cfi;
+  if (!p || !payload || !ahat || !recon || !status || step < 1) return CF_ERR_ARG;
+  if (p->dtype != CF_F32 && p->dtype != CF_BF16) return CF_ERR_ARG;
+  if (p->ef != CF_EF_EXPLICIT && p->ef != CF_EF_IMPLICIT) return CF_ERR_ARG;
+  if (p->lr_int4 != 0 && p->lr_int4 != 1) return CF_ERR_ARG;
+  if (p->iters < 1 || p->iters > 2) return CF_ERR_UNSUPPORTED;
+  if (rows < 128 || cols < 128 || rows % 128 || cols % 128 || cols > kMaxCols) return CF_ERR_SHAPE;
+  if (p->rank < 1 || p->rank > kMaxRank || p->rank > rows || p->rank > cols) return CF_ERR_SHAPE;
+  if (((uintptr_t)payload | (uintptr_t)ahat | (uintptr_t)recon) & 15u) return CF_ERR_ALIGN;
+  LowrankPlan P{};
+  cf_params q = *p;
+  q.role = CF_RECEIVER;
+  q.batch = 1;
+  lowrank_plan(rows, cols, q, &P);
+  if (!P.supported) return CF_ERR_UNSUPPORTED;
+  const size_t R = (size_t)rows, C = (size_t)cols, kp = (size_t)P.kp;
+  const size_t need = pad256(R * kp * 2) * (P.int4 ? 1 : 2) + pad256(C * kp * 2) * 2;
+  if (need > kNoAllocBytes) return CF_ERR_TOO_LARGE;
+  void *scratch = nullptr;
+  const int rc = noalloc_scratch(&scratch);
+  if (rc != CF_OK) return rc;
+  uint8_t *base = static_cast<uint8_t *>(scratch);
+  P.b.uahi = reinterpret_cast<__nv_bfloat16 *>(base);
+  base += pad256(R * kp * 2);
+  if (!P.int4) {
+    P.b.ualo = reinterpret_cast<__nv_bfloat16 *>(base);
+    base += pad256(R * kp * 2);
+  } else {
+    P.b.ualo = P.b.uahi;  // not read: INT4 codes are exact in bf16
+  }
+  P.b.vbhi = reinterpret_cast<__nv_bfloat16 *>(base);
+  base += pad256(C * kp * 2);
+  P.b.vblo = reinterpret_cast<__nv_bfloat16 *>(base);
+  if (!(make_map(&P.tm_uahi, P.b.uahi, kp, R, kTileM) && make_map(&P.tm_ualo, P.b.ualo, kp, R, kTileM) &&
+        make_map(&P.tm_vbhi, P.b.vbhi, kp, C, kReconN) && make_map(&P.tm_vblo, P.b.vblo, kp, C, kReconN)))
+    return CF_ERR_CUDA;
+  // the receiver's expected header (same fields as the stateful decode)
+  Header h{};
+  h.w[0] = kMagic;
+  h.w[1] = (uint32_t)CF_LOWRANK;
+  h.w[2] = 0;
+  h.w[3] = (uint32_t)p->dtype;
+  h.w[4] = (uint32_t)(step & 0xffffffffu);
+  h.w[5] = (uint32_t)(step >> 32);
+  h.w[6] = (uint32_t)((uint64_t)rows & 0xffffffffu);
+  h.w[7] = (uint32_t)((uint64_t)rows >> 32);
+  h.w[8] = (uint32_t)((uint64_t)cols & 0xffffffffu);
+  h.w[9] = (uint32_t)((uint64_t)cols >> 32);
+  h.w[10] = 1;
+  h.w[11] = (uint32_t)p->rank;
+  h.w[12] = (uint32_t)p->lr_int4;
+  h.w[13] = (uint32_t)p->ef;
+  h.w[14] = (uint32_t)p->iters;
+  h.w[15] = 0;
+  const cudaError_t e = dequant_and_recon(P, static_cast<const uint8_t *>(payload), true, h, nullptr, ahat, nullptr,
+                                          recon, status, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return CF_ERR_CUDA;
+  }
+  return CF_OK;
+}

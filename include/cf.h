@@ -104,6 +104,7 @@ extern "C" {
 #define CF_ERR_STATE (-9)        /* handle is not a live state (destroyed or foreign) */
 #define CF_ERR_SIZE (-10)        /* a host buffer size does not match */
 #define CF_ERR_TIMEOUT (-11)     /* (device) a bounded wait for an asynchronous copy gave up */
+#define CF_ERR_TOO_LARGE (-12)   /* problem larger than the allocation-free entry point's fixed scratch */
 
 /* ---- enumerations ---------------------------------------------------- */
 typedef enum { CF_IDENTITY = 0, CF_SIGN1 = 1, CF_Q2 = 2, CF_NM = 3, CF_LOWRANK = 4 } cf_mode;
@@ -207,6 +208,33 @@ CF_API int cf_reset(cf_state *s);
 CF_API int cf_state_bytes(const cf_state *s, size_t *out);
 CF_API int cf_state_export(const cf_state *s, void *host, size_t bytes, void *stream);
 CF_API int cf_state_import(cf_state *s, const void *host, size_t bytes, void *stream);
+
+/* Allocation-free low-rank decode.  The paper has no counterpart: this entry
+ * point exists for callers that cannot allocate device memory at decode
+ * time -- code that runs where cudaMalloc is unavailable or forbidden (inside
+ * a framework that owns every allocation, a fixed-memory serving process, a
+ * library call made from a stream callback or capture-sensitive code path).
+ * It decodes one steady-state low-rank payload exactly as cf_decode does on
+ * a CF_LOWRANK receiver (same kernels, bit-identical ahat and recon), but
+ * with no state object and no allocation: the caller passes the receiver's
+ * reconstruction `ahat` (device fp32 [rows][cols], updated in place), the
+ * output `recon` (device, [rows][cols] in p->dtype), a device status word
+ * `status` (int; the kernels OR in 1 when the payload header does not match
+ * rows, cols, p and `step`, leaving ahat and recon untouched, and 2 when a
+ * bounded wait gave up), the device `payload` and the stream.  p supplies
+ * dtype, ef, rank, iters and lr_int4 (role, batch and workspace are
+ * ignored; batch must be 1).  `step` (>= 1) is the step the payload must
+ * carry; the warm-up step (raw activations) is not handled here.
+ * The dequantised factors go to a fixed scratch array of 8 MiB that every
+ * GPU loading the library holds until exit: (rows*kp*(int4 ? 2 : 4) +
+ * cols*kp*4) bytes, each part rounded up to 256, must fit, where kp is rank
+ * rounded up to 64; larger problems return CF_ERR_TOO_LARGE.  The first call
+ * on a device looks up that array's device address and sets kernel
+ * attributes, so make it before any stream capture.  All calls share the
+ * one array: calls whose work overlaps on the GPU (other streams, other
+ * threads) race; serialise them.  Shape rules as for CF_LOWRANK. */
+CF_API int cf_lowrank_decode_noalloc(int64_t rows, int64_t cols, const cf_params *p, uint64_t step,
+                                     const void *payload, float *ahat, void *recon, int *status, void *stream);
 
 /* Free the state (and its memory, unless it lives in a caller workspace).
  * Synchronises the device first.  Later calls with the handle return

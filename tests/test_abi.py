@@ -34,7 +34,7 @@ def test_every_declared_symbol_is_exported(cf):
 
 def test_strerror_and_version(cf):
     assert "sm_100a" in cf.cf_version()
-    for code in range(0, -12, -1):
+    for code in range(0, -13, -1):
         assert cf.cf_strerror(code) != "unknown status"
     assert cf.cf_strerror(-99) == "unknown status"
 
