@@ -39,7 +39,6 @@ namespace {
 constexpr int kTileM = 128;     // UMMA M and TMA box rows of the A operand
 constexpr int kTileK = 64;      // bf16 per 128-byte swizzled row
 constexpr int kReconN = 128;    // N of a reconstruction tile
-constexpr int kGramRows = 64;   // rows per partial Gram block
 constexpr int kStatusDesync = 1;
 constexpr int kStatusTimeout = 2;
 
@@ -302,98 +301,201 @@ __global__ void __launch_bounds__(128, 1)
 
 // ---------------------------------------------------------------- CholeskyQR2 pieces
 
+// Rows per partial Gram block.
+constexpr int kGramRows = 64;
+
 // X = sum of the nsrc partial slabs (fixed order), stored fp32 [rows][n], and
-// the partial Gram matrix X^T X (fp64) of this block's kGramRows rows.
-__global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc, int64_t rows, int n, float *x,
+// the partial Gram matrix X^T X (fp64) of this block's kGramRows rows: a 16 x
+// 16 thread grid, thread (ty, tx) accumulating the TT x TT sub-block rows
+// ty*TT.., cols tx*TT.. (n = 16 TT) in registers.
+template <int TT>
+__global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc, int64_t rows, float *x,
                                                       double *gpart) {
-  extern __shared__ __align__(16) uint8_t gsm[];
-  float *tile = reinterpret_cast<float *>(gsm);  // [kGramRows][n]
+  constexpr int n = 16 * TT;
+  __shared__ float tile[kGramRows][n + 1];
   const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
   for (int idx = threadIdx.x; idx < kGramRows * n; idx += blockDim.x) {
-    const int64_t off = (r0 + idx / n) * n + idx % n;
+    const int64_t off = r0 * n + idx;
     float acc = src[off];
     for (int p = 1; p < nsrc; p++) acc = __fadd_rn(acc, src[(int64_t)p * rows * n + off]);
-    tile[idx] = acc;
+    tile[idx / n][idx % n] = acc;
     x[off] = acc;
   }
   __syncthreads();
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  double acc[TT][TT];
+#pragma unroll
+  for (int a = 0; a < TT; a++)
+#pragma unroll
+    for (int c = 0; c < TT; c++) acc[a][c] = 0.0;
+  for (int rr = 0; rr < kGramRows; rr++) {
+    double xi[TT], xj[TT];
+#pragma unroll
+    for (int a = 0; a < TT; a++) {
+      xi[a] = (double)tile[rr][ty * TT + a];
+      xj[a] = (double)tile[rr][tx * TT + a];
+    }
+#pragma unroll
+    for (int a = 0; a < TT; a++)
+#pragma unroll
+      for (int c = 0; c < TT; c++) acc[a][c] += xi[a] * xj[c];
+  }
   double *g = gpart + (int64_t)blockIdx.x * n * n;
-  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
-    const int i = e / n, j = e % n;
-    if (j < i) continue;
-    double acc = 0.0;
-    for (int rr = 0; rr < kGramRows; rr++) acc += (double)tile[rr * n + i] * (double)tile[rr * n + j];
-    g[i * n + j] = acc;
-    g[j * n + i] = acc;
-  }
+#pragma unroll
+  for (int a = 0; a < TT; a++)
+#pragma unroll
+    for (int c = 0; c < TT; c++) g[(ty * TT + a) * n + tx * TT + c] = acc[a][c];
 }
 
-// Sum of the partial Gram matrices (fixed order) and its Cholesky factor L
-// (lower, fp64).  A pivot <= 1e-12 G_00 (R_kk <= 1e-6 R_00) marks column k
-// rank deficient: dead[k] = 1, L[k][k] = 1 and L[i][k] = 0 below it.
-__global__ void __launch_bounds__(256) lr_chol_kernel(const double *gpart, int nblk, int n, double *Lout, int *dead) {
+// G = sum over blocks of the partial Gram matrices, in block order.
+__global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart, int nblk, int nn, double *G) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= nn) return;
+  double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+  int b = 0;
+  for (; b + 3 < nblk; b += 4) {
+    a0 += gpart[(int64_t)b * nn + e];
+    a1 += gpart[(int64_t)(b + 1) * nn + e];
+    a2 += gpart[(int64_t)(b + 2) * nn + e];
+    a3 += gpart[(int64_t)(b + 3) * nn + e];
+  }
+  for (; b < nblk; b++) a0 += gpart[(int64_t)b * nn + e];
+  G[e] = (a0 + a1) + (a2 + a3);
+}
+
+// Cholesky factor L of the Gram matrix G (left-looking, fp64) and M = L^-T,
+// in one n x (n+1) shared array: the lower triangle holds G and becomes L;
+// thread c then writes column c of L^-1 into row c of the upper triangle
+// (its diagonal 1/L[c][c] kept apart).  One barrier per column k: thread i
+// >= k forms s_i = G[i][k] - L[i][:k].L[k][:k] and publishes it; after the
+// barrier every thread knows 1/L[k][k] = rsqrt(s_k) and the next row's new
+// entry L[k+1][k] = s_{k+1} / L[k][k] without waiting for it to be stored.
+// A pivot <= 1e-12 G_00 (R_kk <= 1e-6 R_00) marks column k rank deficient:
+// dead[k] = 1, L[k][k] = 1, L[i][k] = 0 below it, and column k of M is zero
+// so that Q's column k is zero.  Writes M fp64 [n][n] (upper triangular).
+__global__ void __launch_bounds__(128) lr_chol_kernel(const double *G, int nblk, int n, double *Mout, int *dead) {
   extern __shared__ __align__(16) uint8_t csm[];
-  double *G = reinterpret_cast<double *>(csm);  // [n][n]
-  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
-    double acc = 0.0;
-    for (int b = 0; b < nblk; b++) acc += gpart[(int64_t)b * n * n + e];
-    G[e] = acc;
+  const int ld = n + 1;                          // padded row stride (bank spread)
+  double *A = reinterpret_cast<double *>(csm);   // [n][ld]
+  __shared__ double sv[2][128];                  // s_i of column k, double-buffered by k's parity
+  __shared__ double rd[128];                     // 1 / L[k][k]
+  __shared__ int dead_s[128];
+  (void)nblk;
+  const int i = threadIdx.x;
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) A[(e / n) * ld + e % n] = G[e];
+  __syncthreads();
+  const double thr = 1e-12 * A[0];
+  double lk_prev = 0.0;  // L[k][k-1] of the row k about to be processed (computed locally)
+  for (int k = 0; k < n; k++) {
+    if (i >= k && i < n) {
+      double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+      int j = 0;
+      const int kk = k - 1;  // columns < k-1 are in shared memory; column k-1 of row k is lk_prev
+      for (; j + 3 < kk; j += 4) {
+        s0 += A[i * ld + j] * A[k * ld + j];
+        s1 += A[i * ld + j + 1] * A[k * ld + j + 1];
+        s2 += A[i * ld + j + 2] * A[k * ld + j + 2];
+        s3 += A[i * ld + j + 3] * A[k * ld + j + 3];
+      }
+      for (; j < kk; j++) s0 += A[i * ld + j] * A[k * ld + j];
+      if (k > 0) s0 += A[i * ld + k - 1] * lk_prev;
+      sv[k & 1][i] = A[i * ld + k] - ((s0 + s1) + (s2 + s3));
+    }
+    // the only barrier of the step: after it, s of column k is known to all;
+    // the next step writes the other half of sv, and a thread can run ahead
+    // into it only after every thread has passed this barrier
+    __syncthreads();
+    const double piv = sv[k & 1][k];
+    const bool dk = !(piv > thr);
+    const double r = dk ? 1.0 : rsqrt(piv);
+    if (i == k) {
+      dead_s[k] = dk ? 1 : 0;
+      rd[k] = r;
+      A[k * ld + k] = dk ? 1.0 : piv * r;
+    } else if (i > k && i < n) {
+      A[i * ld + k] = dk ? 0.0 : sv[k & 1][i] * r;
+    }
+    lk_prev = (k + 1 < n) ? (dk ? 0.0 : sv[k & 1][k + 1] * r) : 0.0;
   }
   __syncthreads();
-  const double thr = 1e-12 * G[0];
-  for (int k = 0; k < n; k++) {
-    const double piv = G[k * n + k];
-    const bool dk = !(piv > thr);
-    __syncthreads();
-    const double lkk = dk ? 1.0 : sqrt(piv);
-    for (int i = k + threadIdx.x; i < n; i += blockDim.x) {
-      if (i == k) G[k * n + k] = lkk;
-      else G[i * n + k] = dk ? 0.0 : G[i * n + k] / lkk;
+  // column c of L^-1 (thread c), forward substitution L x = e_c: x[r] for
+  // r > c goes to A[c][r], x[c] = 1/L[c][c] to rd[c]
+  if (i < n) {
+    for (int r = i + 1; r < n; r++) {
+      double s0 = A[r * ld + i] * rd[i], s1 = 0.0, s2 = 0.0, s3 = 0.0;
+      int j = i + 1;
+      for (; j + 3 < r; j += 4) {
+        s0 += A[r * ld + j] * A[i * ld + j];
+        s1 += A[r * ld + j + 1] * A[i * ld + j + 1];
+        s2 += A[r * ld + j + 2] * A[i * ld + j + 2];
+        s3 += A[r * ld + j + 3] * A[i * ld + j + 3];
+      }
+      for (; j < r; j++) s0 += A[r * ld + j] * A[i * ld + j];
+      A[i * ld + r] = -((s0 + s1) + (s2 + s3)) * rd[r];
     }
-    if (threadIdx.x == 0) dead[k] = dk ? 1 : 0;
-    __syncthreads();
-    const int m = n - k - 1;
-    for (int e = threadIdx.x; e < m * m; e += blockDim.x) {
-      const int i = k + 1 + e / m, j = k + 1 + e % m;
-      if (j <= i) G[i * n + j] -= G[i * n + k] * G[j * n + k];
-    }
-    __syncthreads();
   }
+  __syncthreads();
   for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
-    const int i = e / n, j = e % n;
-    Lout[e] = j <= i ? G[e] : 0.0;
+    const int rr = e / n, c = e % n;  // M[rr][c] = Linv[c][rr]; column c of M zero when c is dead
+    double m = 0.0;
+    if (!dead_s[c]) m = c == rr ? rd[rr] : (c > rr ? A[rr * ld + c] : 0.0);
+    Mout[e] = m;
   }
+  for (int e = threadIdx.x; e < n; e += blockDim.x) dead[e] = dead_s[e];
 }
 
-// Q = X L^-T row by row (forward substitution in fp64); dead columns are 0.
-// Writes Q fp32 [rows][n] and, when qthi != nullptr, Q^T split in bf16
-// ([n][rows], the K-major B operand of V = D^T Q).
-__global__ void lr_apply_kernel(const float *x, const double *L, const int *dead, int64_t rows, int n, float *q,
-                                __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo) {
+// Q = X M (M = L^-T, upper triangular) for 32 rows per block: thread
+// (row, group) computes 10..16 consecutive outputs of its row with
+// independent fp64 accumulators.  Writes Q fp32 [rows][n] and, when
+// qthi != nullptr, Q^T split in bf16 ([n][rows], the K-major B operand of
+// V = D^T Q).
+__global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const double *M, int64_t rows, int n, float *q,
+                                                       __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo) {
   extern __shared__ __align__(16) uint8_t asm_[];
-  double *Ls = reinterpret_cast<double *>(asm_);  // [n][n]
-  double *qs = Ls + n * n;                        // [n][blockDim]
-  int *ds = reinterpret_cast<int *>(qs + (size_t)n * blockDim.x);
-  for (int e = threadIdx.x; e < n * n; e += blockDim.x) Ls[e] = L[e];
-  for (int e = threadIdx.x; e < n; e += blockDim.x) ds[e] = dead[e];
-  __syncthreads();
-  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (row >= rows) return;
-  const int T = blockDim.x;
-  for (int k = 0; k < n; k++) {
-    double acc = (double)x[row * n + k];
-    for (int j = 0; j < k; j++) acc -= Ls[k * n + j] * qs[j * T + threadIdx.x];
-    const double qk = ds[k] ? 0.0 : acc / Ls[k * n + k];
-    qs[k * T + threadIdx.x] = qk;
+  double *Ms = reinterpret_cast<double *>(asm_);  // [n][n]
+  float *xs = reinterpret_cast<float *>(Ms + n * n);  // [32][n]
+  const int64_t r0 = (int64_t)blockIdx.x * 32;
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) Ms[e] = M[e];
+  for (int e = threadIdx.x; e < 32 * n; e += blockDim.x) {
+    const int64_t rr = r0 + e / n;
+    xs[e] = rr < rows ? x[rr * n + e % n] : 0.0f;
   }
-  for (int k = 0; k < n; k++) {
-    const float qf = (float)qs[k * T + threadIdx.x];
-    q[row * n + k] = qf;
-    if (qthi) {
-      __nv_bfloat16 hi, lo;
-      split_bf16(qf, hi, lo);
-      qthi[(int64_t)k * rows + row] = hi;
-      qtlo[(int64_t)k * rows + row] = lo;
+  __syncthreads();
+  const int lr = threadIdx.x >> 3, grp = threadIdx.x & 7;
+  const int per = (n + 7) / 8;  // outputs per thread (<= 16)
+  const int c0 = grp * per;
+  const int64_t row = r0 + lr;
+  double acc[16];
+#pragma unroll
+  for (int t = 0; t < 16; t++) acc[t] = 0.0;
+  // M is upper triangular: rows j < c0 touch every output of the group
+  for (int j = 0; j < c0; j++) {
+    const double xj = (double)xs[lr * n + j];
+    const double *mr = Ms + j * n + c0;
+#pragma unroll
+    for (int t = 0; t < 16; t++)
+      if (t < per) acc[t] += xj * mr[t];
+  }
+  for (int j = c0; j < c0 + per && j < n; j++) {
+    const double xj = (double)xs[lr * n + j];
+    const double *mr = Ms + j * n + c0;
+#pragma unroll
+    for (int t = 0; t < 16; t++)
+      if (t < per && c0 + t >= j && c0 + t < n) acc[t] += xj * mr[t];
+  }
+  if (row >= rows) return;
+#pragma unroll
+  for (int t = 0; t < 16; t++) {
+    const int c = c0 + t;
+    if (t < per && c < n) {
+      const float qf = (float)acc[t];
+      q[row * n + c] = qf;
+      if (qthi) {
+        __nv_bfloat16 hi, lo;
+        split_bf16(qf, hi, lo);
+        qthi[(int64_t)c * rows + row] = hi;
+        qtlo[(int64_t)c * rows + row] = lo;
+      }
     }
   }
 }
@@ -778,8 +880,8 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 size_t thin_smem(int n, int stages) { return (size_t)stages * (2u * kTileM * kTileK * 2 + 2u * n * kTileK * 2) + 1024; }
 int thin_stages(int n) { return n <= 96 ? 4 : 3; }
 size_t recon_smem(int kblocks, int a_split) { return (size_t)kblocks * kTileM * kTileK * 2 * (3 + a_split) + 1024; }
-size_t apply_smem(int n, int threads) { return (size_t)n * n * 8 + (size_t)n * threads * 8 + (size_t)n * 4; }
-int apply_threads(int n) { return n <= 96 ? 128 : 64; }
+size_t apply_smem(int n) { return (size_t)n * n * 8 + (size_t)32 * n * 4; }
+size_t chol_smem(int n) { return (size_t)n * (n + 1) * 8; }
 
 }  // namespace
 
@@ -872,11 +974,10 @@ int lowrank_bind(LowrankPlan *plan, void *scratch) {
                            (int)recon_smem(plan->kp / kTileK, 1)) != cudaSuccess ||
       cudaFuncSetAttribute(lr_recon_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)recon_smem(plan->kp / kTileK, 1)) != cudaSuccess ||
-      cudaFuncSetAttribute(lr_chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rpi * rpi * 8) != cudaSuccess ||
-      cudaFuncSetAttribute(lr_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)apply_smem(rpi, apply_threads(rpi))) != cudaSuccess ||
-      cudaFuncSetAttribute(lr_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kGramRows * rpi * 4) != cudaSuccess) {
+      cudaFuncSetAttribute(lr_chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)chol_smem(rpi)) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(lr_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)apply_smem(rpi)) !=
+          cudaSuccess) {
     (void)cudaGetLastError();
     return CF_ERR_CUDA;
   }
@@ -901,16 +1002,35 @@ cudaError_t launch_thin(const LowrankPlan &P, const CUtensorMap &ah, const CUten
   return cudaGetLastError();
 }
 
+cudaError_t launch_gram(int n, int nblk, const float *src, int nsrc, int64_t rows, float *x, double *gpart,
+                        cudaStream_t st) {
+  switch (n / 16) {
+    case 1: lr_gram_kernel<1><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
+    case 2: lr_gram_kernel<2><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
+    case 3: lr_gram_kernel<3><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
+    case 4: lr_gram_kernel<4><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
+    case 5: lr_gram_kernel<5><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
+    case 6: lr_gram_kernel<6><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
+    case 7: lr_gram_kernel<7><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
+    case 8: lr_gram_kernel<8><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int64_t rows, bool final_pass,
                            cudaStream_t st) {
   const LowrankBufs &b = P.b;
   const int n = P.rp;
   const int nblk = (int)(rows / kGramRows);
-  lr_gram_kernel<<<nblk, 256, kGramRows * n * 4, st>>>(src, nsrc, rows, n, b.xbuf, b.gpart);
-  lr_chol_kernel<<<1, 256, (size_t)n * n * 8, st>>>(b.gpart, nblk, n, b.L, b.dead);
-  const int th = apply_threads(n);
-  lr_apply_kernel<<<(unsigned)((rows + th - 1) / th), th, apply_smem(n, th), st>>>(
-      b.xbuf, b.L, b.dead, rows, n, b.q, final_pass ? b.qthi : nullptr, final_pass ? b.qtlo : nullptr);
+  cudaError_t e = launch_gram(n, nblk, src, nsrc, rows, b.xbuf, b.gpart, st);
+  if (e != cudaSuccess) return e;
+  // the reduced Gram matrix goes to the head of the partial buffer's last
+  // slot region (L, which the Cholesky kernel then overwrites with M)
+  lr_gram_reduce_kernel<<<(n * n + 255) / 256, 256, 0, st>>>(b.gpart, nblk, n * n, b.L);
+  lr_chol_kernel<<<1, 128, chol_smem(n), st>>>(b.L, 1, n, b.L, b.dead);
+  lr_apply_kernel<<<(unsigned)((rows + 31) / 32), 256, apply_smem(n), st>>>(
+      b.xbuf, b.L, rows, n, b.q, final_pass ? b.qthi : nullptr, final_pass ? b.qtlo : nullptr);
   return cudaGetLastError();
 }
 

@@ -281,6 +281,122 @@ def run_cf(args, rank, world, device):
     return stats
 
 
+def _lr_alg_bytes(rows, cols, iters, payload):
+    """Low-rank step's algorithmic bytes: read a, ahat, e and write ahat, e once
+    (sender), re-read the residual as one bf16 copy per GEMM (2 per iteration),
+    read and write the receiver's ahat and write recon, plus the payload twice."""
+    E = rows * cols
+    return E * (2 + 16 + 4 * iters) + E * (4 + 4 + 2) + 2 * payload
+
+
+def run_suite(args, device):
+    """The other workloads, timed the same way (CUDA events around each
+    encode and decode on the launching stream, inputs resident)."""
+    import torch
+
+    import activation_residual_compression_b200 as cf
+    from activation_residual_compression_b200 import inputs
+
+    peak, _ = _peaks()
+    stream = torch.cuda.Stream()
+    out = {}
+
+    def timed(S, R, pay, recs, acts, steps, warm, batched):
+        def one(i, evs=None):
+            a = acts[i % len(acts)]
+            if evs is not None:
+                evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
+            if batched:
+                cf.cf_encode_batched(S, [a[b] for b in range(a.shape[0])], pay, stream)
+            else:
+                cf.cf_encode(S, a, pay, stream)
+            if evs is not None:
+                evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
+            if batched:
+                cf.cf_decode_batched(R, pay, recs, stream)
+            else:
+                cf.cf_decode(R, pay, recs, stream)
+            if evs is not None:
+                evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
+        with torch.cuda.stream(stream):
+            for i in range(warm):
+                one(i)
+            evs = []
+            for i in range(warm, warm + steps):
+                one(i, evs)
+        torch.cuda.synchronize()
+        enc = [evs[3 * k].elapsed_time(evs[3 * k + 1]) for k in range(steps)]
+        dec = [evs[3 * k + 1].elapsed_time(evs[3 * k + 2]) for k in range(steps)]
+        if cf.cf_status(R, stream) != cf.CF_OK or cf.cf_status(S, stream) != cf.CF_OK:
+            raise RuntimeError("suite: a codec reported an error status")
+        return statistics.mean(enc), statistics.mean(dec)
+
+    def make(rows, cols, mode, kw, batch=1):
+        base = dict(dtype=cf.CF_BF16, batch=batch, **kw)
+        S = cf.cf_create(rows, cols, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_SENDER, **base))
+        R = cf.cf_create(rows, cols, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_RECEIVER, **base))
+        pay = torch.empty(max(cf.cf_payload_bytes(S, True), cf.cf_payload_bytes(S, False)), dtype=torch.uint8,
+                          device="cuda")
+        return S, R, pay
+
+    # N:M 1:16 and 2:16 on the FLUX-shaped stream
+    for n in (1, 2):
+        kw = {"nm_n": n, "nm_m": 16}
+        s = inputs.flux("cuda", rows=ROWS, cols=COLS, seed=5)
+        acts = [s.next() for _ in range(24)]
+        S, R, pay = make(ROWS, COLS, "nm", kw)
+        rec = torch.empty(ROWS, COLS, dtype=torch.bfloat16, device="cuda")
+        e_ms, d_ms = timed(S, R, pay, rec, acts, 20, 4, False)
+        alg = encode_bytes("nm", ROWS, COLS, kw) + decode_bytes("nm", ROWS, COLS, kw)
+        P = 64 + _payload_body("nm", ROWS, COLS, kw)
+        out[f"nm{n}_16_flux"] = {"ms_per_step": round(e_ms + d_ms, 5), "encode_ms": round(e_ms, 5),
+                                 "decode_ms": round(d_ms, 5),
+                                 "activation_gbs": round(ROWS * COLS * 2 / ((e_ms + d_ms) / 1e3) / 1e9, 2),
+                                 "roofline_frac": round(alg / ((e_ms + d_ms) / 1e3) / 1e9 / peak, 4),
+                                 "ratio_vs_bf16": round(ROWS * COLS * 2 / P, 2)}
+        cf.cf_destroy(S); cf.cf_destroy(R)
+        del acts
+    # low-rank ~100x on 4096 x 3072, rank 70, INT4, 1 and 2 iterations
+    lr_rows, lr_cols = 4096, 3072
+    for it in (1, 2):
+        s = inputs.ar1("cuda", rows=lr_rows, cols=lr_cols)
+        acts = [s.next() for _ in range(28)]
+        S, R, pay = make(lr_rows, lr_cols, "lowrank", {"rank": 70, "iters": it, "lr_int4": 1, "seed": 7})
+        rec = torch.empty(lr_rows, lr_cols, dtype=torch.bfloat16, device="cuda")
+        e_ms, d_ms = timed(S, R, pay, rec, acts, 20, 5, False)
+        P = cf.cf_payload_bytes(S, False)
+        alg = _lr_alg_bytes(lr_rows, lr_cols, it, P)
+        out[f"lowrank_r70_k{it}"] = {"ms_per_step": round(e_ms + d_ms, 5), "encode_ms": round(e_ms, 5),
+                                     "decode_ms": round(d_ms, 5),
+                                     "activation_gbs": round(lr_rows * lr_cols * 2 / ((e_ms + d_ms) / 1e3) / 1e9, 2),
+                                     "roofline_frac": round(alg / ((e_ms + d_ms) / 1e3) / 1e9 / peak, 4),
+                                     "payload_bytes": P, "ratio_vs_bf16": round(lr_rows * lr_cols * 2 / P, 2),
+                                     "budget_note": "pages quote a ~1 ms compression budget"}
+        cf.cf_destroy(S); cf.cf_destroy(R)
+        del acts
+    # CogVideoX-2b-shaped full step: 60 tensors of 17550 x 1920, Q2, one launch each way
+    if not args.no_cogvideox:
+        B, cr, cc = 60, 17550, 1920
+        s = inputs.cogvideox("cuda")
+        acts = [s.next() for _ in range(3)]
+        del s
+        torch.cuda.empty_cache()
+        S, R, pay = make(cr, cc, "q2", {}, batch=B)
+        recs = [torch.empty(cr, cc, dtype=torch.bfloat16, device="cuda") for _ in range(B)]
+        e_ms, d_ms = timed(S, R, pay, recs, acts, 6, 2, True)
+        E = B * cr * cc
+        alg = B * (encode_bytes("q2", cr, cc, {}) + decode_bytes("q2", cr, cc, {}))
+        out["cogvideox_q2_60x17550x1920"] = {"ms_per_step": round(e_ms + d_ms, 4), "encode_ms": round(e_ms, 4),
+                                             "decode_ms": round(d_ms, 4),
+                                             "activation_gbs": round(E * 2 / ((e_ms + d_ms) / 1e3) / 1e9, 2),
+                                             "roofline_frac": round(alg / ((e_ms + d_ms) / 1e3) / 1e9 / peak, 4),
+                                             "launches_per_step": 2}
+        cf.cf_destroy(S); cf.cf_destroy(R)
+        del acts, recs
+    torch.cuda.empty_cache()
+    return out
+
+
 def cpu_baseline(max_seconds=20.0):
     """The CPU oracle, as it stands, on the same workload: full 4608 x 3072 bf16
     FLUX-shaped stream, both modes, compressed steps until max_seconds of oracle
@@ -362,6 +478,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--max-resident", type=int, default=400, help="pre-generated inputs per mode (cycled)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-suite", action="store_true", help="skip the supplementary workloads")
+    ap.add_argument("--no-cogvideox", action="store_true", help="skip the 60-tensor CogVideoX-shaped step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -433,6 +551,8 @@ def main():
         line["e2e"] = {"value": round(act_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                        "h2d_bytes_per_step": st["e2e"]["h2d"], "d2h_bytes_per_step": st["e2e"]["d2h"],
                        "ms_per_step": round(e2e_ms, 4)}
+    if world == 1 and not args.no_suite:
+        line["suite"] = run_suite(args, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:
