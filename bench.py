@@ -45,6 +45,20 @@ MODES = [("sign1", {}), ("q2", {})]
 WORKLOAD = "flux1dev-4608x3072-bf16"
 METRIC = "activation GB/s and ms/step per mode (encode+EF+decode), % of B200 HBM roofline"
 
+# Timed workloads (--workload): shape, batch, seeded stream and the codecs one
+# step runs (each codec has its own sender/receiver pair and its own stream).
+WORKLOADS = {
+    "flux": dict(name=WORKLOAD, rows=ROWS, cols=COLS, batch=1, stream="flux", codecs=MODES),
+    "nm": dict(name="flux1dev-4608x3072-bf16-nm16", rows=ROWS, cols=COLS, batch=1, stream="flux",
+               codecs=[("nm", {"nm_n": 1, "nm_m": 16}), ("nm", {"nm_n": 2, "nm_m": 16})]),
+    "lowrank": dict(name="ar1-4096x3072-bf16-rank70-int4-k1", rows=4096, cols=3072, batch=1, stream="ar1",
+                    codecs=[("lowrank", {"rank": 70, "iters": 1, "lr_int4": 1, "seed": 7})]),
+    "lowrank2": dict(name="ar1-4096x3072-bf16-rank70-int4-k2", rows=4096, cols=3072, batch=1, stream="ar1",
+                     codecs=[("lowrank", {"rank": 70, "iters": 2, "lr_int4": 1, "seed": 7})]),
+    "cogvideox": dict(name="cogvideox2b-60x17550x1920-bf16", rows=17550, cols=1920, batch=60, stream="cogvideox",
+                      codecs=[("q2", {})]),
+}
+
 
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -159,38 +173,92 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- GPU arm
 
+def _codec_name(mode, kw):
+    if mode == "nm":
+        return f"nm{kw['nm_n']}_{kw['nm_m']}"
+    if mode == "lowrank":
+        return f"lowrank_r{kw['rank']}_k{kw['iters']}"
+    return mode
+
+
+def _make_stream(kind, wl, seed, device="cuda"):
+    from activation_residual_compression_b200 import inputs
+    if kind == "flux":
+        return inputs.flux(device, rows=wl["rows"], cols=wl["cols"], seed=seed)
+    if kind == "ar1":
+        return inputs.ar1(device, rows=wl["rows"], cols=wl["cols"], seed=seed)
+    if kind == "cogvideox":
+        return inputs.cogvideox(device, rows=wl["rows"], cols=wl["cols"], n_tensors=wl["batch"])
+    raise ValueError(kind)
+
+
+def step_bytes(mode, rows, cols, kw, payload):
+    """Algorithmic bytes of one encode + decode of one tensor."""
+    if mode == "lowrank":
+        return _lr_alg_bytes(rows, cols, kw["iters"], payload)
+    return encode_bytes(mode, rows, cols, kw) + decode_bytes(mode, rows, cols, kw)
+
+
+def launches_per_call(mode, kw, encode):
+    """libcf kernels one steady-state cf_encode / cf_decode call launches."""
+    if mode != "lowrank":
+        return 1
+    if not encode:
+        return 2                                   # dequantise, reconstruction
+    return 2 + 11 * kw["iters"] + 2 + 2            # V prep, residual; per sweep: 2 GEMMs, 2 x 4 orth., V sum;
+                                                   # scales, pack; dequantise, reconstruction
+
+
 def run_cf(args, rank, world, device):
     import torch
 
     import activation_residual_compression_b200 as cf
-    from activation_residual_compression_b200 import inputs
 
+    wl = WORKLOADS[args.workload]
+    R_, C_, B_ = wl["rows"], wl["cols"], wl["batch"]
     torch.cuda.set_device(device)
     stream = torch.cuda.Stream()
     K, W = args.steps, args.warmup
-    n_inputs = min(W + K + 1, args.max_resident)
+    in_bytes = B_ * R_ * C_ * 2
+    n_inputs = max(2, min(W + K + 1, args.max_resident, int(args.resident_gb * 1e9 // (in_bytes * len(wl["codecs"])))))
+    batched = B_ > 1
     codecs = []
-    for mi, (mode, kw) in enumerate(MODES):
-        s = inputs.flux("cuda", rows=ROWS, cols=COLS, seed=1 + 100 * mi + 1000 * rank)
+    for mi, (mode, kw) in enumerate(wl["codecs"]):
+        s = _make_stream(wl["stream"], wl, seed=1 + 100 * mi + 1000 * rank)
         acts = [s.next() for _ in range(n_inputs)]
-        base = dict(dtype=cf.CF_BF16, **kw)
-        S = cf.cf_create(ROWS, COLS, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_SENDER, **base))
-        R = cf.cf_create(ROWS, COLS, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_RECEIVER, **base))
+        del s
+        base = dict(dtype=cf.CF_BF16, batch=B_, **kw)
+        S = cf.cf_create(R_, C_, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_SENDER, **base))
+        R = cf.cf_create(R_, C_, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_RECEIVER, **base))
         pay = torch.empty(max(cf.cf_payload_bytes(S, True), cf.cf_payload_bytes(S, False)), dtype=torch.uint8,
                           device="cuda")
-        rec = torch.empty(ROWS, COLS, dtype=torch.bfloat16, device="cuda")
-        codecs.append(dict(mode=mode, kw=kw, S=S, R=R, pay=pay, rec=rec, acts=acts))
+        rec = torch.empty(B_, R_, C_, dtype=torch.bfloat16, device="cuda")
+        codecs.append(dict(mode=mode, kw=kw, name=_codec_name(mode, kw), S=S, R=R, pay=pay, rec=rec, acts=acts,
+                           P=cf.cf_payload_bytes(S, False)))
+    torch.cuda.empty_cache()
     torch.cuda.synchronize()
+
+    def enc(c, a):
+        if batched:
+            cf.cf_encode_batched(c["S"], [a[b] for b in range(B_)], c["pay"], stream)
+        else:
+            cf.cf_encode(c["S"], a, c["pay"], stream)
+
+    def dec(c):
+        if batched:
+            cf.cf_decode_batched(c["R"], c["pay"], [c["rec"][b] for b in range(B_)], stream)
+        else:
+            cf.cf_decode(c["R"], c["pay"], c["rec"], stream)
 
     def step(i, evs=None):
         for c in codecs:
             a = c["acts"][i % n_inputs]
             if evs is not None:
                 evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
-            cf.cf_encode(c["S"], a, c["pay"], stream)
+            enc(c, a)
             if evs is not None:
                 evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
-            cf.cf_decode(c["R"], c["pay"], c["rec"], stream)
+            dec(c)
         if evs is not None:
             evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
 
@@ -222,28 +290,24 @@ def run_cf(args, rank, world, device):
     torch.cuda.synchronize()
     clk = clocks.stop()
     total_ms = t0.elapsed_time(t1)
-    # per-kernel durations: evs per step = [pre_enc0, pre_dec0/post_enc0, pre_enc1 ..., end]
-    nm = len(codecs)
-    per = {c["mode"]: {"enc": [], "dec": []} for c in codecs}
     # events per step: for each codec (before encode, before decode), then one at the end
+    nm = len(codecs)
     stride = 2 * nm + 1
+    per = {c["name"]: {"enc": [], "dec": []} for c in codecs}
     for k in range(K):
         base = k * stride
         for mi, c in enumerate(codecs):
-            e_enc0 = evs[base + 2 * mi]
-            e_dec0 = evs[base + 2 * mi + 1]
-            e_next = evs[base + 2 * mi + 2]
-            per[c["mode"]]["enc"].append(e_enc0.elapsed_time(e_dec0))
-            per[c["mode"]]["dec"].append(e_dec0.elapsed_time(e_next))
+            per[c["name"]]["enc"].append(evs[base + 2 * mi].elapsed_time(evs[base + 2 * mi + 1]))
+            per[c["name"]]["dec"].append(evs[base + 2 * mi + 1].elapsed_time(evs[base + 2 * mi + 2]))
     for c in codecs:
-        if cf.cf_status(c["R"], stream) != cf.CF_OK:
-            raise RuntimeError(f"receiver of {c['mode']} reported a desync")
+        if cf.cf_status(c["R"], stream) != cf.CF_OK or cf.cf_status(c["S"], stream) != cf.CF_OK:
+            raise RuntimeError(f"codec {c['name']} reported an error status")
 
     # e2e: pinned host activations in, pinned host reconstruction out
     e2e = None
     if args.e2e_steps > 0:
         host_in = [c["acts"][0].cpu().pin_memory() for c in codecs]
-        host_out = [torch.empty(ROWS, COLS, dtype=torch.bfloat16).pin_memory() for _ in codecs]
+        host_out = [torch.empty_like(c["rec"], device="cpu").pin_memory() for c in codecs]
         dev_in = [torch.empty_like(h, device="cuda") for h in host_in]
         for c in codecs:
             cf.cf_reset(c["S"]); cf.cf_reset(c["R"])
@@ -251,8 +315,8 @@ def run_cf(args, rank, world, device):
         def e2e_step():
             for ci, c in enumerate(codecs):
                 dev_in[ci].copy_(host_in[ci], non_blocking=True)
-                cf.cf_encode(c["S"], dev_in[ci], c["pay"], stream)
-                cf.cf_decode(c["R"], c["pay"], c["rec"], stream)
+                enc(c, dev_in[ci])
+                dec(c)
                 host_out[ci].copy_(c["rec"], non_blocking=True)
 
         with torch.cuda.stream(stream):
@@ -272,12 +336,15 @@ def run_cf(args, rank, world, device):
         e2e_ms = a0.elapsed_time(a1) / args.e2e_steps
         e2e = dict(ms=e2e_ms, h2d=sum(t.numel() * 2 for t in host_in), d2h=sum(t.numel() * 2 for t in host_out))
 
+    info = [dict(mode=c["mode"], kw=c["kw"], name=c["name"], P=c["P"]) for c in codecs]
     for c in codecs:
         cf.cf_destroy(c["S"]); cf.cf_destroy(c["R"])
+    del codecs
+    torch.cuda.empty_cache()
 
     ms_step = total_ms / K
     stats = dict(ms_step=ms_step, per={m: {k: statistics.mean(v) for k, v in d.items()} for m, d in per.items()},
-                 e2e=e2e, clocks=clk)
+                 e2e=e2e, clocks=clk, codecs=info)
     return stats
 
 
@@ -397,21 +464,29 @@ def run_suite(args, device):
     return out
 
 
-def cpu_baseline(max_seconds=20.0):
-    """The CPU oracle, as it stands, on the same workload: full 4608 x 3072 bf16
-    FLUX-shaped stream, both modes, compressed steps until max_seconds of oracle
-    time (warm-up step untimed)."""
+def cpu_baseline(wl=None, max_seconds=20.0):
+    """The CPU oracle, as it stands, on the same workload (full-size tensors;
+    for the 60-tensor step the first tensors only, tensors being independent),
+    steps until max_seconds of oracle time (the warm-up step untimed)."""
     import numpy as np
     import torch
 
     import oracle
+
+    wl = wl or WORKLOADS["flux"]
+    R_, C_, B_ = wl["rows"], wl["cols"], wl["batch"]
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    nt = 1 if B_ > 1 else B_
     from activation_residual_compression_b200 import inputs
 
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     orcs = []
-    for mi, (mode, kw) in enumerate(MODES):
-        s = inputs.flux("cpu", rows=ROWS, cols=COLS, seed=1 + 100 * mi)
-        o = oracle.Oracle(ROWS, COLS, mode, dtype="bf16", **kw)
+    for mi, (mode, kw) in enumerate(wl["codecs"]):
+        if wl["stream"] == "cogvideox":   # the first tensor of the step (seed and sigma of layer 0)
+            s = inputs.ActivationStream(R_, C_, dtype=torch.bfloat16, device="cpu", seed_per_tensor=[1000],
+                                        sigma_per_tensor=inputs.cogvideox_sigmas(B_)[:1])
+        else:
+            s = _make_stream(wl["stream"], wl, seed=1 + 100 * mi, device="cpu")
+        o = oracle.Oracle(R_, C_, mode, dtype="bf16", batch=nt, **kw)
         a = s.next().view(torch.int16).numpy().view(np.uint16)
         o.decode(o.encode(a))
         orcs.append((s, o))
@@ -423,28 +498,40 @@ def cpu_baseline(max_seconds=20.0):
             o.decode(o.encode(a))
         spent += time.perf_counter() - t
         steps += 1
-    act_bytes = steps * len(MODES) * ROWS * COLS * 2
+    act_bytes = steps * len(orcs) * nt * R_ * C_ * 2
+    what = f"{steps} compressed steps of {nt} full {R_}x{C_} bf16 tensor(s)" + \
+        (f" (of the {B_}-tensor step)" if B_ > 1 else "")
     return {"value": act_bytes / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{steps} compressed steps of the full {ROWS}x{COLS} bf16 stream, modes "
-                      f"{'+'.join(m for m, _ in MODES)} (encode+decode), {spent:.1f} s of oracle time",
+            "sample": f"{what}, modes {'+'.join(_codec_name(m, k) for m, k in wl['codecs'])} (encode+decode), "
+                      f"{spent:.1f} s of oracle time",
             "ms_per_step": spent / steps * 1e3}
 
 
 def run_reference(args):
-    """The oracle as the reference arm: each step = encode+decode in both modes of
-    a 1152-row sample (a quarter of the rows; rows are independent) of the stream."""
+    """The oracle as the reference arm, on the workload's codecs.  Streaming
+    modes: each step is encode + decode of a 1152-row sample of the stream
+    (rows are independent in these modes, so a row sample is the same per-row
+    work); the low-rank mode couples all rows, so its steps are full tensors."""
     import numpy as np
     import torch
 
     import oracle
     from activation_residual_compression_b200 import inputs
 
-    rows = 1152
+    wl = WORKLOADS[args.workload]
+    R_, C_ = wl["rows"], wl["cols"]
+    lowrank = any(m == "lowrank" for m, _ in wl["codecs"])
+    rows = R_ if lowrank else 1152
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     orcs = []
-    for mi, (mode, kw) in enumerate(MODES):
-        s = inputs.flux("cpu", rows=rows, cols=COLS, seed=1 + 100 * mi)
-        orcs.append((s, oracle.Oracle(rows, COLS, mode, dtype="bf16", **kw)))
+    for mi, (mode, kw) in enumerate(wl["codecs"]):
+        sub = dict(wl, rows=rows)
+        if wl["stream"] == "cogvideox":
+            s = inputs.ActivationStream(rows, C_, dtype=torch.bfloat16, device="cpu", seed_per_tensor=[1000],
+                                        sigma_per_tensor=inputs.cogvideox_sigmas(wl["batch"])[:1])
+        else:
+            s = _make_stream(wl["stream"], sub, seed=1 + 100 * mi, device="cpu")
+        orcs.append((s, oracle.Oracle(rows, C_, mode, dtype="bf16", **kw)))
 
     def one():
         ins = [s.next().view(torch.int16).numpy().view(np.uint16) for s, _ in orcs]
@@ -458,13 +545,15 @@ def run_reference(args):
         one()
     spent = sum(one() for _ in range(args.steps))
     ms = spent / args.steps * 1e3
-    val = len(MODES) * rows * COLS * 2 / (ms / 1e3) / 1e9
+    val = len(orcs) * rows * C_ * 2 / (ms / 1e3) / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "modes": [m for m, _ in MODES], "sample_rows": rows},
+            "config": {"workload": wl["name"], "modes": [_codec_name(m, k) for m, k in wl["codecs"]],
+                       "sample_rows": rows},
             "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{rows} of {ROWS} rows x {COLS} bf16 per step, both modes"},
+                             "sample": f"{rows} of {R_} rows x {C_} bf16 per step, "
+                                       f"{'+'.join(_codec_name(m, k) for m, k in wl['codecs'])}"},
             "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -479,6 +568,9 @@ def main():
     ap.add_argument("--max-resident", type=int, default=400, help="pre-generated inputs per mode (cycled)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-suite", action="store_true", help="skip the supplementary workloads")
+    ap.add_argument("--workload", default="flux", choices=sorted(WORKLOADS),
+                    help="timed workload (default: the FLUX-shaped 1-bit + 2-bit step)")
+    ap.add_argument("--resident-gb", type=float, default=12.0, help="device memory for pre-generated inputs")
     ap.add_argument("--no-cogvideox", action="store_true", help="skip the 60-tensor CogVideoX-shaped step")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -505,56 +597,70 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     st = run_cf(args, rank, world, local)
+    wl = WORKLOADS[args.workload]
+    R_, C_, B_ = wl["rows"], wl["cols"], wl["batch"]
     ms = st["ms_step"]
     e2e_ms = st["e2e"]["ms"] if st["e2e"] else None
     if dist:
         t = torch.tensor([ms, e2e_ms or 0.0], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms, e2e_ms = float(t[0]), float(t[1])
-    act_bytes = len(MODES) * ROWS * COLS * 2 * world
+    n_codecs = len(st["codecs"])
+    act_bytes = n_codecs * B_ * R_ * C_ * 2 * world
     value = act_bytes / (ms / 1e3) / 1e9
     peak, peak_kind = _peaks()
-    m0, kw0 = MODES[0]
-    enc_ms = st["per"][m0]["enc"]
-    achieved = encode_bytes(m0, ROWS, COLS, kw0) / (enc_ms / 1e3) / 1e9
-    tr = _traffic_record()
+    c0 = st["codecs"][0]
+    enc_ms = st["per"][c0["name"]]["enc"]
+    if c0["mode"] == "lowrank":
+        E = R_ * C_
+        enc_alg = E * (2 + 16 + 4 * c0["kw"]["iters"]) + c0["P"]
+        kern = f"cf_encode low-rank ({launches_per_call(c0['mode'], c0['kw'], True)} launches)"
+        tr = None
+    else:
+        enc_alg = B_ * encode_bytes(c0["mode"], R_, C_, c0["kw"])
+        kern = f"encode_kernel<{c0['name']}, bf16>"
+        tr = _traffic_record() if args.workload == "flux" else None
+    achieved = enc_alg / (enc_ms / 1e3) / 1e9
     per_mode = {}
-    for m, kw in MODES:
-        pm = st["per"][m]
+    for c in st["codecs"]:
+        pm = st["per"][c["name"]]
         step_ms = pm["enc"] + pm["dec"]
-        alg = encode_bytes(m, ROWS, COLS, kw) + decode_bytes(m, ROWS, COLS, kw)
-        per_mode[m] = {"ms_per_step": round(step_ms, 5), "encode_ms": round(pm["enc"], 5),
-                       "decode_ms": round(pm["dec"], 5),
-                       "activation_gbs": round(ROWS * COLS * 2 / (step_ms / 1e3) / 1e9, 2),
-                       "hbm_gbs": round(alg / (step_ms / 1e3) / 1e9, 1),
-                       "roofline_frac": round(alg / (step_ms / 1e3) / 1e9 / peak, 4),
-                       "payload_bytes": 64 + _payload_body(m, ROWS, COLS, kw),
-                       "ratio_vs_bf16": round(ROWS * COLS * 2 / (64 + _payload_body(m, ROWS, COLS, kw)), 2)}
+        alg = B_ * step_bytes(c["mode"], R_, C_, c["kw"], c["P"])
+        per_mode[c["name"]] = {"ms_per_step": round(step_ms, 5), "encode_ms": round(pm["enc"], 5),
+                               "decode_ms": round(pm["dec"], 5),
+                               "activation_gbs": round(B_ * R_ * C_ * 2 / (step_ms / 1e3) / 1e9, 2),
+                               "hbm_gbs": round(alg / (step_ms / 1e3) / 1e9, 1),
+                               "roofline_frac": round(alg / (step_ms / 1e3) / 1e9 / peak, 4),
+                               "payload_bytes": c["P"],
+                               "ratio_vs_bf16": round(B_ * R_ * C_ * 2 / c["P"], 2)}
+    in_mb = B_ * R_ * C_ * 2 / 1e6
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "activation_dtype": "bf16",
-                   "modes": [m for m, _ in MODES], "error_feedback": "explicit",
+        "config": {"workload": wl["name"], "rows": R_, "cols": C_, "tensors": B_, "activation_dtype": "bf16",
+                   "modes": [c["name"] for c in st["codecs"]], "error_feedback": "explicit",
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "inputs larger than L2: fresh 28 MB input per step, per-kernel working set 170-230 MB",
+                   "l2": f"inputs larger than L2: a fresh {in_mb:.0f} MB input per codec per step, state "
+                         f"{B_ * R_ * C_ * 12 / 1e6:.0f} MB per codec",
                    "inputs_resident": True},
         "per_mode": per_mode,
-        "roofline": {"bound": "hbm", "kernel": f"encode_kernel<{m0}, bf16>", "achieved": round(achieved, 1),
+        "roofline": {"bound": "hbm", "kernel": kern, "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": (tr["bytes_per_launch"] if tr else None),
-                     "algorithmic_bytes": encode_bytes(m0, ROWS, COLS, kw0), "peak_source": peak_kind},
-        "gpu_launches": 2 * len(MODES) * args.steps,
+                     "algorithmic_bytes": enc_alg, "peak_source": peak_kind},
+        "gpu_launches": sum(launches_per_call(c["mode"], c["kw"], True) + launches_per_call(c["mode"], c["kw"], False)
+                            for c in st["codecs"]) * args.steps,
         "clocks": st["clocks"],
     }
     if e2e_ms:
         line["e2e"] = {"value": round(act_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                        "h2d_bytes_per_step": st["e2e"]["h2d"], "d2h_bytes_per_step": st["e2e"]["d2h"],
                        "ms_per_step": round(e2e_ms, 4)}
-    if world == 1 and not args.no_suite:
+    if world == 1 and not args.no_suite and args.workload == "flux":
         line["suite"] = run_suite(args, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
+        line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:
