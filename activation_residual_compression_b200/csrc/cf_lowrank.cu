@@ -677,64 +677,19 @@ struct ReconArgs {
   Header expect;
 };
 
-template <typename T>
-__device__ __forceinline__ void load16_act(const T *p, float (&x)[16]) {
-  if constexpr (sizeof(T) == 2) {
-    const uint4 u0 = reinterpret_cast<const uint4 *>(p)[0], u1 = reinterpret_cast<const uint4 *>(p)[1];
-    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-    for (int k = 0; k < 8; k++) {
-      x[2 * k] = __uint_as_float(w[k] << 16);
-      x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-    }
-  } else {
-    const float4 *q = reinterpret_cast<const float4 *>(p);
-#pragma unroll
-    for (int k = 0; k < 4; k++) {
-      const float4 f = q[k];
-      x[4 * k] = f.x; x[4 * k + 1] = f.y; x[4 * k + 2] = f.z; x[4 * k + 3] = f.w;
-    }
-  }
-}
-
-__device__ __forceinline__ void load16_f32(const float *p, float (&x)[16]) {
-  const float4 *q = reinterpret_cast<const float4 *>(p);
-#pragma unroll
-  for (int k = 0; k < 4; k++) {
-    const float4 f = __ldcs(q + k);
-    x[4 * k] = f.x; x[4 * k + 1] = f.y; x[4 * k + 2] = f.z; x[4 * k + 3] = f.w;
-  }
-}
-
-__device__ __forceinline__ void store16_f32(float *p, const float (&x)[16]) {
-  float4 *q = reinterpret_cast<float4 *>(p);
-#pragma unroll
-  for (int k = 0; k < 4; k++) __stcs(q + k, make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]));
-}
-
-template <typename T>
-__device__ __forceinline__ void store16_act(T *p, const float (&x)[16]) {
-  if constexpr (sizeof(T) == 2) {
-    uint32_t w[8];
-#pragma unroll
-    for (int k = 0; k < 8; k++) {
-      w[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[2 * k])) |
-             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[2 * k + 1])) << 16);
-    }
-    uint4 *q = reinterpret_cast<uint4 *>(p);
-    q[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    q[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  } else {
-    store16_f32(reinterpret_cast<float *>(p), x);
-  }
-}
-
 // C tile (128 rows x 128 cols) = A[rows tile] * B[cols tile]^T over K = kp,
 // products hi*hi + hi*lo (+ lo*hi when A is split), then the fused update:
 // sender: D = (a - ahat) + e recomputed bit for bit; e = D - C; ahat = ahat + C;
 // receiver: ahat = ahat + C; recon = cast(ahat).
+// 8 warps: warp 0 lane 0 loads the operands (TMA) and issues the MMAs; after
+// they complete, warp w drains TMEM lanes 32 (w % 4).., columns 64 (w / 4)..
+// into a padded shared-memory C tile (the operand buffers are free by then),
+// and all warps update whole rows with coalesced 512-byte accesses.
+constexpr int kReconThreads = 256;
+constexpr int kCsLd = kReconN + 4;  // padded C-tile row (floats)
+
 template <typename T>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kReconThreads, 2)
     lr_recon_kernel(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
                     const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
                     const ReconArgs R) {
@@ -812,39 +767,81 @@ __global__ void __launch_bounds__(128, 1)
     return;
   }
   umma::fence_after_sync();
-  const int64_t row = m0 + 32 * warp + lane;
-  const int64_t base_off = row * R.cols + n0;
-  for (int c = 0; c < kReconN; c += 16) {
-    float cv[16];
-    umma::tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, cv);
-    const int64_t off = base_off + c;
-    float h[16];
-    load16_f32(R.ahat + off, h);
-    if (R.role == CF_SENDER) {
-      float x[16], e[16];
-      load16_act(static_cast<const T *>(R.a) + off, x);
-      if (R.ef_explicit) load16_f32(R.err + off, e);
-      float en[16], hn[16];
+  // TMEM -> shared C tile (the MMAs are complete: the operand buffers are free)
+  float *cs = reinterpret_cast<float *>(sm);
+  {
+    const int q = warp & 3, hf = warp >> 2;
+    float *dst = cs + (32 * q + lane) * kCsLd + hf * 64;
 #pragma unroll
-      for (int k = 0; k < 16; k++) {
-        const float tt = __fsub_rn(x[k], h[k]);
-        const float d = R.ef_explicit ? __fadd_rn(tt, e[k]) : tt;
-        en[k] = __fsub_rn(d, cv[k]);
-        hn[k] = __fadd_rn(h[k], cv[k]);
-      }
-      store16_f32(R.err + off, en);
-      store16_f32(R.ahat + off, hn);
-    } else {
-      float hn[16];
-#pragma unroll
-      for (int k = 0; k < 16; k++) hn[k] = __fadd_rn(h[k], cv[k]);
-      store16_f32(R.ahat + off, hn);
-      store16_act(static_cast<T *>(R.recon) + off, hn);
+    for (int c = 0; c < 64; c += 16) {
+      float v[16];
+      umma::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(hf * 64 + c), v);
+      float4 *d4 = reinterpret_cast<float4 *>(dst + c);
+      d4[0] = make_float4(v[0], v[1], v[2], v[3]);
+      d4[1] = make_float4(v[4], v[5], v[6], v[7]);
+      d4[2] = make_float4(v[8], v[9], v[10], v[11]);
+      d4[3] = make_float4(v[12], v[13], v[14], v[15]);
     }
   }
   umma::fence_before_sync();
   __syncthreads();
   if (warp == 0) umma::tmem_dealloc(tmem, 128);
+  // coalesced update: warp w takes rows w, w + 8, ...; lane l columns 4l .. 4l + 3
+  constexpr int kRowsInFlight = 4;
+  for (int r0 = warp; r0 < kTileM; r0 += 8 * kRowsInFlight) {
+    float4 cv[kRowsInFlight], hv[kRowsInFlight], ev[kRowsInFlight];
+    float xv[kRowsInFlight][4];
+    int64_t off[kRowsInFlight];
+#pragma unroll
+    for (int u = 0; u < kRowsInFlight; u++) {
+      const int rr = r0 + 8 * u;
+      off[u] = (m0 + rr) * R.cols + n0 + 4 * lane;
+      cv[u] = *reinterpret_cast<const float4 *>(cs + rr * kCsLd + 4 * lane);
+      hv[u] = __ldcs(reinterpret_cast<const float4 *>(R.ahat + off[u]));
+      if (R.role == CF_SENDER) {
+        ev[u] = R.ef_explicit ? __ldcs(reinterpret_cast<const float4 *>(R.err + off[u])) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if constexpr (sizeof(T) == 2) {
+          const uint2 w = __ldcs(reinterpret_cast<const uint2 *>(static_cast<const T *>(R.a) + off[u]));
+          xv[u][0] = __uint_as_float(w.x << 16);
+          xv[u][1] = __uint_as_float(w.x & 0xffff0000u);
+          xv[u][2] = __uint_as_float(w.y << 16);
+          xv[u][3] = __uint_as_float(w.y & 0xffff0000u);
+        } else {
+          const float4 f = __ldcs(reinterpret_cast<const float4 *>(static_cast<const T *>(R.a) + off[u]));
+          xv[u][0] = f.x; xv[u][1] = f.y; xv[u][2] = f.z; xv[u][3] = f.w;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kRowsInFlight; u++) {
+      const float c[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
+      const float h[4] = {hv[u].x, hv[u].y, hv[u].z, hv[u].w};
+      float hn[4];
+#pragma unroll
+      for (int k = 0; k < 4; k++) hn[k] = __fadd_rn(h[k], c[k]);
+      __stcs(reinterpret_cast<float4 *>(R.ahat + off[u]), make_float4(hn[0], hn[1], hn[2], hn[3]));
+      if (R.role == CF_SENDER) {
+        const float e[4] = {ev[u].x, ev[u].y, ev[u].z, ev[u].w};
+        float en[4];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          const float tt = __fsub_rn(xv[u][k], h[k]);
+          const float d = R.ef_explicit ? __fadd_rn(tt, e[k]) : tt;
+          en[k] = __fsub_rn(d, c[k]);
+        }
+        __stcs(reinterpret_cast<float4 *>(R.err + off[u]), make_float4(en[0], en[1], en[2], en[3]));
+      } else if constexpr (sizeof(T) == 2) {
+        uint2 w;
+        w.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[0])) |
+              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[1])) << 16);
+        w.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[2])) |
+              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[3])) << 16);
+        __stcs(reinterpret_cast<uint2 *>(static_cast<T *>(R.recon) + off[u]), w);
+      } else {
+        __stcs(reinterpret_cast<float4 *>(static_cast<T *>(R.recon) + off[u]), make_float4(hn[0], hn[1], hn[2], hn[3]));
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------- host
@@ -879,7 +876,11 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 size_t thin_smem(int n, int stages) { return (size_t)stages * (2u * kTileM * kTileK * 2 + 2u * n * kTileK * 2) + 1024; }
 int thin_stages(int n) { return n <= 96 ? 4 : 3; }
-size_t recon_smem(int kblocks, int a_split) { return (size_t)kblocks * kTileM * kTileK * 2 * (3 + a_split) + 1024; }
+size_t recon_smem(int kblocks, int a_split) {
+  const size_t ops = (size_t)kblocks * kTileM * kTileK * 2 * (3 + a_split);
+  const size_t ctile = (size_t)kTileM * kCsLd * 4;
+  return (ops > ctile ? ops : ctile) + 1024;
+}
 size_t apply_smem(int n) { return (size_t)n * n * 8 + (size_t)32 * n * 4; }
 size_t chol_smem(int n) { return (size_t)n * (n + 1) * 8; }
 
@@ -1096,9 +1097,9 @@ cudaError_t dequant_and_recon(const LowrankPlan &P, const uint8_t *payload, bool
   const dim3 grid((unsigned)(P.rows / kTileM), (unsigned)(P.cols / kReconN));
   const size_t smem = recon_smem(R.kblocks, R.a_split);
   if (P.dtype == CF_BF16)
-    lr_recon_kernel<__nv_bfloat16><<<grid, 128, smem, st>>>(P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
+    lr_recon_kernel<__nv_bfloat16><<<grid, kReconThreads, smem, st>>>(P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
   else
-    lr_recon_kernel<float><<<grid, 128, smem, st>>>(P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
+    lr_recon_kernel<float><<<grid, kReconThreads, smem, st>>>(P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
   return cudaGetLastError();
 }
 
