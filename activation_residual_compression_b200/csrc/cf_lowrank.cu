@@ -301,44 +301,85 @@ __global__ void __launch_bounds__(128, 1)
 
 // ---------------------------------------------------------------- CholeskyQR2 pieces
 
-// Rows per partial Gram block.
-constexpr int kGramRows = 64;
+// Rows per partial Gram block (rows are a multiple of 128).
+constexpr int kGramRows = 32;
+
+// Shared-memory column index of the Gram tile: the 16 column groups of TT
+// are laid out with an odd stride (TT | 1), so that the 16 groups a warp reads
+// at once fall in distinct banks.
+template <int TT>
+__device__ __forceinline__ int gram_col(int c) {
+  return (c / TT) * (TT | 1) + c % TT;
+}
 
 // X = sum of the nsrc partial slabs (fixed order), stored fp32 [rows][n], and
 // the partial Gram matrix X^T X (fp64) of this block's kGramRows rows: a 16 x
 // 16 thread grid, thread (ty, tx) accumulating the TT x TT sub-block rows
-// ty*TT.., cols tx*TT.. (n = 16 TT) in registers.
+// ty*TT.., cols tx*TT.. (n = 16 TT) in registers.  The products of two fp32
+// values are exact in fp64, so each fused multiply-add rounds once, as a
+// multiply followed by an add would.
 template <int TT>
 __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc, int64_t rows, float *x,
                                                       double *gpart) {
   constexpr int n = 16 * TT;
-  __shared__ float tile[kGramRows][n + 1];
+  constexpr int n4 = n / 4;                          // float4 per row
+  constexpr int NV = (kGramRows * n4 + 255) / 256;   // float4 per thread
+  __shared__ float tile[kGramRows][16 * (TT | 1)];
   const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
-  for (int idx = threadIdx.x; idx < kGramRows * n; idx += blockDim.x) {
-    const int64_t off = r0 * n + idx;
-    float acc = src[off];
-    for (int p = 1; p < nsrc; p++) acc = __fadd_rn(acc, src[(int64_t)p * rows * n + off]);
-    tile[idx / n][idx % n] = acc;
-    x[off] = acc;
+  const float4 *s4 = reinterpret_cast<const float4 *>(src) + r0 * n4;
+  const int64_t slab4 = rows * n4;
+  float4 acc4[NV];
+#pragma unroll
+  for (int v = 0; v < NV; v++) {
+    const int e = threadIdx.x + 256 * v;
+    acc4[v] = e < kGramRows * n4 ? s4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int p = 1; p < nsrc; p++) {
+#pragma unroll
+    for (int v = 0; v < NV; v++) {
+      const int e = threadIdx.x + 256 * v;
+      if (e < kGramRows * n4) {
+        const float4 t = s4[(int64_t)p * slab4 + e];
+        acc4[v].x = __fadd_rn(acc4[v].x, t.x);
+        acc4[v].y = __fadd_rn(acc4[v].y, t.y);
+        acc4[v].z = __fadd_rn(acc4[v].z, t.z);
+        acc4[v].w = __fadd_rn(acc4[v].w, t.w);
+      }
+    }
+  }
+  float4 *x4 = reinterpret_cast<float4 *>(x) + r0 * n4;
+#pragma unroll
+  for (int v = 0; v < NV; v++) {
+    const int e = threadIdx.x + 256 * v;
+    if (e < kGramRows * n4) {
+      x4[e] = acc4[v];
+      const int rr = e / n4, c = (e % n4) * 4;
+      tile[rr][gram_col<TT>(c)] = acc4[v].x;
+      tile[rr][gram_col<TT>(c + 1)] = acc4[v].y;
+      tile[rr][gram_col<TT>(c + 2)] = acc4[v].z;
+      tile[rr][gram_col<TT>(c + 3)] = acc4[v].w;
+    }
   }
   __syncthreads();
   const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  constexpr int S = TT | 1;
   double acc[TT][TT];
 #pragma unroll
   for (int a = 0; a < TT; a++)
 #pragma unroll
     for (int c = 0; c < TT; c++) acc[a][c] = 0.0;
+#pragma unroll 4
   for (int rr = 0; rr < kGramRows; rr++) {
     double xi[TT], xj[TT];
 #pragma unroll
     for (int a = 0; a < TT; a++) {
-      xi[a] = (double)tile[rr][ty * TT + a];
-      xj[a] = (double)tile[rr][tx * TT + a];
+      xi[a] = (double)tile[rr][ty * S + a];
+      xj[a] = (double)tile[rr][tx * S + a];
     }
 #pragma unroll
     for (int a = 0; a < TT; a++)
 #pragma unroll
-      for (int c = 0; c < TT; c++) acc[a][c] += xi[a] * xj[c];
+      for (int c = 0; c < TT; c++) acc[a][c] = fma(xi[a], xj[c], acc[a][c]);
   }
   double *g = gpart + (int64_t)blockIdx.x * n * n;
 #pragma unroll
@@ -347,155 +388,224 @@ __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc
     for (int c = 0; c < TT; c++) g[(ty * TT + a) * n + tx * TT + c] = acc[a][c];
 }
 
-// G = sum over blocks of the partial Gram matrices, in block order.
-__global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart, int nblk, int nn, double *G) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= nn) return;
+// G = sum over the nblk partial Gram matrices, lower triangle only (the
+// Cholesky kernel reads nothing above the diagonal; those entries are set to
+// zero).  A block covers 32 consecutive entries, one per lane; its 8 warps sum
+// 8 contiguous slices of the partials, and the slice sums are added in slice
+// order, so the result does not depend on scheduling.
+__global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart, int nblk, int n, double *G) {
+  __shared__ double part[8][32];
+  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+  const int nn = n * n;
+  const int e = blockIdx.x * 32 + lane;
+  const bool live = e < nn && (e % n) <= (e / n);
+  const int per = (nblk + 7) / 8;
+  const int b0 = wp * per, b1 = min(nblk, b0 + per);
   double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-  int b = 0;
-  for (; b + 3 < nblk; b += 4) {
-    a0 += gpart[(int64_t)b * nn + e];
-    a1 += gpart[(int64_t)(b + 1) * nn + e];
-    a2 += gpart[(int64_t)(b + 2) * nn + e];
-    a3 += gpart[(int64_t)(b + 3) * nn + e];
+  if (live) {
+    int b = b0;
+    for (; b + 3 < b1; b += 4) {
+      a0 += gpart[(int64_t)b * nn + e];
+      a1 += gpart[(int64_t)(b + 1) * nn + e];
+      a2 += gpart[(int64_t)(b + 2) * nn + e];
+      a3 += gpart[(int64_t)(b + 3) * nn + e];
+    }
+    for (; b < b1; b++) a0 += gpart[(int64_t)b * nn + e];
   }
-  for (; b < nblk; b++) a0 += gpart[(int64_t)b * nn + e];
-  G[e] = (a0 + a1) + (a2 + a3);
+  part[wp][lane] = (a0 + a1) + (a2 + a3);
+  __syncthreads();
+  if (wp == 0 && e < nn) {
+    double t = part[0][lane];
+#pragma unroll
+    for (int w = 1; w < 8; w++) t += part[w][lane];
+    G[e] = live ? t : 0.0;
+  }
 }
 
-// Cholesky factor L of the Gram matrix G (left-looking, fp64) and M = L^-T,
-// in one n x (n+1) shared array: the lower triangle holds G and becomes L;
-// thread c then writes column c of L^-1 into row c of the upper triangle
-// (its diagonal 1/L[c][c] kept apart).  One barrier per column k: thread i
-// >= k forms s_i = G[i][k] - L[i][:k].L[k][:k] and publishes it; after the
-// barrier every thread knows 1/L[k][k] = rsqrt(s_k) and the next row's new
-// entry L[k+1][k] = s_{k+1} / L[k][k] without waiting for it to be stored.
-// A pivot <= 1e-12 G_00 (R_kk <= 1e-6 R_00) marks column k rank deficient:
-// dead[k] = 1, L[k][k] = 1, L[i][k] = 0 below it, and column k of M is zero
-// so that Q's column k is zero.  Writes M fp64 [n][n] (upper triangular).
-__global__ void __launch_bounds__(128) lr_chol_kernel(const double *G, int nblk, int n, double *Mout, int *dead) {
-  extern __shared__ __align__(16) uint8_t csm[];
-  const int ld = n + 1;                          // padded row stride (bank spread)
-  double *A = reinterpret_cast<double *>(csm);   // [n][ld]
-  __shared__ double sv[2][128];                  // s_i of column k, double-buffered by k's parity
-  __shared__ double rd[128];                     // 1 / L[k][k]
-  __shared__ int dead_s[128];
-  (void)nblk;
-  const int i = threadIdx.x;
-  for (int e = threadIdx.x; e < n * n; e += blockDim.x) A[(e / n) * ld + e % n] = G[e];
-  __syncthreads();
-  const double thr = 1e-12 * A[0];
-  double lk_prev = 0.0;  // L[k][k-1] of the row k about to be processed (computed locally)
-  for (int k = 0; k < n; k++) {
-    if (i >= k && i < n) {
-      double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-      int j = 0;
-      const int kk = k - 1;  // columns < k-1 are in shared memory; column k-1 of row k is lk_prev
-      for (; j + 3 < kk; j += 4) {
-        s0 += A[i * ld + j] * A[k * ld + j];
-        s1 += A[i * ld + j + 1] * A[k * ld + j + 1];
-        s2 += A[i * ld + j + 2] * A[k * ld + j + 2];
-        s3 += A[i * ld + j + 3] * A[k * ld + j + 3];
-      }
-      for (; j < kk; j++) s0 += A[i * ld + j] * A[k * ld + j];
-      if (k > 0) s0 += A[i * ld + k - 1] * lk_prev;
-      sv[k & 1][i] = A[i * ld + k] - ((s0 + s1) + (s2 + s3));
-    }
-    // the only barrier of the step: after it, s of column k is known to all;
-    // the next step writes the other half of sv, and a thread can run ahead
-    // into it only after every thread has passed this barrier
-    __syncthreads();
-    const double piv = sv[k & 1][k];
-    const bool dk = !(piv > thr);
-    const double r = dk ? 1.0 : rsqrt(piv);
-    if (i == k) {
-      dead_s[k] = dk ? 1 : 0;
-      rd[k] = r;
-      A[k * ld + k] = dk ? 1.0 : piv * r;
-    } else if (i > k && i < n) {
-      A[i * ld + k] = dk ? 0.0 : sv[k & 1][i] * r;
-    }
-    lk_prev = (k + 1 < n) ? (dk ? 0.0 : sv[k & 1][k + 1] * r) : 0.0;
+// Cholesky factor L of the Gram matrix G (fp64) and M = L^-T, by right-
+// looking elimination with the n x n working array W held in registers: a
+// 16 x 16 thread grid, thread (ty, tx) owning the TT x TT block rows
+// ty*TT.., columns tx*TT.. (n = 16 TT).  W starts as the lower triangle of
+// G.  At step k, with d the pivot and c_i = W[i][k] (i > k) the column below
+// it, every row i > k takes W[i][j] -= (c_i / d) v_j for all j, where v is
+// row k of W left of the diagonal (j < k), the column c right of it (j > k)
+// and 0 at j = k.  In the trailing part (j > k) this is the Cholesky update;
+// left of it, W carries L^-1 by forward elimination of the identity, each of
+// its columns j stored scaled by -d_j (L^-1[i][j] = -W[i][j] / (d_j sqrt(d_i))
+// once row i is final), which makes the update uniform over j.  The owners of
+// column k+1 and of row k+1 publish v for the next step into a double-
+// buffered shared vector, so each step costs one barrier and TT^2 fused
+// multiply-adds per thread.  A pivot <= 1e-12 G_00 (R_kk <= 1e-6 R_00) marks
+// column k rank deficient: dead[k] = 1, the step's multiplier is zero (L's
+// column k below the diagonal is zero) and column k of M is zero, so that
+// Q's column k is zero.  Writes M fp64 [n][n] (upper triangular); G and M
+// may alias (G is read into registers before the first barrier).
+template <int TT>
+__global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double *Mout, int *dead) {
+  constexpr int n = 16 * TT;
+  constexpr int S = TT | 1;  // odd block stride of the shared vector: no bank conflicts
+  __shared__ double u[2][16 * S];
+  __shared__ double piv[2];
+  __shared__ double rd[n];   // 1 / sqrt(d_k), 0 for a dead column
+  __shared__ int dead_s[n];
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  const int i0 = ty * TT, j0 = tx * TT;
+  double w[TT][TT];
+#pragma unroll
+  for (int a = 0; a < TT; a++)
+#pragma unroll
+    for (int c = 0; c < TT; c++) w[a][c] = (j0 + c <= i0 + a) ? G[(i0 + a) * n + j0 + c] : 0.0;
+  if (tx == 0) {
+#pragma unroll
+    for (int a = 0; a < TT; a++) u[0][ty * S + a] = (i0 + a == 0) ? 0.0 : w[a][0];
   }
+  if (threadIdx.x == 0) piv[0] = w[0][0];
+  const double thr = 1e-12 * G[0];
+  const bool lower = tx <= ty;  // blocks above the diagonal hold nothing
   __syncthreads();
-  // column c of L^-1 (thread c), forward substitution L x = e_c: x[r] for
-  // r > c goes to A[c][r], x[c] = 1/L[c][c] to rd[c]
-  if (i < n) {
-    for (int r = i + 1; r < n; r++) {
-      double s0 = A[r * ld + i] * rd[i], s1 = 0.0, s2 = 0.0, s3 = 0.0;
-      int j = i + 1;
-      for (; j + 3 < r; j += 4) {
-        s0 += A[r * ld + j] * A[i * ld + j];
-        s1 += A[r * ld + j + 1] * A[i * ld + j + 1];
-        s2 += A[r * ld + j + 2] * A[i * ld + j + 2];
-        s3 += A[r * ld + j + 3] * A[i * ld + j + 3];
+  for (int kb = 0; kb < 16; kb++) {
+#pragma unroll
+    for (int kr = 0; kr < TT; kr++) {  // unrolled: the next column's register index is static
+      const int k = kb * TT + kr;
+      const double *uk = u[k & 1];
+      const double d = piv[k & 1];
+      const bool dk = !(d > thr);
+      const double r = dk ? 0.0 : rsqrt(d);
+      const double invd = r * r;
+      if (threadIdx.x == 0) {
+        rd[k] = r;
+        dead_s[k] = dk ? 1 : 0;
       }
-      for (; j < r; j++) s0 += A[r * ld + j] * A[i * ld + j];
-      A[i * ld + r] = -((s0 + s1) + (s2 + s3)) * rd[r];
+      if (lower && i0 + TT - 1 > k) {
+        double vj[TT];
+#pragma unroll
+        for (int c = 0; c < TT; c++) vj[c] = uk[tx * S + c];
+#pragma unroll
+        for (int a = 0; a < TT; a++) {
+          // rows <= k are final; a zero multiplier leaves them as they are
+          const double sa = (i0 + a > k) ? -(uk[ty * S + a] * invd) : 0.0;
+#pragma unroll
+          for (int c = 0; c < TT; c++) w[a][c] = fma(sa, vj[c], w[a][c]);
+        }
+      }
+      const int k1 = k + 1;
+      const int cn = (kr + 1 == TT) ? 0 : kr + 1;
+      const int b1 = (kr + 1 == TT) ? kb + 1 : kb;
+      if (k1 < n) {
+        double *un = u[k1 & 1];
+        if (tx == b1) {  // column k1 below the diagonal; its diagonal is the next pivot
+#pragma unroll
+          for (int a = 0; a < TT; a++) {
+            const double x = w[a][cn];
+            if (i0 + a > k1) un[ty * S + a] = x;
+            if (i0 + a == k1) {
+              un[ty * S + a] = 0.0;
+              piv[k1 & 1] = x;
+            }
+          }
+        }
+        if (ty == b1) {  // row k1 left of the diagonal
+#pragma unroll
+          for (int c = 0; c < TT; c++)
+            if (j0 + c < k1) un[tx * S + c] = w[cn][c];
+        }
+      }
+      __syncthreads();
     }
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
-    const int rr = e / n, c = e % n;  // M[rr][c] = Linv[c][rr]; column c of M zero when c is dead
-    double m = 0.0;
-    if (!dead_s[c]) m = c == rr ? rd[rr] : (c > rr ? A[rr * ld + c] : 0.0);
-    Mout[e] = m;
+#pragma unroll
+  for (int a = 0; a < TT; a++) {
+    const int gi = i0 + a;
+    const bool dki = dead_s[gi] != 0;
+    const double ri = rd[gi];
+#pragma unroll
+    for (int c = 0; c < TT; c++) {
+      const int gj = j0 + c;
+      const double rj = rd[gj];
+      double m = 0.0;  // M[gj][gi] = L^-1[gi][gj]
+      if (gj <= gi && !dki) m = gj == gi ? ri : (-w[a][c] * (rj * rj)) * ri;
+      Mout[gj * n + gi] = m;
+    }
   }
   for (int e = threadIdx.x; e < n; e += blockDim.x) dead[e] = dead_s[e];
 }
 
-// Q = X M (M = L^-T, upper triangular) for 32 rows per block: thread
-// (row, group) computes 10..16 consecutive outputs of its row with
-// independent fp64 accumulators.  Writes Q fp32 [rows][n] and, when
-// qthi != nullptr, Q^T split in bf16 ([n][rows], the K-major B operand of
-// V = D^T Q).
-__global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const double *M, int64_t rows, int n, float *q,
+// Rows per apply block.
+constexpr int kApplyRows = 32;
+template <int TT>
+__host__ __device__ constexpr int apply_xld() {
+  return 16 * TT + 4;  // padded row stride of the X tile (bank spread, 16-byte rows)
+}
+
+// Q = X M (M = L^-T, upper triangular, zero below the diagonal) for 32 rows
+// per block.  M and the block's rows of X are staged in shared memory;
+// thread (row, group) computes the 2 TT outputs c = 16 t + 2 group + {0, 1}
+// of its row (conflict-free paired loads of M) with fp64 accumulators over
+// all n terms in ascending order (the zeros below M's diagonal add nothing).
+// Writes Q fp32 [rows][n] and, when qthi != nullptr, Q^T split in bf16
+// ([n][rows], the K-major B operand of V = D^T Q), transposed through shared
+// memory so that those stores are row-contiguous.
+template <int TT>
+__global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const double *M, int64_t rows, float *q,
                                                        __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo) {
+  constexpr int n = 16 * TT, xld = apply_xld<TT>(), qld = kApplyRows + 1;
   extern __shared__ __align__(16) uint8_t asm_[];
-  double *Ms = reinterpret_cast<double *>(asm_);  // [n][n]
-  float *xs = reinterpret_cast<float *>(Ms + n * n);  // [32][n]
-  const int64_t r0 = (int64_t)blockIdx.x * 32;
-  for (int e = threadIdx.x; e < n * n; e += blockDim.x) Ms[e] = M[e];
-  for (int e = threadIdx.x; e < 32 * n; e += blockDim.x) {
-    const int64_t rr = r0 + e / n;
-    xs[e] = rr < rows ? x[rr * n + e % n] : 0.0f;
+  double *Ms = reinterpret_cast<double *>(asm_);      // [n][n]
+  float *xs = reinterpret_cast<float *>(Ms + n * n);  // [32][xld]; reused as Q^T [n][qld]
+  const int64_t r0 = (int64_t)blockIdx.x * kApplyRows;
+  {
+    const double2 *M2 = reinterpret_cast<const double2 *>(M);
+    double2 *Ms2 = reinterpret_cast<double2 *>(Ms);
+#pragma unroll 4
+    for (int e = threadIdx.x; e < n * n / 2; e += 256) Ms2[e] = M2[e];
+    const float4 *x4 = reinterpret_cast<const float4 *>(x) + r0 * (n / 4);
+    for (int e = threadIdx.x; e < kApplyRows * n / 4; e += 256) {
+      const int rr = e / (n / 4), c = (e % (n / 4)) * 4;
+      const float4 v = r0 + rr < rows ? x4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4 *>(xs + rr * xld + c) = v;
+    }
   }
   __syncthreads();
   const int lr = threadIdx.x >> 3, grp = threadIdx.x & 7;
-  const int per = (n + 7) / 8;  // outputs per thread (<= 16)
-  const int c0 = grp * per;
+  double acc[2 * TT];
+#pragma unroll
+  for (int t = 0; t < 2 * TT; t++) acc[t] = 0.0;
+#pragma unroll 2
+  for (int j = 0; j < n; j++) {
+    const double xj = (double)xs[lr * xld + j];
+    const double2 *mr = reinterpret_cast<const double2 *>(Ms + j * n + 2 * grp);
+#pragma unroll
+    for (int t = 0; t < TT; t++) {
+      const double2 m = mr[8 * t];  // columns 16 t + 2 grp, +1
+      acc[2 * t] = fma(xj, m.x, acc[2 * t]);
+      acc[2 * t + 1] = fma(xj, m.y, acc[2 * t + 1]);
+    }
+  }
   const int64_t row = r0 + lr;
-  double acc[16];
+  if (row < rows) {
 #pragma unroll
-  for (int t = 0; t < 16; t++) acc[t] = 0.0;
-  // M is upper triangular: rows j < c0 touch every output of the group
-  for (int j = 0; j < c0; j++) {
-    const double xj = (double)xs[lr * n + j];
-    const double *mr = Ms + j * n + c0;
-#pragma unroll
-    for (int t = 0; t < 16; t++)
-      if (t < per) acc[t] += xj * mr[t];
+    for (int t = 0; t < TT; t++) {
+      const int c = 16 * t + 2 * grp;
+      *reinterpret_cast<float2 *>(q + row * n + c) = make_float2((float)acc[2 * t], (float)acc[2 * t + 1]);
+    }
   }
-  for (int j = c0; j < c0 + per && j < n; j++) {
-    const double xj = (double)xs[lr * n + j];
-    const double *mr = Ms + j * n + c0;
+  if (qthi == nullptr) return;  // uniform over the block
+  __syncthreads();              // every thread is done with xs
+  float *qs = xs;               // Q^T tile [n][qld]
 #pragma unroll
-    for (int t = 0; t < 16; t++)
-      if (t < per && c0 + t >= j && c0 + t < n) acc[t] += xj * mr[t];
+  for (int t = 0; t < TT; t++) {
+    const int c = 16 * t + 2 * grp;
+    qs[c * qld + lr] = (float)acc[2 * t];
+    qs[(c + 1) * qld + lr] = (float)acc[2 * t + 1];
   }
-  if (row >= rows) return;
-#pragma unroll
-  for (int t = 0; t < 16; t++) {
-    const int c = c0 + t;
-    if (t < per && c < n) {
-      const float qf = (float)acc[t];
-      q[row * n + c] = qf;
-      if (qthi) {
-        __nv_bfloat16 hi, lo;
-        split_bf16(qf, hi, lo);
-        qthi[(int64_t)c * rows + row] = hi;
-        qtlo[(int64_t)c * rows + row] = lo;
-      }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n * kApplyRows; e += 256) {
+    const int c = e / kApplyRows, rr = e % kApplyRows;
+    if (r0 + rr < rows) {
+      __nv_bfloat16 hi, lo;
+      split_bf16(qs[c * qld + rr], hi, lo);
+      qthi[(int64_t)c * rows + r0 + rr] = hi;
+      qtlo[(int64_t)c * rows + r0 + rr] = lo;
     }
   }
 }
@@ -881,8 +991,10 @@ size_t recon_smem(int kblocks, int a_split) {
   const size_t ctile = (size_t)kTileM * kCsLd * 4;
   return (ops > ctile ? ops : ctile) + 1024;
 }
-size_t apply_smem(int n) { return (size_t)n * n * 8 + (size_t)32 * n * 4; }
-size_t chol_smem(int n) { return (size_t)n * (n + 1) * 8; }
+size_t apply_smem(int n) {
+  const size_t xt = (size_t)kApplyRows * (n + 4) * 4, qt = (size_t)n * (kApplyRows + 1) * 4;
+  return (size_t)n * n * 8 + (xt > qt ? xt : qt);
+}
 
 }  // namespace
 
@@ -927,6 +1039,30 @@ void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *p
   plan->enc_scratch_bytes = enc;
   plan->dec_scratch_bytes = dec;
 }
+
+namespace {
+
+template <int TT>
+cudaError_t set_apply_smem_tt() {
+  return cudaFuncSetAttribute(lr_apply_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)apply_smem(16 * TT));
+}
+
+cudaError_t set_apply_smem(int n) {
+  switch (n / 16) {
+    case 1: return set_apply_smem_tt<1>();
+    case 2: return set_apply_smem_tt<2>();
+    case 3: return set_apply_smem_tt<3>();
+    case 4: return set_apply_smem_tt<4>();
+    case 5: return set_apply_smem_tt<5>();
+    case 6: return set_apply_smem_tt<6>();
+    case 7: return set_apply_smem_tt<7>();
+    case 8: return set_apply_smem_tt<8>();
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
 
 int lowrank_bind(LowrankPlan *plan, void *scratch) {
   uint8_t *p = static_cast<uint8_t *>(scratch);
@@ -975,10 +1111,7 @@ int lowrank_bind(LowrankPlan *plan, void *scratch) {
                            (int)recon_smem(plan->kp / kTileK, 1)) != cudaSuccess ||
       cudaFuncSetAttribute(lr_recon_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)recon_smem(plan->kp / kTileK, 1)) != cudaSuccess ||
-      cudaFuncSetAttribute(lr_chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)chol_smem(rpi)) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(lr_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)apply_smem(rpi)) !=
-          cudaSuccess) {
+      set_apply_smem(rpi) != cudaSuccess) {
     (void)cudaGetLastError();
     return CF_ERR_CUDA;
   }
@@ -1019,6 +1152,39 @@ cudaError_t launch_gram(int n, int nblk, const float *src, int nsrc, int64_t row
   return cudaGetLastError();
 }
 
+cudaError_t launch_chol(int n, double *L, int *dead, cudaStream_t st) {
+  switch (n / 16) {
+    case 1: lr_chol_kernel<1><<<1, 256, 0, st>>>(L, L, dead); break;
+    case 2: lr_chol_kernel<2><<<1, 256, 0, st>>>(L, L, dead); break;
+    case 3: lr_chol_kernel<3><<<1, 256, 0, st>>>(L, L, dead); break;
+    case 4: lr_chol_kernel<4><<<1, 256, 0, st>>>(L, L, dead); break;
+    case 5: lr_chol_kernel<5><<<1, 256, 0, st>>>(L, L, dead); break;
+    case 6: lr_chol_kernel<6><<<1, 256, 0, st>>>(L, L, dead); break;
+    case 7: lr_chol_kernel<7><<<1, 256, 0, st>>>(L, L, dead); break;
+    case 8: lr_chol_kernel<8><<<1, 256, 0, st>>>(L, L, dead); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_apply(int n, const float *x, const double *M, int64_t rows, float *q, __nv_bfloat16 *qthi,
+                         __nv_bfloat16 *qtlo, cudaStream_t st) {
+  const unsigned grid = (unsigned)((rows + kApplyRows - 1) / kApplyRows);
+  const size_t sm = apply_smem(n);
+  switch (n / 16) {
+    case 1: lr_apply_kernel<1><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
+    case 2: lr_apply_kernel<2><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
+    case 3: lr_apply_kernel<3><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
+    case 4: lr_apply_kernel<4><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
+    case 5: lr_apply_kernel<5><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
+    case 6: lr_apply_kernel<6><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
+    case 7: lr_apply_kernel<7><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
+    case 8: lr_apply_kernel<8><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int64_t rows, bool final_pass,
                            cudaStream_t st) {
   const LowrankBufs &b = P.b;
@@ -1026,13 +1192,12 @@ cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int
   const int nblk = (int)(rows / kGramRows);
   cudaError_t e = launch_gram(n, nblk, src, nsrc, rows, b.xbuf, b.gpart, st);
   if (e != cudaSuccess) return e;
-  // the reduced Gram matrix goes to the head of the partial buffer's last
-  // slot region (L, which the Cholesky kernel then overwrites with M)
-  lr_gram_reduce_kernel<<<(n * n + 255) / 256, 256, 0, st>>>(b.gpart, nblk, n * n, b.L);
-  lr_chol_kernel<<<1, 128, chol_smem(n), st>>>(b.L, 1, n, b.L, b.dead);
-  lr_apply_kernel<<<(unsigned)((rows + 31) / 32), 256, apply_smem(n), st>>>(
-      b.xbuf, b.L, rows, n, b.q, final_pass ? b.qthi : nullptr, final_pass ? b.qtlo : nullptr);
-  return cudaGetLastError();
+  // the reduced Gram matrix goes to L, which the Cholesky kernel then
+  // overwrites with M = L^-T
+  lr_gram_reduce_kernel<<<(unsigned)((n * n + 31) / 32), 256, 0, st>>>(b.gpart, nblk, n, b.L);
+  e = launch_chol(n, b.L, b.dead, st);
+  if (e != cudaSuccess) return e;
+  return launch_apply(n, b.xbuf, b.L, rows, b.q, final_pass ? b.qthi : nullptr, final_pass ? b.qtlo : nullptr, st);
 }
 
 PackArgs pack_args(const LowrankPlan &P, uint8_t *payload, const Header &hdr) {
