@@ -28,6 +28,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <utility>
 #include <mutex>
 
 #include "cf_lowrank.h"
@@ -84,10 +85,39 @@ __device__ __forceinline__ float v0_entry(uint64_t seed, int64_t j, int r, int k
 
 // ---------------------------------------------------------------- V preparation
 
+// Programmatic dependent launch.  Every kernel of the encode and decode
+// chains starts here: it waits until the kernel before it in the stream has
+// completed and its writes are visible, then lets the kernel after it be
+// scheduled, so that launch latency overlaps the tail of the running grid.
+// Without the launch attribute both instructions return at once.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch with the programmatic-stream-serialisation attribute (the kernel
+// must begin with pdl_enter()).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Vt (split bf16, [rp][cols]) from the warm start: the previous step's V
 // (fp32 [cols][r]), or V0 on the first step and for any all-zero column.
 __global__ void __launch_bounds__(256) lr_vprep_kernel(const float *vprev, int64_t cols, int r, int rp, int first,
                                                        uint64_t seed, __nv_bfloat16 *vthi, __nv_bfloat16 *vtlo) {
+  pdl_enter();
   const int k = blockIdx.x;
   __shared__ int nonzero;
   if (threadIdx.x == 0) nonzero = 0;
@@ -120,6 +150,7 @@ __global__ void __launch_bounds__(256) lr_delta_kernel(const T *a, const float *
                                                        int64_t rows, int64_t cols, __nv_bfloat16 *dhi,
                                                        __nv_bfloat16 *dlo, __nv_bfloat16 *dthi,
                                                        __nv_bfloat16 *dtlo) {
+  pdl_enter();
   __shared__ __nv_bfloat16 shi[64][72];
   __shared__ __nv_bfloat16 slo[64][72];
   const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
@@ -200,6 +231,7 @@ __global__ void __launch_bounds__(128, 1)
     lr_thin_gemm_kernel(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
                         const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
                         const ThinArgs A) {
+  pdl_enter();
   extern __shared__ __align__(1024) uint8_t dsm[];
   __shared__ __align__(8) uint64_t full[4], empty[4], accb;
   __shared__ uint32_t tmem_base;
@@ -321,6 +353,7 @@ __device__ __forceinline__ int gram_col(int c) {
 template <int TT>
 __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc, int64_t rows, float *x,
                                                       double *gpart) {
+  pdl_enter();
   constexpr int n = 16 * TT;
   constexpr int n4 = n / 4;                          // float4 per row
   constexpr int NV = (kGramRows * n4 + 255) / 256;   // float4 per thread
@@ -394,6 +427,7 @@ __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc
 // 8 contiguous slices of the partials, and the slice sums are added in slice
 // order, so the result does not depend on scheduling.
 __global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart, int nblk, int n, double *G) {
+  pdl_enter();
   __shared__ double part[8][32];
   const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
   const int nn = n * n;
@@ -442,6 +476,7 @@ __global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart
 // may alias (G is read into registers before the first barrier).
 template <int TT>
 __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double *Mout, int *dead) {
+  pdl_enter();
   constexpr int n = 16 * TT;
   constexpr int S = TT | 1;  // odd block stride of the shared vector: no bank conflicts
   __shared__ double u[2][16 * S];
@@ -548,6 +583,7 @@ __host__ __device__ constexpr int apply_xld() {
 template <int TT>
 __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const double *M, int64_t rows, float *q,
                                                        __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo) {
+  pdl_enter();
   constexpr int n = 16 * TT, xld = apply_xld<TT>(), qld = kApplyRows + 1;
   extern __shared__ __align__(16) uint8_t asm_[];
   double *Ms = reinterpret_cast<double *>(asm_);      // [n][n]
@@ -616,6 +652,7 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
 __global__ void __launch_bounds__(256) lr_vsum_kernel(const float *vpart, int nsrc, int64_t cols, int n, int r,
                                                       float *v, float *vprev, __nv_bfloat16 *vthi,
                                                       __nv_bfloat16 *vtlo) {
+  pdl_enter();
   const int64_t total = cols * n;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
     float acc = vpart[idx];
@@ -648,6 +685,7 @@ struct PackArgs {
 // Per-column scales s_k = fp32(absmax_k / 7) of U (blocks 0..r-1) and V
 // (blocks r..2r-1), into the payload's scale section.
 __global__ void __launch_bounds__(256) lr_scale_kernel(PackArgs P) {
+  pdl_enter();
   const int k = blockIdx.x % P.r;
   const bool isv = blockIdx.x >= P.r;
   const float *m = isv ? P.v : P.q;
@@ -677,6 +715,7 @@ __device__ __forceinline__ uint32_t int4_code(float x, float s) {
 // Nibbles of U and V (element (i,k) is nibble i*r + k, low nibble first) or
 // the fp32 factors, padding bytes zero, and the header.
 __global__ void __launch_bounds__(256) lr_pack_kernel(PackArgs P) {
+  pdl_enter();
   uint8_t *body = P.payload + kHdrBytes;
   if (blockIdx.x == 0 && threadIdx.x < 16) reinterpret_cast<uint32_t *>(P.payload)[threadIdx.x] = P.hdr.w[threadIdx.x];
   const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
@@ -735,6 +774,7 @@ struct DequantArgs {
 };
 
 __global__ void __launch_bounds__(256) lr_dequant_kernel(DequantArgs D) {
+  pdl_enter();
   if (D.check_header && !lr_header_ok(D.payload, D.expect, D.status)) return;
   const uint8_t *body = D.payload + kHdrBytes;
   const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
@@ -803,6 +843,7 @@ __global__ void __launch_bounds__(kReconThreads, 2)
     lr_recon_kernel(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
                     const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
                     const ReconArgs R) {
+  pdl_enter();
   extern __shared__ __align__(1024) uint8_t dsm[];
   __shared__ __align__(8) uint64_t full, accb;
   __shared__ uint32_t tmem_base;
@@ -1131,7 +1172,7 @@ cudaError_t launch_thin(const LowrankPlan &P, const CUtensorMap &ah, const CUten
   A.splits = splits;
   A.stages = thin_stages(P.rp);
   A.status = status;
-  lr_thin_gemm_kernel<<<dim3((unsigned)(M / kTileM), (unsigned)splits), 128, thin_smem(P.rp, A.stages), st>>>(
+  launch_pdl(lr_thin_gemm_kernel, dim3(dim3((unsigned)(M / kTileM), (unsigned)splits)), dim3(128), thin_smem(P.rp, A.stages), st, 
       ah, al, bh, bl, A);
   return cudaGetLastError();
 }
@@ -1139,14 +1180,14 @@ cudaError_t launch_thin(const LowrankPlan &P, const CUtensorMap &ah, const CUten
 cudaError_t launch_gram(int n, int nblk, const float *src, int nsrc, int64_t rows, float *x, double *gpart,
                         cudaStream_t st) {
   switch (n / 16) {
-    case 1: lr_gram_kernel<1><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
-    case 2: lr_gram_kernel<2><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
-    case 3: lr_gram_kernel<3><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
-    case 4: lr_gram_kernel<4><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
-    case 5: lr_gram_kernel<5><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
-    case 6: lr_gram_kernel<6><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
-    case 7: lr_gram_kernel<7><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
-    case 8: lr_gram_kernel<8><<<nblk, 256, 0, st>>>(src, nsrc, rows, x, gpart); break;
+    case 1: launch_pdl(lr_gram_kernel<1>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
+    case 2: launch_pdl(lr_gram_kernel<2>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
+    case 3: launch_pdl(lr_gram_kernel<3>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
+    case 4: launch_pdl(lr_gram_kernel<4>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
+    case 5: launch_pdl(lr_gram_kernel<5>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
+    case 6: launch_pdl(lr_gram_kernel<6>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
+    case 7: launch_pdl(lr_gram_kernel<7>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
+    case 8: launch_pdl(lr_gram_kernel<8>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -1154,14 +1195,14 @@ cudaError_t launch_gram(int n, int nblk, const float *src, int nsrc, int64_t row
 
 cudaError_t launch_chol(int n, double *L, int *dead, cudaStream_t st) {
   switch (n / 16) {
-    case 1: lr_chol_kernel<1><<<1, 256, 0, st>>>(L, L, dead); break;
-    case 2: lr_chol_kernel<2><<<1, 256, 0, st>>>(L, L, dead); break;
-    case 3: lr_chol_kernel<3><<<1, 256, 0, st>>>(L, L, dead); break;
-    case 4: lr_chol_kernel<4><<<1, 256, 0, st>>>(L, L, dead); break;
-    case 5: lr_chol_kernel<5><<<1, 256, 0, st>>>(L, L, dead); break;
-    case 6: lr_chol_kernel<6><<<1, 256, 0, st>>>(L, L, dead); break;
-    case 7: lr_chol_kernel<7><<<1, 256, 0, st>>>(L, L, dead); break;
-    case 8: lr_chol_kernel<8><<<1, 256, 0, st>>>(L, L, dead); break;
+    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), 0, st, L, L, dead); break;
+    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), 0, st, L, L, dead); break;
+    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), 0, st, L, L, dead); break;
+    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), 0, st, L, L, dead); break;
+    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), 0, st, L, L, dead); break;
+    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), 0, st, L, L, dead); break;
+    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), 0, st, L, L, dead); break;
+    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), 0, st, L, L, dead); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -1172,14 +1213,14 @@ cudaError_t launch_apply(int n, const float *x, const double *M, int64_t rows, f
   const unsigned grid = (unsigned)((rows + kApplyRows - 1) / kApplyRows);
   const size_t sm = apply_smem(n);
   switch (n / 16) {
-    case 1: lr_apply_kernel<1><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
-    case 2: lr_apply_kernel<2><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
-    case 3: lr_apply_kernel<3><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
-    case 4: lr_apply_kernel<4><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
-    case 5: lr_apply_kernel<5><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
-    case 6: lr_apply_kernel<6><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
-    case 7: lr_apply_kernel<7><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
-    case 8: lr_apply_kernel<8><<<grid, 256, sm, st>>>(x, M, rows, q, qthi, qtlo); break;
+    case 1: launch_pdl(lr_apply_kernel<1>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
+    case 2: launch_pdl(lr_apply_kernel<2>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
+    case 3: launch_pdl(lr_apply_kernel<3>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
+    case 4: launch_pdl(lr_apply_kernel<4>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
+    case 5: launch_pdl(lr_apply_kernel<5>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
+    case 6: launch_pdl(lr_apply_kernel<6>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
+    case 7: launch_pdl(lr_apply_kernel<7>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
+    case 8: launch_pdl(lr_apply_kernel<8>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -1194,7 +1235,7 @@ cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int
   if (e != cudaSuccess) return e;
   // the reduced Gram matrix goes to L, which the Cholesky kernel then
   // overwrites with M = L^-T
-  lr_gram_reduce_kernel<<<(unsigned)((n * n + 31) / 32), 256, 0, st>>>(b.gpart, nblk, n, b.L);
+  launch_pdl(lr_gram_reduce_kernel, dim3((unsigned)((n * n + 31) / 32)), dim3(256), 0, st, b.gpart, nblk, n, b.L);
   e = launch_chol(n, b.L, b.dead, st);
   if (e != cudaSuccess) return e;
   return launch_apply(n, b.xbuf, b.L, rows, b.q, final_pass ? b.qthi : nullptr, final_pass ? b.qtlo : nullptr, st);
@@ -1243,7 +1284,7 @@ cudaError_t dequant_and_recon(const LowrankPlan &P, const uint8_t *payload, bool
   D.check_header = receiver;
   D.expect = expect;
   D.status = status;
-  lr_dequant_kernel<<<1184, 256, 0, st>>>(D);
+  launch_pdl(lr_dequant_kernel, dim3(1184), dim3(256), 0, st, D);
   ReconArgs R{};
   R.rows = P.rows;
   R.cols = P.cols;
@@ -1262,9 +1303,9 @@ cudaError_t dequant_and_recon(const LowrankPlan &P, const uint8_t *payload, bool
   const dim3 grid((unsigned)(P.rows / kTileM), (unsigned)(P.cols / kReconN));
   const size_t smem = recon_smem(R.kblocks, R.a_split);
   if (P.dtype == CF_BF16)
-    lr_recon_kernel<__nv_bfloat16><<<grid, kReconThreads, smem, st>>>(P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
+    launch_pdl(lr_recon_kernel<__nv_bfloat16>, dim3(grid), dim3(kReconThreads), smem, st, P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
   else
-    lr_recon_kernel<float><<<grid, kReconThreads, smem, st>>>(P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
+    launch_pdl(lr_recon_kernel<float>, dim3(grid), dim3(kReconThreads), smem, st, P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
   return cudaGetLastError();
 }
 
@@ -1275,13 +1316,13 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
   if (tab) return cudaErrorNotSupported;  // batch 1 only
   const LowrankBufs &b = P.b;
   const int64_t R = P.rows, C = P.cols;
-  lr_vprep_kernel<<<P.rp, 256, 0, st>>>(vprev, C, P.rank, P.rp, step == 1 ? 1 : 0, seed, b.vthi, b.vtlo);
+  launch_pdl(lr_vprep_kernel, dim3(P.rp), dim3(256), 0, st, vprev, C, P.rank, P.rp, step == 1 ? 1 : 0, seed, b.vthi, b.vtlo);
   const dim3 dg((unsigned)(C / 64), (unsigned)(R / 64));
   if (P.dtype == CF_BF16)
-    lr_delta_kernel<__nv_bfloat16><<<dg, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(args.a), args.ahat, args.err,
+    launch_pdl(lr_delta_kernel<__nv_bfloat16>, dim3(dg), dim3(256), 0, st, static_cast<const __nv_bfloat16 *>(args.a), args.ahat, args.err,
                                                         P.ef_explicit, R, C, b.dhi, b.dlo, b.dthi, b.dtlo);
   else
-    lr_delta_kernel<float><<<dg, 256, 0, st>>>(static_cast<const float *>(args.a), args.ahat, args.err, P.ef_explicit,
+    launch_pdl(lr_delta_kernel<float>, dim3(dg), dim3(256), 0, st, static_cast<const float *>(args.a), args.ahat, args.err, P.ef_explicit,
                                                R, C, b.dhi, b.dlo, b.dthi, b.dtlo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1298,14 +1339,14 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
         cudaSuccess)
       return e;
     const bool more = it + 1 < P.iters;
-    lr_vsum_kernel<<<592, 256, 0, st>>>(b.vpart, P.sv, C, P.rp, P.rank, b.v, vprev, more ? b.vthi : nullptr,
+    launch_pdl(lr_vsum_kernel, dim3(592), dim3(256), 0, st, b.vpart, P.sv, C, P.rp, P.rank, b.v, vprev, more ? b.vthi : nullptr,
                                         more ? b.vtlo : nullptr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // INT4 (or fp32) factors into the payload
   const PackArgs pa = pack_args(P, args.payload, args.hdr);
-  if (P.int4) lr_scale_kernel<<<2 * P.rank, 256, 0, st>>>(pa);
-  lr_pack_kernel<<<592, 256, 0, st>>>(pa);
+  if (P.int4) launch_pdl(lr_scale_kernel, dim3(2 * P.rank), dim3(256), 0, st, pa);
+  launch_pdl(lr_pack_kernel, dim3(592), dim3(256), 0, st, pa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // sender reconstruction from the payload bytes
   return dequant_and_recon(P, args.payload, false, args.hdr, args.a, args.ahat, args.err, nullptr, args.status, st);
