@@ -115,27 +115,39 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 
 // Vt (split bf16, [rp][cols]) from the warm start: the previous step's V
 // (fp32 [cols][r]), or V0 on the first step and for any all-zero column.
-__global__ void __launch_bounds__(256) lr_vprep_kernel(const float *vprev, int64_t cols, int r, int rp, int first,
-                                                       uint64_t seed, __nv_bfloat16 *vthi, __nv_bfloat16 *vtlo) {
+constexpr int kVprepThreads = 1024;
+constexpr int kVprepPer = 8;
+static_assert(kVprepThreads * kVprepPer >= kMaxCols, "one vprep block holds a whole column");
+__global__ void __launch_bounds__(kVprepThreads) lr_vprep_kernel(const float *vprev, int64_t cols, int r, int rp,
+                                                                 int first, uint64_t seed, __nv_bfloat16 *vthi,
+                                                                 __nv_bfloat16 *vtlo, unsigned *amax) {
   pdl_enter();
   const int k = blockIdx.x;
-  __shared__ int nonzero;
-  if (threadIdx.x == 0) nonzero = 0;
-  __syncthreads();
-  if (k < r && !first) {
-    int nz = 0;
-    for (int64_t j = threadIdx.x; j < cols; j += blockDim.x) nz |= vprev[j * r + k] != 0.0f;
-    if (__syncthreads_or(nz) && threadIdx.x == 0) nonzero = 1;
+  if (threadIdx.x == 0) {  // this encode's column maxima start from zero
+    amax[k] = 0u;
+    amax[rp + k] = 0u;
   }
-  __syncthreads();
-  const bool use_prev = nonzero != 0;
-  for (int64_t j = threadIdx.x; j < cols; j += blockDim.x) {
-    float x = 0.0f;
-    if (k < r) x = use_prev ? vprev[j * r + k] : v0_entry(seed, j, r, k);
-    __nv_bfloat16 hi, lo;
-    split_bf16(x, hi, lo);
-    vthi[(int64_t)k * cols + j] = hi;
-    vtlo[(int64_t)k * cols + j] = lo;
+  float x[kVprepPer];
+  int nz = 0;
+#pragma unroll
+  for (int t = 0; t < kVprepPer; t++) {
+    const int64_t j = threadIdx.x + (int64_t)t * kVprepThreads;
+    x[t] = (k < r && !first && j < cols) ? vprev[j * r + k] : 0.0f;
+    nz |= x[t] != 0.0f;
+  }
+  // a column of V_prev that is entirely zero (a dead direction) restarts from V0
+  const bool use_prev = __syncthreads_or(nz) != 0;
+#pragma unroll
+  for (int t = 0; t < kVprepPer; t++) {
+    const int64_t j = threadIdx.x + (int64_t)t * kVprepThreads;
+    if (j < cols) {
+      float v = 0.0f;
+      if (k < r) v = use_prev ? x[t] : v0_entry(seed, j, r, k);
+      __nv_bfloat16 hi, lo;
+      split_bf16(v, hi, lo);
+      vthi[(int64_t)k * cols + j] = hi;
+      vtlo[(int64_t)k * cols + j] = lo;
+    }
   }
 }
 
@@ -657,8 +669,8 @@ __global__ void __launch_bounds__(256) lr_vsum_kernel(const float *vpart, int ns
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
     float acc = vpart[idx];
     for (int p = 1; p < nsrc; p++) acc = __fadd_rn(acc, vpart[(int64_t)p * total + idx]);
-    const int64_t j = idx / n;
-    const int k = (int)(idx % n);
+    const uint32_t j = (uint32_t)idx / (uint32_t)n;
+    const int k = (int)((uint32_t)idx - j * (uint32_t)n);
     v[idx] = acc;
     if (k < r) vprev[j * r + k] = acc;
     if (vthi) {
@@ -680,29 +692,50 @@ struct PackArgs {
   int r, n, int4;
   int64_t sec1, sec2, body;
   Header hdr;
+  unsigned *amax;  // [2 n]: column absmax bit patterns of Q, then of V (zeroed by lr_vprep_kernel)
 };
 
-// Per-column scales s_k = fp32(absmax_k / 7) of U (blocks 0..r-1) and V
-// (blocks r..2r-1), into the payload's scale section.
+// Column absmax of Q (blocks 0 .. rows/32 - 1) and of V (the rest), one
+// 32-row tile per block: thread (row lane, column group) keeps the maxima of
+// its four columns over its rows in registers (coalesced float4 loads), the
+// block combines them in shared memory, and one atomicMax per column goes to
+// P.amax.  The values are non-negative, so their bit patterns order like the
+// values and the result does not depend on the order of the updates.
+constexpr int kScaleRows = 32;
 __global__ void __launch_bounds__(256) lr_scale_kernel(PackArgs P) {
   pdl_enter();
-  const int k = blockIdx.x % P.r;
-  const bool isv = blockIdx.x >= P.r;
-  const float *m = isv ? P.v : P.q;
-  const int64_t len = isv ? P.cols : P.rows;
-  float amax = 0.0f;
-  for (int64_t i = threadIdx.x; i < len; i += blockDim.x) amax = fmaxf(amax, fabsf(m[i * P.n + k]));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  __shared__ float wm[8];
-  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = amax;
+  __shared__ unsigned cm[128];
+  const int nq = (int)(P.rows / kScaleRows);
+  const bool isv = (int)blockIdx.x >= nq;
+  const int64_t r0 = (int64_t)(isv ? blockIdx.x - nq : blockIdx.x) * kScaleRows;
+  const float4 *m4 = reinterpret_cast<const float4 *>((isv ? P.v : P.q) + r0 * P.n);
+  const int n4 = P.n / 4, lanes = (int)blockDim.x / n4;  // row lanes (n4 <= 32)
+  const int cg = threadIdx.x % n4, rl = threadIdx.x / n4;
+  for (int k = threadIdx.x; k < P.n; k += blockDim.x) cm[k] = 0u;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < (int)(blockDim.x >> 5); w++) amax = fmaxf(amax, wm[w]);
-    amax = fmaxf(amax, wm[0]);
-    float *sc = reinterpret_cast<float *>(P.payload + kHdrBytes);
-    sc[(isv ? P.r : 0) + k] = (float)((double)amax / 7.0);
+  if (rl < lanes) {
+    float mx = 0.f, my = 0.f, mz = 0.f, mw = 0.f;
+    for (int rr = rl; rr < kScaleRows; rr += lanes) {
+      const float4 v = m4[rr * n4 + cg];
+      mx = fmaxf(mx, fabsf(v.x));
+      my = fmaxf(my, fabsf(v.y));
+      mz = fmaxf(mz, fabsf(v.z));
+      mw = fmaxf(mw, fabsf(v.w));
+    }
+    atomicMax(&cm[4 * cg], __float_as_uint(mx));
+    atomicMax(&cm[4 * cg + 1], __float_as_uint(my));
+    atomicMax(&cm[4 * cg + 2], __float_as_uint(mz));
+    atomicMax(&cm[4 * cg + 3], __float_as_uint(mw));
   }
+  __syncthreads();
+  for (int k = threadIdx.x; k < P.r; k += blockDim.x)
+    if (cm[k]) atomicMax(&P.amax[(isv ? P.n : 0) + k], cm[k]);
+}
+
+// Scale s_k = fp32(absmax_k / 7) of column k of U (k < r) or V (k >= r).
+__device__ __forceinline__ float lr_scale_of(const PackArgs &P, int k) {
+  const unsigned bits = k < P.r ? P.amax[k] : P.amax[P.n + k - P.r];
+  return (float)((double)__uint_as_float(bits) / 7.0);
 }
 
 __device__ __forceinline__ uint32_t int4_code(float x, float s) {
@@ -721,24 +754,27 @@ __global__ void __launch_bounds__(256) lr_pack_kernel(PackArgs P) {
   const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (P.int4) {
-    const float *sc = reinterpret_cast<const float *>(body);
+    // the scale section: block 0 writes the 2r scales, every thread computes
+    // the ones it needs the same way
+    float *sc = reinterpret_cast<float *>(body);
+    if (blockIdx.x == 0)
+      for (int k = threadIdx.x; k < 2 * P.r; k += blockDim.x) sc[k] = lr_scale_of(P, k);
     // scale section padding
     for (int64_t b = (int64_t)P.r * 8 + tid; b < P.sec1; b += nthr) body[b] = 0;
-    const int64_t ubytes = P.sec2 - P.sec1, vbytes = P.body - P.sec2;
-    const int64_t un = P.rows * P.r, vn = P.cols * P.r;
-    for (int64_t b = tid; b < ubytes + vbytes; b += nthr) {
+    const uint32_t ubytes = (uint32_t)(P.sec2 - P.sec1), vbytes = (uint32_t)(P.body - P.sec2);
+    const uint32_t un = (uint32_t)(P.rows * P.r), vn = (uint32_t)(P.cols * P.r), r = (uint32_t)P.r;
+    for (uint32_t b = (uint32_t)tid; b < ubytes + vbytes; b += (uint32_t)nthr) {
       const bool isv = b >= ubytes;
-      const int64_t bb = isv ? b - ubytes : b;
-      const int64_t nel = isv ? vn : un;
+      const uint32_t bb = isv ? b - ubytes : b;
+      const uint32_t nel = isv ? vn : un;
       const float *m = isv ? P.v : P.q;
       uint32_t byte = 0;
 #pragma unroll
       for (int h = 0; h < 2; h++) {
-        const int64_t e = 2 * bb + h;
+        const uint32_t e = 2 * bb + h;
         if (e < nel) {
-          const int64_t i = e / P.r;
-          const int k = (int)(e % P.r);
-          byte |= int4_code(m[i * P.n + k], sc[(isv ? P.r : 0) + k]) << (4 * h);
+          const uint32_t i = e / r, k = e - i * r;
+          byte |= int4_code(m[(int64_t)i * P.n + k], lr_scale_of(P, (int)k + (isv ? P.r : 0))) << (4 * h);
         }
       }
       body[(isv ? P.sec2 : P.sec1) + bb] = (uint8_t)byte;
@@ -777,34 +813,36 @@ __global__ void __launch_bounds__(256) lr_dequant_kernel(DequantArgs D) {
   pdl_enter();
   if (D.check_header && !lr_header_ok(D.payload, D.expect, D.status)) return;
   const uint8_t *body = D.payload + kHdrBytes;
-  const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
-  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t un = D.rows * D.kp, vn = D.cols * D.kp;
   const float *sc = reinterpret_cast<const float *>(body);
-  for (int64_t e = tid; e < un + vn; e += nthr) {
-    const bool isv = e >= un;
-    const int64_t ee = isv ? e - un : e;
-    const int64_t i = ee / D.kp;
-    const int k = (int)(ee % D.kp);
-    float x = 0.0f;
-    if (k < D.r) {
-      if (D.int4) {
-        const uint8_t *nb = body + (isv ? D.sec2 : D.sec1);
-        const int q = nibble_at(nb, i * D.r + k);
-        x = isv ? (float)((double)q * (double)sc[k] * (double)sc[D.r + k]) : (float)q;
-      } else {
-        const float *f = reinterpret_cast<const float *>(body + (isv ? D.sec2 : 0));
-        x = f[i * D.r + k];
+  // one warp per row: rows of U first, then rows of V; lanes over the kp columns
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarp = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t total = D.rows + D.cols;
+  for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < total; row += nwarp) {
+    const bool isv = row >= D.rows;
+    const int64_t i = isv ? row - D.rows : row;
+    const uint8_t *nb = body + (isv ? D.sec2 : D.sec1);
+    const float *f = reinterpret_cast<const float *>(body + (isv ? D.sec2 : 0));
+    for (int k = lane; k < D.kp; k += 32) {
+      float x = 0.0f;
+      if (k < D.r) {
+        if (D.int4) {
+          const int q = nibble_at(nb, i * D.r + k);
+          x = isv ? (float)((double)q * (double)sc[k] * (double)sc[D.r + k]) : (float)q;
+        } else {
+          x = f[i * D.r + k];
+        }
       }
-    }
-    __nv_bfloat16 hi, lo;
-    split_bf16(x, hi, lo);
-    if (isv) {
-      D.vbhi[ee] = hi;
-      D.vblo[ee] = lo;
-    } else {
-      D.uahi[ee] = hi;
-      if (D.ualo) D.ualo[ee] = lo;
+      __nv_bfloat16 hi, lo;
+      split_bf16(x, hi, lo);
+      const int64_t o = i * D.kp + k;
+      if (isv) {
+        D.vbhi[o] = hi;
+        D.vblo[o] = lo;
+      } else {
+        D.uahi[o] = hi;
+        if (D.ualo) D.ualo[o] = lo;
+      }
     }
   }
 }
@@ -1052,12 +1090,21 @@ void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *p
   plan->rp = round_up(p.rank < 16 ? 16 : p.rank, 16);
   plan->kp = round_up(p.rank, kTileK);
   plan->supported = rows % 128 == 0 && cols % 128 == 0 && rows >= 128 && cols >= 128 && p.batch == 1 &&
-                    p.rank >= 1 && p.rank <= 128 && rows < (1ll << 30) && cols < (1ll << 30);
+                    p.rank >= 1 && p.rank <= 128 && rows < (1ll << 30) && cols < (1ll << 30) &&
+                    (rows + cols) * (int64_t)round_up(p.rank, kTileK) < (1ll << 31);  // 32-bit factor indices
   // split-K so that each thin GEMM fills the SMs: (tiles of 128 rows) x splits
   const int ty = (int)(rows / kTileM), tv = (int)(cols / kTileM);
   const int kby = (int)(cols / kTileK), kbv = (int)(rows / kTileK);
-  auto splits = [](int tiles, int kblocks) {
-    int s = (144 + tiles - 1) / tiles;
+  // one CTA per SM (the operand ring takes most of the shared memory): the
+  // largest split count that keeps tiles x splits within one wave
+  int nsm = 148, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) !=
+                                               cudaSuccess || nsm < 1) {
+    (void)cudaGetLastError();
+    nsm = 148;
+  }
+  auto splits = [nsm](int tiles, int kblocks) {
+    int s = nsm / tiles;
     if (s > kblocks) s = kblocks;
     return s < 1 ? 1 : s;
   };
@@ -1077,6 +1124,7 @@ void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *p
   enc += pad256(mx * rp * 4) * 2 + pad256(C * rp * 4);        // xbuf, q, v
   enc += pad256((size_t)plan->nblk_gram * rp * rp * 8);       // gpart
   enc += pad256(rp * rp * 8) + pad256(rp * 4);                // L, dead
+  enc += pad256(2 * rp * 4);                                  // amax
   plan->enc_scratch_bytes = enc;
   plan->dec_scratch_bytes = dec;
 }
@@ -1138,6 +1186,7 @@ int lowrank_bind(LowrankPlan *plan, void *scratch) {
     b.gpart = reinterpret_cast<double *>(take((size_t)plan->nblk_gram * rp * rp * 8));
     b.L = reinterpret_cast<double *>(take(rp * rp * 8));
     b.dead = reinterpret_cast<int *>(take(rp * 4));
+    b.amax = reinterpret_cast<unsigned *>(take(2 * rp * 4));
     ok = ok && make_map(&plan->tm_dhi, b.dhi, C, R, kTileM) && make_map(&plan->tm_dlo, b.dlo, C, R, kTileM) &&
          make_map(&plan->tm_vthi, b.vthi, C, rp, (uint32_t)rp) && make_map(&plan->tm_vtlo, b.vtlo, C, rp, (uint32_t)rp) &&
          make_map(&plan->tm_dthi, b.dthi, R, C, kTileM) && make_map(&plan->tm_dtlo, b.dtlo, R, C, kTileM) &&
@@ -1262,6 +1311,7 @@ PackArgs pack_args(const LowrankPlan &P, uint8_t *payload, const Header &hdr) {
     A.body = A.sec2 + (int64_t)pad16(C * r * 4);
   }
   A.hdr = hdr;
+  A.amax = P.b.amax;
   return A;
 }
 
@@ -1316,7 +1366,8 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
   if (tab) return cudaErrorNotSupported;  // batch 1 only
   const LowrankBufs &b = P.b;
   const int64_t R = P.rows, C = P.cols;
-  launch_pdl(lr_vprep_kernel, dim3(P.rp), dim3(256), 0, st, vprev, C, P.rank, P.rp, step == 1 ? 1 : 0, seed, b.vthi, b.vtlo);
+  launch_pdl(lr_vprep_kernel, dim3(P.rp), dim3(kVprepThreads), 0, st, vprev, C, P.rank, P.rp, step == 1 ? 1 : 0, seed, b.vthi, b.vtlo,
+             b.amax);
   const dim3 dg((unsigned)(C / 64), (unsigned)(R / 64));
   if (P.dtype == CF_BF16)
     launch_pdl(lr_delta_kernel<__nv_bfloat16>, dim3(dg), dim3(256), 0, st, static_cast<const __nv_bfloat16 *>(args.a), args.ahat, args.err,
@@ -1345,7 +1396,7 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
   }
   // INT4 (or fp32) factors into the payload
   const PackArgs pa = pack_args(P, args.payload, args.hdr);
-  if (P.int4) launch_pdl(lr_scale_kernel, dim3(2 * P.rank), dim3(256), 0, st, pa);
+  if (P.int4) launch_pdl(lr_scale_kernel, dim3((unsigned)((R + C) / kScaleRows)), dim3(256), 0, st, pa);
   launch_pdl(lr_pack_kernel, dim3(592), dim3(256), 0, st, pa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // sender reconstruction from the payload bytes

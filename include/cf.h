@@ -153,6 +153,7 @@ CF_API int cf_workspace_bytes(int64_t rows, int64_t cols, int mode, const cf_par
  * rules: rows >= 1; cols % 8 == 0 and cols <= 8192; CF_SIGN1 cols % 32 == 0;
  * CF_Q2 cols % 16 == 0; CF_NM cols % M == 0 and (cols/M) N log2(M) % 32 == 0;
  * CF_LOWRANK rows % 128 == 0, cols % 128 == 0, rank <= min(rows, cols, 128),
+ * (rows + cols) * round_up(rank, 64) < 2^31 (32-bit factor indices),
  * batch 1 (the low-rank state also holds its factor scratch: about
  * 8 rows*cols bytes for a sender).  The state owns its tensors (in `workspace`
  * when given, else in memory it allocates with cudaMalloc) and starts at
