@@ -31,7 +31,7 @@ CF_ERR_TOO_LARGE = -12
 CF_IDENTITY, CF_SIGN1, CF_Q2, CF_NM, CF_LOWRANK = 0, 1, 2, 3, 4
 CF_F32, CF_BF16 = 0, 1
 CF_SENDER, CF_RECEIVER = 0, 1
-CF_EF_EXPLICIT, CF_EF_IMPLICIT = 0, 1
+CF_EF_EXPLICIT, CF_EF_IMPLICIT, CF_EF_OFF = 0, 1, 2
 CF_T_RECON, CF_T_ERROR, CF_T_VPREV = 0, 1, 2
 
 MODE_NAMES = {"identity": CF_IDENTITY, "sign1": CF_SIGN1, "q2": CF_Q2, "nm": CF_NM, "lowrank": CF_LOWRANK}

@@ -101,7 +101,7 @@ int validate(int64_t rows, int64_t cols, int mode, const cf_params *p) {
   if (mode < CF_IDENTITY || mode > CF_LOWRANK) return CF_ERR_ARG;
   if (p->dtype != CF_F32 && p->dtype != CF_BF16) return CF_ERR_ARG;
   if (p->role != CF_SENDER && p->role != CF_RECEIVER) return CF_ERR_ARG;
-  if (p->ef != CF_EF_EXPLICIT && p->ef != CF_EF_IMPLICIT) return CF_ERR_ARG;
+  if (p->ef != CF_EF_EXPLICIT && p->ef != CF_EF_IMPLICIT && p->ef != CF_EF_OFF) return CF_ERR_ARG;
   if (p->batch < 1 || p->batch > kMaxBatch * 1024) return CF_ERR_ARG;
   if (rows < 1 || cols < 8) return CF_ERR_SHAPE;
   if (cols % 8) return CF_ERR_SHAPE;
@@ -201,6 +201,7 @@ EncArgs enc_args(cf_state *s, const void *a, void *payload, bool warm) {
   A.sec1 = (int64_t)s->lay.sec1;
   A.batch = s->p.batch;
   A.ef_explicit = s->p.ef == CF_EF_EXPLICIT;
+  A.ef_off = s->p.ef == CF_EF_OFF;
   A.team_log2 = s->cfg.team_log2;
   A.status = s->status;
   A.hdr = header_of(s, warm, s->step);

@@ -48,6 +48,7 @@ struct EncArgs {
   int64_t sec1;           // offset of codes / indices in a body
   int batch;
   int ef_explicit;
+  int ef_off;             // CF_EF_OFF: ahat <- fp32(a), e untouched
   int team_log2;          // threads per row = 1 << team_log2 (>= 32)
   int64_t padA_off, padA_len;  // alignment padding inside each body, zeroed by the encoder
   int64_t padB_off, padB_len;

@@ -855,6 +855,7 @@ struct ReconArgs {
   int a_split;        // 1: A carries a lo term (fp32 factors)
   int role;           // CF_SENDER: e, ahat update; CF_RECEIVER: ahat, recon
   int ef_explicit;
+  int ef_off;  // CF_EF_OFF: ahat <- fp32(a), e untouched
   const void *a;      // sender: activations [rows][cols]
   float *ahat;
   float *err;
@@ -1008,6 +1009,10 @@ __global__ void __launch_bounds__(kReconThreads, 2)
       float hn[4];
 #pragma unroll
       for (int k = 0; k < 4; k++) hn[k] = __fadd_rn(h[k], c[k]);
+      if (R.role == CF_SENDER && R.ef_off) {  // no error feedback: the state is the activation
+        __stcs(reinterpret_cast<float4 *>(R.ahat + off[u]), make_float4(xv[u][0], xv[u][1], xv[u][2], xv[u][3]));
+        continue;
+      }
       __stcs(reinterpret_cast<float4 *>(R.ahat + off[u]), make_float4(hn[0], hn[1], hn[2], hn[3]));
       if (R.role == CF_SENDER) {
         const float e[4] = {ev[u].x, ev[u].y, ev[u].z, ev[u].w};
@@ -1087,6 +1092,7 @@ void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *p
   plan->role = p.role;
   plan->dtype = p.dtype;
   plan->ef_explicit = p.ef == CF_EF_EXPLICIT;
+  plan->ef_off = p.ef == CF_EF_OFF;
   plan->rp = round_up(p.rank < 16 ? 16 : p.rank, 16);
   plan->kp = round_up(p.rank, kTileK);
   plan->supported = rows % 128 == 0 && cols % 128 == 0 && rows >= 128 && cols >= 128 && p.batch == 1 &&
@@ -1342,6 +1348,7 @@ cudaError_t dequant_and_recon(const LowrankPlan &P, const uint8_t *payload, bool
   R.a_split = P.int4 ? 0 : 1;
   R.role = receiver ? CF_RECEIVER : CF_SENDER;
   R.ef_explicit = P.ef_explicit;
+  R.ef_off = P.ef_off;
   R.a = a;
   R.ahat = ahat;
   R.err = err;
@@ -1462,7 +1469,7 @@ extern "C" int cf_lowrank_decode_noalloc(int64_t rows, int64_t cols, const cf_pa
   using namespace cfi;
   if (!p || !payload || !ahat || !recon || !status || step < 1) return CF_ERR_ARG;
   if (p->dtype != CF_F32 && p->dtype != CF_BF16) return CF_ERR_ARG;
-  if (p->ef != CF_EF_EXPLICIT && p->ef != CF_EF_IMPLICIT) return CF_ERR_ARG;
+  if (p->ef != CF_EF_EXPLICIT && p->ef != CF_EF_IMPLICIT && p->ef != CF_EF_OFF) return CF_ERR_ARG;
   if (p->lr_int4 != 0 && p->lr_int4 != 1) return CF_ERR_ARG;
   if (p->iters < 1 || p->iters > 2) return CF_ERR_UNSUPPORTED;
   if (rows < 128 || cols < 128 || rows % 128 || cols % 128 || cols > kMaxCols) return CF_ERR_SHAPE;

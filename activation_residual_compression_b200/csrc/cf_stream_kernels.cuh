@@ -315,7 +315,8 @@ __device__ __forceinline__ void zero_padding(const EncArgs &A) {
 
 // One row of the fused encode, given the thread's raw inputs (a, ahat, e of
 // its vectors v = t + j * TEAM): residual with error feedback, row statistic,
-// encode, payload stores, e = D - C and ahat = ahat + C stores.  Every thread
+// encode, payload stores, e = D - C and ahat = ahat + C stores (with
+// CF_EF_OFF: ahat = fp32(a) and no e store).  Every thread
 // of the block calls this together (team reductions use __syncthreads).
 template <int MODE, typename T, int VPT, int NM_M, int NM_N>
 __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const int tlog, const bool row_ok,
@@ -338,7 +339,9 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
                          re[j][1].x, re[j][1].y, re[j][1].z, re[j][1].w};
 #pragma unroll
     for (int k = 0; k < 8; k++) {
-      h[j][k] = hv[k];
+      // without error feedback the new state is the activation itself; it
+      // takes the registers of ahat, which the update then does not need
+      h[j][k] = A.ef_off ? x[k] : hv[k];
       const float tt = __fsub_rn(x[k], hv[k]);
       d[j][k] = A.ef_explicit ? __fadd_rn(tt, ev[k]) : tt;
     }
@@ -568,9 +571,9 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
 #pragma unroll
       for (int k = 0; k < 8; k++) {
         en[k] = __fsub_rn(d[j][k], c[j][k]);
-        hn[k] = __fadd_rn(h[j][k], c[j][k]);
+        hn[k] = A.ef_off ? h[j][k] : __fadd_rn(h[j][k], c[j][k]);
       }
-      store_f32x8(erow + v * 8, en);
+      if (!A.ef_off) store_f32x8(erow + v * 8, en);
       store_f32x8(hrow + v * 8, hn);
     }
   }

@@ -83,10 +83,13 @@ def _payload_body(mode, rows, cols, kw):
     raise ValueError(mode)
 
 
-def encode_bytes(mode, rows, cols, kw, act_size=2):
-    """Algorithmic bytes of one encode launch: read a, ahat, e; write ahat, e, payload."""
+def encode_bytes(mode, rows, cols, kw, act_size=2, ef="explicit"):
+    """Algorithmic bytes of one encode launch: read a, ahat, e; write ahat, e, payload.
+    Implicit feedback does not read e; without feedback e is neither read nor written."""
     E = rows * cols
-    return E * (act_size + 4 + 4 + 4 + 4) + 64 + _payload_body(mode, rows, cols, kw)
+    e_rd = 4 if ef == "explicit" else 0
+    e_wr = 0 if ef == "off" else 4
+    return E * (act_size + 4 + e_rd + 4 + e_wr) + 64 + _payload_body(mode, rows, cols, kw)
 
 
 def decode_bytes(mode, rows, cols, kw, act_size=2):
@@ -173,6 +176,9 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- GPU arm
 
+EF_CODES = {"explicit": 0, "implicit": 1, "off": 2}
+
+
 def _codec_name(mode, kw):
     if mode == "nm":
         return f"nm{kw['nm_n']}_{kw['nm_m']}"
@@ -192,11 +198,12 @@ def _make_stream(kind, wl, seed, device="cuda"):
     raise ValueError(kind)
 
 
-def step_bytes(mode, rows, cols, kw, payload):
-    """Algorithmic bytes of one encode + decode of one tensor."""
+def step_bytes(mode, rows, cols, kw, payload, ef="explicit"):
+    """Algorithmic bytes of one encode + decode of one tensor (low-rank: the
+    explicit-feedback figure)."""
     if mode == "lowrank":
         return _lr_alg_bytes(rows, cols, kw["iters"], payload)
-    return encode_bytes(mode, rows, cols, kw) + decode_bytes(mode, rows, cols, kw)
+    return encode_bytes(mode, rows, cols, kw, ef=ef) + decode_bytes(mode, rows, cols, kw)
 
 
 def launches_per_call(mode, kw, encode):
@@ -227,7 +234,7 @@ def run_cf(args, rank, world, device):
         s = _make_stream(wl["stream"], wl, seed=1 + 100 * mi + 1000 * rank)
         acts = [s.next() for _ in range(n_inputs)]
         del s
-        base = dict(dtype=cf.CF_BF16, batch=B_, **kw)
+        base = dict(dtype=cf.CF_BF16, batch=B_, ef=EF_CODES[args.ef], **kw)
         S = cf.cf_create(R_, C_, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_SENDER, **base))
         R = cf.cf_create(R_, C_, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_RECEIVER, **base))
         pay = torch.empty(max(cf.cf_payload_bytes(S, True), cf.cf_payload_bytes(S, False)), dtype=torch.uint8,
@@ -464,6 +471,53 @@ def run_suite(args, device):
     return out
 
 
+EF_STUDY_MODES = [("sign1", {}), ("q2", {}), ("nm", {"nm_n": 1, "nm_m": 16}), ("nm", {"nm_n": 2, "nm_m": 16}),
+                  ("lowrank", {"rank": 70, "iters": 1, "lr_int4": 1, "seed": 7})]
+EF_STUDY_STEPS = (1, 2, 5, 10, 20, 27, 40, 49)
+
+
+def run_ef_study(args, device, T=50):
+    """Receiver error ||recon_t - a_t|| / ||a_t|| of the CUDA codec (C ABI) over
+    T steps of the stationary AR(1) stream (rho = sqrt(0.99), innovations
+    0.1 N(0, 1), so sigma_Delta / sigma_a ~ 0.1) for every mode and feedback
+    form: explicit (the recurrence as specified), implicit (residual against
+    the reconstruction only) and off (residual against the previous
+    activation).  Streaming modes on 4608 x 3072 bf16, low-rank on 4096 x 3072."""
+    import torch
+
+    import activation_residual_compression_b200 as cf
+    from activation_residual_compression_b200 import inputs
+    torch.cuda.set_device(device)
+    out = {}
+    for mode, kw in EF_STUDY_MODES:
+        rows, cols = (4096, 3072) if mode == "lowrank" else (ROWS, COLS)
+        row = {}
+        for ef in ("explicit", "implicit", "off"):
+            base = dict(dtype=cf.CF_BF16, ef=EF_CODES[ef], **kw)
+            S = cf.cf_create(rows, cols, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_SENDER, **base))
+            R = cf.cf_create(rows, cols, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_RECEIVER, **base))
+            pay = torch.empty(max(cf.cf_payload_bytes(S, True), cf.cf_payload_bytes(S, False)), dtype=torch.uint8,
+                              device="cuda")
+            rec = torch.empty(1, rows, cols, dtype=torch.bfloat16, device="cuda")
+            s = inputs.ar1("cuda", rows=rows, cols=cols, seed=1)
+            rel = []
+            for _ in range(T):
+                a = s.next()
+                cf.cf_encode(S, a, pay)
+                cf.cf_decode(R, pay, rec)
+                af = a.float()
+                rel.append(float(torch.linalg.vector_norm(rec.float() - af) / torch.linalg.vector_norm(af)))
+            if cf.cf_status(R) != cf.CF_OK or cf.cf_status(S) != cf.CF_OK:
+                raise RuntimeError(f"{mode} {ef}: codec reported an error status")
+            cf.cf_destroy(S)
+            cf.cf_destroy(R)
+            row[ef] = {str(t): (round(rel[t], 5) if rel[t] < 1e6 else float(f"{rel[t]:.3e}")) for t in EF_STUDY_STEPS}
+        out[_codec_name(mode, kw)] = row
+    print(json.dumps({"ef_study": out, "metric": "receiver relative L2 error ||recon_t - a_t|| / ||a_t|| at step t",
+                      "stream": "ar1 rho=sqrt(0.99) sigma=0.1 (stationary, sigma_Delta/sigma_a ~ 0.1)",
+                      "steps": T, "data": "synthetic"}), flush=True)
+
+
 def cpu_baseline(wl=None, max_seconds=20.0):
     """The CPU oracle, as it stands, on the same workload (full-size tensors;
     for the 60-tensor step the first tensors only, tensors being independent),
@@ -572,6 +626,10 @@ def main():
                     help="timed workload (default: the FLUX-shaped 1-bit + 2-bit step)")
     ap.add_argument("--resident-gb", type=float, default=12.0, help="device memory for pre-generated inputs")
     ap.add_argument("--no-cogvideox", action="store_true", help="skip the 60-tensor CogVideoX-shaped step")
+    ap.add_argument("--ef", default="explicit", choices=sorted(EF_CODES),
+                    help="error-feedback form of the timed codecs (default: explicit)")
+    ap.add_argument("--ef-study", action="store_true",
+                    help="instead of timing: receiver error per step of every mode and feedback form")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -588,6 +646,10 @@ def main():
     import torch
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
+    if args.ef_study:
+        if rank == 0:
+            run_ef_study(args, local)
+        return
     dist = None
     if world > 1:
         import datetime
@@ -617,15 +679,15 @@ def main():
         kern = f"cf_encode low-rank ({launches_per_call(c0['mode'], c0['kw'], True)} launches)"
         tr = None
     else:
-        enc_alg = B_ * encode_bytes(c0["mode"], R_, C_, c0["kw"])
+        enc_alg = B_ * encode_bytes(c0["mode"], R_, C_, c0["kw"], ef=args.ef)
         kern = f"encode_kernel<{c0['name']}, bf16>"
-        tr = _traffic_record() if args.workload == "flux" else None
+        tr = _traffic_record() if args.workload == "flux" and args.ef == "explicit" else None
     achieved = enc_alg / (enc_ms / 1e3) / 1e9
     per_mode = {}
     for c in st["codecs"]:
         pm = st["per"][c["name"]]
         step_ms = pm["enc"] + pm["dec"]
-        alg = B_ * step_bytes(c["mode"], R_, C_, c["kw"], c["P"])
+        alg = B_ * step_bytes(c["mode"], R_, C_, c["kw"], c["P"], ef=args.ef)
         per_mode[c["name"]] = {"ms_per_step": round(step_ms, 5), "encode_ms": round(pm["enc"], 5),
                                "decode_ms": round(pm["dec"], 5),
                                "activation_gbs": round(B_ * R_ * C_ * 2 / (step_ms / 1e3) / 1e9, 2),
@@ -639,7 +701,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": wl["name"], "rows": R_, "cols": C_, "tensors": B_, "activation_dtype": "bf16",
-                   "modes": [c["name"] for c in st["codecs"]], "error_feedback": "explicit",
+                   "modes": [c["name"] for c in st["codecs"]], "error_feedback": args.ef,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": f"inputs larger than L2: a fresh {in_mb:.0f} MB input per codec per step, state "
                          f"{B_ * R_ * C_ * 12 / 1e6:.0f} MB per codec",
@@ -657,7 +719,7 @@ def main():
         line["e2e"] = {"value": round(act_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                        "h2d_bytes_per_step": st["e2e"]["h2d"], "d2h_bytes_per_step": st["e2e"]["d2h"],
                        "ms_per_step": round(e2e_ms, 4)}
-    if world == 1 and not args.no_suite and args.workload == "flux":
+    if world == 1 and not args.no_suite and args.workload == "flux" and args.ef == "explicit":
         line["suite"] = run_suite(args, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)

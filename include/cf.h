@@ -112,8 +112,14 @@ typedef enum { CF_F32 = 0, CF_BF16 = 1 } cf_dtype;
 typedef enum { CF_SENDER = 0, CF_RECEIVER = 1 } cf_role;
 /* Error-feedback form ("Key design: error feedback"):
  *   CF_EF_EXPLICIT  D = (a - ahat) + e   (default; the recurrence as stated)
- *   CF_EF_IMPLICIT  D = a - ahat; e = D - C is still recorded. */
-typedef enum { CF_EF_EXPLICIT = 0, CF_EF_IMPLICIT = 1 } cf_ef;
+ *   CF_EF_IMPLICIT  D = a - ahat; e = D - C is still recorded.
+ *   CF_EF_OFF       residual compression without error feedback, the
+ *                   variant whose error the page says grows linearly with
+ *                   the step count: the sender's ahat slot holds fp32 of the
+ *                   previous activation, D = a_t - a_{t-1}, and the sender's
+ *                   update is ahat = fp32(a_t); e is neither read nor
+ *                   written.  The receiver is the same for all three. */
+typedef enum { CF_EF_EXPLICIT = 0, CF_EF_IMPLICIT = 1, CF_EF_OFF = 2 } cf_ef;
 
 /* which tensor cf_tensor() returns */
 typedef enum { CF_T_RECON = 0, CF_T_ERROR = 1, CF_T_VPREV = 2 } cf_which;

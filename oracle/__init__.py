@@ -28,7 +28,7 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
 MODES = {"identity": 0, "sign1": 1, "q2": 2, "nm": 3, "lowrank": 4}
 DTYPES = {"f32": 0, "bf16": 1}
-EFS = {"explicit": 0, "implicit": 1}
+EFS = {"explicit": 0, "implicit": 1, "off": 2}
 
 
 def build(force: bool = False) -> str:

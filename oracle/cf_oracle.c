@@ -17,7 +17,10 @@
  *             e = D - C;  ahat_S = ahat_S + C  (fp32 RN)
  *   receiver: ahat_R = ahat_R + dec(payload);  recon = cast(ahat_R)
  * With implicit error feedback D = a_t - ahat_S (the error already lives in
- * the reconstruction) and e is only recorded.
+ * the reconstruction) and e is only recorded.  Without error feedback (the
+ * variant whose error the page says grows linearly with the step count) the
+ * sender's ahat slot holds fp32(a_{t-1}): D = a_t - a_{t-1}, and the update
+ * is ahat_S = fp32(a_t); e stays zero.
  *
  * The pages give no bit layouts, scales or rounding rules.  The encodings
  * below are the readings this project fixes (IEEE round-to-nearest-even in
@@ -52,6 +55,7 @@
 
 #define ORC_EF_EXPLICIT 0
 #define ORC_EF_IMPLICIT 1
+#define ORC_EF_OFF 2 /* residual against the previous activation, no feedback */
 
 #define ORC_MAGIC 0x31504643u /* bytes 'C','F','P','1' */
 #define ORC_HDR 64
@@ -256,7 +260,7 @@ orc_state *orc_create(int64_t rows, int64_t cols, int mode, int dtype, int ef, i
     if (rows < 1 || cols < 1 || batch < 1) return NULL;
     if (mode < ORC_IDENTITY || mode > ORC_LOWRANK) return NULL;
     if (dtype != ORC_F32 && dtype != ORC_BF16) return NULL;
-    if (ef != ORC_EF_EXPLICIT && ef != ORC_EF_IMPLICIT) return NULL;
+    if (ef != ORC_EF_EXPLICIT && ef != ORC_EF_IMPLICIT && ef != ORC_EF_OFF) return NULL;
     if (cols % 8) return NULL;
     if (mode == ORC_SIGN1 && cols % 32) return NULL;
     if (mode == ORC_Q2 && cols % 16) return NULL;
@@ -687,8 +691,15 @@ int orc_encode(orc_state *o, const void *a, uint8_t *payload)
             for (int64_t r = 0; r < o->rows; r++) encode_row(o, d + r * o->cols, body, r, C + r * o->cols);
         }
         for (int64_t i = 0; i < E; i++) {
-            er[i] = d[i] - C[i];
-            ah[i] = ah[i] + C[i];
+            if (o->ef == ORC_EF_OFF) {
+                /* "Key design: error feedback" names what happens without
+                 * feedback: the untransmitted error is dropped, and the
+                 * next residual is taken against this step's activation */
+                ah[i] = load_act(a, o->dtype, (int64_t)b * E + i);
+            } else {
+                er[i] = d[i] - C[i];
+                ah[i] = ah[i] + C[i];
+            }
         }
     }
     free(d); free(C);

@@ -39,7 +39,7 @@ class GpuPair:
         self.mode = cf.MODE_NAMES[mode]
         self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
         kw = dict(dtype=cf.CF_BF16 if dtype == "bf16" else cf.CF_F32,
-                  ef=cf.CF_EF_EXPLICIT if ef == "explicit" else cf.CF_EF_IMPLICIT,
+                  ef={"explicit": cf.CF_EF_EXPLICIT, "implicit": cf.CF_EF_IMPLICIT, "off": cf.CF_EF_OFF}[ef],
                   nm_n=nm_n, nm_m=nm_m, batch=batch, rank=rank, iters=iters, lr_int4=lr_int4, seed=seed)
         self.S = cf.cf_create(rows, cols, self.mode, cf.cf_params_init(role=cf.CF_SENDER, **kw))
         self.R = cf.cf_create(rows, cols, self.mode, cf.cf_params_init(role=cf.CF_RECEIVER, **kw))

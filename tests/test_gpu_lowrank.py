@@ -121,6 +121,38 @@ def test_teacher_forced_matches_oracle(rows, cols, rank, iters):
     print(f"worst teacher-forced rel Frobenius {worst:.3e}")
 
 
+def test_error_feedback_off_teacher_forced():
+    """No feedback: D = a_t - a_{t-1}; the sender's state becomes fp32(a_t)
+    exactly, e stays zero, the payload stands for the oracle's C within the
+    low-rank tolerance, and the receiver adds C(payload)."""
+    rows, cols, rank = 512, 384, 40
+    pair = GpuPair(rows, cols, "lowrank", dtype="bf16", ef="off", rank=rank, iters=1, lr_int4=1, seed=7)
+    orc = oracle.Oracle(rows, cols, "lowrank", dtype="bf16", ef="off", rank=rank, iters=1, lr_int4=1, seed=7)
+    s = inputs.ar1("cuda", rows=rows, cols=cols)
+    try:
+        for t in range(6):
+            a = s.next()
+            a_np = to_np(a)
+            if t == 0:
+                pair.step(a)
+                continue
+            p_o = _teacher_force(orc, pair, a_np, t)
+            ah_r_pre = pair.state("R")[0][0].copy()
+            pair.step(a)
+            torch.cuda.synchronize()
+            p_g = pair.payload_np(False)
+            assert np.array_equal(p_g[:64], p_o[:64])
+            C_g = orc.meaning(p_g)
+            assert _rel(C_g, orc.meaning(p_o)) <= 2e-2, t
+            ah_s, e_s = pair.state("S")
+            assert np.array_equal(ah_s[0].view(np.uint32), oracle.f32_from_bf16(a_np[0]).view(np.uint32))
+            assert not np.any(e_s)
+            assert _rel(pair.state("R")[0][0] - ah_r_pre, C_g) < 1e-4
+        assert cf.cf_status(pair.R) == cf.CF_OK and cf.cf_status(pair.S) == cf.CF_OK
+    finally:
+        pair.close()
+
+
 def test_closed_loop_quality_matches_oracle():
     """Run GPU and oracle independently on the same stream.  Their states are not
     compared (INT4 ties that round differently make the two error-feedback

@@ -23,7 +23,8 @@ def _np_act(a: torch.Tensor):
     return to_np(a)
 
 
-def _run_and_compare(pair: GpuPair, orc: oracle.Oracle, stream_next, steps, check_state_every=1):
+def _run_and_compare(pair: GpuPair, orc: oracle.Oracle, stream_next, steps, check_state_every=1,
+                     sender_tracks_receiver=True):
     for t in range(steps):
         a = stream_next()
         pair.step(a)
@@ -44,7 +45,8 @@ def _run_and_compare(pair: GpuPair, orc: oracle.Oracle, stream_next, steps, chec
             assert np.array_equal(ah_s.view(np.uint32), orc.ahat_s.view(np.uint32)), f"ahat_S differs at step {t}"
             assert np.array_equal(e_s.view(np.uint32), orc.err.view(np.uint32)), f"e differs at step {t}"
             assert np.array_equal(ah_r.view(np.uint32), orc.ahat_r.view(np.uint32)), f"ahat_R differs at step {t}"
-            assert np.array_equal(ah_s.view(np.uint32), ah_r.view(np.uint32))
+            if sender_tracks_receiver:
+                assert np.array_equal(ah_s.view(np.uint32), ah_r.view(np.uint32))
     assert pair.guards_ok(), "a kernel wrote outside its buffers"
 
 
@@ -98,14 +100,34 @@ def test_modes_and_shapes_bit_exact(mode, kw, rows, cols, dtype):
         pair.close()
 
 
-@pytest.mark.parametrize("mode,kw", [("sign1", {}), ("q2", {}), ("nm", {"nm_n": 2, "nm_m": 16})])
-def test_implicit_error_feedback_bit_exact(mode, kw):
+@pytest.mark.parametrize("ef", ["implicit", "off"])
+@pytest.mark.parametrize("mode,kw", [("sign1", {}), ("q2", {}), ("nm", {"nm_n": 2, "nm_m": 16}),
+                                     ("nm", {"nm_n": 1, "nm_m": 4}), ("identity", {})])
+def test_other_error_feedback_forms_bit_exact(mode, kw, ef):
+    """Implicit feedback, and no feedback (the sender's state is the previous
+    activation, e stays zero): payloads and both states bit-identical."""
     rows, cols = 65, 3072
     s = inputs.ActivationStream(rows, cols, dtype=torch.bfloat16, device="cuda", seed=5)
-    pair = GpuPair(rows, cols, mode, dtype="bf16", ef="implicit", **kw)
-    orc = oracle.Oracle(rows, cols, mode, dtype="bf16", ef="implicit", **kw)
+    pair = GpuPair(rows, cols, mode, dtype="bf16", ef=ef, **kw)
+    orc = oracle.Oracle(rows, cols, mode, dtype="bf16", ef=ef, **kw)
     try:
-        _run_and_compare(pair, orc, s.next, 5)
+        _run_and_compare(pair, orc, s.next, 5, sender_tracks_receiver=ef != "off")
+        if ef == "off":
+            _, e_s = pair.state("S")
+            assert not np.any(e_s)
+    finally:
+        pair.close()
+
+
+@pytest.mark.parametrize("mode,kw", [("sign1", {}), ("q2", {})])
+def test_error_feedback_off_batched_fp32_bit_exact(mode, kw):
+    """No feedback in the batched launch with fp32 activations."""
+    rows, cols, batch = 40, 512, 3
+    s = inputs.ActivationStream(rows, cols, dtype=torch.float32, device="cuda", seed=8, batch=batch)
+    pair = GpuPair(rows, cols, mode, dtype="f32", ef="off", batch=batch, **kw)
+    orc = oracle.Oracle(rows, cols, mode, dtype="f32", ef="off", batch=batch, **kw)
+    try:
+        _run_and_compare(pair, orc, s.next, 4, sender_tracks_receiver=False)
     finally:
         pair.close()
 
