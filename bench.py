@@ -518,6 +518,59 @@ def run_ef_study(args, device, T=50):
                       "steps": T, "data": "synthetic"}), flush=True)
 
 
+# Low-rank settings at (about) one payload: INT4 factors at rank 70 against fp32
+# factors at rank 9 (the rank that fits the same bytes), one and two sweeps,
+# plus INT4 at rank 128 as the larger-payload point.
+LR_SWEEP = [(70, 1, 1), (70, 2, 1), (9, 1, 0), (9, 2, 0), (128, 1, 1), (128, 2, 1), (35, 2, 1)]
+
+
+def run_lr_sweep(args, device, T=50, ef="implicit"):
+    """Low-rank quality sweep ("coverage over precision"): receiver error of
+    the CUDA codec on the stationary AR(1) stream (4096 x 3072 bf16) for rank,
+    sweeps and factor precision, with the payload bytes and the encode time."""
+    import torch
+
+    import activation_residual_compression_b200 as cf
+    from activation_residual_compression_b200 import inputs
+    torch.cuda.set_device(device)
+    rows, cols = 4096, 3072
+    out = []
+    for rank, iters, int4 in LR_SWEEP:
+        base = dict(dtype=cf.CF_BF16, ef=EF_CODES[ef], rank=rank, iters=iters, lr_int4=int4, seed=7)
+        S = cf.cf_create(rows, cols, cf.MODE_NAMES["lowrank"], cf.cf_params_init(role=cf.CF_SENDER, **base))
+        R = cf.cf_create(rows, cols, cf.MODE_NAMES["lowrank"], cf.cf_params_init(role=cf.CF_RECEIVER, **base))
+        P = cf.cf_payload_bytes(S, False)
+        pay = torch.empty(max(cf.cf_payload_bytes(S, True), P), dtype=torch.uint8, device="cuda")
+        rec = torch.empty(1, rows, cols, dtype=torch.bfloat16, device="cuda")
+        s = inputs.ar1("cuda", rows=rows, cols=cols, seed=1)
+        rel, enc_ms = [], []
+        for t in range(T):
+            a = s.next()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            cf.cf_encode(S, a, pay)
+            e1.record()
+            cf.cf_decode(R, pay, rec)
+            af = a.float()
+            rel.append(float(torch.linalg.vector_norm(rec.float() - af) / torch.linalg.vector_norm(af)))
+            torch.cuda.synchronize()
+            if t >= 3:
+                enc_ms.append(e0.elapsed_time(e1))
+        if cf.cf_status(R) != cf.CF_OK or cf.cf_status(S) != cf.CF_OK:
+            raise RuntimeError(f"rank {rank} iters {iters}: codec reported an error status")
+        cf.cf_destroy(S)
+        cf.cf_destroy(R)
+        out.append({"rank": rank, "iters": iters, "factors": "int4" if int4 else "fp32", "payload_bytes": P,
+                    "ratio_vs_bf16": round(rows * cols * 2 / P, 1),
+                    "rel_err": {str(t): round(rel[t], 5) for t in EF_STUDY_STEPS},
+                    "steady_rel_err": round(statistics.mean(rel[T // 2:]), 5),
+                    "encode_ms": round(statistics.median(enc_ms), 4)})
+    print(json.dumps({"lr_sweep": out, "metric": "receiver relative L2 error ||recon_t - a_t|| / ||a_t||",
+                      "stream": "ar1 4096x3072 bf16 rho=sqrt(0.99) sigma=0.1", "error_feedback": ef,
+                      "steps": T, "data": "synthetic"}), flush=True)
+
+
 def cpu_baseline(wl=None, max_seconds=20.0):
     """The CPU oracle, as it stands, on the same workload (full-size tensors;
     for the 60-tensor step the first tensors only, tensors being independent),
@@ -630,6 +683,8 @@ def main():
                     help="error-feedback form of the timed codecs (default: explicit)")
     ap.add_argument("--ef-study", action="store_true",
                     help="instead of timing: receiver error per step of every mode and feedback form")
+    ap.add_argument("--lr-sweep", action="store_true",
+                    help="instead of timing: low-rank receiver error over rank, sweeps and factor precision")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -646,9 +701,9 @@ def main():
     import torch
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
-    if args.ef_study:
+    if args.ef_study or args.lr_sweep:
         if rank == 0:
-            run_ef_study(args, local)
+            (run_ef_study if args.ef_study else run_lr_sweep)(args, local)
         return
     dist = None
     if world > 1:
