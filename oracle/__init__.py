@@ -17,6 +17,7 @@ Activations are numpy arrays: float32, or uint16 holding bfloat16 bit patterns.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 
@@ -26,7 +27,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "cf_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
-MODES = {"identity": 0, "sign1": 1, "q2": 2, "nm": 3, "lowrank": 4}
+MODES = {"identity": 0, "sign1": 1, "q2": 2, "nm": 3, "lowrank": 4, "blocksel": 5}
 DTYPES = {"f32": 0, "bf16": 1}
 EFS = {"explicit": 0, "implicit": 1, "off": 2}
 
@@ -95,6 +96,14 @@ def lib():
         L.orc_lr_v0.argtypes = [c.c_uint64, c.c_int64, c.c_int, c.c_int]
         L.orc_householder_qr.argtypes = [P, c.c_int64, c.c_int, c.c_double, P, P, P]
         L.orc_subspace_iteration.argtypes = [P, c.c_int64, c.c_int64, c.c_int, c.c_int, P, P]
+        L.orc_next_is_warm.restype = c.c_int
+        L.orc_next_is_warm.argtypes = [P, c.c_int]
+        L.orc_set_blocksel.restype = c.c_int
+        L.orc_set_blocksel.argtypes = [P, c.c_int, c.c_int, c.c_int, c.c_int]
+        L.orc_blocksel_sent.restype = P
+        L.orc_blocksel_sent.argtypes = [P]
+        L.orc_blocksel_dissimilarity.restype = c.c_int
+        L.orc_blocksel_dissimilarity.argtypes = [P, P, P, P]
         _lib = L
     return _lib
 
@@ -189,7 +198,7 @@ class Oracle:
     """
 
     def __init__(self, rows, cols, mode, dtype="bf16", ef="explicit", nm_n=1, nm_m=16,
-                 rank=1, iters=1, lr_int4=1, batch=1, seed=0):
+                 rank=1, iters=1, lr_int4=1, batch=1, seed=0, bs_h=0, bs_block=8, bs_k=0, bs_warm=5):
         self.rows, self.cols, self.batch = int(rows), int(cols), int(batch)
         self.mode = mode
         self.dtype = dtype
@@ -198,6 +207,16 @@ class Oracle:
                                    nm_n, nm_m, rank, iters, lr_int4, batch, seed)
         if not self._h:
             raise ValueError("oracle rejected the configuration")
+        if mode == "blocksel":
+            # the grid defaults to square; k to a quarter of the blocks ("k/K = 1/4")
+            h = int(bs_h) or math.isqrt(self.rows)
+            K = (h // bs_block) * ((self.rows // h) // bs_block) if h else 0
+            self.bs_h, self.bs_w, self.bs_b = h, (self.rows // h if h else 0), int(bs_block)
+            self.bs_K = K
+            self.bs_k = int(bs_k) or max(1, K // 4)
+            self.bs_warm = int(bs_warm)
+            if lib().orc_set_blocksel(self._h, h, self.bs_b, self.bs_k, self.bs_warm) != 0:
+                raise ValueError("oracle rejected the block-selection configuration")
 
     def __del__(self):
         h = getattr(self, "_h", None)
@@ -224,7 +243,7 @@ class Oracle:
     def encode(self, a) -> np.ndarray:
         a = np.ascontiguousarray(a, dtype=self.np_act)
         assert a.size == self.batch * self.rows * self.cols
-        warm = self.step() == 0
+        warm = lib().orc_next_is_warm(self._h, 0) != 0
         out = np.zeros(self.payload_bytes(warm), dtype=np.uint8)
         lib().orc_encode(self._h, _ptr(a), _ptr(out))
         return out
@@ -264,6 +283,20 @@ class Oracle:
     @property
     def vprev(self):
         return self._buf(3, (self.batch, self.cols, self.rank))
+
+    @property
+    def sent(self):
+        """BLOCKSEL: live view of the per-block 'sent this round' flags."""
+        p = lib().orc_blocksel_sent(self._h)
+        return np.ctypeslib.as_array((ctypes.c_uint8 * self.bs_K).from_address(p))
+
+    def dissimilarity(self, prev: np.ndarray, cur: np.ndarray) -> np.ndarray:
+        """BLOCKSEL: cosine dissimilarity of every block between two fp32 activations."""
+        prev = np.ascontiguousarray(prev, dtype=np.float32)
+        cur = np.ascontiguousarray(cur, dtype=np.float32)
+        d = np.empty(self.bs_K, dtype=np.float64)
+        assert lib().orc_blocksel_dissimilarity(self._h, _ptr(prev), _ptr(cur), _ptr(d)) == 0
+        return d
 
     def set_vprev_valid(self, v: bool):
         lib().orc_set_vprev_valid(self._h, 1 if v else 0)

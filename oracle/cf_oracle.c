@@ -36,6 +36,13 @@
  *           are quantised to INT4 per column.
  *   IDENTITY: payload = D (fp32), C = D.
  *
+ *   BLOCKSEL: Otil's selective transmission ("Informative sub-block
+ *           selection", "Dynamic round-robin"): the token grid H x W (rows =
+ *           H*W in raster order) is cut into b x b blocks (all channels); per
+ *           step the k blocks of largest cosine dissimilarity against the
+ *           previous activation, among the blocks not yet sent this round,
+ *           are sent raw; the round restarts once every block has been sent.
+ *
  * Parity pins live in tests/test_oracle_*.py; every function here is checked
  * there against brute force, closed forms or a library routine.
  */
@@ -49,6 +56,7 @@
 #define ORC_Q2 2
 #define ORC_NM 3
 #define ORC_LOWRANK 4
+#define ORC_BLOCKSEL 5 /* Otil-style block selection (second workload) */
 
 #define ORC_F32 0
 #define ORC_BF16 1
@@ -216,6 +224,8 @@ typedef struct {
     float *err;      /* [batch][rows][cols] error-feedback memory */
     float *ahat_r;   /* [batch][rows][cols] receiver reconstruction */
     float *vprev;    /* LOWRANK: [batch][cols][rank] fp32 warm start */
+    int bs_h, bs_w, bs_b, bs_k, bs_warm, bs_K; /* BLOCKSEL grid, block side, blocks per step */
+    uint8_t *bs_sent; /* BLOCKSEL: [K] 1 = sent in the current round */
     int vprev_valid;
     uint64_t step_s, step_r;
     int status;      /* 0 ok; nonzero after a header mismatch */
@@ -244,8 +254,20 @@ size_t orc_tensor_body_bytes(const orc_state *o)
             return pad16((size_t)o->rank * 8u) + pad16((size_t)((R * o->rank + 1) / 2)) +
                    pad16((size_t)((Cc * o->rank + 1) / 2));
         return pad16((size_t)(R * o->rank) * 4u) + pad16((size_t)(Cc * o->rank) * 4u);
+    case ORC_BLOCKSEL:
+        return pad16((size_t)o->bs_k * 4u) +
+               (size_t)o->bs_k * (size_t)o->bs_b * (size_t)o->bs_b * (size_t)Cc * act_size(o->dtype);
     }
     return 0;
+}
+
+/* number of leading steps sent in full */
+static uint64_t warm_steps(const orc_state *o) { return o->mode == ORC_BLOCKSEL ? (uint64_t)o->bs_warm : 1u; }
+
+/* 1 if the next encode (receiver: decode) is a full-size warm-up step */
+int orc_next_is_warm(const orc_state *o, int receiver)
+{
+    return (receiver ? o->step_r : o->step_s) < warm_steps(o);
 }
 
 size_t orc_payload_bytes(const orc_state *o, int warmup)
@@ -258,7 +280,7 @@ orc_state *orc_create(int64_t rows, int64_t cols, int mode, int dtype, int ef, i
                       int rank, int iters, int lr_int4, int batch, uint64_t seed)
 {
     if (rows < 1 || cols < 1 || batch < 1) return NULL;
-    if (mode < ORC_IDENTITY || mode > ORC_LOWRANK) return NULL;
+    if (mode < ORC_IDENTITY || mode > ORC_BLOCKSEL) return NULL;
     if (dtype != ORC_F32 && dtype != ORC_BF16) return NULL;
     if (ef != ORC_EF_EXPLICIT && ef != ORC_EF_IMPLICIT && ef != ORC_EF_OFF) return NULL;
     if (cols % 8) return NULL;
@@ -286,7 +308,7 @@ orc_state *orc_create(int64_t rows, int64_t cols, int mode, int dtype, int ef, i
 void orc_destroy(orc_state *o)
 {
     if (!o) return;
-    free(o->ahat_s); free(o->err); free(o->ahat_r); free(o->vprev);
+    free(o->ahat_s); free(o->err); free(o->ahat_r); free(o->vprev); free(o->bs_sent);
     free(o);
 }
 
@@ -306,6 +328,26 @@ float *orc_buffer(orc_state *o, int which)
 }
 
 void orc_set_vprev_valid(orc_state *o, int v) { o->vprev_valid = v; }
+
+/* BLOCKSEL configuration (required before the first step): token grid
+ * h x (rows / h), block side b, k blocks per step, `warm` leading steps sent
+ * in full.  Returns 0, or -1 if the grid is not cut evenly into blocks, k is
+ * out of range or the state is not a single-tensor BLOCKSEL state. */
+int orc_set_blocksel(orc_state *o, int h, int b, int k, int warm)
+{
+    if (o->mode != ORC_BLOCKSEL || o->batch != 1) return -1;
+    if (h < 1 || b < 1 || warm < 1 || o->rows % h) return -1;
+    int w = (int)(o->rows / h);
+    if (h % b || w % b) return -1;
+    int K = (h / b) * (w / b);
+    if (k < 1 || k > K) return -1;
+    o->bs_h = h; o->bs_w = w; o->bs_b = b; o->bs_k = k; o->bs_warm = warm; o->bs_K = K;
+    free(o->bs_sent);
+    o->bs_sent = (uint8_t *)calloc((size_t)K, 1);
+    return 0;
+}
+
+uint8_t *orc_blocksel_sent(orc_state *o) { return o->bs_sent; }
 void orc_set_step(orc_state *o, uint64_t s_send, uint64_t s_recv) { o->step_s = s_send; o->step_r = s_recv; }
 
 static float load_act(const void *a, int dtype, int64_t i)
@@ -326,7 +368,8 @@ static void write_u64(uint8_t *p, uint64_t v) { memcpy(p, &v, 8); }
 /* 64-byte payload header (little-endian):
  *   0 magic | 4 mode | 8 flags (bit0 warm-up) | 12 dtype | 16 step (u64)
  *  24 rows (u64) | 32 cols (u64) | 40 batch | 44 p0 | 48 p1 | 52 ef | 56 p2 | 60 zero
- *  p0/p1/p2: NM -> N, M, 0; LOWRANK -> rank, int4 flag, iterations; else 0. */
+ *  p0/p1/p2: NM -> N, M, 0; LOWRANK -> rank, int4 flag, iterations;
+ *  BLOCKSEL -> grid height, block side, blocks per step; else 0. */
 static void write_header(const orc_state *o, uint8_t *p, int warm, uint64_t step)
 {
     memset(p, 0, ORC_HDR);
@@ -341,6 +384,7 @@ static void write_header(const orc_state *o, uint8_t *p, int warm, uint64_t step
     uint32_t p0 = 0, p1 = 0, p2 = 0;
     if (o->mode == ORC_NM) { p0 = (uint32_t)o->nm_n; p1 = (uint32_t)o->nm_m; }
     if (o->mode == ORC_LOWRANK) { p0 = (uint32_t)o->rank; p1 = (uint32_t)o->lr_int4; p2 = (uint32_t)o->iters; }
+    if (o->mode == ORC_BLOCKSEL) { p0 = (uint32_t)o->bs_h; p1 = (uint32_t)o->bs_b; p2 = (uint32_t)o->bs_k; }
     write_u32(p + 44, p0);
     write_u32(p + 48, p1);
     write_u32(p + 52, (uint32_t)o->ef);
@@ -651,10 +695,134 @@ static void lowrank_encode(orc_state *o, const float *d, float *vprev, uint8_t *
 
 /* Sender step: a = [batch][rows][cols] in the state's dtype; payload gets
  * orc_payload_bytes(o, step==0) bytes.  Returns 0. */
+/* ------------------------------------------------------------------ */
+/* block selection                                                     */
+/* ------------------------------------------------------------------ */
+
+#define ORC_BS_NONE 0xffffffffu /* index of an unused payload slot */
+
+/* token (row) index of element (y, x) of block i */
+static int64_t bs_token(const orc_state *o, int i, int y, int x)
+{
+    int nbx = o->bs_w / o->bs_b;
+    int by = i / nbx, bx = i % nbx;
+    return (int64_t)(by * o->bs_b + y) * o->bs_w + bx * o->bs_b + x;
+}
+
+/* Cosine dissimilarity of block i between the previous activation p and the
+ * current one a ("Informative sub-block selection"): d = 1 - <p, a>_F /
+ * (||p||_F ||a||_F), the Frobenius sums over the block's tokens in raster
+ * order and all channels, in fp64 (each product of two fp32 values is exact).
+ * Readings for the cases the formula leaves open: a block whose values are
+ * all unchanged has d = 0; a block with exactly one zero norm has d = 1. */
+static double bs_dissimilarity(const orc_state *o, int i, const float *p, const float *a)
+{
+    double dot = 0.0, np_ = 0.0, na = 0.0;
+    int changed = 0;
+    for (int y = 0; y < o->bs_b; y++)
+        for (int x = 0; x < o->bs_b; x++) {
+            int64_t t = bs_token(o, i, y, x);
+            for (int64_t c = 0; c < o->cols; c++) {
+                double u = p[t * o->cols + c], v = a[t * o->cols + c];
+                if (u != v) changed = 1;
+                dot += u * v;
+                np_ += u * u;
+                na += v * v;
+            }
+        }
+    if (!changed) return 0.0;
+    if (np_ == 0.0 || na == 0.0) return 1.0;
+    return 1.0 - dot / (sqrt(np_) * sqrt(na));
+}
+
+typedef struct { double d; int i; } bs_cand;
+
+/* larger dissimilarity first; on equal dissimilarity the lower block index */
+static int bs_cmp(const void *x, const void *y)
+{
+    const bs_cand *a = (const bs_cand *)x, *b = (const bs_cand *)y;
+    if (a->d > b->d) return -1;
+    if (a->d < b->d) return 1;
+    return (a->i > b->i) - (a->i < b->i);
+}
+
+static int bs_cmp_index(const void *x, const void *y)
+{
+    int a = *(const int *)x, b = *(const int *)y;
+    return (a > b) - (a < b);
+}
+
+/* One selective step: the top-k of the unsent blocks ("Dynamic round-robin":
+ * selection only from the blocks not yet sent this round; when every block
+ * has been sent the round restarts), their raw values in ascending block
+ * order, unused slots (the last step of a round may have fewer than k
+ * blocks left) marked ORC_BS_NONE and zero.  The sender's state becomes
+ * fp32(a_t). */
+static void blocksel_encode(orc_state *o, const void *a, uint8_t *body)
+{
+    int K = o->bs_K, k = o->bs_k, b = o->bs_b;
+    int64_t E = elems(o);
+    float *cur = (float *)malloc(sizeof(float) * (size_t)E);
+    for (int64_t i = 0; i < E; i++) cur[i] = load_act(a, o->dtype, i);
+    bs_cand *cand = (bs_cand *)malloc(sizeof(bs_cand) * (size_t)K);
+    int nc = 0;
+    for (int i = 0; i < K; i++)
+        if (!o->bs_sent[i]) {
+            cand[nc].d = bs_dissimilarity(o, i, o->ahat_s, cur);
+            cand[nc].i = i;
+            nc++;
+        }
+    qsort(cand, (size_t)nc, sizeof(bs_cand), bs_cmp);
+    int m = nc < k ? nc : k;
+    int *sel = (int *)malloc(sizeof(int) * (size_t)(m > 0 ? m : 1));
+    for (int j = 0; j < m; j++) sel[j] = cand[j].i;
+    qsort(sel, (size_t)m, sizeof(int), bs_cmp_index);
+    size_t asz = act_size(o->dtype);
+    size_t blk = (size_t)b * b * (size_t)o->cols * asz;
+    uint8_t *data = body + pad16((size_t)k * 4u);
+    memset(body, 0, orc_tensor_body_bytes(o));
+    for (int j = 0; j < k; j++) write_u32(body + 4 * j, j < m ? (uint32_t)sel[j] : ORC_BS_NONE);
+    for (int j = 0; j < m; j++)
+        for (int y = 0; y < b; y++)
+            for (int x = 0; x < b; x++) {
+                int64_t t = bs_token(o, sel[j], y, x);
+                memcpy(data + (size_t)j * blk + ((size_t)y * b + x) * (size_t)o->cols * asz,
+                       (const uint8_t *)a + (size_t)t * (size_t)o->cols * asz, (size_t)o->cols * asz);
+            }
+    for (int j = 0; j < m; j++) o->bs_sent[sel[j]] = 1;
+    int all = 1;
+    for (int i = 0; i < K; i++) all &= o->bs_sent[i];
+    if (all) memset(o->bs_sent, 0, (size_t)K);
+    memcpy(o->ahat_s, cur, sizeof(float) * (size_t)E);
+    free(cur); free(cand); free(sel);
+}
+
+/* Receiver side: the sent blocks replace the receiver's values; every other
+ * block keeps the value it last received. */
+static void blocksel_decode(orc_state *o, const uint8_t *body)
+{
+    int K = o->bs_K, k = o->bs_k, b = o->bs_b;
+    size_t asz = act_size(o->dtype);
+    size_t blk = (size_t)b * b * (size_t)o->cols * asz;
+    const uint8_t *data = body + pad16((size_t)k * 4u);
+    for (int j = 0; j < k; j++) {
+        uint32_t i;
+        memcpy(&i, body + 4 * j, 4);
+        if (i == ORC_BS_NONE || i >= (uint32_t)K) continue;
+        for (int y = 0; y < b; y++)
+            for (int x = 0; x < b; x++) {
+                int64_t t = bs_token(o, (int)i, y, x);
+                const uint8_t *src = data + (size_t)j * blk + ((size_t)y * b + x) * (size_t)o->cols * asz;
+                for (int64_t c = 0; c < o->cols; c++) o->ahat_r[t * o->cols + c] = load_act(src, o->dtype, c);
+            }
+    }
+}
+
 int orc_encode(orc_state *o, const void *a, uint8_t *payload)
 {
     int64_t E = elems(o);
-    int warm = o->step_s == 0;
+    int warm = o->step_s < warm_steps(o);
+    if (o->mode == ORC_BLOCKSEL && !o->bs_sent) return -1;
     write_header(o, payload, warm, o->step_s);
     uint8_t *body0 = payload + ORC_HDR;
     if (warm) {
@@ -672,6 +840,11 @@ int orc_encode(orc_state *o, const void *a, uint8_t *payload)
         return 0;
     }
     size_t tb = orc_tensor_body_bytes(o);
+    if (o->mode == ORC_BLOCKSEL) {
+        blocksel_encode(o, a, body0);
+        o->step_s++;
+        return 0;
+    }
     float *d = (float *)malloc(sizeof(float) * (size_t)E);
     float *C = (float *)malloc(sizeof(float) * (size_t)E);
     for (int b = 0; b < o->batch; b++) {
@@ -714,7 +887,8 @@ int orc_encode(orc_state *o, const void *a, uint8_t *payload)
 int orc_decode(orc_state *o, const uint8_t *payload, void *recon)
 {
     int64_t E = elems(o);
-    int warm = o->step_r == 0;
+    int warm = o->step_r < warm_steps(o);
+    if (o->mode == ORC_BLOCKSEL && !o->bs_sent) return -1;
     if (!check_header(o, payload, warm, o->step_r)) {
         o->status = 1;
         o->step_r++;
@@ -733,6 +907,12 @@ int orc_decode(orc_state *o, const uint8_t *payload, void *recon)
         return 0;
     }
     size_t tb = orc_tensor_body_bytes(o);
+    if (o->mode == ORC_BLOCKSEL) {
+        blocksel_decode(o, body0);
+        for (int64_t i = 0; i < E; i++) store_act(recon, o->dtype, i, o->ahat_r[i]);
+        o->step_r++;
+        return 0;
+    }
     float *C = (float *)malloc(sizeof(float) * (size_t)E);
     for (int b = 0; b < o->batch; b++) {
         const uint8_t *body = body0 + tb * b;
@@ -762,6 +942,7 @@ int orc_decode(orc_state *o, const uint8_t *payload, void *recon)
  * without touching any state: used by tests that compare payload meaning. */
 int orc_payload_meaning(const orc_state *o, const uint8_t *payload, int b, float *C)
 {
+    if (o->mode == ORC_BLOCKSEL) return -1; /* a selection carries values, not a residual */
     const uint8_t *body = payload + ORC_HDR + orc_tensor_body_bytes(o) * (size_t)b;
     if (o->mode == ORC_LOWRANK) {
         int r = o->rank;
@@ -801,6 +982,15 @@ void orc_subspace_iteration(const float *D, int64_t m, int64_t n, int r, int ite
             }
     }
     free(Y); free(rd); free(dead);
+}
+
+/* BLOCKSEL pin helper: the dissimilarity of every block between two caller
+ * activations p and a (fp32 [rows][cols]) into d[K]. */
+int orc_blocksel_dissimilarity(const orc_state *o, const float *p, const float *a, double *d)
+{
+    if (o->mode != ORC_BLOCKSEL || !o->bs_sent) return -1;
+    for (int i = 0; i < o->bs_K; i++) d[i] = bs_dissimilarity(o, i, p, a);
+    return 0;
 }
 
 /* Array helpers for the tests (elementwise, no arithmetic of their own). */
