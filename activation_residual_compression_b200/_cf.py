@@ -28,13 +28,14 @@ CF_ERR_SIZE = -10
 CF_ERR_TIMEOUT = -11
 CF_ERR_TOO_LARGE = -12
 
-CF_IDENTITY, CF_SIGN1, CF_Q2, CF_NM, CF_LOWRANK = 0, 1, 2, 3, 4
+CF_IDENTITY, CF_SIGN1, CF_Q2, CF_NM, CF_LOWRANK, CF_BLOCKSEL = 0, 1, 2, 3, 4, 5
 CF_F32, CF_BF16 = 0, 1
 CF_SENDER, CF_RECEIVER = 0, 1
 CF_EF_EXPLICIT, CF_EF_IMPLICIT, CF_EF_OFF = 0, 1, 2
 CF_T_RECON, CF_T_ERROR, CF_T_VPREV = 0, 1, 2
 
-MODE_NAMES = {"identity": CF_IDENTITY, "sign1": CF_SIGN1, "q2": CF_Q2, "nm": CF_NM, "lowrank": CF_LOWRANK}
+MODE_NAMES = {"identity": CF_IDENTITY, "sign1": CF_SIGN1, "q2": CF_Q2, "nm": CF_NM, "lowrank": CF_LOWRANK,
+              "blocksel": CF_BLOCKSEL}
 
 
 class cf_params(ctypes.Structure):
@@ -51,6 +52,10 @@ class cf_params(ctypes.Structure):
         ("seed", ctypes.c_uint64),
         ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
+        ("bs_grid_h", ctypes.c_int),
+        ("bs_block", ctypes.c_int),
+        ("bs_k", ctypes.c_int),
+        ("bs_warm", ctypes.c_int),
     ]
 
 

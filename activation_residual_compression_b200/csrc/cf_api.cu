@@ -13,6 +13,7 @@
 #include <unordered_set>
 
 #include "cf.h"
+#include "cf_blocksel.h"
 #include "cf_internal.h"
 #include "cf_lowrank.h"
 
@@ -37,6 +38,7 @@ struct cf_state {
   StreamCfg cfg{};
   Layout lay{};
   LowrankPlan lr{};
+  BlockselPlan bs{};
 };
 
 namespace {
@@ -60,6 +62,10 @@ int ilog2(int m) {
 
 size_t act_size(int dtype) { return dtype == CF_BF16 ? 2u : 4u; }
 
+int bs_plan_of(int64_t rows, int64_t cols, const cf_params &p, BlockselPlan *P) {
+  return blocksel_plan(rows, cols, p.dtype, p.batch, p.bs_grid_h, p.bs_block, p.bs_k, p.bs_warm, P);
+}
+
 Layout layout_of(int64_t rows, int64_t cols, int mode, const cf_params &p) {
   Layout L{};
   switch (mode) {
@@ -81,6 +87,14 @@ Layout layout_of(int64_t rows, int64_t cols, int mode, const cf_params &p) {
       L.body = L.sec1 + pad16((size_t)(rows * words) * 4u);
       break;
     }
+    case CF_BLOCKSEL: {
+      BlockselPlan bp{};
+      if (bs_plan_of(rows, cols, p, &bp) == CF_OK) {
+        L.sec1 = pad16((size_t)bp.k * 4u);
+        L.body = blocksel_body_bytes(bp);
+      }
+      break;
+    }
     case CF_LOWRANK:
       if (p.lr_int4) {
         L.sec1 = pad16((size_t)p.rank * 8u);
@@ -98,7 +112,7 @@ Layout layout_of(int64_t rows, int64_t cols, int mode, const cf_params &p) {
 
 int validate(int64_t rows, int64_t cols, int mode, const cf_params *p) {
   if (!p) return CF_ERR_ARG;
-  if (mode < CF_IDENTITY || mode > CF_LOWRANK) return CF_ERR_ARG;
+  if (mode < CF_IDENTITY || mode > CF_BLOCKSEL) return CF_ERR_ARG;
   if (p->dtype != CF_F32 && p->dtype != CF_BF16) return CF_ERR_ARG;
   if (p->role != CF_SENDER && p->role != CF_RECEIVER) return CF_ERR_ARG;
   if (p->ef != CF_EF_EXPLICIT && p->ef != CF_EF_IMPLICIT && p->ef != CF_EF_OFF) return CF_ERR_ARG;
@@ -114,6 +128,11 @@ int validate(int64_t rows, int64_t cols, int mode, const cf_params *p) {
     if (cols % p->nm_m) return CF_ERR_SHAPE;
     if (((cols / p->nm_m) * p->nm_n * ilog2(p->nm_m)) % 32) return CF_ERR_SHAPE;
   }
+  if (mode == CF_BLOCKSEL) {
+    BlockselPlan bp{};
+    const int rc = bs_plan_of(rows, cols, *p, &bp);
+    if (rc != CF_OK) return rc;
+  }
   if (mode == CF_LOWRANK) {
     if (p->rank < 1 || p->rank > kMaxRank || p->rank > rows || p->rank > cols) return CF_ERR_SHAPE;
     if (rows % 128 || cols % 128) return CF_ERR_SHAPE;
@@ -128,10 +147,11 @@ int validate(int64_t rows, int64_t cols, int mode, const cf_params *p) {
 }
 
 struct Carve {
-  size_t status, ahat, err, vprev, lr, total;
+  size_t status, ahat, err, vprev, lr, bs, total;
 };
 
-Carve carve_of(int64_t rows, int64_t cols, int mode, const cf_params &p, const LowrankPlan &lr) {
+Carve carve_of(int64_t rows, int64_t cols, int mode, const cf_params &p, const LowrankPlan &lr,
+               const BlockselPlan &bs) {
   Carve c{};
   const size_t E = (size_t)(rows * cols) * (size_t)p.batch;
   size_t off = 0;
@@ -139,7 +159,7 @@ Carve carve_of(int64_t rows, int64_t cols, int mode, const cf_params &p, const L
   off += 256;
   c.ahat = off;
   off += pad256(E * 4u);
-  if (p.role == CF_SENDER) {
+  if (p.role == CF_SENDER && mode != CF_BLOCKSEL) {  // block selection keeps no error term
     c.err = off;
     off += pad256(E * 4u);
     if (mode == CF_LOWRANK) {
@@ -150,6 +170,10 @@ Carve carve_of(int64_t rows, int64_t cols, int mode, const cf_params &p, const L
   if (mode == CF_LOWRANK) {
     c.lr = off;
     off += pad256(p.role == CF_SENDER ? lr.enc_scratch_bytes : lr.dec_scratch_bytes);
+  }
+  if (mode == CF_BLOCKSEL && p.role == CF_SENDER) {
+    c.bs = off;
+    off += pad256(blocksel_scratch_bytes(bs));
   }
   c.total = off;
   return c;
@@ -171,6 +195,7 @@ Header header_of(const cf_state *s, bool warm, uint64_t step) {
   uint32_t p0 = 0, p1 = 0, p2 = 0;
   if (s->mode == CF_NM) { p0 = (uint32_t)s->p.nm_n; p1 = (uint32_t)s->p.nm_m; }
   if (s->mode == CF_LOWRANK) { p0 = (uint32_t)s->p.rank; p1 = (uint32_t)s->p.lr_int4; p2 = (uint32_t)s->p.iters; }
+  if (s->mode == CF_BLOCKSEL) { p0 = (uint32_t)s->bs.H; p1 = (uint32_t)s->bs.b; p2 = (uint32_t)s->bs.k; }
   h.w[11] = p0;
   h.w[12] = p1;
   h.w[13] = (uint32_t)s->p.ef;
@@ -188,6 +213,9 @@ int cuda_err(cudaError_t e) {
 }
 
 size_t warm_body(const cf_state *s) { return pad16((size_t)(s->rows * s->cols) * act_size(s->p.dtype)); }
+
+// leading steps sent in full (block selection: bs_warm; every other mode: 1)
+uint64_t warm_steps(const cf_state *s) { return s->mode == CF_BLOCKSEL ? (uint64_t)s->bs.warm : 1u; }
 
 EncArgs enc_args(cf_state *s, const void *a, void *payload, bool warm) {
   EncArgs A{};
@@ -253,11 +281,14 @@ int do_encode(cf_state *s, const void *a, const PtrTable *tab, void *payload, cu
   if (!aligned16(payload) || (a && !aligned16(a))) return CF_ERR_ALIGN;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != s->device) return CF_ERR_ARG;
-  const bool warm = s->step == 0;
+  const bool warm = s->step < warm_steps(s);
+  if (s->mode == CF_BLOCKSEL && tab) return CF_ERR_UNSUPPORTED;
   EncArgs A = enc_args(s, a, payload, warm);
   cudaError_t e;
   if (warm) {
     e = launch_warm_encode(s->p.dtype, s->cfg, A, tab, st);
+  } else if (s->mode == CF_BLOCKSEL) {
+    e = blocksel_encode(s->bs, a, s->ahat, static_cast<uint8_t *>(payload), A.hdr, st);
   } else if (s->mode == CF_LOWRANK) {
     e = lowrank_encode(s->lr, A, tab, s->vprev, s->step, s->p.seed, st);
   } else {
@@ -275,11 +306,14 @@ int do_decode(cf_state *s, const void *payload, void *recon, const PtrTable *tab
   if (!aligned16(payload) || (recon && !aligned16(recon))) return CF_ERR_ALIGN;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != s->device) return CF_ERR_ARG;
-  const bool warm = s->step == 0;
+  const bool warm = s->step < warm_steps(s);
+  if (s->mode == CF_BLOCKSEL && tab) return CF_ERR_UNSUPPORTED;
   DecArgs A = dec_args(s, payload, recon, warm);
   cudaError_t e;
   if (warm) {
     e = launch_warm_decode(s->p.dtype, s->cfg, A, tab, st);
+  } else if (s->mode == CF_BLOCKSEL) {
+    e = blocksel_decode(s->bs, static_cast<const uint8_t *>(payload), s->ahat, recon, A.expect, s->status, st);
   } else if (s->mode == CF_LOWRANK) {
     e = lowrank_decode(s->lr, A, tab, st);
   } else {
@@ -352,6 +386,10 @@ int cf_params_init(cf_params *p) {
   p->lr_int4 = 1;
   p->batch = 1;
   p->seed = 0;
+  p->bs_grid_h = 0;
+  p->bs_block = 8;
+  p->bs_k = 0;
+  p->bs_warm = 5;
   return CF_OK;
 }
 
@@ -360,8 +398,10 @@ int cf_workspace_bytes(int64_t rows, int64_t cols, int mode, const cf_params *p,
   const int v = validate(rows, cols, mode, p);
   if (v != CF_OK) return v;
   LowrankPlan lr{};
+  BlockselPlan bs{};
   if (mode == CF_LOWRANK) lowrank_plan(rows, cols, *p, &lr);
-  *out = carve_of(rows, cols, mode, *p, lr).total;
+  if (mode == CF_BLOCKSEL) bs_plan_of(rows, cols, *p, &bs);
+  *out = carve_of(rows, cols, mode, *p, lr, bs).total;
   return CF_OK;
 }
 
@@ -383,6 +423,7 @@ int cf_create(int64_t rows, int64_t cols, int mode, const cf_params *p, cf_state
     return CF_ERR_CUDA;
   }
   if (mode == CF_LOWRANK) lowrank_plan(rows, cols, *p, &s->lr);
+  if (mode == CF_BLOCKSEL) bs_plan_of(rows, cols, *p, &s->bs);
   s->lay = layout_of(rows, cols, mode, *p);
   const int rc = stream_config(mode, p->dtype, p->nm_m, p->nm_n, rows, cols, p->batch, s->sm_count,
                                p->ef == CF_EF_EXPLICIT, &s->cfg);
@@ -390,7 +431,7 @@ int cf_create(int64_t rows, int64_t cols, int mode, const cf_params *p, cf_state
     delete s;
     return rc;
   }
-  const Carve c = carve_of(rows, cols, mode, *p, s->lr);
+  const Carve c = carve_of(rows, cols, mode, *p, s->lr, s->bs);
   if (p->workspace) {
     if (p->workspace_bytes < c.total || ((uintptr_t)p->workspace & 255u)) {
       delete s;
@@ -410,9 +451,17 @@ int cf_create(int64_t rows, int64_t cols, int mode, const cf_params *p, cf_state
   uint8_t *base = static_cast<uint8_t *>(s->slab);
   s->status = reinterpret_cast<int *>(base + c.status);
   s->ahat = reinterpret_cast<float *>(base + c.ahat);
-  s->err = p->role == CF_SENDER ? reinterpret_cast<float *>(base + c.err) : nullptr;
+  s->err = (p->role == CF_SENDER && mode != CF_BLOCKSEL) ? reinterpret_cast<float *>(base + c.err) : nullptr;
   s->vprev = (p->role == CF_SENDER && mode == CF_LOWRANK) ? reinterpret_cast<float *>(base + c.vprev) : nullptr;
   s->lr_scratch = mode == CF_LOWRANK ? static_cast<void *>(base + c.lr) : nullptr;
+  if (mode == CF_BLOCKSEL && p->role == CF_SENDER) {
+    const int rc2 = blocksel_bind(&s->bs, base + c.bs);
+    if (rc2 != CF_OK) {
+      if (s->own_slab) cudaFree(s->slab);
+      delete s;
+      return rc2;
+    }
+  }
   if (mode == CF_LOWRANK) {
     const int rc2 = lowrank_bind(&s->lr, s->lr_scratch);
     if (rc2 != CF_OK) {
@@ -525,6 +574,7 @@ static size_t export_tensor_bytes(const cf_state *s) {
   size_t b = E * 4u;
   if (s->err) b += E * 4u;
   if (s->vprev) b += (size_t)s->cols * s->p.rank * 4u * s->p.batch;
+  if (s->bs.sent) b += (size_t)s->bs.K;
   return b;
 }
 
@@ -561,7 +611,11 @@ int cf_state_export(const cf_state *s, void *host, size_t bytes, void *stream) {
   if (s->vprev) {
     const size_t vb = (size_t)s->cols * s->p.rank * 4u * s->p.batch;
     if (cudaMemcpy(dst, s->vprev, vb, cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_err(cudaErrorUnknown);
+    dst += vb;
   }
+  if (s->bs.sent &&
+      cudaMemcpy(dst, s->bs.sent, (size_t)s->bs.K, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return cuda_err(cudaErrorUnknown);
   return CF_OK;
 }
 
@@ -589,7 +643,11 @@ int cf_state_import(cf_state *s, const void *host, size_t bytes, void *stream) {
   if (s->vprev) {
     const size_t vb = (size_t)s->cols * s->p.rank * 4u * s->p.batch;
     if (cudaMemcpy(s->vprev, src, vb, cudaMemcpyHostToDevice) != cudaSuccess) return cuda_err(cudaErrorUnknown);
+    src += vb;
   }
+  if (s->bs.sent &&
+      cudaMemcpy(s->bs.sent, src, (size_t)s->bs.K, cudaMemcpyHostToDevice) != cudaSuccess)
+    return cuda_err(cudaErrorUnknown);
   if (cudaMemcpy(s->status, &h.status, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return cuda_err(cudaErrorUnknown);
   s->step = h.step;
   return CF_OK;

@@ -1,0 +1,443 @@
+// cf_blocksel.cu -- kernels of the block-selection mode (Otil page:
+// "Informative sub-block selection", "Dynamic round-robin").
+//
+// Encode = three launches on the caller's stream:
+//   bs_partial_kernel  one CTA per (block, token row of the block): the fp64
+//                      Frobenius sums <p, a>, ||p||^2, ||a||^2 and a changed
+//                      flag over the row's b tokens x all channels, and the
+//                      state update p = fp32(a) (the row is read once);
+//   bs_select_kernel   one CTA: d per block from the partials (fixed order),
+//                      bitonic sort of the unsent blocks by (d desc, index
+//                      asc), the first min(k, unsent) blocks in ascending
+//                      order, the round-robin flags, the payload header and
+//                      index section;
+//   bs_pack_kernel     one CTA per (slot, token row): raw block rows into the
+//                      payload (unused slots zeroed).
+// Decode = one launch: bs_decode_kernel, one CTA per (block, token row): the
+// row comes from the payload when its block was sent, else from ahat; ahat
+// and recon are written.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "cf.h"
+#include "cf_blocksel.h"
+#include "cf_launch.cuh"
+
+namespace cfi {
+namespace {
+
+constexpr int kBsThreads = 256;
+constexpr int kSelThreads = 1024;
+
+size_t pad16(size_t x) { return (x + 15u) & ~(size_t)15u; }
+size_t pad256(size_t x) { return (x + 255u) & ~(size_t)255u; }
+
+// 8 consecutive activations as fp32, and their raw bits
+template <typename T>
+struct Vec8;
+template <>
+struct Vec8<__nv_bfloat16> {
+  using Raw = uint4;
+  static __device__ __forceinline__ Raw load(const __nv_bfloat16 *p) { return *reinterpret_cast<const uint4 *>(p); }
+  static __device__ __forceinline__ void store(__nv_bfloat16 *p, const Raw &r) { *reinterpret_cast<uint4 *>(p) = r; }
+  static __device__ __forceinline__ void to_f32(const Raw &r, float (&x)[8]) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  // fp32 values that are bf16 numbers (received raw values): exact conversion
+  static __device__ __forceinline__ Raw from_f32(const float (&x)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++)
+      w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[2 * i])) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[2 * i + 1])) << 16);
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+template <>
+struct Vec8<float> {
+  struct Raw {
+    float4 a, b;
+  };
+  static __device__ __forceinline__ Raw load(const float *p) {
+    return Raw{reinterpret_cast<const float4 *>(p)[0], reinterpret_cast<const float4 *>(p)[1]};
+  }
+  static __device__ __forceinline__ void store(float *p, const Raw &r) {
+    reinterpret_cast<float4 *>(p)[0] = r.a;
+    reinterpret_cast<float4 *>(p)[1] = r.b;
+  }
+  static __device__ __forceinline__ void to_f32(const Raw &r, float (&x)[8]) {
+    x[0] = r.a.x; x[1] = r.a.y; x[2] = r.a.z; x[3] = r.a.w;
+    x[4] = r.b.x; x[5] = r.b.y; x[6] = r.b.z; x[7] = r.b.w;
+  }
+  static __device__ __forceinline__ Raw from_f32(const float (&x)[8]) {
+    return Raw{make_float4(x[0], x[1], x[2], x[3]), make_float4(x[4], x[5], x[6], x[7])};
+  }
+};
+
+__device__ __forceinline__ void load_f32x8(const float *p, float (&x)[8]) {
+  const float4 u = reinterpret_cast<const float4 *>(p)[0], v = reinterpret_cast<const float4 *>(p)[1];
+  x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+  x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+}
+__device__ __forceinline__ void store_f32x8(float *p, const float (&x)[8]) {
+  reinterpret_cast<float4 *>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
+  reinterpret_cast<float4 *>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
+}
+
+// first token of row y of block i (the row's b tokens are consecutive)
+__device__ __forceinline__ int64_t block_row_token(int i, int y, int W, int b) {
+  const int nbx = W / b;
+  const int by = i / nbx, bx = i - by * nbx;
+  return (int64_t)(by * b + y) * W + (int64_t)bx * b;
+}
+
+// ------------------------------------------------------------------ encode
+
+// Sums over one token row of one block, state update fused.  Each product of
+// two fp32 values is exact in fp64, so each fused multiply-add rounds once;
+// the CTA adds its threads' sums in a fixed order (deterministic).
+template <typename T>
+__global__ void __launch_bounds__(kBsThreads) bs_partial_kernel(const T *a, float *prev, int W, int b,
+                                                                 int64_t cols, double *part) {
+  pdl_enter();
+  const int i = blockIdx.x / b, y = blockIdx.x - (blockIdx.x / b) * b;
+  const int64_t e0 = block_row_token(i, y, W, b) * cols;
+  const int64_t n8 = (int64_t)b * cols / 8;
+  double dot = 0.0, np_ = 0.0, na = 0.0;
+  int changed = 0;
+  for (int64_t v = threadIdx.x; v < n8; v += kBsThreads) {
+    const int64_t e = e0 + v * 8;
+    float x[8], p[8];
+    Vec8<T>::to_f32(Vec8<T>::load(a + e), x);
+    load_f32x8(prev + e, p);
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      changed |= p[k] != x[k];
+      dot = fma((double)p[k], (double)x[k], dot);
+      np_ = fma((double)p[k], (double)p[k], np_);
+      na = fma((double)x[k], (double)x[k], na);
+    }
+    store_f32x8(prev + e, x);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    np_ += __shfl_xor_sync(0xffffffffu, np_, o);
+    na += __shfl_xor_sync(0xffffffffu, na, o);
+    changed |= __shfl_xor_sync(0xffffffffu, changed, o);
+  }
+  __shared__ double ws[kBsThreads / 32][4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    ws[warp][0] = dot;
+    ws[warp][1] = np_;
+    ws[warp][2] = na;
+    ws[warp][3] = changed ? 1.0 : 0.0;
+  }
+  __syncthreads();
+  if (threadIdx.x < 4) {
+    double s = ws[0][threadIdx.x];
+    for (int w = 1; w < kBsThreads / 32; w++)
+      s = threadIdx.x == 3 ? fmax(s, ws[w][3]) : s + ws[w][threadIdx.x];
+    part[(int64_t)blockIdx.x * 4 + threadIdx.x] = s;
+  }
+}
+
+// Order-preserving key of a double (larger d -> larger key); 0 marks "not a
+// candidate" (no finite d maps to it).
+__device__ __forceinline__ unsigned long long sort_key(double d) {
+  const unsigned long long u = (unsigned long long)__double_as_longlong(d);
+  return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+// entry x goes before entry y: larger dissimilarity, then lower block index
+__device__ __forceinline__ bool before(unsigned long long kx, int ix, unsigned long long ky, int iy) {
+  return kx > ky || (kx == ky && ix < iy);
+}
+
+__global__ void __launch_bounds__(kSelThreads) bs_select_kernel(const double *part, int K, int K2, int b, int k,
+                                                                 uint8_t *sent, uint32_t *sel, uint8_t *payload,
+                                                                 const Header hdr) {
+  pdl_enter();
+  extern __shared__ __align__(16) uint8_t smem[];
+  unsigned long long *key = reinterpret_cast<unsigned long long *>(smem);  // [K2]
+  int *idx = reinterpret_cast<int *>(key + K2);                           // [K2]
+  uint8_t *pick = reinterpret_cast<uint8_t *>(idx + K2);                  // [K2]
+  __shared__ int wsum[kSelThreads / 32];
+  const int tid = threadIdx.x;
+  // dissimilarities of the unsent blocks
+  int mine = 0;
+  for (int i = tid; i < K2; i += kSelThreads) {
+    unsigned long long kk = 0ull;
+    if (i < K && !sent[i]) {
+      double dot = 0.0, np_ = 0.0, na = 0.0, ch = 0.0;
+      for (int y = 0; y < b; y++) {
+        const double *q = part + ((int64_t)i * b + y) * 4;
+        dot += q[0];
+        np_ += q[1];
+        na += q[2];
+        ch = fmax(ch, q[3]);
+      }
+      double d;
+      if (ch == 0.0) d = 0.0;                       // every value unchanged
+      else if (np_ == 0.0 || na == 0.0) d = 1.0;    // exactly one zero norm
+      else d = 1.0 - dot / (sqrt(np_) * sqrt(na));
+      kk = sort_key(d);
+      mine++;
+    }
+    key[i] = kk;
+    idx[i] = i;
+    pick[i] = 0;
+  }
+  (void)mine;
+  // bitonic sort of K2 (a power of two) entries into "before" order
+  for (int size = 2; size <= K2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      __syncthreads();
+      for (int i = tid; i < K2; i += kSelThreads) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const bool jfirst = before(key[j], idx[j], key[i], idx[i]);
+          const bool ifirst = before(key[i], idx[i], key[j], idx[j]);
+          if (up ? jfirst : ifirst) {
+            const unsigned long long tk = key[i];
+            key[i] = key[j];
+            key[j] = tk;
+            const int ti = idx[i];
+            idx[i] = idx[j];
+            idx[j] = ti;
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // candidates sort first (key > 0); the first min(k, candidates) are picked
+  for (int r = tid; r < K2; r += kSelThreads)
+    if (r < k && key[r] != 0ull) pick[idx[r]] = 1;
+  __syncthreads();
+  // ascending list of the picked blocks: each thread owns a contiguous chunk
+  const int chunk = (K2 + kSelThreads - 1) / kSelThreads;
+  const int c0 = tid * chunk;
+  int cnt = 0;
+  for (int i = c0; i < c0 + chunk && i < K2; i++) cnt += pick[i];
+  // exclusive scan of cnt over the CTA
+  const int lane = tid & 31, warp = tid >> 5;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < warp; w++) base += wsum[w];
+  int m = 0;
+  for (int w = 0; w < kSelThreads / 32; w++) m += wsum[w];
+  int pos = base + incl - cnt;
+  uint32_t *slots = reinterpret_cast<uint32_t *>(payload + kHdrBytes);
+  for (int i = c0; i < c0 + chunk && i < K2; i++)
+    if (pick[i]) {
+      sel[pos] = (uint32_t)i;
+      slots[pos] = (uint32_t)i;
+      pos++;
+    }
+  for (int j = m + tid; j < k; j += kSelThreads) {
+    sel[j] = kBsNone;
+    slots[j] = kBsNone;
+  }
+  // index-section padding
+  for (int bb = 4 * k + tid; bb < (int)((4 * k + 15) & ~15); bb += kSelThreads) payload[kHdrBytes + bb] = 0;
+  if (tid < 16) reinterpret_cast<uint32_t *>(payload)[tid] = hdr.w[tid];
+  // round-robin flags: mark this step's blocks; restart the round once all are sent
+  int all_sent = 1;
+  for (int i = tid; i < K; i += kSelThreads) {
+    const uint8_t s = (uint8_t)(sent[i] | pick[i]);
+    sent[i] = s;
+    all_sent &= s;
+  }
+  if (__syncthreads_and(all_sent))
+    for (int i = tid; i < K; i += kSelThreads) sent[i] = 0;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kBsThreads) bs_pack_kernel(const T *a, const uint32_t *sel, int W, int b,
+                                                              int64_t cols, T *data) {
+  pdl_enter();
+  const int j = blockIdx.x / b, y = blockIdx.x - (blockIdx.x / b) * b;
+  const uint32_t blk = sel[j];
+  const int64_t n8 = (int64_t)b * cols / 8;
+  T *dst = data + ((int64_t)j * b * b + (int64_t)y * b) * cols;
+  if (blk == kBsNone) {
+    float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const typename Vec8<T>::Raw zr = Vec8<T>::from_f32(z);
+    for (int64_t v = threadIdx.x; v < n8; v += kBsThreads) Vec8<T>::store(dst + v * 8, zr);
+    return;
+  }
+  const T *src = a + block_row_token((int)blk, y, W, b) * cols;
+  for (int64_t v = threadIdx.x; v < n8; v += kBsThreads) Vec8<T>::store(dst + v * 8, Vec8<T>::load(src + v * 8));
+}
+
+// ------------------------------------------------------------------ decode
+
+template <typename T>
+__global__ void __launch_bounds__(kBsThreads) bs_decode_kernel(const uint8_t *payload, float *ahat, T *recon,
+                                                                int W, int b, int64_t cols, int k, int K,
+                                                                const Header expect, int *status) {
+  __shared__ int slot;
+  const int i = blockIdx.x / b, y = blockIdx.x - (blockIdx.x / b) * b;
+  int bad = 0;
+  if (threadIdx.x < 16) bad = reinterpret_cast<const uint32_t *>(payload)[threadIdx.x] != expect.w[threadIdx.x];
+  if (__syncthreads_or(bad)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, 1);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    // the slot of block i in the ascending index list (unused slots sort last)
+    const uint32_t *slots = reinterpret_cast<const uint32_t *>(payload + kHdrBytes);
+    int lo = 0, hi = k - 1, found = -1;
+    while (lo <= hi) {
+      const int mid = (lo + hi) >> 1;
+      const uint32_t v = slots[mid];
+      if (v == (uint32_t)i) {
+        found = mid;
+        break;
+      }
+      if (v < (uint32_t)i) lo = mid + 1;
+      else hi = mid - 1;
+    }
+    slot = (i < K) ? found : -1;
+  }
+  __syncthreads();
+  const int64_t e0 = block_row_token(i, y, W, b) * cols;
+  const int64_t n8 = (int64_t)b * cols / 8;
+  if (slot >= 0) {
+    const T *src = reinterpret_cast<const T *>(payload + kHdrBytes + ((4 * (size_t)k + 15) & ~(size_t)15)) +
+                   ((int64_t)slot * b * b + (int64_t)y * b) * cols;
+    for (int64_t v = threadIdx.x; v < n8; v += kBsThreads) {
+      const typename Vec8<T>::Raw r = Vec8<T>::load(src + v * 8);
+      float x[8];
+      Vec8<T>::to_f32(r, x);
+      store_f32x8(ahat + e0 + v * 8, x);
+      Vec8<T>::store(recon + e0 + v * 8, r);
+    }
+  } else {
+    for (int64_t v = threadIdx.x; v < n8; v += kBsThreads) {
+      float x[8];
+      load_f32x8(ahat + e0 + v * 8, x);
+      Vec8<T>::store(recon + e0 + v * 8, Vec8<T>::from_f32(x));
+    }
+  }
+}
+
+int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+size_t select_smem(int K2) { return (size_t)K2 * (8 + 4 + 1); }
+
+}  // namespace
+
+int blocksel_plan(int64_t rows, int64_t cols, int dtype, int batch, int grid_h, int block, int k, int warm,
+                  BlockselPlan *P) {
+  if (batch != 1) return CF_ERR_UNSUPPORTED;
+  if (block != 4 && block != 8 && block != 16) return CF_ERR_UNSUPPORTED;
+  if (warm < 1) return CF_ERR_ARG;
+  int64_t h = grid_h;
+  if (h == 0) {  // square grid
+    h = 1;
+    while ((h + 1) * (h + 1) <= rows) h++;
+    if (h * h != rows) return CF_ERR_SHAPE;
+  }
+  if (h < 1 || rows % h) return CF_ERR_SHAPE;
+  const int64_t w = rows / h;
+  if (h % block || w % block) return CF_ERR_SHAPE;
+  const int64_t K = (h / block) * (w / block);
+  if (K < 1 || K > kBsMaxBlocks) return CF_ERR_UNSUPPORTED;
+  const int kk = k == 0 ? (int)(K / 4 > 0 ? K / 4 : 1) : k;
+  if (kk < 1 || kk > K) return CF_ERR_ARG;
+  P->rows = rows;
+  P->cols = cols;
+  P->H = (int)h;
+  P->W = (int)w;
+  P->b = block;
+  P->K = (int)K;
+  P->k = kk;
+  P->warm = warm;
+  P->dtype = dtype;
+  return CF_OK;
+}
+
+size_t blocksel_body_bytes(const BlockselPlan &P) {
+  const size_t asz = P.dtype == CF_BF16 ? 2u : 4u;
+  return pad16((size_t)P.k * 4u) + (size_t)P.k * P.b * P.b * (size_t)P.cols * asz;
+}
+
+size_t blocksel_scratch_bytes(const BlockselPlan &P) {
+  return pad256((size_t)P.K) + pad256((size_t)P.K * P.b * 4 * 8) + pad256((size_t)P.k * 4);
+}
+
+int blocksel_bind(BlockselPlan *P, void *scratch) {
+  uint8_t *p = static_cast<uint8_t *>(scratch);
+  P->sent = p;
+  p += pad256((size_t)P->K);
+  P->part = reinterpret_cast<double *>(p);
+  p += pad256((size_t)P->K * P->b * 4 * 8);
+  P->sel = reinterpret_cast<uint32_t *>(p);
+  if (cudaFuncSetAttribute(bs_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)select_smem(next_pow2(P->K))) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return CF_ERR_CUDA;
+  }
+  return CF_OK;
+}
+
+cudaError_t blocksel_encode(const BlockselPlan &P, const void *a, float *prev, uint8_t *payload, const Header &hdr,
+                            cudaStream_t st) {
+  const int K2 = next_pow2(P.K);
+  const unsigned rows_grid = (unsigned)(P.K * P.b), pack_grid = (unsigned)(P.k * P.b);
+  if (P.dtype == CF_BF16) {
+    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a);
+    launch_pdl(bs_partial_kernel<__nv_bfloat16>, dim3(rows_grid), dim3(kBsThreads), 0, st, x, prev, P.W, P.b, P.cols,
+               P.part);
+    launch_pdl(bs_select_kernel, dim3(1), dim3(kSelThreads), select_smem(K2), st, (const double *)P.part, P.K, K2,
+               P.b, P.k, P.sent, P.sel, payload, hdr);
+    __nv_bfloat16 *data = reinterpret_cast<__nv_bfloat16 *>(payload + kHdrBytes + pad16((size_t)P.k * 4u));
+    launch_pdl(bs_pack_kernel<__nv_bfloat16>, dim3(pack_grid), dim3(kBsThreads), 0, st, x, (const uint32_t *)P.sel,
+               P.W, P.b, P.cols, data);
+  } else {
+    const float *x = static_cast<const float *>(a);
+    launch_pdl(bs_partial_kernel<float>, dim3(rows_grid), dim3(kBsThreads), 0, st, x, prev, P.W, P.b, P.cols, P.part);
+    launch_pdl(bs_select_kernel, dim3(1), dim3(kSelThreads), select_smem(K2), st, (const double *)P.part, P.K, K2,
+               P.b, P.k, P.sent, P.sel, payload, hdr);
+    float *data = reinterpret_cast<float *>(payload + kHdrBytes + pad16((size_t)P.k * 4u));
+    launch_pdl(bs_pack_kernel<float>, dim3(pack_grid), dim3(kBsThreads), 0, st, x, (const uint32_t *)P.sel, P.W,
+               P.b, P.cols, data);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t blocksel_decode(const BlockselPlan &P, const uint8_t *payload, float *ahat, void *recon,
+                            const Header &expect, int *status, cudaStream_t st) {
+  const unsigned grid = (unsigned)(P.K * P.b);
+  if (P.dtype == CF_BF16)
+    bs_decode_kernel<__nv_bfloat16><<<grid, kBsThreads, 0, st>>>(payload, ahat, static_cast<__nv_bfloat16 *>(recon),
+                                                                 P.W, P.b, P.cols, P.k, P.K, expect, status);
+  else
+    bs_decode_kernel<float><<<grid, kBsThreads, 0, st>>>(payload, ahat, static_cast<float *>(recon), P.W, P.b, P.cols,
+                                                         P.k, P.K, expect, status);
+  return cudaGetLastError();
+}
+
+}  // namespace cfi

@@ -32,6 +32,7 @@
 #include <mutex>
 
 #include "cf_lowrank.h"
+#include "cf_launch.cuh"
 #include "cf_umma.cuh"
 
 namespace cfi {
@@ -85,33 +86,6 @@ __device__ __forceinline__ float v0_entry(uint64_t seed, int64_t j, int r, int k
 
 // ---------------------------------------------------------------- V preparation
 
-// Programmatic dependent launch.  Every kernel of the encode and decode
-// chains starts here: it waits until the kernel before it in the stream has
-// completed and its writes are visible, then lets the kernel after it be
-// scheduled, so that launch latency overlaps the tail of the running grid.
-// Without the launch attribute both instructions return at once.
-__device__ __forceinline__ void pdl_enter() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-// Launch with the programmatic-stream-serialisation attribute (the kernel
-// must begin with pdl_enter()).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                       Args &&...args) {
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-}
 
 // Vt (split bf16, [rp][cols]) from the warm start: the previous step's V
 // (fp32 [cols][r]), or V0 on the first step and for any all-zero column.

@@ -117,7 +117,7 @@ int stream_config(int mode, int dtype, int nm_m, int nm_n, int64_t rows, int64_t
   const int64_t n_rg = ((int64_t)batch * rows + tpb - 1) / tpb;
   auto cap = [&](int64_t g) -> int { return (int)(g < n_rg ? g : n_rg); };
   cfg->enc_grid = cfg->dec_grid = 1;
-  if (mode != CF_LOWRANK) {
+  if (mode != CF_LOWRANK && mode != CF_BLOCKSEL) {
     const void *efn = kernel_any(true, mode, dtype, nm_m, nm_n, best_v, false);
     const void *dfn = kernel_any(false, mode, dtype, nm_m, nm_n, best_v, false);
     if (!efn || !dfn) return CF_ERR_UNSUPPORTED;

@@ -866,7 +866,7 @@ __global__ void __launch_bounds__(kBlock) warm_encode_kernel(const EncArgs A, co
         Act<T>::store_raw(prow + v * 8, raw);
         store_f32x8(A.ahat + gr * cols + v * 8, x);
         const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        store_f32x8(A.err + gr * cols + v * 8, z);
+        if (A.err) store_f32x8(A.err + gr * cols + v * 8, z);  // block selection keeps no e
       }
     }
   }

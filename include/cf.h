@@ -107,7 +107,18 @@ extern "C" {
 #define CF_ERR_TOO_LARGE (-12)   /* problem larger than the allocation-free entry point's fixed scratch */
 
 /* ---- enumerations ---------------------------------------------------- */
-typedef enum { CF_IDENTITY = 0, CF_SIGN1 = 1, CF_Q2 = 2, CF_NM = 3, CF_LOWRANK = 4 } cf_mode;
+/* CF_BLOCKSEL is Otil's selective transmission ("Informative sub-block
+ * selection", "Dynamic round-robin"): not a residual codec.  The rows are a
+ * token grid bs_grid_h x (rows / bs_grid_h) in raster order, cut into
+ * bs_block x bs_block blocks spanning all channels; each selective step sends
+ * the bs_k blocks whose cosine dissimilarity d = 1 - <x_{t-1}, x_t>_F /
+ * (||x_{t-1}|| ||x_t||) against the previous activation is largest, among the
+ * blocks not yet sent in the current round (ties: lower block index; a block
+ * with all values unchanged has d = 0, one with exactly one zero norm d = 1);
+ * the round restarts once every block has been sent; the receiver keeps
+ * every other block as last received.  The first bs_warm steps are sent in
+ * full.  Error feedback does not apply (ef is ignored). */
+typedef enum { CF_IDENTITY = 0, CF_SIGN1 = 1, CF_Q2 = 2, CF_NM = 3, CF_LOWRANK = 4, CF_BLOCKSEL = 5 } cf_mode;
 typedef enum { CF_F32 = 0, CF_BF16 = 1 } cf_dtype;
 typedef enum { CF_SENDER = 0, CF_RECEIVER = 1 } cf_role;
 /* Error-feedback form ("Key design: error feedback"):
@@ -137,6 +148,10 @@ typedef struct {
     uint64_t seed;             /* CF_LOWRANK: seed of the first step's V */
     void *workspace;           /* optional caller-owned device memory for the state, or NULL */
     size_t workspace_bytes;    /* its size; must be >= cf_workspace_bytes() */
+    int bs_grid_h;             /* CF_BLOCKSEL: token-grid height; 0 = square grid (rows a square) */
+    int bs_block;              /* CF_BLOCKSEL: block side in tokens, 4, 8 or 16 (default 8) */
+    int bs_k;                  /* CF_BLOCKSEL: blocks per step, 1..K; 0 = K/4 ("k/K = 1/4") */
+    int bs_warm;               /* CF_BLOCKSEL: leading steps sent in full, >= 1 (default 5) */
 } cf_params;
 
 typedef struct cf_state cf_state;
@@ -158,6 +173,8 @@ CF_API int cf_workspace_bytes(int64_t rows, int64_t cols, int mode, const cf_par
 /* Create a sender or receiver state on the current CUDA device.  Shape
  * rules: rows >= 1; cols % 8 == 0 and cols <= 8192; CF_SIGN1 cols % 32 == 0;
  * CF_Q2 cols % 16 == 0; CF_NM cols % M == 0 and (cols/M) N log2(M) % 32 == 0;
+ * CF_BLOCKSEL: the grid and both of its sides divisible by bs_block,
+ * K = (H/b)(W/b) <= 4096 blocks, batch 1;
  * CF_LOWRANK rows % 128 == 0, cols % 128 == 0, rank <= min(rows, cols, 128),
  * (rows + cols) * round_up(rank, 64) < 2^31 (32-bit factor indices),
  * batch 1 (the low-rank state also holds its factor scratch: about

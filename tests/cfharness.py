@@ -34,13 +34,14 @@ class GpuPair:
     """A sender and a receiver state of the CUDA codec plus guarded device buffers."""
 
     def __init__(self, rows, cols, mode, dtype="bf16", ef="explicit", nm_n=1, nm_m=16, batch=1,
-                 rank=70, iters=1, lr_int4=1, seed=0):
+                 rank=70, iters=1, lr_int4=1, seed=0, **extra):
         self.rows, self.cols, self.batch = rows, cols, batch
         self.mode = cf.MODE_NAMES[mode]
         self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
         kw = dict(dtype=cf.CF_BF16 if dtype == "bf16" else cf.CF_F32,
                   ef={"explicit": cf.CF_EF_EXPLICIT, "implicit": cf.CF_EF_IMPLICIT, "off": cf.CF_EF_OFF}[ef],
-                  nm_n=nm_n, nm_m=nm_m, batch=batch, rank=rank, iters=iters, lr_int4=lr_int4, seed=seed)
+                  nm_n=nm_n, nm_m=nm_m, batch=batch, rank=rank, iters=iters, lr_int4=lr_int4, seed=seed, **extra)
+        self.has_err = mode != "blocksel"       # block selection keeps no error term
         self.S = cf.cf_create(rows, cols, self.mode, cf.cf_params_init(role=cf.CF_SENDER, **kw))
         self.R = cf.cf_create(rows, cols, self.mode, cf.cf_params_init(role=cf.CF_RECEIVER, **kw))
         self.pb_warm = cf.cf_payload_bytes(self.S, True)
@@ -75,12 +76,19 @@ class GpuPair:
         n = self.batch * self.rows * self.cols
         ahat = ten[:4 * n].view(np.float32).reshape(self.batch, self.rows, self.cols)
         err = None
-        if which == "S":
+        if which == "S" and self.has_err:
             err = ten[4 * n:8 * n].view(np.float32).reshape(self.batch, self.rows, self.cols)
         if with_vprev:
             vp = ten[8 * n:].view(np.float32).reshape(self.batch, self.cols, -1)
             return ahat, err, vp
         return ahat, err
+
+    def sent_flags(self) -> np.ndarray:
+        """Block selection (sender): the per-block 'sent this round' flags (the export's tail)."""
+        buf = self.export("S")
+        tb = int(buf[80:88].view(np.uint64)[0])
+        ten = buf[len(buf) - tb:]
+        return ten[4 * self.batch * self.rows * self.cols:].copy()
 
     def guards_ok(self) -> bool:
         return canaries_intact(self.pay_whole) and canaries_intact(self.rec_whole)
