@@ -217,6 +217,10 @@ size_t warm_body(const cf_state *s) { return pad16((size_t)(s->rows * s->cols) *
 // leading steps sent in full (block selection: bs_warm; every other mode: 1)
 uint64_t warm_steps(const cf_state *s) { return s->mode == CF_BLOCKSEL ? (uint64_t)s->bs.warm : 1u; }
 
+// bytes per element of the ahat tensor: fp32, except block selection, whose
+// state holds raw activations in their own dtype
+size_t ahat_elem_bytes(const cf_state *s) { return s->mode == CF_BLOCKSEL ? act_size(s->p.dtype) : 4u; }
+
 EncArgs enc_args(cf_state *s, const void *a, void *payload, bool warm) {
   EncArgs A{};
   A.a = a;
@@ -285,10 +289,10 @@ int do_encode(cf_state *s, const void *a, const PtrTable *tab, void *payload, cu
   if (s->mode == CF_BLOCKSEL && tab) return CF_ERR_UNSUPPORTED;
   EncArgs A = enc_args(s, a, payload, warm);
   cudaError_t e;
-  if (warm) {
+  if (s->mode == CF_BLOCKSEL) {
+    e = blocksel_encode(s->bs, a, s->ahat, static_cast<uint8_t *>(payload), A.hdr, warm, st);
+  } else if (warm) {
     e = launch_warm_encode(s->p.dtype, s->cfg, A, tab, st);
-  } else if (s->mode == CF_BLOCKSEL) {
-    e = blocksel_encode(s->bs, a, s->ahat, static_cast<uint8_t *>(payload), A.hdr, st);
   } else if (s->mode == CF_LOWRANK) {
     e = lowrank_encode(s->lr, A, tab, s->vprev, s->step, s->p.seed, st);
   } else {
@@ -310,10 +314,10 @@ int do_decode(cf_state *s, const void *payload, void *recon, const PtrTable *tab
   if (s->mode == CF_BLOCKSEL && tab) return CF_ERR_UNSUPPORTED;
   DecArgs A = dec_args(s, payload, recon, warm);
   cudaError_t e;
-  if (warm) {
+  if (s->mode == CF_BLOCKSEL) {
+    e = blocksel_decode(s->bs, static_cast<const uint8_t *>(payload), s->ahat, recon, A.expect, warm, s->status, st);
+  } else if (warm) {
     e = launch_warm_decode(s->p.dtype, s->cfg, A, tab, st);
-  } else if (s->mode == CF_BLOCKSEL) {
-    e = blocksel_decode(s->bs, static_cast<const uint8_t *>(payload), s->ahat, recon, A.expect, s->status, st);
   } else if (s->mode == CF_LOWRANK) {
     e = lowrank_decode(s->lr, A, tab, st);
   } else {
@@ -538,7 +542,7 @@ int cf_tensor(cf_state *s, int which, void **dptr, size_t *bytes) {
   switch (which) {
     case CF_T_RECON:
       *dptr = s->ahat;
-      *bytes = E * 4u;
+      *bytes = E * ahat_elem_bytes(s);
       return CF_OK;
     case CF_T_ERROR:
       if (!s->err) return CF_ERR_ROLE;
@@ -571,7 +575,7 @@ int cf_reset(cf_state *s) {
 
 static size_t export_tensor_bytes(const cf_state *s) {
   const size_t E = (size_t)(s->rows * s->cols) * (size_t)s->p.batch;
-  size_t b = E * 4u;
+  size_t b = E * ahat_elem_bytes(s);
   if (s->err) b += E * 4u;
   if (s->vprev) b += (size_t)s->cols * s->p.rank * 4u * s->p.batch;
   if (s->bs.sent) b += (size_t)s->bs.K;
@@ -602,8 +606,9 @@ int cf_state_export(const cf_state *s, void *host, size_t bytes, void *stream) {
   std::memcpy(dst, &h, sizeof(h));
   dst += sizeof(h);
   const size_t E = (size_t)(s->rows * s->cols) * (size_t)s->p.batch;
-  if (cudaMemcpy(dst, s->ahat, E * 4u, cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_err(cudaErrorUnknown);
-  dst += E * 4u;
+  const size_t hb = E * ahat_elem_bytes(s);
+  if (cudaMemcpy(dst, s->ahat, hb, cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_err(cudaErrorUnknown);
+  dst += hb;
   if (s->err) {
     if (cudaMemcpy(dst, s->err, E * 4u, cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_err(cudaErrorUnknown);
     dst += E * 4u;
@@ -634,8 +639,9 @@ int cf_state_import(cf_state *s, const void *host, size_t bytes, void *stream) {
   if (cudaStreamSynchronize(st) != cudaSuccess) return cuda_err(cudaErrorUnknown);
   const uint8_t *src = static_cast<const uint8_t *>(host) + sizeof(h);
   const size_t E = (size_t)(s->rows * s->cols) * (size_t)s->p.batch;
-  if (cudaMemcpy(s->ahat, src, E * 4u, cudaMemcpyHostToDevice) != cudaSuccess) return cuda_err(cudaErrorUnknown);
-  src += E * 4u;
+  const size_t hb = E * ahat_elem_bytes(s);
+  if (cudaMemcpy(s->ahat, src, hb, cudaMemcpyHostToDevice) != cudaSuccess) return cuda_err(cudaErrorUnknown);
+  src += hb;
   if (s->err) {
     if (cudaMemcpy(s->err, src, E * 4u, cudaMemcpyHostToDevice) != cudaSuccess) return cuda_err(cudaErrorUnknown);
     src += E * 4u;

@@ -1,18 +1,22 @@
 // cf_blocksel.cu -- kernels of the block-selection mode (Otil page:
 // "Informative sub-block selection", "Dynamic round-robin").
 //
-// Encode = three launches on the caller's stream:
-//   bs_partial_kernel  one CTA per (block, token row of the block): the fp64
+// The state (the sender's previous activation, the receiver's values) is
+// kept in the activation dtype: it only ever holds raw activations, which that
+// dtype represents exactly.
+//
+// Encode = two launches on the caller's stream:
+//   bs_encode_kernel   one CTA per (block, token row of the block): the fp64
 //                      Frobenius sums <p, a>, ||p||^2, ||a||^2 and a changed
 //                      flag over the row's b tokens x all channels, and the
-//                      state update p = fp32(a) (the row is read once);
-//   bs_select_kernel   one CTA: d per block from the partials (fixed order),
-//                      bitonic sort of the unsent blocks by (d desc, index
-//                      asc), the first min(k, unsent) blocks in ascending
-//                      order, the round-robin flags, the payload header and
-//                      index section;
-//   bs_pack_kernel     one CTA per (slot, token row): raw block rows into the
-//                      payload (unused slots zeroed).
+//                      state update p = a (the row is read once); the CTA
+//                      that finishes last runs the selection: d per block
+//                      from the partials (fixed order), bitonic sort of the
+//                      unsent blocks by (d desc, index asc), the first
+//                      min(k, unsent) in ascending order, the round-robin
+//                      flags, the payload header and index section;
+//   bs_pack_kernel     one CTA per (slot, token-row quarter): raw block rows
+//                      into the payload (unused slots zeroed).
 // Decode = one launch: bs_decode_kernel, one CTA per (block, token row): the
 // row comes from the payload when its block was sent, else from ahat; ahat
 // and recon are written.
@@ -29,7 +33,7 @@ namespace cfi {
 namespace {
 
 constexpr int kBsThreads = 256;
-constexpr int kSelThreads = 1024;
+constexpr int kSelThreads = 1024;  // the largest selection CTA
 
 size_t pad16(size_t x) { return (x + 15u) & ~(size_t)15u; }
 size_t pad256(size_t x) { return (x + 255u) & ~(size_t)255u; }
@@ -100,56 +104,6 @@ __device__ __forceinline__ int64_t block_row_token(int i, int y, int W, int b) {
 
 // ------------------------------------------------------------------ encode
 
-// Sums over one token row of one block, state update fused.  Each product of
-// two fp32 values is exact in fp64, so each fused multiply-add rounds once;
-// the CTA adds its threads' sums in a fixed order (deterministic).
-template <typename T>
-__global__ void __launch_bounds__(kBsThreads) bs_partial_kernel(const T *a, float *prev, int W, int b,
-                                                                 int64_t cols, double *part) {
-  pdl_enter();
-  const int i = blockIdx.x / b, y = blockIdx.x - (blockIdx.x / b) * b;
-  const int64_t e0 = block_row_token(i, y, W, b) * cols;
-  const int64_t n8 = (int64_t)b * cols / 8;
-  double dot = 0.0, np_ = 0.0, na = 0.0;
-  int changed = 0;
-  for (int64_t v = threadIdx.x; v < n8; v += kBsThreads) {
-    const int64_t e = e0 + v * 8;
-    float x[8], p[8];
-    Vec8<T>::to_f32(Vec8<T>::load(a + e), x);
-    load_f32x8(prev + e, p);
-#pragma unroll
-    for (int k = 0; k < 8; k++) {
-      changed |= p[k] != x[k];
-      dot = fma((double)p[k], (double)x[k], dot);
-      np_ = fma((double)p[k], (double)p[k], np_);
-      na = fma((double)x[k], (double)x[k], na);
-    }
-    store_f32x8(prev + e, x);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    np_ += __shfl_xor_sync(0xffffffffu, np_, o);
-    na += __shfl_xor_sync(0xffffffffu, na, o);
-    changed |= __shfl_xor_sync(0xffffffffu, changed, o);
-  }
-  __shared__ double ws[kBsThreads / 32][4];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) {
-    ws[warp][0] = dot;
-    ws[warp][1] = np_;
-    ws[warp][2] = na;
-    ws[warp][3] = changed ? 1.0 : 0.0;
-  }
-  __syncthreads();
-  if (threadIdx.x < 4) {
-    double s = ws[0][threadIdx.x];
-    for (int w = 1; w < kBsThreads / 32; w++)
-      s = threadIdx.x == 3 ? fmax(s, ws[w][3]) : s + ws[w][threadIdx.x];
-    part[(int64_t)blockIdx.x * 4 + threadIdx.x] = s;
-  }
-}
-
 // Order-preserving key of a double (larger d -> larger key); 0 marks "not a
 // candidate" (no finite d maps to it).
 __device__ __forceinline__ unsigned long long sort_key(double d) {
@@ -162,46 +116,58 @@ __device__ __forceinline__ bool before(unsigned long long kx, int ix, unsigned l
   return kx > ky || (kx == ky && ix < iy);
 }
 
-__global__ void __launch_bounds__(kSelThreads) bs_select_kernel(const double *part, int K, int K2, int b, int k,
-                                                                 uint8_t *sent, uint32_t *sel, uint8_t *payload,
-                                                                 const Header hdr) {
-  pdl_enter();
-  extern __shared__ __align__(16) uint8_t smem[];
+// The selection, run by one CTA of kBsThreads threads once every partial is
+// written: d per unsent block from its b partials (in order), bitonic sort of
+// K2 (a power of two) entries by (d desc, index asc), the first min(k,
+// unsent) blocks in ascending order into sel and the payload's index
+// section, the round-robin flags (restarting the round when all are sent)
+// and the payload header.
+__device__ void select_blocks(const double *part, int K, int K2, int b, int k, uint8_t *sent, uint32_t *sel,
+                              uint8_t *payload, const Header &hdr, uint8_t *smem) {
   unsigned long long *key = reinterpret_cast<unsigned long long *>(smem);  // [K2]
   int *idx = reinterpret_cast<int *>(key + K2);                           // [K2]
   uint8_t *pick = reinterpret_cast<uint8_t *>(idx + K2);                  // [K2]
-  __shared__ int wsum[kSelThreads / 32];
+  __shared__ int wsum[kBsThreads / 32];
   const int tid = threadIdx.x;
-  // dissimilarities of the unsent blocks
-  int mine = 0;
-  for (int i = tid; i < K2; i += kSelThreads) {
+  for (int i = tid; i < K2; i += kBsThreads) {
     unsigned long long kk = 0ull;
     if (i < K && !sent[i]) {
+      const double4 *src = reinterpret_cast<const double4 *>(part) + (int64_t)i * b;
       double dot = 0.0, np_ = 0.0, na = 0.0, ch = 0.0;
-      for (int y = 0; y < b; y++) {
-        const double *q = part + ((int64_t)i * b + y) * 4;
-        dot += q[0];
-        np_ += q[1];
-        na += q[2];
-        ch = fmax(ch, q[3]);
+      for (int r0 = 0; r0 < b; r0 += 8) {
+        double4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+          v[u] = make_double4(0.0, 0.0, 0.0, 0.0);
+          if (r0 + u < b) {  // written by other CTAs of this grid: read through L2
+            const double2 *q2 = reinterpret_cast<const double2 *>(src + r0 + u);
+            const double2 lo = __ldcg(q2), hi = __ldcg(q2 + 1);
+            v[u] = make_double4(lo.x, lo.y, hi.x, hi.y);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; u++)
+          if (r0 + u < b) {
+            dot += v[u].x;
+            np_ += v[u].y;
+            na += v[u].z;
+            ch = fmax(ch, v[u].w);
+          }
       }
       double d;
       if (ch == 0.0) d = 0.0;                       // every value unchanged
       else if (np_ == 0.0 || na == 0.0) d = 1.0;    // exactly one zero norm
       else d = 1.0 - dot / (sqrt(np_) * sqrt(na));
       kk = sort_key(d);
-      mine++;
     }
     key[i] = kk;
     idx[i] = i;
     pick[i] = 0;
   }
-  (void)mine;
-  // bitonic sort of K2 (a power of two) entries into "before" order
   for (int size = 2; size <= K2; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       __syncthreads();
-      for (int i = tid; i < K2; i += kSelThreads) {
+      for (int i = tid; i < K2; i += kBsThreads) {
         const int j = i ^ stride;
         if (j > i) {
           const bool up = (i & size) == 0;
@@ -221,15 +187,14 @@ __global__ void __launch_bounds__(kSelThreads) bs_select_kernel(const double *pa
   }
   __syncthreads();
   // candidates sort first (key > 0); the first min(k, candidates) are picked
-  for (int r = tid; r < K2; r += kSelThreads)
+  for (int r = tid; r < K2; r += kBsThreads)
     if (r < k && key[r] != 0ull) pick[idx[r]] = 1;
   __syncthreads();
   // ascending list of the picked blocks: each thread owns a contiguous chunk
-  const int chunk = (K2 + kSelThreads - 1) / kSelThreads;
+  const int chunk = (K2 + kBsThreads - 1) / kBsThreads;
   const int c0 = tid * chunk;
   int cnt = 0;
   for (int i = c0; i < c0 + chunk && i < K2; i++) cnt += pick[i];
-  // exclusive scan of cnt over the CTA
   const int lane = tid & 31, warp = tid >> 5;
   int incl = cnt;
 #pragma unroll
@@ -239,10 +204,11 @@ __global__ void __launch_bounds__(kSelThreads) bs_select_kernel(const double *pa
   }
   if (lane == 31) wsum[warp] = incl;
   __syncthreads();
-  int base = 0;
-  for (int w = 0; w < warp; w++) base += wsum[w];
-  int m = 0;
-  for (int w = 0; w < kSelThreads / 32; w++) m += wsum[w];
+  int base = 0, m = 0;
+  for (int w = 0; w < kBsThreads / 32; w++) {
+    if (w < warp) base += wsum[w];
+    m += wsum[w];
+  }
   int pos = base + incl - cnt;
   uint32_t *slots = reinterpret_cast<uint32_t *>(payload + kHdrBytes);
   for (int i = c0; i < c0 + chunk && i < K2; i++)
@@ -251,72 +217,176 @@ __global__ void __launch_bounds__(kSelThreads) bs_select_kernel(const double *pa
       slots[pos] = (uint32_t)i;
       pos++;
     }
-  for (int j = m + tid; j < k; j += kSelThreads) {
+  for (int j = m + tid; j < k; j += kBsThreads) {
     sel[j] = kBsNone;
     slots[j] = kBsNone;
   }
-  // index-section padding
-  for (int bb = 4 * k + tid; bb < (int)((4 * k + 15) & ~15); bb += kSelThreads) payload[kHdrBytes + bb] = 0;
+  for (int bb = 4 * k + tid; bb < (int)((4 * k + 15) & ~15); bb += kBsThreads) payload[kHdrBytes + bb] = 0;
   if (tid < 16) reinterpret_cast<uint32_t *>(payload)[tid] = hdr.w[tid];
-  // round-robin flags: mark this step's blocks; restart the round once all are sent
   int all_sent = 1;
-  for (int i = tid; i < K; i += kSelThreads) {
-    const uint8_t s = (uint8_t)(sent[i] | pick[i]);
-    sent[i] = s;
-    all_sent &= s;
+  for (int i = tid; i < K; i += kBsThreads) {
+    const uint8_t f = (uint8_t)(sent[i] | pick[i]);
+    sent[i] = f;
+    all_sent &= f;
   }
   if (__syncthreads_and(all_sent))
-    for (int i = tid; i < K; i += kSelThreads) sent[i] = 0;
+    for (int i = tid; i < K; i += kBsThreads) sent[i] = 0;
 }
 
+// One CTA per (block, token row of the block): the row's Frobenius sums in
+// fp64 (each product of two fp32 values is exact, so each fused
+// multiply-add rounds once; the CTA adds its threads' sums in a fixed
+// order) and the state update prev = a (the row is read once).  The CTA
+// that finishes last (an atomic count after a fence) then runs the
+// selection on the complete set of partials, still in L2.
+template <typename T>
+__global__ void __launch_bounds__(kBsThreads) bs_encode_kernel(const T *a, T *prev, int W, int b, int64_t cols,
+                                                                int K, int K2, int k, double *part,
+                                                                unsigned *counter, uint8_t *sent, uint32_t *sel,
+                                                                uint8_t *payload, const Header hdr) {
+  pdl_enter();
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ int last;
+  const int i = blockIdx.x / b, y = blockIdx.x - (blockIdx.x / b) * b;
+  const int64_t e0 = block_row_token(i, y, W, b) * cols;
+  const int64_t n8 = (int64_t)b * cols / 8;
+  double dot = 0.0, np_ = 0.0, na = 0.0;
+  int changed = 0;
+  constexpr int U = 4;  // vectors in flight per thread
+  for (int64_t v0 = threadIdx.x; v0 < n8; v0 += (int64_t)U * kBsThreads) {
+    typename Vec8<T>::Raw ra[U], rp[U];
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int64_t v = v0 + (int64_t)u * kBsThreads;
+      if (v < n8) {
+        ra[u] = Vec8<T>::load(a + e0 + v * 8);
+        rp[u] = Vec8<T>::load(prev + e0 + v * 8);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int64_t v = v0 + (int64_t)u * kBsThreads;
+      if (v < n8) {
+        float x[8], p[8];
+        Vec8<T>::to_f32(ra[u], x);
+        Vec8<T>::to_f32(rp[u], p);
+#pragma unroll
+        for (int q = 0; q < 8; q++) {
+          changed |= p[q] != x[q];
+          dot = fma((double)p[q], (double)x[q], dot);
+          np_ = fma((double)p[q], (double)p[q], np_);
+          na = fma((double)x[q], (double)x[q], na);
+        }
+        Vec8<T>::store(prev + e0 + v * 8, ra[u]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    np_ += __shfl_xor_sync(0xffffffffu, np_, o);
+    na += __shfl_xor_sync(0xffffffffu, na, o);
+    changed |= __shfl_xor_sync(0xffffffffu, changed, o);
+  }
+  __shared__ double ws[kBsThreads / 32][4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    ws[warp][0] = dot;
+    ws[warp][1] = np_;
+    ws[warp][2] = na;
+    ws[warp][3] = changed ? 1.0 : 0.0;
+  }
+  __syncthreads();
+  if (threadIdx.x < 4) {
+    double sacc = ws[0][threadIdx.x];
+    for (int w = 1; w < kBsThreads / 32; w++)
+      sacc = threadIdx.x == 3 ? fmax(sacc, ws[w][3]) : sacc + ws[w][threadIdx.x];
+    part[(int64_t)blockIdx.x * 4 + threadIdx.x] = sacc;
+  }
+  // the last CTA to finish selects
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(counter, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  select_blocks(part, K, K2, b, k, sent, sel, payload, hdr, smem);
+  if (threadIdx.x == 0) *counter = 0u;  // for the next step
+}
+
+constexpr int kPackSplit = 4;  // CTAs per (slot, token row)
 template <typename T>
 __global__ void __launch_bounds__(kBsThreads) bs_pack_kernel(const T *a, const uint32_t *sel, int W, int b,
                                                               int64_t cols, T *data) {
   pdl_enter();
-  const int j = blockIdx.x / b, y = blockIdx.x - (blockIdx.x / b) * b;
+  const int row = blockIdx.x / kPackSplit, piece = blockIdx.x - row * kPackSplit;
+  const int j = row / b, y = row - (row / b) * b;
   const uint32_t blk = sel[j];
   const int64_t n8 = (int64_t)b * cols / 8;
+  const int64_t v0 = n8 * piece / kPackSplit, v1 = n8 * (piece + 1) / kPackSplit;
   T *dst = data + ((int64_t)j * b * b + (int64_t)y * b) * cols;
   if (blk == kBsNone) {
     float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     const typename Vec8<T>::Raw zr = Vec8<T>::from_f32(z);
-    for (int64_t v = threadIdx.x; v < n8; v += kBsThreads) Vec8<T>::store(dst + v * 8, zr);
+    for (int64_t v = v0 + threadIdx.x; v < v1; v += kBsThreads) Vec8<T>::store(dst + v * 8, zr);
     return;
   }
   const T *src = a + block_row_token((int)blk, y, W, b) * cols;
-  for (int64_t v = threadIdx.x; v < n8; v += kBsThreads) Vec8<T>::store(dst + v * 8, Vec8<T>::load(src + v * 8));
+  for (int64_t v = v0 + threadIdx.x; v < v1; v += kBsThreads) Vec8<T>::store(dst + v * 8, Vec8<T>::load(src + v * 8));
 }
 
-// ------------------------------------------------------------------ decode
+// Full-size leading steps: payload body = a, state = a (sender); state =
+// recon = body (receiver, after the header check).
+template <typename T>
+__global__ void __launch_bounds__(kBsThreads) bs_warm_encode_kernel(const T *a, T *prev, uint8_t *payload, int64_t E,
+                                                                     const Header hdr) {
+  if (blockIdx.x == 0 && threadIdx.x < 16) reinterpret_cast<uint32_t *>(payload)[threadIdx.x] = hdr.w[threadIdx.x];
+  T *body = reinterpret_cast<T *>(payload + kHdrBytes);
+  const int64_t n8 = E / 8;
+  for (int64_t v = (int64_t)blockIdx.x * kBsThreads + threadIdx.x; v < n8; v += (int64_t)gridDim.x * kBsThreads) {
+    const typename Vec8<T>::Raw r = Vec8<T>::load(a + v * 8);
+    Vec8<T>::store(body + v * 8, r);
+    Vec8<T>::store(prev + v * 8, r);
+  }
+}
 
 template <typename T>
-__global__ void __launch_bounds__(kBsThreads) bs_decode_kernel(const uint8_t *payload, float *ahat, T *recon,
-                                                                int W, int b, int64_t cols, int k, int K,
-                                                                const Header expect, int *status) {
-  __shared__ int slot;
-  const int i = blockIdx.x / b, y = blockIdx.x - (blockIdx.x / b) * b;
+__global__ void __launch_bounds__(kBsThreads) bs_warm_decode_kernel(const uint8_t *payload, T *ahat, T *recon,
+                                                                     int64_t E, const Header expect, int *status) {
   int bad = 0;
   if (threadIdx.x < 16) bad = reinterpret_cast<const uint32_t *>(payload)[threadIdx.x] != expect.w[threadIdx.x];
   if (__syncthreads_or(bad)) {
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, 1);
     return;
   }
-  if (threadIdx.x == 0) {
-    // the slot of block i in the ascending index list (unused slots sort last)
-    const uint32_t *slots = reinterpret_cast<const uint32_t *>(payload + kHdrBytes);
-    int lo = 0, hi = k - 1, found = -1;
-    while (lo <= hi) {
-      const int mid = (lo + hi) >> 1;
-      const uint32_t v = slots[mid];
-      if (v == (uint32_t)i) {
-        found = mid;
-        break;
-      }
-      if (v < (uint32_t)i) lo = mid + 1;
-      else hi = mid - 1;
-    }
-    slot = (i < K) ? found : -1;
+  const T *body = reinterpret_cast<const T *>(payload + kHdrBytes);
+  const int64_t n8 = E / 8;
+  for (int64_t v = (int64_t)blockIdx.x * kBsThreads + threadIdx.x; v < n8; v += (int64_t)gridDim.x * kBsThreads) {
+    const typename Vec8<T>::Raw r = Vec8<T>::load(body + v * 8);
+    Vec8<T>::store(ahat + v * 8, r);
+    Vec8<T>::store(recon + v * 8, r);
   }
+}
+
+// ------------------------------------------------------------------ decode
+
+template <typename T>
+__global__ void __launch_bounds__(kBsThreads) bs_decode_kernel(const uint8_t *payload, T *ahat, T *recon, int W,
+                                                                int b, int64_t cols, int k, int K,
+                                                                const Header expect, int *status) {
+  __shared__ int slot;
+  const int i = blockIdx.x / b, y = blockIdx.x - (blockIdx.x / b) * b;
+  int bad = 0;
+  if (threadIdx.x < 16) bad = reinterpret_cast<const uint32_t *>(payload)[threadIdx.x] != expect.w[threadIdx.x];
+  if (threadIdx.x == 0) slot = -1;
+  if (__syncthreads_or(bad)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, 1);
+    return;
+  }
+  // the slot of block i in the index list (each index appears at most once)
+  const uint32_t *slots = reinterpret_cast<const uint32_t *>(payload + kHdrBytes);
+  for (int j = threadIdx.x; j < k; j += kBsThreads)
+    if (slots[j] == (uint32_t)i && i < K) atomicMax(&slot, j);
   __syncthreads();
   const int64_t e0 = block_row_token(i, y, W, b) * cols;
   const int64_t n8 = (int64_t)b * cols / 8;
@@ -325,17 +395,12 @@ __global__ void __launch_bounds__(kBsThreads) bs_decode_kernel(const uint8_t *pa
                    ((int64_t)slot * b * b + (int64_t)y * b) * cols;
     for (int64_t v = threadIdx.x; v < n8; v += kBsThreads) {
       const typename Vec8<T>::Raw r = Vec8<T>::load(src + v * 8);
-      float x[8];
-      Vec8<T>::to_f32(r, x);
-      store_f32x8(ahat + e0 + v * 8, x);
+      Vec8<T>::store(ahat + e0 + v * 8, r);
       Vec8<T>::store(recon + e0 + v * 8, r);
     }
   } else {
-    for (int64_t v = threadIdx.x; v < n8; v += kBsThreads) {
-      float x[8];
-      load_f32x8(ahat + e0 + v * 8, x);
-      Vec8<T>::store(recon + e0 + v * 8, Vec8<T>::from_f32(x));
-    }
+    for (int64_t v = threadIdx.x; v < n8; v += kBsThreads)
+      Vec8<T>::store(recon + e0 + v * 8, Vec8<T>::load(ahat + e0 + v * 8));
   }
 }
 
@@ -346,6 +411,11 @@ int next_pow2(int x) {
 }
 
 size_t select_smem(int K2) { return (size_t)K2 * (8 + 4 + 1); }
+
+unsigned warm_grid(int64_t E) {
+  const int64_t n = (E / 8 + kBsThreads - 1) / kBsThreads;
+  return (unsigned)(n < 148 * 8 ? (n > 0 ? n : 1) : 148 * 8);
+}
 
 }  // namespace
 
@@ -385,7 +455,7 @@ size_t blocksel_body_bytes(const BlockselPlan &P) {
 }
 
 size_t blocksel_scratch_bytes(const BlockselPlan &P) {
-  return pad256((size_t)P.K) + pad256((size_t)P.K * P.b * 4 * 8) + pad256((size_t)P.k * 4);
+  return pad256((size_t)P.K) + pad256((size_t)P.K * P.b * 4 * 8) + pad256((size_t)P.k * 4) + 256;
 }
 
 int blocksel_bind(BlockselPlan *P, void *scratch) {
@@ -395,48 +465,73 @@ int blocksel_bind(BlockselPlan *P, void *scratch) {
   P->part = reinterpret_cast<double *>(p);
   p += pad256((size_t)P->K * P->b * 4 * 8);
   P->sel = reinterpret_cast<uint32_t *>(p);
-  if (cudaFuncSetAttribute(bs_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)select_smem(next_pow2(P->K))) != cudaSuccess) {
+  p += pad256((size_t)P->k * 4);
+  P->counter = reinterpret_cast<unsigned *>(p);
+  const int sm = (int)select_smem(next_pow2(P->K));
+  if (cudaFuncSetAttribute(bs_encode_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(bs_encode_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess) {
     (void)cudaGetLastError();
     return CF_ERR_CUDA;
   }
   return CF_OK;
 }
 
-cudaError_t blocksel_encode(const BlockselPlan &P, const void *a, float *prev, uint8_t *payload, const Header &hdr,
-                            cudaStream_t st) {
+namespace {
+
+template <typename T>
+cudaError_t encode_t(const BlockselPlan &P, const T *a, T *prev, uint8_t *payload, const Header &hdr,
+                     cudaStream_t st) {
   const int K2 = next_pow2(P.K);
-  const unsigned rows_grid = (unsigned)(P.K * P.b), pack_grid = (unsigned)(P.k * P.b);
-  if (P.dtype == CF_BF16) {
-    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a);
-    launch_pdl(bs_partial_kernel<__nv_bfloat16>, dim3(rows_grid), dim3(kBsThreads), 0, st, x, prev, P.W, P.b, P.cols,
-               P.part);
-    launch_pdl(bs_select_kernel, dim3(1), dim3(kSelThreads), select_smem(K2), st, (const double *)P.part, P.K, K2,
-               P.b, P.k, P.sent, P.sel, payload, hdr);
-    __nv_bfloat16 *data = reinterpret_cast<__nv_bfloat16 *>(payload + kHdrBytes + pad16((size_t)P.k * 4u));
-    launch_pdl(bs_pack_kernel<__nv_bfloat16>, dim3(pack_grid), dim3(kBsThreads), 0, st, x, (const uint32_t *)P.sel,
-               P.W, P.b, P.cols, data);
-  } else {
-    const float *x = static_cast<const float *>(a);
-    launch_pdl(bs_partial_kernel<float>, dim3(rows_grid), dim3(kBsThreads), 0, st, x, prev, P.W, P.b, P.cols, P.part);
-    launch_pdl(bs_select_kernel, dim3(1), dim3(kSelThreads), select_smem(K2), st, (const double *)P.part, P.K, K2,
-               P.b, P.k, P.sent, P.sel, payload, hdr);
-    float *data = reinterpret_cast<float *>(payload + kHdrBytes + pad16((size_t)P.k * 4u));
-    launch_pdl(bs_pack_kernel<float>, dim3(pack_grid), dim3(kBsThreads), 0, st, x, (const uint32_t *)P.sel, P.W,
-               P.b, P.cols, data);
-  }
+  launch_pdl(bs_encode_kernel<T>, dim3((unsigned)(P.K * P.b)), dim3(kBsThreads), select_smem(K2), st, a, prev, P.W,
+             P.b, P.cols, P.K, K2, P.k, P.part, P.counter, P.sent, P.sel, payload, hdr);
+  T *data = reinterpret_cast<T *>(payload + kHdrBytes + pad16((size_t)P.k * 4u));
+  launch_pdl(bs_pack_kernel<T>, dim3((unsigned)(P.k * P.b * kPackSplit)), dim3(kBsThreads), 0, st, a,
+             (const uint32_t *)P.sel, P.W, P.b, P.cols, data);
   return cudaGetLastError();
 }
 
-cudaError_t blocksel_decode(const BlockselPlan &P, const uint8_t *payload, float *ahat, void *recon,
-                            const Header &expect, int *status, cudaStream_t st) {
+}  // namespace
+
+cudaError_t blocksel_encode(const BlockselPlan &P, const void *a, void *prev, uint8_t *payload, const Header &hdr,
+                            bool warm, cudaStream_t st) {
+  const int64_t E = P.rows * P.cols;
+  if (P.dtype == CF_BF16) {
+    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a);
+    __nv_bfloat16 *pv = static_cast<__nv_bfloat16 *>(prev);
+    if (warm) {
+      bs_warm_encode_kernel<__nv_bfloat16><<<warm_grid(E), kBsThreads, 0, st>>>(x, pv, payload, E, hdr);
+      return cudaGetLastError();
+    }
+    return encode_t(P, x, pv, payload, hdr, st);
+  }
+  const float *x = static_cast<const float *>(a);
+  float *pv = static_cast<float *>(prev);
+  if (warm) {
+    bs_warm_encode_kernel<float><<<warm_grid(E), kBsThreads, 0, st>>>(x, pv, payload, E, hdr);
+    return cudaGetLastError();
+  }
+  return encode_t(P, x, pv, payload, hdr, st);
+}
+
+cudaError_t blocksel_decode(const BlockselPlan &P, const uint8_t *payload, void *ahat, void *recon,
+                            const Header &expect, bool warm, int *status, cudaStream_t st) {
+  const int64_t E = P.rows * P.cols;
   const unsigned grid = (unsigned)(P.K * P.b);
-  if (P.dtype == CF_BF16)
-    bs_decode_kernel<__nv_bfloat16><<<grid, kBsThreads, 0, st>>>(payload, ahat, static_cast<__nv_bfloat16 *>(recon),
-                                                                 P.W, P.b, P.cols, P.k, P.K, expect, status);
+  if (P.dtype == CF_BF16) {
+    __nv_bfloat16 *h = static_cast<__nv_bfloat16 *>(ahat), *r = static_cast<__nv_bfloat16 *>(recon);
+    if (warm)
+      bs_warm_decode_kernel<__nv_bfloat16><<<warm_grid(E), kBsThreads, 0, st>>>(payload, h, r, E, expect, status);
+    else
+      bs_decode_kernel<__nv_bfloat16><<<grid, kBsThreads, 0, st>>>(payload, h, r, P.W, P.b, P.cols, P.k, P.K, expect,
+                                                                   status);
+    return cudaGetLastError();
+  }
+  float *h = static_cast<float *>(ahat), *r = static_cast<float *>(recon);
+  if (warm)
+    bs_warm_decode_kernel<float><<<warm_grid(E), kBsThreads, 0, st>>>(payload, h, r, E, expect, status);
   else
-    bs_decode_kernel<float><<<grid, kBsThreads, 0, st>>>(payload, ahat, static_cast<float *>(recon), P.W, P.b, P.cols,
-                                                         P.k, P.K, expect, status);
+    bs_decode_kernel<float><<<grid, kBsThreads, 0, st>>>(payload, h, r, P.W, P.b, P.cols, P.k, P.K, expect, status);
   return cudaGetLastError();
 }
 

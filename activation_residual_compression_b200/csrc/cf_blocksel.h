@@ -27,6 +27,7 @@ struct BlockselPlan {
   uint8_t *sent = nullptr;   // [K] 1 = sent in the current round (part of the state)
   double *part = nullptr;    // [K][b][4] per block row: <p, a>, ||p||^2, ||a||^2, changed
   uint32_t *sel = nullptr;   // [k] this step's blocks, ascending; kBsNone = unused slot
+  unsigned *counter = nullptr;  // CTAs of the current encode that have written their partials
 };
 
 // Checks the configuration and fills the plan; CF_OK or an error code.
@@ -36,12 +37,14 @@ size_t blocksel_body_bytes(const BlockselPlan &P);
 size_t blocksel_scratch_bytes(const BlockselPlan &P);  // sender
 int blocksel_bind(BlockselPlan *P, void *scratch);     // sender; CF_OK or CF_ERR_CUDA
 
-// One selective step (sender): dissimilarities, selection, payload; prev
-// (fp32 [rows][cols], the state) becomes fp32(a).
-cudaError_t blocksel_encode(const BlockselPlan &P, const void *a, float *prev, uint8_t *payload, const Header &hdr,
-                            cudaStream_t st);
-// Receiver: the sent blocks replace ahat's; recon = cast(ahat) everywhere.
-cudaError_t blocksel_decode(const BlockselPlan &P, const uint8_t *payload, float *ahat, void *recon,
-                            const Header &expect, int *status, cudaStream_t st);
+// One step (sender).  warm: the payload is a itself.  Otherwise the
+// dissimilarities, the selection and the payload.  Either way prev ([rows]
+// [cols] in the activation dtype, the state) becomes a.
+cudaError_t blocksel_encode(const BlockselPlan &P, const void *a, void *prev, uint8_t *payload, const Header &hdr,
+                            bool warm, cudaStream_t st);
+// Receiver: warm, ahat = recon = the payload; otherwise the sent blocks
+// replace ahat's and recon = ahat everywhere (ahat in the activation dtype).
+cudaError_t blocksel_decode(const BlockselPlan &P, const uint8_t *payload, void *ahat, void *recon,
+                            const Header &expect, bool warm, int *status, cudaStream_t st);
 
 }  // namespace cfi

@@ -81,6 +81,39 @@ class ActivationStream:
         return out
 
 
+class BlockStream(ActivationStream):
+    """A random walk whose innovation scale is constant within each b x b block
+    of an H x W token grid (rows = H*W, raster order) and log-uniform over
+    blocks in [lo, hi]: the changes between steps concentrate in a few regions."""
+
+    def __init__(self, H, W, cols, *, block=8, lo=0.01, hi=0.3, dtype=torch.bfloat16, device="cpu", seed=0):
+        super().__init__(H * W, cols, dtype=dtype, device=device, seed=seed, sigma=1.0, seed_per_tensor=[seed])
+        g = torch.Generator().manual_seed(int(seed) + 1)
+        K = (H // block) * (W // block)
+        u = torch.rand(K, generator=g, dtype=torch.float64)
+        scale = torch.exp(math.log(lo) + u * (math.log(hi) - math.log(lo))).to(torch.float32)
+        grid = scale.reshape(H // block, W // block).repeat_interleave(block, 0).repeat_interleave(block, 1)
+        self.row_scale = grid.reshape(H * W, 1).to(self.device)
+
+    def next(self, out: torch.Tensor | None = None) -> torch.Tensor:
+        z = self._normal(0)
+        if self.t == 0:
+            self.state[0] = z
+        else:
+            self.state[0].add_(z * self.row_scale)
+        self.t += 1
+        if out is None:
+            return self.state.to(self.dtype, copy=True)
+        out.copy_(self.state)
+        return out
+
+
+def blocksel(device="cpu", H=64, W=64, cols=3072, block=8, seed=4):
+    """Token-grid stream for the block-selection mode: 64 x 64 tokens x 3072
+    channels bf16, per-8x8-block innovation scales log-uniform in [0.01, 0.3]."""
+    return BlockStream(H, W, cols, block=block, device=device, seed=seed)
+
+
 def tiny(device="cpu"):
     """256 x 64 fp32 random walk, sigma 0.1, seed 0."""
     return ActivationStream(256, 64, dtype=torch.float32, device=device, seed=0, sigma=0.1,

@@ -57,6 +57,8 @@ WORKLOADS = {
                      codecs=[("lowrank", {"rank": 70, "iters": 2, "lr_int4": 1, "seed": 7})]),
     "cogvideox": dict(name="cogvideox2b-60x17550x1920-bf16", rows=17550, cols=1920, batch=60, stream="cogvideox",
                       codecs=[("q2", {})]),
+    "blocksel": dict(name="otil-grid64x64-3072ch-bf16-b8-k16", rows=4096, cols=3072, batch=1, stream="blocksel",
+                     codecs=[("blocksel", {"bs_grid_h": 64, "bs_block": 8, "bs_k": 16, "bs_warm": 5})]),
 }
 
 
@@ -80,21 +82,40 @@ def _payload_body(mode, rows, cols, kw):
         return pad(rows * cols // m * n * 2) + pad(rows * (cols // m * n * (m.bit_length() - 1) // 32) * 4)
     if mode == "identity":
         return rows * cols * 4
+    if mode == "blocksel":
+        b, k = kw["bs_block"], kw["bs_k"]
+        return pad(4 * k) + k * b * b * cols * 2
     raise ValueError(mode)
+
+
+def _bs_frac(rows, kw):
+    H = kw["bs_grid_h"]
+    K = (H // kw["bs_block"]) * ((rows // H) // kw["bs_block"])
+    return kw["bs_k"] / K
 
 
 def encode_bytes(mode, rows, cols, kw, act_size=2, ef="explicit"):
     """Algorithmic bytes of one encode launch: read a, ahat, e; write ahat, e, payload.
-    Implicit feedback does not read e; without feedback e is neither read nor written."""
+    Implicit feedback does not read e; without feedback e is neither read nor written.
+    Block selection: read a and the previous activation (kept in the
+    activation dtype), write it, and read + write the sent fraction f of a into
+    the payload."""
     E = rows * cols
+    if mode == "blocksel":
+        return int(E * 3 * act_size + 2 * _bs_frac(rows, kw) * E * act_size) + 64 + 16
     e_rd = 4 if ef == "explicit" else 0
     e_wr = 0 if ef == "off" else 4
     return E * (act_size + 4 + e_rd + 4 + e_wr) + 64 + _payload_body(mode, rows, cols, kw)
 
 
 def decode_bytes(mode, rows, cols, kw, act_size=2):
-    """Algorithmic bytes of one decode launch: read payload, ahat; write ahat, recon."""
+    """Algorithmic bytes of one decode launch: read payload, ahat; write ahat, recon.
+    Block selection (state in the activation dtype): unsent blocks read ahat and
+    write recon; sent blocks read the payload and write ahat and recon."""
     E = rows * cols
+    if mode == "blocksel":
+        f = _bs_frac(rows, kw)
+        return int(E * ((1 - f) * 2 * act_size + f * 3 * act_size)) + 64
     return E * (4 + 4 + act_size) + 64 + _payload_body(mode, rows, cols, kw)
 
 
@@ -180,6 +201,8 @@ EF_CODES = {"explicit": 0, "implicit": 1, "off": 2}
 
 
 def _codec_name(mode, kw):
+    if mode == "blocksel":
+        return f"blocksel_b{kw['bs_block']}_k{kw['bs_k']}"
     if mode == "nm":
         return f"nm{kw['nm_n']}_{kw['nm_m']}"
     if mode == "lowrank":
@@ -195,6 +218,8 @@ def _make_stream(kind, wl, seed, device="cuda"):
         return inputs.ar1(device, rows=wl["rows"], cols=wl["cols"], seed=seed)
     if kind == "cogvideox":
         return inputs.cogvideox(device, rows=wl["rows"], cols=wl["cols"], n_tensors=wl["batch"])
+    if kind == "blocksel":
+        return inputs.blocksel(device, H=64, W=wl["rows"] // 64, cols=wl["cols"], seed=seed)
     raise ValueError(kind)
 
 
@@ -208,6 +233,8 @@ def step_bytes(mode, rows, cols, kw, payload, ef="explicit"):
 
 def launches_per_call(mode, kw, encode):
     """libcf kernels one steady-state cf_encode / cf_decode call launches."""
+    if mode == "blocksel":
+        return 3 if encode else 1                 # block sums, selection, pack; decode
     if mode != "lowrank":
         return 1
     if not encode:
@@ -273,8 +300,11 @@ def run_cf(args, rank, world, device):
     if world > 1:
         import torch.distributed as dist
 
+    # untimed steps: at least the warm-up, and past every codec's full-size
+    # leading steps (block selection sends bs_warm steps in full)
+    W_run = max([W] + [kw.get("bs_warm", 1) for _, kw in wl["codecs"]])
     with torch.cuda.stream(stream):
-        for i in range(W):
+        for i in range(W_run):
             step(i)
     torch.cuda.synchronize()
     if dist:
@@ -288,7 +318,7 @@ def run_cf(args, rank, world, device):
     t1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         t0.record(stream)
-        for i in range(W, W + K):
+        for i in range(W_run, W_run + K):
             step(i, evs)
         t1.record(stream)
     torch.cuda.synchronize()
@@ -327,7 +357,7 @@ def run_cf(args, rank, world, device):
                 host_out[ci].copy_(c["rec"], non_blocking=True)
 
         with torch.cuda.stream(stream):
-            for _ in range(3):
+            for _ in range(max(3, W_run)):
                 e2e_step()
         torch.cuda.synchronize()
         if dist:
@@ -571,6 +601,63 @@ def run_lr_sweep(args, device, T=50, ef="implicit"):
                       "steps": T, "data": "synthetic"}), flush=True)
 
 
+def _oracle_kw(mode, kw):
+    """The oracle's names for a codec's parameters."""
+    if mode == "blocksel":
+        return {"bs_h": kw["bs_grid_h"], "bs_block": kw["bs_block"], "bs_k": kw["bs_k"], "bs_warm": kw["bs_warm"]}
+    return kw
+
+
+BS_STUDY_K = (4, 8, 16, 32, 64)   # of K = 64 blocks: k/K = 1/16, 1/8, 1/4, 1/2, 1
+
+
+def run_bs_study(args, device, T=50):
+    """Block selection (Otil page, "Ablation: transmitted fraction k/K"): receiver
+    error and step time of the CUDA codec on the block-scaled random walk
+    (64 x 64 tokens x 3072 channels bf16, 8 x 8 blocks) for several k."""
+    import torch
+
+    import activation_residual_compression_b200 as cf
+    from activation_residual_compression_b200 import inputs
+    torch.cuda.set_device(device)
+    rows, cols = 4096, 3072
+    out = []
+    for k in BS_STUDY_K:
+        kw = {"bs_grid_h": 64, "bs_block": 8, "bs_k": k, "bs_warm": 5}
+        base = dict(dtype=cf.CF_BF16, **kw)
+        S = cf.cf_create(rows, cols, cf.MODE_NAMES["blocksel"], cf.cf_params_init(role=cf.CF_SENDER, **base))
+        R = cf.cf_create(rows, cols, cf.MODE_NAMES["blocksel"], cf.cf_params_init(role=cf.CF_RECEIVER, **base))
+        P = cf.cf_payload_bytes(S, False)
+        pay = torch.empty(max(cf.cf_payload_bytes(S, True), P), dtype=torch.uint8, device="cuda")
+        rec = torch.empty(1, rows, cols, dtype=torch.bfloat16, device="cuda")
+        s = inputs.blocksel("cuda", seed=1)
+        rel, ms = [], []
+        for t in range(T):
+            a = s.next()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            cf.cf_encode(S, a, pay)
+            cf.cf_decode(R, pay, rec)
+            e1.record()
+            af = a.float()
+            rel.append(float(torch.linalg.vector_norm(rec.float() - af) / torch.linalg.vector_norm(af)))
+            torch.cuda.synchronize()
+            if t >= kw["bs_warm"] + 2:
+                ms.append(e0.elapsed_time(e1))
+        if cf.cf_status(R) != cf.CF_OK:
+            raise RuntimeError(f"k {k}: codec reported an error status")
+        cf.cf_destroy(S)
+        cf.cf_destroy(R)
+        out.append({"k": k, "k_over_K": f"{k}/64", "payload_bytes": P, "ratio_vs_bf16": round(rows * cols * 2 / P, 2),
+                    "rel_err": {str(t): round(rel[t], 5) for t in EF_STUDY_STEPS},
+                    "steady_rel_err": round(statistics.mean(rel[T // 2:]), 5),
+                    "ms_per_step": round(statistics.median(ms), 4)})
+    print(json.dumps({"bs_study": out, "metric": "receiver relative L2 error ||recon_t - a_t|| / ||a_t||",
+                      "stream": "random walk, per-8x8-block innovation scale log-uniform in [0.01, 0.3]",
+                      "steps": T, "data": "synthetic"}), flush=True)
+
+
 def cpu_baseline(wl=None, max_seconds=20.0):
     """The CPU oracle, as it stands, on the same workload (full-size tensors;
     for the 60-tensor step the first tensors only, tensors being independent),
@@ -593,9 +680,10 @@ def cpu_baseline(wl=None, max_seconds=20.0):
                                         sigma_per_tensor=inputs.cogvideox_sigmas(B_)[:1])
         else:
             s = _make_stream(wl["stream"], wl, seed=1 + 100 * mi, device="cpu")
-        o = oracle.Oracle(R_, C_, mode, dtype="bf16", batch=nt, **kw)
-        a = s.next().view(torch.int16).numpy().view(np.uint16)
-        o.decode(o.encode(a))
+        o = oracle.Oracle(R_, C_, mode, dtype="bf16", batch=nt, **_oracle_kw(mode, kw))
+        for _ in range(kw.get("bs_warm", 1)):     # the full-size leading steps, untimed
+            a = s.next().view(torch.int16).numpy().view(np.uint16)
+            o.decode(o.encode(a))
         orcs.append((s, o))
     spent, steps = 0.0, 0
     while spent < max_seconds and steps < 27:
@@ -627,8 +715,8 @@ def run_reference(args):
 
     wl = WORKLOADS[args.workload]
     R_, C_ = wl["rows"], wl["cols"]
-    lowrank = any(m == "lowrank" for m, _ in wl["codecs"])
-    rows = R_ if lowrank else 1152
+    coupled = any(m in ("lowrank", "blocksel") for m, _ in wl["codecs"])   # rows not independent
+    rows = R_ if coupled else 1152
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     orcs = []
     for mi, (mode, kw) in enumerate(wl["codecs"]):
@@ -638,7 +726,7 @@ def run_reference(args):
                                         sigma_per_tensor=inputs.cogvideox_sigmas(wl["batch"])[:1])
         else:
             s = _make_stream(wl["stream"], sub, seed=1 + 100 * mi, device="cpu")
-        orcs.append((s, oracle.Oracle(rows, C_, mode, dtype="bf16", **kw)))
+        orcs.append((s, oracle.Oracle(rows, C_, mode, dtype="bf16", **_oracle_kw(mode, kw))))
 
     def one():
         ins = [s.next().view(torch.int16).numpy().view(np.uint16) for s, _ in orcs]
@@ -647,7 +735,8 @@ def run_reference(args):
             o.decode(o.encode(a))
         return time.perf_counter() - t
 
-    one()  # the stream's raw first step
+    for _ in range(max([1] + [kw.get("bs_warm", 1) for _, kw in wl["codecs"]])):
+        one()  # the stream's full-size leading steps
     for _ in range(args.warmup):
         one()
     spent = sum(one() for _ in range(args.steps))
@@ -685,6 +774,8 @@ def main():
                     help="instead of timing: receiver error per step of every mode and feedback form")
     ap.add_argument("--lr-sweep", action="store_true",
                     help="instead of timing: low-rank receiver error over rank, sweeps and factor precision")
+    ap.add_argument("--bs-study", action="store_true",
+                    help="instead of timing: block-selection receiver error and step time over k/K")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -701,9 +792,9 @@ def main():
     import torch
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
-    if args.ef_study or args.lr_sweep:
+    if args.ef_study or args.lr_sweep or args.bs_study:
         if rank == 0:
-            (run_ef_study if args.ef_study else run_lr_sweep)(args, local)
+            (run_ef_study if args.ef_study else run_lr_sweep if args.lr_sweep else run_bs_study)(args, local)
         return
     dist = None
     if world > 1:
@@ -732,6 +823,10 @@ def main():
         E = R_ * C_
         enc_alg = E * (2 + 16 + 4 * c0["kw"]["iters"]) + c0["P"]
         kern = f"cf_encode low-rank ({launches_per_call(c0['mode'], c0['kw'], True)} launches)"
+        tr = None
+    elif c0["mode"] == "blocksel":
+        enc_alg = encode_bytes(c0["mode"], R_, C_, c0["kw"])
+        kern = f"cf_encode block selection ({launches_per_call(c0['mode'], c0['kw'], True)} launches)"
         tr = None
     else:
         enc_alg = B_ * encode_bytes(c0["mode"], R_, C_, c0["kw"], ef=args.ef)

@@ -42,6 +42,8 @@ class GpuPair:
                   ef={"explicit": cf.CF_EF_EXPLICIT, "implicit": cf.CF_EF_IMPLICIT, "off": cf.CF_EF_OFF}[ef],
                   nm_n=nm_n, nm_m=nm_m, batch=batch, rank=rank, iters=iters, lr_int4=lr_int4, seed=seed, **extra)
         self.has_err = mode != "blocksel"       # block selection keeps no error term
+        # block selection keeps its state (raw activations) in the activation dtype
+        self.state_esz = (2 if dtype == "bf16" else 4) if mode == "blocksel" else 4
         self.S = cf.cf_create(rows, cols, self.mode, cf.cf_params_init(role=cf.CF_SENDER, **kw))
         self.R = cf.cf_create(rows, cols, self.mode, cf.cf_params_init(role=cf.CF_RECEIVER, **kw))
         self.pb_warm = cf.cf_payload_bytes(self.S, True)
@@ -74,7 +76,11 @@ class GpuPair:
         tb = int(buf[80:88].view(np.uint64)[0])
         ten = buf[len(buf) - tb:]
         n = self.batch * self.rows * self.cols
-        ahat = ten[:4 * n].view(np.float32).reshape(self.batch, self.rows, self.cols)
+        if self.state_esz == 2:
+            ahat = (ten[:2 * n].view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+            ahat = ahat.reshape(self.batch, self.rows, self.cols)
+        else:
+            ahat = ten[:4 * n].view(np.float32).reshape(self.batch, self.rows, self.cols)
         err = None
         if which == "S" and self.has_err:
             err = ten[4 * n:8 * n].view(np.float32).reshape(self.batch, self.rows, self.cols)
@@ -88,7 +94,7 @@ class GpuPair:
         buf = self.export("S")
         tb = int(buf[80:88].view(np.uint64)[0])
         ten = buf[len(buf) - tb:]
-        return ten[4 * self.batch * self.rows * self.cols:].copy()
+        return ten[self.state_esz * self.batch * self.rows * self.cols:].copy()
 
     def guards_ok(self) -> bool:
         return canaries_intact(self.pay_whole) and canaries_intact(self.rec_whole)
