@@ -56,6 +56,7 @@ class cf_params(ctypes.Structure):
         ("bs_block", ctypes.c_int),
         ("bs_k", ctypes.c_int),
         ("bs_warm", ctypes.c_int),
+        ("state_dtype", ctypes.c_int),
     ]
 
 

@@ -128,6 +128,9 @@ int validate(int64_t rows, int64_t cols, int mode, const cf_params *p) {
     if (cols % p->nm_m) return CF_ERR_SHAPE;
     if (((cols / p->nm_m) * p->nm_n * ilog2(p->nm_m)) % 32) return CF_ERR_SHAPE;
   }
+  if (p->state_dtype != CF_F32 && p->state_dtype != CF_BF16) return CF_ERR_ARG;
+  if (p->state_dtype == CF_BF16 && (p->dtype != CF_BF16 || mode == CF_LOWRANK || mode == CF_BLOCKSEL))
+    return CF_ERR_UNSUPPORTED;  // the bf16 state is an option of the streaming modes on bf16 activations
   if (mode == CF_BLOCKSEL) {
     BlockselPlan bp{};
     const int rc = bs_plan_of(rows, cols, *p, &bp);
@@ -157,11 +160,12 @@ Carve carve_of(int64_t rows, int64_t cols, int mode, const cf_params &p, const L
   size_t off = 0;
   c.status = off;
   off += 256;
+  const size_t esz = p.state_dtype == CF_BF16 ? 2u : 4u;
   c.ahat = off;
-  off += pad256(E * 4u);
+  off += pad256(E * esz);
   if (p.role == CF_SENDER && mode != CF_BLOCKSEL) {  // block selection keeps no error term
     c.err = off;
-    off += pad256(E * 4u);
+    off += pad256(E * esz);
     if (mode == CF_LOWRANK) {
       c.vprev = off;
       off += pad256((size_t)cols * p.rank * 4u * p.batch);
@@ -219,7 +223,10 @@ uint64_t warm_steps(const cf_state *s) { return s->mode == CF_BLOCKSEL ? (uint64
 
 // bytes per element of the ahat tensor: fp32, except block selection, whose
 // state holds raw activations in their own dtype
-size_t ahat_elem_bytes(const cf_state *s) { return s->mode == CF_BLOCKSEL ? act_size(s->p.dtype) : 4u; }
+size_t ahat_elem_bytes(const cf_state *s) {
+  if (s->mode == CF_BLOCKSEL) return act_size(s->p.dtype);
+  return s->p.state_dtype == CF_BF16 ? 2u : 4u;
+}
 
 EncArgs enc_args(cf_state *s, const void *a, void *payload, bool warm) {
   EncArgs A{};
@@ -348,7 +355,7 @@ struct ExportHeader {
   int32_t mode, dtype, role, ef, nm_n, nm_m, rank, iters, lr_int4, batch;
   uint64_t step;
   int32_t status;
-  int32_t pad;
+  int32_t state_dtype;
   uint64_t tensor_bytes;
 };
 
@@ -394,6 +401,7 @@ int cf_params_init(cf_params *p) {
   p->bs_block = 8;
   p->bs_k = 0;
   p->bs_warm = 5;
+  p->state_dtype = CF_F32;
   return CF_OK;
 }
 
@@ -430,7 +438,7 @@ int cf_create(int64_t rows, int64_t cols, int mode, const cf_params *p, cf_state
   if (mode == CF_BLOCKSEL) bs_plan_of(rows, cols, *p, &s->bs);
   s->lay = layout_of(rows, cols, mode, *p);
   const int rc = stream_config(mode, p->dtype, p->nm_m, p->nm_n, rows, cols, p->batch, s->sm_count,
-                               p->ef == CF_EF_EXPLICIT, &s->cfg);
+                               p->state_dtype == CF_BF16, &s->cfg);
   if (rc != CF_OK) {
     delete s;
     return rc;
@@ -547,7 +555,7 @@ int cf_tensor(cf_state *s, int which, void **dptr, size_t *bytes) {
     case CF_T_ERROR:
       if (!s->err) return CF_ERR_ROLE;
       *dptr = s->err;
-      *bytes = E * 4u;
+      *bytes = E * ahat_elem_bytes(s);
       return CF_OK;
     case CF_T_VPREV:
       if (!s->vprev) return CF_ERR_ROLE;
@@ -576,7 +584,7 @@ int cf_reset(cf_state *s) {
 static size_t export_tensor_bytes(const cf_state *s) {
   const size_t E = (size_t)(s->rows * s->cols) * (size_t)s->p.batch;
   size_t b = E * ahat_elem_bytes(s);
-  if (s->err) b += E * 4u;
+  if (s->err) b += E * ahat_elem_bytes(s);
   if (s->vprev) b += (size_t)s->cols * s->p.rank * 4u * s->p.batch;
   if (s->bs.sent) b += (size_t)s->bs.K;
   return b;
@@ -599,7 +607,7 @@ int cf_state_export(const cf_state *s, void *host, size_t bytes, void *stream) {
   h.magic = kExportMagic;
   h.rows = s->rows; h.cols = s->cols; h.mode = s->mode; h.dtype = s->p.dtype; h.role = s->p.role;
   h.ef = s->p.ef; h.nm_n = s->p.nm_n; h.nm_m = s->p.nm_m; h.rank = s->p.rank; h.iters = s->p.iters;
-  h.lr_int4 = s->p.lr_int4; h.batch = s->p.batch; h.step = s->step;
+  h.lr_int4 = s->p.lr_int4; h.batch = s->p.batch; h.step = s->step; h.state_dtype = s->p.state_dtype;
   h.tensor_bytes = export_tensor_bytes(s);
   if (cudaMemcpy(&h.status, s->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_err(cudaErrorUnknown);
   uint8_t *dst = static_cast<uint8_t *>(host);
@@ -610,8 +618,8 @@ int cf_state_export(const cf_state *s, void *host, size_t bytes, void *stream) {
   if (cudaMemcpy(dst, s->ahat, hb, cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_err(cudaErrorUnknown);
   dst += hb;
   if (s->err) {
-    if (cudaMemcpy(dst, s->err, E * 4u, cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_err(cudaErrorUnknown);
-    dst += E * 4u;
+    if (cudaMemcpy(dst, s->err, hb, cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_err(cudaErrorUnknown);
+    dst += hb;
   }
   if (s->vprev) {
     const size_t vb = (size_t)s->cols * s->p.rank * 4u * s->p.batch;
@@ -633,7 +641,7 @@ int cf_state_import(cf_state *s, const void *host, size_t bytes, void *stream) {
   if (h.magic != kExportMagic || h.rows != s->rows || h.cols != s->cols || h.mode != s->mode ||
       h.dtype != s->p.dtype || h.role != s->p.role || h.ef != s->p.ef || h.nm_n != s->p.nm_n ||
       h.nm_m != s->p.nm_m || h.rank != s->p.rank || h.iters != s->p.iters || h.lr_int4 != s->p.lr_int4 ||
-      h.batch != s->p.batch || h.tensor_bytes != export_tensor_bytes(s))
+      h.batch != s->p.batch || h.state_dtype != s->p.state_dtype || h.tensor_bytes != export_tensor_bytes(s))
     return CF_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return cuda_err(cudaErrorUnknown);
@@ -643,8 +651,8 @@ int cf_state_import(cf_state *s, const void *host, size_t bytes, void *stream) {
   if (cudaMemcpy(s->ahat, src, hb, cudaMemcpyHostToDevice) != cudaSuccess) return cuda_err(cudaErrorUnknown);
   src += hb;
   if (s->err) {
-    if (cudaMemcpy(s->err, src, E * 4u, cudaMemcpyHostToDevice) != cudaSuccess) return cuda_err(cudaErrorUnknown);
-    src += E * 4u;
+    if (cudaMemcpy(s->err, src, hb, cudaMemcpyHostToDevice) != cudaSuccess) return cuda_err(cudaErrorUnknown);
+    src += hb;
   }
   if (s->vprev) {
     const size_t vb = (size_t)s->cols * s->p.rank * 4u * s->p.batch;

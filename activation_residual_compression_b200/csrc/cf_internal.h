@@ -77,11 +77,12 @@ struct StreamCfg {
   int enc_grid;
   int dec_grid;
   int warm_grid;
+  bool state_bf16;  // ahat and e stored as bf16 (the bf16-state option)
 };
 
 // ---- streaming kernels (cf_stream.cu) ----
 int stream_config(int mode, int dtype, int nm_m, int nm_n, int64_t rows, int64_t cols, int batch,
-                  int sm_count, int ef_explicit, StreamCfg *cfg);
+                  int sm_count, int state_bf16, StreamCfg *cfg);
 cudaError_t launch_encode(int mode, int dtype, int nm_m, int nm_n, const StreamCfg &cfg,
                           const EncArgs &args, const PtrTable *tab, cudaStream_t st);
 cudaError_t launch_decode(int mode, int dtype, int nm_m, int nm_n, const StreamCfg &cfg,

@@ -38,30 +38,35 @@ namespace {
 
 // ---------------------------------------------------------------- dispatch
 
-const void *kernel_any(bool enc, int mode, int dtype, int nm_m, int nm_n, int vpt, bool table) {
+const void *kernel_any(bool enc, int mode, int dtype, int nm_m, int nm_n, int vpt, bool table, bool sb) {
   switch (mode) {
-    case CF_IDENTITY: return stream_kernel_id(enc, dtype, nm_m, nm_n, vpt, table);
-    case CF_SIGN1: return stream_kernel_s1(enc, dtype, nm_m, nm_n, vpt, table);
-    case CF_Q2: return stream_kernel_q2(enc, dtype, nm_m, nm_n, vpt, table);
-    case CF_NM: return stream_kernel_nm(enc, dtype, nm_m, nm_n, vpt, table);
+    case CF_IDENTITY: return stream_kernel_id(enc, dtype, nm_m, nm_n, vpt, table, sb);
+    case CF_SIGN1: return stream_kernel_s1(enc, dtype, nm_m, nm_n, vpt, table, sb);
+    case CF_Q2: return stream_kernel_q2(enc, dtype, nm_m, nm_n, vpt, table, sb);
+    case CF_NM: return stream_kernel_nm(enc, dtype, nm_m, nm_n, vpt, table, sb);
   }
   return nullptr;
 }
 
-template <typename T, typename Tab>
+template <typename T, typename Tab, typename S>
 const void *warm_for(bool enc, int vpt) {
   switch (vpt) {
-    case 1: return enc ? (const void *)&warm_encode_kernel<T, 1, Tab> : (const void *)&warm_decode_kernel<T, 1, Tab>;
-    case 2: return enc ? (const void *)&warm_encode_kernel<T, 2, Tab> : (const void *)&warm_decode_kernel<T, 2, Tab>;
-    case 3: return enc ? (const void *)&warm_encode_kernel<T, 3, Tab> : (const void *)&warm_decode_kernel<T, 3, Tab>;
-    case 4: return enc ? (const void *)&warm_encode_kernel<T, 4, Tab> : (const void *)&warm_decode_kernel<T, 4, Tab>;
+    case 1: return enc ? (const void *)&warm_encode_kernel<T, 1, Tab, S> : (const void *)&warm_decode_kernel<T, 1, Tab, S>;
+    case 2: return enc ? (const void *)&warm_encode_kernel<T, 2, Tab, S> : (const void *)&warm_decode_kernel<T, 2, Tab, S>;
+    case 3: return enc ? (const void *)&warm_encode_kernel<T, 3, Tab, S> : (const void *)&warm_decode_kernel<T, 3, Tab, S>;
+    case 4: return enc ? (const void *)&warm_encode_kernel<T, 4, Tab, S> : (const void *)&warm_decode_kernel<T, 4, Tab, S>;
   }
   return nullptr;
 }
 
-const void *warm_any(bool enc, int dtype, int vpt, bool table) {
-  if (dtype == CF_BF16) return table ? warm_for<__nv_bfloat16, PtrTable>(enc, vpt) : warm_for<__nv_bfloat16, NoTable>(enc, vpt);
-  return table ? warm_for<float, PtrTable>(enc, vpt) : warm_for<float, NoTable>(enc, vpt);
+const void *warm_any(bool enc, int dtype, int vpt, bool table, bool sb) {
+  if (dtype == CF_BF16) {
+    if (sb) return table ? warm_for<__nv_bfloat16, PtrTable, __nv_bfloat16>(enc, vpt)
+                         : warm_for<__nv_bfloat16, NoTable, __nv_bfloat16>(enc, vpt);
+    return table ? warm_for<__nv_bfloat16, PtrTable, float>(enc, vpt) : warm_for<__nv_bfloat16, NoTable, float>(enc, vpt);
+  }
+  if (sb) return nullptr;
+  return table ? warm_for<float, PtrTable, float>(enc, vpt) : warm_for<float, NoTable, float>(enc, vpt);
 }
 
 template <typename Args>
@@ -89,8 +94,8 @@ int occupancy(const void *fn, size_t smem) {
 // 128 threads per row, then wider teams), then size each persistent grid as
 // (resident blocks per SM) x (SM count), capped by the number of row groups.
 int stream_config(int mode, int dtype, int nm_m, int nm_n, int64_t rows, int64_t cols, int batch, int sm_count,
-                  int ef_explicit, StreamCfg *cfg) {
-  (void)ef_explicit;
+                  int state_bf16, StreamCfg *cfg) {
+  cfg->state_bf16 = state_bf16 != 0;
   const int64_t V = cols / 8;
   int best_t = -1, best_v = 0;
   int64_t best_key[3] = {0, 0, 0};
@@ -118,34 +123,36 @@ int stream_config(int mode, int dtype, int nm_m, int nm_n, int64_t rows, int64_t
   auto cap = [&](int64_t g) -> int { return (int)(g < n_rg ? g : n_rg); };
   cfg->enc_grid = cfg->dec_grid = 1;
   if (mode != CF_LOWRANK && mode != CF_BLOCKSEL) {
-    const void *efn = kernel_any(true, mode, dtype, nm_m, nm_n, best_v, false);
-    const void *dfn = kernel_any(false, mode, dtype, nm_m, nm_n, best_v, false);
+    const void *efn = kernel_any(true, mode, dtype, nm_m, nm_n, best_v, false, cfg->state_bf16);
+    const void *dfn = kernel_any(false, mode, dtype, nm_m, nm_n, best_v, false, cfg->state_bf16);
     if (!efn || !dfn) return CF_ERR_UNSUPPORTED;
     cfg->enc_grid = cap((int64_t)occupancy(efn, 0) * sm_count);
     cfg->dec_grid = cap((int64_t)occupancy(dfn, 0) * sm_count);
   }
-  cfg->warm_grid = cap((int64_t)occupancy(warm_any(true, dtype, best_v, false), 0) * sm_count);
+  const void *wfn = warm_any(true, dtype, best_v, false, cfg->state_bf16);
+  if (!wfn) return CF_ERR_UNSUPPORTED;
+  cfg->warm_grid = cap((int64_t)occupancy(wfn, 0) * sm_count);
   return CF_OK;
 }
 
 cudaError_t launch_encode(int mode, int dtype, int nm_m, int nm_n, const StreamCfg &cfg, const EncArgs &args,
                           const PtrTable *tab, cudaStream_t st) {
-  return launch(kernel_any(true, mode, dtype, nm_m, nm_n, cfg.vpt, tab != nullptr), cfg.enc_grid, 0, args, tab, st);
+  return launch(kernel_any(true, mode, dtype, nm_m, nm_n, cfg.vpt, tab != nullptr, cfg.state_bf16), cfg.enc_grid, 0, args, tab, st);
 }
 
 cudaError_t launch_decode(int mode, int dtype, int nm_m, int nm_n, const StreamCfg &cfg, const DecArgs &args,
                           const PtrTable *tab, cudaStream_t st) {
-  return launch(kernel_any(false, mode, dtype, nm_m, nm_n, cfg.vpt, tab != nullptr), cfg.dec_grid, 0, args, tab, st);
+  return launch(kernel_any(false, mode, dtype, nm_m, nm_n, cfg.vpt, tab != nullptr, cfg.state_bf16), cfg.dec_grid, 0, args, tab, st);
 }
 
 cudaError_t launch_warm_encode(int dtype, const StreamCfg &cfg, const EncArgs &args, const PtrTable *tab,
                                cudaStream_t st) {
-  return launch(warm_any(true, dtype, cfg.vpt, tab != nullptr), cfg.warm_grid, 0, args, tab, st);
+  return launch(warm_any(true, dtype, cfg.vpt, tab != nullptr, cfg.state_bf16), cfg.warm_grid, 0, args, tab, st);
 }
 
 cudaError_t launch_warm_decode(int dtype, const StreamCfg &cfg, const DecArgs &args, const PtrTable *tab,
                                cudaStream_t st) {
-  return launch(warm_any(false, dtype, cfg.vpt, tab != nullptr), cfg.warm_grid, 0, args, tab, st);
+  return launch(warm_any(false, dtype, cfg.vpt, tab != nullptr, cfg.state_bf16), cfg.warm_grid, 0, args, tab, st);
 }
 
 }  // namespace cfi

@@ -122,6 +122,20 @@ __device__ __forceinline__ void store_f32x8(float *p, const float (&x)[8]) {
   __stcs(q + 1, make_float4(x[4], x[5], x[6], x[7]));
 }
 
+// The codec state (ahat, e) is fp32, or bf16 when the caller asks for the
+// bf16-state option: loads widen exactly, stores round to nearest even.
+template <typename S>
+__device__ __forceinline__ void load_state8(const S *p, float4 (&r)[2]) {
+  float x[8];
+  Act<S>::to_f32(Act<S>::load(p), x);
+  r[0] = make_float4(x[0], x[1], x[2], x[3]);
+  r[1] = make_float4(x[4], x[5], x[6], x[7]);
+}
+template <typename S>
+__device__ __forceinline__ void store_state8(S *p, const float (&x)[8]) {
+  Act<S>::store_f32(p, x);
+}
+
 template <typename T, typename Tab>
 __device__ __forceinline__ const T *act_tensor(const void *base, const Tab &tab, int64_t b, int64_t E);
 template <>
@@ -318,9 +332,9 @@ __device__ __forceinline__ void zero_padding(const EncArgs &A) {
 // encode, payload stores, e = D - C and ahat = ahat + C stores (with
 // CF_EF_OFF: ahat = fp32(a) and no e store).  Every thread
 // of the block calls this together (team reductions use __syncthreads).
-template <int MODE, typename T, int VPT, int NM_M, int NM_N>
+template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename S>
 __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const int tlog, const bool row_ok,
-                                           const int64_t r, float *hrow, float *erow, uint8_t *body,
+                                           const int64_t r, S *hrow, S *erow, uint8_t *body,
                                            const typename Act<T>::Raw (&ra)[VPT], const float4 (&rh)[VPT][2],
                                            const float4 (&re)[VPT][2], float *sm_f, unsigned long long *sm_u) {
   using P = Pack<MODE, NM_M, NM_N>;
@@ -573,8 +587,8 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
         en[k] = __fsub_rn(d[j][k], c[j][k]);
         hn[k] = A.ef_off ? h[j][k] : __fadd_rn(h[j][k], c[j][k]);
       }
-      if (!A.ef_off) store_f32x8(erow + v * 8, en);
-      store_f32x8(hrow + v * 8, hn);
+      if (!A.ef_off) store_state8(erow + v * 8, en);
+      store_state8(hrow + v * 8, hn);
     }
   }
 }
@@ -585,7 +599,7 @@ struct EncMinBlocks {
   static constexpr int value = (MODE == CF_Q2 || VPT <= 2) ? 3 : 2;
 };
 
-template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename Tab>
+template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename Tab, typename S = float>
 __global__ void __launch_bounds__(kBlock, EncMinBlocks<MODE, VPT>::value) encode_kernel(const EncArgs A, const __grid_constant__ Tab tab) {
   __shared__ float sm_f[kBlock / 32];
   __shared__ unsigned long long sm_u[kBlock / 32];
@@ -609,8 +623,8 @@ __global__ void __launch_bounds__(kBlock, EncMinBlocks<MODE, VPT>::value) encode
     int64_t b = 0, r = 0;
     if (row_ok) split_row(gr, A.rows, A.batch, b, r);
     const T *arow = act_tensor<T, Tab>(A.a, tab, b, E) + r * cols;
-    float *hrow = A.ahat + (row_ok ? gr : 0) * cols;
-    float *erow = A.err + (row_ok ? gr : 0) * cols;
+    S *hrow = reinterpret_cast<S *>(A.ahat) + (row_ok ? gr : 0) * cols;
+    S *erow = reinterpret_cast<S *>(A.err) + (row_ok ? gr : 0) * cols;
     uint8_t *body = A.payload + kHdrBytes + b * A.body_bytes;
     typename Act<T>::Raw ra[VPT];
     float4 rh[VPT][2], re[VPT][2];
@@ -622,17 +636,11 @@ __global__ void __launch_bounds__(kBlock, EncMinBlocks<MODE, VPT>::value) encode
       rh[j][0] = rh[j][1] = re[j][0] = re[j][1] = z;
       if (row_ok && v < V) {
         ra[j] = Act<T>::load(arow + v * 8);
-        const float4 *hp = reinterpret_cast<const float4 *>(hrow + v * 8);
-        rh[j][0] = __ldcs(hp);
-        rh[j][1] = __ldcs(hp + 1);
-        if (A.ef_explicit) {
-          const float4 *ep = reinterpret_cast<const float4 *>(erow + v * 8);
-          re[j][0] = __ldcs(ep);
-          re[j][1] = __ldcs(ep + 1);
-        }
+        load_state8(hrow + v * 8, rh[j]);
+        if (A.ef_explicit) load_state8(erow + v * 8, re[j]);
       }
     }
-    encode_row<MODE, T, VPT, NM_M, NM_N>(A, t, tlog, row_ok, r, hrow, erow, body, ra, rh, re, sm_f, sm_u);
+    encode_row<MODE, T, VPT, NM_M, NM_N, S>(A, t, tlog, row_ok, r, hrow, erow, body, ra, rh, re, sm_f, sm_u);
   }
 }
 
@@ -719,8 +727,8 @@ __device__ __forceinline__ float bf16_half(uint32_t w, int hi) { return __uint_a
 
 // One row of the decode: C from the payload, ahat = ahat + C (fp32 RN),
 // recon = cast(ahat).  rp holds the identity mode's fp32 payload vectors.
-template <int MODE, typename T, int VPT, int NM_M, int NM_N>
-__device__ __forceinline__ void decode_row(const DecArgs &A, const int t, const int tlog, float *hrow, T *rrow,
+template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename S>
+__device__ __forceinline__ void decode_row(const DecArgs &A, const int t, const int tlog, S *hrow, T *rrow,
                                            const float4 (&rh)[VPT][2], const float4 (&rp)[VPT][2],
                                            const DecIn<VPT> &in) {
   using P = Pack<MODE, NM_M, NM_N>;
@@ -785,12 +793,12 @@ __device__ __forceinline__ void decode_row(const DecArgs &A, const int t, const 
     float hn[8];
 #pragma unroll
     for (int k = 0; k < 8; k++) hn[k] = __fadd_rn(hv[k], c[k]);
-    store_f32x8(hrow + v * 8, hn);
-    Act<T>::store_f32(rrow + v * 8, hn);
+    store_state8(hrow + v * 8, hn);
+    Act<T>::store_f32(rrow + v * 8, hn);  // a bf16 state and a bf16 recon round alike
   }
 }
 
-template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename Tab>
+template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename Tab, typename S = float>
 __global__ void __launch_bounds__(kBlock, CF_DEC_MIN_BLOCKS) decode_kernel(const DecArgs A, const __grid_constant__ Tab tab) {
   if (!header_ok(A)) return;
   const int tlog = A.team_log2;
@@ -810,7 +818,7 @@ __global__ void __launch_bounds__(kBlock, CF_DEC_MIN_BLOCKS) decode_kernel(const
     split_row(gr, A.rows, A.batch, b, r);
     const uint8_t *body = A.payload + kHdrBytes + b * A.body_bytes;
     T *rrow = static_cast<T *>(recon_tensor<Tab>(A.recon, tab, b, E * (int64_t)sizeof(T))) + r * cols;
-    float *hrow = A.ahat + gr * cols;
+    S *hrow = reinterpret_cast<S *>(A.ahat) + gr * cols;
     DecIn<VPT> in;
     load_dec_in<MODE, VPT, NM_M, NM_N>(A, body, r, t, tlog, true, in);
     float4 rh[VPT][2], rp[VPT][2];
@@ -820,9 +828,7 @@ __global__ void __launch_bounds__(kBlock, CF_DEC_MIN_BLOCKS) decode_kernel(const
       const int v = t + (j << tlog);
       rh[j][0] = rh[j][1] = rp[j][0] = rp[j][1] = z;
       if (v < V) {
-        const float4 *hp = reinterpret_cast<const float4 *>(hrow + v * 8);
-        rh[j][0] = __ldcs(hp);
-        rh[j][1] = __ldcs(hp + 1);
+        load_state8(hrow + v * 8, rh[j]);
         if constexpr (MODE == M_ID) {
           const float4 *pp = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(body) + r * cols + v * 8);
           rp[j][0] = __ldcs(pp);
@@ -830,14 +836,14 @@ __global__ void __launch_bounds__(kBlock, CF_DEC_MIN_BLOCKS) decode_kernel(const
         }
       }
     }
-    decode_row<MODE, T, VPT, NM_M, NM_N>(A, t, tlog, hrow, rrow, rh, rp, in);
+    decode_row<MODE, T, VPT, NM_M, NM_N, S>(A, t, tlog, hrow, rrow, rh, rp, in);
   }
 }
 
 // ---------------------------------------------------------------- warm-up kernels
 
 // Step 0: payload body = raw a; ahat = fp32(a); e = 0.
-template <typename T, int VPT, typename Tab>
+template <typename T, int VPT, typename Tab, typename S = float>
 __global__ void __launch_bounds__(kBlock) warm_encode_kernel(const EncArgs A, const __grid_constant__ Tab tab) {
   const int tlog = A.team_log2;
   const int TEAM = 1 << tlog;
@@ -864,16 +870,16 @@ __global__ void __launch_bounds__(kBlock) warm_encode_kernel(const EncArgs A, co
         float x[8];
         Act<T>::to_f32(raw, x);
         Act<T>::store_raw(prow + v * 8, raw);
-        store_f32x8(A.ahat + gr * cols + v * 8, x);
+        store_state8(reinterpret_cast<S *>(A.ahat) + gr * cols + v * 8, x);
         const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (A.err) store_f32x8(A.err + gr * cols + v * 8, z);  // block selection keeps no e
+        if (A.err) store_state8(reinterpret_cast<S *>(A.err) + gr * cols + v * 8, z);
       }
     }
   }
 }
 
 // Step 0 receiver: ahat = fp32(body); recon = body.
-template <typename T, int VPT, typename Tab>
+template <typename T, int VPT, typename Tab, typename S = float>
 __global__ void __launch_bounds__(kBlock) warm_decode_kernel(const DecArgs A, const __grid_constant__ Tab tab) {
   if (!header_ok(A)) return;
   const int tlog = A.team_log2;
@@ -899,7 +905,7 @@ __global__ void __launch_bounds__(kBlock) warm_decode_kernel(const DecArgs A, co
         const typename Act<T>::Raw raw = Act<T>::load(prow + v * 8);
         float x[8];
         Act<T>::to_f32(raw, x);
-        store_f32x8(A.ahat + gr * cols + v * 8, x);
+        store_state8(reinterpret_cast<S *>(A.ahat) + gr * cols + v * 8, x);
         Act<T>::store_raw(rrow + v * 8, raw);
       }
     }
@@ -909,36 +915,42 @@ __global__ void __launch_bounds__(kBlock) warm_decode_kernel(const DecArgs A, co
 }  // namespace
 
 // Kernel of one mode family (defined in cf_stream_mode_<mode>.cu).
-const void *stream_kernel_id(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table);
-const void *stream_kernel_s1(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table);
-const void *stream_kernel_q2(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table);
-const void *stream_kernel_nm(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table);
+const void *stream_kernel_id(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table, bool state_bf16);
+const void *stream_kernel_s1(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table, bool state_bf16);
+const void *stream_kernel_q2(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table, bool state_bf16);
+const void *stream_kernel_nm(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table, bool state_bf16);
 
 namespace {
-template <int MODE, int NM_M, int NM_N, typename T, typename Tab, int VPT>
+template <int MODE, int NM_M, int NM_N, typename T, typename Tab, typename S, int VPT>
 const void *pick_one(bool enc) {
-  if (enc) return reinterpret_cast<const void *>(&encode_kernel<MODE, T, VPT, NM_M, NM_N, Tab>);
-  return reinterpret_cast<const void *>(&decode_kernel<MODE, T, VPT, NM_M, NM_N, Tab>);
+  if (enc) return reinterpret_cast<const void *>(&encode_kernel<MODE, T, VPT, NM_M, NM_N, Tab, S>);
+  return reinterpret_cast<const void *>(&decode_kernel<MODE, T, VPT, NM_M, NM_N, Tab, S>);
 }
 
-template <int MODE, int NM_M, int NM_N, typename T, typename Tab>
+template <int MODE, int NM_M, int NM_N, typename T, typename Tab, typename S>
 const void *pick(bool enc, int vpt) {
   switch (vpt) {
-    case 1: return pick_one<MODE, NM_M, NM_N, T, Tab, 1>(enc);
-    case 2: return pick_one<MODE, NM_M, NM_N, T, Tab, 2>(enc);
-    case 3: return pick_one<MODE, NM_M, NM_N, T, Tab, 3>(enc);
-    case 4: return pick_one<MODE, NM_M, NM_N, T, Tab, 4>(enc);
+    case 1: return pick_one<MODE, NM_M, NM_N, T, Tab, S, 1>(enc);
+    case 2: return pick_one<MODE, NM_M, NM_N, T, Tab, S, 2>(enc);
+    case 3: return pick_one<MODE, NM_M, NM_N, T, Tab, S, 3>(enc);
+    case 4: return pick_one<MODE, NM_M, NM_N, T, Tab, S, 4>(enc);
   }
   return nullptr;
 }
 
+// The bf16-state option exists for bf16 activations only.
 template <int MODE, int NM_M, int NM_N>
-const void *pick_any(bool enc, int dtype, int vpt, bool table) {
-  if (dtype == CF_BF16)
-    return table ? pick<MODE, NM_M, NM_N, __nv_bfloat16, PtrTable>(enc, vpt)
-                 : pick<MODE, NM_M, NM_N, __nv_bfloat16, NoTable>(enc, vpt);
-  return table ? pick<MODE, NM_M, NM_N, float, PtrTable>(enc, vpt)
-               : pick<MODE, NM_M, NM_N, float, NoTable>(enc, vpt);
+const void *pick_any(bool enc, int dtype, int vpt, bool table, bool state_bf16) {
+  if (dtype == CF_BF16) {
+    if (state_bf16)
+      return table ? pick<MODE, NM_M, NM_N, __nv_bfloat16, PtrTable, __nv_bfloat16>(enc, vpt)
+                   : pick<MODE, NM_M, NM_N, __nv_bfloat16, NoTable, __nv_bfloat16>(enc, vpt);
+    return table ? pick<MODE, NM_M, NM_N, __nv_bfloat16, PtrTable, float>(enc, vpt)
+                 : pick<MODE, NM_M, NM_N, __nv_bfloat16, NoTable, float>(enc, vpt);
+  }
+  if (state_bf16) return nullptr;
+  return table ? pick<MODE, NM_M, NM_N, float, PtrTable, float>(enc, vpt)
+               : pick<MODE, NM_M, NM_N, float, NoTable, float>(enc, vpt);
 }
 }  // namespace
 

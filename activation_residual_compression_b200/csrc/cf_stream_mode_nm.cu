@@ -4,11 +4,11 @@
 
 namespace cfi {
 
-const void *stream_kernel_nm(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table) {
-  if (nm_m == 16 && nm_n == 1) return pick_any<M_NM, 16, 1>(enc, dtype, vpt, table);
-  if (nm_m == 16 && nm_n == 2) return pick_any<M_NM, 16, 2>(enc, dtype, vpt, table);
-  if (nm_m == 4 && nm_n == 1) return pick_any<M_NM, 4, 1>(enc, dtype, vpt, table);
-  if (nm_m == 4 && nm_n == 2) return pick_any<M_NM, 4, 2>(enc, dtype, vpt, table);
+const void *stream_kernel_nm(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table, bool state_bf16) {
+  if (nm_m == 16 && nm_n == 1) return pick_any<M_NM, 16, 1>(enc, dtype, vpt, table, state_bf16);
+  if (nm_m == 16 && nm_n == 2) return pick_any<M_NM, 16, 2>(enc, dtype, vpt, table, state_bf16);
+  if (nm_m == 4 && nm_n == 1) return pick_any<M_NM, 4, 1>(enc, dtype, vpt, table, state_bf16);
+  if (nm_m == 4 && nm_n == 2) return pick_any<M_NM, 4, 2>(enc, dtype, vpt, table, state_bf16);
   return nullptr;
 }
 

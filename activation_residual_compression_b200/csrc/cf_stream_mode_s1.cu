@@ -4,10 +4,10 @@
 
 namespace cfi {
 
-const void *stream_kernel_s1(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table) {
+const void *stream_kernel_s1(bool enc, int dtype, int nm_m, int nm_n, int vpt, bool table, bool state_bf16) {
   (void)nm_m;
   (void)nm_n;
-  return pick_any<M_S1, 0, 0>(enc, dtype, vpt, table);
+  return pick_any<M_S1, 0, 0>(enc, dtype, vpt, table, state_bf16);
 }
 
 }  // namespace cfi

@@ -94,7 +94,7 @@ def _bs_frac(rows, kw):
     return kw["bs_k"] / K
 
 
-def encode_bytes(mode, rows, cols, kw, act_size=2, ef="explicit"):
+def encode_bytes(mode, rows, cols, kw, act_size=2, ef="explicit", state_size=4):
     """Algorithmic bytes of one encode launch: read a, ahat, e; write ahat, e, payload.
     Implicit feedback does not read e; without feedback e is neither read nor written.
     Block selection: read a and the previous activation (kept in the
@@ -103,12 +103,13 @@ def encode_bytes(mode, rows, cols, kw, act_size=2, ef="explicit"):
     E = rows * cols
     if mode == "blocksel":
         return int(E * 3 * act_size + 2 * _bs_frac(rows, kw) * E * act_size) + 64 + 16
-    e_rd = 4 if ef == "explicit" else 0
-    e_wr = 0 if ef == "off" else 4
-    return E * (act_size + 4 + e_rd + 4 + e_wr) + 64 + _payload_body(mode, rows, cols, kw)
+    z = state_size
+    e_rd = z if ef == "explicit" else 0
+    e_wr = 0 if ef == "off" else z
+    return E * (act_size + z + e_rd + z + e_wr) + 64 + _payload_body(mode, rows, cols, kw)
 
 
-def decode_bytes(mode, rows, cols, kw, act_size=2):
+def decode_bytes(mode, rows, cols, kw, act_size=2, state_size=4):
     """Algorithmic bytes of one decode launch: read payload, ahat; write ahat, recon.
     Block selection (state in the activation dtype): unsent blocks read ahat and
     write recon; sent blocks read the payload and write ahat and recon."""
@@ -116,7 +117,7 @@ def decode_bytes(mode, rows, cols, kw, act_size=2):
     if mode == "blocksel":
         f = _bs_frac(rows, kw)
         return int(E * ((1 - f) * 2 * act_size + f * 3 * act_size)) + 64
-    return E * (4 + 4 + act_size) + 64 + _payload_body(mode, rows, cols, kw)
+    return E * (2 * state_size + act_size) + 64 + _payload_body(mode, rows, cols, kw)
 
 
 def _kernel_sources_sha256():
@@ -223,12 +224,13 @@ def _make_stream(kind, wl, seed, device="cuda"):
     raise ValueError(kind)
 
 
-def step_bytes(mode, rows, cols, kw, payload, ef="explicit"):
+def step_bytes(mode, rows, cols, kw, payload, ef="explicit", state_size=4):
     """Algorithmic bytes of one encode + decode of one tensor (low-rank: the
     explicit-feedback figure)."""
     if mode == "lowrank":
         return _lr_alg_bytes(rows, cols, kw["iters"], payload)
-    return encode_bytes(mode, rows, cols, kw, ef=ef) + decode_bytes(mode, rows, cols, kw)
+    return (encode_bytes(mode, rows, cols, kw, ef=ef, state_size=state_size) +
+            decode_bytes(mode, rows, cols, kw, state_size=state_size))
 
 
 def launches_per_call(mode, kw, encode):
@@ -262,6 +264,8 @@ def run_cf(args, rank, world, device):
         acts = [s.next() for _ in range(n_inputs)]
         del s
         base = dict(dtype=cf.CF_BF16, batch=B_, ef=EF_CODES[args.ef], **kw)
+        if args.state == "bf16":
+            base["state_dtype"] = cf.CF_BF16
         S = cf.cf_create(R_, C_, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_SENDER, **base))
         R = cf.cf_create(R_, C_, cf.MODE_NAMES[mode], cf.cf_params_init(role=cf.CF_RECEIVER, **base))
         pay = torch.empty(max(cf.cf_payload_bytes(S, True), cf.cf_payload_bytes(S, False)), dtype=torch.uint8,
@@ -770,6 +774,8 @@ def main():
     ap.add_argument("--no-cogvideox", action="store_true", help="skip the 60-tensor CogVideoX-shaped step")
     ap.add_argument("--ef", default="explicit", choices=sorted(EF_CODES),
                     help="error-feedback form of the timed codecs (default: explicit)")
+    ap.add_argument("--state", default="f32", choices=["f32", "bf16"],
+                    help="state dtype of the timed streaming codecs (default fp32; bf16: the bf16-state option)")
     ap.add_argument("--ef-study", action="store_true",
                     help="instead of timing: receiver error per step of every mode and feedback form")
     ap.add_argument("--lr-sweep", action="store_true",
@@ -829,15 +835,17 @@ def main():
         kern = f"cf_encode block selection ({launches_per_call(c0['mode'], c0['kw'], True)} launches)"
         tr = None
     else:
-        enc_alg = B_ * encode_bytes(c0["mode"], R_, C_, c0["kw"], ef=args.ef)
-        kern = f"encode_kernel<{c0['name']}, bf16>"
-        tr = _traffic_record() if args.workload == "flux" and args.ef == "explicit" else None
+        zs = 2 if args.state == "bf16" else 4
+        enc_alg = B_ * encode_bytes(c0["mode"], R_, C_, c0["kw"], ef=args.ef, state_size=zs)
+        kern = f"encode_kernel<{c0['name']}, bf16" + (", bf16 state>" if zs == 2 else ">")
+        tr = _traffic_record() if args.workload == "flux" and args.ef == "explicit" and zs == 4 else None
     achieved = enc_alg / (enc_ms / 1e3) / 1e9
     per_mode = {}
     for c in st["codecs"]:
         pm = st["per"][c["name"]]
         step_ms = pm["enc"] + pm["dec"]
-        alg = B_ * step_bytes(c["mode"], R_, C_, c["kw"], c["P"], ef=args.ef)
+        alg = B_ * step_bytes(c["mode"], R_, C_, c["kw"], c["P"], ef=args.ef,
+                              state_size=2 if args.state == "bf16" else 4)
         per_mode[c["name"]] = {"ms_per_step": round(step_ms, 5), "encode_ms": round(pm["enc"], 5),
                                "decode_ms": round(pm["dec"], 5),
                                "activation_gbs": round(B_ * R_ * C_ * 2 / (step_ms / 1e3) / 1e9, 2),
@@ -852,6 +860,7 @@ def main():
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": wl["name"], "rows": R_, "cols": C_, "tensors": B_, "activation_dtype": "bf16",
                    "modes": [c["name"] for c in st["codecs"]], "error_feedback": args.ef,
+                   "state_dtype": args.state,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": f"inputs larger than L2: a fresh {in_mb:.0f} MB input per codec per step, state "
                          f"{B_ * R_ * C_ * 12 / 1e6:.0f} MB per codec",
@@ -869,7 +878,7 @@ def main():
         line["e2e"] = {"value": round(act_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                        "h2d_bytes_per_step": st["e2e"]["h2d"], "d2h_bytes_per_step": st["e2e"]["d2h"],
                        "ms_per_step": round(e2e_ms, 4)}
-    if world == 1 and not args.no_suite and args.workload == "flux" and args.ef == "explicit":
+    if world == 1 and not args.no_suite and args.workload == "flux" and args.ef == "explicit" and args.state == "f32":
         line["suite"] = run_suite(args, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)

@@ -152,6 +152,10 @@ typedef struct {
     int bs_block;              /* CF_BLOCKSEL: block side in tokens, 4, 8 or 16 (default 8) */
     int bs_k;                  /* CF_BLOCKSEL: blocks per step, 1..K; 0 = K/4 ("k/K = 1/4") */
     int bs_warm;               /* CF_BLOCKSEL: leading steps sent in full, >= 1 (default 5) */
+    int state_dtype;           /* CF_F32 (default): ahat and e in fp32.  CF_BF16: the bf16-state
+                                  option of the streaming modes with bf16 activations -- every
+                                  state update rounds to bf16 (nearest even), on both sides
+                                  alike; state traffic 8 instead of 16 bytes per element */
 } cf_params;
 
 typedef struct cf_state cf_state;

@@ -96,6 +96,8 @@ def lib():
         L.orc_lr_v0.argtypes = [c.c_uint64, c.c_int64, c.c_int, c.c_int]
         L.orc_householder_qr.argtypes = [P, c.c_int64, c.c_int, c.c_double, P, P, P]
         L.orc_subspace_iteration.argtypes = [P, c.c_int64, c.c_int64, c.c_int, c.c_int, P, P]
+        L.orc_set_state_bf16.restype = c.c_int
+        L.orc_set_state_bf16.argtypes = [P, c.c_int]
         L.orc_next_is_warm.restype = c.c_int
         L.orc_next_is_warm.argtypes = [P, c.c_int]
         L.orc_set_blocksel.restype = c.c_int
@@ -198,7 +200,8 @@ class Oracle:
     """
 
     def __init__(self, rows, cols, mode, dtype="bf16", ef="explicit", nm_n=1, nm_m=16,
-                 rank=1, iters=1, lr_int4=1, batch=1, seed=0, bs_h=0, bs_block=8, bs_k=0, bs_warm=5):
+                 rank=1, iters=1, lr_int4=1, batch=1, seed=0, bs_h=0, bs_block=8, bs_k=0, bs_warm=5,
+                 state_dtype="f32"):
         self.rows, self.cols, self.batch = int(rows), int(cols), int(batch)
         self.mode = mode
         self.dtype = dtype
@@ -207,6 +210,8 @@ class Oracle:
                                    nm_n, nm_m, rank, iters, lr_int4, batch, seed)
         if not self._h:
             raise ValueError("oracle rejected the configuration")
+        if state_dtype != "f32" and lib().orc_set_state_bf16(self._h, 1) != 0:
+            raise ValueError("the bf16 state needs a streaming mode on bf16 activations")
         if mode == "blocksel":
             # the grid defaults to square; k to a quarter of the blocks ("k/K = 1/4")
             h = int(bs_h) or math.isqrt(self.rows)

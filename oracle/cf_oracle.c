@@ -226,6 +226,7 @@ typedef struct {
     float *vprev;    /* LOWRANK: [batch][cols][rank] fp32 warm start */
     int bs_h, bs_w, bs_b, bs_k, bs_warm, bs_K; /* BLOCKSEL grid, block side, blocks per step */
     uint8_t *bs_sent; /* BLOCKSEL: [K] 1 = sent in the current round */
+    int state_bf16;   /* the bf16-state option: every state update rounds to bf16 */
     int vprev_valid;
     uint64_t step_s, step_r;
     int status;      /* 0 ok; nonzero after a header mismatch */
@@ -348,6 +349,22 @@ int orc_set_blocksel(orc_state *o, int h, int b, int k, int warm)
 }
 
 uint8_t *orc_blocksel_sent(orc_state *o) { return o->bs_sent; }
+
+/* The bf16-state option (streaming modes, bf16 activations): ahat_S, e and
+ * ahat_R are rounded to bf16 (nearest even) after every update, on both
+ * sides alike.  Returns 0, or -1 for a configuration without the option. */
+int orc_set_state_bf16(orc_state *o, int on)
+{
+    if (on && (o->dtype != ORC_BF16 || o->mode == ORC_LOWRANK || o->mode == ORC_BLOCKSEL)) return -1;
+    o->state_bf16 = on ? 1 : 0;
+    return 0;
+}
+
+/* the state's storage rounding */
+static float st_round(const orc_state *o, float x)
+{
+    return o->state_bf16 ? orc_f32_from_bf16(orc_bf16_from_f32(x)) : x;
+}
 void orc_set_step(orc_state *o, uint64_t s_send, uint64_t s_recv) { o->step_s = s_send; o->step_r = s_recv; }
 
 static float load_act(const void *a, int dtype, int64_t i)
@@ -868,10 +885,10 @@ int orc_encode(orc_state *o, const void *a, uint8_t *payload)
                 /* "Key design: error feedback" names what happens without
                  * feedback: the untransmitted error is dropped, and the
                  * next residual is taken against this step's activation */
-                ah[i] = load_act(a, o->dtype, (int64_t)b * E + i);
+                ah[i] = st_round(o, load_act(a, o->dtype, (int64_t)b * E + i));
             } else {
-                er[i] = d[i] - C[i];
-                ah[i] = ah[i] + C[i];
+                er[i] = st_round(o, d[i] - C[i]);
+                ah[i] = st_round(o, ah[i] + C[i]);
             }
         }
     }
@@ -929,7 +946,7 @@ int orc_decode(orc_state *o, const uint8_t *payload, void *recon)
         }
         float *ah = o->ahat_r + (int64_t)b * E;
         for (int64_t i = 0; i < E; i++) {
-            ah[i] = ah[i] + C[i];
+            ah[i] = st_round(o, ah[i] + C[i]);
             store_act(recon, o->dtype, (int64_t)b * E + i, ah[i]);
         }
     }

@@ -38,12 +38,16 @@ class GpuPair:
         self.rows, self.cols, self.batch = rows, cols, batch
         self.mode = cf.MODE_NAMES[mode]
         self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        bf16_state = extra.get("state_dtype") == "bf16"
+        if "state_dtype" in extra:
+            extra["state_dtype"] = cf.CF_BF16 if bf16_state else cf.CF_F32
         kw = dict(dtype=cf.CF_BF16 if dtype == "bf16" else cf.CF_F32,
                   ef={"explicit": cf.CF_EF_EXPLICIT, "implicit": cf.CF_EF_IMPLICIT, "off": cf.CF_EF_OFF}[ef],
                   nm_n=nm_n, nm_m=nm_m, batch=batch, rank=rank, iters=iters, lr_int4=lr_int4, seed=seed, **extra)
         self.has_err = mode != "blocksel"       # block selection keeps no error term
-        # block selection keeps its state (raw activations) in the activation dtype
-        self.state_esz = (2 if dtype == "bf16" else 4) if mode == "blocksel" else 4
+        # block selection keeps its state (raw activations) in the activation dtype;
+        # the bf16-state option stores ahat and e as bf16
+        self.state_esz = (2 if dtype == "bf16" else 4) if mode == "blocksel" else (2 if bf16_state else 4)
         self.S = cf.cf_create(rows, cols, self.mode, cf.cf_params_init(role=cf.CF_SENDER, **kw))
         self.R = cf.cf_create(rows, cols, self.mode, cf.cf_params_init(role=cf.CF_RECEIVER, **kw))
         self.pb_warm = cf.cf_payload_bytes(self.S, True)
@@ -76,16 +80,21 @@ class GpuPair:
         tb = int(buf[80:88].view(np.uint64)[0])
         ten = buf[len(buf) - tb:]
         n = self.batch * self.rows * self.cols
-        if self.state_esz == 2:
-            ahat = (ten[:2 * n].view(np.uint16).astype(np.uint32) << 16).view(np.float32)
-            ahat = ahat.reshape(self.batch, self.rows, self.cols)
-        else:
-            ahat = ten[:4 * n].view(np.float32).reshape(self.batch, self.rows, self.cols)
+        z = self.state_esz
+
+        def tensor(k):
+            raw = ten[k * z * n:(k + 1) * z * n]
+            if z == 2:
+                return (raw.view(np.uint16).astype(np.uint32) << 16).view(np.float32).reshape(
+                    self.batch, self.rows, self.cols)
+            return raw.view(np.float32).reshape(self.batch, self.rows, self.cols)
+
+        ahat = tensor(0)
         err = None
         if which == "S" and self.has_err:
-            err = ten[4 * n:8 * n].view(np.float32).reshape(self.batch, self.rows, self.cols)
+            err = tensor(1)
         if with_vprev:
-            vp = ten[8 * n:].view(np.float32).reshape(self.batch, self.cols, -1)
+            vp = ten[2 * z * n:].view(np.float32).reshape(self.batch, self.cols, -1)
             return ahat, err, vp
         return ahat, err
 

@@ -132,6 +132,33 @@ def test_error_feedback_off_batched_fp32_bit_exact(mode, kw):
         pair.close()
 
 
+@pytest.mark.parametrize("ef", ["explicit", "implicit", "off"])
+@pytest.mark.parametrize("mode,kw", [("sign1", {}), ("q2", {}), ("nm", {"nm_n": 1, "nm_m": 16}),
+                                     ("nm", {"nm_n": 2, "nm_m": 4}), ("identity", {})])
+def test_bf16_state_bit_exact(mode, kw, ef):
+    """The bf16-state option: every state update rounds to bf16 on both sides."""
+    rows, cols = 33, 1920
+    s = inputs.ActivationStream(rows, cols, dtype=torch.bfloat16, device="cuda", seed=12)
+    pair = GpuPair(rows, cols, mode, dtype="bf16", ef=ef, state_dtype="bf16", **kw)
+    orc = oracle.Oracle(rows, cols, mode, dtype="bf16", ef=ef, state_dtype="bf16", **kw)
+    try:
+        _run_and_compare(pair, orc, s.next, 6, sender_tracks_receiver=ef != "off")
+    finally:
+        pair.close()
+
+
+@pytest.mark.parametrize("mode,kw", [("sign1", {}), ("q2", {}), ("nm", {"nm_n": 2, "nm_m": 16})])
+def test_bf16_state_batched_bit_exact(mode, kw):
+    rows, cols, B = 24, 3072, 3
+    s = inputs.ActivationStream(rows, cols, batch=B, dtype=torch.bfloat16, device="cuda", seed=13)
+    pair = GpuPair(rows, cols, mode, dtype="bf16", batch=B, state_dtype="bf16", **kw)
+    orc = oracle.Oracle(rows, cols, mode, dtype="bf16", batch=B, state_dtype="bf16", **kw)
+    try:
+        _run_and_compare(pair, orc, s.next, 4)
+    finally:
+        pair.close()
+
+
 def test_degenerate_inputs_bit_exact():
     """Constant activations (all-zero residual), exact zeros, sign flips, huge and tiny values."""
     rows, cols = 16, 256
