@@ -233,6 +233,10 @@ class Oracle:
     def np_act(self):
         return np.uint16 if self.dtype == "bf16" else np.float32
 
+    def next_is_warm(self, receiver: bool = False) -> bool:
+        """The next encode (receiver: decode) is a full-size warm-up step."""
+        return lib().orc_next_is_warm(self._h, 1 if receiver else 0) != 0
+
     def payload_bytes(self, warmup: bool) -> int:
         return int(lib().orc_payload_bytes(self._h, 1 if warmup else 0))
 

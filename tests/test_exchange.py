@@ -1,0 +1,118 @@
+"""Host logic of the sequence-parallel payload exchange
+(``activation_residual_compression_b200.exchange``), on CPU with two gloo ranks.
+
+The exchange is codec-agnostic; here each rank drives it with the CPU oracle
+as the codec (test infrastructure), so no GPU is needed.  Every rank checks
+that the reconstruction it received for each peer's shard is bit-identical
+to an independent replay of that peer's seeded stream through a local
+sender/receiver pair, and that its own slot is its exact shard -- for two
+tensors per step, warm-up steps included.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROWS, COLS, STEPS = 64, 64, 9
+CASES = [("q2", {}), ("blocksel", {"bs_grid_h": 8, "bs_block": 4, "bs_k": 1, "bs_warm": 3})]
+
+
+class OracleCodec:
+    """The exchange's codec interface over the CPU oracle (one role used)."""
+
+    def __init__(self, rows, cols, mode, role, **params):
+        import oracle
+        kw = dict(params)
+        if "bs_grid_h" in kw:
+            kw["bs_h"] = kw.pop("bs_grid_h")
+        self.o = oracle.Oracle(rows, cols, mode, dtype="bf16", **kw)
+        self.role = role
+
+    def payload_bytes(self, warm):
+        return self.o.payload_bytes(warm)
+
+    def next_is_warm(self):
+        return self.o.next_is_warm(receiver=False)
+
+    def encode(self, a, payload, stream=None):
+        p = self.o.encode(a.view(torch.int16).numpy().view(np.uint16))
+        payload.copy_(torch.from_numpy(p))
+
+    def decode(self, payload, recon, stream=None):
+        r, st = self.o.decode(payload.numpy())
+        assert st == 0
+        recon.copy_(torch.from_numpy(r.reshape(recon.shape).view(np.int16)).view(torch.bfloat16))
+
+    def status(self, stream=None):
+        return self.o.status()
+
+    def close(self):
+        pass
+
+
+def _shard(rank, tensor, t):
+    g = torch.Generator().manual_seed(1000 * rank + 17 * tensor)
+    base = torch.randn(ROWS, COLS, generator=g)
+    walk = torch.zeros(ROWS, COLS)
+    for _ in range(t + 1):
+        walk += 0.1 * torch.randn(ROWS, COLS, generator=g)
+    return (base + walk).to(torch.bfloat16)
+
+
+def _worker(rank, world, port, mode, kw, q):
+    try:
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        from activation_residual_compression_b200.exchange import SPExchange
+        ex = SPExchange(ROWS, COLS, mode, n_tensors=2, device="cpu", codec_factory=OracleCodec, **kw)
+        # independent replay of every peer's stream: a local sender/receiver pair per (peer, tensor)
+        replay = {(p, i): (OracleCodec(ROWS, COLS, mode, 0, **kw), OracleCodec(ROWS, COLS, mode, 1, **kw))
+                  for p in range(world) if p != rank for i in range(2)}
+        for t in range(STEPS):
+            shards = [_shard(rank, i, t) for i in range(2)]
+            outs = ex.step(shards)
+            for i in range(2):
+                assert torch.equal(outs[i][rank], shards[i])
+                for p in range(world):
+                    if p == rank:
+                        continue
+                    s, r = replay[(p, i)]
+                    a = _shard(p, i, t)
+                    P = s.payload_bytes(s.next_is_warm())
+                    buf = torch.empty(P, dtype=torch.uint8)
+                    s.encode(a, buf)
+                    rec = torch.empty(ROWS, COLS, dtype=torch.bfloat16)
+                    r.decode(buf, rec)
+                    assert torch.equal(outs[i][p], rec), (rank, p, i, t)
+        assert ex.status() == 0
+        ex.close()
+        dist.barrier()
+        dist.destroy_process_group()
+        q.put((rank, "ok"))
+    except BaseException as e:  # report to the parent instead of hanging it
+        q.put((rank, repr(e)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("mode,kw", CASES)
+def test_two_rank_exchange_matches_independent_replay(mode, kw):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, mode, kw, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+    assert results == {0: "ok", 1: "ok"}, results
