@@ -162,17 +162,25 @@ __device__ __forceinline__ const __nv_bfloat16 *act_tensor<__nv_bfloat16, PtrTab
 // ---------------------------------------------------------------- reductions
 
 // Max over the team (all threads of the block call this together).
+// Barrier of one team only (named barrier 1 + team index; a block holds at
+// most kBlock / 64 = 4 multi-warp teams), so that the teams of a block do not
+// wait for one another.
+static_assert(kBlock / 64 <= 15, "named team barriers use ids 1 .. kBlock / 64");
+__device__ __forceinline__ void team_bar(int team_log2) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + (int)(threadIdx.x >> team_log2)), "r"(1 << team_log2) : "memory");
+}
+
 __device__ __forceinline__ float team_max(float x, int team_log2, float *sm) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
   if (team_log2 > 5) {
     const int warp = threadIdx.x >> 5, wpt = 1 << (team_log2 - 5);
     if ((threadIdx.x & 31) == 0) sm[warp] = x;
-    __syncthreads();
+    team_bar(team_log2);
     const int w0 = warp & ~(wpt - 1);
     x = sm[w0];
     for (int w = 1; w < wpt; w++) x = fmaxf(x, sm[w0 + w]);
-    __syncthreads();
+    team_bar(team_log2);
   }
   return x;
 }
@@ -184,11 +192,11 @@ __device__ __forceinline__ unsigned long long team_sum_u64(unsigned long long x,
   if (team_log2 > 5) {
     const int warp = threadIdx.x >> 5, wpt = 1 << (team_log2 - 5);
     if ((threadIdx.x & 31) == 0) sm[warp] = x;
-    __syncthreads();
+    team_bar(team_log2);
     const int w0 = warp & ~(wpt - 1);
     x = sm[w0];
     for (int w = 1; w < wpt; w++) x += sm[w0 + w];
-    __syncthreads();
+    team_bar(team_log2);
   }
   return x;
 }
@@ -331,7 +339,7 @@ __device__ __forceinline__ void zero_padding(const EncArgs &A) {
 // its vectors v = t + j * TEAM): residual with error feedback, row statistic,
 // encode, payload stores, e = D - C and ahat = ahat + C stores (with
 // CF_EF_OFF: ahat = fp32(a) and no e store).  Every thread
-// of the block calls this together (team reductions use __syncthreads).
+// of the team calls this together (team reductions use the team's barrier).
 template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename S>
 __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const int tlog, const bool row_ok,
                                            const int64_t r, S *hrow, S *erow, uint8_t *body,
