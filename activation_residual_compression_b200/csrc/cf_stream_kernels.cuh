@@ -370,7 +370,15 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
   }
 
   // ---- encode; c[j][k] = C(D) from the encoded values ----
-  float c[VPT][8];
+  // C(D) for the state update below.  The 2-bit and N:M modes rebuild it
+  // there from compact per-vector data (the 2-bit codes and two levels; the
+  // kept mask) rather than holding VPT x 8 floats; the 1-bit mode keeps its
+  // +-S values (measured faster for it on B200).
+  float cL2 = 0.0f, cL3 = 0.0f;
+  uint32_t cinfo[VPT];
+  float cs1[MODE == M_S1 ? VPT : 1][8];
+#pragma unroll
+  for (int j = 0; j < VPT; j++) cinfo[j] = 0;
   uint32_t cbits[VPT];
 #pragma unroll
   for (int j = 0; j < VPT; j++) cbits[j] = 0;
@@ -380,7 +388,6 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
     for (int j = 0; j < VPT; j++) {
       const int v = t + (j << tlog);
 #pragma unroll
-      for (int k = 0; k < 8; k++) c[j][k] = d[j][k];
       if (row_ok && v < V) store_f32x8(reinterpret_cast<float *>(body) + r * cols + v * 8, d[j]);
     }
   } else if constexpr (MODE == M_S1) {
@@ -427,7 +434,7 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
       for (int k = 0; k < 8; k++) {
         const bool neg = d[j][k] < 0.0f;
         byte |= (uint32_t)neg << k;
-        c[j][k] = neg ? -S : S;
+        cs1[j][k] = neg ? -S : S;
       }
       const int v = t + (j << tlog);
       cbits[j] = byte << ((v % P::G) * P::bpv);
@@ -444,6 +451,8 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
     if (row_ok && t == 0) reinterpret_cast<uint16_t *>(body)[r] = sbits;
     float L[4];
     q2_levels(S, L);
+    cL2 = L[2];
+    cL3 = L[3];
     const float k1 = S != 0.0f ? __fdiv_rn(1.5f, S) : 0.0f;
 #pragma unroll
     for (int j = 0; j < VPT; j++) {
@@ -452,8 +461,8 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
       for (int k = 0; k < 8; k++) {
         const float qf = S != 0.0f ? q2_code(d[j][k], S, k1) : 0.0f;
         codes |= small_uint(qf) << (2 * k);
-        c[j][k] = q2_level(qf, L[2], L[3]);
       }
+      cinfo[j] = codes;
       const int v = t + (j << tlog);
       cbits[j] = codes << ((v % P::G) * P::bpv);
     }
@@ -464,8 +473,6 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
     for (int j = 0; j < VPT; j++) {
       const int v = t + (j << tlog);
       const bool ok = row_ok && v < V;
-#pragma unroll
-      for (int k = 0; k < 8; k++) c[j][k] = 0.0f;
       if constexpr (NM_M == 16) {
         // a block of 16 columns spans the vector pair (v even, v odd) held by lanes (t, t^1)
         float bv[2];
@@ -516,7 +523,7 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
           const int gk = k + 8 * half;
           bool keep = gk == ki[0];
           if (NM_N == 2) keep = keep || gk == ki[1];
-          if (keep) c[j][k] = __bfloat162float(__float2bfloat16_rn(d[j][k]));
+          if (keep) cinfo[j] |= 1u << k;
         }
         if (half == 0) {
           const int blk = v >> 1;
@@ -553,7 +560,7 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
             fields |= (uint32_t)ki[s] << (2 * (qb * NM_N + s));
 #pragma unroll
             for (int k = 0; k < 4; k++)
-              if (k == ki[s]) c[j][4 * qb + k] = __bfloat162float(bb);
+              if (k == ki[s]) cinfo[j] |= 1u << (4 * qb + k);
           }
         }
         cbits[j] = fields << ((v % P::G) * P::bpv);
@@ -589,11 +596,19 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
   for (int j = 0; j < VPT; j++) {
     const int v = t + (j << tlog);
     if (row_ok && v < V) {
+      float c[8];
+#pragma unroll
+      for (int k = 0; k < 8; k++) {
+        if constexpr (MODE == M_ID) c[k] = d[j][k];
+        else if constexpr (MODE == M_S1) c[k] = cs1[j][k];
+        else if constexpr (MODE == M_Q2) c[k] = q2_level((float)((cinfo[j] >> (2 * k)) & 3u), cL2, cL3);
+        else c[k] = ((cinfo[j] >> k) & 1u) ? __bfloat162float(__float2bfloat16_rn(d[j][k])) : 0.0f;
+      }
       float en[8], hn[8];
 #pragma unroll
       for (int k = 0; k < 8; k++) {
-        en[k] = __fsub_rn(d[j][k], c[j][k]);
-        hn[k] = A.ef_off ? h[j][k] : __fadd_rn(h[j][k], c[j][k]);
+        en[k] = __fsub_rn(d[j][k], c[k]);
+        hn[k] = A.ef_off ? h[j][k] : __fadd_rn(h[j][k], c[k]);
       }
       if (!A.ef_off) store_state8(erow + v * 8, en);
       store_state8(hrow + v * 8, hn);

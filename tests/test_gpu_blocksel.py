@@ -88,6 +88,13 @@ def test_full_size_grid_bit_exact():
     _run(64, 64, 3072, 8, 16, "bf16", T=10, warm=5)
 
 
+def test_largest_block_count_bit_exact():
+    """K = 4096 blocks (the limit of the in-CTA sort): a 512 x 512 grid of 8 x 8
+    blocks, 16 channels, k = 1000 (not a divisor of K: rounds end with fewer
+    blocks and unused slots)."""
+    _run(512, 512, 16, 8, 1000, "bf16", T=9, warm=1)
+
+
 def test_ties_and_zero_blocks_bit_exact():
     """Unchanged activations (every d = 0: the lowest unsent indices win), blocks
     that become or stay zero (d = 1 / d = 0), then ordinary steps."""
