@@ -33,12 +33,10 @@
 
 #include "cf_internal.h"
 
-// Resident blocks per SM the compiler must allow (register budget) for the
-// streaming decode kernels; the encode kernels take 3 for the 2-bit mode and
-// for up to two vectors per thread, else 2 (measured on B200).
-#ifndef CF_DEC_MIN_BLOCKS
-#define CF_DEC_MIN_BLOCKS 3
-#endif
+// Resident blocks per SM the compiler must allow (register budget), measured
+// on B200: the decode kernels take 4 for N:M with two kept values per block
+// and 3 otherwise; the encode kernels take 3 for the 2-bit mode and for up to
+// two vectors per thread, else 2 (EncMinBlocks below).
 
 namespace cfi {
 namespace {
@@ -821,8 +819,13 @@ __device__ __forceinline__ void decode_row(const DecArgs &A, const int t, const 
   }
 }
 
+template <int MODE, int NM_N>
+struct DecMinBlocks {
+  static constexpr int value = (MODE == M_NM && NM_N == 2) ? 4 : 3;
+};
+
 template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename Tab, typename S = float>
-__global__ void __launch_bounds__(kBlock, CF_DEC_MIN_BLOCKS) decode_kernel(const DecArgs A, const __grid_constant__ Tab tab) {
+__global__ void __launch_bounds__(kBlock, DecMinBlocks<MODE, NM_N>::value) decode_kernel(const DecArgs A, const __grid_constant__ Tab tab) {
   if (!header_ok(A)) return;
   const int tlog = A.team_log2;
   const int TEAM = 1 << tlog;
