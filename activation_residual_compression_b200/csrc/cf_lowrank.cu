@@ -28,6 +28,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <type_traits>
 #include <utility>
 #include <mutex>
 
@@ -321,6 +322,10 @@ __global__ void __launch_bounds__(128, 1)
 
 // Rows per partial Gram block (rows are a multiple of 128).
 constexpr int kGramRows = 32;
+// Second CholeskyQR pass: largest |Q1^T Q1 - I| entry for which the first-
+// order factor is used (its orthogonality error, about 3 n 2^-32 per entry,
+// is at the fp32 rounding of the stored Q).
+constexpr double kNearIdentity = 1.0 / 65536.0;
 
 // Shared-memory column index of the Gram tile: the 16 column groups of TT
 // are laid out with an odd stride (TT | 1), so that the 16 groups a warp reads
@@ -458,10 +463,21 @@ __global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart
 // multiply-adds per thread.  A pivot <= 1e-12 G_00 (R_kk <= 1e-6 R_00) marks
 // column k rank deficient: dead[k] = 1, the step's multiplier is zero (L's
 // column k below the diagonal is zero) and column k of M is zero, so that
-// Q's column k is zero.  Writes M fp64 [n][n] (upper triangular); G and M
-// may alias (G is read into registers before the first barrier).
+// Q's column k is zero.
+//
+// near_id > 0 (the second pass of CholeskyQR2, where G = Q1^T Q1 is close to
+// the identity): if every entry of E = G - I between nonzero columns has
+// |E_ij| <= near_id, M is the first-order factor instead: with G = L L^T and
+// L = I + F, F = strict_lower(E) + diag(E) / 2 + O(|E|^2), so L^-1 = I - F +
+// O(|E|^2), and Q1 M has an orthogonality error of about 3 n near_id^2 per
+// entry.  A column of G that is exactly zero (a column of Q1 zeroed as rank
+// deficient by the first pass) is dead, as in the elimination.  Otherwise
+// the elimination runs.
+//
+// Writes M fp64 [n][n] (upper triangular); G and M may alias (G is read into
+// registers before the first barrier).
 template <int TT>
-__global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double *Mout, int *dead) {
+__global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double *Mout, int *dead, double near_id) {
   pdl_enter();
   constexpr int n = 16 * TT;
   constexpr int S = TT | 1;  // odd block stride of the shared vector: no bank conflicts
@@ -476,13 +492,47 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double
   for (int a = 0; a < TT; a++)
 #pragma unroll
     for (int c = 0; c < TT; c++) w[a][c] = (j0 + c <= i0 + a) ? G[(i0 + a) * n + j0 + c] : 0.0;
+  const bool lower = tx <= ty;  // blocks above the diagonal hold nothing
+  if (near_id > 0.0) {
+    int far = 0;
+    if (lower) {
+#pragma unroll
+      for (int a = 0; a < TT; a++)
+#pragma unroll
+        for (int c = 0; c < TT; c++) {
+          const int gi = i0 + a, gj = j0 + c;
+          const double g = w[a][c];
+          if (gj < gi ? !(fabs(g) <= near_id) : (gj == gi && g != 0.0 && !(fabs(g - 1.0) <= near_id))) far = 1;
+        }
+    }
+    if (!__syncthreads_or(far)) {
+      // first-order factor; zero diagonal entries mark dead columns
+      if (tx == ty) {
+#pragma unroll
+        for (int a = 0; a < TT; a++) dead_s[i0 + a] = w[a][a] == 0.0 ? 1 : 0;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int a = 0; a < TT; a++) {
+        const int gi = i0 + a;
+#pragma unroll
+        for (int c = 0; c < TT; c++) {
+          const int gj = j0 + c;
+          double m = 0.0;  // M[gj][gi] = L^-1[gi][gj]
+          if (gj <= gi && !dead_s[gi] && !dead_s[gj]) m = gj == gi ? 1.0 - 0.5 * (w[a][c] - 1.0) : -w[a][c];
+          Mout[gj * n + gi] = m;
+        }
+      }
+      for (int e = threadIdx.x; e < n; e += blockDim.x) dead[e] = dead_s[e];
+      return;
+    }
+  }
+  const double thr = 1e-12 * G[0];
   if (tx == 0) {
 #pragma unroll
     for (int a = 0; a < TT; a++) u[0][ty * S + a] = (i0 + a == 0) ? 0.0 : w[a][0];
   }
   if (threadIdx.x == 0) piv[0] = w[0][0];
-  const double thr = 1e-12 * G[0];
-  const bool lower = tx <= ty;  // blocks above the diagonal hold nothing
   __syncthreads();
   for (int kb = 0; kb < 16; kb++) {
 #pragma unroll
@@ -827,7 +877,6 @@ struct ReconArgs {
   int64_t rows, cols;
   int kblocks;        // kp / 64
   int a_split;        // 1: A carries a lo term (fp32 factors)
-  int role;           // CF_SENDER: e, ahat update; CF_RECEIVER: ahat, recon
   int ef_explicit;
   int ef_off;  // CF_EF_OFF: ahat <- fp32(a), e untouched
   const void *a;      // sender: activations [rows][cols]
@@ -847,11 +896,52 @@ struct ReconArgs {
 // 8 warps: warp 0 lane 0 loads the operands (TMA) and issues the MMAs; after
 // they complete, warp w drains TMEM lanes 32 (w % 4).., columns 64 (w / 4)..
 // into a padded shared-memory C tile (the operand buffers are free by then),
-// and all warps update whole rows with coalesced 512-byte accesses.
+// and all warps update whole rows with coalesced 512-byte accesses, in
+// batches of rows whose HBM operands are loaded together (the first batch
+// before the MMAs).  The role is a template parameter so that the receiver,
+// which loads only the state, takes larger batches.
 constexpr int kReconThreads = 256;
 constexpr int kCsLd = kReconN + 4;  // padded C-tile row (floats)
+constexpr int kReconBatchSender = 4;  // rows per warp and batch of the update
+constexpr int kReconBatchReceiver = 8;
 
-template <typename T>
+// The update's global operands for one batch of a warp's rows (lane l:
+// columns 4l .. 4l + 3): the state, and for the sender the error (explicit
+// feedback) and the activation.
+template <typename T, bool SENDER>
+struct ReconRows {
+  static constexpr int B = SENDER ? kReconBatchSender : kReconBatchReceiver;
+  static constexpr int NB = kTileM / (8 * B);
+  static_assert(NB * 8 * B == kTileM, "update batches must cover the tile");
+  using X = typename std::conditional<sizeof(T) == 2, uint2, float4>::type;
+  float4 h[B];
+  float4 e[SENDER ? B : 1];
+  X x[SENDER ? B : 1];  // the activation as loaded
+  __device__ __forceinline__ void load(const ReconArgs &R, int64_t m0, int64_t n0, int warp, int lane, int b) {
+#pragma unroll
+    for (int u = 0; u < B; u++) {
+      const int rr = warp + 8 * (B * b + u);
+      const int64_t off = (m0 + rr) * R.cols + n0 + 4 * lane;
+      h[u] = __ldcs(reinterpret_cast<const float4 *>(R.ahat + off));
+      if constexpr (SENDER) {
+        e[u] = R.ef_explicit ? __ldcs(reinterpret_cast<const float4 *>(R.err + off)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[u] = __ldcs(reinterpret_cast<const X *>(static_cast<const T *>(R.a) + off));
+      }
+    }
+  }
+  __device__ __forceinline__ void act(int u, float (&v)[4]) const {
+    if constexpr (sizeof(T) == 2) {
+      v[0] = __uint_as_float(x[u].x << 16);
+      v[1] = __uint_as_float(x[u].x & 0xffff0000u);
+      v[2] = __uint_as_float(x[u].y << 16);
+      v[3] = __uint_as_float(x[u].y & 0xffff0000u);
+    } else {
+      v[0] = x[u].x; v[1] = x[u].y; v[2] = x[u].z; v[3] = x[u].w;
+    }
+  }
+};
+
+template <typename T, bool SENDER>
 __global__ void __launch_bounds__(kReconThreads, 2)
     lr_recon_kernel(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
                     const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
@@ -885,6 +975,8 @@ __global__ void __launch_bounds__(kReconThreads, 2)
   __syncthreads();
   umma::fence_after_sync();
   const uint32_t tmem = tmem_base;
+  ReconRows<T, SENDER> L;
+  L.load(R, m0, n0, warp, lane, 0);
   int ok = 1;
   if (warp == 0 && lane == 0) {
     umma::mbar_arrive_expect_tx(&full, total);
@@ -950,63 +1042,50 @@ __global__ void __launch_bounds__(kReconThreads, 2)
   umma::fence_before_sync();
   __syncthreads();
   if (warp == 0) umma::tmem_dealloc(tmem, 128);
-  // coalesced update: warp w takes rows w, w + 8, ...; lane l columns 4l .. 4l + 3
-  constexpr int kRowsInFlight = 4;
-  for (int r0 = warp; r0 < kTileM; r0 += 8 * kRowsInFlight) {
-    float4 cv[kRowsInFlight], hv[kRowsInFlight], ev[kRowsInFlight];
-    float xv[kRowsInFlight][4];
-    int64_t off[kRowsInFlight];
+  // coalesced update: warp w takes rows w + 8 j; lane l columns 4l .. 4l + 3;
+  // batch b = rows j in [B b, B (b + 1))
+  constexpr int B = ReconRows<T, SENDER>::B;
+  for (int b = 0; b < ReconRows<T, SENDER>::NB; b++) {
+    if (b > 0) L.load(R, m0, n0, warp, lane, b);
 #pragma unroll
-    for (int u = 0; u < kRowsInFlight; u++) {
-      const int rr = r0 + 8 * u;
-      off[u] = (m0 + rr) * R.cols + n0 + 4 * lane;
-      cv[u] = *reinterpret_cast<const float4 *>(cs + rr * kCsLd + 4 * lane);
-      hv[u] = __ldcs(reinterpret_cast<const float4 *>(R.ahat + off[u]));
-      if (R.role == CF_SENDER) {
-        ev[u] = R.ef_explicit ? __ldcs(reinterpret_cast<const float4 *>(R.err + off[u])) : make_float4(0.f, 0.f, 0.f, 0.f);
-        if constexpr (sizeof(T) == 2) {
-          const uint2 w = __ldcs(reinterpret_cast<const uint2 *>(static_cast<const T *>(R.a) + off[u]));
-          xv[u][0] = __uint_as_float(w.x << 16);
-          xv[u][1] = __uint_as_float(w.x & 0xffff0000u);
-          xv[u][2] = __uint_as_float(w.y << 16);
-          xv[u][3] = __uint_as_float(w.y & 0xffff0000u);
-        } else {
-          const float4 f = __ldcs(reinterpret_cast<const float4 *>(static_cast<const T *>(R.a) + off[u]));
-          xv[u][0] = f.x; xv[u][1] = f.y; xv[u][2] = f.z; xv[u][3] = f.w;
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kRowsInFlight; u++) {
-      const float c[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
-      const float h[4] = {hv[u].x, hv[u].y, hv[u].z, hv[u].w};
+    for (int u = 0; u < B; u++) {
+      const int rr = warp + 8 * (B * b + u);
+      const int64_t off = (m0 + rr) * R.cols + n0 + 4 * lane;
+      const float4 cv = *reinterpret_cast<const float4 *>(cs + rr * kCsLd + 4 * lane);
+      const float c[4] = {cv.x, cv.y, cv.z, cv.w};
+      const float h[4] = {L.h[u].x, L.h[u].y, L.h[u].z, L.h[u].w};
       float hn[4];
 #pragma unroll
       for (int k = 0; k < 4; k++) hn[k] = __fadd_rn(h[k], c[k]);
-      if (R.role == CF_SENDER && R.ef_off) {  // no error feedback: the state is the activation
-        __stcs(reinterpret_cast<float4 *>(R.ahat + off[u]), make_float4(xv[u][0], xv[u][1], xv[u][2], xv[u][3]));
-        continue;
-      }
-      __stcs(reinterpret_cast<float4 *>(R.ahat + off[u]), make_float4(hn[0], hn[1], hn[2], hn[3]));
-      if (R.role == CF_SENDER) {
-        const float e[4] = {ev[u].x, ev[u].y, ev[u].z, ev[u].w};
+      if constexpr (SENDER) {
+        float xv[4];
+        L.act(u, xv);
+        if (R.ef_off) {  // no error feedback: the state is the activation
+          __stcs(reinterpret_cast<float4 *>(R.ahat + off), make_float4(xv[0], xv[1], xv[2], xv[3]));
+          continue;
+        }
+        __stcs(reinterpret_cast<float4 *>(R.ahat + off), make_float4(hn[0], hn[1], hn[2], hn[3]));
+        const float e[4] = {L.e[u].x, L.e[u].y, L.e[u].z, L.e[u].w};
         float en[4];
 #pragma unroll
         for (int k = 0; k < 4; k++) {
-          const float tt = __fsub_rn(xv[u][k], h[k]);
+          const float tt = __fsub_rn(xv[k], h[k]);
           const float d = R.ef_explicit ? __fadd_rn(tt, e[k]) : tt;
           en[k] = __fsub_rn(d, c[k]);
         }
-        __stcs(reinterpret_cast<float4 *>(R.err + off[u]), make_float4(en[0], en[1], en[2], en[3]));
-      } else if constexpr (sizeof(T) == 2) {
-        uint2 w;
-        w.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[0])) |
-              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[1])) << 16);
-        w.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[2])) |
-              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[3])) << 16);
-        __stcs(reinterpret_cast<uint2 *>(static_cast<T *>(R.recon) + off[u]), w);
+        __stcs(reinterpret_cast<float4 *>(R.err + off), make_float4(en[0], en[1], en[2], en[3]));
       } else {
-        __stcs(reinterpret_cast<float4 *>(static_cast<T *>(R.recon) + off[u]), make_float4(hn[0], hn[1], hn[2], hn[3]));
+        __stcs(reinterpret_cast<float4 *>(R.ahat + off), make_float4(hn[0], hn[1], hn[2], hn[3]));
+        if constexpr (sizeof(T) == 2) {
+          uint2 w;
+          w.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[0])) |
+                ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[1])) << 16);
+          w.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[2])) |
+                ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hn[3])) << 16);
+          __stcs(reinterpret_cast<uint2 *>(static_cast<T *>(R.recon) + off), w);
+        } else {
+          __stcs(reinterpret_cast<float4 *>(static_cast<T *>(R.recon) + off), make_float4(hn[0], hn[1], hn[2], hn[3]));
+        }
       }
     }
   }
@@ -1048,6 +1127,16 @@ size_t recon_smem(int kblocks, int a_split) {
   const size_t ops = (size_t)kblocks * kTileM * kTileK * 2 * (3 + a_split);
   const size_t ctile = (size_t)kTileM * kCsLd * 4;
   return (ops > ctile ? ops : ctile) + 1024;
+}
+cudaError_t set_recon_smem(int smem) {
+  const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(lr_recon_kernel<__nv_bfloat16, true>, attr, smem)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(lr_recon_kernel<__nv_bfloat16, false>, attr, smem)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(lr_recon_kernel<float, true>, attr, smem)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(lr_recon_kernel<float, false>, attr, smem)) != cudaSuccess)
+    return e;
+  return cudaSuccess;
 }
 size_t apply_smem(int n) {
   const size_t xt = (size_t)kApplyRows * (n + 4) * 4, qt = (size_t)n * (kApplyRows + 1) * 4;
@@ -1177,10 +1266,7 @@ int lowrank_bind(LowrankPlan *plan, void *scratch) {
   const int rpi = plan->rp;
   if (cudaFuncSetAttribute(lr_thin_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)thin_smem(rpi, thin_stages(rpi))) != cudaSuccess ||
-      cudaFuncSetAttribute(lr_recon_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)recon_smem(plan->kp / kTileK, 1)) != cudaSuccess ||
-      cudaFuncSetAttribute(lr_recon_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)recon_smem(plan->kp / kTileK, 1)) != cudaSuccess ||
+      set_recon_smem((int)recon_smem(plan->kp / kTileK, 1)) != cudaSuccess ||
       set_apply_smem(rpi) != cudaSuccess) {
     (void)cudaGetLastError();
     return CF_ERR_CUDA;
@@ -1222,16 +1308,16 @@ cudaError_t launch_gram(int n, int nblk, const float *src, int nsrc, int64_t row
   return cudaGetLastError();
 }
 
-cudaError_t launch_chol(int n, double *L, int *dead, cudaStream_t st) {
+cudaError_t launch_chol(int n, double *L, int *dead, double near_id, cudaStream_t st) {
   switch (n / 16) {
-    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), 0, st, L, L, dead); break;
-    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), 0, st, L, L, dead); break;
-    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), 0, st, L, L, dead); break;
-    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), 0, st, L, L, dead); break;
-    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), 0, st, L, L, dead); break;
-    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), 0, st, L, L, dead); break;
-    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), 0, st, L, L, dead); break;
-    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), 0, st, L, L, dead); break;
+    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
+    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
+    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
+    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
+    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
+    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
+    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
+    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -1265,7 +1351,7 @@ cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int
   // the reduced Gram matrix goes to L, which the Cholesky kernel then
   // overwrites with M = L^-T
   launch_pdl(lr_gram_reduce_kernel, dim3((unsigned)((n * n + 31) / 32)), dim3(256), 0, st, b.gpart, nblk, n, b.L);
-  e = launch_chol(n, b.L, b.dead, st);
+  e = launch_chol(n, b.L, b.dead, final_pass ? kNearIdentity : 0.0, st);
   if (e != cudaSuccess) return e;
   return launch_apply(n, b.xbuf, b.L, rows, b.q, final_pass ? b.qthi : nullptr, final_pass ? b.qtlo : nullptr, st);
 }
@@ -1320,7 +1406,6 @@ cudaError_t dequant_and_recon(const LowrankPlan &P, const uint8_t *payload, bool
   R.cols = P.cols;
   R.kblocks = P.kp / kTileK;
   R.a_split = P.int4 ? 0 : 1;
-  R.role = receiver ? CF_RECEIVER : CF_SENDER;
   R.ef_explicit = P.ef_explicit;
   R.ef_off = P.ef_off;
   R.a = a;
@@ -1333,10 +1418,9 @@ cudaError_t dequant_and_recon(const LowrankPlan &P, const uint8_t *payload, bool
   R.expect = expect;
   const dim3 grid((unsigned)(P.rows / kTileM), (unsigned)(P.cols / kReconN));
   const size_t smem = recon_smem(R.kblocks, R.a_split);
-  if (P.dtype == CF_BF16)
-    launch_pdl(lr_recon_kernel<__nv_bfloat16>, dim3(grid), dim3(kReconThreads), smem, st, P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
-  else
-    launch_pdl(lr_recon_kernel<float>, dim3(grid), dim3(kReconThreads), smem, st, P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
+  auto *kern = P.dtype == CF_BF16 ? (receiver ? lr_recon_kernel<__nv_bfloat16, false> : lr_recon_kernel<__nv_bfloat16, true>)
+                                  : (receiver ? lr_recon_kernel<float, false> : lr_recon_kernel<float, true>);
+  launch_pdl(kern, dim3(grid), dim3(kReconThreads), smem, st, P.tm_uahi, P.tm_ualo, P.tm_vbhi, P.tm_vblo, R);
   return cudaGetLastError();
 }
 
@@ -1422,10 +1506,7 @@ int noalloc_scratch(void **out) {
       return CF_ERR_CUDA;
     }
     const int smem = (int)recon_smem(2, 1);
-    if (cudaFuncSetAttribute(lr_recon_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(lr_recon_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess) {
+    if (set_recon_smem(smem) != cudaSuccess) {
       (void)cudaGetLastError();
       return CF_ERR_CUDA;
     }
