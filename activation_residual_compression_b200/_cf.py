@@ -57,6 +57,7 @@ class cf_params(ctypes.Structure):
         ("bs_k", ctypes.c_int),
         ("bs_warm", ctypes.c_int),
         ("state_dtype", ctypes.c_int),
+        ("lr_qr2_tol", ctypes.c_double),
     ]
 
 

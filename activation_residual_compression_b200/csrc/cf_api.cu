@@ -141,6 +141,7 @@ int validate(int64_t rows, int64_t cols, int mode, const cf_params *p) {
     if (rows % 128 || cols % 128) return CF_ERR_SHAPE;
     if (p->iters < 1 || p->iters > 2) return CF_ERR_UNSUPPORTED;
     if (p->lr_int4 != 0 && p->lr_int4 != 1) return CF_ERR_ARG;
+    if (!(p->lr_qr2_tol >= 0.0 && p->lr_qr2_tol <= 1.0 / 4096.0)) return CF_ERR_ARG;  // NaN fails too
     if (p->batch != 1) return CF_ERR_UNSUPPORTED;
     LowrankPlan plan{};
     lowrank_plan(rows, cols, *p, &plan);
@@ -402,6 +403,7 @@ int cf_params_init(cf_params *p) {
   p->bs_k = 0;
   p->bs_warm = 5;
   p->state_dtype = CF_F32;
+  p->lr_qr2_tol = 1.0 / 65536.0;
   return CF_OK;
 }
 

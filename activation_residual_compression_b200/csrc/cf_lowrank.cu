@@ -322,10 +322,6 @@ __global__ void __launch_bounds__(128, 1)
 
 // Rows per partial Gram block (rows are a multiple of 128).
 constexpr int kGramRows = 32;
-// Second CholeskyQR pass: largest |Q1^T Q1 - I| entry for which the first-
-// order factor is used (its orthogonality error, about 3 n 2^-32 per entry,
-// is at the fp32 rounding of the stored Q).
-constexpr double kNearIdentity = 1.0 / 65536.0;
 
 // Shared-memory column index of the Gram tile: the 16 column groups of TT
 // are laid out with an odd stride (TT | 1), so that the 16 groups a warp reads
@@ -1156,6 +1152,7 @@ void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *p
   plan->dtype = p.dtype;
   plan->ef_explicit = p.ef == CF_EF_EXPLICIT;
   plan->ef_off = p.ef == CF_EF_OFF;
+  plan->qr2_tol = p.lr_qr2_tol;
   plan->rp = round_up(p.rank < 16 ? 16 : p.rank, 16);
   plan->kp = round_up(p.rank, kTileK);
   plan->supported = rows % 128 == 0 && cols % 128 == 0 && rows >= 128 && cols >= 128 && p.batch == 1 &&
@@ -1351,7 +1348,7 @@ cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int
   // the reduced Gram matrix goes to L, which the Cholesky kernel then
   // overwrites with M = L^-T
   launch_pdl(lr_gram_reduce_kernel, dim3((unsigned)((n * n + 31) / 32)), dim3(256), 0, st, b.gpart, nblk, n, b.L);
-  e = launch_chol(n, b.L, b.dead, final_pass ? kNearIdentity : 0.0, st);
+  e = launch_chol(n, b.L, b.dead, final_pass ? P.qr2_tol : 0.0, st);
   if (e != cudaSuccess) return e;
   return launch_apply(n, b.xbuf, b.L, rows, b.q, final_pass ? b.qthi : nullptr, final_pass ? b.qtlo : nullptr, st);
 }

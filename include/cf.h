@@ -156,6 +156,11 @@ typedef struct {
                                   option of the streaming modes with bf16 activations -- every
                                   state update rounds to bf16 (nearest even), on both sides
                                   alike; state traffic 8 instead of 16 bytes per element */
+    double lr_qr2_tol;         /* CF_LOWRANK: the second CholeskyQR pass uses the first-order
+                                  factor of Q1^T Q1 when every entry of Q1^T Q1 - I is at most
+                                  this (orthogonality error about 3 rank tol^2 per entry);
+                                  0 = always the full elimination; 0 <= tol <= 2^-12
+                                  (default 2^-16) */
 } cf_params;
 
 typedef struct cf_state cf_state;
@@ -167,7 +172,8 @@ CF_API const char *cf_version(void);
 CF_API const char *cf_strerror(int status);
 
 /* Defaults: bf16, sender, explicit EF, N:M 2:16, rank 70, 1 sweep, INT4,
- * batch 1, seed 0, no workspace.  Returns CF_ERR_ARG if p is NULL. */
+ * batch 1, seed 0, no workspace, block selection 8x8 blocks with k = K/4 and
+ * 5 full steps, fp32 state, lr_qr2_tol 2^-16.  Returns CF_ERR_ARG if p is NULL. */
 CF_API int cf_params_init(cf_params *p);
 
 /* Device bytes a state of this configuration needs (state tensors, status

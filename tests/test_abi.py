@@ -43,6 +43,17 @@ def test_params_defaults(cf):
     p = cf.cf_params_init()
     assert (p.dtype, p.role, p.ef, p.nm_n, p.nm_m, p.rank, p.iters, p.lr_int4, p.batch) == \
         (cf.CF_BF16, cf.CF_SENDER, cf.CF_EF_EXPLICIT, 2, 16, 70, 1, 1, 1)
+    assert (p.bs_grid_h, p.bs_block, p.bs_k, p.bs_warm, p.state_dtype) == (0, 8, 0, 5, cf.CF_F32)
+    assert p.lr_qr2_tol == 2.0 ** -16
+
+
+def test_lowrank_qr2_tolerance_range(cf):
+    ok = _ws(cf, 512, 384, cf.CF_LOWRANK, rank=40)
+    assert ok[0] == cf.CF_OK
+    for tol in (0.0, 2.0 ** -12):
+        assert _ws(cf, 512, 384, cf.CF_LOWRANK, rank=40, lr_qr2_tol=tol) == ok
+    for tol in (-1e-9, 2.0 ** -12 * 1.001, float("nan"), float("inf")):
+        assert _ws(cf, 512, 384, cf.CF_LOWRANK, rank=40, lr_qr2_tol=tol)[0] == cf.CF_ERR_ARG, tol
 
 
 def _ws(cf, rows, cols, mode, **kw):
