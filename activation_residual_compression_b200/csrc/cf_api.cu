@@ -39,6 +39,13 @@ struct cf_state {
   Layout lay{};
   LowrankPlan lr{};
   BlockselPlan bs{};
+  // Low-rank sender: the encode chain (17 launches for one sweep) runs as
+  // one CUDA graph, captured on a private stream at each call and swapped
+  // into the executable graph with cudaGraphExecUpdate (same topology, new
+  // arguments), so that the chain pays one graph launch instead of a stream
+  // launch per kernel.
+  cudaStream_t cap = nullptr;
+  cudaGraphExec_t gexec = nullptr;
 };
 
 namespace {
@@ -286,6 +293,42 @@ DecArgs dec_args(cf_state *s, const void *payload, void *recon, bool warm) {
   return A;
 }
 
+// Runs chain(stream) as a CUDA graph launched on st (see cf_state::gexec).
+// When st is itself being captured, the launches go straight into the
+// caller's graph.
+template <typename F>
+cudaError_t graph_run(cf_state *s, cudaStream_t st, F &&chain) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  if (cs != cudaStreamCaptureStatusNone) return chain(st);
+  if (!s->cap && (e = cudaStreamCreateWithFlags(&s->cap, cudaStreamNonBlocking)) != cudaSuccess) {
+    s->cap = nullptr;
+    return e;
+  }
+  if ((e = cudaStreamBeginCapture(s->cap, cudaStreamCaptureModeThreadLocal)) != cudaSuccess) return e;
+  const cudaError_t le = chain(s->cap);
+  cudaGraph_t g = nullptr;
+  e = cudaStreamEndCapture(s->cap, &g);
+  if (le != cudaSuccess || e != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    (void)cudaGetLastError();
+    return le != cudaSuccess ? le : e;
+  }
+  if (s->gexec) {
+    cudaGraphExecUpdateResultInfo info{};
+    if (cudaGraphExecUpdate(s->gexec, g, &info) != cudaSuccess) {  // topology changed: instantiate anew
+      (void)cudaGetLastError();
+      cudaGraphExecDestroy(s->gexec);
+      s->gexec = nullptr;
+    }
+  }
+  if (!s->gexec && (e = cudaGraphInstantiate(&s->gexec, g, 0)) != cudaSuccess) s->gexec = nullptr;
+  cudaGraphDestroy(g);
+  if (e != cudaSuccess) return e;
+  return cudaGraphLaunch(s->gexec, st);
+}
+
 int do_encode(cf_state *s, const void *a, const PtrTable *tab, void *payload, cudaStream_t st) {
   if (!live(s)) return CF_ERR_STATE;
   if (s->p.role != CF_SENDER) return CF_ERR_ROLE;
@@ -302,7 +345,7 @@ int do_encode(cf_state *s, const void *a, const PtrTable *tab, void *payload, cu
   } else if (warm) {
     e = launch_warm_encode(s->p.dtype, s->cfg, A, tab, st);
   } else if (s->mode == CF_LOWRANK) {
-    e = lowrank_encode(s->lr, A, tab, s->vprev, s->step, s->p.seed, st);
+    e = graph_run(s, st, [&](cudaStream_t cs) { return lowrank_encode(s->lr, A, tab, s->vprev, s->step, s->p.seed, cs); });
   } else {
     e = launch_encode(s->mode, s->p.dtype, s->p.nm_m, s->p.nm_n, s->cfg, A, tab, st);
   }
@@ -327,7 +370,7 @@ int do_decode(cf_state *s, const void *payload, void *recon, const PtrTable *tab
   } else if (warm) {
     e = launch_warm_decode(s->p.dtype, s->cfg, A, tab, st);
   } else if (s->mode == CF_LOWRANK) {
-    e = lowrank_decode(s->lr, A, tab, st);
+    e = lowrank_decode(s->lr, A, tab, st);  // two launches: a graph would not pay off
   } else {
     e = launch_decode(s->mode, s->p.dtype, s->p.nm_m, s->p.nm_n, s->cfg, A, tab, st);
   }
@@ -676,6 +719,8 @@ int cf_destroy(cf_state *s) {
     g_live.erase(s);
   }
   cudaDeviceSynchronize();
+  if (s->gexec) cudaGraphExecDestroy(s->gexec);
+  if (s->cap) cudaStreamDestroy(s->cap);
   if (s->own_slab) cudaFree(s->slab);
   (void)cudaGetLastError();
   delete s;

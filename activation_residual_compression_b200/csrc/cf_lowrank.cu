@@ -354,16 +354,25 @@ __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc
     const int e = threadIdx.x + 256 * v;
     acc4[v] = e < kGramRows * n4 ? s4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int p = 1; p < nsrc; p++) {
+  for (int p0 = 1; p0 < nsrc; p0 += 4) {  // four slabs' loads in flight, added in slab order
+    float4 t[4][NV];
 #pragma unroll
-    for (int v = 0; v < NV; v++) {
-      const int e = threadIdx.x + 256 * v;
-      if (e < kGramRows * n4) {
-        const float4 t = s4[(int64_t)p * slab4 + e];
-        acc4[v].x = __fadd_rn(acc4[v].x, t.x);
-        acc4[v].y = __fadd_rn(acc4[v].y, t.y);
-        acc4[v].z = __fadd_rn(acc4[v].z, t.z);
-        acc4[v].w = __fadd_rn(acc4[v].w, t.w);
+    for (int u = 0; u < 4; u++)
+#pragma unroll
+      for (int v = 0; v < NV; v++) {
+        const int e = threadIdx.x + 256 * v;
+        t[u][v] = (p0 + u < nsrc && e < kGramRows * n4) ? s4[(int64_t)(p0 + u) * slab4 + e]
+                                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+      if (p0 + u >= nsrc) break;
+#pragma unroll
+      for (int v = 0; v < NV; v++) {
+        acc4[v].x = __fadd_rn(acc4[v].x, t[u][v].x);
+        acc4[v].y = __fadd_rn(acc4[v].y, t[u][v].y);
+        acc4[v].z = __fadd_rn(acc4[v].z, t[u][v].z);
+        acc4[v].w = __fadd_rn(acc4[v].w, t[u][v].w);
       }
     }
   }
@@ -598,74 +607,79 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double
 }
 
 // Rows per apply block.
-constexpr int kApplyRows = 32;
+constexpr int kApplyRows = 16;
 template <int TT>
 __host__ __device__ constexpr int apply_xld() {
   return 16 * TT + 4;  // padded row stride of the X tile (bank spread, 16-byte rows)
 }
 
-// Q = X M (M = L^-T, upper triangular, zero below the diagonal) for 32 rows
+// Q = X M (M = L^-T, upper triangular, zero below the diagonal) for 16 rows
 // per block.  M and the block's rows of X are staged in shared memory;
-// thread (row, group) computes the 2 TT outputs c = 16 t + 2 group + {0, 1}
-// of its row (conflict-free paired loads of M) with fp64 accumulators over
-// all n terms in ascending order (the zeros below M's diagonal add nothing).
-// Writes Q fp32 [rows][n] and, when qthi != nullptr, Q^T split in bf16
-// ([n][rows], the K-major B operand of V = D^T Q), transposed through shared
-// memory so that those stores are row-contiguous.
+// thread (row, q) computes the TT outputs c = q + 16 t of its row (the 16
+// threads of a row read 16 consecutive entries of a row of M) with fp64
+// accumulators over all n terms, the two halves of the term range in
+// separate accumulators added at the end (the zeros below M's diagonal add
+// nothing).  Writes Q fp32 [rows][n] and, when qthi != nullptr, Q^T split in
+// bf16 ([n][rows], the K-major B operand of V = D^T Q), transposed through
+// shared memory so that those stores are row-contiguous.
 template <int TT>
 __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const double *M, int64_t rows, float *q,
                                                        __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo) {
   pdl_enter();
-  constexpr int n = 16 * TT, xld = apply_xld<TT>(), qld = kApplyRows + 1;
+  constexpr int n = 16 * TT, xld = apply_xld<TT>(), qld = kApplyRows + 1, h = n / 2;
   extern __shared__ __align__(16) uint8_t asm_[];
   double *Ms = reinterpret_cast<double *>(asm_);      // [n][n]
-  float *xs = reinterpret_cast<float *>(Ms + n * n);  // [32][xld]; reused as Q^T [n][qld]
+  float *xs = reinterpret_cast<float *>(Ms + n * n);  // [16][xld]; reused as Q^T [n][qld]
   const int64_t r0 = (int64_t)blockIdx.x * kApplyRows;
   {
     const double2 *M2 = reinterpret_cast<const double2 *>(M);
     double2 *Ms2 = reinterpret_cast<double2 *>(Ms);
-#pragma unroll 4
-    for (int e = threadIdx.x; e < n * n / 2; e += 256) Ms2[e] = M2[e];
+    constexpr int NM = n * n / 2;
+#pragma unroll
+    for (int v = 0; v < (NM + 255) / 256; v++) {
+      const int e = threadIdx.x + 256 * v;
+      if (e < NM) Ms2[e] = M2[e];
+    }
     const float4 *x4 = reinterpret_cast<const float4 *>(x) + r0 * (n / 4);
-    for (int e = threadIdx.x; e < kApplyRows * n / 4; e += 256) {
-      const int rr = e / (n / 4), c = (e % (n / 4)) * 4;
-      const float4 v = r0 + rr < rows ? x4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
-      *reinterpret_cast<float4 *>(xs + rr * xld + c) = v;
+    constexpr int NX = kApplyRows * n / 4;
+#pragma unroll
+    for (int v = 0; v < (NX + 255) / 256; v++) {
+      const int e = threadIdx.x + 256 * v;
+      if (e < NX) {
+        const int rr = e / (n / 4), c = (e % (n / 4)) * 4;
+        const float4 val = r0 + rr < rows ? x4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(xs + rr * xld + c) = val;
+      }
     }
   }
   __syncthreads();
-  const int lr = threadIdx.x >> 3, grp = threadIdx.x & 7;
-  double acc[2 * TT];
+  const int lr = threadIdx.x >> 4, qc = threadIdx.x & 15;
+  double acc0[TT], acc1[TT];
 #pragma unroll
-  for (int t = 0; t < 2 * TT; t++) acc[t] = 0.0;
+  for (int t = 0; t < TT; t++) acc0[t] = acc1[t] = 0.0;
 #pragma unroll 2
-  for (int j = 0; j < n; j++) {
-    const double xj = (double)xs[lr * xld + j];
-    const double2 *mr = reinterpret_cast<const double2 *>(Ms + j * n + 2 * grp);
+  for (int j = 0; j < h; j++) {
+    const double x0 = (double)xs[lr * xld + j], x1 = (double)xs[lr * xld + h + j];
+    const double *m0 = Ms + j * n + qc, *m1 = Ms + (h + j) * n + qc;
 #pragma unroll
     for (int t = 0; t < TT; t++) {
-      const double2 m = mr[8 * t];  // columns 16 t + 2 grp, +1
-      acc[2 * t] = fma(xj, m.x, acc[2 * t]);
-      acc[2 * t + 1] = fma(xj, m.y, acc[2 * t + 1]);
+      acc0[t] = fma(x0, m0[16 * t], acc0[t]);
+      acc1[t] = fma(x1, m1[16 * t], acc1[t]);
     }
   }
+  float res[TT];
+#pragma unroll
+  for (int t = 0; t < TT; t++) res[t] = (float)(acc0[t] + acc1[t]);
   const int64_t row = r0 + lr;
   if (row < rows) {
 #pragma unroll
-    for (int t = 0; t < TT; t++) {
-      const int c = 16 * t + 2 * grp;
-      *reinterpret_cast<float2 *>(q + row * n + c) = make_float2((float)acc[2 * t], (float)acc[2 * t + 1]);
-    }
+    for (int t = 0; t < TT; t++) q[row * n + qc + 16 * t] = res[t];
   }
   if (qthi == nullptr) return;  // uniform over the block
   __syncthreads();              // every thread is done with xs
   float *qs = xs;               // Q^T tile [n][qld]
 #pragma unroll
-  for (int t = 0; t < TT; t++) {
-    const int c = 16 * t + 2 * grp;
-    qs[c * qld + lr] = (float)acc[2 * t];
-    qs[(c + 1) * qld + lr] = (float)acc[2 * t + 1];
-  }
+  for (int t = 0; t < TT; t++) qs[(qc + 16 * t) * qld + lr] = res[t];
   __syncthreads();
   for (int e = threadIdx.x; e < n * kApplyRows; e += 256) {
     const int c = e / kApplyRows, rr = e % kApplyRows;
