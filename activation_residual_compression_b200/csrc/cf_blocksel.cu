@@ -11,8 +11,9 @@
 //                      flag over the row's b tokens x all channels, and the
 //                      state update p = a (the row is read once); the CTA
 //                      that finishes last runs the selection: d per block
-//                      from the partials (fixed order), bitonic sort of the
-//                      unsent blocks by (d desc, index asc), the first
+//                      from the partials (fixed order), the unsent blocks
+//                      ordered by (d desc, index asc) (all pairs compared
+//                      when K <= 256, else a bitonic sort), the first
 //                      min(k, unsent) in ascending order, the round-robin
 //                      flags, the payload header and index section;
 //   bs_pack_kernel     one CTA per (slot, token-row quarter): raw block rows
@@ -33,7 +34,6 @@ namespace cfi {
 namespace {
 
 constexpr int kBsThreads = 256;
-constexpr int kSelThreads = 1024;  // the largest selection CTA
 
 size_t pad16(size_t x) { return (x + 15u) & ~(size_t)15u; }
 size_t pad256(size_t x) { return (x + 255u) & ~(size_t)255u; }
@@ -85,16 +85,6 @@ struct Vec8<float> {
   }
 };
 
-__device__ __forceinline__ void load_f32x8(const float *p, float (&x)[8]) {
-  const float4 u = reinterpret_cast<const float4 *>(p)[0], v = reinterpret_cast<const float4 *>(p)[1];
-  x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
-  x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
-}
-__device__ __forceinline__ void store_f32x8(float *p, const float (&x)[8]) {
-  reinterpret_cast<float4 *>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
-  reinterpret_cast<float4 *>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
-}
-
 // first token of row y of block i (the row's b tokens are consecutive)
 __device__ __forceinline__ int64_t block_row_token(int i, int y, int W, int b) {
   const int nbx = W / b;
@@ -103,6 +93,13 @@ __device__ __forceinline__ int64_t block_row_token(int i, int y, int W, int b) {
 }
 
 // ------------------------------------------------------------------ encode
+
+// Device-scope acquire-release fetch-and-add.
+__device__ __forceinline__ unsigned atomic_add_acq_rel(unsigned *p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 
 // Order-preserving key of a double (larger d -> larger key); 0 marks "not a
 // candidate" (no finite d maps to it).
@@ -116,10 +113,43 @@ __device__ __forceinline__ bool before(unsigned long long kx, int ix, unsigned l
   return kx > ky || (kx == ky && ix < iy);
 }
 
+// d of block i from its b row partials, added in row order: 0 when every
+// value is unchanged, 1 when exactly one of the two norms is zero, else
+// 1 - <p, a> / (||p|| ||a||).  The partials were written by other CTAs of
+// this grid: read through L2.
+__device__ double block_dissimilarity(const double *part, int i, int b) {
+  const double4 *src = reinterpret_cast<const double4 *>(part) + (int64_t)i * b;
+  double dot = 0.0, np_ = 0.0, na = 0.0, ch = 0.0;
+  for (int r0 = 0; r0 < b; r0 += 8) {
+    double4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; u++) {
+      v[u] = make_double4(0.0, 0.0, 0.0, 0.0);
+      if (r0 + u < b) {
+        const double2 *q2 = reinterpret_cast<const double2 *>(src + r0 + u);
+        const double2 lo = __ldcg(q2), hi = __ldcg(q2 + 1);
+        v[u] = make_double4(lo.x, lo.y, hi.x, hi.y);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; u++)
+      if (r0 + u < b) {
+        dot += v[u].x;
+        np_ += v[u].y;
+        na += v[u].z;
+        ch = fmax(ch, v[u].w);
+      }
+  }
+  if (ch == 0.0) return 0.0;                     // every value unchanged
+  if (np_ == 0.0 || na == 0.0) return 1.0;       // exactly one zero norm
+  return 1.0 - dot / (sqrt(np_) * sqrt(na));
+}
+
 // The selection, run by one CTA of kBsThreads threads once every partial is
-// written: d per unsent block from its b partials (in order), bitonic sort of
-// K2 (a power of two) entries by (d desc, index asc), the first min(k,
-// unsent) blocks in ascending order into sel and the payload's index
+// written: d per unsent block, the unsent blocks ordered by (d desc, index
+// asc) -- for K2 <= kBsThreads each thread ranks one block against all
+// others, else a bitonic sort of K2 (a power of two) entries -- the first
+// min(k, unsent) blocks in ascending order into sel and the payload's index
 // section, the round-robin flags (restarting the round when all are sent)
 // and the payload header.
 __device__ void select_blocks(const double *part, int K, int K2, int b, int k, uint8_t *sent, uint32_t *sel,
@@ -130,65 +160,48 @@ __device__ void select_blocks(const double *part, int K, int K2, int b, int k, u
   __shared__ int wsum[kBsThreads / 32];
   const int tid = threadIdx.x;
   for (int i = tid; i < K2; i += kBsThreads) {
-    unsigned long long kk = 0ull;
-    if (i < K && !sent[i]) {
-      const double4 *src = reinterpret_cast<const double4 *>(part) + (int64_t)i * b;
-      double dot = 0.0, np_ = 0.0, na = 0.0, ch = 0.0;
-      for (int r0 = 0; r0 < b; r0 += 8) {
-        double4 v[8];
-#pragma unroll
-        for (int u = 0; u < 8; u++) {
-          v[u] = make_double4(0.0, 0.0, 0.0, 0.0);
-          if (r0 + u < b) {  // written by other CTAs of this grid: read through L2
-            const double2 *q2 = reinterpret_cast<const double2 *>(src + r0 + u);
-            const double2 lo = __ldcg(q2), hi = __ldcg(q2 + 1);
-            v[u] = make_double4(lo.x, lo.y, hi.x, hi.y);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; u++)
-          if (r0 + u < b) {
-            dot += v[u].x;
-            np_ += v[u].y;
-            na += v[u].z;
-            ch = fmax(ch, v[u].w);
-          }
-      }
-      double d;
-      if (ch == 0.0) d = 0.0;                       // every value unchanged
-      else if (np_ == 0.0 || na == 0.0) d = 1.0;    // exactly one zero norm
-      else d = 1.0 - dot / (sqrt(np_) * sqrt(na));
-      kk = sort_key(d);
-    }
-    key[i] = kk;
+    // 0 marks "not a candidate": sent in this round, or padding
+    key[i] = (i < K && !sent[i]) ? sort_key(block_dissimilarity(part, i, b)) : 0ull;
     idx[i] = i;
     pick[i] = 0;
   }
-  for (int size = 2; size <= K2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      __syncthreads();
-      for (int i = tid; i < K2; i += kBsThreads) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool up = (i & size) == 0;
-          const bool jfirst = before(key[j], idx[j], key[i], idx[i]);
-          const bool ifirst = before(key[i], idx[i], key[j], idx[j]);
-          if (up ? jfirst : ifirst) {
-            const unsigned long long tk = key[i];
-            key[i] = key[j];
-            key[j] = tk;
-            const int ti = idx[i];
-            idx[i] = idx[j];
-            idx[j] = ti;
+  __syncthreads();
+  if (K2 <= kBsThreads) {
+    // rank of block tid among all K2 entries; candidates (key > 0) rank first
+    if (tid < K2) {
+      const unsigned long long kt = key[tid];
+      int rank = 0;
+#pragma unroll 8
+      for (int j = 0; j < K2; j++) rank += before(key[j], j, kt, tid) ? 1 : 0;
+      if (rank < k && kt != 0ull) pick[tid] = 1;
+    }
+  } else {
+    for (int size = 2; size <= K2; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        __syncthreads();
+        for (int i = tid; i < K2; i += kBsThreads) {
+          const int j = i ^ stride;
+          if (j > i) {
+            const bool up = (i & size) == 0;
+            const bool jfirst = before(key[j], idx[j], key[i], idx[i]);
+            const bool ifirst = before(key[i], idx[i], key[j], idx[j]);
+            if (up ? jfirst : ifirst) {
+              const unsigned long long tk = key[i];
+              key[i] = key[j];
+              key[j] = tk;
+              const int ti = idx[i];
+              idx[i] = idx[j];
+              idx[j] = ti;
+            }
           }
         }
       }
     }
+    __syncthreads();
+    // candidates sort first (key > 0); the first min(k, candidates) are picked
+    for (int r = tid; r < K2; r += kBsThreads)
+      if (r < k && key[r] != 0ull) pick[idx[r]] = 1;
   }
-  __syncthreads();
-  // candidates sort first (key > 0); the first min(k, candidates) are picked
-  for (int r = tid; r < K2; r += kBsThreads)
-    if (r < k && key[r] != 0ull) pick[idx[r]] = 1;
   __syncthreads();
   // ascending list of the picked blocks: each thread owns a contiguous chunk
   const int chunk = (K2 + kBsThreads - 1) / kBsThreads;
@@ -237,7 +250,7 @@ __device__ void select_blocks(const double *part, int K, int K2, int b, int k, u
 // fp64 (each product of two fp32 values is exact, so each fused
 // multiply-add rounds once; the CTA adds its threads' sums in a fixed
 // order) and the state update prev = a (the row is read once).  The CTA
-// that finishes last (an atomic count after a fence) then runs the
+// that finishes last (an acquire-release atomic count) then runs the
 // selection on the complete set of partials, still in L2.
 template <typename T>
 __global__ void __launch_bounds__(kBsThreads) bs_encode_kernel(const T *a, T *prev, int W, int b, int64_t cols,
@@ -303,13 +316,14 @@ __global__ void __launch_bounds__(kBsThreads) bs_encode_kernel(const T *a, T *pr
       sacc = threadIdx.x == 3 ? fmax(sacc, ws[w][3]) : sacc + ws[w][threadIdx.x];
     part[(int64_t)blockIdx.x * 4 + threadIdx.x] = sacc;
   }
-  // the last CTA to finish selects
-  __threadfence();
+  // The last CTA to finish selects.  The count is an acquire-release atomic
+  // after the CTA barrier: it releases this CTA's partial (the barrier orders
+  // the writing threads before thread 0), and the last CTA's acquires every
+  // other CTA's; the selection then reads the partials through L2.
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(counter, 1u) == gridDim.x - 1;
+  if (threadIdx.x == 0) last = atomic_add_acq_rel(counter, 1u) == gridDim.x - 1;
   __syncthreads();
   if (!last) return;
-  __threadfence();
   select_blocks(part, K, K2, b, k, sent, sel, payload, hdr, smem);
   if (threadIdx.x == 0) *counter = 0u;  // for the next step
 }
@@ -332,7 +346,20 @@ __global__ void __launch_bounds__(kBsThreads) bs_pack_kernel(const T *a, const u
     return;
   }
   const T *src = a + block_row_token((int)blk, y, W, b) * cols;
-  for (int64_t v = v0 + threadIdx.x; v < v1; v += kBsThreads) Vec8<T>::store(dst + v * 8, Vec8<T>::load(src + v * 8));
+  constexpr int U = 4;  // vectors in flight per thread
+  for (int64_t v0t = v0 + threadIdx.x; v0t < v1; v0t += (int64_t)U * kBsThreads) {
+    typename Vec8<T>::Raw r[U];
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int64_t v = v0t + (int64_t)u * kBsThreads;
+      if (v < v1) r[u] = Vec8<T>::load(src + v * 8);
+    }
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int64_t v = v0t + (int64_t)u * kBsThreads;
+      if (v < v1) Vec8<T>::store(dst + v * 8, r[u]);
+    }
+  }
 }
 
 // Full-size leading steps: payload body = a, state = a (sender); state =
@@ -388,19 +415,29 @@ __global__ void __launch_bounds__(kBsThreads) bs_decode_kernel(const uint8_t *pa
   for (int j = threadIdx.x; j < k; j += kBsThreads)
     if (slots[j] == (uint32_t)i && i < K) atomicMax(&slot, j);
   __syncthreads();
-  const int64_t e0 = block_row_token(i, y, W, b) * cols;
   const int64_t n8 = (int64_t)b * cols / 8;
-  if (slot >= 0) {
-    const T *src = reinterpret_cast<const T *>(payload + kHdrBytes + ((4 * (size_t)k + 15) & ~(size_t)15)) +
-                   ((int64_t)slot * b * b + (int64_t)y * b) * cols;
-    for (int64_t v = threadIdx.x; v < n8; v += kBsThreads) {
-      const typename Vec8<T>::Raw r = Vec8<T>::load(src + v * 8);
-      Vec8<T>::store(ahat + e0 + v * 8, r);
-      Vec8<T>::store(recon + e0 + v * 8, r);
+  const int64_t e0 = block_row_token(i, y, W, b) * cols;
+  // the row comes from the payload (its block was sent) or from ahat
+  const bool from_payload = slot >= 0;
+  const T *src = from_payload ? reinterpret_cast<const T *>(payload + kHdrBytes + ((4 * (size_t)k + 15) & ~(size_t)15)) +
+                                    ((int64_t)slot * b * b + (int64_t)y * b) * cols
+                              : ahat + e0;
+  constexpr int U = 4;  // vectors in flight per thread
+  for (int64_t v0 = threadIdx.x; v0 < n8; v0 += (int64_t)U * kBsThreads) {
+    typename Vec8<T>::Raw r[U];
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int64_t v = v0 + (int64_t)u * kBsThreads;
+      if (v < n8) r[u] = Vec8<T>::load(src + v * 8);
     }
-  } else {
-    for (int64_t v = threadIdx.x; v < n8; v += kBsThreads)
-      Vec8<T>::store(recon + e0 + v * 8, Vec8<T>::load(ahat + e0 + v * 8));
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int64_t v = v0 + (int64_t)u * kBsThreads;
+      if (v < n8) {
+        if (from_payload) Vec8<T>::store(ahat + e0 + v * 8, r[u]);
+        Vec8<T>::store(recon + e0 + v * 8, r[u]);
+      }
+    }
   }
 }
 

@@ -233,10 +233,18 @@ def step_bytes(mode, rows, cols, kw, payload, ef="explicit", state_size=4):
             decode_bytes(mode, rows, cols, kw, state_size=state_size))
 
 
+def state_bytes_per_elem(args):
+    """Sender + receiver state bytes per element of one codec pair."""
+    if args.workload == "blocksel":
+        return 2 + 2                               # previous activation (sender), values (receiver), bf16
+    esz = 2 if args.state == "bf16" else 4
+    return esz * (3 if args.ef == "explicit" or args.ef == "implicit" else 2)  # ahat + e (sender), ahat (receiver)
+
+
 def launches_per_call(mode, kw, encode):
     """libcf kernels one steady-state cf_encode / cf_decode call launches."""
     if mode == "blocksel":
-        return 3 if encode else 1                 # block sums, selection, pack; decode
+        return 2 if encode else 1                 # block sums with the selection in the last CTA, pack; decode
     if mode != "lowrank":
         return 1
     if not encode:
@@ -859,11 +867,12 @@ def main():
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": wl["name"], "rows": R_, "cols": C_, "tensors": B_, "activation_dtype": "bf16",
-                   "modes": [c["name"] for c in st["codecs"]], "error_feedback": args.ef,
-                   "state_dtype": args.state,
+                   "modes": [c["name"] for c in st["codecs"]],
+                   **({"selection": "raw blocks, no error feedback, state in the activation dtype"}
+                      if args.workload == "blocksel" else {"error_feedback": args.ef, "state_dtype": args.state}),
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": f"inputs larger than L2: a fresh {in_mb:.0f} MB input per codec per step, state "
-                         f"{B_ * R_ * C_ * 12 / 1e6:.0f} MB per codec",
+                         f"{B_ * R_ * C_ * state_bytes_per_elem(args) / 1e6:.0f} MB per codec",
                    "inputs_resident": True},
         "per_mode": per_mode,
         "roofline": {"bound": "hbm", "kernel": kern, "achieved": round(achieved, 1),

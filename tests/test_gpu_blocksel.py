@@ -78,7 +78,10 @@ def _run(H, W, C, b, k, dtype, T, seq=None, warm=3, seed=1):
 
 @pytest.mark.parametrize("H,W,C,b,k,dtype", [(16, 16, 64, 8, 1, "f32"), (32, 32, 64, 8, 0, "bf16"),
                                              (24, 40, 32, 8, 4, "f32"), (12, 8, 16, 4, 2, "bf16"),
-                                             (48, 32, 1920, 16, 0, "bf16"), (64, 64, 256, 8, 3, "bf16")])
+                                             (48, 32, 1920, 16, 0, "bf16"), (64, 64, 256, 8, 3, "bf16"),
+                                             # around the switch from all-pairs ranking (K <= 256) to the sort
+                                             (80, 160, 32, 8, 0, "f32"), (128, 128, 32, 8, 50, "bf16"),
+                                             (136, 128, 16, 8, 7, "bf16")])
 def test_block_selection_bit_exact(H, W, C, b, k, dtype):
     _run(H, W, C, b, k, dtype, T=14)
 
