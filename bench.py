@@ -16,7 +16,9 @@ value  = activation bytes (rows*cols*2 per mode) / device time per step,
          CUDA events on the launching stream, max over ranks.
 e2e    = the same metric with the activation in pinned host memory: each
          step copies a_t host->device, encodes, decodes and copies the
-         reconstruction device->host, inside the timed region.
+         reconstruction device->host, inside the timed region; the copies
+         run on their own streams (two buffer slots), so step i's compute
+         overlaps step i+1's upload and step i-1's download.
 roofline = the encode kernel of the first mode: algorithmic bytes per launch
          (read a, ahat, e; write ahat, e, payload) / its mean event-timed
          duration, against the measured copy bandwidth.
@@ -290,11 +292,12 @@ def run_cf(args, rank, world, device):
         else:
             cf.cf_encode(c["S"], a, c["pay"], stream)
 
-    def dec(c):
+    def dec(c, out=None):
+        out = c["rec"] if out is None else out
         if batched:
-            cf.cf_decode_batched(c["R"], c["pay"], [c["rec"][b] for b in range(B_)], stream)
+            cf.cf_decode_batched(c["R"], c["pay"], [out[b] for b in range(B_)], stream)
         else:
-            cf.cf_decode(c["R"], c["pay"], c["rec"], stream)
+            cf.cf_decode(c["R"], c["pay"], out, stream)
 
     def step(i, evs=None):
         for c in codecs:
@@ -352,38 +355,67 @@ def run_cf(args, rank, world, device):
         if cf.cf_status(c["R"], stream) != cf.CF_OK or cf.cf_status(c["S"], stream) != cf.CF_OK:
             raise RuntimeError(f"codec {c['name']} reported an error status")
 
-    # e2e: pinned host activations in, pinned host reconstruction out
+    # e2e: pinned host activations in, pinned host reconstruction out, every
+    # step.  Three streams and two buffer slots: the host-to-device copy of
+    # step i+1 and the device-to-host copy of step i-1 run while step i is
+    # encoded and decoded (PCIe is full duplex); each slot is reused only
+    # after its previous contents were consumed.
     e2e = None
     if args.e2e_steps > 0:
-        host_in = [c["acts"][0].cpu().pin_memory() for c in codecs]
-        host_out = [torch.empty_like(c["rec"], device="cpu").pin_memory() for c in codecs]
-        dev_in = [torch.empty_like(h, device="cuda") for h in host_in]
+        nslot = 2
+        host_in = [[c["acts"][sl % n_inputs].cpu().pin_memory() for c in codecs] for sl in range(nslot)]
+        host_out = [[torch.empty_like(c["rec"], device="cpu").pin_memory() for c in codecs] for sl in range(nslot)]
+        dev_in = [[torch.empty_like(c["acts"][0]) for c in codecs] for _ in range(nslot)]
+        dev_out = [[torch.empty_like(c["rec"]) for c in codecs] for _ in range(nslot)]
+        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(nslot)]     # the slot's inputs are on the device
+        ev_done = [torch.cuda.Event() for _ in range(nslot)]   # encode + decode of the slot finished
+        ev_out = [torch.cuda.Event() for _ in range(nslot)]    # the slot's outputs are on the host
         for c in codecs:
             cf.cf_reset(c["S"]); cf.cf_reset(c["R"])
 
-        def e2e_step():
-            for ci, c in enumerate(codecs):
-                dev_in[ci].copy_(host_in[ci], non_blocking=True)
-                enc(c, dev_in[ci])
-                dec(c)
-                host_out[ci].copy_(c["rec"], non_blocking=True)
+        def e2e_step(i):
+            sl = i % nslot
+            with torch.cuda.stream(h2d):
+                if i >= nslot:
+                    h2d.wait_event(ev_done[sl])
+                for ci in range(len(codecs)):
+                    dev_in[sl][ci].copy_(host_in[sl][ci], non_blocking=True)
+                ev_in[sl].record(h2d)
+            stream.wait_event(ev_in[sl])
+            if i >= nslot:
+                stream.wait_event(ev_out[sl])
+            with torch.cuda.stream(stream):
+                for ci, c in enumerate(codecs):
+                    enc(c, dev_in[sl][ci])
+                    dec(c, dev_out[sl][ci])
+                ev_done[sl].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(ev_done[sl])
+                for ci in range(len(codecs)):
+                    host_out[sl][ci].copy_(dev_out[sl][ci], non_blocking=True)
+                ev_out[sl].record(d2h)
 
-        with torch.cuda.stream(stream):
-            for _ in range(max(3, W_run)):
-                e2e_step()
+        n_warm = max(3, W_run)
+        for i in range(n_warm):
+            e2e_step(i)
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            a0.record(stream)
-            for _ in range(args.e2e_steps):
-                e2e_step()
-            a1.record(stream)
+        a0.record(h2d)
+        for i in range(n_warm, n_warm + args.e2e_steps):
+            e2e_step(i)
+        # the last device-to-host copy depends on every earlier copy and step
+        a1.record(d2h)
         torch.cuda.synchronize()
         e2e_ms = a0.elapsed_time(a1) / args.e2e_steps
-        e2e = dict(ms=e2e_ms, h2d=sum(t.numel() * 2 for t in host_in), d2h=sum(t.numel() * 2 for t in host_out))
+        e2e = dict(ms=e2e_ms, h2d=sum(t.numel() * t.element_size() for t in host_in[0]),
+                   d2h=sum(t.numel() * t.element_size() for t in host_out[0]))
+        for c in codecs:
+            if cf.cf_status(c["R"], stream) != cf.CF_OK or cf.cf_status(c["S"], stream) != cf.CF_OK:
+                raise RuntimeError(f"codec {c['name']} reported an error status in the e2e run")
 
     info = [dict(mode=c["mode"], kw=c["kw"], name=c["name"], P=c["P"]) for c in codecs]
     for c in codecs:
