@@ -235,6 +235,15 @@ def step_bytes(mode, rows, cols, kw, payload, ef="explicit", state_size=4):
             decode_bytes(mode, rows, cols, kw, state_size=state_size))
 
 
+def workload_config(args, wl, world):
+    """The `config` keys both arms report for a workload."""
+    return {"workload": wl["name"], "rows": wl["rows"], "cols": wl["cols"], "tensors": wl["batch"],
+            "activation_dtype": "bf16", "modes": [_codec_name(m, k) for m, k in wl["codecs"]],
+            **({"selection": "raw blocks, no error feedback, state in the activation dtype"}
+               if args.workload == "blocksel" else {"error_feedback": args.ef, "state_dtype": args.state}),
+            "parallelism": f"replicas{world}" if world > 1 else "single"}
+
+
 def state_bytes_per_elem(args):
     """Sender + receiver state bytes per element of one codec pair."""
     if args.workload == "blocksel":
@@ -770,7 +779,12 @@ def run_reference(args):
                                         sigma_per_tensor=inputs.cogvideox_sigmas(wl["batch"])[:1])
         else:
             s = _make_stream(wl["stream"], sub, seed=1 + 100 * mi, device="cpu")
-        orcs.append((s, oracle.Oracle(rows, C_, mode, dtype="bf16", **_oracle_kw(mode, kw))))
+        okw = dict(_oracle_kw(mode, kw))
+        if mode != "blocksel":
+            okw["ef"] = args.ef
+            if args.state == "bf16" and mode != "lowrank":
+                okw["state_dtype"] = "bf16"
+        orcs.append((s, oracle.Oracle(rows, C_, mode, dtype="bf16", **okw)))
 
     def one():
         ins = [s.next().view(torch.int16).numpy().view(np.uint16) for s, _ in orcs]
@@ -789,8 +803,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl["name"], "modes": [_codec_name(m, k) for m, k in wl["codecs"]],
-                       "sample_rows": rows},
+            "config": {**workload_config(args, wl, args.gpus), "sample_rows": rows},
             "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": f"{rows} of {R_} rows x {C_} bf16 per step, "
                                        f"{'+'.join(_codec_name(m, k) for m, k in wl['codecs'])}"},
@@ -898,11 +911,7 @@ def main():
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": wl["name"], "rows": R_, "cols": C_, "tensors": B_, "activation_dtype": "bf16",
-                   "modes": [c["name"] for c in st["codecs"]],
-                   **({"selection": "raw blocks, no error feedback, state in the activation dtype"}
-                      if args.workload == "blocksel" else {"error_feedback": args.ef, "state_dtype": args.state}),
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
+        "config": {**workload_config(args, wl, world),
                    "l2": f"inputs larger than L2: a fresh {in_mb:.0f} MB input per codec per step, state "
                          f"{B_ * R_ * C_ * state_bytes_per_elem(args) / 1e6:.0f} MB per codec",
                    "inputs_resident": True},
