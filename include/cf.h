@@ -201,7 +201,11 @@ CF_API int cf_payload_bytes(const cf_state *s, int warmup, size_t *out);
  * activations a ([batch][rows][cols], contiguous, state dtype), writes the
  * device payload (cf_payload_bytes(s, step == 0) bytes), and updates the
  * sender's ahat and e in place.  One fused kernel per call for the
- * streaming modes.  Asynchronous on `stream`. */
+ * streaming modes.  Asynchronous on `stream`.  CF_LOWRANK: the launch chain
+ * is captured on a stream the state owns and run as one CUDA graph on
+ * `stream` (the state keeps the executable graph and updates it in place
+ * each call); when `stream` is itself being captured, the kernels are
+ * recorded into the caller's graph instead. */
 CF_API int cf_encode(cf_state *s, const void *a, void *payload, void *stream);
 
 /* Receiver step: reads the device payload, updates the receiver's ahat and
