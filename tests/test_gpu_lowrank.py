@@ -314,3 +314,35 @@ def test_lowrank_desync_detected():
         assert np.array_equal(before.view(np.uint32), after.view(np.uint32))
     finally:
         pair.close()
+
+
+def test_encode_captured_into_a_caller_graph():
+    """A low-rank cf_encode / cf_decode issued on a stream that the caller is
+    capturing (torch.cuda.graph) records the kernels into the caller's graph;
+    replaying it gives the bytes of the same step run directly."""
+    rows, cols, rank = 512, 384, 40
+    s = inputs.ar1("cuda", rows=rows, cols=cols)
+    acts = [s.next() for _ in range(3)]
+    direct, captured = _lr_pair(rows, cols, rank, 1, 1), _lr_pair(rows, cols, rank, 1, 1)
+    try:
+        for p in (direct, captured):
+            p.step(acts[0])
+            p.step(acts[1])
+        direct.step(acts[2])
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side), torch.cuda.graph(g, stream=side):
+            captured.step(acts[2], torch.cuda.current_stream())
+        g.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(direct.payload_np(False), captured.payload_np(False))
+        assert torch.equal(direct.recon, captured.recon)
+        for which in ("S", "R"):
+            assert np.array_equal(direct.export(which), captured.export(which)), which
+        for p in (direct, captured):
+            assert cf.cf_status(p.R) == cf.CF_OK and cf.cf_status(p.S) == cf.CF_OK
+        del g
+    finally:
+        direct.close()
+        captured.close()
