@@ -621,11 +621,15 @@ __host__ __device__ constexpr int apply_xld() {
 // separate accumulators added at the end (the zeros below M's diagonal add
 // nothing).  Writes Q fp32 [rows][n] and, when qthi != nullptr, Q^T split in
 // bf16 ([n][rows], the K-major B operand of V = D^T Q), transposed through
-// shared memory so that those stores are row-contiguous.
+// shared memory so that those stores are row-contiguous; when amax !=
+// nullptr, the absmax of each of Q's first r columns (the INT4 scales'
+// input) goes to amax, one atomicMax per column and block.
 template <int TT>
 __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const double *M, int64_t rows, float *q,
-                                                       __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo) {
+                                                       __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo, int r,
+                                                       unsigned *amax) {
   pdl_enter();
+  __shared__ unsigned cmax[16 * TT];
   constexpr int n = 16 * TT, xld = apply_xld<TT>(), qld = kApplyRows + 1, h = n / 2;
   extern __shared__ __align__(16) uint8_t asm_[];
   double *Ms = reinterpret_cast<double *>(asm_);      // [n][n]
@@ -675,6 +679,17 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
 #pragma unroll
     for (int t = 0; t < TT; t++) q[row * n + qc + 16 * t] = res[t];
   }
+  if (amax != nullptr) {  // uniform over the block: the INT4 column maxima of Q (non-negative bit patterns)
+    for (int c = threadIdx.x; c < n; c += 256) cmax[c] = 0u;
+    __syncthreads();
+    if (row < rows) {
+#pragma unroll
+      for (int t = 0; t < TT; t++) atomicMax(&cmax[qc + 16 * t], __float_as_uint(fabsf(res[t])));
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < r; c += 256)
+      if (cmax[c]) atomicMax(&amax[c], cmax[c]);
+  }
   if (qthi == nullptr) return;  // uniform over the block
   __syncthreads();              // every thread is done with xs
   float *qs = xs;               // Q^T tile [n][qld]
@@ -694,25 +709,45 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
 
 // V = sum of the partial slabs (fixed order) [cols][n]; V_prev (state,
 // [cols][r]) = V[:, :r]; when vthi != nullptr also V^T split for the next
-// iteration's Y = D V.
+// iteration's Y = D V; when amax != nullptr the absmax of each of V's first r
+// columns (the INT4 scales' input) goes to amax, one atomicMax per column
+// and block.
 __global__ void __launch_bounds__(256) lr_vsum_kernel(const float *vpart, int nsrc, int64_t cols, int n, int r,
                                                       float *v, float *vprev, __nv_bfloat16 *vthi,
-                                                      __nv_bfloat16 *vtlo) {
+                                                      __nv_bfloat16 *vtlo, unsigned *amax) {
   pdl_enter();
+  __shared__ unsigned cmax[kMaxRank];  // n <= kMaxRank
+  if (amax != nullptr) {  // uniform over the grid
+    for (int c = threadIdx.x; c < n; c += blockDim.x) cmax[c] = 0u;
+    __syncthreads();
+  }
   const int64_t total = cols * n;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
     float acc = vpart[idx];
-    for (int p = 1; p < nsrc; p++) acc = __fadd_rn(acc, vpart[(int64_t)p * total + idx]);
+    for (int p0 = 1; p0 < nsrc; p0 += 4) {  // four slabs' loads in flight, added in slab order
+      float t[4];
+#pragma unroll
+      for (int u = 0; u < 4; u++) t[u] = p0 + u < nsrc ? vpart[(int64_t)(p0 + u) * total + idx] : 0.0f;
+#pragma unroll
+      for (int u = 0; u < 4; u++)
+        if (p0 + u < nsrc) acc = __fadd_rn(acc, t[u]);
+    }
     const uint32_t j = (uint32_t)idx / (uint32_t)n;
     const int k = (int)((uint32_t)idx - j * (uint32_t)n);
     v[idx] = acc;
     if (k < r) vprev[j * r + k] = acc;
+    if (amax != nullptr) atomicMax(&cmax[k], __float_as_uint(fabsf(acc)));
     if (vthi) {
       __nv_bfloat16 hi, lo;
       split_bf16(k < r ? acc : 0.0f, hi, lo);
       vthi[(int64_t)k * cols + j] = hi;
       vtlo[(int64_t)k * cols + j] = lo;
     }
+  }
+  if (amax != nullptr) {  // the block's column maxima, one atomicMax per column
+    __syncthreads();
+    for (int c = threadIdx.x; c < r; c += blockDim.x)
+      if (cmax[c]) atomicMax(&amax[c], cmax[c]);
   }
 }
 
@@ -727,44 +762,11 @@ struct PackArgs {
   int64_t sec1, sec2, body;
   Header hdr;
   unsigned *amax;  // [2 n]: column absmax bit patterns of Q, then of V (zeroed by lr_vprep_kernel)
+  // the sender's reconstruction operands, written from the packed values (the
+  // dequantisation of the payload, see lr_dequant_kernel); k >= r stays zero
+  int kp;
+  __nv_bfloat16 *uahi, *ualo, *vbhi, *vblo;
 };
-
-// Column absmax of Q (blocks 0 .. rows/32 - 1) and of V (the rest), one
-// 32-row tile per block: thread (row lane, column group) keeps the maxima of
-// its four columns over its rows in registers (coalesced float4 loads), the
-// block combines them in shared memory, and one atomicMax per column goes to
-// P.amax.  The values are non-negative, so their bit patterns order like the
-// values and the result does not depend on the order of the updates.
-constexpr int kScaleRows = 32;
-__global__ void __launch_bounds__(256) lr_scale_kernel(PackArgs P) {
-  pdl_enter();
-  __shared__ unsigned cm[128];
-  const int nq = (int)(P.rows / kScaleRows);
-  const bool isv = (int)blockIdx.x >= nq;
-  const int64_t r0 = (int64_t)(isv ? blockIdx.x - nq : blockIdx.x) * kScaleRows;
-  const float4 *m4 = reinterpret_cast<const float4 *>((isv ? P.v : P.q) + r0 * P.n);
-  const int n4 = P.n / 4, lanes = (int)blockDim.x / n4;  // row lanes (n4 <= 32)
-  const int cg = threadIdx.x % n4, rl = threadIdx.x / n4;
-  for (int k = threadIdx.x; k < P.n; k += blockDim.x) cm[k] = 0u;
-  __syncthreads();
-  if (rl < lanes) {
-    float mx = 0.f, my = 0.f, mz = 0.f, mw = 0.f;
-    for (int rr = rl; rr < kScaleRows; rr += lanes) {
-      const float4 v = m4[rr * n4 + cg];
-      mx = fmaxf(mx, fabsf(v.x));
-      my = fmaxf(my, fabsf(v.y));
-      mz = fmaxf(mz, fabsf(v.z));
-      mw = fmaxf(mw, fabsf(v.w));
-    }
-    atomicMax(&cm[4 * cg], __float_as_uint(mx));
-    atomicMax(&cm[4 * cg + 1], __float_as_uint(my));
-    atomicMax(&cm[4 * cg + 2], __float_as_uint(mz));
-    atomicMax(&cm[4 * cg + 3], __float_as_uint(mw));
-  }
-  __syncthreads();
-  for (int k = threadIdx.x; k < P.r; k += blockDim.x)
-    if (cm[k]) atomicMax(&P.amax[(isv ? P.n : 0) + k], cm[k]);
-}
 
 // Scale s_k = fp32(absmax_k / 7) of column k of U (k < r) or V (k >= r).
 __device__ __forceinline__ float lr_scale_of(const PackArgs &P, int k) {
@@ -779,8 +781,20 @@ __device__ __forceinline__ uint32_t int4_code(float x, float s) {
   return (uint32_t)((int)t & 0xF);
 }
 
+// Reconstruction operand entry (i, k) of U (isv false) or of the scaled V
+// from the value the payload carries: INT4, the code q (U: q, exact in bf16;
+// V: fp32(q sU_k sV_k), products in fp64); fp32 factors, the value itself.
+__device__ __forceinline__ void lr_operand_store(__nv_bfloat16 *hi_out, __nv_bfloat16 *lo_out, int64_t o, float x) {
+  __nv_bfloat16 hi, lo;
+  split_bf16(x, hi, lo);
+  hi_out[o] = hi;
+  if (lo_out) lo_out[o] = lo;
+}
+
 // Nibbles of U and V (element (i,k) is nibble i*r + k, low nibble first) or
-// the fp32 factors, padding bytes zero, and the header.
+// the fp32 factors, padding bytes zero, and the header; and the sender's
+// reconstruction operands from the same values, exactly as the dequantisation
+// of the payload computes them.
 __global__ void __launch_bounds__(256) lr_pack_kernel(PackArgs P) {
   pdl_enter();
   uint8_t *body = P.payload + kHdrBytes;
@@ -808,7 +822,15 @@ __global__ void __launch_bounds__(256) lr_pack_kernel(PackArgs P) {
         const uint32_t e = 2 * bb + h;
         if (e < nel) {
           const uint32_t i = e / r, k = e - i * r;
-          byte |= int4_code(m[(int64_t)i * P.n + k], lr_scale_of(P, (int)k + (isv ? P.r : 0))) << (4 * h);
+          const uint32_t c = int4_code(m[(int64_t)i * P.n + k], lr_scale_of(P, (int)k + (isv ? P.r : 0)));
+          byte |= c << (4 * h);
+          const int q = (c & 0x8) ? (int)c - 16 : (int)c;
+          const int64_t o = (int64_t)i * P.kp + k;
+          if (isv)
+            lr_operand_store(P.vbhi, P.vblo, o,
+                             (float)((double)q * (double)lr_scale_of(P, (int)k) * (double)lr_scale_of(P, P.r + (int)k)));
+          else
+            lr_operand_store(P.uahi, nullptr, o, (float)q);
         }
       }
       body[(isv ? P.sec2 : P.sec1) + bb] = (uint8_t)byte;
@@ -817,8 +839,18 @@ __global__ void __launch_bounds__(256) lr_pack_kernel(PackArgs P) {
     float *u = reinterpret_cast<float *>(body);
     float *vv = reinterpret_cast<float *>(body + P.sec2);
     const int64_t un = P.rows * P.r, vn = P.cols * P.r;
-    for (int64_t e = tid; e < un; e += nthr) u[e] = P.q[(e / P.r) * P.n + e % P.r];
-    for (int64_t e = tid; e < vn; e += nthr) vv[e] = P.v[(e / P.r) * P.n + e % P.r];
+    for (int64_t e = tid; e < un; e += nthr) {
+      const int64_t i = e / P.r, k = e % P.r;
+      const float x = P.q[i * P.n + k];
+      u[e] = x;
+      lr_operand_store(P.uahi, P.ualo, i * P.kp + k, x);
+    }
+    for (int64_t e = tid; e < vn; e += nthr) {
+      const int64_t i = e / P.r, k = e % P.r;
+      const float x = P.v[i * P.n + k];
+      vv[e] = x;
+      lr_operand_store(P.vbhi, P.vblo, i * P.kp + k, x);
+    }
     for (int64_t b = un * 4 + tid; b < P.sec2; b += nthr) body[b] = 0;
     for (int64_t b = P.sec2 + vn * 4 + tid; b < P.body; b += nthr) body[b] = 0;
   }
@@ -829,7 +861,8 @@ __device__ __forceinline__ int nibble_at(const uint8_t *base, int64_t idx) {
   return (v & 0x8) ? v - 16 : v;
 }
 
-// Reconstruction operands from the payload alone (both roles): A = U
+// Reconstruction operands from the payload alone (the receiver; the sender's
+// pack kernel writes the same values): A = U
 // ([rows][kp]; INT4: the integer codes, exact in bf16; fp32 factors: split),
 // B = V scaled ([cols][kp], split; INT4: fp32(qV * sU * sV) per entry).
 struct DequantArgs {
@@ -1335,25 +1368,25 @@ cudaError_t launch_chol(int n, double *L, int *dead, double near_id, cudaStream_
 }
 
 cudaError_t launch_apply(int n, const float *x, const double *M, int64_t rows, float *q, __nv_bfloat16 *qthi,
-                         __nv_bfloat16 *qtlo, cudaStream_t st) {
+                         __nv_bfloat16 *qtlo, int r, unsigned *amax, cudaStream_t st) {
   const unsigned grid = (unsigned)((rows + kApplyRows - 1) / kApplyRows);
   const size_t sm = apply_smem(n);
   switch (n / 16) {
-    case 1: launch_pdl(lr_apply_kernel<1>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
-    case 2: launch_pdl(lr_apply_kernel<2>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
-    case 3: launch_pdl(lr_apply_kernel<3>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
-    case 4: launch_pdl(lr_apply_kernel<4>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
-    case 5: launch_pdl(lr_apply_kernel<5>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
-    case 6: launch_pdl(lr_apply_kernel<6>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
-    case 7: launch_pdl(lr_apply_kernel<7>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
-    case 8: launch_pdl(lr_apply_kernel<8>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo); break;
+    case 1: launch_pdl(lr_apply_kernel<1>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
+    case 2: launch_pdl(lr_apply_kernel<2>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
+    case 3: launch_pdl(lr_apply_kernel<3>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
+    case 4: launch_pdl(lr_apply_kernel<4>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
+    case 5: launch_pdl(lr_apply_kernel<5>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
+    case 6: launch_pdl(lr_apply_kernel<6>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
+    case 7: launch_pdl(lr_apply_kernel<7>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
+    case 8: launch_pdl(lr_apply_kernel<8>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }
 
 cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int64_t rows, bool final_pass,
-                           cudaStream_t st) {
+                           unsigned *amax, cudaStream_t st) {
   const LowrankBufs &b = P.b;
   const int n = P.rp;
   const int nblk = (int)(rows / kGramRows);
@@ -1364,7 +1397,8 @@ cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int
   launch_pdl(lr_gram_reduce_kernel, dim3((unsigned)((n * n + 31) / 32)), dim3(256), 0, st, b.gpart, nblk, n, b.L);
   e = launch_chol(n, b.L, b.dead, final_pass ? P.qr2_tol : 0.0, st);
   if (e != cudaSuccess) return e;
-  return launch_apply(n, b.xbuf, b.L, rows, b.q, final_pass ? b.qthi : nullptr, final_pass ? b.qtlo : nullptr, st);
+  return launch_apply(n, b.xbuf, b.L, rows, b.q, final_pass ? b.qthi : nullptr, final_pass ? b.qtlo : nullptr, P.rank,
+                      amax, st);
 }
 
 PackArgs pack_args(const LowrankPlan &P, uint8_t *payload, const Header &hdr) {
@@ -1389,6 +1423,11 @@ PackArgs pack_args(const LowrankPlan &P, uint8_t *payload, const Header &hdr) {
   }
   A.hdr = hdr;
   A.amax = P.b.amax;
+  A.kp = P.kp;
+  A.uahi = P.b.uahi;
+  A.ualo = P.int4 ? nullptr : P.b.ualo;
+  A.vbhi = P.b.vbhi;
+  A.vblo = P.b.vblo;
   return A;
 }
 
@@ -1411,7 +1450,8 @@ cudaError_t dequant_and_recon(const LowrankPlan &P, const uint8_t *payload, bool
   D.check_header = receiver;
   D.expect = expect;
   D.status = status;
-  launch_pdl(lr_dequant_kernel, dim3(1184), dim3(256), 0, st, D);
+  // the sender's operands were written by the pack kernel from the same values
+  if (receiver) launch_pdl(lr_dequant_kernel, dim3(1184), dim3(256), 0, st, D);
   ReconArgs R{};
   R.rows = P.rows;
   R.cols = P.cols;
@@ -1458,21 +1498,24 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
     if ((e = launch_thin(P, P.tm_dhi, P.tm_dlo, P.tm_vthi, P.tm_vtlo, b.ypart, R, C, P.sy, args.status, st)) !=
         cudaSuccess)
       return e;
+    // the last sweep's Q and V feed the INT4 scales: their column maxima are
+    // taken where they are written
+    const bool more = it + 1 < P.iters;
+    unsigned *amax_q = (P.int4 && !more) ? b.amax : nullptr;
+    unsigned *amax_v = (P.int4 && !more) ? b.amax + P.rp : nullptr;
     // Q = orth(Y): CholeskyQR2
-    if ((e = orthonormalise(P, b.ypart, P.sy, R, false, st)) != cudaSuccess) return e;
-    if ((e = orthonormalise(P, b.q, 1, R, true, st)) != cudaSuccess) return e;
+    if ((e = orthonormalise(P, b.ypart, P.sy, R, false, nullptr, st)) != cudaSuccess) return e;
+    if ((e = orthonormalise(P, b.q, 1, R, true, amax_q, st)) != cudaSuccess) return e;
     // V = D^T Q
     if ((e = launch_thin(P, P.tm_dthi, P.tm_dtlo, P.tm_qthi, P.tm_qtlo, b.vpart, C, R, P.sv, args.status, st)) !=
         cudaSuccess)
       return e;
-    const bool more = it + 1 < P.iters;
     launch_pdl(lr_vsum_kernel, dim3(592), dim3(256), 0, st, b.vpart, P.sv, C, P.rp, P.rank, b.v, vprev, more ? b.vthi : nullptr,
-                                        more ? b.vtlo : nullptr);
+                                        more ? b.vtlo : nullptr, amax_v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // INT4 (or fp32) factors into the payload
   const PackArgs pa = pack_args(P, args.payload, args.hdr);
-  if (P.int4) launch_pdl(lr_scale_kernel, dim3((unsigned)((R + C) / kScaleRows)), dim3(256), 0, st, pa);
   launch_pdl(lr_pack_kernel, dim3(592), dim3(256), 0, st, pa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // sender reconstruction from the payload bytes
