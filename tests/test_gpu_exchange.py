@@ -1,7 +1,7 @@
 """The sequence-parallel exchange on the GPU path: libcf codecs, NCCL
-all-gather on a communication stream.  Every gpurun call has one GPU, so this
-runs a world of one (the collective degenerates to a copy); the multi-rank
-host logic is covered on CPU by test_exchange.py."""
+all-gather on a communication stream.  The test runs a world of one rank on
+one GPU (the collective degenerates to a copy); the multi-rank host logic is
+covered on the CPU by test_exchange.py."""
 import os
 import socket
 
