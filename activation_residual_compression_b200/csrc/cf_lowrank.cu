@@ -128,18 +128,15 @@ __global__ void __launch_bounds__(kVprepThreads) lr_vprep_kernel(const float *vp
 
 // ---------------------------------------------------------------- residual pass
 
-// D = (a - ahat) + e for a 64 x 64 tile, written as split bf16 both
-// row-major ([rows][cols], the K-major A operand of Y = D V) and transposed
-// ([cols][rows], the K-major A operand of V = D^T Q).  The fp32 D is not
-// stored: the reconstruction pass recomputes it bit for bit.
+// D = (a - ahat) + e split in two bf16 terms, row-major ([rows][cols]): the
+// K-major A operand of Y = D V and the MN-major A operand of V = D^T Q.  A
+// block covers 64 rows x 64 columns (4 per thread per row pass).  The fp32 D
+// is not stored: the reconstruction pass recomputes it bit for bit.
 template <typename T>
 __global__ void __launch_bounds__(256) lr_delta_kernel(const T *a, const float *ahat, const float *err, int ef_explicit,
                                                        int64_t rows, int64_t cols, __nv_bfloat16 *dhi,
-                                                       __nv_bfloat16 *dlo, __nv_bfloat16 *dthi,
-                                                       __nv_bfloat16 *dtlo) {
+                                                       __nv_bfloat16 *dlo) {
   pdl_enter();
-  __shared__ __nv_bfloat16 shi[64][72];
-  __shared__ __nv_bfloat16 slo[64][72];
   const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll
@@ -166,8 +163,6 @@ __global__ void __launch_bounds__(256) lr_delta_kernel(const T *a, const float *
       const float tt = __fsub_rn(x[k], hv[k]);
       const float d = ef_explicit ? __fadd_rn(tt, ev[k]) : tt;
       split_bf16(d, hi[k], lo[k]);
-      shi[lr][4 * tx + k] = hi[k];
-      slo[lr][4 * tx + k] = lo[k];
     }
     uint2 ph, pl;
     ph.x = (uint32_t)__bfloat16_as_ushort(hi[0]) | ((uint32_t)__bfloat16_as_ushort(hi[1]) << 16);
@@ -177,23 +172,6 @@ __global__ void __launch_bounds__(256) lr_delta_kernel(const T *a, const float *
     *reinterpret_cast<uint2 *>(dhi + off) = ph;
     *reinterpret_cast<uint2 *>(dlo + off) = pl;
   }
-  __syncthreads();
-  // transposed: output row c0 + oc holds rows r0 .. r0 + 63 of column oc
-  const int oc = threadIdx.x >> 2, part = threadIdx.x & 3;
-  uint32_t wh[8], wl[8];
-#pragma unroll
-  for (int k = 0; k < 8; k++) {
-    const int rr = part * 16 + 2 * k;
-    wh[k] = (uint32_t)__bfloat16_as_ushort(shi[rr][oc]) | ((uint32_t)__bfloat16_as_ushort(shi[rr + 1][oc]) << 16);
-    wl[k] = (uint32_t)__bfloat16_as_ushort(slo[rr][oc]) | ((uint32_t)__bfloat16_as_ushort(slo[rr + 1][oc]) << 16);
-  }
-  const int64_t toff = (c0 + oc) * rows + r0 + part * 16;
-  uint4 *th = reinterpret_cast<uint4 *>(dthi + toff);
-  uint4 *tl = reinterpret_cast<uint4 *>(dtlo + toff);
-  th[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-  th[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
-  tl[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-  tl[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
 }
 
 // ---------------------------------------------------------------- thin GEMM (tcgen05)
@@ -205,11 +183,13 @@ struct ThinArgs {
   int kblocks;    // K / 64
   int splits;
   int stages;
+  int a_mn;       // A stored K x M (M contiguous): loaded in 64 x 64 boxes, MN-major descriptors
   int *status;
 };
 
 // out[s] = A[:, K_s] * B[:, K_s]^T for the s-th K range, A = ahi + alo
-// ([M][K] bf16, K-major), B = bhi + blo ([n][K] bf16, K-major), summing the
+// ([M][K] bf16, K-major; or, with a_mn, [K][M], MN-major), B = bhi + blo
+// ([n][K] bf16, K-major), summing the
 // products hi*hi + hi*lo + lo*hi in fp32 tensor memory.  One CTA per
 // (128-row tile, K split); warp 0 lane 0 streams tiles with TMA into a ring
 // of shared-memory stages, warp 1 lane 0 issues the MMAs, all four warps
@@ -264,14 +244,21 @@ __global__ void __launch_bounds__(128, 1)
       uint8_t *base = sm + (size_t)st * stage_bytes;
       umma::mbar_arrive_expect_tx(&full[st], stage_bytes);
       const int kc = (kb0 + i) * kTileK;
-      umma::tma_load_2d(base, &ta_hi, kc, m0, &full[st]);
-      umma::tma_load_2d(base + a_bytes, &ta_lo, kc, m0, &full[st]);
+      if (A.a_mn) {  // two 64-column halves of the M tile, 64 K rows each
+        umma::tma_load_2d(base, &ta_hi, m0, kc, &full[st]);
+        umma::tma_load_2d(base + a_bytes / 2, &ta_hi, m0 + kTileK, kc, &full[st]);
+        umma::tma_load_2d(base + a_bytes, &ta_lo, m0, kc, &full[st]);
+        umma::tma_load_2d(base + a_bytes + a_bytes / 2, &ta_lo, m0 + kTileK, kc, &full[st]);
+      } else {
+        umma::tma_load_2d(base, &ta_hi, kc, m0, &full[st]);
+        umma::tma_load_2d(base + a_bytes, &ta_lo, kc, m0, &full[st]);
+      }
       umma::tma_load_2d(base + 2 * a_bytes, &tb_hi, kc, 0, &full[st]);
       umma::tma_load_2d(base + 2 * a_bytes + b_bytes, &tb_lo, kc, 0, &full[st]);
     }
   } else if (warp == 1 && lane == 0) {
     // MMA issuer
-    const uint32_t idesc = umma::idesc_bf16_f32(kTileM, A.n);
+    const uint32_t idesc = umma::idesc_bf16_f32(kTileM, A.n, A.a_mn != 0);
     for (int i = 0; i < nk && ok; i++) {
       const int st = i % ST;
       if (!umma::mbar_wait(&full[st], (uint32_t)((i / ST) & 1))) { ok = 0; break; }
@@ -279,8 +266,12 @@ __global__ void __launch_bounds__(128, 1)
       const uint32_t base = umma::saddr(sm + (size_t)st * stage_bytes);
 #pragma unroll
       for (int kk = 0; kk < kTileK / 16; kk++) {
-        const uint64_t ah = umma::desc_kmajor_sw128(base + kk * 32);
-        const uint64_t al = umma::desc_kmajor_sw128(base + a_bytes + kk * 32);
+        // K-major: the k-th 16-column slice is 32 bytes into each row; MN-major:
+        // 16 K rows (2048 bytes) further, the M halves a_bytes / 2 apart
+        const uint64_t ah = A.a_mn ? umma::desc_mnmajor_sw128(base + kk * 2048, a_bytes / 2)
+                                   : umma::desc_kmajor_sw128(base + kk * 32);
+        const uint64_t al = A.a_mn ? umma::desc_mnmajor_sw128(base + a_bytes + kk * 2048, a_bytes / 2)
+                                   : umma::desc_kmajor_sw128(base + a_bytes + kk * 32);
         const uint64_t bh = umma::desc_kmajor_sw128(base + 2 * a_bytes + kk * 32);
         const uint64_t bl = umma::desc_kmajor_sw128(base + 2 * a_bytes + b_bytes + kk * 32);
         umma::mma_bf16(tmem, ah, bh, idesc, (i > 0 || kk > 0) ? 1u : 0u);
@@ -1230,7 +1221,7 @@ void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *p
   dec += pad256(R * kp * 2) * 2;  // uahi, ualo
   dec += pad256(C * kp * 2) * 2;  // vbhi, vblo
   size_t enc = dec;
-  enc += pad256(R * C * 2) * 4;                               // dhi dlo dthi dtlo
+  enc += pad256(R * C * 2) * 2;                               // dhi dlo
   enc += pad256(rp * C * 2) * 2 + pad256(rp * R * 2) * 2;     // vt, qt
   enc += pad256((size_t)plan->sy * R * rp * 4);               // ypart
   enc += pad256((size_t)plan->sv * C * rp * 4);               // vpart
@@ -1285,8 +1276,6 @@ int lowrank_bind(LowrankPlan *plan, void *scratch) {
   if (plan->role == CF_SENDER) {
     b.dhi = reinterpret_cast<__nv_bfloat16 *>(take(R * C * 2));
     b.dlo = reinterpret_cast<__nv_bfloat16 *>(take(R * C * 2));
-    b.dthi = reinterpret_cast<__nv_bfloat16 *>(take(R * C * 2));
-    b.dtlo = reinterpret_cast<__nv_bfloat16 *>(take(R * C * 2));
     b.vthi = reinterpret_cast<__nv_bfloat16 *>(take(rp * C * 2));
     b.vtlo = reinterpret_cast<__nv_bfloat16 *>(take(rp * C * 2));
     b.qthi = reinterpret_cast<__nv_bfloat16 *>(take(rp * R * 2));
@@ -1302,7 +1291,7 @@ int lowrank_bind(LowrankPlan *plan, void *scratch) {
     b.amax = reinterpret_cast<unsigned *>(take(2 * rp * 4));
     ok = ok && make_map(&plan->tm_dhi, b.dhi, C, R, kTileM) && make_map(&plan->tm_dlo, b.dlo, C, R, kTileM) &&
          make_map(&plan->tm_vthi, b.vthi, C, rp, (uint32_t)rp) && make_map(&plan->tm_vtlo, b.vtlo, C, rp, (uint32_t)rp) &&
-         make_map(&plan->tm_dthi, b.dthi, R, C, kTileM) && make_map(&plan->tm_dtlo, b.dtlo, R, C, kTileM) &&
+         make_map(&plan->tm_dmhi, b.dhi, C, R, kTileK) && make_map(&plan->tm_dmlo, b.dlo, C, R, kTileK) &&
          make_map(&plan->tm_qthi, b.qthi, R, rp, (uint32_t)rp) && make_map(&plan->tm_qtlo, b.qtlo, R, rp, (uint32_t)rp);
   }
   if (!ok) return CF_ERR_CUDA;
@@ -1322,7 +1311,7 @@ namespace {
 
 cudaError_t launch_thin(const LowrankPlan &P, const CUtensorMap &ah, const CUtensorMap &al, const CUtensorMap &bh,
                         const CUtensorMap &bl, float *out, int64_t M, int64_t K, int splits, int *status,
-                        cudaStream_t st) {
+                        cudaStream_t st, bool a_mn = false) {
   ThinArgs A{};
   A.out = out;
   A.M = M;
@@ -1330,6 +1319,7 @@ cudaError_t launch_thin(const LowrankPlan &P, const CUtensorMap &ah, const CUten
   A.kblocks = (int)(K / kTileK);
   A.splits = splits;
   A.stages = thin_stages(P.rp);
+  A.a_mn = a_mn ? 1 : 0;
   A.status = status;
   launch_pdl(lr_thin_gemm_kernel, dim3(dim3((unsigned)(M / kTileM), (unsigned)splits)), dim3(128), thin_smem(P.rp, A.stages), st, 
       ah, al, bh, bl, A);
@@ -1487,10 +1477,10 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
   const dim3 dg((unsigned)(C / 64), (unsigned)(R / 64));
   if (P.dtype == CF_BF16)
     launch_pdl(lr_delta_kernel<__nv_bfloat16>, dim3(dg), dim3(256), 0, st, static_cast<const __nv_bfloat16 *>(args.a), args.ahat, args.err,
-                                                        P.ef_explicit, R, C, b.dhi, b.dlo, b.dthi, b.dtlo);
+                                                        P.ef_explicit, R, C, b.dhi, b.dlo);
   else
     launch_pdl(lr_delta_kernel<float>, dim3(dg), dim3(256), 0, st, static_cast<const float *>(args.a), args.ahat, args.err, P.ef_explicit,
-                                               R, C, b.dhi, b.dlo, b.dthi, b.dtlo);
+                                               R, C, b.dhi, b.dlo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   for (int it = 0; it < P.iters; it++) {
@@ -1507,7 +1497,7 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
     if ((e = orthonormalise(P, b.ypart, P.sy, R, false, nullptr, st)) != cudaSuccess) return e;
     if ((e = orthonormalise(P, b.q, 1, R, true, amax_q, st)) != cudaSuccess) return e;
     // V = D^T Q
-    if ((e = launch_thin(P, P.tm_dthi, P.tm_dtlo, P.tm_qthi, P.tm_qtlo, b.vpart, C, R, P.sv, args.status, st)) !=
+    if ((e = launch_thin(P, P.tm_dmhi, P.tm_dmlo, P.tm_qthi, P.tm_qtlo, b.vpart, C, R, P.sv, args.status, st, true)) !=
         cudaSuccess)
       return e;
     launch_pdl(lr_vsum_kernel, dim3(592), dim3(256), 0, st, b.vpart, P.sv, C, P.rp, P.rank, b.v, vprev, more ? b.vthi : nullptr,

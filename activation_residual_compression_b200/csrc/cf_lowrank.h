@@ -14,7 +14,6 @@ namespace cfi {
 struct LowrankBufs {
   // sender only
   __nv_bfloat16 *dhi = nullptr, *dlo = nullptr;    // residual D split in two bf16 terms, [rows][cols]
-  __nv_bfloat16 *dthi = nullptr, *dtlo = nullptr;  // the same, transposed [cols][rows]
   __nv_bfloat16 *vthi = nullptr, *vtlo = nullptr;  // V^T split, [rp][cols]
   __nv_bfloat16 *qthi = nullptr, *qtlo = nullptr;  // Q^T split, [rp][rows]
   float *ypart = nullptr;                          // split-K partial products [sy][rows][rp]
@@ -43,7 +42,7 @@ struct LowrankPlan {
   bool supported = false;
   LowrankBufs b;
   CUtensorMap tm_dhi, tm_dlo, tm_vthi, tm_vtlo;    // Y = D V
-  CUtensorMap tm_dthi, tm_dtlo, tm_qthi, tm_qtlo;  // V = D^T Q
+  CUtensorMap tm_dmhi, tm_dmlo, tm_qthi, tm_qtlo;  // V = D^T Q (D read MN-major: 64 x 64 boxes)
   CUtensorMap tm_uahi, tm_ualo, tm_vbhi, tm_vblo;  // C = U V^T
 };
 

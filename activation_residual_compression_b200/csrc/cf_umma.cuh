@@ -1,7 +1,8 @@
 // cf_umma.cuh -- sm_100a primitives for the low-rank mode's GEMMs: mbarriers,
 // 2-D TMA tile loads (no multicast), tcgen05 (UMMA) issue / commit, tensor
 // memory allocation and loads, and the shared-memory / instruction
-// descriptors for K-major bf16 tiles in the 128-byte swizzled layout.
+// descriptors for K-major and MN-major bf16 tiles in the 128-byte swizzled
+// layout.
 //
 // Tile convention: a K-major operand tile is R rows x 64 bf16 (128 bytes per
 // row) written by TMA with 128-byte swizzling into a 1024-byte aligned
@@ -135,11 +136,28 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t smem_addr) {
   return d;
 }
 
+// Shared-memory descriptor of an MN-major bf16 tile in the 128-byte swizzled
+// layout, as TMA writes boxes of 64 MN-contiguous elements x K rows: each
+// K row is one 128-byte swizzle row, 8 K rows form a 1024-byte group (the
+// stride byte offset, between groups along K), and the leading byte offset
+// is the distance between consecutive 64-element blocks along MN.  A K = 16
+// slice starts 2048 bytes (16 rows) after the previous one.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t smem_addr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo & 0x3FFFFu) >> 4) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
 // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
-// (bits 7-9 = 1, 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits
-// 17-22, M >> 4 at bits 24-28.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+// (bits 7-9 = 1, 10-12 = 1), B K-major (bit 16 = 0), A K-major or, with
+// a_mn, MN-major (bit 15), N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace umma
