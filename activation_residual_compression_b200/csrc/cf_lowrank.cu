@@ -130,8 +130,10 @@ __global__ void __launch_bounds__(kVprepThreads) lr_vprep_kernel(const float *vp
 
 // D = (a - ahat) + e split in two bf16 terms, row-major ([rows][cols]): the
 // K-major A operand of Y = D V and the MN-major A operand of V = D^T Q.  A
-// block covers 64 rows x 64 columns (4 per thread per row pass).  The fp32 D
-// is not stored: the reconstruction pass recomputes it bit for bit.
+// block covers 64 rows x 64 columns (4 per thread per row pass).  The inputs
+// are read once (evict-first loads), so the split, which both products read
+// next, is more likely to stay in L2.  The fp32 D is not stored: the
+// reconstruction pass recomputes it bit for bit.
 template <typename T>
 __global__ void __launch_bounds__(256) lr_delta_kernel(const T *a, const float *ahat, const float *err, int ef_explicit,
                                                        int64_t rows, int64_t cols, __nv_bfloat16 *dhi,
@@ -145,17 +147,17 @@ __global__ void __launch_bounds__(256) lr_delta_kernel(const T *a, const float *
     const int64_t off = (r0 + lr) * cols + c0 + 4 * tx;
     float x[4];
     if constexpr (sizeof(T) == 2) {
-      const uint2 raw = *reinterpret_cast<const uint2 *>(a + off);
+      const uint2 raw = __ldcs(reinterpret_cast<const uint2 *>(a + off));
       x[0] = __uint_as_float(raw.x << 16);
       x[1] = __uint_as_float(raw.x & 0xffff0000u);
       x[2] = __uint_as_float(raw.y << 16);
       x[3] = __uint_as_float(raw.y & 0xffff0000u);
     } else {
-      const float4 f = *reinterpret_cast<const float4 *>(a + off);
+      const float4 f = __ldcs(reinterpret_cast<const float4 *>(a + off));
       x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
     }
-    const float4 h = *reinterpret_cast<const float4 *>(ahat + off);
-    const float4 e = ef_explicit ? *reinterpret_cast<const float4 *>(err + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 h = __ldcs(reinterpret_cast<const float4 *>(ahat + off));
+    const float4 e = ef_explicit ? __ldcs(reinterpret_cast<const float4 *>(err + off)) : make_float4(0.f, 0.f, 0.f, 0.f);
     const float hv[4] = {h.x, h.y, h.z, h.w}, ev[4] = {e.x, e.y, e.z, e.w};
     __nv_bfloat16 hi[4], lo[4];
 #pragma unroll
