@@ -186,6 +186,7 @@ struct ThinArgs {
   int splits;
   int stages;
   int a_mn;       // A stored K x M (M contiguous): loaded in 64 x 64 boxes, MN-major descriptors
+  int a_l2;       // L2 priority of A's lines: 0 default, 1 keep (read again later), 2 last use
   int *status;
 };
 
@@ -240,6 +241,11 @@ __global__ void __launch_bounds__(128, 1)
 
   if (warp == 0 && lane == 0) {
     // producer
+    const uint64_t pol = A.a_l2 == 1 ? umma::policy_evict_last() : umma::policy_evict_first();
+    auto load_a = [&](void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
+      if (A.a_l2) umma::tma_load_2d_hint(dst, map, c0, c1, bar, pol);
+      else umma::tma_load_2d(dst, map, c0, c1, bar);
+    };
     for (int i = 0; i < nk && ok; i++) {
       const int st = i % ST;
       if (i >= ST && !umma::mbar_wait(&empty[st], (uint32_t)(((i / ST) - 1) & 1))) { ok = 0; break; }
@@ -247,13 +253,13 @@ __global__ void __launch_bounds__(128, 1)
       umma::mbar_arrive_expect_tx(&full[st], stage_bytes);
       const int kc = (kb0 + i) * kTileK;
       if (A.a_mn) {  // two 64-column halves of the M tile, 64 K rows each
-        umma::tma_load_2d(base, &ta_hi, m0, kc, &full[st]);
-        umma::tma_load_2d(base + a_bytes / 2, &ta_hi, m0 + kTileK, kc, &full[st]);
-        umma::tma_load_2d(base + a_bytes, &ta_lo, m0, kc, &full[st]);
-        umma::tma_load_2d(base + a_bytes + a_bytes / 2, &ta_lo, m0 + kTileK, kc, &full[st]);
+        load_a(base, &ta_hi, m0, kc, &full[st]);
+        load_a(base + a_bytes / 2, &ta_hi, m0 + kTileK, kc, &full[st]);
+        load_a(base + a_bytes, &ta_lo, m0, kc, &full[st]);
+        load_a(base + a_bytes + a_bytes / 2, &ta_lo, m0 + kTileK, kc, &full[st]);
       } else {
-        umma::tma_load_2d(base, &ta_hi, kc, m0, &full[st]);
-        umma::tma_load_2d(base + a_bytes, &ta_lo, kc, m0, &full[st]);
+        load_a(base, &ta_hi, kc, m0, &full[st]);
+        load_a(base + a_bytes, &ta_lo, kc, m0, &full[st]);
       }
       umma::tma_load_2d(base + 2 * a_bytes, &tb_hi, kc, 0, &full[st]);
       umma::tma_load_2d(base + 2 * a_bytes + b_bytes, &tb_lo, kc, 0, &full[st]);
@@ -1313,7 +1319,7 @@ namespace {
 
 cudaError_t launch_thin(const LowrankPlan &P, const CUtensorMap &ah, const CUtensorMap &al, const CUtensorMap &bh,
                         const CUtensorMap &bl, float *out, int64_t M, int64_t K, int splits, int *status,
-                        cudaStream_t st, bool a_mn = false) {
+                        cudaStream_t st, bool a_mn = false, int a_l2 = 0) {
   ThinArgs A{};
   A.out = out;
   A.M = M;
@@ -1322,6 +1328,7 @@ cudaError_t launch_thin(const LowrankPlan &P, const CUtensorMap &ah, const CUten
   A.splits = splits;
   A.stages = thin_stages(P.rp);
   A.a_mn = a_mn ? 1 : 0;
+  A.a_l2 = a_l2;
   A.status = status;
   launch_pdl(lr_thin_gemm_kernel, dim3(dim3((unsigned)(M / kTileM), (unsigned)splits)), dim3(128), thin_smem(P.rp, A.stages), st, 
       ah, al, bh, bl, A);
@@ -1487,7 +1494,8 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
   if (e != cudaSuccess) return e;
   for (int it = 0; it < P.iters; it++) {
     // Y = D V
-    if ((e = launch_thin(P, P.tm_dhi, P.tm_dlo, P.tm_vthi, P.tm_vtlo, b.ypart, R, C, P.sy, args.status, st)) !=
+    if ((e = launch_thin(P, P.tm_dhi, P.tm_dlo, P.tm_vthi, P.tm_vtlo, b.ypart, R, C, P.sy, args.status, st, false,
+                         1)) !=
         cudaSuccess)
       return e;
     // the last sweep's Q and V feed the INT4 scales: their column maxima are
@@ -1499,7 +1507,8 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
     if ((e = orthonormalise(P, b.ypart, P.sy, R, false, nullptr, st)) != cudaSuccess) return e;
     if ((e = orthonormalise(P, b.q, 1, R, true, amax_q, st)) != cudaSuccess) return e;
     // V = D^T Q
-    if ((e = launch_thin(P, P.tm_dmhi, P.tm_dmlo, P.tm_qthi, P.tm_qtlo, b.vpart, C, R, P.sv, args.status, st, true)) !=
+    if ((e = launch_thin(P, P.tm_dmhi, P.tm_dmlo, P.tm_qthi, P.tm_qtlo, b.vpart, C, R, P.sv, args.status, st, true,
+                         2)) !=
         cudaSuccess)
       return e;
     launch_pdl(lr_vsum_kernel, dim3(592), dim3(256), 0, st, b.vpart, P.sv, C, P.rp, P.rank, b.v, vprev, more ? b.vthi : nullptr,
