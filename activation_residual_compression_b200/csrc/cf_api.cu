@@ -39,7 +39,7 @@ struct cf_state {
   Layout lay{};
   LowrankPlan lr{};
   BlockselPlan bs{};
-  // Low-rank sender: the encode chain (15 launches for one sweep) runs as
+  // Low-rank sender: the encode chain (14 launches for one sweep) runs as
   // one CUDA graph, captured on a private stream at each call and swapped
   // into the executable graph with cudaGraphExecUpdate (same topology, new
   // arguments), so that the chain pays one graph launch instead of a stream

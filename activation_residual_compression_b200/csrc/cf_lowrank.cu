@@ -706,6 +706,96 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
   }
 }
 
+// The first CholeskyQR pass's Q1 = X M for kGramRows rows per block, with
+// the sums of lr_apply_kernel (each output's two halves of the term range in
+// separate fp64 accumulators, added at the end; thread (row, q) takes the 2 TT
+// outputs c = q + 8 t), and the partial Gram matrix Q1^T Q1 of these rows from
+// the fp32 values it stores, with the sums of lr_gram_kernel: the second pass
+// needs no Gram kernel, and both results are bit-identical to the separate
+// kernels'.
+template <int TT>
+__global__ void __launch_bounds__(256) lr_apply_gram_kernel(const float *x, const double *M, int64_t rows, float *q,
+                                                            double *gpart) {
+  pdl_enter();
+  constexpr int n = 16 * TT, xld = apply_xld<TT>(), h = n / 2, S = TT | 1;
+  extern __shared__ __align__(16) uint8_t asm_[];
+  double *Ms = reinterpret_cast<double *>(asm_);                          // [n][n]
+  float *xs = reinterpret_cast<float *>(Ms + n * n);                      // [kGramRows][xld]
+  float (*tile)[16 * S] = reinterpret_cast<float (*)[16 * S]>(xs + kGramRows * xld);  // [kGramRows][16 S]
+  const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
+  {
+    const double2 *M2 = reinterpret_cast<const double2 *>(M);
+    double2 *Ms2 = reinterpret_cast<double2 *>(Ms);
+    constexpr int NM = n * n / 2;
+#pragma unroll
+    for (int v = 0; v < (NM + 255) / 256; v++) {
+      const int e = threadIdx.x + 256 * v;
+      if (e < NM) Ms2[e] = M2[e];
+    }
+    const float4 *x4 = reinterpret_cast<const float4 *>(x) + r0 * (n / 4);
+    constexpr int NX = kGramRows * n / 4;
+#pragma unroll
+    for (int v = 0; v < (NX + 255) / 256; v++) {
+      const int e = threadIdx.x + 256 * v;
+      if (e < NX) {
+        const int rr = e / (n / 4), c = (e % (n / 4)) * 4;
+        const float4 val = r0 + rr < rows ? x4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(xs + rr * xld + c) = val;
+      }
+    }
+  }
+  __syncthreads();
+  {
+    const int lr = threadIdx.x >> 3, qc = threadIdx.x & 7;
+    double acc0[2 * TT], acc1[2 * TT];
+#pragma unroll
+    for (int t = 0; t < 2 * TT; t++) acc0[t] = acc1[t] = 0.0;
+#pragma unroll 2
+    for (int j = 0; j < h; j++) {
+      const double x0 = (double)xs[lr * xld + j], x1 = (double)xs[lr * xld + h + j];
+      const double *m0 = Ms + j * n + qc, *m1 = Ms + (h + j) * n + qc;
+#pragma unroll
+      for (int t = 0; t < 2 * TT; t++) {
+        acc0[t] = fma(x0, m0[8 * t], acc0[t]);
+        acc1[t] = fma(x1, m1[8 * t], acc1[t]);
+      }
+    }
+    const int64_t row = r0 + lr;
+#pragma unroll
+    for (int t = 0; t < 2 * TT; t++) {
+      const int c = qc + 8 * t;
+      const float v = row < rows ? (float)(acc0[t] + acc1[t]) : 0.0f;
+      if (row < rows) q[row * n + c] = v;
+      tile[lr][gram_col<TT>(c)] = v;
+    }
+  }
+  __syncthreads();
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  double acc[TT][TT];
+#pragma unroll
+  for (int a = 0; a < TT; a++)
+#pragma unroll
+    for (int c = 0; c < TT; c++) acc[a][c] = 0.0;
+#pragma unroll 4
+  for (int rr = 0; rr < kGramRows; rr++) {
+    double xi[TT], xj[TT];
+#pragma unroll
+    for (int a = 0; a < TT; a++) {
+      xi[a] = (double)tile[rr][ty * S + a];
+      xj[a] = (double)tile[rr][tx * S + a];
+    }
+#pragma unroll
+    for (int a = 0; a < TT; a++)
+#pragma unroll
+      for (int c = 0; c < TT; c++) acc[a][c] = fma(xi[a], xj[c], acc[a][c]);
+  }
+  double *g = gpart + (int64_t)blockIdx.x * n * n;
+#pragma unroll
+  for (int a = 0; a < TT; a++)
+#pragma unroll
+    for (int c = 0; c < TT; c++) g[(ty * TT + a) * n + tx * TT + c] = acc[a][c];
+}
+
 // V = sum of the partial slabs (fixed order) [cols][n]; V_prev (state,
 // [cols][r]) = V[:, :r]; when vthi != nullptr also V^T split for the next
 // iteration's Y = D V; when amax != nullptr the absmax of each of V's first r
@@ -1184,6 +1274,10 @@ size_t apply_smem(int n) {
   const size_t xt = (size_t)kApplyRows * (n + 4) * 4, qt = (size_t)n * (kApplyRows + 1) * 4;
   return (size_t)n * n * 8 + (xt > qt ? xt : qt);
 }
+size_t apply_gram_smem(int n) {
+  const int tt = n / 16, s = tt | 1;
+  return (size_t)n * n * 8 + (size_t)kGramRows * (n + 4) * 4 + (size_t)kGramRows * 16 * s * 4;
+}
 
 }  // namespace
 
@@ -1245,8 +1339,11 @@ namespace {
 
 template <int TT>
 cudaError_t set_apply_smem_tt() {
-  return cudaFuncSetAttribute(lr_apply_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)apply_smem(16 * TT));
+  cudaError_t e = cudaFuncSetAttribute(lr_apply_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)apply_smem(16 * TT));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(lr_apply_gram_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)apply_gram_smem(16 * TT));
 }
 
 cudaError_t set_apply_smem(int n) {
@@ -1384,20 +1481,40 @@ cudaError_t launch_apply(int n, const float *x, const double *M, int64_t rows, f
   return cudaGetLastError();
 }
 
+cudaError_t launch_apply_gram(int n, const float *x, const double *M, int64_t rows, float *q, double *gpart,
+                              cudaStream_t st) {
+  const unsigned grid = (unsigned)(rows / kGramRows);
+  const size_t sm = apply_gram_smem(n);
+  switch (n / 16) {
+    case 1: launch_pdl(lr_apply_gram_kernel<1>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
+    case 2: launch_pdl(lr_apply_gram_kernel<2>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
+    case 3: launch_pdl(lr_apply_gram_kernel<3>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
+    case 4: launch_pdl(lr_apply_gram_kernel<4>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
+    case 5: launch_pdl(lr_apply_gram_kernel<5>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
+    case 6: launch_pdl(lr_apply_gram_kernel<6>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
+    case 7: launch_pdl(lr_apply_gram_kernel<7>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
+    case 8: launch_pdl(lr_apply_gram_kernel<8>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int64_t rows, bool final_pass,
                            unsigned *amax, cudaStream_t st) {
   const LowrankBufs &b = P.b;
   const int n = P.rp;
   const int nblk = (int)(rows / kGramRows);
-  cudaError_t e = launch_gram(n, nblk, src, nsrc, rows, b.xbuf, b.gpart, st);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  // the first pass's partial Gram matrices come from the Gram kernel (over the
+  // split-K partials of Y), the second pass's from the first pass's apply
+  if (!final_pass && (e = launch_gram(n, nblk, src, nsrc, rows, b.xbuf, b.gpart, st)) != cudaSuccess) return e;
   // the reduced Gram matrix goes to L, which the Cholesky kernel then
   // overwrites with M = L^-T
   launch_pdl(lr_gram_reduce_kernel, dim3((unsigned)((n * n + 31) / 32)), dim3(256), 0, st, b.gpart, nblk, n, b.L);
   e = launch_chol(n, b.L, b.dead, final_pass ? P.qr2_tol : 0.0, st);
   if (e != cudaSuccess) return e;
-  return launch_apply(n, b.xbuf, b.L, rows, b.q, final_pass ? b.qthi : nullptr, final_pass ? b.qtlo : nullptr, P.rank,
-                      amax, st);
+  if (!final_pass) return launch_apply_gram(n, b.xbuf, b.L, rows, b.q, b.gpart, st);
+  return launch_apply(n, b.q, b.L, rows, b.q, b.qthi, b.qtlo, P.rank, amax, st);
 }
 
 PackArgs pack_args(const LowrankPlan &P, uint8_t *payload, const Header &hdr) {

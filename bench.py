@@ -260,8 +260,8 @@ def launches_per_call(mode, kw, encode):
         return 1
     if not encode:
         return 2                                   # dequantise, reconstruction
-    return 2 + 11 * kw["iters"] + 2                # V prep, residual; per sweep: 2 GEMMs, 2 x 4 orth., V sum;
-                                                   # pack (with the sender's operands), reconstruction
+    return 2 + 10 * kw["iters"] + 2                # V prep, residual; per sweep: 2 GEMMs, Gram, 2 x (reduce,
+                                                   # Cholesky, apply), V sum; pack, reconstruction
 
 
 def run_cf(args, rank, world, device):
