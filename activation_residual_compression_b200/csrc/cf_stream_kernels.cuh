@@ -788,11 +788,11 @@ __device__ __forceinline__ void decode_row(const DecArgs &A, const int t, const 
         for (int s = 0; s < NM_N; s++) {
           const int idx = int((fields >> (4 * s)) & 15u);
           const float val = bf16_half(in.nv[j].x, s);
-          if ((idx >> 3) == half) {
+          // position in this half, or 8 (nowhere) when the kept value is in the other
+          // half: selects only, no divergent branch
+          const int pos = ((idx >> 3) == half) ? (idx & 7) : 8;
 #pragma unroll
-            for (int k = 0; k < 8; k++)
-              if (k == (idx & 7)) c[k] = val;
-          }
+          for (int k = 0; k < 8; k++) c[k] = (k == pos) ? val : c[k];
         }
       } else {  // NM_M == 4
         const uint32_t fields = (in.w[j] >> ((v % P::G) * P::bpv)) & ((1u << P::bpv) - 1u);
