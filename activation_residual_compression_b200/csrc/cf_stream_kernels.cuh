@@ -291,14 +291,16 @@ template <int N>
 __device__ __forceinline__ void local_topn(const float (&x)[8], int k0, int cnt, float (&bv)[2], int (&bi)[2]) {
   bv[0] = -1.0f; bv[1] = -1.0f; bi[0] = 0; bi[1] = 0;
 #pragma unroll
-  for (int k = 0; k < cnt; k++) {
+  for (int k = 0; k < cnt; k++) {  // selects, no divergent branch; strict > keeps the lower index on ties
     const float a = fabsf(x[k0 + k]);
-    if (a > bv[0]) {
-      bv[1] = bv[0]; bi[1] = bi[0];
-      bv[0] = a; bi[0] = k;
-    } else if (N == 2 && a > bv[1]) {
-      bv[1] = a; bi[1] = k;
-    }
+    const bool gt0 = a > bv[0];
+    const bool gt1 = N == 2 && !gt0 && a > bv[1];
+    const float v1 = gt0 ? bv[0] : (gt1 ? a : bv[1]);
+    const int i1 = gt0 ? bi[0] : (gt1 ? k : bi[1]);
+    bv[0] = gt0 ? a : bv[0];
+    bi[0] = gt0 ? k : bi[0];
+    bv[1] = v1;
+    bi[1] = i1;
   }
 }
 
@@ -505,16 +507,19 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
             const float bvv = ib == 0 ? pv[0] : pv[1];
             const int bii = ib == 0 ? pi[0] : pi[1];
             const float bdd = ib == 0 ? pd[0] : pd[1];
-            if (better(av, ai, bvv, bii)) {
-              ki[s] = ai; kd[s] = ad; ia++;
-            } else {
-              ki[s] = bii; kd[s] = bdd; ib++;
-            }
+            const bool take_a = better(av, ai, bvv, bii);  // selects, no divergent branch
+            ki[s] = take_a ? ai : bii;
+            kd[s] = take_a ? ad : bdd;
+            ia += take_a ? 1 : 0;
+            ib += take_a ? 0 : 1;
           }
         }
-        if (NM_N == 2 && ki[0] > ki[1]) {
-          const int ti = ki[0]; ki[0] = ki[1]; ki[1] = ti;
-          const float td = kd[0]; kd[0] = kd[1]; kd[1] = td;
+        if (NM_N == 2) {  // ascending indices
+          const bool sw = ki[0] > ki[1];
+          const int i0 = sw ? ki[1] : ki[0], i1 = sw ? ki[0] : ki[1];
+          const float d0 = sw ? kd[1] : kd[0], d1 = sw ? kd[0] : kd[1];
+          ki[0] = i0; ki[1] = i1;
+          kd[0] = d0; kd[1] = d1;
         }
 #pragma unroll
         for (int k = 0; k < 8; k++) {
@@ -546,7 +551,11 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
           int bi[2];
           local_topn<NM_N>(d[j], 4 * qb, 4, bv, bi);
           int ki[2] = {bi[0], bi[1]};
-          if (NM_N == 2 && ki[0] > ki[1]) { const int ti = ki[0]; ki[0] = ki[1]; ki[1] = ti; }
+          if (NM_N == 2) {  // ascending indices, by selects
+            const bool sw = ki[0] > ki[1];
+            const int i0 = sw ? ki[1] : ki[0], i1 = sw ? ki[0] : ki[1];
+            ki[0] = i0; ki[1] = i1;
+          }
 #pragma unroll
           for (int s = 0; s < NM_N; s++) {
             float dv = d[j][4 * qb];
