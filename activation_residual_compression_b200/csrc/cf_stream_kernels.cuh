@@ -387,7 +387,6 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
 #pragma unroll
     for (int j = 0; j < VPT; j++) {
       const int v = t + (j << tlog);
-#pragma unroll
       if (row_ok && v < V) store_f32x8(reinterpret_cast<float *>(body) + r * cols + v * 8, d[j]);
     }
   } else if constexpr (MODE == M_S1) {
@@ -397,7 +396,7 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
 #pragma unroll
       for (int k = 0; k < 8; k++) m = fmaxf(m, fabsf(d[j][k]));
     m = team_max(m, tlog, sm_f);
-    float S = 0.0f;
+    float Sc = 0.0f;
     unsigned long long q = 0;
     const int Ex = m > 0.0f ? floor_log2_f32(m) : 0;
     if (m > 0.0f) {
@@ -424,7 +423,7 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
       const double p2 = __hiloint2double((Ex - kFxF + 1023) << 20, 0);
       const double mean = __ddiv_rn(__dmul_rn(__ull2double_rn(q), p2), (double)cols);
       sbits = __bfloat16_as_ushort(__float2bfloat16_rn(__double2float_rn(mean)));
-      S = __uint_as_float((uint32_t)sbits << 16);
+      Sc = __uint_as_float((uint32_t)sbits << 16);
     }
     if (row_ok && t == 0) reinterpret_cast<uint16_t *>(body)[r] = sbits;
 #pragma unroll
@@ -434,7 +433,7 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
       for (int k = 0; k < 8; k++) {
         const bool neg = d[j][k] < 0.0f;
         byte |= (uint32_t)neg << k;
-        cs1[j][k] = neg ? -S : S;
+        cs1[j][k] = neg ? -Sc : Sc;
       }
       const int v = t + (j << tlog);
       cbits[j] = byte << ((v % P::G) * P::bpv);
@@ -447,19 +446,19 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
       for (int k = 0; k < 8; k++) m = fmaxf(m, fabsf(d[j][k]));
     m = team_max(m, tlog, sm_f);
     const uint16_t sbits = __bfloat16_as_ushort(__float2bfloat16_rn(m));
-    const float S = __uint_as_float((uint32_t)sbits << 16);
+    const float Sc = __uint_as_float((uint32_t)sbits << 16);
     if (row_ok && t == 0) reinterpret_cast<uint16_t *>(body)[r] = sbits;
     float L[4];
-    q2_levels(S, L);
+    q2_levels(Sc, L);
     cL2 = L[2];
     cL3 = L[3];
-    const float k1 = S != 0.0f ? __fdiv_rn(1.5f, S) : 0.0f;
+    const float k1 = Sc != 0.0f ? __fdiv_rn(1.5f, Sc) : 0.0f;
 #pragma unroll
     for (int j = 0; j < VPT; j++) {
       uint32_t codes = 0;
 #pragma unroll
       for (int k = 0; k < 8; k++) {
-        const float qf = S != 0.0f ? q2_code(d[j][k], S, k1) : 0.0f;
+        const float qf = Sc != 0.0f ? q2_code(d[j][k], Sc, k1) : 0.0f;
         codes |= small_uint(qf) << (2 * k);
       }
       cinfo[j] = codes;
