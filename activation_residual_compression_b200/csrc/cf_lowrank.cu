@@ -478,10 +478,15 @@ __global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart
 // deficient by the first pass) is dead, as in the elimination.  Otherwise
 // the elimination runs.
 //
+// Columns nlive .. n-1 must be zero in G (the padding of the rank): they are
+// marked dead and the elimination stops after column nlive - 1, which gives
+// the same M as running the remaining steps (each would find a zero pivot).
+//
 // Writes M fp64 [n][n] (upper triangular); G and M may alias (G is read into
 // registers before the first barrier).
 template <int TT>
-__global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double *Mout, int *dead, double near_id) {
+__global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double *Mout, int *dead, double near_id,
+                                                         int nlive) {
   pdl_enter();
   constexpr int n = 16 * TT;
   constexpr int S = TT | 1;  // odd block stride of the shared vector: no bank conflicts
@@ -537,11 +542,17 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double
     for (int a = 0; a < TT; a++) u[0][ty * S + a] = (i0 + a == 0) ? 0.0 : w[a][0];
   }
   if (threadIdx.x == 0) piv[0] = w[0][0];
+  // columns from nlive on (the rank's padding) are zero in G: dead without elimination steps
+  for (int k = nlive + threadIdx.x; k < n; k += blockDim.x) {
+    rd[k] = 0.0;
+    dead_s[k] = 1;
+  }
   __syncthreads();
-  for (int kb = 0; kb < 16; kb++) {
+  for (int kb = 0; kb < 16 && kb * TT < nlive; kb++) {
 #pragma unroll
     for (int kr = 0; kr < TT; kr++) {  // unrolled: the next column's register index is static
       const int k = kb * TT + kr;
+      if (k >= nlive) break;  // uniform over the block
       const double *uk = u[k & 1];
       const double d = piv[k & 1];
       const bool dk = !(d > thr);
@@ -1448,16 +1459,16 @@ cudaError_t launch_gram(int n, int nblk, const float *src, int nsrc, int64_t row
   return cudaGetLastError();
 }
 
-cudaError_t launch_chol(int n, double *L, int *dead, double near_id, cudaStream_t st) {
+cudaError_t launch_chol(int n, double *L, int *dead, double near_id, int nlive, cudaStream_t st) {
   switch (n / 16) {
-    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
-    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
-    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
-    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
-    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
-    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
-    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
-    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), 0, st, L, L, dead, near_id); break;
+    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
+    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
+    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
+    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
+    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
+    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
+    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
+    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -1511,7 +1522,7 @@ cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int
   // the reduced Gram matrix goes to L, which the Cholesky kernel then
   // overwrites with M = L^-T
   launch_pdl(lr_gram_reduce_kernel, dim3((unsigned)((n * n + 31) / 32)), dim3(256), 0, st, b.gpart, nblk, n, b.L);
-  e = launch_chol(n, b.L, b.dead, final_pass ? P.qr2_tol : 0.0, st);
+  e = launch_chol(n, b.L, b.dead, final_pass ? P.qr2_tol : 0.0, P.rank, st);
   if (e != cudaSuccess) return e;
   if (!final_pass) return launch_apply_gram(n, b.xbuf, b.L, rows, b.q, b.gpart, st);
   return launch_apply(n, b.q, b.L, rows, b.q, b.qthi, b.qtlo, P.rank, amax, st);
