@@ -322,20 +322,70 @@ __global__ void __launch_bounds__(128, 1)
 // Rows per partial Gram block (rows are a multiple of 128).
 constexpr int kGramRows = 32;
 
-// Shared-memory column index of the Gram tile: the 16 column groups of TT
-// are laid out with an odd stride (TT | 1), so that the 16 groups a warp reads
-// at once fall in distinct banks.
+// The fp64 products of the orthonormalisation (the Gram matrices X^T X and
+// Q = X M) run on the fp64 tensor-core MMA: tcgen05 has no f64 kind, so this
+// is the warp-level mma.sync of shape m8n8k4.  One call adds A B to the 8 x 8
+// tile D, A 8 x 4 and B 4 x 8; lane l holds A[l / 4][l % 4], B[l % 4][l / 4]
+// and D[l / 4][2 (l % 4)], D[l / 4][2 (l % 4) + 1].  Every result below is
+// the same sequence of these calls wherever it is computed, so the kernels
+// that fuse two steps give bit-identical values to the separate ones.
+__device__ __forceinline__ void dmma_8x8x4(double &d0, double &d1, double a, double b) {
+  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
+      : "+d"(d0), "+d"(d1)
+      : "d"(a), "d"(b));
+}
+
+// Row stride (floats) of a Gram input tile [kGramRows][n]: n + 8 is 8 or 24
+// modulo 32, so the 4 rows x 8 columns a fragment load touches fall in 32
+// distinct banks.
 template <int TT>
-__device__ __forceinline__ int gram_col(int c) {
-  return (c / TT) * (TT | 1) + c % TT;
+__host__ __device__ constexpr int gram_ld() {
+  return 16 * TT + 8;
+}
+
+// Partial Gram matrix X^T X of the kGramRows rows of xs (fp32 [kGramRows][ld],
+// ld = gram_ld) into g (fp64 [n][n], n = 16 TT): the 8 x 8 tiles on and below
+// the diagonal (the reduction reads nothing else), dealt round-robin in
+// row-major order to the block's 8 warps, each tile the sum over the rows in
+// steps of 4 from zero.  The products of two fp32 values are exact in fp64.
+template <int TT>
+__device__ __forceinline__ void gram_tiles(const float *xs, double *g, int warp, int lane) {
+  constexpr int n = 16 * TT, ld = gram_ld<TT>(), CT = 2 * TT, T = CT * (CT + 1) / 2, TPW = (T + 7) / 8;
+  const int gq = lane >> 2, t4 = lane & 3;
+  int ti[TPW], tj[TPW];
+  double acc[TPW][2];
+#pragma unroll
+  for (int u = 0; u < TPW; u++) {
+    int t = warp + 8 * u, I = 0;
+    if (t < T) {
+      while (t >= I + 1) {
+        t -= I + 1;
+        I++;
+      }
+      ti[u] = I;
+      tj[u] = t;
+    } else {
+      ti[u] = -1;
+      tj[u] = 0;
+    }
+    acc[u][0] = acc[u][1] = 0.0;
+  }
+#pragma unroll
+  for (int k0 = 0; k0 < kGramRows; k0 += 4) {
+    const float *xr = xs + (k0 + t4) * ld + gq;
+#pragma unroll
+    for (int u = 0; u < TPW; u++)
+      if (ti[u] >= 0) dmma_8x8x4(acc[u][0], acc[u][1], (double)xr[8 * ti[u]], (double)xr[8 * tj[u]]);
+  }
+#pragma unroll
+  for (int u = 0; u < TPW; u++)
+    if (ti[u] >= 0)
+      *reinterpret_cast<double2 *>(g + (8 * ti[u] + gq) * n + 8 * tj[u] + 2 * t4) = make_double2(acc[u][0], acc[u][1]);
 }
 
 // X = sum of the nsrc partial slabs (fixed order), stored fp32 [rows][n], and
-// the partial Gram matrix X^T X (fp64) of this block's kGramRows rows: a 16 x
-// 16 thread grid, thread (ty, tx) accumulating the TT x TT sub-block rows
-// ty*TT.., cols tx*TT.. (n = 16 TT) in registers.  The products of two fp32
-// values are exact in fp64, so each fused multiply-add rounds once, as a
-// multiply followed by an add would.
+// the partial Gram matrix X^T X (fp64, gram_tiles) of this block's kGramRows
+// rows.
 template <int TT>
 __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc, int64_t rows, float *x,
                                                       double *gpart) {
@@ -343,7 +393,7 @@ __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc
   constexpr int n = 16 * TT;
   constexpr int n4 = n / 4;                          // float4 per row
   constexpr int NV = (kGramRows * n4 + 255) / 256;   // float4 per thread
-  __shared__ float tile[kGramRows][16 * (TT | 1)];
+  __shared__ __align__(16) float tile[kGramRows * gram_ld<TT>()];
   const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
   const float4 *s4 = reinterpret_cast<const float4 *>(src) + r0 * n4;
   const int64_t slab4 = rows * n4;
@@ -382,38 +432,11 @@ __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc
     if (e < kGramRows * n4) {
       x4[e] = acc4[v];
       const int rr = e / n4, c = (e % n4) * 4;
-      tile[rr][gram_col<TT>(c)] = acc4[v].x;
-      tile[rr][gram_col<TT>(c + 1)] = acc4[v].y;
-      tile[rr][gram_col<TT>(c + 2)] = acc4[v].z;
-      tile[rr][gram_col<TT>(c + 3)] = acc4[v].w;
+      *reinterpret_cast<float4 *>(tile + rr * gram_ld<TT>() + c) = acc4[v];
     }
   }
   __syncthreads();
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  constexpr int S = TT | 1;
-  double acc[TT][TT];
-#pragma unroll
-  for (int a = 0; a < TT; a++)
-#pragma unroll
-    for (int c = 0; c < TT; c++) acc[a][c] = 0.0;
-#pragma unroll 4
-  for (int rr = 0; rr < kGramRows; rr++) {
-    double xi[TT], xj[TT];
-#pragma unroll
-    for (int a = 0; a < TT; a++) {
-      xi[a] = (double)tile[rr][ty * S + a];
-      xj[a] = (double)tile[rr][tx * S + a];
-    }
-#pragma unroll
-    for (int a = 0; a < TT; a++)
-#pragma unroll
-      for (int c = 0; c < TT; c++) acc[a][c] = fma(xi[a], xj[c], acc[a][c]);
-  }
-  double *g = gpart + (int64_t)blockIdx.x * n * n;
-#pragma unroll
-  for (int a = 0; a < TT; a++)
-#pragma unroll
-    for (int c = 0; c < TT; c++) g[(ty * TT + a) * n + tx * TT + c] = acc[a][c];
+  gram_tiles<TT>(tile, gpart + (int64_t)blockIdx.x * n * n, threadIdx.x >> 5, threadIdx.x & 31);
 }
 
 // G = sum over the nblk partial Gram matrices, lower triangle only (the
@@ -620,18 +643,76 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double
 constexpr int kApplyRows = 16;
 template <int TT>
 __host__ __device__ constexpr int apply_xld() {
-  return 16 * TT + 4;  // padded row stride of the X tile (bank spread, 16-byte rows)
+  return 16 * TT + 4;  // X tile row stride (floats): 4 or 20 mod 32, a fragment's 8 rows x 4 in distinct banks
+}
+template <int TT>
+__host__ __device__ constexpr int apply_mld() {
+  return 16 * TT + 4;  // M row stride (doubles): each half-warp's 4 rows x 4 fragment entries in distinct banks
 }
 
-// Q = X M (M = L^-T, upper triangular, zero below the diagonal) for 16 rows
-// per block.  M and the block's rows of X are staged in shared memory;
-// thread (row, q) computes the TT outputs c = q + 16 t of its row (the 16
-// threads of a row read 16 consecutive entries of a row of M) with fp64
-// accumulators over all n terms, the two halves of the term range in
-// separate accumulators added at the end (the zeros below M's diagonal add
-// nothing).  Writes Q fp32 [rows][n] and, when qthi != nullptr, Q^T split in
-// bf16 ([n][rows], the K-major B operand of V = D^T Q), transposed through
-// shared memory so that those stores are row-contiguous; when amax !=
+// Stage M (fp64 [n][n]) into Ms (row stride apply_mld) and the block's nx
+// rows of X (fp32 [rows][n], from row r0; rows past the end read as zero) into
+// xs (row stride apply_xld).
+template <int TT>
+__device__ __forceinline__ void apply_stage(const float *x, const double *M, int64_t rows, int64_t r0, int nx,
+                                            double *Ms, float *xs) {
+  constexpr int n = 16 * TT, mld = apply_mld<TT>(), xld = apply_xld<TT>();
+  const double2 *M2 = reinterpret_cast<const double2 *>(M);
+  for (int e = threadIdx.x; e < n * n / 2; e += blockDim.x) {
+    const int rr = (2 * e) / n, c = (2 * e) % n;
+    *reinterpret_cast<double2 *>(Ms + rr * mld + c) = M2[e];
+  }
+  const float4 *x4 = reinterpret_cast<const float4 *>(x) + r0 * (n / 4);
+  for (int e = threadIdx.x; e < nx * n / 4; e += blockDim.x) {
+    const int rr = e / (n / 4), c = (e % (n / 4)) * 4;
+    const float4 val = r0 + rr < rows ? x4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4 *>(xs + rr * xld + c) = val;
+  }
+}
+
+// Column tile (of 8) that warp w computes in its round jt of Q = X M: the
+// 2 TT tiles are dealt in descending order (the widest term ranges first),
+// snake-wise over the 8 warps; -1 past the last.
+template <int TT>
+__device__ __forceinline__ int apply_ctile(int w, int jt) {
+  const int s = 8 * jt + ((jt & 1) ? 7 - w : w);
+  return s < 2 * TT ? 2 * TT - 1 - s : -1;
+}
+template <int TT>
+__host__ __device__ constexpr int apply_rounds() {
+  return (2 * TT + 7) / 8;
+}
+
+// Q = X M for the 8 RT rows of xs (M upper triangular): warp w computes its
+// column tiles (apply_ctile) for all RT row tiles, each output the sum from
+// zero over M's rows 0 .. 8 J + 7 in steps of 4 (the rows below add zeros).
+template <int TT, int RT>
+__device__ __forceinline__ void apply_tiles(const float *xs, const double *Ms, int warp, int lane,
+                                            double (&acc)[apply_rounds<TT>()][RT][2]) {
+  constexpr int mld = apply_mld<TT>(), xld = apply_xld<TT>();
+  const int gq = lane >> 2, t4 = lane & 3;
+#pragma unroll
+  for (int jt = 0; jt < apply_rounds<TT>(); jt++) {
+#pragma unroll
+    for (int i = 0; i < RT; i++) acc[jt][i][0] = acc[jt][i][1] = 0.0;
+    const int J = apply_ctile<TT>(warp, jt);
+    if (J < 0) continue;  // uniform over the warp
+    const double *mp = Ms + t4 * mld + 8 * J + gq;
+    const float *xp = xs + gq * xld + t4;
+#pragma unroll 2
+    for (int k0 = 0; k0 < 8 * J + 8; k0 += 4) {
+      const double b = mp[k0 * mld];
+#pragma unroll
+      for (int i = 0; i < RT; i++) dmma_8x8x4(acc[jt][i][0], acc[jt][i][1], (double)xp[8 * i * xld + k0], b);
+    }
+  }
+}
+
+// Q = X M (M = L^-T, upper triangular, zero below the diagonal) for
+// kApplyRows rows per block (apply_tiles; M and the rows of X staged in
+// shared memory).  Writes Q fp32 [rows][n] and, when qthi != nullptr, Q^T
+// split in bf16 ([n][rows], the K-major B operand of V = D^T Q), transposed
+// through shared memory so that those stores are row-contiguous; when amax !=
 // nullptr, the absmax of each of Q's first r columns (the INT4 scales'
 // input) goes to amax, one atomicMax per column and block.
 template <int TT>
@@ -640,62 +721,39 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
                                                        unsigned *amax) {
   pdl_enter();
   __shared__ unsigned cmax[16 * TT];
-  constexpr int n = 16 * TT, xld = apply_xld<TT>(), qld = kApplyRows + 1, h = n / 2;
+  constexpr int n = 16 * TT, mld = apply_mld<TT>(), qld = kApplyRows + 1, RT = kApplyRows / 8;
+  constexpr int JR = apply_rounds<TT>();
   extern __shared__ __align__(16) uint8_t asm_[];
-  double *Ms = reinterpret_cast<double *>(asm_);      // [n][n]
-  float *xs = reinterpret_cast<float *>(Ms + n * n);  // [16][xld]; reused as Q^T [n][qld]
+  double *Ms = reinterpret_cast<double *>(asm_);        // [n][mld]
+  float *xs = reinterpret_cast<float *>(Ms + n * mld);  // [kApplyRows][xld]; reused as Q^T [n][qld]
   const int64_t r0 = (int64_t)blockIdx.x * kApplyRows;
-  {
-    const double2 *M2 = reinterpret_cast<const double2 *>(M);
-    double2 *Ms2 = reinterpret_cast<double2 *>(Ms);
-    constexpr int NM = n * n / 2;
+  apply_stage<TT>(x, M, rows, r0, kApplyRows, Ms, xs);
+  if (amax != nullptr)
+    for (int c = threadIdx.x; c < n; c += 256) cmax[c] = 0u;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t4 = lane & 3;
+  double acc[JR][RT][2];
+  apply_tiles<TT, RT>(xs, Ms, warp, lane, acc);
+  float res[JR][RT][2];
 #pragma unroll
-    for (int v = 0; v < (NM + 255) / 256; v++) {
-      const int e = threadIdx.x + 256 * v;
-      if (e < NM) Ms2[e] = M2[e];
-    }
-    const float4 *x4 = reinterpret_cast<const float4 *>(x) + r0 * (n / 4);
-    constexpr int NX = kApplyRows * n / 4;
+  for (int jt = 0; jt < JR; jt++) {
+    const int J = apply_ctile<TT>(warp, jt);
 #pragma unroll
-    for (int v = 0; v < (NX + 255) / 256; v++) {
-      const int e = threadIdx.x + 256 * v;
-      if (e < NX) {
-        const int rr = e / (n / 4), c = (e % (n / 4)) * 4;
-        const float4 val = r0 + rr < rows ? x4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4 *>(xs + rr * xld + c) = val;
+    for (int i = 0; i < RT; i++) {
+      res[jt][i][0] = (float)acc[jt][i][0];
+      res[jt][i][1] = (float)acc[jt][i][1];
+      const int64_t row = r0 + 8 * i + gq;
+      if (J >= 0 && row < rows) {
+        const int c = 8 * J + 2 * t4;
+        *reinterpret_cast<float2 *>(q + row * n + c) = make_float2(res[jt][i][0], res[jt][i][1]);
+        if (amax != nullptr) {  // the INT4 column maxima of Q (non-negative bit patterns)
+          atomicMax(&cmax[c], __float_as_uint(fabsf(res[jt][i][0])));
+          atomicMax(&cmax[c + 1], __float_as_uint(fabsf(res[jt][i][1])));
+        }
       }
     }
   }
-  __syncthreads();
-  const int lr = threadIdx.x >> 4, qc = threadIdx.x & 15;
-  double acc0[TT], acc1[TT];
-#pragma unroll
-  for (int t = 0; t < TT; t++) acc0[t] = acc1[t] = 0.0;
-#pragma unroll 2
-  for (int j = 0; j < h; j++) {
-    const double x0 = (double)xs[lr * xld + j], x1 = (double)xs[lr * xld + h + j];
-    const double *m0 = Ms + j * n + qc, *m1 = Ms + (h + j) * n + qc;
-#pragma unroll
-    for (int t = 0; t < TT; t++) {
-      acc0[t] = fma(x0, m0[16 * t], acc0[t]);
-      acc1[t] = fma(x1, m1[16 * t], acc1[t]);
-    }
-  }
-  float res[TT];
-#pragma unroll
-  for (int t = 0; t < TT; t++) res[t] = (float)(acc0[t] + acc1[t]);
-  const int64_t row = r0 + lr;
-  if (row < rows) {
-#pragma unroll
-    for (int t = 0; t < TT; t++) q[row * n + qc + 16 * t] = res[t];
-  }
-  if (amax != nullptr) {  // uniform over the block: the INT4 column maxima of Q (non-negative bit patterns)
-    for (int c = threadIdx.x; c < n; c += 256) cmax[c] = 0u;
-    __syncthreads();
-    if (row < rows) {
-#pragma unroll
-      for (int t = 0; t < TT; t++) atomicMax(&cmax[qc + 16 * t], __float_as_uint(fabsf(res[t])));
-    }
+  if (amax != nullptr) {  // uniform over the block
     __syncthreads();
     for (int c = threadIdx.x; c < r; c += 256)
       if (cmax[c]) atomicMax(&amax[c], cmax[c]);
@@ -704,7 +762,16 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
   __syncthreads();              // every thread is done with xs
   float *qs = xs;               // Q^T tile [n][qld]
 #pragma unroll
-  for (int t = 0; t < TT; t++) qs[(qc + 16 * t) * qld + lr] = res[t];
+  for (int jt = 0; jt < JR; jt++) {
+    const int J = apply_ctile<TT>(warp, jt);
+    if (J < 0) continue;
+#pragma unroll
+    for (int i = 0; i < RT; i++) {
+      const int c = 8 * J + 2 * t4;
+      qs[c * qld + 8 * i + gq] = res[jt][i][0];
+      qs[(c + 1) * qld + 8 * i + gq] = res[jt][i][1];
+    }
+  }
   __syncthreads();
   for (int e = threadIdx.x; e < n * kApplyRows; e += 256) {
     const int c = e / kApplyRows, rr = e % kApplyRows;
@@ -717,94 +784,44 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
   }
 }
 
-// The first CholeskyQR pass's Q1 = X M for kGramRows rows per block, with
-// the sums of lr_apply_kernel (each output's two halves of the term range in
-// separate fp64 accumulators, added at the end; thread (row, q) takes the 2 TT
-// outputs c = q + 8 t), and the partial Gram matrix Q1^T Q1 of these rows from
-// the fp32 values it stores, with the sums of lr_gram_kernel: the second pass
-// needs no Gram kernel, and both results are bit-identical to the separate
-// kernels'.
+// The first CholeskyQR pass's Q1 = X M for kGramRows rows per block, with the
+// sums of lr_apply_kernel (apply_tiles), and the partial Gram matrix Q1^T Q1
+// of these rows from the fp32 values it stores, with the sums of
+// lr_gram_kernel (gram_tiles): the second pass needs no Gram kernel, and both
+// results are bit-identical to the separate kernels'.
 template <int TT>
 __global__ void __launch_bounds__(256) lr_apply_gram_kernel(const float *x, const double *M, int64_t rows, float *q,
                                                             double *gpart) {
   pdl_enter();
-  constexpr int n = 16 * TT, xld = apply_xld<TT>(), h = n / 2, S = TT | 1;
+  constexpr int n = 16 * TT, mld = apply_mld<TT>(), xld = apply_xld<TT>(), RT = kGramRows / 8;
+  constexpr int JR = apply_rounds<TT>();
   extern __shared__ __align__(16) uint8_t asm_[];
-  double *Ms = reinterpret_cast<double *>(asm_);                          // [n][n]
-  float *xs = reinterpret_cast<float *>(Ms + n * n);                      // [kGramRows][xld]
-  float (*tile)[16 * S] = reinterpret_cast<float (*)[16 * S]>(xs + kGramRows * xld);  // [kGramRows][16 S]
+  double *Ms = reinterpret_cast<double *>(asm_);        // [n][mld]
+  float *xs = reinterpret_cast<float *>(Ms + n * mld);  // [kGramRows][xld]
+  float *gs = xs + kGramRows * xld;                     // Q1 [kGramRows][gram_ld]
   const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
+  apply_stage<TT>(x, M, rows, r0, kGramRows, Ms, xs);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t4 = lane & 3;
   {
-    const double2 *M2 = reinterpret_cast<const double2 *>(M);
-    double2 *Ms2 = reinterpret_cast<double2 *>(Ms);
-    constexpr int NM = n * n / 2;
+    double acc[JR][RT][2];
+    apply_tiles<TT, RT>(xs, Ms, warp, lane, acc);
 #pragma unroll
-    for (int v = 0; v < (NM + 255) / 256; v++) {
-      const int e = threadIdx.x + 256 * v;
-      if (e < NM) Ms2[e] = M2[e];
-    }
-    const float4 *x4 = reinterpret_cast<const float4 *>(x) + r0 * (n / 4);
-    constexpr int NX = kGramRows * n / 4;
+    for (int jt = 0; jt < JR; jt++) {
+      const int J = apply_ctile<TT>(warp, jt);
+      if (J < 0) continue;
 #pragma unroll
-    for (int v = 0; v < (NX + 255) / 256; v++) {
-      const int e = threadIdx.x + 256 * v;
-      if (e < NX) {
-        const int rr = e / (n / 4), c = (e % (n / 4)) * 4;
-        const float4 val = r0 + rr < rows ? x4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4 *>(xs + rr * xld + c) = val;
+      for (int i = 0; i < RT; i++) {
+        const int64_t row = r0 + 8 * i + gq;
+        const int c = 8 * J + 2 * t4;
+        const float2 v = row < rows ? make_float2((float)acc[jt][i][0], (float)acc[jt][i][1]) : make_float2(0.f, 0.f);
+        if (row < rows) *reinterpret_cast<float2 *>(q + row * n + c) = v;
+        *reinterpret_cast<float2 *>(gs + (8 * i + gq) * gram_ld<TT>() + c) = v;
       }
     }
   }
   __syncthreads();
-  {
-    const int lr = threadIdx.x >> 3, qc = threadIdx.x & 7;
-    double acc0[2 * TT], acc1[2 * TT];
-#pragma unroll
-    for (int t = 0; t < 2 * TT; t++) acc0[t] = acc1[t] = 0.0;
-#pragma unroll 2
-    for (int j = 0; j < h; j++) {
-      const double x0 = (double)xs[lr * xld + j], x1 = (double)xs[lr * xld + h + j];
-      const double *m0 = Ms + j * n + qc, *m1 = Ms + (h + j) * n + qc;
-#pragma unroll
-      for (int t = 0; t < 2 * TT; t++) {
-        acc0[t] = fma(x0, m0[8 * t], acc0[t]);
-        acc1[t] = fma(x1, m1[8 * t], acc1[t]);
-      }
-    }
-    const int64_t row = r0 + lr;
-#pragma unroll
-    for (int t = 0; t < 2 * TT; t++) {
-      const int c = qc + 8 * t;
-      const float v = row < rows ? (float)(acc0[t] + acc1[t]) : 0.0f;
-      if (row < rows) q[row * n + c] = v;
-      tile[lr][gram_col<TT>(c)] = v;
-    }
-  }
-  __syncthreads();
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  double acc[TT][TT];
-#pragma unroll
-  for (int a = 0; a < TT; a++)
-#pragma unroll
-    for (int c = 0; c < TT; c++) acc[a][c] = 0.0;
-#pragma unroll 4
-  for (int rr = 0; rr < kGramRows; rr++) {
-    double xi[TT], xj[TT];
-#pragma unroll
-    for (int a = 0; a < TT; a++) {
-      xi[a] = (double)tile[rr][ty * S + a];
-      xj[a] = (double)tile[rr][tx * S + a];
-    }
-#pragma unroll
-    for (int a = 0; a < TT; a++)
-#pragma unroll
-      for (int c = 0; c < TT; c++) acc[a][c] = fma(xi[a], xj[c], acc[a][c]);
-  }
-  double *g = gpart + (int64_t)blockIdx.x * n * n;
-#pragma unroll
-  for (int a = 0; a < TT; a++)
-#pragma unroll
-    for (int c = 0; c < TT; c++) g[(ty * TT + a) * n + tx * TT + c] = acc[a][c];
+  gram_tiles<TT>(gs, gpart + (int64_t)blockIdx.x * n * n, warp, lane);
 }
 
 // V = sum of the partial slabs (fixed order) [cols][n]; V_prev (state,
@@ -1281,13 +1298,12 @@ cudaError_t set_recon_smem(int smem) {
     return e;
   return cudaSuccess;
 }
-size_t apply_smem(int n) {
+size_t apply_smem(int n) {  // n = 16 TT: apply_mld = apply_xld = n + 4
   const size_t xt = (size_t)kApplyRows * (n + 4) * 4, qt = (size_t)n * (kApplyRows + 1) * 4;
-  return (size_t)n * n * 8 + (xt > qt ? xt : qt);
+  return (size_t)n * (n + 4) * 8 + (xt > qt ? xt : qt);
 }
-size_t apply_gram_smem(int n) {
-  const int tt = n / 16, s = tt | 1;
-  return (size_t)n * n * 8 + (size_t)kGramRows * (n + 4) * 4 + (size_t)kGramRows * 16 * s * 4;
+size_t apply_gram_smem(int n) {  // gram_ld = n + 8
+  return (size_t)n * (n + 4) * 8 + (size_t)kGramRows * (n + 4) * 4 + (size_t)kGramRows * (n + 8) * 4;
 }
 
 }  // namespace
