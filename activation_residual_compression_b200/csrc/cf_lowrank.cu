@@ -474,23 +474,99 @@ __global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart
   }
 }
 
-// Cholesky factor L of the Gram matrix G (fp64) and M = L^-T, by right-
-// looking elimination with the n x n working array W held in registers: a
-// 16 x 16 thread grid, thread (ty, tx) owning the TT x TT block rows
-// ty*TT.., columns tx*TT.. (n = 16 TT).  W starts as the lower triangle of
-// G.  At step k, with d the pivot and c_i = W[i][k] (i > k) the column below
-// it, every row i > k takes W[i][j] -= (c_i / d) v_j for all j, where v is
-// row k of W left of the diagonal (j < k), the column c right of it (j > k)
-// and 0 at j = k.  In the trailing part (j > k) this is the Cholesky update;
-// left of it, W carries L^-1 by forward elimination of the identity, each of
-// its columns j stored scaled by -d_j (L^-1[i][j] = -W[i][j] / (d_j sqrt(d_i))
-// once row i is final), which makes the update uniform over j.  The owners of
-// column k+1 and of row k+1 publish v for the next step into a double-
-// buffered shared vector, so each step costs one barrier and TT^2 fused
-// multiply-adds per thread.  A pivot <= 1e-12 G_00 (R_kk <= 1e-6 R_00) marks
-// column k rank deficient: dead[k] = 1, the step's multiplier is zero (L's
-// column k below the diagonal is zero) and column k of M is zero, so that
-// Q's column k is zero.
+// ---- Cholesky factor of the Gram matrix and its inverse (fp64)
+//
+// Blocked right-looking elimination on 8 x 8 tiles.  The working matrix A
+// (the lower triangle of G) and X = L^-1 live in shared memory as packed
+// lower-triangular arrays of tiles, tile (I, J), J <= I, at index
+// I (I + 1) / 2 + J, each 8 rows of chol_tld doubles.  For each block column
+// b of the nbl = ceil(nlive / 8) live ones:
+//   diagonal  one warp factors the 8 x 8 block A_bb = L_bb L_bb^T column by
+//             column in registers (lane i holds row i) and forms X_bb =
+//             L_bb^-1 by forward substitution of the identity, row k of it
+//             being r_k (e_k - sum_{m<k} L_km X_m) with r_k = 1 / L_kk;
+//   panel     L_ib = A_ib X_bb^T for the tiles below, and the finished row
+//             of the inverse X_bj = X_bb X_bj (j < b);
+//   trailing  A_ij -= L_ib L_jb^T (b < j <= i) and X_ij -= L_ib X_bj
+//             (i > b, j <= b); the warp that updates the next diagonal tile
+//             factors it at once.
+// Each phase ends with one block barrier; the tile products run on the fp64
+// MMA.  A pivot <= 1e-12 G_00 (R_kk <= 1e-6 R_00), or a column at or past
+// nlive (the rank's zero padding), marks column k rank deficient: dead[k] =
+// 1, r_k = 0, so row k of X and column k of L (hence of X) are zero and the
+// column updates nothing; the other columns are the Cholesky factor of G
+// restricted to them.
+constexpr int kCholTld = 9;  // tile row stride (doubles): a half-warp's 4 x 4 fragment in distinct banks
+
+template <int TT>
+__host__ __device__ constexpr int chol_ntiles() {
+  return (2 * TT) * (2 * TT + 1) / 2;
+}
+__host__ __device__ constexpr size_t chol_smem_tt(int tt) {
+  return (size_t)2 * ((2 * tt) * (2 * tt + 1) / 2) * 8 * kCholTld * 8;
+}
+
+__device__ __forceinline__ int chol_tile(int I, int J) {
+  return (I * (I + 1) / 2 + J) * 8 * kCholTld;
+}
+
+// D += a B for an 8 x 8 tile: P row-major (A operand P[g][4 kc + t4]), R either
+// transposed (B[k][c] = R[c][k]) or not; sa = -1 subtracts the product.
+__device__ __forceinline__ void chol_tile_mma(double &d0, double &d1, const double *P, const double *R, bool rt,
+                                              double sa, int gq, int t4) {
+#pragma unroll
+  for (int kc = 0; kc < 2; kc++) {
+    const double a = sa * P[gq * kCholTld + 4 * kc + t4];
+    const double b = rt ? R[gq * kCholTld + 4 * kc + t4] : R[(4 * kc + t4) * kCholTld + gq];
+    dmma_8x8x4(d0, d1, a, b);
+  }
+}
+
+// Factor the diagonal tile of block column b (one warp): reads A_bb, writes
+// X_bb = L_bb^-1 and the dead flags of its 8 columns.
+__device__ __forceinline__ void chol_diag(const double *Ab, double *Xb, int b, int nlive, double thr, int lane,
+                                          int *dead_s) {
+  const int i = lane;
+  double a[8], y[8], l[8];
+#pragma unroll
+  for (int j = 0; j < 8; j++) {
+    a[j] = (i < 8 && j <= i) ? Ab[i * kCholTld + j] : 0.0;
+    y[j] = (i == j) ? 1.0 : 0.0;
+  }
+  unsigned dmask = 0;
+#pragma unroll
+  for (int k = 0; k < 8; k++) {
+    const double d = __shfl_sync(0xffffffffu, a[k], k);
+    const bool dk = 8 * b + k >= nlive || !(d > thr);
+    const double r = dk ? 0.0 : rsqrt(d);
+    dmask |= dk ? 1u << k : 0u;
+    l[k] = i > k ? a[k] * r : 0.0;  // L[i][k]
+    // row k of the inverse, then its subtraction from the rows below
+    double xk[8];
+#pragma unroll
+    for (int j = 0; j <= k; j++) xk[j] = __shfl_sync(0xffffffffu, y[j], k) * r;
+    if (i == k) {
+#pragma unroll
+      for (int j = 0; j <= k; j++) y[j] = xk[j];
+    }
+#pragma unroll
+    for (int j = 0; j <= k; j++)
+      if (i > k) y[j] = fma(-l[k], xk[j], y[j]);
+#pragma unroll
+    for (int j = k + 1; j < 8; j++) {
+      const double lj = __shfl_sync(0xffffffffu, l[k], j);
+      if (i >= j) a[j] = fma(-l[k], lj, a[j]);
+    }
+  }
+  if (i < 8) {
+#pragma unroll
+    for (int j = 0; j < 8; j++) Xb[i * kCholTld + j] = j <= i ? y[j] : 0.0;
+    dead_s[8 * b + i] = (dmask >> i) & 1u;
+  }
+}
+
+// Cholesky factor L of the Gram matrix G (fp64, lower triangle read) and M =
+// L^-T (fp64 [n][n], upper triangular), with the dead flags.
 //
 // near_id > 0 (the second pass of CholeskyQR2, where G = Q1^T Q1 is close to
 // the identity): if every entry of E = G - I between nonzero columns has
@@ -499,33 +575,26 @@ __global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart
 // O(|E|^2), and Q1 M has an orthogonality error of about 3 n near_id^2 per
 // entry.  A column of G that is exactly zero (a column of Q1 zeroed as rank
 // deficient by the first pass) is dead, as in the elimination.  Otherwise
-// the elimination runs.
+// the blocked elimination runs.
 //
-// Columns nlive .. n-1 must be zero in G (the padding of the rank): they are
-// marked dead and the elimination stops after column nlive - 1, which gives
-// the same M as running the remaining steps (each would find a zero pivot).
-//
-// Writes M fp64 [n][n] (upper triangular); G and M may alias (G is read into
-// registers before the first barrier).
+// Columns nlive .. n-1 must be zero in G (the padding of the rank).  G and M
+// may alias (G is read before the first barrier).
 template <int TT>
 __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double *Mout, int *dead, double near_id,
                                                          int nlive) {
   pdl_enter();
   constexpr int n = 16 * TT;
-  constexpr int S = TT | 1;  // odd block stride of the shared vector: no bank conflicts
-  __shared__ double u[2][16 * S];
-  __shared__ double piv[2];
-  __shared__ double rd[n];   // 1 / sqrt(d_k), 0 for a dead column
   __shared__ int dead_s[n];
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  const int i0 = ty * TT, j0 = tx * TT;
-  double w[TT][TT];
-#pragma unroll
-  for (int a = 0; a < TT; a++)
-#pragma unroll
-    for (int c = 0; c < TT; c++) w[a][c] = (j0 + c <= i0 + a) ? G[(i0 + a) * n + j0 + c] : 0.0;
-  const bool lower = tx <= ty;  // blocks above the diagonal hold nothing
+  extern __shared__ __align__(16) uint8_t csm[];
   if (near_id > 0.0) {
+    const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+    const int i0 = ty * TT, j0 = tx * TT;
+    const bool lower = tx <= ty;  // blocks above the diagonal hold nothing
+    double w[TT][TT];
+#pragma unroll
+    for (int a = 0; a < TT; a++)
+#pragma unroll
+      for (int c = 0; c < TT; c++) w[a][c] = (lower && j0 + c <= i0 + a) ? G[(i0 + a) * n + j0 + c] : 0.0;
     int far = 0;
     if (lower) {
 #pragma unroll
@@ -559,82 +628,90 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double
       return;
     }
   }
+  double *A = reinterpret_cast<double *>(csm);  // packed tiles of the working matrix
+  double *X = A + chol_ntiles<TT>() * 8 * kCholTld;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t4 = lane & 3;
+  const int nbl = (min(max(nlive, 0), n) + 7) / 8;
+  const int nl = 8 * nbl;
   const double thr = 1e-12 * G[0];
-  if (tx == 0) {
-#pragma unroll
-    for (int a = 0; a < TT; a++) u[0][ty * S + a] = (i0 + a == 0) ? 0.0 : w[a][0];
+  for (int e = threadIdx.x; e < nl * nl; e += blockDim.x) {
+    const int gi = e / nl, gj = e % nl;
+    if ((gj >> 3) <= (gi >> 3)) {
+      const int o = chol_tile(gi >> 3, gj >> 3) + (gi & 7) * kCholTld + (gj & 7);
+      A[o] = gj <= gi ? G[gi * n + gj] : 0.0;
+      X[o] = 0.0;
+    }
   }
-  if (threadIdx.x == 0) piv[0] = w[0][0];
-  // columns from nlive on (the rank's padding) are zero in G: dead without elimination steps
-  for (int k = nlive + threadIdx.x; k < n; k += blockDim.x) {
-    rd[k] = 0.0;
-    dead_s[k] = 1;
-  }
+  for (int k = nl + threadIdx.x; k < n; k += blockDim.x) dead_s[k] = 1;
   __syncthreads();
-  for (int kb = 0; kb < 16 && kb * TT < nlive; kb++) {
-#pragma unroll
-    for (int kr = 0; kr < TT; kr++) {  // unrolled: the next column's register index is static
-      const int k = kb * TT + kr;
-      if (k >= nlive) break;  // uniform over the block
-      const double *uk = u[k & 1];
-      const double d = piv[k & 1];
-      const bool dk = !(d > thr);
-      const double r = dk ? 0.0 : rsqrt(d);
-      const double invd = r * r;
-      if (threadIdx.x == 0) {
-        rd[k] = r;
-        dead_s[k] = dk ? 1 : 0;
-      }
-      if (lower && i0 + TT - 1 > k) {
-        double vj[TT];
-#pragma unroll
-        for (int c = 0; c < TT; c++) vj[c] = uk[tx * S + c];
-#pragma unroll
-        for (int a = 0; a < TT; a++) {
-          // rows <= k are final; a zero multiplier leaves them as they are
-          const double sa = (i0 + a > k) ? -(uk[ty * S + a] * invd) : 0.0;
-#pragma unroll
-          for (int c = 0; c < TT; c++) w[a][c] = fma(sa, vj[c], w[a][c]);
-        }
-      }
-      const int k1 = k + 1;
-      const int cn = (kr + 1 == TT) ? 0 : kr + 1;
-      const int b1 = (kr + 1 == TT) ? kb + 1 : kb;
-      if (k1 < n) {
-        double *un = u[k1 & 1];
-        if (tx == b1) {  // column k1 below the diagonal; its diagonal is the next pivot
-#pragma unroll
-          for (int a = 0; a < TT; a++) {
-            const double x = w[a][cn];
-            if (i0 + a > k1) un[ty * S + a] = x;
-            if (i0 + a == k1) {
-              un[ty * S + a] = 0.0;
-              piv[k1 & 1] = x;
-            }
+  if (nbl > 0 && warp == 0) chol_diag(A, X, 0, nlive, thr, lane, dead_s);
+  __syncthreads();
+  for (int b = 0; b < nbl; b++) {
+    const int m = nbl - 1 - b;  // block rows below the diagonal
+    const double *Xbb = X + chol_tile(b, b);
+    // panel L_ib = A_ib X_bb^T (i > b) and the inverse's row X_bj = X_bb X_bj (j < b)
+    for (int t = warp; t < m + b; t += 8) {
+      double *T = t < m ? A + chol_tile(b + 1 + t, b) : X + chol_tile(b, t - m);
+      double d0 = 0.0, d1 = 0.0;
+      if (t < m)
+        chol_tile_mma(d0, d1, T, Xbb, true, 1.0, gq, t4);
+      else
+        chol_tile_mma(d0, d1, Xbb, T, false, 1.0, gq, t4);
+      __syncwarp();
+      T[gq * kCholTld + 2 * t4] = d0;
+      T[gq * kCholTld + 2 * t4 + 1] = d1;
+    }
+    __syncthreads();
+    if (m == 0) break;  // uniform
+    // trailing A_ij -= L_ib L_jb^T (b < j <= i) and X_ij -= L_ib X_bj (i > b, j <= b); warp 0 takes the
+    // next diagonal tile and factors it, warps 1..7 the rest
+    const int ntr = m * (m + 1) / 2, ntask = ntr - 1 + m * (b + 1);
+    if (warp == 0) {
+      double *T = A + chol_tile(b + 1, b + 1);
+      const double *Lb = A + chol_tile(b + 1, b);
+      double d0 = T[gq * kCholTld + 2 * t4], d1 = T[gq * kCholTld + 2 * t4 + 1];
+      chol_tile_mma(d0, d1, Lb, Lb, true, -1.0, gq, t4);
+      T[gq * kCholTld + 2 * t4] = d0;
+      T[gq * kCholTld + 2 * t4 + 1] = d1;
+      __syncwarp();
+      chol_diag(T, X + chol_tile(b + 1, b + 1), b + 1, nlive, thr, lane, dead_s);
+    } else {
+      for (int t = warp - 1; t < ntask; t += 7) {
+        int i, j;
+        double *T;
+        const double *R;
+        bool rt;
+        if (t < ntr - 1) {  // trailing tile, row-major over the triangle after the next diagonal tile
+          int u = t + 1, ii = 0;
+          while (u >= ii + 1) {
+            u -= ii + 1;
+            ii++;
           }
+          i = b + 1 + ii;
+          j = b + 1 + u;
+          T = A + chol_tile(i, j);
+          R = A + chol_tile(j, b);
+          rt = true;
+        } else {
+          const int u = t - (ntr - 1);
+          i = b + 1 + u / (b + 1);
+          j = u % (b + 1);
+          T = X + chol_tile(i, j);
+          R = X + chol_tile(b, j);
+          rt = false;
         }
-        if (ty == b1) {  // row k1 left of the diagonal
-#pragma unroll
-          for (int c = 0; c < TT; c++)
-            if (j0 + c < k1) un[tx * S + c] = w[cn][c];
-        }
+        double d0 = T[gq * kCholTld + 2 * t4], d1 = T[gq * kCholTld + 2 * t4 + 1];
+        chol_tile_mma(d0, d1, A + chol_tile(i, b), R, rt, -1.0, gq, t4);
+        T[gq * kCholTld + 2 * t4] = d0;
+        T[gq * kCholTld + 2 * t4 + 1] = d1;
       }
-      __syncthreads();
     }
+    __syncthreads();
   }
-#pragma unroll
-  for (int a = 0; a < TT; a++) {
-    const int gi = i0 + a;
-    const bool dki = dead_s[gi] != 0;
-    const double ri = rd[gi];
-#pragma unroll
-    for (int c = 0; c < TT; c++) {
-      const int gj = j0 + c;
-      const double rj = rd[gj];
-      double m = 0.0;  // M[gj][gi] = L^-1[gi][gj]
-      if (gj <= gi && !dki) m = gj == gi ? ri : (-w[a][c] * (rj * rj)) * ri;
-      Mout[gj * n + gi] = m;
-    }
+  // M[gj][gi] = X[gi][gj]
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+    const int gj = e / n, gi = e % n;
+    Mout[e] = (gi < nl && gj <= gi) ? X[chol_tile(gi >> 3, gj >> 3) + (gi & 7) * kCholTld + (gj & 7)] : 0.0;
   }
   for (int e = threadIdx.x; e < n; e += blockDim.x) dead[e] = dead_s[e];
 }
@@ -1369,8 +1446,10 @@ cudaError_t set_apply_smem_tt() {
   cudaError_t e = cudaFuncSetAttribute(lr_apply_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)apply_smem(16 * TT));
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(lr_apply_gram_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)apply_gram_smem(16 * TT));
+  e = cudaFuncSetAttribute(lr_apply_gram_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)apply_gram_smem(16 * TT));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(lr_chol_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)chol_smem_tt(TT));
 }
 
 cudaError_t set_apply_smem(int n) {
@@ -1477,14 +1556,14 @@ cudaError_t launch_gram(int n, int nblk, const float *src, int nsrc, int64_t row
 
 cudaError_t launch_chol(int n, double *L, int *dead, double near_id, int nlive, cudaStream_t st) {
   switch (n / 16) {
-    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
-    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
-    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
-    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
-    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
-    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
-    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
-    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), 0, st, L, L, dead, near_id, nlive); break;
+    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), chol_smem_tt(1), st, L, L, dead, near_id, nlive); break;
+    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), chol_smem_tt(2), st, L, L, dead, near_id, nlive); break;
+    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), chol_smem_tt(3), st, L, L, dead, near_id, nlive); break;
+    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), chol_smem_tt(4), st, L, L, dead, near_id, nlive); break;
+    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), chol_smem_tt(5), st, L, L, dead, near_id, nlive); break;
+    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), chol_smem_tt(6), st, L, L, dead, near_id, nlive); break;
+    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), chol_smem_tt(7), st, L, L, dead, near_id, nlive); break;
+    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), chol_smem_tt(8), st, L, L, dead, near_id, nlive); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
