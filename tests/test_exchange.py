@@ -1,5 +1,5 @@
 """Host logic of the sequence-parallel payload exchange
-(``activation_residual_compression_b200.exchange``), on CPU with two gloo ranks.
+(``activation_residual_compression_b200.exchange``), on CPU with two and three gloo ranks.
 
 The exchange is codec-agnostic; here each rank drives it with the CPU oracle
 as the codec (test infrastructure), so no GPU is needed.  Every rank checks
@@ -104,15 +104,24 @@ def _free_port():
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("mode,kw", CASES)
-def test_two_rank_exchange_matches_independent_replay(mode, kw):
+def _run(world, mode, kw):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, mode, kw, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, mode, kw, q)) for r in range(world)]
     for p in procs:
         p.start()
     results = dict(q.get(timeout=180) for _ in procs)
     for p in procs:
         p.join(timeout=60)
-    assert results == {0: "ok", 1: "ok"}, results
+    assert results == {r: "ok" for r in range(world)}, results
+
+
+@pytest.mark.parametrize("mode,kw", CASES)
+def test_two_rank_exchange_matches_independent_replay(mode, kw):
+    _run(2, mode, kw)
+
+
+def test_three_rank_exchange_matches_independent_replay():
+    """An odd world: every rank receives two peers' shards per tensor."""
+    _run(3, "sign1", {})
