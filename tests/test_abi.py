@@ -80,6 +80,44 @@ def test_shape_rules_rejected_on_host(cf):
     assert _ws(cf, 4, 64, cf.CF_Q2, batch=0)[0] == cf.CF_ERR_ARG
 
 
+def test_lowrank_shape_rules_rejected_on_host(cf):
+    """CF_LOWRANK: rows and cols multiples of 128, 1 <= rank <= min(rows, cols, 128),
+    1 or 2 sweeps, INT4 or fp32 factors, batch 1."""
+    L = cf.CF_LOWRANK
+    assert _ws(cf, 4096, 3072, L)[0] == cf.CF_OK
+    assert _ws(cf, 4096 + 64, 3072, L)[0] == cf.CF_ERR_SHAPE
+    assert _ws(cf, 4096, 3072 + 64, L)[0] == cf.CF_ERR_SHAPE
+    assert _ws(cf, 4096, 3072, L, rank=128)[0] == cf.CF_OK
+    assert _ws(cf, 128, 3072, L, rank=128)[0] == cf.CF_OK
+    for rank in (0, 129):
+        assert _ws(cf, 4096, 3072, L, rank=rank)[0] == cf.CF_ERR_SHAPE, rank
+    assert _ws(cf, 4096, 3072, L, iters=2)[0] == cf.CF_OK
+    for iters in (0, 3):
+        assert _ws(cf, 4096, 3072, L, iters=iters)[0] == cf.CF_ERR_UNSUPPORTED, iters
+    assert _ws(cf, 4096, 3072, L, lr_int4=0)[0] == cf.CF_OK
+    assert _ws(cf, 4096, 3072, L, lr_int4=2)[0] == cf.CF_ERR_ARG
+    assert _ws(cf, 4096, 3072, L, batch=2)[0] == cf.CF_ERR_UNSUPPORTED
+
+
+def test_blocksel_shape_rules_rejected_on_host(cf):
+    """CF_BLOCKSEL: the grid and its sides divisible by the block side (4, 8 or 16),
+    K <= 4096 blocks, 1 <= k <= K, at least one leading full step, batch 1."""
+    B = cf.CF_BLOCKSEL
+    assert _ws(cf, 4096, 3072, B)[0] == cf.CF_OK                      # 64 x 64 grid, b = 8
+    assert _ws(cf, 4096, 3072, B, bs_block=16)[0] == cf.CF_OK
+    assert _ws(cf, 4096, 3072, B, bs_block=5)[0] == cf.CF_ERR_UNSUPPORTED
+    assert _ws(cf, 4096 + 8, 3072, B)[0] == cf.CF_ERR_SHAPE           # not a square grid
+    assert _ws(cf, 4096, 3072, B, bs_grid_h=32)[0] == cf.CF_OK        # 32 x 128 grid
+    assert _ws(cf, 4096, 3072, B, bs_grid_h=48)[0] == cf.CF_ERR_SHAPE  # 48 does not divide 4096
+    assert _ws(cf, 256 * 256, 64, B, bs_block=4)[0] == cf.CF_OK       # K = 4096
+    assert _ws(cf, 512 * 512, 64, B, bs_block=4)[0] == cf.CF_ERR_UNSUPPORTED  # K = 16384
+    assert _ws(cf, 4096, 3072, B, bs_k=64)[0] == cf.CF_OK             # k = K
+    for k in (65, -1):
+        assert _ws(cf, 4096, 3072, B, bs_k=k)[0] == cf.CF_ERR_ARG, k
+    assert _ws(cf, 4096, 3072, B, bs_warm=0)[0] == cf.CF_ERR_ARG
+    assert _ws(cf, 4096, 3072, B, batch=2)[0] == cf.CF_ERR_UNSUPPORTED
+
+
 def test_workspace_sizes(cf):
     E = 4608 * 3072
     rc, s = _ws(cf, 4608, 3072, cf.CF_SIGN1, role=cf.CF_SENDER)
