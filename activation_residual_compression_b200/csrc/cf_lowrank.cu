@@ -510,8 +510,8 @@ __device__ __forceinline__ int chol_tile(int I, int J) {
   return (I * (I + 1) / 2 + J) * 8 * kCholTld;
 }
 
-// D += a B for an 8 x 8 tile: P row-major (A operand P[g][4 kc + t4]), R either
-// transposed (B[k][c] = R[c][k]) or not; sa = -1 subtracts the product.
+// D += sa P R^T (rt) or D += sa P R (!rt) for 8 x 8 tiles P, R of the packed
+// arrays, D in this lane's two accumulator entries; sa = -1 subtracts.
 __device__ __forceinline__ void chol_tile_mma(double &d0, double &d1, const double *P, const double *R, bool rt,
                                               double sa, int gq, int t4) {
 #pragma unroll
