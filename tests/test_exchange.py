@@ -6,7 +6,8 @@ as the codec (test infrastructure), so no GPU is needed.  Every rank checks
 that the reconstruction it received for each peer's shard is bit-identical
 to an independent replay of that peer's seeded stream through a local
 sender/receiver pair, and that its own slot is its exact shard -- for two
-tensors per step, warm-up steps included.
+tensors per step, warm-up steps included -- and that a payload corrupted in
+transit is reported by the receiving rank's status.
 """
 import os
 import socket
@@ -125,3 +126,76 @@ def test_two_rank_exchange_matches_independent_replay(mode, kw):
 def test_three_rank_exchange_matches_independent_replay():
     """An odd world: every rank receives two peers' shards per tensor."""
     _run(3, "sign1", {})
+
+
+T_FAULT = 4
+
+
+class CorruptingCodec(OracleCodec):
+    """Rank 1's sender flips a byte of the payload header at step T_FAULT (a
+    host-made fault in transit); receivers record the decode status instead of
+    asserting it."""
+
+    rank = 0
+
+    def __init__(self, *a, **kw):
+        super().__init__(*a, **kw)
+        self.t = 0
+        self.statuses = []
+
+    def encode(self, a, payload, stream=None):
+        super().encode(a, payload, stream)
+        if self.rank == 1 and self.t == T_FAULT:
+            payload[0] ^= 0x5A
+        self.t += 1
+
+    def decode(self, payload, recon, stream=None):
+        r, st = self.o.decode(payload.numpy())
+        self.statuses.append(st)
+        if st == 0:
+            recon.copy_(torch.from_numpy(r.reshape(recon.shape).view(np.int16)).view(torch.bfloat16))
+
+
+def _fault_worker(rank, world, port, q):
+    try:
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        from activation_residual_compression_b200.exchange import SPExchange
+        CorruptingCodec.rank = rank
+        ex = SPExchange(ROWS, COLS, "q2", n_tensors=1, device="cpu", codec_factory=CorruptingCodec)
+        seen = []
+        for t in range(STEPS):
+            ex.step([_shard(rank, 0, t)])
+            seen.append(ex.status())
+        rx = ex.channels[0].receivers
+        per_step = {p: c.statuses for p, c in rx.items()}
+        ex.close()
+        dist.barrier()
+        dist.destroy_process_group()
+        q.put((rank, (seen, per_step)))
+    except BaseException as e:  # report to the parent instead of hanging it
+        q.put((rank, repr(e)))
+
+
+def test_corrupted_payload_is_reported_by_the_receiving_rank_only():
+    """A payload whose header was altered in transit fails that step's decode
+    on the receiving rank (the receiver keeps its state) and sets its status,
+    which stays set: later payloads decode, but the exchange's status reports
+    the desync at every following step.  The sending rank sees nothing."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_fault_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+    assert all(isinstance(v, tuple) for v in results.values()), results
+    seen0, dec0 = results[0]
+    seen1, dec1 = results[1]
+    assert dec0 == {1: [0] * T_FAULT + [1] + [0] * (STEPS - T_FAULT - 1)}, dec0
+    assert seen0[:T_FAULT] == [0] * T_FAULT
+    assert all(st != 0 for st in seen0[T_FAULT:]), seen0
+    assert seen1 == [0] * STEPS and dec1 == {0: [0] * STEPS}
