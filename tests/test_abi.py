@@ -134,3 +134,33 @@ def test_null_handles_rejected(cf):
     assert cf.raw("cf_status")(P(12345), None) == cf.CF_ERR_STATE
     out = ctypes.c_size_t()
     assert cf.raw("cf_payload_bytes")(P(12345), 0, ctypes.byref(out)) == cf.CF_ERR_STATE
+
+
+def test_params_layout_and_constants_match_the_header(cf, tmp_path):
+    """The ctypes mirror of cf_params and the binding's constants against the
+    header itself, compiled as C: every field's offset, the struct size, and
+    every CF_* value the binding defines."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc") or shutil.which("cc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    fields = [f[0] for f in cf.cf_params._fields_]
+    consts = sorted(n for n in dir(cf) if n.startswith("CF_") and isinstance(getattr(cf, n), int))
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "cf.h"', "int main(void) {",
+             '  printf("size %zu\\n", sizeof(cf_params));']
+    lines += [f'  printf("off.{f} %zu\\n", offsetof(cf_params, {f}));' for f in fields]
+    lines += [f'  printf("const.{c} %d\\n", (int)({c}));' for c in consts]
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    inc = os.path.join(ROOT, "include")
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Werror", "-I", inc, str(src), "-o", str(exe)], check=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], check=True, capture_output=True,
+                                                       text=True).stdout.splitlines())
+    assert int(got["size"]) == ctypes.sizeof(cf.cf_params)
+    for f in fields:
+        assert int(got[f"off.{f}"]) == getattr(cf.cf_params, f).offset, f
+    for c in consts:
+        assert int(got[f"const.{c}"]) == getattr(cf, c), c
