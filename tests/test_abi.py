@@ -164,3 +164,17 @@ def test_params_layout_and_constants_match_the_header(cf, tmp_path):
         assert int(got[f"off.{f}"]) == getattr(cf.cf_params, f).offset, f
     for c in consts:
         assert int(got[f"const.{c}"]) == getattr(cf, c), c
+
+
+def test_missing_library_raises_instead_of_falling_back(tmp_path):
+    """Without libcf.so the binding raises on its first call; nothing runs on the CPU instead."""
+    import subprocess
+    import sys
+    code = ("import activation_residual_compression_b200 as m\n"
+            "try:\n"
+            f"    m._cf.load({str(tmp_path / 'libcf.so')!r})\n"
+            "except ImportError as e:\n"
+            "    print('raised', 'no CPU fallback' in str(e))\n")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == "raised True"
