@@ -548,3 +548,52 @@ def test_householder_first_column_along_e1(orc):
     Qn, Rn = np.linalg.qr(Y)
     Qn = Qn * np.sign(np.diag(Rn))
     assert np.abs(Q - Qn).max() < 1e-12
+
+
+def _pad16(n):
+    return (n + 15) // 16 * 16
+
+
+def _nibbles(buf, count):
+    """Two's-complement 4-bit values, low nibble first."""
+    b = np.frombuffer(buf, dtype=np.uint8)[: (count + 1) // 2]
+    v = np.empty(2 * len(b), dtype=np.int64)
+    v[0::2] = b & 0xF
+    v[1::2] = b >> 4
+    v = v[:count]
+    return np.where(v >= 8, v - 16, v)
+
+
+@pytest.mark.parametrize("int4", [1, 0])
+def test_lowrank_payload_layout_hand_parsed(orc, int4):
+    """The low-rank payload parsed by hand from its documented layout (64-byte
+    header; INT4: fp32 scales sU[r], sV[r], then U and V as nibbles, element
+    (i, k) at nibble i r + k, low nibble first, each part padded to 16 bytes;
+    fp32: U [rows][r] then V [cols][r]) gives the C the oracle's own decoder
+    reads from it, and every code lies in [-7, 7]."""
+    rows, cols, r = 48, 40, 5
+    o = orc.Oracle(rows, cols, "lowrank", dtype="f32", rank=r, iters=1, lr_int4=int4, seed=3)
+    s = _walk(rows, cols, 3, 21)
+    o.encode(s[0])
+    o.encode(s[1])
+    p = o.encode(s[2])
+    body = bytes(p[64:])
+    if int4:
+        assert len(p) == 64 + _pad16(8 * r) + _pad16((rows * r + 1) // 2) + _pad16((cols * r + 1) // 2)
+        sc = np.frombuffer(body[: 8 * r], dtype=np.float32)
+        sU, sV = sc[:r].astype(np.float64), sc[r:].astype(np.float64)
+        o1 = _pad16(8 * r)
+        qU = _nibbles(body[o1:], rows * r).reshape(rows, r)
+        o2 = o1 + _pad16((rows * r + 1) // 2)
+        qV = _nibbles(body[o2:], cols * r).reshape(cols, r)
+        assert qU.min() >= -7 and qU.max() <= 7 and qV.min() >= -7 and qV.max() <= 7
+        assert np.abs(qU).max() == 7 and np.abs(qV).max() == 7   # absmax scaling reaches the end code
+        U, V = qU * sU, qV * sV
+    else:
+        assert len(p) == 64 + _pad16(4 * rows * r) + _pad16(4 * cols * r)
+        U = np.frombuffer(body[: 4 * rows * r], dtype=np.float32).reshape(rows, r).astype(np.float64)
+        o1 = _pad16(4 * rows * r)
+        V = np.frombuffer(body[o1: o1 + 4 * cols * r], dtype=np.float32).reshape(cols, r).astype(np.float64)
+    C = U @ V.T
+    ref = o.meaning(p).astype(np.float64)
+    assert np.abs(C - ref).max() <= 1e-5 * np.abs(ref).max()
