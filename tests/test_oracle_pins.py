@@ -69,6 +69,61 @@ def test_lr_v0_range_and_exactness(orc):
     assert abs(float(V.mean())) < 0.1 and 0.25 < float(V.var()) < 0.42  # U[-1,1): var 1/3
 
 
+def _v0_exact(orc, seed, cols, r, index=lambda j, k, cols, r: j * r + k, mix=lambda s, i: s ^ i):
+    """V0[j, k] = 2 (splitmix64(seed xor (j r + k)) >> 40) 2^-24 - 1 in exact rational
+    arithmetic, from the published splitmix64 (pinned above against its reference
+    vector); `index` and `mix` are swappable so the test can show that a plausible
+    misreading of either gives different values."""
+    out = np.empty((cols, r), dtype=np.float64)
+    for j in range(cols):
+        for k in range(r):
+            z = orc.splitmix64(mix(seed, index(j, k, cols, r)) % 2 ** 64)
+            out[j, k] = float(Fraction(2 * (z >> 40), 2 ** 24) - 1)
+    return out
+
+
+@pytest.mark.parametrize("seed,cols,r", [(0, 16, 3), (42, 64, 5), (7, 5, 9), (2 ** 63 + 12345, 33, 17),
+                                         (0xDEADBEEFCAFEF00D, 128, 70)])
+def test_lr_v0_element_index_and_seed_mix(orc, seed, cols, r):
+    """The first step's V (the low-rank strategy leaves it open; this library's reading):
+    element (j, k) of the cols x r factor takes counter j r + k, xor-ed into the seed.
+    The exact values match element for element; the transposed counter k cols + j and
+    (for seeds with low bits set) the additive mix seed + (j r + k) are both told apart."""
+    got = orc.lr_v0(seed, cols, r).astype(np.float64)
+    want = _v0_exact(orc, seed, cols, r)
+    assert np.array_equal(got, want)
+    transposed = _v0_exact(orc, seed, cols, r, index=lambda j, k, cols, r: k * cols + j)
+    additive = _v0_exact(orc, seed, cols, r, mix=lambda s, i: s + i)
+    assert not np.array_equal(got, transposed)
+    if seed & 0xFFFF:  # with no low seed bits, xor and add of a small counter coincide
+        assert not np.array_equal(got, additive)
+
+
+def test_lowrank_first_step_starts_from_v0(orc):
+    """The oracle's first compressed low-rank step (fp32 factors, one sweep) starts its
+    subspace iteration from V0 with the state's seed: the factors it transmits equal
+    Q = orth(D V0) (positive diag R, numpy QR) and V = D^T Q computed here in fp64
+    from the exact V0 of the pin above."""
+    rows, cols, r, seed = 48, 40, 6, 0x1234_5678_9ABC
+    o = orc.Oracle(rows, cols, "lowrank", dtype="f32", rank=r, iters=1, lr_int4=0, seed=seed)
+    s = _walk(rows, cols, 2, 23)
+    o.encode(s[0])
+    d = ((s[1] - o.ahat_s[0]) + o.err[0]).astype(np.float32).astype(np.float64)
+    p = o.encode(s[1])
+    body = bytes(p[64:])
+    U = np.frombuffer(body[: 4 * rows * r], dtype=np.float32).reshape(rows, r).astype(np.float64)
+    o1 = (4 * rows * r + 15) // 16 * 16
+    V = np.frombuffer(body[o1: o1 + 4 * cols * r], dtype=np.float32).reshape(cols, r).astype(np.float64)
+    Qn, Rn = np.linalg.qr(d @ _v0_exact(orc, seed, cols, r))
+    Qn = Qn * np.sign(np.diag(Rn))
+    Vn = d.T @ Qn
+    assert np.abs(U - Qn).max() <= 1e-6
+    assert np.abs(V - Vn).max() <= 1e-6 * np.abs(Vn).max()
+    # a different seed gives a different first step
+    Qs, Rs = np.linalg.qr(d @ _v0_exact(orc, seed + 1, cols, r))
+    assert np.abs(U - Qs * np.sign(np.diag(Rs))).max() > 1e-3
+
+
 # ------------------------------------------------------------------ SIGN1
 
 def _exact_mean_abs(d):
