@@ -1124,6 +1124,8 @@ struct ReconArgs {
   const uint8_t *payload;
   int check_header;
   Header expect;
+  uint32_t spin_limit;  // polls of the operand wait
+  int withhold_copies;  // test hook: issue no operand copy, so that wait runs out
 };
 
 // C tile (128 rows x 128 cols) = A[rows tile] * B[cols tile]^T over K = kp,
@@ -1217,13 +1219,15 @@ __global__ void __launch_bounds__(kReconThreads, 2)
   int ok = 1;
   if (warp == 0 && lane == 0) {
     umma::mbar_arrive_expect_tx(&full, total);
-    for (int kb = 0; kb < nkb; kb++) {
+    // (with the test hook no copy is issued: the barrier's transaction count
+    // stays pending, the wait below gives up, and nothing is left in flight)
+    for (int kb = 0; kb < nkb && !R.withhold_copies; kb++) {
       umma::tma_load_2d(sm + kb * tile, &ta_hi, kb * kTileK, (int)m0, &full);
       if (R.a_split) umma::tma_load_2d(sm + off_al + kb * tile, &ta_lo, kb * kTileK, (int)m0, &full);
       umma::tma_load_2d(sm + off_bh + kb * tile, &tb_hi, kb * kTileK, (int)n0, &full);
       umma::tma_load_2d(sm + off_bl + kb * tile, &tb_lo, kb * kTileK, (int)n0, &full);
     }
-    if (!umma::mbar_wait(&full, 0)) {
+    if (!umma::mbar_wait(&full, 0, R.spin_limit)) {
       ok = 0;
     } else {
       umma::fence_after_sync();
@@ -1375,6 +1379,24 @@ cudaError_t set_recon_smem(int smem) {
     return e;
   return cudaSuccess;
 }
+// The dynamic shared-memory limit is one setting per kernel and device,
+// shared by every low-rank state (and the allocation-free decode).  The
+// kernels whose request depends on the rank -- the thin GEMM and the
+// reconstruction -- therefore get the largest request of any supported rank,
+// so that setting up a state of one rank never lowers the limit below what a
+// live state of another rank launches with.  The value is the same on every
+// call, so concurrent set-ups agree.
+cudaError_t set_shared_smem_limits() {
+  size_t thin = 0;
+  for (int n = 16; n <= kMaxRank; n += 16) {
+    const size_t b = thin_smem(n, thin_stages(n));
+    if (b > thin) thin = b;
+  }
+  const cudaError_t e =
+      cudaFuncSetAttribute(lr_thin_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)thin);
+  if (e != cudaSuccess) return e;
+  return set_recon_smem((int)recon_smem(kMaxRank / kTileK, 1));
+}
 size_t apply_smem(int n) {  // n = 16 TT: apply_mld = apply_xld = n + 4
   const size_t xt = (size_t)kApplyRows * (n + 4) * 4, qt = (size_t)n * (kApplyRows + 1) * 4;
   return (size_t)n * (n + 4) * 8 + (xt > qt ? xt : qt);
@@ -1508,10 +1530,7 @@ int lowrank_bind(LowrankPlan *plan, void *scratch) {
   if (!ok) return CF_ERR_CUDA;
   // kernels that need more than 48 KiB of dynamic shared memory
   const int rpi = plan->rp;
-  if (cudaFuncSetAttribute(lr_thin_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)thin_smem(rpi, thin_stages(rpi))) != cudaSuccess ||
-      set_recon_smem((int)recon_smem(plan->kp / kTileK, 1)) != cudaSuccess ||
-      set_apply_smem(rpi) != cudaSuccess) {
+  if (set_shared_smem_limits() != cudaSuccess || set_apply_smem(rpi) != cudaSuccess) {
     (void)cudaGetLastError();
     return CF_ERR_CUDA;
   }
@@ -1689,6 +1708,8 @@ cudaError_t dequant_and_recon(const LowrankPlan &P, const uint8_t *payload, bool
   R.payload = payload;
   R.check_header = receiver;
   R.expect = expect;
+  R.spin_limit = P.test_wait_polls ? P.test_wait_polls : umma::kSpinLimit;
+  R.withhold_copies = P.test_wait_polls != 0;
   const dim3 grid((unsigned)(P.rows / kTileM), (unsigned)(P.cols / kReconN));
   const size_t smem = recon_smem(R.kblocks, R.a_split);
   auto *kern = P.dtype == CF_BF16 ? (receiver ? lr_recon_kernel<__nv_bfloat16, false> : lr_recon_kernel<__nv_bfloat16, true>)
@@ -1783,8 +1804,7 @@ int noalloc_scratch(void **out) {
       (void)cudaGetLastError();
       return CF_ERR_CUDA;
     }
-    const int smem = (int)recon_smem(2, 1);
-    if (set_recon_smem(smem) != cudaSuccess) {
+    if (set_shared_smem_limits() != cudaSuccess) {
       (void)cudaGetLastError();
       return CF_ERR_CUDA;
     }

@@ -126,9 +126,9 @@ def flux(device="cpu", rows=4608, cols=3072, seed=1):
                             outlier_frac=0.01, seed_per_tensor=[seed])
 
 
-def ar1(device="cpu", rows=4096, cols=3072, seed=3):
+def ar1(device="cpu", rows=4096, cols=3072, seed=3, dtype=torch.bfloat16):
     """Stationary AR(1) stream for the low-rank mode."""
-    return ActivationStream(rows, cols, dtype=torch.bfloat16, device=device, seed=seed, sigma=0.1,
+    return ActivationStream(rows, cols, dtype=dtype, device=device, seed=seed, sigma=0.1,
                             rho=math.sqrt(0.99), seed_per_tensor=[seed])
 
 

@@ -239,6 +239,18 @@ CF_API int cf_step(const cf_state *s, uint64_t *out);
  * is cleared.  Synchronous (device memset on the legacy stream). */
 CF_API int cf_reset(cf_state *s);
 
+/* Test hook for the failure detection of the low-rank kernels (the pages
+ * have no counterpart: this is the library's own bounded-wait check).  With
+ * polls > 0, every later reconstruction launch of this CF_LOWRANK state (the
+ * receiver's decode; the last kernel of a sender's encode) issues none of its
+ * operand copies and waits at most `polls` polls for them, so its bounded
+ * wait gives up: the kernel records the timeout in the state's status word
+ * (cf_status then returns CF_ERR_TIMEOUT), frees its tensor memory and
+ * returns without writing ahat, e or recon.  No copy or MMA is left in
+ * flight.  polls = 0 restores normal operation; cf_reset clears the status.
+ * Returns CF_ERR_UNSUPPORTED for the other modes. */
+CF_API int cf_test_wait_timeout(cf_state *s, uint32_t polls);
+
 /* Checkpoint / resume: cf_state_bytes gives the host buffer size;
  * cf_state_export copies the state (step, status and tensors) into it,
  * cf_state_import restores a state of the same configuration.  Both
@@ -261,8 +273,9 @@ CF_API int cf_state_import(cf_state *s, const void *host, size_t bytes, void *st
  * rows, cols, p and `step`, leaving ahat and recon untouched, and 2 when a
  * bounded wait gave up), the device `payload` and the stream.  p supplies
  * dtype, ef, rank, iters and lr_int4 (role, batch and workspace are
- * ignored; batch must be 1).  `step` (>= 1) is the step the payload must
- * carry; the warm-up step (raw activations) is not handled here.
+ * ignored: this decode always handles one tensor).  `step` (>= 1) is the
+ * step the payload must carry; the warm-up step (raw activations) is not
+ * handled here.
  * The dequantised factors go to a fixed scratch array of 8 MiB that every
  * GPU loading the library holds until exit: (rows*kp*(int4 ? 2 : 4) +
  * cols*kp*4) bytes, each part rounded up to 256, must fit, where kp is rank

@@ -90,6 +90,8 @@ def lib():
         L.orc_q2_level.restype = c.c_float
         L.orc_q2_level.argtypes = [c.c_int, c.c_float]
         L.orc_nm_select.argtypes = [P, c.c_int, c.c_int, P]
+        L.orc_set_threads.restype = c.c_int
+        L.orc_set_threads.argtypes = [c.c_int]
         L.orc_splitmix64.restype = c.c_uint64
         L.orc_splitmix64.argtypes = [c.c_uint64]
         L.orc_lr_v0.restype = c.c_float
@@ -155,6 +157,11 @@ def nm_select(d, n: int) -> list[int]:
     out = np.zeros(n, dtype=np.int32)
     lib().orc_nm_select(_ptr(d), d.size, n, _ptr(out))
     return [int(v) for v in out]
+
+
+def set_threads(n: int) -> int:
+    """Threads of the oracle's row-parallel loops (timing only); returns the count in effect."""
+    return int(lib().orc_set_threads(int(n)))
 
 
 def splitmix64(x: int) -> int:
@@ -226,8 +233,11 @@ class Oracle:
     def __del__(self):
         h = getattr(self, "_h", None)
         if h:
-            lib().orc_destroy(h)
             self._h = None
+            try:
+                lib().orc_destroy(h)
+            except TypeError:   # interpreter shutdown: the module globals are gone
+                pass
 
     @property
     def np_act(self):

@@ -266,6 +266,53 @@ def test_closed_loop_quality_matches_oracle():
         pair.close()
 
 
+def _closed_loop(rows, cols, rank, iters, ef, T, seed=3):
+    """GPU and oracle run independently on one stream; returns the per-step relative
+    state distance ||ahat_gpu - ahat_orc|| / ||ahat_orc|| (receiver states), with the
+    GPU's sender and receiver checked bit-equal at the end."""
+    pair = GpuPair(rows, cols, "lowrank", dtype="bf16", ef=ef, rank=rank, iters=iters, lr_int4=1, seed=7)
+    orc = oracle.Oracle(rows, cols, "lowrank", dtype="bf16", ef=ef, rank=rank, iters=iters, lr_int4=1, seed=7)
+    s = inputs.ar1("cuda", rows=rows, cols=cols, seed=seed)
+    dist = []
+    try:
+        for t in range(T):
+            a = s.next()
+            pair.step(a)
+            orc.decode(orc.encode(to_np(a)))
+            torch.cuda.synchronize()
+            dist.append(_rel(pair.state("R")[0][0], orc.ahat_r[0]))
+        ah_s, _ = pair.state("S")
+        ah_r, _ = pair.state("R")
+        assert np.array_equal(ah_s.view(np.uint32), ah_r.view(np.uint32))
+        assert cf.cf_status(pair.R) == cf.CF_OK and cf.cf_status(pair.S) == cf.CF_OK
+    finally:
+        pair.close()
+    return dist
+
+
+@pytest.mark.parametrize("ef", ["explicit", "implicit"])
+@pytest.mark.parametrize("iters", [1, 2])
+def test_closed_loop_state_distance(ef, iters):
+    """Closed loop, 1024 x 768 rank 70 INT4, 28 steps (1 warm-up + 27 compressed):
+    the GPU's reconstruction stays within 2e-2 (relative) of the oracle's own,
+    although neither is ever reset to the other."""
+    dist = _closed_loop(1024, 768, 70, iters, ef, 28)
+    print(f"closed loop {ef} k={iters}: state distance at T {dist[-1]:.3e}, max {max(dist):.3e}")
+    assert dist[0] == 0.0                                    # the warm-up step is exact
+    assert dist[-1] <= 2e-2, dist
+
+
+@pytest.mark.parametrize("iters", [1, 2])
+def test_full_size_closed_loop_state_distance(iters):
+    """The low-rank configuration at full size (4096 x 3072 bf16 AR(1), rank 70,
+    INT4, 28 steps, explicit feedback) in closed loop: GPU and fp64 oracle each run
+    the whole stream; the relative distance of their reconstructions at T is gated
+    at 2e-2."""
+    dist = _closed_loop(4096, 3072, 70, iters, "explicit", 28)
+    print(f"full-size closed loop k={iters}: " + " ".join(f"{d:.2e}" for d in dist))
+    assert dist[-1] <= 2e-2, dist
+
+
 @pytest.mark.parametrize("iters", [1, 2])
 def test_full_size_config_teacher_forced(iters):
     """4096 x 3072 bf16 AR(1) stream, rank 70, INT4, 28 steps; the oracle is
@@ -296,6 +343,40 @@ def test_full_size_config_teacher_forced(iters):
         assert pair.pb == 64 + 560 + 143360 + 107520                   # 100.06x smaller than the bf16 tensor
     finally:
         pair.close()
+
+
+def test_live_states_of_different_ranks():
+    """The thin GEMM's and the reconstruction's shared-memory limits are one setting
+    per kernel: a rank-128 state created after a rank-70 one (which needs the larger
+    GEMM operand ring) must leave the rank-70 state working.  Its payloads and
+    reconstructions equal those of a rank-70 state run with no other state alive."""
+    rows, cols = 512, 384
+    s = inputs.ar1("cuda", rows=rows, cols=cols)
+    acts = [s.next() for _ in range(4)]
+    ref = _lr_pair(rows, cols, 70, 1, 1)
+    want = []
+    try:
+        for a in acts:
+            ref.step(a)
+            torch.cuda.synchronize()
+            want.append((ref.payload_np(ref.t == 1).copy(), to_np(ref.recon).copy()))
+        assert cf.cf_status(ref.S) == cf.CF_OK and cf.cf_status(ref.R) == cf.CF_OK
+    finally:
+        ref.close()
+    p70 = _lr_pair(rows, cols, 70, 1, 1)
+    p128 = _lr_pair(rows, cols, 128, 1, 1)
+    try:
+        for t, a in enumerate(acts):
+            p70.step(a)
+            p128.step(a)
+            torch.cuda.synchronize()
+            assert np.array_equal(p70.payload_np(t == 0), want[t][0]), t
+            assert np.array_equal(to_np(p70.recon), want[t][1]), t
+        for p in (p70, p128):
+            assert cf.cf_status(p.S) == cf.CF_OK and cf.cf_status(p.R) == cf.CF_OK
+    finally:
+        p70.close()
+        p128.close()
 
 
 def test_lowrank_desync_detected():
