@@ -72,7 +72,7 @@ _lib = None
 EXPORTS = ["cf_version", "cf_strerror", "cf_params_init", "cf_workspace_bytes", "cf_create", "cf_payload_bytes",
            "cf_encode", "cf_decode", "cf_encode_batched", "cf_decode_batched", "cf_status", "cf_tensor",
            "cf_step", "cf_reset", "cf_state_bytes", "cf_state_export", "cf_state_import", "cf_destroy",
-           "cf_lowrank_decode_noalloc"]
+           "cf_lowrank_decode_noalloc", "cf_test_wait_timeout"]
 
 
 def load(path: str = LIB_PATH):
@@ -108,6 +108,7 @@ def load(path: str = LIB_PATH):
     L.cf_state_import.argtypes = [P, P, c.c_size_t, P]
     L.cf_destroy.argtypes = [P]
     L.cf_lowrank_decode_noalloc.argtypes = [c.c_int64, c.c_int64, c.POINTER(cf_params), c.c_uint64, P, P, P, P, P]
+    L.cf_test_wait_timeout.argtypes = [P, c.c_uint32]
     for name in EXPORTS:
         if name not in ("cf_version", "cf_strerror"):
             getattr(L, name).restype = c.c_int
@@ -255,6 +256,12 @@ def cf_lowrank_decode_noalloc(rows: int, cols: int, params: cf_params, step: int
     return _check("cf_lowrank_decode_noalloc", load().cf_lowrank_decode_noalloc(
         rows, cols, ctypes.byref(params), step, _ptr(payload), _ptr(ahat), _ptr(recon), _ptr(status),
         _stream(stream)))
+
+
+def cf_test_wait_timeout(state, polls: int) -> int:
+    """Low-rank failure-detection test hook (see include/cf.h): polls > 0 makes the
+    reconstruction kernel's bounded operand wait run out; 0 restores it."""
+    return _check("cf_test_wait_timeout", load().cf_test_wait_timeout(state, polls))
 
 
 def raw(name: str):

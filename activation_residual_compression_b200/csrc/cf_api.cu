@@ -626,6 +626,13 @@ int cf_reset(cf_state *s) {
   return CF_OK;
 }
 
+int cf_test_wait_timeout(cf_state *s, uint32_t polls) {
+  if (!live(s)) return CF_ERR_STATE;
+  if (s->mode != CF_LOWRANK) return CF_ERR_UNSUPPORTED;
+  s->lr.test_wait_polls = polls;
+  return CF_OK;
+}
+
 static size_t export_tensor_bytes(const cf_state *s) {
   const size_t E = (size_t)(s->rows * s->cols) * (size_t)s->p.batch;
   size_t b = E * ahat_elem_bytes(s);

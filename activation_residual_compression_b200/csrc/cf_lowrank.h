@@ -35,6 +35,7 @@ struct LowrankPlan {
   int rank = 0, rp = 0, kp = 0, iters = 1, int4 = 1, batch = 1;
   int role = 0, ef_explicit = 1, ef_off = 0, dtype = CF_BF16;
   double qr2_tol = 0.0;          // near-identity bound of the second CholeskyQR pass (0: full)
+  uint32_t test_wait_polls = 0;  // test hook: > 0 makes the reconstruction's operand wait run out
   int sy = 1, sv = 1;            // split-K factors of the two thin GEMMs
   int nblk_gram = 1;             // row blocks of the partial Gram matrices
   size_t enc_scratch_bytes = 0;

@@ -42,13 +42,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: gives up after kSpinLimit polls (each poll may suspend the
-// thread for a hardware-defined interval), so a copy or MMA that never
-// completes cannot hang the GPU; the caller records the failure and leaves.
+// Bounded wait: gives up after `limit` polls (kSpinLimit unless a caller
+// passes a shorter one; each poll may suspend the thread for a
+// hardware-defined interval), so a copy or MMA that never completes cannot
+// hang the GPU; the caller records the failure and leaves.
 constexpr uint32_t kSpinLimit = 1u << 22;
 
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it)
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit = kSpinLimit) {
+  for (uint32_t it = 0; it < limit; ++it)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }

@@ -1,7 +1,8 @@
 """Host-made faults and state management on the GPU path: every failure is
 injected on the host (a corrupted header, a skipped step, a wrong role, a
-misaligned or missing pointer, a destroyed handle); no kernel traps, spins or
-faults.  Also checkpoint/resume and reset."""
+misaligned or missing pointer, a destroyed handle) or is a bounded device wait
+made to run out with nothing in flight; no kernel traps, spins without a limit
+or faults.  Also checkpoint/resume and reset."""
 import ctypes
 
 import numpy as np
@@ -52,6 +53,60 @@ def test_header_mismatch_sets_desync_and_leaves_receiver(corrupt):
         pair.step(s.next())
         pair.step(s.next())
         assert cf.cf_status(pair.R) == cf.CF_OK
+    finally:
+        pair.close()
+
+
+@pytest.mark.parametrize("role", ["receiver", "sender"])
+def test_lowrank_bounded_wait_runs_out(role):
+    """The low-rank reconstruction kernel's bounded wait for its operand copies,
+    made to run out by the test hook (no copy is issued, so nothing is in flight;
+    a limit of 256 polls): the kernel returns, cf_status reports CF_ERR_TIMEOUT
+    for that state only, and the state it would have updated (receiver: ahat and
+    recon; sender: ahat and e) is unchanged.  With the hook off and both states
+    reset, a clean request runs and reports no error."""
+    rows, cols = 256, 256
+    pair = GpuPair(rows, cols, "lowrank", dtype="bf16", rank=16, iters=1, lr_int4=1, seed=3)
+    s = inputs.ar1("cuda", rows=rows, cols=cols)
+    try:
+        pair.step(s.next())
+        pair.step(s.next())
+        torch.cuda.synchronize()
+        hooked, other = (pair.R, pair.S) if role == "receiver" else (pair.S, pair.R)
+        which = "R" if role == "receiver" else "S"
+        before = pair.state(which)
+        rec_before = to_np(pair.recon).copy()
+        cf.cf_test_wait_timeout(hooked, 256)
+        a = s.next()
+        cf.cf_encode(pair.S, a, pair.payload)
+        if role == "receiver":
+            cf.cf_decode(pair.R, pair.payload, pair.recon)
+        assert cf.cf_status(hooked) == cf.CF_ERR_TIMEOUT
+        assert cf.cf_status(other) == cf.CF_OK
+        after = pair.state(which)
+        assert np.array_equal(before[0].view(np.uint32), after[0].view(np.uint32))
+        if role == "sender":
+            assert np.array_equal(before[1].view(np.uint32), after[1].view(np.uint32))
+        assert np.array_equal(rec_before, to_np(pair.recon))
+        # the context is still usable: hook off, both sides reset, a clean request
+        cf.cf_test_wait_timeout(hooked, 0)
+        cf.cf_reset(pair.S)
+        cf.cf_reset(pair.R)
+        for _ in range(3):
+            pair.step(s.next())
+        assert cf.cf_status(pair.S) == cf.CF_OK and cf.cf_status(pair.R) == cf.CF_OK
+        ah_s, _ = pair.state("S")
+        ah_r, _ = pair.state("R")
+        assert np.array_equal(ah_s.view(np.uint32), ah_r.view(np.uint32))
+        assert cf.raw("cf_test_wait_timeout")(pair.S, 0) == cf.CF_OK
+    finally:
+        pair.close()
+
+
+def test_wait_timeout_hook_is_lowrank_only():
+    pair, _ = _pair_after(1)
+    try:
+        assert cf.raw("cf_test_wait_timeout")(pair.S, 16) == cf.CF_ERR_UNSUPPORTED
     finally:
         pair.close()
 
