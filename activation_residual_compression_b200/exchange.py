@@ -20,6 +20,10 @@ The host logic (payload sizes, warm-up steps, ordering, per-peer states) is
 independent of the codec: ``codec_factory`` builds the per-tensor codec; the
 default is the CUDA library (``CfCodec``).  Payloads travel as uint8 tensors;
 no TMA multicast or peer-memory loads are involved (NCCL moves the bytes).
+On a group whose backend cannot gather device tensors (gloo), device payloads
+are staged through host memory: copied to the host, gathered there, and
+copied back before the peers' decodes (a synchronous transport, used when
+several ranks share one GPU or have no NVLink path).
 """
 from __future__ import annotations
 
@@ -56,6 +60,10 @@ class CfCodec:
 
     def status(self, stream=None) -> int:
         return cf.cf_status(self.h, stream)
+
+    def reset(self):
+        """New request: the next call is the warm-up step again."""
+        cf.cf_reset(self.h)
 
     def close(self):
         if self.h is not None:
@@ -97,7 +105,9 @@ class SPExchange:
             self.channels.append(_Channel(
                 s, rx, torch.empty(n, dtype=torch.uint8, device=self.device),
                 torch.empty(self.world, n, dtype=torch.uint8, device=self.device)))
-        self.comm = torch.cuda.Stream(self.device) if self.cuda else None
+        # device payloads over a backend without device collectives go through the host
+        self.host_staged = self.cuda and dist.get_backend(group) == "gloo"
+        self.comm = torch.cuda.Stream(self.device) if self.cuda and not self.host_staged else None
         self.t = 0
 
     def step(self, shards):
@@ -116,7 +126,9 @@ class SPExchange:
             P = ch.sender.payload_bytes(warm)
             sizes.append(P)
             ch.sender.encode(a, ch.send_buf[:P], compute)
-            if self.cuda:
+            if self.host_staged:
+                work = _host_staged_gather(_flat(ch.gather_buf, P), ch.send_buf[:P], self.world, self.group)
+            elif self.cuda:
                 self.comm.wait_stream(compute)
                 with torch.cuda.stream(self.comm):
                     work = dist.all_gather_into_tensor(_flat(ch.gather_buf, P), ch.send_buf[:P], group=self.group,
@@ -128,7 +140,7 @@ class SPExchange:
         # decode the peers' payloads of each tensor once its gather is complete
         for ch, a, out, P, work in zip(self.channels, shards, outs, sizes, gathered):
             work.wait()
-            if self.cuda:
+            if self.comm is not None:
                 compute.wait_stream(self.comm)
             flat = _flat(ch.gather_buf, P).view(self.world, P)
             for p, rx in ch.receivers.items():
@@ -136,6 +148,14 @@ class SPExchange:
             out[self.rank].copy_(a)
         self.t += 1
         return outs
+
+    def reset(self):
+        """Start a new request on every state of this rank (the next step is a
+        warm-up step again); every rank must reset before the same step."""
+        for ch in self.channels:
+            for c in [ch.sender] + list(ch.receivers.values()):
+                c.reset()
+        self.t = 0
 
     def status(self) -> int:
         """First nonzero device status of this rank's states (libcf codes)."""
@@ -151,6 +171,24 @@ class SPExchange:
             for c in [ch.sender] + list(ch.receivers.values()):
                 c.close()
         self.channels = []
+
+
+class _Done:
+    """A completed collective (the synchronous host-staged transport)."""
+
+    def wait(self):
+        return True
+
+
+def _host_staged_gather(out: torch.Tensor, send: torch.Tensor, world: int, group) -> _Done:
+    """All-gather of device bytes through host memory: the device-to-host copy
+    waits for the encode on the current stream; the gathered bytes are copied
+    back on the current stream, ahead of the decodes enqueued after it."""
+    h_send = send.cpu()
+    h_out = torch.empty(world * h_send.numel(), dtype=torch.uint8)
+    dist.all_gather_into_tensor(h_out, h_send, group=group)
+    out.copy_(h_out.to(out.device, non_blocking=False))
+    return _Done()
 
 
 def _flat(gather_buf: torch.Tensor, P: int) -> torch.Tensor:

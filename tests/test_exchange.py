@@ -31,6 +31,7 @@ class OracleCodec:
         if "bs_grid_h" in kw:
             kw["bs_h"] = kw.pop("bs_grid_h")
         self.o = oracle.Oracle(rows, cols, mode, dtype="bf16", **kw)
+        self.kw = kw
         self.role = role
 
     def payload_bytes(self, warm):
@@ -50,6 +51,11 @@ class OracleCodec:
 
     def status(self, stream=None):
         return self.o.status()
+
+    def reset(self):
+        import oracle
+        o = self.o
+        self.o = oracle.Oracle(o.rows, o.cols, o.mode, dtype="bf16", **self.kw)
 
     def close(self):
         pass
@@ -199,3 +205,47 @@ def test_corrupted_payload_is_reported_by_the_receiving_rank_only():
     assert seen0[:T_FAULT] == [0] * T_FAULT
     assert all(st != 0 for st in seen0[T_FAULT:]), seen0
     assert seen1 == [0] * STEPS and dec1 == {0: [0] * STEPS}
+
+
+def _bench_worker(rank, world, port, q):
+    try:
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        import bench
+        from activation_residual_compression_b200.exchange import SPExchange
+        ex = SPExchange(ROWS, COLS, "q2", n_tensors=2, device="cpu", codec_factory=OracleCodec)
+        res = bench.exchange_bench(ex, lambda t: [_shard(rank, i, t) for i in range(2)], 4, 3, "cpu")
+        # the exchange still works after the bench's resets: a fresh request decodes every peer exactly
+        outs = ex.step([_shard(rank, i, 0) for i in range(2)])
+        for i in range(2):
+            for p in range(world):
+                assert torch.equal(outs[i][p], _shard(p, i, 0))      # warm-up step: raw activations
+        ex.close()
+        dist.barrier()
+        dist.destroy_process_group()
+        q.put((rank, res))
+    except BaseException as e:  # report to the parent instead of hanging it
+        q.put((rank, repr(e)))
+
+
+def test_exchange_bench_on_two_gloo_ranks():
+    """bench.py's exchange timing (the --exchange leg) on two CPU ranks with the
+    oracle as the codec: it runs, agrees across ranks (times are maxima over
+    ranks), reports positive step and codec times, no error status, and leaves
+    the exchange usable."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bench_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = dict(q.get(timeout=240) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+    assert all(isinstance(v, dict) for v in results.values()), results
+    r0, r1 = results[0], results[1]
+    assert r0["ms_per_step"] == r1["ms_per_step"] and r0["codec_ms_per_step"] == r1["codec_ms_per_step"]
+    assert r0["ms_per_step"] > 0 and r0["codec_ms_per_step"] > 0 and r0["status"] == 0
+    assert r0["activation_gbs_per_rank"] > 0
+    assert r0["payload_bytes_per_tensor"] == 64 + 16 * ((ROWS * 2 + 15) // 16) + ROWS * COLS // 4
