@@ -45,6 +45,8 @@ sys.path.insert(0, ROOT)
 ROWS, COLS = 4608, 3072
 MODES = [("sign1", {}), ("q2", {})]
 WORKLOAD = "flux1dev-4608x3072-bf16"
+SEQ_STEPS = 27          # compressed steps of a 28-step request (one warm-up step + 27)
+DATASHEET_GBS = 8000.0  # B200 HBM3e datasheet bandwidth (context beside the measured copy peak)
 METRIC = "activation GB/s and ms/step per mode (encode+EF+decode), % of B200 HBM roofline"
 
 # Timed workloads (--workload): shape, batch, seeded stream and the codecs one
@@ -275,7 +277,8 @@ def run_cf(args, rank, world, device):
     stream = torch.cuda.Stream()
     K, W = args.steps, args.warmup
     in_bytes = B_ * R_ * C_ * 2
-    n_inputs = max(2, min(W + K + 1, args.max_resident, int(args.resident_gb * 1e9 // (in_bytes * len(wl["codecs"])))))
+    want = max(W + K + 1, SEQ_STEPS + 1 if args.sequences > 0 else 0)
+    n_inputs = max(2, min(want, args.max_resident, int(args.resident_gb * 1e9 // (in_bytes * len(wl["codecs"])))))
     batched = B_ > 1
     codecs = []
     for mi, (mode, kw) in enumerate(wl["codecs"]):
@@ -364,6 +367,35 @@ def run_cf(args, rank, world, device):
         if cf.cf_status(c["R"], stream) != cf.CF_OK or cf.cf_status(c["S"], stream) != cf.CF_OK:
             raise RuntimeError(f"codec {c['name']} reported an error status")
 
+    # full sequences: each a new request (both states reset, the warm-up step
+    # untimed) of SEQ_STEPS compressed steps, every encode and decode bracketed
+    # by events; the median over sequences of the mean step time
+    seq = None
+    if args.sequences > 0:
+        W_seq = max(kw.get("bs_warm", 1) for _, kw in wl["codecs"])
+        seq_step, seq_per = [], {c["name"]: [] for c in codecs}
+        for q in range(args.sequences):
+            for c in codecs:
+                cf.cf_reset(c["S"]); cf.cf_reset(c["R"])
+            sev = []
+            with torch.cuda.stream(stream):
+                for i in range(W_seq):
+                    step(i)
+                for i in range(W_seq, W_seq + SEQ_STEPS):
+                    step(i, sev)
+            torch.cuda.synchronize()
+            tot = 0.0
+            for mi, c in enumerate(codecs):
+                ms_c = sum(sev[k * stride + 2 * mi].elapsed_time(sev[k * stride + 2 * mi + 2])
+                           for k in range(SEQ_STEPS)) / SEQ_STEPS
+                seq_per[c["name"]].append(ms_c)
+                tot += ms_c
+            seq_step.append(tot)
+        for c in codecs:
+            if cf.cf_status(c["R"], stream) != cf.CF_OK or cf.cf_status(c["S"], stream) != cf.CF_OK:
+                raise RuntimeError(f"codec {c['name']} reported an error status in the sequence runs")
+        seq = dict(n=args.sequences, steps=SEQ_STEPS, step_ms=seq_step, per=seq_per)
+
     # e2e: pinned host activations in, pinned host reconstruction out, every
     # step.  Three streams and two buffer slots: the host-to-device copy of
     # step i+1 and the device-to-host copy of step i-1 run while step i is
@@ -434,16 +466,18 @@ def run_cf(args, rank, world, device):
 
     ms_step = total_ms / K
     stats = dict(ms_step=ms_step, per={m: {k: statistics.mean(v) for k, v in d.items()} for m, d in per.items()},
-                 e2e=e2e, clocks=clk, codecs=info)
+                 e2e=e2e, clocks=clk, codecs=info, seq=seq)
     return stats
 
 
-def _lr_alg_bytes(rows, cols, iters, payload):
+def _lr_alg_bytes(rows, cols, iters, payload, ef="explicit"):
     """Low-rank step's algorithmic bytes: read a, ahat, e and write ahat, e once
-    (sender), re-read the residual as one bf16 copy per GEMM (2 per iteration),
-    read and write the receiver's ahat and write recon, plus the payload twice."""
+    (sender; implicit feedback reads no e), re-read the residual as one bf16
+    copy per GEMM (2 per iteration), read and write the receiver's ahat and
+    write recon, plus the payload twice."""
     E = rows * cols
-    return E * (2 + 16 + 4 * iters) + E * (4 + 4 + 2) + 2 * payload
+    sender = 2 + 4 + (4 if ef == "explicit" else 0) + 4 + 4
+    return E * (sender + 4 * iters) + E * (4 + 4 + 2) + 2 * payload
 
 
 def run_suite(args, device):
@@ -496,6 +530,39 @@ def run_suite(args, device):
                           device="cuda")
         return S, R, pay
 
+    def entry(e_ms, d_ms, alg, act_bytes, P, **extra):
+        t = (e_ms + d_ms) / 1e3
+        return {"ms_per_step": round(e_ms + d_ms, 5), "encode_ms": round(e_ms, 5), "decode_ms": round(d_ms, 5),
+                "activation_gbs": round(act_bytes / t / 1e9, 2), "roofline_frac": round(alg / t / 1e9 / peak, 4),
+                "roofline_frac_datasheet": round(alg / t / 1e9 / DATASHEET_GBS, 4),
+                "payload_bytes": P, "ratio_vs_bf16": round(act_bytes / P, 2), **extra}
+
+    # implicit error feedback on the FLUX-shaped stream: the form that settles to a
+    # bounded steady state in every mode (the explicit recurrence diverges for N:M)
+    for mode, kw in (("sign1", {}), ("q2", {}), ("nm", {"nm_n": 1, "nm_m": 16}), ("nm", {"nm_n": 2, "nm_m": 16})):
+        s = inputs.flux("cuda", rows=ROWS, cols=COLS, seed=6)
+        acts = [s.next() for _ in range(24)]
+        S, R, pay = make(ROWS, COLS, mode, dict(kw, ef=EF_CODES["implicit"]))
+        rec = torch.empty(ROWS, COLS, dtype=torch.bfloat16, device="cuda")
+        e_ms, d_ms = timed(S, R, pay, rec, acts, 20, 4, False)
+        alg = encode_bytes(mode, ROWS, COLS, kw, ef="implicit") + decode_bytes(mode, ROWS, COLS, kw)
+        out[f"{_codec_name(mode, kw)}_flux_implicit"] = entry(e_ms, d_ms, alg, ROWS * COLS * 2,
+                                                              cf.cf_payload_bytes(S, False))
+        cf.cf_destroy(S); cf.cf_destroy(R)
+        del acts
+    # block selection (the Otil page): 64 x 64 token grid x 3072 channels, 8 x 8 blocks, k/K = 16/64
+    bkw = {"bs_grid_h": 64, "bs_block": 8, "bs_k": 16, "bs_warm": 5}
+    s = inputs.blocksel("cuda", seed=1)
+    acts = [s.next() for _ in range(28)]
+    S, R, pay = make(4096, 3072, "blocksel", bkw)
+    rec = torch.empty(4096, 3072, dtype=torch.bfloat16, device="cuda")
+    e_ms, d_ms = timed(S, R, pay, rec, acts, 20, bkw["bs_warm"] + 2, False)
+    alg = encode_bytes("blocksel", 4096, 3072, bkw) + decode_bytes("blocksel", 4096, 3072, bkw)
+    out["blocksel_grid64x64_3072_b8_k16"] = entry(e_ms, d_ms, alg, 4096 * 3072 * 2, cf.cf_payload_bytes(S, False),
+                                                  launches_per_step=3)
+    cf.cf_destroy(S); cf.cf_destroy(R)
+    del acts
+
     # N:M 1:16 and 2:16 on the FLUX-shaped stream
     for n in (1, 2):
         kw = {"nm_n": n, "nm_m": 16}
@@ -506,29 +573,25 @@ def run_suite(args, device):
         e_ms, d_ms = timed(S, R, pay, rec, acts, 20, 4, False)
         alg = encode_bytes("nm", ROWS, COLS, kw) + decode_bytes("nm", ROWS, COLS, kw)
         P = 64 + _payload_body("nm", ROWS, COLS, kw)
-        out[f"nm{n}_16_flux"] = {"ms_per_step": round(e_ms + d_ms, 5), "encode_ms": round(e_ms, 5),
-                                 "decode_ms": round(d_ms, 5),
-                                 "activation_gbs": round(ROWS * COLS * 2 / ((e_ms + d_ms) / 1e3) / 1e9, 2),
-                                 "roofline_frac": round(alg / ((e_ms + d_ms) / 1e3) / 1e9 / peak, 4),
-                                 "ratio_vs_bf16": round(ROWS * COLS * 2 / P, 2)}
+        out[f"nm{n}_16_flux"] = entry(e_ms, d_ms, alg, ROWS * COLS * 2, P)
         cf.cf_destroy(S); cf.cf_destroy(R)
         del acts
-    # low-rank ~100x on 4096 x 3072, rank 70, INT4, 1 and 2 iterations
+    # low-rank ~100x on 4096 x 3072, rank 70, INT4, 1 and 2 iterations (explicit
+    # feedback, as specified), and 1 iteration with implicit feedback
     lr_rows, lr_cols = 4096, 3072
-    for it in (1, 2):
+    for it, ef in ((1, "explicit"), (2, "explicit"), (1, "implicit")):
         s = inputs.ar1("cuda", rows=lr_rows, cols=lr_cols)
         acts = [s.next() for _ in range(28)]
-        S, R, pay = make(lr_rows, lr_cols, "lowrank", {"rank": 70, "iters": it, "lr_int4": 1, "seed": 7})
+        S, R, pay = make(lr_rows, lr_cols, "lowrank", {"rank": 70, "iters": it, "lr_int4": 1, "seed": 7,
+                                                       "ef": EF_CODES[ef]})
         rec = torch.empty(lr_rows, lr_cols, dtype=torch.bfloat16, device="cuda")
         e_ms, d_ms = timed(S, R, pay, rec, acts, 20, 5, False)
         P = cf.cf_payload_bytes(S, False)
-        alg = _lr_alg_bytes(lr_rows, lr_cols, it, P)
-        out[f"lowrank_r70_k{it}"] = {"ms_per_step": round(e_ms + d_ms, 5), "encode_ms": round(e_ms, 5),
-                                     "decode_ms": round(d_ms, 5),
-                                     "activation_gbs": round(lr_rows * lr_cols * 2 / ((e_ms + d_ms) / 1e3) / 1e9, 2),
-                                     "roofline_frac": round(alg / ((e_ms + d_ms) / 1e3) / 1e9 / peak, 4),
-                                     "payload_bytes": P, "ratio_vs_bf16": round(lr_rows * lr_cols * 2 / P, 2),
-                                     "budget_note": "pages quote a ~1 ms compression budget"}
+        alg = _lr_alg_bytes(lr_rows, lr_cols, it, P, ef=ef)
+        name = f"lowrank_r70_k{it}" + ("" if ef == "explicit" else "_implicit")
+        out[name] = entry(e_ms, d_ms, alg, lr_rows * lr_cols * 2, P,
+                          launches_per_step=launches_per_call("lowrank", {"iters": it}, True) + 2,
+                          budget_note="pages quote a ~1 ms compression budget")
         cf.cf_destroy(S); cf.cf_destroy(R)
         del acts
     # CogVideoX-2b-shaped full step: 60 tensors of 17550 x 1920, Q2, one launch each way
@@ -543,11 +606,8 @@ def run_suite(args, device):
         e_ms, d_ms = timed(S, R, pay, recs, acts, 6, 2, True)
         E = B * cr * cc
         alg = B * (encode_bytes("q2", cr, cc, {}) + decode_bytes("q2", cr, cc, {}))
-        out["cogvideox_q2_60x17550x1920"] = {"ms_per_step": round(e_ms + d_ms, 4), "encode_ms": round(e_ms, 4),
-                                             "decode_ms": round(d_ms, 4),
-                                             "activation_gbs": round(E * 2 / ((e_ms + d_ms) / 1e3) / 1e9, 2),
-                                             "roofline_frac": round(alg / ((e_ms + d_ms) / 1e3) / 1e9 / peak, 4),
-                                             "launches_per_step": 2}
+        out["cogvideox_q2_60x17550x1920"] = entry(e_ms, d_ms, alg, E * 2, cf.cf_payload_bytes(S, False),
+                                                  launches_per_step=2)
         cf.cf_destroy(S); cf.cf_destroy(R)
         del acts, recs
     torch.cuda.empty_cache()
@@ -654,6 +714,97 @@ def run_lr_sweep(args, device, T=50, ef="implicit"):
                       "steps": T, "data": "synthetic"}), flush=True)
 
 
+# Sequence-parallel exchange: one token shard per rank of the FLUX-shaped activation
+# (4608 tokens over the pages' 4 GPUs: 1152 rows x 3072 channels bf16), the per-rank
+# shard fixed as ranks are added (weak scaling), several exchanged tensors per step.
+EXCHANGE = dict(rows=1152, cols=3072, tensors=4, mode="q2", kw={})
+
+
+def exchange_bench(ex, shards_at, steps, warmup, device, group=None):
+    """Time the exchange `ex` (an SPExchange) over `steps` steps after `warmup`
+    untimed ones; `shards_at(t)` gives the rank's shards of step t.  Two timed
+    passes on the same inputs: the exchange step itself, and the same codec
+    work with no collective (the rank's encodes and one decode per peer from
+    its own payload), so that exposed communication = step - codec work.
+    Times are the max over ranks (CUDA events on a GPU, wall clock on a CPU)."""
+    import torch
+    import torch.distributed as dist
+
+    cuda = torch.device(device).type == "cuda"
+
+    def clock(fn, n, t0):
+        if cuda:
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for t in range(t0, t0 + n):
+                fn(t)
+            b.record()
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b)
+        else:
+            t = time.perf_counter()
+            for k in range(t0, t0 + n):
+                fn(k)
+            ms = (time.perf_counter() - t) * 1e3
+        m = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(m, op=dist.ReduceOp.MAX, group=group)
+        return float(m[0]) / n
+
+    def codec_only(t):
+        for ch, a in zip(ex.channels, shards_at(t)):
+            P = ch.sender.payload_bytes(ch.sender.next_is_warm())
+            ch.sender.encode(a, ch.send_buf[:P], torch.cuda.current_stream() if cuda else None)
+            for p, rx in ch.receivers.items():
+                rx.decode(ch.send_buf[:P], ch.scratch_out, torch.cuda.current_stream() if cuda else None)
+
+    for t in range(warmup):
+        ex.step(shards_at(t))
+    step_ms = clock(lambda t: ex.step(shards_at(t)), steps, warmup)
+    st = ex.status()
+    # the codec-only pass runs fresh states (receivers fed by this rank's own payloads)
+    ex.reset()
+    for ch in ex.channels:
+        ch.scratch_out = torch.empty(ex.rows, ex.cols, dtype=ex.act_dtype, device=device)
+    for t in range(warmup):
+        codec_only(t)
+    codec_ms = clock(codec_only, steps, warmup)
+    ex.reset()
+    world = ex.world
+    act = len(ex.channels) * world * ex.rows * ex.cols * 2
+    return {"ms_per_step": round(step_ms, 5), "codec_ms_per_step": round(codec_ms, 5),
+            "exposed_comm_ms": round(max(step_ms - codec_ms, 0.0), 5),
+            "activation_gbs_per_rank": round(act / (step_ms / 1e3) / 1e9, 3),
+            "activation_gbs_all_ranks": round(world * act / (step_ms / 1e3) / 1e9, 3),
+            "payload_bytes_per_tensor": ex.channels[0].sender.payload_bytes(False),
+            "status": st}
+
+
+def run_exchange(args, rank, world, local):
+    """The payload exchange over NCCL on this node's GPUs (one rank per GPU)."""
+    import torch
+    import torch.distributed as dist
+
+    from activation_residual_compression_b200 import inputs
+    from activation_residual_compression_b200.exchange import SPExchange
+
+    X = EXCHANGE
+    streams = [inputs.flux("cuda", rows=X["rows"], cols=X["cols"], seed=11 + 100 * i + 1000 * rank)
+               for i in range(X["tensors"])]
+    n = args.warmup + args.steps
+    acts = [[s.next()[0] for _ in range(n)] for s in streams]
+    del streams
+    ex = SPExchange(X["rows"], X["cols"], X["mode"], n_tensors=X["tensors"], **X["kw"])
+    try:
+        res = exchange_bench(ex, lambda t: [a[t % n] for a in acts], args.steps, args.warmup, f"cuda:{local}")
+    finally:
+        ex.close()
+    res.update({"ranks": world, "transport": "nccl all_gather_into_tensor on a communication stream",
+                "shard": f"{X['rows']}x{X['cols']} bf16 per rank per tensor", "tensors": X["tensors"],
+                "mode": X["mode"], "scaling": "weak (fixed shard per rank)"})
+    return res
+
+
 def _oracle_kw(mode, kw):
     """The oracle's names for a codec's parameters."""
     if mode == "blocksel":
@@ -711,21 +862,30 @@ def run_bs_study(args, device, T=50):
                       "steps": T, "data": "synthetic"}), flush=True)
 
 
-def cpu_baseline(wl=None, max_seconds=20.0):
-    """The CPU oracle, as it stands, on the same workload (full-size tensors;
-    for the 60-tensor step the first tensors only, tensors being independent),
-    steps until max_seconds of oracle time (the warm-up step untimed)."""
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _oracle_leg(wl, max_seconds, max_steps=SEQ_STEPS):
+    """The CPU oracle, as it stands, on full-size tensors of a workload's stream
+    (for a many-tensor step its first tensor only: tensors are independent);
+    compressed steps until max_seconds of oracle time, at least one (the
+    leading full-size steps untimed).  Returns (activation GB/s, steps, seconds)."""
     import numpy as np
     import torch
 
     import oracle
-
-    wl = wl or WORKLOADS["flux"]
-    R_, C_, B_ = wl["rows"], wl["cols"], wl["batch"]
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    nt = 1 if B_ > 1 else B_
     from activation_residual_compression_b200 import inputs
 
+    R_, C_, B_ = wl["rows"], wl["cols"], wl["batch"]
     orcs = []
     for mi, (mode, kw) in enumerate(wl["codecs"]):
         if wl["stream"] == "cogvideox":   # the first tensor of the step (seed and sigma of layer 0)
@@ -733,26 +893,52 @@ def cpu_baseline(wl=None, max_seconds=20.0):
                                         sigma_per_tensor=inputs.cogvideox_sigmas(B_)[:1])
         else:
             s = _make_stream(wl["stream"], wl, seed=1 + 100 * mi, device="cpu")
-        o = oracle.Oracle(R_, C_, mode, dtype="bf16", batch=nt, **_oracle_kw(mode, kw))
+        o = oracle.Oracle(R_, C_, mode, dtype="bf16", batch=1, **_oracle_kw(mode, kw))
         for _ in range(kw.get("bs_warm", 1)):     # the full-size leading steps, untimed
             a = s.next().view(torch.int16).numpy().view(np.uint16)
             o.decode(o.encode(a))
         orcs.append((s, o))
     spent, steps = 0.0, 0
-    while spent < max_seconds and steps < 27:
+    while steps < 1 or (spent < max_seconds and steps < max_steps):
         ins = [s.next().view(torch.int16).numpy().view(np.uint16) for s, _ in orcs]
         t = time.perf_counter()
         for (s, o), a in zip(orcs, ins):
             o.decode(o.encode(a))
         spent += time.perf_counter() - t
         steps += 1
-    act_bytes = steps * len(orcs) * nt * R_ * C_ * 2
-    what = f"{steps} compressed steps of {nt} full {R_}x{C_} bf16 tensor(s)" + \
-        (f" (of the {B_}-tensor step)" if B_ > 1 else "")
-    return {"value": act_bytes / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{what}, modes {'+'.join(_codec_name(m, k) for m, k in wl['codecs'])} (encode+decode), "
-                      f"{spent:.1f} s of oracle time",
-            "ms_per_step": spent / steps * 1e3}
+    return steps * len(orcs) * R_ * C_ * 2 / spent / 1e9, steps, spent
+
+
+def cpu_baseline(wl=None, max_seconds=10.0, per_workload_seconds=4.0):
+    """The oracle timed on the host cores, as a baseline (not the target): the
+    timed workload with every core and with one thread, and a bounded sample of
+    each other workload (every core)."""
+    import oracle
+
+    wl = wl or WORKLOADS["flux"]
+    cores = oracle.set_threads(int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)))
+    val, steps, spent = _oracle_leg(wl, max_seconds)
+    oracle.set_threads(1)
+    val1, steps1, spent1 = _oracle_leg(wl, max_seconds)
+    oracle.set_threads(cores)
+    modes = "+".join(_codec_name(m, k) for m, k in wl["codecs"])
+    others = {}
+    for key in ("nm", "lowrank", "cogvideox", "blocksel"):
+        w = WORKLOADS[key]
+        if w["name"] == wl["name"]:
+            continue
+        v, n, t = _oracle_leg(w, per_workload_seconds)
+        others[w["name"]] = {"value": round(v, 5), "unit": "GB/s", "steps": n, "seconds": round(t, 2),
+                             "modes": "+".join(_codec_name(m, k) for m, k in w["codecs"]),
+                             **({"tensors_of_step": f"1 of {w['batch']}"} if w["batch"] > 1 else {})}
+    return {"value": round(val, 5), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{steps} compressed steps of one full {wl['rows']}x{wl['cols']} bf16 tensor"
+                      + (f" (of the {wl['batch']}-tensor step)" if wl["batch"] > 1 else "")
+                      + f", modes {modes} (encode+decode), {spent:.1f} s of oracle time",
+            "ms_per_step": round(spent / steps * 1e3, 2), "cpu_model": _cpu_model(),
+            "single_thread": {"value": round(val1, 5), "unit": "GB/s", "cores": 1, "steps": steps1,
+                              "seconds": round(spent1, 2)},
+            "other_workloads": others}
 
 
 def run_reference(args):
@@ -818,6 +1004,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cf", choices=["cf", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--sequences", type=int, default=5,
+                    help="full request sequences (27 compressed steps each) timed after the main region; 0: none")
     ap.add_argument("--max-resident", type=int, default=400, help="pre-generated inputs per mode (cycled)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-suite", action="store_true", help="skip the supplementary workloads")
@@ -833,6 +1021,8 @@ def main():
                     help="instead of timing: receiver error per step of every mode and feedback form")
     ap.add_argument("--lr-sweep", action="store_true",
                     help="instead of timing: low-rank receiver error over rank, sweeps and factor precision")
+    ap.add_argument("--exchange", action="store_true",
+                    help="also time the sequence-parallel payload exchange (always on with several GPUs)")
     ap.add_argument("--bs-study", action="store_true",
                     help="instead of timing: block-selection receiver error and step time over k/K")
     args = ap.parse_args()
@@ -904,6 +1094,7 @@ def main():
                                "activation_gbs": round(B_ * R_ * C_ * 2 / (step_ms / 1e3) / 1e9, 2),
                                "hbm_gbs": round(alg / (step_ms / 1e3) / 1e9, 1),
                                "roofline_frac": round(alg / (step_ms / 1e3) / 1e9 / peak, 4),
+                               "roofline_frac_datasheet": round(alg / (step_ms / 1e3) / 1e9 / DATASHEET_GBS, 4),
                                "payload_bytes": c["P"],
                                "ratio_vs_bf16": round(B_ * R_ * C_ * 2 / c["P"], 2)}
     in_mb = B_ * R_ * C_ * 2 / 1e6
@@ -919,15 +1110,50 @@ def main():
         "roofline": {"bound": "hbm", "kernel": kern, "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": (tr["bytes_per_launch"] if tr else None),
-                     "algorithmic_bytes": enc_alg, "peak_source": peak_kind},
+                     "algorithmic_bytes": enc_alg, "peak_source": peak_kind,
+                     "datasheet_peak": DATASHEET_GBS, "frac_of_datasheet": round(achieved / DATASHEET_GBS, 4)},
         "gpu_launches": sum(launches_per_call(c["mode"], c["kw"], True) + launches_per_call(c["mode"], c["kw"], False)
                             for c in st["codecs"]) * args.steps,
         "clocks": st["clocks"],
     }
+    if st["seq"]:
+        sq = st["seq"]
+        med = statistics.median(sq["step_ms"])
+        line["sequences"] = {
+            "n": sq["n"], "compressed_steps_each": sq["steps"],
+            "what": "each a new request (states reset, warm-up step untimed); per sequence the mean "
+                    "encode+decode time per step over all codecs",
+            "ms_per_step_median": round(med, 5), "ms_per_step_min": round(min(sq["step_ms"]), 5),
+            "ms_per_step_max": round(max(sq["step_ms"]), 5),
+            "activation_gbs_median": round(n_codecs * B_ * R_ * C_ * 2 / (med / 1e3) / 1e9, 2),
+            "per_mode_ms_median": {m: round(statistics.median(v), 5) for m, v in sq["per"].items()},
+            "per_mode_roofline_frac_median": {
+                c["name"]: round(B_ * step_bytes(c["mode"], R_, C_, c["kw"], c["P"], ef=args.ef,
+                                                 state_size=2 if args.state == "bf16" else 4)
+                                 / (statistics.median(sq["per"][c["name"]]) / 1e3) / 1e9 / peak, 4)
+                for c in st["codecs"]}}
     if e2e_ms:
         line["e2e"] = {"value": round(act_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                        "h2d_bytes_per_step": st["e2e"]["h2d"], "d2h_bytes_per_step": st["e2e"]["d2h"],
                        "ms_per_step": round(e2e_ms, 4)}
+    if args.exchange or world > 1:
+        own_group = dist is None
+        if own_group:   # a one-rank NCCL group for the exchange on this GPU
+            import datetime
+            import socket
+
+            import torch.distributed as dist
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                port = sk.getsockname()[1]
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ["MASTER_PORT"] = str(port)
+            dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        line["exchange"] = run_exchange(args, rank, world, local)
+        if own_group:
+            dist.destroy_process_group()
+            dist = None
     if world == 1 and not args.no_suite and args.workload == "flux" and args.ef == "explicit" and args.state == "f32":
         line["suite"] = run_suite(args, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -50,6 +50,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_IDENTITY 0
 #define ORC_SIGN1 1
@@ -315,6 +318,21 @@ void orc_destroy(orc_state *o)
 
 uint64_t orc_step(const orc_state *o, int receiver) { return receiver ? o->step_r : o->step_s; }
 int orc_status(const orc_state *o) { return o->status; }
+
+/* Threads of the row-parallel loops for the calling thread's later calls
+ * (timing only: every parallel loop writes disjoint rows, so the results do
+ * not depend on it).  Returns the thread count now in effect. */
+int orc_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
 
 /* which: 0 ahat_S, 1 e, 2 ahat_R, 3 V_prev.  Copies the whole batch. */
 float *orc_buffer(orc_state *o, int which)
