@@ -18,6 +18,9 @@ CogVideoX-2b finding):
                an i.i.d. (high-rank) Gaussian innovation
 * cogvideox -- 60 tensors (30 layers x 2) of 17550 x 1920 bf16, per-tensor
                residual ratio drawn U[0.05, 0.2]
+* lowrank_walk -- a random walk whose innovation is dominated by a fixed
+               rank-k structure with a decaying spectrum, plus a small i.i.d.
+               part: a residual whose leading subspace is well separated
 
 Rows are tokens, columns are channels (the hidden dimension).  The walk state
 is kept in fp32 and cast to the stream dtype each step.
@@ -28,7 +31,7 @@ import math
 
 import torch
 
-__all__ = ["ActivationStream", "tiny", "flux", "ar1", "cogvideox"]
+__all__ = ["ActivationStream", "LowRankWalk", "tiny", "flux", "ar1", "cogvideox", "lowrank_walk"]
 
 
 class ActivationStream:
@@ -112,6 +115,43 @@ def blocksel(device="cpu", H=64, W=64, cols=3072, block=8, seed=4):
     """Token-grid stream for the block-selection mode: 64 x 64 tokens x 3072
     channels bf16, per-8x8-block innovation scales log-uniform in [0.01, 0.3]."""
     return BlockStream(H, W, cols, block=block, device=device, seed=seed)
+
+
+class LowRankWalk(ActivationStream):
+    """a_0 ~ N(0,1); a_t = a_{t-1} + U diag(s z_t) W^T + noise N(0,1), with fixed
+    Gaussian factors U (rows x k) and W (cols x k) scaled by 1/sqrt(rows) and
+    1/sqrt(cols), per-step random signs z_t in {-1, +1}^k and weights
+    s_i = amp decay^i: the innovation's spectrum decays, every direction is
+    present at every step, and its leading subspace stays put, unlike the
+    i.i.d. innovation of the AR(1) stream."""
+
+    def __init__(self, rows, cols, *, rank=70, amp=20.0, decay=0.96, noise=1e-3, dtype=torch.bfloat16,
+                 device="cpu", seed=0):
+        super().__init__(rows, cols, dtype=dtype, device=device, seed=seed, sigma=noise, seed_per_tensor=[seed])
+        g = torch.Generator().manual_seed(int(seed) + 1)
+        self.U = (torch.randn(rows, rank, generator=g) / math.sqrt(rows)).to(self.device)
+        self.W = (torch.randn(cols, rank, generator=g) / math.sqrt(cols)).to(self.device)
+        self.s = (amp * decay ** torch.arange(rank, dtype=torch.float32)).to(self.device)
+        self.zgen = torch.Generator().manual_seed(int(seed) + 2)
+
+    def next(self, out: torch.Tensor | None = None) -> torch.Tensor:
+        z = self._normal(0)
+        if self.t == 0:
+            self.state[0] = z
+        else:
+            sg = torch.randint(0, 2, (self.U.shape[1],), generator=self.zgen).to(torch.float32) * 2 - 1
+            c = sg.to(self.device) * self.s
+            self.state[0].add_(z * self.sigmas[0]).add_((self.U * c) @ self.W.T)
+        self.t += 1
+        if out is None:
+            return self.state.to(self.dtype, copy=True)
+        out.copy_(self.state)
+        return out
+
+
+def lowrank_walk(device="cpu", rows=1024, cols=768, seed=5, **kw):
+    """Random walk with a well-separated low-rank innovation (see LowRankWalk)."""
+    return LowRankWalk(rows, cols, device=device, seed=seed, **kw)
 
 
 def tiny(device="cpu"):
