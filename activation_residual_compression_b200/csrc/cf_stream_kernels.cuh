@@ -35,8 +35,8 @@
 
 // Resident blocks per SM the compiler must allow (register budget), measured
 // on B200: the decode kernels take 4 for N:M with two kept values per block
-// and 3 otherwise; the encode kernels take 3 for the 2-bit mode and for up to
-// two vectors per thread, else 2 (EncMinBlocks below).
+// and 3 otherwise; the encode kernels take 3 for the 1-bit and 2-bit modes and
+// for up to two vectors per thread, else 2 (EncMinBlocks below).
 
 namespace cfi {
 namespace {
@@ -370,13 +370,14 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
   }
 
   // ---- encode; c[j][k] = C(D) from the encoded values ----
-  // C(D) for the state update below.  The 2-bit and N:M modes rebuild it
-  // there from compact per-vector data (the 2-bit codes and two levels; the
-  // kept mask) rather than holding VPT x 8 floats; the 1-bit mode keeps its
-  // +-S values (measured faster for it on B200).
+  // C(D) for the state update below, rebuilt there from compact data rather
+  // than held as VPT x 8 floats: the 1-bit value from the sign of D and the
+  // scale, the 2-bit value from its code and two levels, the N:M value from
+  // the kept mask (fewer live registers: the 1-bit encode fits the budget of
+  // three resident blocks per SM).
   float cL2 = 0.0f, cL3 = 0.0f;
   uint32_t cinfo[VPT];
-  float cs1[MODE == M_S1 ? VPT : 1][8];
+  float cS1 = 0.0f;
 #pragma unroll
   for (int j = 0; j < VPT; j++) cinfo[j] = 0;
   uint32_t cbits[VPT];
@@ -426,6 +427,7 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
       Sc = __uint_as_float((uint32_t)sbits << 16);
     }
     if (row_ok && t == 0) reinterpret_cast<uint16_t *>(body)[r] = sbits;
+    cS1 = Sc;
 #pragma unroll
     for (int j = 0; j < VPT; j++) {
       uint32_t byte = 0;
@@ -433,7 +435,6 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
       for (int k = 0; k < 8; k++) {
         const bool neg = d[j][k] < 0.0f;
         byte |= (uint32_t)neg << k;
-        cs1[j][k] = neg ? -Sc : Sc;
       }
       const int v = t + (j << tlog);
       cbits[j] = byte << ((v % P::G) * P::bpv);
@@ -606,7 +607,7 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
 #pragma unroll
       for (int k = 0; k < 8; k++) {
         if constexpr (MODE == M_ID) c[k] = d[j][k];
-        else if constexpr (MODE == M_S1) c[k] = cs1[j][k];
+        else if constexpr (MODE == M_S1) c[k] = d[j][k] < 0.0f ? -cS1 : cS1;
         else if constexpr (MODE == M_Q2) c[k] = q2_level((float)((cinfo[j] >> (2 * k)) & 3u), cL2, cL3);
         else c[k] = ((cinfo[j] >> k) & 1u) ? __bfloat162float(__float2bfloat16_rn(d[j][k])) : 0.0f;
       }
@@ -625,7 +626,7 @@ __device__ __forceinline__ void encode_row(const EncArgs &A, const int t, const 
 // Register path: each thread loads its vectors straight from global memory.
 template <int MODE, int VPT>
 struct EncMinBlocks {
-  static constexpr int value = (MODE == CF_Q2 || VPT <= 2) ? 3 : 2;
+  static constexpr int value = (MODE == CF_Q2 || MODE == CF_SIGN1 || VPT <= 2) ? 3 : 2;
 };
 
 template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename Tab, typename S = float>
