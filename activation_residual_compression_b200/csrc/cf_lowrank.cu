@@ -90,39 +90,35 @@ __device__ __forceinline__ float v0_entry(uint64_t seed, int64_t j, int r, int k
 
 // Vt (split bf16, [rp][cols]) from the warm start: the previous step's V
 // (fp32 [cols][r]), or V0 on the first step and for any all-zero column.
-constexpr int kVprepThreads = 1024;
-constexpr int kVprepPer = 8;
-static_assert(kVprepThreads * kVprepPer >= kMaxCols, "one vprep block holds a whole column");
-__global__ void __launch_bounds__(kVprepThreads) lr_vprep_kernel(const float *vprev, int64_t cols, int r, int rp,
-                                                                 int first, uint64_t seed, __nv_bfloat16 *vthi,
-                                                                 __nv_bfloat16 *vtlo, unsigned *amax) {
-  pdl_enter();
-  const int k = blockIdx.x;
+// One 256-thread block per column k of the rp padded ones (the leading
+// blocks of the residual kernel's grid, so the two run as one launch).  The
+// column is read twice (the zero test, then the values, from cache) so that
+// these blocks hold no more registers than the residual tiles.
+struct VprepArgs {
+  const float *vprev;
+  int64_t cols;
+  int r, rp, first;
+  uint64_t seed;
+  __nv_bfloat16 *vthi, *vtlo;
+  unsigned *amax;
+};
+__device__ __forceinline__ void vprep_column(const VprepArgs &V, int k) {
   if (threadIdx.x == 0) {  // this encode's column maxima start from zero
-    amax[k] = 0u;
-    amax[rp + k] = 0u;
+    V.amax[k] = 0u;
+    V.amax[V.rp + k] = 0u;
   }
-  float x[kVprepPer];
   int nz = 0;
-#pragma unroll
-  for (int t = 0; t < kVprepPer; t++) {
-    const int64_t j = threadIdx.x + (int64_t)t * kVprepThreads;
-    x[t] = (k < r && !first && j < cols) ? vprev[j * r + k] : 0.0f;
-    nz |= x[t] != 0.0f;
-  }
+  if (k < V.r && !V.first)
+    for (int64_t j = threadIdx.x; j < V.cols; j += 256) nz |= V.vprev[j * V.r + k] != 0.0f;
   // a column of V_prev that is entirely zero (a dead direction) restarts from V0
   const bool use_prev = __syncthreads_or(nz) != 0;
-#pragma unroll
-  for (int t = 0; t < kVprepPer; t++) {
-    const int64_t j = threadIdx.x + (int64_t)t * kVprepThreads;
-    if (j < cols) {
-      float v = 0.0f;
-      if (k < r) v = use_prev ? x[t] : v0_entry(seed, j, r, k);
-      __nv_bfloat16 hi, lo;
-      split_bf16(v, hi, lo);
-      vthi[(int64_t)k * cols + j] = hi;
-      vtlo[(int64_t)k * cols + j] = lo;
-    }
+  for (int64_t j = threadIdx.x; j < V.cols; j += 256) {
+    float v = 0.0f;
+    if (k < V.r) v = use_prev ? V.vprev[j * V.r + k] : v0_entry(V.seed, j, V.r, k);
+    __nv_bfloat16 hi, lo;
+    split_bf16(v, hi, lo);
+    V.vthi[(int64_t)k * V.cols + j] = hi;
+    V.vtlo[(int64_t)k * V.cols + j] = lo;
   }
 }
 
@@ -130,16 +126,22 @@ __global__ void __launch_bounds__(kVprepThreads) lr_vprep_kernel(const float *vp
 
 // D = (a - ahat) + e split in two bf16 terms, row-major ([rows][cols]): the
 // K-major A operand of Y = D V and the MN-major A operand of V = D^T Q.  A
-// block covers 64 rows x 64 columns (4 per thread per row pass).  The inputs
+// block covers 64 rows x 64 columns (4 per thread per row pass); the grid's
+// first rp blocks prepare the warm start instead (vprep_column).  The inputs
 // are read once (evict-first loads), so the split, which both products read
 // next, is more likely to stay in L2.  The fp32 D is not stored: the
 // reconstruction pass recomputes it bit for bit.
 template <typename T>
-__global__ void __launch_bounds__(256) lr_delta_kernel(const T *a, const float *ahat, const float *err, int ef_explicit,
+__global__ void __launch_bounds__(256, 8) lr_delta_kernel(const T *a, const float *ahat, const float *err, int ef_explicit,
                                                        int64_t rows, int64_t cols, __nv_bfloat16 *dhi,
-                                                       __nv_bfloat16 *dlo) {
+                                                       __nv_bfloat16 *dlo, const VprepArgs V) {
   pdl_enter();
-  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+  if ((int)blockIdx.x < V.rp) {  // uniform over the block
+    vprep_column(V, (int)blockIdx.x);
+    return;
+  }
+  const int tile = (int)blockIdx.x - V.rp, tiles_x = (int)(cols / 64);
+  const int64_t r0 = (int64_t)(tile / tiles_x) * 64, c0 = (int64_t)(tile % tiles_x) * 64;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll
   for (int i = 0; i < 4; i++) {
@@ -444,8 +446,10 @@ __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc
 // zero).  A block covers 32 consecutive entries, one per lane; its 8 warps sum
 // 8 contiguous slices of the partials, and the slice sums are added in slice
 // order, so the result does not depend on scheduling.
-__global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart, int nblk, int n, double *G) {
+__global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart, int nblk, int n, double *G,
+                                                              const int *skip2) {
   pdl_enter();
+  if (skip2 != nullptr && *skip2) return;  // second pass not needed (uniform over the grid)
   __shared__ double part[8][32];
   const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
   const int nn = n * n;
@@ -579,12 +583,24 @@ __device__ __forceinline__ void chol_diag(const double *Ab, double *Xb, int b, i
 //
 // Columns nlive .. n-1 must be zero in G (the padding of the rank).  G and M
 // may alias (G is read before the first barrier).
+//
+// First pass of a sweep (first_pass): the elimination also bounds the
+// condition number of X (the matrix being orthonormalised) by B =
+// ||L||_F ||L^-1||_F >= kappa_2(L) = kappa_2(X), with ||L||_F^2 the trace of G
+// over the live columns, and sets *skip2 when B^2 <= kappa2_max (0: never).
+// Then Q1 = X L^-T is orthonormal to within about n kappa^2 2^-53 per entry
+// (the fp64 Gram matrix and elimination), far below the fp32 rounding of the
+// stored Q (2^-24), and the second pass is skipped: its kernels return at
+// once (second pass: !first_pass, *skip2 set).
 template <int TT>
 __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double *Mout, int *dead, double near_id,
-                                                         int nlive) {
+                                                         int nlive, int *skip2, int first_pass, double kappa2_max) {
   pdl_enter();
+  if (!first_pass && *skip2) return;  // uniform over the block
   constexpr int n = 16 * TT;
   __shared__ int dead_s[n];
+  __shared__ double gdiag[n];
+  __shared__ double red[8];
   extern __shared__ __align__(16) uint8_t csm[];
   if (near_id > 0.0) {
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
@@ -634,15 +650,29 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double
   const int nbl = (min(max(nlive, 0), n) + 7) / 8;
   const int nl = 8 * nbl;
   const double thr = 1e-12 * G[0];
-  for (int e = threadIdx.x; e < nl * nl; e += blockDim.x) {
-    const int gi = e / nl, gj = e % nl;
-    if ((gj >> 3) <= (gi >> 3)) {
-      const int o = chol_tile(gi >> 3, gj >> 3) + (gi & 7) * kCholTld + (gj & 7);
-      A[o] = gj <= gi ? G[gi * n + gj] : 0.0;
-      X[o] = 0.0;
+  // the working matrix from G: eight loads in flight per thread before the
+  // stores into the tiles
+  for (int e0 = 0; e0 < nl * nl; e0 += 8 * 256) {
+    double g[8];
+#pragma unroll
+    for (int u = 0; u < 8; u++) {
+      const int e = e0 + u * 256 + (int)threadIdx.x;
+      const int gi = e / nl, gj = e - (e / nl) * nl;
+      g[u] = (e < nl * nl && gj <= gi) ? G[gi * n + gj] : 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; u++) {
+      const int e = e0 + u * 256 + (int)threadIdx.x;
+      const int gi = e / nl, gj = e - (e / nl) * nl;
+      if (e < nl * nl && (gj >> 3) <= (gi >> 3)) {
+        const int o = chol_tile(gi >> 3, gj >> 3) + (gi & 7) * kCholTld + (gj & 7);
+        A[o] = g[u];
+        X[o] = 0.0;
+      }
     }
   }
   for (int k = nl + threadIdx.x; k < n; k += blockDim.x) dead_s[k] = 1;
+  for (int k = threadIdx.x; k < nl; k += blockDim.x) gdiag[k] = G[k * n + k];
   __syncthreads();
   if (nbl > 0 && warp == 0) chol_diag(A, X, 0, nlive, thr, lane, dead_s);
   __syncthreads();
@@ -709,15 +739,37 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double
     __syncthreads();
   }
   // M[gj][gi] = X[gi][gj]
+  double sx = 0.0;  // this thread's part of ||X||_F^2
   for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
     const int gj = e / n, gi = e % n;
-    Mout[e] = (gi < nl && gj <= gi) ? X[chol_tile(gi >> 3, gj >> 3) + (gi & 7) * kCholTld + (gj & 7)] : 0.0;
+    const double xv = (gi < nl && gj <= gi) ? X[chol_tile(gi >> 3, gj >> 3) + (gi & 7) * kCholTld + (gj & 7)] : 0.0;
+    Mout[e] = xv;
+    sx = fma(xv, xv, sx);
   }
   for (int e = threadIdx.x; e < n; e += blockDim.x) dead[e] = dead_s[e];
+  if (first_pass) {  // uniform over the block
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, o);
+    if (lane == 0) red[warp] = sx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double xs2 = 0.0, tr = 0.0;
+      for (int w = 0; w < 8; w++) xs2 += red[w];
+      for (int k = 0; k < nl; k++)
+        if (!dead_s[k]) tr += gdiag[k];
+      *skip2 = (kappa2_max > 0.0 && tr * xs2 <= kappa2_max) ? 1 : 0;
+    }
+  }
 }
 
 // Rows per apply block.
 constexpr int kApplyRows = 16;
+
+// The second CholeskyQR pass of a sweep is skipped when the first pass bounds
+// the condition number of the matrix it orthonormalises by this (see
+// lr_chol_kernel): its orthogonality error is then about n kSkipKappa^2 2^-53
+// <= 2^-30 per entry for n <= 128, against the 2^-24 of the stored fp32 Q.
+constexpr double kSkipKappa = 256.0;
 template <int TT>
 __host__ __device__ constexpr int apply_xld() {
   return 16 * TT + 4;  // X tile row stride (floats): 4 or 20 mod 32, a fragment's 8 rows x 4 in distinct banks
@@ -792,25 +844,21 @@ __device__ __forceinline__ void apply_tiles(const float *xs, const double *Ms, i
 // through shared memory so that those stores are row-contiguous; when amax !=
 // nullptr, the absmax of each of Q's first r columns (the INT4 scales'
 // input) goes to amax, one atomicMax per column and block.
-template <int TT>
-__global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const double *M, int64_t rows, float *q,
-                                                       __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo, int r,
-                                                       unsigned *amax) {
-  pdl_enter();
-  __shared__ unsigned cmax[16 * TT];
-  constexpr int n = 16 * TT, mld = apply_mld<TT>(), qld = kApplyRows + 1, RT = kApplyRows / 8;
-  constexpr int JR = apply_rounds<TT>();
-  extern __shared__ __align__(16) uint8_t asm_[];
-  double *Ms = reinterpret_cast<double *>(asm_);        // [n][mld]
-  float *xs = reinterpret_cast<float *>(Ms + n * mld);  // [kApplyRows][xld]; reused as Q^T [n][qld]
-  const int64_t r0 = (int64_t)blockIdx.x * kApplyRows;
-  apply_stage<TT>(x, M, rows, r0, kApplyRows, Ms, xs);
-  if (amax != nullptr)
-    for (int c = threadIdx.x; c < n; c += 256) cmax[c] = 0u;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t4 = lane & 3;
-  double acc[JR][RT][2];
-  apply_tiles<TT, RT>(xs, Ms, warp, lane, acc);
+// The outputs of Q = X M for the 8 RT rows of one block from r0, from the
+// accumulators of apply_tiles: Q fp32 [rows][n]; when amax != nullptr the
+// absmax of each of Q's first r columns (the INT4 scales' input), one
+// atomicMax per column and block (cmax: n entries of shared memory, zeroed
+// before the block's last barrier); when qthi != nullptr Q^T split in bf16
+// ([n][rows], the K-major B operand of V = D^T Q), transposed through qs
+// (shared, n x (8 RT + 1) floats, free once every thread has passed the
+// first barrier here) so that those stores are row-contiguous.  Every thread
+// of the block calls this (amax and qthi are uniform).
+template <int TT, int RT>
+__device__ __forceinline__ void apply_store(const double (&acc)[apply_rounds<TT>()][RT][2], int64_t r0, int64_t rows,
+                                            float *q, __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo, int r,
+                                            unsigned *amax, unsigned *cmax, float *qs, int warp, int lane) {
+  constexpr int n = 16 * TT, NR = 8 * RT, qld = NR + 1, JR = apply_rounds<TT>();
+  const int gq = lane >> 2, t4 = lane & 3;
   float res[JR][RT][2];
 #pragma unroll
   for (int jt = 0; jt < JR; jt++) {
@@ -830,14 +878,12 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
       }
     }
   }
+  __syncthreads();  // the column maxima are complete, and every thread is done with the buffer under qs
   if (amax != nullptr) {  // uniform over the block
-    __syncthreads();
     for (int c = threadIdx.x; c < r; c += 256)
       if (cmax[c]) atomicMax(&amax[c], cmax[c]);
   }
   if (qthi == nullptr) return;  // uniform over the block
-  __syncthreads();              // every thread is done with xs
-  float *qs = xs;               // Q^T tile [n][qld]
 #pragma unroll
   for (int jt = 0; jt < JR; jt++) {
     const int J = apply_ctile<TT>(warp, jt);
@@ -850,8 +896,8 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
     }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < n * kApplyRows; e += 256) {
-    const int c = e / kApplyRows, rr = e % kApplyRows;
+  for (int e = threadIdx.x; e < n * NR; e += 256) {
+    const int c = e / NR, rr = e % NR;
     if (r0 + rr < rows) {
       __nv_bfloat16 hi, lo;
       split_bf16(qs[c * qld + rr], hi, lo);
@@ -861,25 +907,69 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
   }
 }
 
+// Q = X M (M = L^-T, upper triangular, zero below the diagonal) for
+// kApplyRows rows per block (apply_tiles; M and the rows of X staged in
+// shared memory), with the stores of apply_store.  The second CholeskyQR
+// pass of a sweep whose first pass was accurate enough (*skip2 set by the
+// first pass's factor kernel) has nothing to do: that pass's apply already
+// wrote these outputs.
+template <int TT>
+__global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const double *M, int64_t rows, float *q,
+                                                       __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo, int r,
+                                                       unsigned *amax, const int *skip2) {
+  pdl_enter();
+  if (skip2 != nullptr && *skip2) return;  // uniform over the grid
+  __shared__ unsigned cmax[16 * TT];
+  constexpr int n = 16 * TT, mld = apply_mld<TT>(), RT = kApplyRows / 8;
+  constexpr int JR = apply_rounds<TT>();
+  extern __shared__ __align__(16) uint8_t asm_[];
+  double *Ms = reinterpret_cast<double *>(asm_);        // [n][mld]
+  float *xs = reinterpret_cast<float *>(Ms + n * mld);  // [kApplyRows][xld]; reused as Q^T [n][kApplyRows + 1]
+  const int64_t r0 = (int64_t)blockIdx.x * kApplyRows;
+  apply_stage<TT>(x, M, rows, r0, kApplyRows, Ms, xs);
+  if (amax != nullptr)
+    for (int c = threadIdx.x; c < n; c += 256) cmax[c] = 0u;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  double acc[JR][RT][2];
+  apply_tiles<TT, RT>(xs, Ms, warp, lane, acc);
+  apply_store<TT, RT>(acc, r0, rows, q, qthi, qtlo, r, amax, cmax, xs, warp, lane);
+}
+
 // The first CholeskyQR pass's Q1 = X M for kGramRows rows per block, with the
 // sums of lr_apply_kernel (apply_tiles), and the partial Gram matrix Q1^T Q1
 // of these rows from the fp32 values it stores, with the sums of
 // lr_gram_kernel (gram_tiles): the second pass needs no Gram kernel, and both
-// results are bit-identical to the separate kernels'.
+// results are bit-identical to the separate kernels'.  When the first pass's
+// factor kernel found the pass accurate enough (*skip2), Q1 is the sweep's Q:
+// the block writes the final pass's outputs instead (apply_store: Q, its
+// INT4 column maxima when amax != nullptr, Q^T split) and no Gram matrix.
 template <int TT>
 __global__ void __launch_bounds__(256) lr_apply_gram_kernel(const float *x, const double *M, int64_t rows, float *q,
-                                                            double *gpart) {
+                                                            double *gpart, const int *skip2, __nv_bfloat16 *qthi,
+                                                            __nv_bfloat16 *qtlo, int r, unsigned *amax) {
   pdl_enter();
+  __shared__ unsigned cmax[16 * TT];
   constexpr int n = 16 * TT, mld = apply_mld<TT>(), xld = apply_xld<TT>(), RT = kGramRows / 8;
   constexpr int JR = apply_rounds<TT>();
+  static_assert(kGramRows * xld >= n * (kGramRows + 1), "the X tile holds the transposed Q tile");
   extern __shared__ __align__(16) uint8_t asm_[];
   double *Ms = reinterpret_cast<double *>(asm_);        // [n][mld]
   float *xs = reinterpret_cast<float *>(Ms + n * mld);  // [kGramRows][xld]
   float *gs = xs + kGramRows * xld;                     // Q1 [kGramRows][gram_ld]
   const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
+  const bool final_q = *skip2 != 0;                     // uniform over the grid
   apply_stage<TT>(x, M, rows, r0, kGramRows, Ms, xs);
+  if (final_q && amax != nullptr)
+    for (int c = threadIdx.x; c < n; c += 256) cmax[c] = 0u;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t4 = lane & 3;
+  if (final_q) {
+    double acc[JR][RT][2];
+    apply_tiles<TT, RT>(xs, Ms, warp, lane, acc);
+    apply_store<TT, RT>(acc, r0, rows, q, qthi, qtlo, r, amax, cmax, xs, warp, lane);
+    return;
+  }
   {
     double acc[JR][RT][2];
     apply_tiles<TT, RT>(xs, Ms, warp, lane, acc);
@@ -955,7 +1045,7 @@ struct PackArgs {
   int r, n, int4;
   int64_t sec1, sec2, body;
   Header hdr;
-  unsigned *amax;  // [2 n]: column absmax bit patterns of Q, then of V (zeroed by lr_vprep_kernel)
+  unsigned *amax;  // [2 n]: column absmax bit patterns of Q, then of V (zeroed by vprep_column)
   // the sender's reconstruction operands, written from the packed values (the
   // dequantisation of the payload, see lr_dequant_kernel); k >= r stays zero
   int kp;
@@ -1455,7 +1545,7 @@ void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *p
   enc += pad256((size_t)plan->sv * C * rp * 4);               // vpart
   enc += pad256(mx * rp * 4) * 2 + pad256(C * rp * 4);        // xbuf, q, v
   enc += pad256((size_t)plan->nblk_gram * rp * rp * 8);       // gpart
-  enc += pad256(rp * rp * 8) + pad256(rp * 4);                // L, dead
+  enc += pad256(rp * rp * 8) + pad256(rp * 4) + pad256(4);    // L, dead, skip flag
   enc += pad256(2 * rp * 4);                                  // amax
   plan->enc_scratch_bytes = enc;
   plan->dec_scratch_bytes = dec;
@@ -1521,6 +1611,7 @@ int lowrank_bind(LowrankPlan *plan, void *scratch) {
     b.gpart = reinterpret_cast<double *>(take((size_t)plan->nblk_gram * rp * rp * 8));
     b.L = reinterpret_cast<double *>(take(rp * rp * 8));
     b.dead = reinterpret_cast<int *>(take(rp * 4));
+    b.skip2 = reinterpret_cast<int *>(take(4));
     b.amax = reinterpret_cast<unsigned *>(take(2 * rp * 4));
     ok = ok && make_map(&plan->tm_dhi, b.dhi, C, R, kTileM) && make_map(&plan->tm_dlo, b.dlo, C, R, kTileM) &&
          make_map(&plan->tm_vthi, b.vthi, C, rp, (uint32_t)rp) && make_map(&plan->tm_vtlo, b.vtlo, C, rp, (uint32_t)rp) &&
@@ -1573,52 +1664,54 @@ cudaError_t launch_gram(int n, int nblk, const float *src, int nsrc, int64_t row
   return cudaGetLastError();
 }
 
-cudaError_t launch_chol(int n, double *L, int *dead, double near_id, int nlive, cudaStream_t st) {
+cudaError_t launch_chol(int n, double *L, int *dead, double near_id, int nlive, int *skip2, int first_pass,
+                        double kappa2_max, cudaStream_t st) {
   switch (n / 16) {
-    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), chol_smem_tt(1), st, L, L, dead, near_id, nlive); break;
-    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), chol_smem_tt(2), st, L, L, dead, near_id, nlive); break;
-    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), chol_smem_tt(3), st, L, L, dead, near_id, nlive); break;
-    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), chol_smem_tt(4), st, L, L, dead, near_id, nlive); break;
-    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), chol_smem_tt(5), st, L, L, dead, near_id, nlive); break;
-    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), chol_smem_tt(6), st, L, L, dead, near_id, nlive); break;
-    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), chol_smem_tt(7), st, L, L, dead, near_id, nlive); break;
-    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), chol_smem_tt(8), st, L, L, dead, near_id, nlive); break;
+    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), chol_smem_tt(1), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), chol_smem_tt(2), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), chol_smem_tt(3), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), chol_smem_tt(4), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), chol_smem_tt(5), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), chol_smem_tt(6), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), chol_smem_tt(7), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), chol_smem_tt(8), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_apply(int n, const float *x, const double *M, int64_t rows, float *q, __nv_bfloat16 *qthi,
-                         __nv_bfloat16 *qtlo, int r, unsigned *amax, cudaStream_t st) {
+                         __nv_bfloat16 *qtlo, int r, unsigned *amax, const int *skip2, cudaStream_t st) {
   const unsigned grid = (unsigned)((rows + kApplyRows - 1) / kApplyRows);
   const size_t sm = apply_smem(n);
   switch (n / 16) {
-    case 1: launch_pdl(lr_apply_kernel<1>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
-    case 2: launch_pdl(lr_apply_kernel<2>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
-    case 3: launch_pdl(lr_apply_kernel<3>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
-    case 4: launch_pdl(lr_apply_kernel<4>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
-    case 5: launch_pdl(lr_apply_kernel<5>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
-    case 6: launch_pdl(lr_apply_kernel<6>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
-    case 7: launch_pdl(lr_apply_kernel<7>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
-    case 8: launch_pdl(lr_apply_kernel<8>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax); break;
+    case 1: launch_pdl(lr_apply_kernel<1>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
+    case 2: launch_pdl(lr_apply_kernel<2>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
+    case 3: launch_pdl(lr_apply_kernel<3>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
+    case 4: launch_pdl(lr_apply_kernel<4>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
+    case 5: launch_pdl(lr_apply_kernel<5>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
+    case 6: launch_pdl(lr_apply_kernel<6>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
+    case 7: launch_pdl(lr_apply_kernel<7>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
+    case 8: launch_pdl(lr_apply_kernel<8>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_apply_gram(int n, const float *x, const double *M, int64_t rows, float *q, double *gpart,
+                              const int *skip2, __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo, int r, unsigned *amax,
                               cudaStream_t st) {
   const unsigned grid = (unsigned)(rows / kGramRows);
   const size_t sm = apply_gram_smem(n);
   switch (n / 16) {
-    case 1: launch_pdl(lr_apply_gram_kernel<1>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
-    case 2: launch_pdl(lr_apply_gram_kernel<2>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
-    case 3: launch_pdl(lr_apply_gram_kernel<3>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
-    case 4: launch_pdl(lr_apply_gram_kernel<4>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
-    case 5: launch_pdl(lr_apply_gram_kernel<5>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
-    case 6: launch_pdl(lr_apply_gram_kernel<6>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
-    case 7: launch_pdl(lr_apply_gram_kernel<7>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
-    case 8: launch_pdl(lr_apply_gram_kernel<8>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart); break;
+    case 1: launch_pdl(lr_apply_gram_kernel<1>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
+    case 2: launch_pdl(lr_apply_gram_kernel<2>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
+    case 3: launch_pdl(lr_apply_gram_kernel<3>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
+    case 4: launch_pdl(lr_apply_gram_kernel<4>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
+    case 5: launch_pdl(lr_apply_gram_kernel<5>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
+    case 6: launch_pdl(lr_apply_gram_kernel<6>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
+    case 7: launch_pdl(lr_apply_gram_kernel<7>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
+    case 8: launch_pdl(lr_apply_gram_kernel<8>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -1634,12 +1727,15 @@ cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int
   // split-K partials of Y), the second pass's from the first pass's apply
   if (!final_pass && (e = launch_gram(n, nblk, src, nsrc, rows, b.xbuf, b.gpart, st)) != cudaSuccess) return e;
   // the reduced Gram matrix goes to L, which the Cholesky kernel then
-  // overwrites with M = L^-T
-  launch_pdl(lr_gram_reduce_kernel, dim3((unsigned)((n * n + 31) / 32)), dim3(256), 0, st, b.gpart, nblk, n, b.L);
-  e = launch_chol(n, b.L, b.dead, final_pass ? P.qr2_tol : 0.0, P.rank, st);
+  // overwrites with M = L^-T; the first pass decides whether the second one
+  // runs (lr_qr2_tol = 0: always, the full CholeskyQR2)
+  launch_pdl(lr_gram_reduce_kernel, dim3((unsigned)((n * n + 31) / 32)), dim3(256), 0, st, b.gpart, nblk, n, b.L,
+             final_pass ? b.skip2 : nullptr);
+  const double kappa2_max = P.qr2_tol > 0.0 ? kSkipKappa * kSkipKappa : 0.0;
+  e = launch_chol(n, b.L, b.dead, final_pass ? P.qr2_tol : 0.0, P.rank, b.skip2, final_pass ? 0 : 1, kappa2_max, st);
   if (e != cudaSuccess) return e;
-  if (!final_pass) return launch_apply_gram(n, b.xbuf, b.L, rows, b.q, b.gpart, st);
-  return launch_apply(n, b.q, b.L, rows, b.q, b.qthi, b.qtlo, P.rank, amax, st);
+  if (!final_pass) return launch_apply_gram(n, b.xbuf, b.L, rows, b.q, b.gpart, b.skip2, b.qthi, b.qtlo, P.rank, amax, st);
+  return launch_apply(n, b.q, b.L, rows, b.q, b.qthi, b.qtlo, P.rank, amax, b.skip2, st);
 }
 
 PackArgs pack_args(const LowrankPlan &P, uint8_t *payload, const Header &hdr) {
@@ -1725,15 +1821,23 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
   if (tab) return cudaErrorNotSupported;  // batch 1 only
   const LowrankBufs &b = P.b;
   const int64_t R = P.rows, C = P.cols;
-  launch_pdl(lr_vprep_kernel, dim3(P.rp), dim3(kVprepThreads), 0, st, vprev, C, P.rank, P.rp, step == 1 ? 1 : 0, seed, b.vthi, b.vtlo,
-             b.amax);
-  const dim3 dg((unsigned)(C / 64), (unsigned)(R / 64));
+  VprepArgs V{};
+  V.vprev = vprev;
+  V.cols = C;
+  V.r = P.rank;
+  V.rp = P.rp;
+  V.first = step == 1 ? 1 : 0;
+  V.seed = seed;
+  V.vthi = b.vthi;
+  V.vtlo = b.vtlo;
+  V.amax = b.amax;
+  const dim3 dg((unsigned)(P.rp + (C / 64) * (R / 64)));
   if (P.dtype == CF_BF16)
-    launch_pdl(lr_delta_kernel<__nv_bfloat16>, dim3(dg), dim3(256), 0, st, static_cast<const __nv_bfloat16 *>(args.a), args.ahat, args.err,
-                                                        P.ef_explicit, R, C, b.dhi, b.dlo);
+    launch_pdl(lr_delta_kernel<__nv_bfloat16>, dim3(dg), dim3(256), 0, st, static_cast<const __nv_bfloat16 *>(args.a),
+               args.ahat, args.err, P.ef_explicit, R, C, b.dhi, b.dlo, V);
   else
-    launch_pdl(lr_delta_kernel<float>, dim3(dg), dim3(256), 0, st, static_cast<const float *>(args.a), args.ahat, args.err, P.ef_explicit,
-                                               R, C, b.dhi, b.dlo);
+    launch_pdl(lr_delta_kernel<float>, dim3(dg), dim3(256), 0, st, static_cast<const float *>(args.a), args.ahat, args.err,
+               P.ef_explicit, R, C, b.dhi, b.dlo, V);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   for (int it = 0; it < P.iters; it++) {
@@ -1748,7 +1852,7 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
     unsigned *amax_q = (P.int4 && !more) ? b.amax : nullptr;
     unsigned *amax_v = (P.int4 && !more) ? b.amax + P.rp : nullptr;
     // Q = orth(Y): CholeskyQR2
-    if ((e = orthonormalise(P, b.ypart, P.sy, R, false, nullptr, st)) != cudaSuccess) return e;
+    if ((e = orthonormalise(P, b.ypart, P.sy, R, false, amax_q, st)) != cudaSuccess) return e;
     if ((e = orthonormalise(P, b.q, 1, R, true, amax_q, st)) != cudaSuccess) return e;
     // V = D^T Q
     if ((e = launch_thin(P, P.tm_dmhi, P.tm_dmlo, P.tm_qthi, P.tm_qtlo, b.vpart, C, R, P.sv, args.status, st, true,

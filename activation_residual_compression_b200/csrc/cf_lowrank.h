@@ -24,6 +24,7 @@ struct LowrankBufs {
   double *gpart = nullptr;                         // partial Gram matrices [nblk][rp][rp]
   double *L = nullptr;                             // Cholesky factor [rp][rp]
   int *dead = nullptr;                             // rank-deficient column flags [rp]
+  int *skip2 = nullptr;                            // the sweep's first CholeskyQR pass suffices (set on the device)
   unsigned *amax = nullptr;                        // column absmax bit patterns of Q [rp] and V [rp]
   // both roles: reconstruction operands dequantised from the payload
   __nv_bfloat16 *uahi = nullptr, *ualo = nullptr;  // [rows][kp]
