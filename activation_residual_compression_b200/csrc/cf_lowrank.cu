@@ -441,13 +441,22 @@ __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc
   gram_tiles<TT>(tile, gpart + (int64_t)blockIdx.x * n * n, threadIdx.x >> 5, threadIdx.x & 31);
 }
 
+// Offset of entry (i, j), j <= i, in the Cholesky kernel's packed array of
+// 8 x 8 tiles (tile (I, J), J <= I, at I (I + 1) / 2 + J; rows of kCholTld
+// doubles).
+constexpr int kCholTld = 9;  // tile row stride (doubles): a half-warp's 4 x 4 fragment in distinct banks
+__host__ __device__ constexpr int chol_tile(int I, int J) { return (I * (I + 1) / 2 + J) * 8 * kCholTld; }
+__device__ __forceinline__ int chol_entry(int i, int j) { return chol_tile(i >> 3, j >> 3) + (i & 7) * kCholTld + (j & 7); }
+
 // G = sum over the nblk partial Gram matrices, lower triangle only (the
 // Cholesky kernel reads nothing above the diagonal; those entries are set to
-// zero).  A block covers 32 consecutive entries, one per lane; its 8 warps sum
-// 8 contiguous slices of the partials, and the slice sums are added in slice
-// order, so the result does not depend on scheduling.
+// zero), row-major into G and, in the Cholesky kernel's packed tile layout,
+// into Gp (the lower tiles; entries above the diagonal of a diagonal tile are
+// zero).  A block covers 32 consecutive entries, one per lane; its 8 warps
+// sum 8 contiguous slices of the partials, and the slice sums are added in
+// slice order, so the result does not depend on scheduling.
 __global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart, int nblk, int n, double *G,
-                                                              const int *skip2) {
+                                                              double *Gp, const int *skip2) {
   pdl_enter();
   if (skip2 != nullptr && *skip2) return;  // second pass not needed (uniform over the grid)
   __shared__ double part[8][32];
@@ -475,6 +484,8 @@ __global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart
 #pragma unroll
     for (int w = 1; w < 8; w++) t += part[w][lane];
     G[e] = live ? t : 0.0;
+    const int gi = e / n, gj = e - (e / n) * n;
+    if ((gj >> 3) <= (gi >> 3)) Gp[chol_entry(gi, gj)] = live ? t : 0.0;
   }
 }
 
@@ -500,7 +511,6 @@ __global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart
 // 1, r_k = 0, so row k of X and column k of L (hence of X) are zero and the
 // column updates nothing; the other columns are the Cholesky factor of G
 // restricted to them.
-constexpr int kCholTld = 9;  // tile row stride (doubles): a half-warp's 4 x 4 fragment in distinct banks
 
 template <int TT>
 __host__ __device__ constexpr int chol_ntiles() {
@@ -510,9 +520,6 @@ __host__ __device__ constexpr size_t chol_smem_tt(int tt) {
   return (size_t)2 * ((2 * tt) * (2 * tt + 1) / 2) * 8 * kCholTld * 8;
 }
 
-__device__ __forceinline__ int chol_tile(int I, int J) {
-  return (I * (I + 1) / 2 + J) * 8 * kCholTld;
-}
 
 // D += sa P R^T (rt) or D += sa P R (!rt) for 8 x 8 tiles P, R of the packed
 // arrays, D in this lane's two accumulator entries; sa = -1 subtracts.
@@ -593,8 +600,9 @@ __device__ __forceinline__ void chol_diag(const double *Ab, double *Xb, int b, i
 // stored Q (2^-24), and the second pass is skipped: its kernels return at
 // once (second pass: !first_pass, *skip2 set).
 template <int TT>
-__global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double *Mout, int *dead, double near_id,
-                                                         int nlive, int *skip2, int first_pass, double kappa2_max) {
+__global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, const double *Gp, double *Mout, int *dead,
+                                                         double near_id, int nlive, int *skip2, int first_pass,
+                                                         double kappa2_max) {
   pdl_enter();
   if (!first_pass && *skip2) return;  // uniform over the block
   constexpr int n = 16 * TT;
@@ -649,30 +657,28 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t4 = lane & 3;
   const int nbl = (min(max(nlive, 0), n) + 7) / 8;
   const int nl = 8 * nbl;
-  const double thr = 1e-12 * G[0];
-  // the working matrix from G: eight loads in flight per thread before the
-  // stores into the tiles
-  for (int e0 = 0; e0 < nl * nl; e0 += 8 * 256) {
+  const double thr = 1e-12 * Gp[0];
+  // the working matrix: the live tiles of G's packed copy (the first
+  // nbl (nbl + 1) / 2 tiles of both arrays), eight loads in flight per thread
+  const int nlt = nbl * (nbl + 1) / 2 * 8 * kCholTld;
+  for (int e0 = 0; e0 < nlt; e0 += 8 * 256) {
     double g[8];
 #pragma unroll
     for (int u = 0; u < 8; u++) {
       const int e = e0 + u * 256 + (int)threadIdx.x;
-      const int gi = e / nl, gj = e - (e / nl) * nl;
-      g[u] = (e < nl * nl && gj <= gi) ? G[gi * n + gj] : 0.0;
+      g[u] = e < nlt ? Gp[e] : 0.0;
     }
 #pragma unroll
     for (int u = 0; u < 8; u++) {
       const int e = e0 + u * 256 + (int)threadIdx.x;
-      const int gi = e / nl, gj = e - (e / nl) * nl;
-      if (e < nl * nl && (gj >> 3) <= (gi >> 3)) {
-        const int o = chol_tile(gi >> 3, gj >> 3) + (gi & 7) * kCholTld + (gj & 7);
-        A[o] = g[u];
-        X[o] = 0.0;
+      if (e < nlt) {
+        A[e] = g[u];
+        X[e] = 0.0;
       }
     }
   }
   for (int k = nl + threadIdx.x; k < n; k += blockDim.x) dead_s[k] = 1;
-  for (int k = threadIdx.x; k < nl; k += blockDim.x) gdiag[k] = G[k * n + k];
+  for (int k = threadIdx.x; k < nl; k += blockDim.x) gdiag[k] = Gp[chol_entry(k, k)];
   __syncthreads();
   if (nbl > 0 && warp == 0) chol_diag(A, X, 0, nlive, thr, lane, dead_s);
   __syncthreads();
@@ -752,12 +758,17 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, double
     for (int o = 16; o > 0; o >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, o);
     if (lane == 0) red[warp] = sx;
     __syncthreads();
-    if (threadIdx.x == 0) {
-      double xs2 = 0.0, tr = 0.0;
-      for (int w = 0; w < 8; w++) xs2 += red[w];
-      for (int k = 0; k < nl; k++)
+    if (warp == 0) {
+      double tr = 0.0;  // trace of G over the live columns
+      for (int k = lane; k < nl; k += 32)
         if (!dead_s[k]) tr += gdiag[k];
-      *skip2 = (kappa2_max > 0.0 && tr * xs2 <= kappa2_max) ? 1 : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) tr += __shfl_xor_sync(0xffffffffu, tr, o);
+      if (lane == 0) {
+        double xs2 = 0.0;
+        for (int w = 0; w < 8; w++) xs2 += red[w];
+        *skip2 = (kappa2_max > 0.0 && tr * xs2 <= kappa2_max) ? 1 : 0;
+      }
     }
   }
 }
@@ -1452,6 +1463,10 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, 
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
+// Bytes of G in the Cholesky kernel's packed layout: the lower 8 x 8 tiles of
+// an rp x rp matrix, rows of kCholTld doubles.
+size_t gpk_bytes(size_t rp) { return (rp / 8) * (rp / 8 + 1) / 2 * 8 * kCholTld * 8; }
+
 size_t thin_smem(int n, int stages) { return (size_t)stages * (2u * kTileM * kTileK * 2 + 2u * n * kTileK * 2) + 1024; }
 int thin_stages(int n) { return n <= 96 ? 4 : 3; }
 size_t recon_smem(int kblocks, int a_split) {
@@ -1546,6 +1561,7 @@ void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *p
   enc += pad256(mx * rp * 4) * 2 + pad256(C * rp * 4);        // xbuf, q, v
   enc += pad256((size_t)plan->nblk_gram * rp * rp * 8);       // gpart
   enc += pad256(rp * rp * 8) + pad256(rp * 4) + pad256(4);    // L, dead, skip flag
+  enc += pad256(gpk_bytes(rp));                                // G in packed tiles
   enc += pad256(2 * rp * 4);                                  // amax
   plan->enc_scratch_bytes = enc;
   plan->dec_scratch_bytes = dec;
@@ -1612,6 +1628,7 @@ int lowrank_bind(LowrankPlan *plan, void *scratch) {
     b.L = reinterpret_cast<double *>(take(rp * rp * 8));
     b.dead = reinterpret_cast<int *>(take(rp * 4));
     b.skip2 = reinterpret_cast<int *>(take(4));
+    b.gpk = reinterpret_cast<double *>(take(gpk_bytes(rp)));
     b.amax = reinterpret_cast<unsigned *>(take(2 * rp * 4));
     ok = ok && make_map(&plan->tm_dhi, b.dhi, C, R, kTileM) && make_map(&plan->tm_dlo, b.dlo, C, R, kTileM) &&
          make_map(&plan->tm_vthi, b.vthi, C, rp, (uint32_t)rp) && make_map(&plan->tm_vtlo, b.vtlo, C, rp, (uint32_t)rp) &&
@@ -1664,17 +1681,17 @@ cudaError_t launch_gram(int n, int nblk, const float *src, int nsrc, int64_t row
   return cudaGetLastError();
 }
 
-cudaError_t launch_chol(int n, double *L, int *dead, double near_id, int nlive, int *skip2, int first_pass,
-                        double kappa2_max, cudaStream_t st) {
+cudaError_t launch_chol(int n, double *L, const double *Gp, int *dead, double near_id, int nlive, int *skip2,
+                        int first_pass, double kappa2_max, cudaStream_t st) {
   switch (n / 16) {
-    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), chol_smem_tt(1), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), chol_smem_tt(2), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), chol_smem_tt(3), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), chol_smem_tt(4), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), chol_smem_tt(5), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), chol_smem_tt(6), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), chol_smem_tt(7), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), chol_smem_tt(8), st, L, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), chol_smem_tt(1), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), chol_smem_tt(2), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), chol_smem_tt(3), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), chol_smem_tt(4), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), chol_smem_tt(5), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), chol_smem_tt(6), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), chol_smem_tt(7), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
+    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), chol_smem_tt(8), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -1730,9 +1747,10 @@ cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int
   // overwrites with M = L^-T; the first pass decides whether the second one
   // runs (lr_qr2_tol = 0: always, the full CholeskyQR2)
   launch_pdl(lr_gram_reduce_kernel, dim3((unsigned)((n * n + 31) / 32)), dim3(256), 0, st, b.gpart, nblk, n, b.L,
-             final_pass ? b.skip2 : nullptr);
+             b.gpk, final_pass ? b.skip2 : nullptr);
   const double kappa2_max = P.qr2_tol > 0.0 ? kSkipKappa * kSkipKappa : 0.0;
-  e = launch_chol(n, b.L, b.dead, final_pass ? P.qr2_tol : 0.0, P.rank, b.skip2, final_pass ? 0 : 1, kappa2_max, st);
+  e = launch_chol(n, b.L, b.gpk, b.dead, final_pass ? P.qr2_tol : 0.0, P.rank, b.skip2, final_pass ? 0 : 1,
+                  kappa2_max, st);
   if (e != cudaSuccess) return e;
   if (!final_pass) return launch_apply_gram(n, b.xbuf, b.L, rows, b.q, b.gpart, b.skip2, b.qthi, b.qtlo, P.rank, amax, st);
   return launch_apply(n, b.q, b.L, rows, b.q, b.qthi, b.qtlo, P.rank, amax, b.skip2, st);
