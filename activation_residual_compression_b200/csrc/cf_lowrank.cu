@@ -503,14 +503,23 @@ __global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart
 //   panel     L_ib = A_ib X_bb^T for the tiles below, and the finished row
 //             of the inverse X_bj = X_bb X_bj (j < b);
 //   trailing  A_ij -= L_ib L_jb^T (b < j <= i) and X_ij -= L_ib X_bj
-//             (i > b, j <= b); the warp that updates the next diagonal tile
-//             factors it at once.
-// Each phase ends with one block barrier; the tile products run on the fp64
-// MMA.  A pivot <= 1e-12 G_00 (R_kk <= 1e-6 R_00), or a column at or past
-// nlive (the rank's zero padding), marks column k rank deficient: dead[k] =
-// 1, r_k = 0, so row k of X and column k of L (hence of X) are zero and the
-// column updates nothing; the other columns are the Cholesky factor of G
-// restricted to them.
+//             (i > b, j <= b).
+// The diagonal chain is the critical path, so warp 0 runs one block column
+// ahead of the rest: in the step of column b it forms the panel tile
+// L_{b+1,b}, applies it to A_{b+1,b+1} and factors that tile, while warps
+// 1-7 form the other panel tiles and then (after a named barrier that warp
+// 0 arrives at once L_{b+1,b} is stored) the other trailing updates; one
+// block barrier ends the step.  Every tile receives the same products in
+// the same order as in a plain blocked elimination.  The tile products run
+// on the fp64 MMA.  A pivot <= 1e-12 G_00 (R_kk <= 1e-6 R_00), or a column
+// at or past nlive (the rank's zero padding), marks column k rank
+// deficient: dead[k] = 1, r_k = 0, so row k of X and column k of L (hence
+// of X) are zero and the column updates nothing; the other columns are the
+// Cholesky factor of G restricted to them.
+//
+// The factor leaves the kernel as X in the same packed tile layout (all
+// chol_ntiles tiles, those past the live ones zero): a flat copy here, and
+// the apply kernels stage M = X^T from it.
 
 template <int TT>
 __host__ __device__ constexpr int chol_ntiles() {
@@ -576,20 +585,27 @@ __device__ __forceinline__ void chol_diag(const double *Ab, double *Xb, int b, i
   }
 }
 
-// Cholesky factor L of the Gram matrix G (fp64, lower triangle read) and M =
-// L^-T (fp64 [n][n], upper triangular), with the dead flags.
+// Named barrier 1 over the whole block: warps 1-7 wait in it, warp 0 only
+// arrives (after its shared-memory stores, which the barrier publishes).
+__device__ __forceinline__ void chol_bar_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void chol_bar_arrive() { asm volatile("bar.arrive 1, 256;" ::: "memory"); }
+
+// Cholesky factor L of the Gram matrix G (fp64, lower triangle read) and X =
+// L^-1 (fp64, packed lower tiles into Xout, as described above), with the
+// dead flags.
 //
 // near_id > 0 (the second pass of CholeskyQR2, where G = Q1^T Q1 is close to
 // the identity): if every entry of E = G - I between nonzero columns has
-// |E_ij| <= near_id, M is the first-order factor instead: with G = L L^T and
+// |E_ij| <= near_id, X is the first-order factor instead: with G = L L^T and
 // L = I + F, F = strict_lower(E) + diag(E) / 2 + O(|E|^2), so L^-1 = I - F +
-// O(|E|^2), and Q1 M has an orthogonality error of about 3 n near_id^2 per
+// O(|E|^2), and Q1 X^T has an orthogonality error of about 3 n near_id^2 per
 // entry.  A column of G that is exactly zero (a column of Q1 zeroed as rank
 // deficient by the first pass) is dead, as in the elimination.  Otherwise
 // the blocked elimination runs.
 //
-// Columns nlive .. n-1 must be zero in G (the padding of the rank).  G and M
-// may alias (G is read before the first barrier).
+// Columns nlive .. n-1 must be zero in G (the padding of the rank).  G
+// (row-major, read only by the first-order test) and Xout may alias: G is
+// read before the first barrier.
 //
 // First pass of a sweep (first_pass): the elimination also bounds the
 // condition number of X (the matrix being orthonormalised) by B =
@@ -600,12 +616,13 @@ __device__ __forceinline__ void chol_diag(const double *Ab, double *Xb, int b, i
 // stored Q (2^-24), and the second pass is skipped: its kernels return at
 // once (second pass: !first_pass, *skip2 set).
 template <int TT>
-__global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, const double *Gp, double *Mout, int *dead,
+__global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, const double *Gp, double *Xout, int *dead,
                                                          double near_id, int nlive, int *skip2, int first_pass,
                                                          double kappa2_max) {
   pdl_enter();
   if (!first_pass && *skip2) return;  // uniform over the block
   constexpr int n = 16 * TT;
+  constexpr int nall = chol_ntiles<TT>() * 8 * kCholTld;  // doubles of the whole packed array
   __shared__ int dead_s[n];
   __shared__ double gdiag[n];
   __shared__ double red[8];
@@ -637,15 +654,18 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, const 
         for (int a = 0; a < TT; a++) dead_s[i0 + a] = w[a][a] == 0.0 ? 1 : 0;
       }
       __syncthreads();
+      // every entry of the packed tiles (the part above the diagonal of a
+      // diagonal tile is zero); the tiles' padding column is never read
 #pragma unroll
       for (int a = 0; a < TT; a++) {
         const int gi = i0 + a;
 #pragma unroll
         for (int c = 0; c < TT; c++) {
           const int gj = j0 + c;
-          double m = 0.0;  // M[gj][gi] = L^-1[gi][gj]
-          if (gj <= gi && !dead_s[gi] && !dead_s[gj]) m = gj == gi ? 1.0 - 0.5 * (w[a][c] - 1.0) : -w[a][c];
-          Mout[gj * n + gi] = m;
+          if ((gj >> 3) > (gi >> 3)) continue;
+          double m = 0.0;  // X[gi][gj] = L^-1[gi][gj]
+          if (lower && gj <= gi && !dead_s[gi] && !dead_s[gj]) m = gj == gi ? 1.0 - 0.5 * (w[a][c] - 1.0) : -w[a][c];
+          Xout[chol_entry(gi, gj)] = m;
         }
       }
       for (int e = threadIdx.x; e < n; e += blockDim.x) dead[e] = dead_s[e];
@@ -657,19 +677,18 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, const 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t4 = lane & 3;
   const int nbl = (min(max(nlive, 0), n) + 7) / 8;
   const int nl = 8 * nbl;
-  const double thr = 1e-12 * Gp[0];
   // the working matrix: the live tiles of G's packed copy (the first
-  // nbl (nbl + 1) / 2 tiles of both arrays), eight loads in flight per thread
+  // nbl (nbl + 1) / 2 tiles of both arrays), sixteen loads in flight per thread
   const int nlt = nbl * (nbl + 1) / 2 * 8 * kCholTld;
-  for (int e0 = 0; e0 < nlt; e0 += 8 * 256) {
-    double g[8];
+  for (int e0 = 0; e0 < nlt; e0 += 16 * 256) {
+    double g[16];
 #pragma unroll
-    for (int u = 0; u < 8; u++) {
+    for (int u = 0; u < 16; u++) {
       const int e = e0 + u * 256 + (int)threadIdx.x;
       g[u] = e < nlt ? Gp[e] : 0.0;
     }
 #pragma unroll
-    for (int u = 0; u < 8; u++) {
+    for (int u = 0; u < 16; u++) {
       const int e = e0 + u * 256 + (int)threadIdx.x;
       if (e < nlt) {
         A[e] = g[u];
@@ -678,78 +697,90 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, const 
     }
   }
   for (int k = nl + threadIdx.x; k < n; k += blockDim.x) dead_s[k] = 1;
-  for (int k = threadIdx.x; k < nl; k += blockDim.x) gdiag[k] = Gp[chol_entry(k, k)];
   __syncthreads();
+  // G's diagonal (for the condition bound), read before any update of A
+  for (int k = threadIdx.x; k < nl; k += blockDim.x) gdiag[k] = A[chol_entry(k, k)];
+  const double thr = 1e-12 * A[0];
   if (nbl > 0 && warp == 0) chol_diag(A, X, 0, nlive, thr, lane, dead_s);
   __syncthreads();
   for (int b = 0; b < nbl; b++) {
     const int m = nbl - 1 - b;  // block rows below the diagonal
     const double *Xbb = X + chol_tile(b, b);
-    // panel L_ib = A_ib X_bb^T (i > b) and the inverse's row X_bj = X_bb X_bj (j < b)
-    for (int t = warp; t < m + b; t += 8) {
-      double *T = t < m ? A + chol_tile(b + 1 + t, b) : X + chol_tile(b, t - m);
-      double d0 = 0.0, d1 = 0.0;
-      if (t < m)
-        chol_tile_mma(d0, d1, T, Xbb, true, 1.0, gq, t4);
-      else
-        chol_tile_mma(d0, d1, Xbb, T, false, 1.0, gq, t4);
-      __syncwarp();
-      T[gq * kCholTld + 2 * t4] = d0;
-      T[gq * kCholTld + 2 * t4 + 1] = d1;
-    }
-    __syncthreads();
-    if (m == 0) break;  // uniform
-    // trailing A_ij -= L_ib L_jb^T (b < j <= i) and X_ij -= L_ib X_bj (i > b, j <= b); warp 0 takes the
-    // next diagonal tile and factors it, warps 1..7 the rest
-    const int ntr = m * (m + 1) / 2, ntask = ntr - 1 + m * (b + 1);
     if (warp == 0) {
-      double *T = A + chol_tile(b + 1, b + 1);
-      const double *Lb = A + chol_tile(b + 1, b);
-      double d0 = T[gq * kCholTld + 2 * t4], d1 = T[gq * kCholTld + 2 * t4 + 1];
-      chol_tile_mma(d0, d1, Lb, Lb, true, -1.0, gq, t4);
-      T[gq * kCholTld + 2 * t4] = d0;
-      T[gq * kCholTld + 2 * t4 + 1] = d1;
-      __syncwarp();
-      chol_diag(T, X + chol_tile(b + 1, b + 1), b + 1, nlive, thr, lane, dead_s);
-    } else {
-      for (int t = warp - 1; t < ntask; t += 7) {
-        int i, j;
-        double *T;
-        const double *R;
-        bool rt;
-        if (t < ntr - 1) {  // trailing tile, row-major over the triangle after the next diagonal tile
-          int u = t + 1, ii = 0;
-          while (u >= ii + 1) {
-            u -= ii + 1;
-            ii++;
-          }
-          i = b + 1 + ii;
-          j = b + 1 + u;
-          T = A + chol_tile(i, j);
-          R = A + chol_tile(j, b);
-          rt = true;
-        } else {
-          const int u = t - (ntr - 1);
-          i = b + 1 + u / (b + 1);
-          j = u % (b + 1);
-          T = X + chol_tile(i, j);
-          R = X + chol_tile(b, j);
-          rt = false;
-        }
+      if (m > 0) {  // uniform: the next diagonal tile's chain
+        double *P = A + chol_tile(b + 1, b);
+        double p0 = 0.0, p1 = 0.0;
+        chol_tile_mma(p0, p1, P, Xbb, true, 1.0, gq, t4);
+        __syncwarp();
+        P[gq * kCholTld + 2 * t4] = p0;
+        P[gq * kCholTld + 2 * t4 + 1] = p1;
+        __syncwarp();
+        chol_bar_arrive();  // L_{b+1,b} is stored: warps 1-7 may start the trailing updates
+        double *T = A + chol_tile(b + 1, b + 1);
         double d0 = T[gq * kCholTld + 2 * t4], d1 = T[gq * kCholTld + 2 * t4 + 1];
-        chol_tile_mma(d0, d1, A + chol_tile(i, b), R, rt, -1.0, gq, t4);
+        chol_tile_mma(d0, d1, P, P, true, -1.0, gq, t4);
         T[gq * kCholTld + 2 * t4] = d0;
         T[gq * kCholTld + 2 * t4 + 1] = d1;
+        __syncwarp();
+        chol_diag(T, X + chol_tile(b + 1, b + 1), b + 1, nlive, thr, lane, dead_s);
+      }
+    } else {
+      // panel L_ib = A_ib X_bb^T (i >= b + 2) and the inverse's row X_bj = X_bb X_bj (j < b)
+      const int mp = m > 0 ? m - 1 : 0;
+      for (int t = warp - 1; t < mp + b; t += 7) {
+        double *T = t < mp ? A + chol_tile(b + 2 + t, b) : X + chol_tile(b, t - mp);
+        double d0 = 0.0, d1 = 0.0;
+        if (t < mp)
+          chol_tile_mma(d0, d1, T, Xbb, true, 1.0, gq, t4);
+        else
+          chol_tile_mma(d0, d1, Xbb, T, false, 1.0, gq, t4);
+        __syncwarp();
+        T[gq * kCholTld + 2 * t4] = d0;
+        T[gq * kCholTld + 2 * t4 + 1] = d1;
+      }
+      if (m > 0) {  // uniform
+        chol_bar_sync();  // every panel tile of column b is stored
+        // trailing A_ij -= L_ib L_jb^T (b < j <= i, all but the next diagonal tile) and X_ij -= L_ib X_bj
+        // (i > b, j <= b)
+        const int ntr = m * (m + 1) / 2, ntask = ntr - 1 + m * (b + 1);
+        for (int t = warp - 1; t < ntask; t += 7) {
+          int i, j;
+          double *T;
+          const double *R;
+          bool rt;
+          if (t < ntr - 1) {  // trailing tile, row-major over the triangle after the next diagonal tile
+            int u = t + 1, ii = 0;
+            while (u >= ii + 1) {
+              u -= ii + 1;
+              ii++;
+            }
+            i = b + 1 + ii;
+            j = b + 1 + u;
+            T = A + chol_tile(i, j);
+            R = A + chol_tile(j, b);
+            rt = true;
+          } else {
+            const int u = t - (ntr - 1);
+            i = b + 1 + u / (b + 1);
+            j = u % (b + 1);
+            T = X + chol_tile(i, j);
+            R = X + chol_tile(b, j);
+            rt = false;
+          }
+          double d0 = T[gq * kCholTld + 2 * t4], d1 = T[gq * kCholTld + 2 * t4 + 1];
+          chol_tile_mma(d0, d1, A + chol_tile(i, b), R, rt, -1.0, gq, t4);
+          T[gq * kCholTld + 2 * t4] = d0;
+          T[gq * kCholTld + 2 * t4 + 1] = d1;
+        }
       }
     }
     __syncthreads();
   }
-  // M[gj][gi] = X[gi][gj]
-  double sx = 0.0;  // this thread's part of ||X||_F^2
-  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
-    const int gj = e / n, gi = e % n;
-    const double xv = (gi < nl && gj <= gi) ? X[chol_tile(gi >> 3, gj >> 3) + (gi & 7) * kCholTld + (gj & 7)] : 0.0;
-    Mout[e] = xv;
+  // X to Xout, the whole packed array (tiles past the live ones zero)
+  double sx = 0.0;  // this thread's part of ||X||_F^2 (the padding column and the zeros add nothing)
+  for (int e = threadIdx.x; e < nall; e += blockDim.x) {
+    const double xv = e < nlt ? X[e] : 0.0;
+    Xout[e] = xv;
     sx = fma(xv, xv, sx);
   }
   for (int e = threadIdx.x; e < n; e += blockDim.x) dead[e] = dead_s[e];
@@ -790,17 +821,35 @@ __host__ __device__ constexpr int apply_mld() {
   return 16 * TT + 4;  // M row stride (doubles): each half-warp's 4 rows x 4 fragment entries in distinct banks
 }
 
-// Stage M (fp64 [n][n]) into Ms (row stride apply_mld) and the block's nx
-// rows of X (fp32 [rows][n], from row r0; rows past the end read as zero) into
-// xs (row stride apply_xld).
+// Stage M = L^-T into Ms (row stride apply_mld) from the factor kernel's
+// packed tiles of X = L^-1 (tile (I, J) of X is the transpose of M's tile
+// (J, I); the entries of M below its diagonal tiles are never read), and the
+// block's nx rows of X (fp32 [rows][n], from row r0; rows past the end read
+// as zero) into xs (row stride apply_xld).
 template <int TT>
-__device__ __forceinline__ void apply_stage(const float *x, const double *M, int64_t rows, int64_t r0, int nx,
+__device__ __forceinline__ void apply_stage(const float *x, const double *Xp, int64_t rows, int64_t r0, int nx,
                                             double *Ms, float *xs) {
   constexpr int n = 16 * TT, mld = apply_mld<TT>(), xld = apply_xld<TT>();
-  const double2 *M2 = reinterpret_cast<const double2 *>(M);
-  for (int e = threadIdx.x; e < n * n / 2; e += blockDim.x) {
-    const int rr = (2 * e) / n, c = (2 * e) % n;
-    *reinterpret_cast<double2 *>(Ms + rr * mld + c) = M2[e];
+  constexpr int NT = chol_ntiles<TT>(), NE = NT * 64, NU = (NE + 255) / 256;
+  double v[NU];
+#pragma unroll
+  for (int u = 0; u < NU; u++) {  // all loads in flight first
+    const int e = (int)threadIdx.x + 256 * u;
+    const int t = e >> 6, w = e & 63;
+    v[u] = e < NE ? Xp[t * 8 * kCholTld + (w & 7) * kCholTld + (w >> 3)] : 0.0;
+  }
+#pragma unroll
+  for (int u = 0; u < NU; u++) {
+    const int e = (int)threadIdx.x + 256 * u;
+    if (e < NE) {
+      const int t = e >> 6, w = e & 63;
+      int I = 0, J = t;  // t = I (I + 1) / 2 + J, J <= I
+      while (J > I) {
+        J -= I + 1;
+        I++;
+      }
+      Ms[(8 * J + (w >> 3)) * mld + 8 * I + (w & 7)] = v[u];
+    }
   }
   const float4 *x4 = reinterpret_cast<const float4 *>(x) + r0 * (n / 4);
   for (int e = threadIdx.x; e < nx * n / 4; e += blockDim.x) {
@@ -848,13 +897,6 @@ __device__ __forceinline__ void apply_tiles(const float *xs, const double *Ms, i
   }
 }
 
-// Q = X M (M = L^-T, upper triangular, zero below the diagonal) for
-// kApplyRows rows per block (apply_tiles; M and the rows of X staged in
-// shared memory).  Writes Q fp32 [rows][n] and, when qthi != nullptr, Q^T
-// split in bf16 ([n][rows], the K-major B operand of V = D^T Q), transposed
-// through shared memory so that those stores are row-contiguous; when amax !=
-// nullptr, the absmax of each of Q's first r columns (the INT4 scales'
-// input) goes to amax, one atomicMax per column and block.
 // The outputs of Q = X M for the 8 RT rows of one block from r0, from the
 // accumulators of apply_tiles: Q fp32 [rows][n]; when amax != nullptr the
 // absmax of each of Q's first r columns (the INT4 scales' input), one
@@ -918,14 +960,15 @@ __device__ __forceinline__ void apply_store(const double (&acc)[apply_rounds<TT>
   }
 }
 
-// Q = X M (M = L^-T, upper triangular, zero below the diagonal) for
-// kApplyRows rows per block (apply_tiles; M and the rows of X staged in
-// shared memory), with the stores of apply_store.  The second CholeskyQR
+// Q = X M (M = L^-T, upper triangular, zero below the diagonal; staged from
+// the factor kernel's packed L^-1) for kApplyRows rows per block
+// (apply_tiles; M and the rows of X staged in shared memory), with the
+// stores of apply_store.  The second CholeskyQR
 // pass of a sweep whose first pass was accurate enough (*skip2 set by the
 // first pass's factor kernel) has nothing to do: that pass's apply already
 // wrote these outputs.
 template <int TT>
-__global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const double *M, int64_t rows, float *q,
+__global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const double *Xp, int64_t rows, float *q,
                                                        __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo, int r,
                                                        unsigned *amax, const int *skip2) {
   pdl_enter();
@@ -937,7 +980,7 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
   double *Ms = reinterpret_cast<double *>(asm_);        // [n][mld]
   float *xs = reinterpret_cast<float *>(Ms + n * mld);  // [kApplyRows][xld]; reused as Q^T [n][kApplyRows + 1]
   const int64_t r0 = (int64_t)blockIdx.x * kApplyRows;
-  apply_stage<TT>(x, M, rows, r0, kApplyRows, Ms, xs);
+  apply_stage<TT>(x, Xp, rows, r0, kApplyRows, Ms, xs);
   if (amax != nullptr)
     for (int c = threadIdx.x; c < n; c += 256) cmax[c] = 0u;
   __syncthreads();
@@ -956,7 +999,7 @@ __global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const dou
 // the block writes the final pass's outputs instead (apply_store: Q, its
 // INT4 column maxima when amax != nullptr, Q^T split) and no Gram matrix.
 template <int TT>
-__global__ void __launch_bounds__(256) lr_apply_gram_kernel(const float *x, const double *M, int64_t rows, float *q,
+__global__ void __launch_bounds__(256) lr_apply_gram_kernel(const float *x, const double *Xp, int64_t rows, float *q,
                                                             double *gpart, const int *skip2, __nv_bfloat16 *qthi,
                                                             __nv_bfloat16 *qtlo, int r, unsigned *amax) {
   pdl_enter();
@@ -970,7 +1013,7 @@ __global__ void __launch_bounds__(256) lr_apply_gram_kernel(const float *x, cons
   float *gs = xs + kGramRows * xld;                     // Q1 [kGramRows][gram_ld]
   const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
   const bool final_q = *skip2 != 0;                     // uniform over the grid
-  apply_stage<TT>(x, M, rows, r0, kGramRows, Ms, xs);
+  apply_stage<TT>(x, Xp, rows, r0, kGramRows, Ms, xs);
   if (final_q && amax != nullptr)
     for (int c = threadIdx.x; c < n; c += 256) cmax[c] = 0u;
   __syncthreads();
@@ -1743,9 +1786,10 @@ cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int
   // the first pass's partial Gram matrices come from the Gram kernel (over the
   // split-K partials of Y), the second pass's from the first pass's apply
   if (!final_pass && (e = launch_gram(n, nblk, src, nsrc, rows, b.xbuf, b.gpart, st)) != cudaSuccess) return e;
-  // the reduced Gram matrix goes to L, which the Cholesky kernel then
-  // overwrites with M = L^-T; the first pass decides whether the second one
-  // runs (lr_qr2_tol = 0: always, the full CholeskyQR2)
+  // the reduced Gram matrix goes to L (row-major) and gpk (packed tiles);
+  // the Cholesky kernel then overwrites L with X = L^-1 in packed tiles; the
+  // first pass decides whether the second one runs (lr_qr2_tol = 0: always,
+  // the full CholeskyQR2)
   launch_pdl(lr_gram_reduce_kernel, dim3((unsigned)((n * n + 31) / 32)), dim3(256), 0, st, b.gpart, nblk, n, b.L,
              b.gpk, final_pass ? b.skip2 : nullptr);
   const double kappa2_max = P.qr2_tol > 0.0 ? kSkipKappa * kSkipKappa : 0.0;
