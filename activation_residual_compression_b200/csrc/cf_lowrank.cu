@@ -101,11 +101,13 @@ struct VprepArgs {
   uint64_t seed;
   __nv_bfloat16 *vthi, *vtlo;
   unsigned *amax;
+  unsigned *gbar;  // the orthonormalisation kernels' barrier counters (one per sweep)
 };
 __device__ __forceinline__ void vprep_column(const VprepArgs &V, int k) {
-  if (threadIdx.x == 0) {  // this encode's column maxima start from zero
+  if (threadIdx.x == 0) {  // this encode's column maxima and barrier counters start from zero
     V.amax[k] = 0u;
     V.amax[V.rp + k] = 0u;
+    if (k < 2) V.gbar[k] = 0u;
   }
   int nz = 0;
   if (k < V.r && !V.first)
@@ -385,25 +387,24 @@ __device__ __forceinline__ void gram_tiles(const float *xs, double *g, int warp,
       *reinterpret_cast<double2 *>(g + (8 * ti[u] + gq) * n + 8 * tj[u] + 2 * t4) = make_double2(acc[u][0], acc[u][1]);
 }
 
-// X = sum of the nsrc partial slabs (fixed order), stored fp32 [rows][n], and
-// the partial Gram matrix X^T X (fp64, gram_tiles) of this block's kGramRows
-// rows.
+// Row block rb (kGramRows rows): X = sum of the nsrc partial slabs of src
+// (fixed order), stored fp32 [rows][n], and the partial Gram matrix X^T X
+// (fp64, gram_tiles) of these rows into gpart[rb]; tile: kGramRows x gram_ld
+// floats of shared memory.  Called by every thread of the block.
 template <int TT>
-__global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc, int64_t rows, float *x,
-                                                      double *gpart) {
-  pdl_enter();
+__device__ __forceinline__ void gram_rows(const float *src, int nsrc, int64_t rows, int rb, float *x, double *gpart,
+                                          float *tile) {
   constexpr int n = 16 * TT;
   constexpr int n4 = n / 4;                          // float4 per row
   constexpr int NV = (kGramRows * n4 + 255) / 256;   // float4 per thread
-  __shared__ __align__(16) float tile[kGramRows * gram_ld<TT>()];
-  const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
+  const int64_t r0 = (int64_t)rb * kGramRows;
   const float4 *s4 = reinterpret_cast<const float4 *>(src) + r0 * n4;
   const int64_t slab4 = rows * n4;
   float4 acc4[NV];
 #pragma unroll
   for (int v = 0; v < NV; v++) {
     const int e = threadIdx.x + 256 * v;
-    acc4[v] = e < kGramRows * n4 ? s4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+    acc4[v] = e < kGramRows * n4 ? __ldcg(s4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   for (int p0 = 1; p0 < nsrc; p0 += 4) {  // four slabs' loads in flight, added in slab order
     float4 t[4][NV];
@@ -412,7 +413,7 @@ __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc
 #pragma unroll
       for (int v = 0; v < NV; v++) {
         const int e = threadIdx.x + 256 * v;
-        t[u][v] = (p0 + u < nsrc && e < kGramRows * n4) ? s4[(int64_t)(p0 + u) * slab4 + e]
+        t[u][v] = (p0 + u < nsrc && e < kGramRows * n4) ? __ldcg(s4 + (int64_t)(p0 + u) * slab4 + e)
                                                          : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
@@ -428,6 +429,7 @@ __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc
     }
   }
   float4 *x4 = reinterpret_cast<float4 *>(x) + r0 * n4;
+  __syncthreads();  // the previous row block's Gram products are done with the tile
 #pragma unroll
   for (int v = 0; v < NV; v++) {
     const int e = threadIdx.x + 256 * v;
@@ -438,7 +440,7 @@ __global__ void __launch_bounds__(256) lr_gram_kernel(const float *src, int nsrc
     }
   }
   __syncthreads();
-  gram_tiles<TT>(tile, gpart + (int64_t)blockIdx.x * n * n, threadIdx.x >> 5, threadIdx.x & 31);
+  gram_tiles<TT>(tile, gpart + (int64_t)rb * n * n, threadIdx.x >> 5, threadIdx.x & 31);
 }
 
 // Offset of entry (i, j), j <= i, in the Cholesky kernel's packed array of
@@ -448,35 +450,46 @@ constexpr int kCholTld = 9;  // tile row stride (doubles): a half-warp's 4 x 4 f
 __host__ __device__ constexpr int chol_tile(int I, int J) { return (I * (I + 1) / 2 + J) * 8 * kCholTld; }
 __device__ __forceinline__ int chol_entry(int i, int j) { return chol_tile(i >> 3, j >> 3) + (i & 7) * kCholTld + (j & 7); }
 
+// Entry group g (32 consecutive entries of the n x n matrix, one per lane):
 // G = sum over the nblk partial Gram matrices, lower triangle only (the
-// Cholesky kernel reads nothing above the diagonal; those entries are set to
-// zero), row-major into G and, in the Cholesky kernel's packed tile layout,
+// Cholesky factor reads nothing above the diagonal; those entries are set to
+// zero), row-major into G and, in the Cholesky factor's packed tile layout,
 // into Gp (the lower tiles; entries above the diagonal of a diagonal tile are
-// zero).  A block covers 32 consecutive entries, one per lane; its 8 warps
-// sum 8 contiguous slices of the partials, and the slice sums are added in
-// slice order, so the result does not depend on scheduling.
-__global__ void __launch_bounds__(256) lr_gram_reduce_kernel(const double *gpart, int nblk, int n, double *G,
-                                                              double *Gp, const int *skip2) {
-  pdl_enter();
-  if (skip2 != nullptr && *skip2) return;  // second pass not needed (uniform over the grid)
-  __shared__ double part[8][32];
+// zero).  The block's 8 warps sum 8 contiguous slices of the partials (four
+// interleaved accumulators, sixteen loads in flight), and the slice sums are
+// added in slice order, so the result does not depend on scheduling.  part:
+// 8 x 32 doubles of shared memory.  Called by every thread of the block.
+__device__ __forceinline__ void reduce_group(const double *gpart, int nblk, int n, double *G, double *Gp, int g,
+                                             double (*part)[32]) {
   const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
   const int nn = n * n;
-  const int e = blockIdx.x * 32 + lane;
+  const int e = g * 32 + lane;
   const bool live = e < nn && (e % n) <= (e / n);
   const int per = (nblk + 7) / 8;
   const int b0 = wp * per, b1 = min(nblk, b0 + per);
   double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
   if (live) {
-    int b = b0;
-    for (; b + 3 < b1; b += 4) {
-      a0 += gpart[(int64_t)b * nn + e];
-      a1 += gpart[(int64_t)(b + 1) * nn + e];
-      a2 += gpart[(int64_t)(b + 2) * nn + e];
-      a3 += gpart[(int64_t)(b + 3) * nn + e];
+    for (int c0 = b0; c0 < b1; c0 += 16) {
+      double t[16];
+#pragma unroll
+      for (int u = 0; u < 16; u++) t[u] = c0 + u < b1 ? __ldcg(gpart + (int64_t)(c0 + u) * nn + e) : 0.0;
+      // the partials in order, partial b to accumulator (b - b0) % 4 (b1 - b0 is not always a multiple of 4)
+#pragma unroll
+      for (int u = 0; u < 16; u += 4) {
+        if (c0 + u + 3 < b1) {
+          a0 += t[u];
+          a1 += t[u + 1];
+          a2 += t[u + 2];
+          a3 += t[u + 3];
+        } else {
+#pragma unroll
+          for (int w = 0; w < 4; w++)
+            if (c0 + u + w < b1) a0 += t[u + w];
+        }
+      }
     }
-    for (; b < b1; b++) a0 += gpart[(int64_t)b * nn + e];
   }
+  __syncthreads();  // the previous group's slice sums have been read
   part[wp][lane] = (a0 + a1) + (a2 + a3);
   __syncthreads();
   if (wp == 0 && e < nn) {
@@ -613,20 +626,17 @@ __device__ __forceinline__ void chol_bar_arrive() { asm volatile("bar.arrive 1, 
 // over the live columns, and sets *skip2 when B^2 <= kappa2_max (0: never).
 // Then Q1 = X L^-T is orthonormal to within about n kappa^2 2^-53 per entry
 // (the fp64 Gram matrix and elimination), far below the fp32 rounding of the
-// stored Q (2^-24), and the second pass is skipped: its kernels return at
-// once (second pass: !first_pass, *skip2 set).
+// stored Q (2^-24), and the second pass is skipped.
+//
+// Run by one block of 256 threads; csm: chol_smem_tt(TT) bytes of shared
+// memory (16-byte aligned), dead_s and gdiag: n entries, red: 8.  G and Gp
+// were written by other blocks of the same grid: they are read through L2.
 template <int TT>
-__global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, const double *Gp, double *Xout, int *dead,
-                                                         double near_id, int nlive, int *skip2, int first_pass,
-                                                         double kappa2_max) {
-  pdl_enter();
-  if (!first_pass && *skip2) return;  // uniform over the block
+__device__ __forceinline__ void chol_factor(const double *G, const double *Gp, double *Xout, int *dead,
+                                            double near_id, int nlive, int *skip2, int first_pass, double kappa2_max,
+                                            uint8_t *csm, int *dead_s, double *gdiag, double *red) {
   constexpr int n = 16 * TT;
   constexpr int nall = chol_ntiles<TT>() * 8 * kCholTld;  // doubles of the whole packed array
-  __shared__ int dead_s[n];
-  __shared__ double gdiag[n];
-  __shared__ double red[8];
-  extern __shared__ __align__(16) uint8_t csm[];
   if (near_id > 0.0) {
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
     const int i0 = ty * TT, j0 = tx * TT;
@@ -635,7 +645,7 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, const 
 #pragma unroll
     for (int a = 0; a < TT; a++)
 #pragma unroll
-      for (int c = 0; c < TT; c++) w[a][c] = (lower && j0 + c <= i0 + a) ? G[(i0 + a) * n + j0 + c] : 0.0;
+      for (int c = 0; c < TT; c++) w[a][c] = (lower && j0 + c <= i0 + a) ? __ldcg(G + (i0 + a) * n + j0 + c) : 0.0;
     int far = 0;
     if (lower) {
 #pragma unroll
@@ -685,7 +695,7 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, const 
 #pragma unroll
     for (int u = 0; u < 16; u++) {
       const int e = e0 + u * 256 + (int)threadIdx.x;
-      g[u] = e < nlt ? Gp[e] : 0.0;
+      g[u] = e < nlt ? __ldcg(Gp + e) : 0.0;
     }
 #pragma unroll
     for (int u = 0; u < 16; u++) {
@@ -804,12 +814,9 @@ __global__ void __launch_bounds__(256, 1) lr_chol_kernel(const double *G, const 
   }
 }
 
-// Rows per apply block.
-constexpr int kApplyRows = 16;
-
 // The second CholeskyQR pass of a sweep is skipped when the first pass bounds
 // the condition number of the matrix it orthonormalises by this (see
-// lr_chol_kernel): its orthogonality error is then about n kSkipKappa^2 2^-53
+// chol_factor): its orthogonality error is then about n kSkipKappa^2 2^-53
 // <= 2^-30 per entry for n <= 128, against the 2^-24 of the stored fp32 Q.
 constexpr double kSkipKappa = 256.0;
 template <int TT>
@@ -821,22 +828,36 @@ __host__ __device__ constexpr int apply_mld() {
   return 16 * TT + 4;  // M row stride (doubles): each half-warp's 4 rows x 4 fragment entries in distinct banks
 }
 
-// Stage M = L^-T into Ms (row stride apply_mld) from the factor kernel's
+// Stage M = L^-T into Ms (row stride apply_mld) from the Cholesky factor's
 // packed tiles of X = L^-1 (tile (I, J) of X is the transpose of M's tile
-// (J, I); the entries of M below its diagonal tiles are never read), and the
-// block's nx rows of X (fp32 [rows][n], from row r0; rows past the end read
-// as zero) into xs (row stride apply_xld).
+// (J, I); the entries of M below its diagonal tiles are never read), and
+// with it the kGramRows rows of X from row r0 (apply_stage_x), all loads in
+// flight at once.  Xp was written by another block of the grid: it is read
+// through L2.
 template <int TT>
-__device__ __forceinline__ void apply_stage(const float *x, const double *Xp, int64_t rows, int64_t r0, int nx,
-                                            double *Ms, float *xs) {
+__device__ __forceinline__ void apply_stage_mx(const double *Xp, double *Ms, const float *x, int64_t rows, int64_t r0,
+                                               float *xs) {
   constexpr int n = 16 * TT, mld = apply_mld<TT>(), xld = apply_xld<TT>();
   constexpr int NT = chol_ntiles<TT>(), NE = NT * 64, NU = (NE + 255) / 256;
+  constexpr int NX = kGramRows * n / 4, NXU = (NX + 255) / 256;
   double v[NU];
+  float4 xv[NXU];
 #pragma unroll
   for (int u = 0; u < NU; u++) {  // all loads in flight first
     const int e = (int)threadIdx.x + 256 * u;
     const int t = e >> 6, w = e & 63;
-    v[u] = e < NE ? Xp[t * 8 * kCholTld + (w & 7) * kCholTld + (w >> 3)] : 0.0;
+    v[u] = e < NE ? __ldcg(Xp + t * 8 * kCholTld + (w & 7) * kCholTld + (w >> 3)) : 0.0;
+  }
+  const float4 *x4 = reinterpret_cast<const float4 *>(x) + r0 * (n / 4);
+#pragma unroll
+  for (int u = 0; u < NXU; u++) {
+    const int e = (int)threadIdx.x + 256 * u;
+    xv[u] = (e < NX && r0 + e / (n / 4) < rows) ? x4[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int u = 0; u < NXU; u++) {
+    const int e = (int)threadIdx.x + 256 * u;
+    if (e < NX) *reinterpret_cast<float4 *>(xs + (e / (n / 4)) * xld + (e % (n / 4)) * 4) = xv[u];
   }
 #pragma unroll
   for (int u = 0; u < NU; u++) {
@@ -851,6 +872,13 @@ __device__ __forceinline__ void apply_stage(const float *x, const double *Xp, in
       Ms[(8 * J + (w >> 3)) * mld + 8 * I + (w & 7)] = v[u];
     }
   }
+}
+
+// Stage the nx rows of X (fp32 [rows][n]) from row r0 into xs (row stride
+// apply_xld); rows past the end read as zero.
+template <int TT>
+__device__ __forceinline__ void apply_stage_x(const float *x, int64_t rows, int64_t r0, int nx, float *xs) {
+  constexpr int n = 16 * TT, xld = apply_xld<TT>();
   const float4 *x4 = reinterpret_cast<const float4 *>(x) + r0 * (n / 4);
   for (int e = threadIdx.x; e < nx * n / 4; e += blockDim.x) {
     const int rr = e / (n / 4), c = (e % (n / 4)) * 4;
@@ -960,73 +988,44 @@ __device__ __forceinline__ void apply_store(const double (&acc)[apply_rounds<TT>
   }
 }
 
-// Q = X M (M = L^-T, upper triangular, zero below the diagonal; staged from
-// the factor kernel's packed L^-1) for kApplyRows rows per block
-// (apply_tiles; M and the rows of X staged in shared memory), with the
-// stores of apply_store.  The second CholeskyQR
-// pass of a sweep whose first pass was accurate enough (*skip2 set by the
-// first pass's factor kernel) has nothing to do: that pass's apply already
-// wrote these outputs.
+// Q = X M (M = L^-T, upper triangular, zero below the diagonal; staged once
+// from the packed factor Xp) for the grid's row blocks of kGramRows rows
+// (apply_tiles; the rows of X staged in shared memory).  final_q: the
+// outputs of apply_store (Q, its INT4 column maxima when amax != nullptr,
+// Q^T split when qthi != nullptr); otherwise (the first pass of a sweep
+// whose second pass runs) Q and the partial Gram matrix Q^T Q of each row
+// block from the fp32 values it stores, with the sums of gram_tiles, into
+// gpart.  x and q may alias (a block reads its rows before it writes them).
+// sm: apply_gram_smem(n) bytes of shared memory; cmax: n entries.  Called by
+// every thread of the block.
 template <int TT>
-__global__ void __launch_bounds__(256) lr_apply_kernel(const float *x, const double *Xp, int64_t rows, float *q,
-                                                       __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo, int r,
-                                                       unsigned *amax, const int *skip2) {
-  pdl_enter();
-  if (skip2 != nullptr && *skip2) return;  // uniform over the grid
-  __shared__ unsigned cmax[16 * TT];
-  constexpr int n = 16 * TT, mld = apply_mld<TT>(), RT = kApplyRows / 8;
-  constexpr int JR = apply_rounds<TT>();
-  extern __shared__ __align__(16) uint8_t asm_[];
-  double *Ms = reinterpret_cast<double *>(asm_);        // [n][mld]
-  float *xs = reinterpret_cast<float *>(Ms + n * mld);  // [kApplyRows][xld]; reused as Q^T [n][kApplyRows + 1]
-  const int64_t r0 = (int64_t)blockIdx.x * kApplyRows;
-  apply_stage<TT>(x, Xp, rows, r0, kApplyRows, Ms, xs);
-  if (amax != nullptr)
-    for (int c = threadIdx.x; c < n; c += 256) cmax[c] = 0u;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  double acc[JR][RT][2];
-  apply_tiles<TT, RT>(xs, Ms, warp, lane, acc);
-  apply_store<TT, RT>(acc, r0, rows, q, qthi, qtlo, r, amax, cmax, xs, warp, lane);
-}
-
-// The first CholeskyQR pass's Q1 = X M for kGramRows rows per block, with the
-// sums of lr_apply_kernel (apply_tiles), and the partial Gram matrix Q1^T Q1
-// of these rows from the fp32 values it stores, with the sums of
-// lr_gram_kernel (gram_tiles): the second pass needs no Gram kernel, and both
-// results are bit-identical to the separate kernels'.  When the first pass's
-// factor kernel found the pass accurate enough (*skip2), Q1 is the sweep's Q:
-// the block writes the final pass's outputs instead (apply_store: Q, its
-// INT4 column maxima when amax != nullptr, Q^T split) and no Gram matrix.
-template <int TT>
-__global__ void __launch_bounds__(256) lr_apply_gram_kernel(const float *x, const double *Xp, int64_t rows, float *q,
-                                                            double *gpart, const int *skip2, __nv_bfloat16 *qthi,
-                                                            __nv_bfloat16 *qtlo, int r, unsigned *amax) {
-  pdl_enter();
-  __shared__ unsigned cmax[16 * TT];
+__device__ __forceinline__ void apply_phase(const float *x, const double *Xp, int64_t rows, int nblk, float *q,
+                                            double *gpart, bool final_q, __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo,
+                                            int r, unsigned *amax, uint8_t *sm, unsigned *cmax) {
   constexpr int n = 16 * TT, mld = apply_mld<TT>(), xld = apply_xld<TT>(), RT = kGramRows / 8;
   constexpr int JR = apply_rounds<TT>();
   static_assert(kGramRows * xld >= n * (kGramRows + 1), "the X tile holds the transposed Q tile");
-  extern __shared__ __align__(16) uint8_t asm_[];
-  double *Ms = reinterpret_cast<double *>(asm_);        // [n][mld]
+  double *Ms = reinterpret_cast<double *>(sm);          // [n][mld]
   float *xs = reinterpret_cast<float *>(Ms + n * mld);  // [kGramRows][xld]
   float *gs = xs + kGramRows * xld;                     // Q1 [kGramRows][gram_ld]
-  const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
-  const bool final_q = *skip2 != 0;                     // uniform over the grid
-  apply_stage<TT>(x, Xp, rows, r0, kGramRows, Ms, xs);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t4 = lane & 3;
+  if ((int)blockIdx.x >= nblk) return;  // uniform: no row block here
+  apply_stage_mx<TT>(Xp, Ms, x, rows, (int64_t)blockIdx.x * kGramRows, xs);
   if (final_q && amax != nullptr)
     for (int c = threadIdx.x; c < n; c += 256) cmax[c] = 0u;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t4 = lane & 3;
-  if (final_q) {
+  for (int rb = blockIdx.x; rb < nblk; rb += gridDim.x) {
+    const int64_t r0 = (int64_t)rb * kGramRows;
+    if (rb != (int)blockIdx.x) {
+      __syncthreads();  // the previous row block is done with xs and gs
+      apply_stage_x<TT>(x, rows, r0, kGramRows, xs);
+    }
+    __syncthreads();
     double acc[JR][RT][2];
     apply_tiles<TT, RT>(xs, Ms, warp, lane, acc);
-    apply_store<TT, RT>(acc, r0, rows, q, qthi, qtlo, r, amax, cmax, xs, warp, lane);
-    return;
-  }
-  {
-    double acc[JR][RT][2];
-    apply_tiles<TT, RT>(xs, Ms, warp, lane, acc);
+    if (final_q) {
+      apply_store<TT, RT>(acc, r0, rows, q, qthi, qtlo, r, amax, cmax, xs, warp, lane);
+      continue;
+    }
 #pragma unroll
     for (int jt = 0; jt < JR; jt++) {
       const int J = apply_ctile<TT>(warp, jt);
@@ -1040,9 +1039,111 @@ __global__ void __launch_bounds__(256) lr_apply_gram_kernel(const float *x, cons
         *reinterpret_cast<float2 *>(gs + (8 * i + gq) * gram_ld<TT>() + c) = v;
       }
     }
+    __syncthreads();
+    gram_tiles<TT>(gs, gpart + (int64_t)rb * n * n, warp, lane);
+  }
+}
+
+// ---- the orthonormalisation of one sweep as one persistent kernel
+//
+// CholeskyQR2 of the split-K partials of Y: the first pass (Gram matrix of X
+// = their sum, Cholesky factor, Q1 = X L^-T) and, unless the first pass
+// bounds kappa(X) by kSkipKappa, the second (the same on Q1).  Its phases
+// are separated by grid-wide barriers instead of kernel boundaries: the
+// Gram rows (every block), the reduction of the partial Gram matrices (every
+// block), the factor (block 0), the apply (every block), and so on.  All
+// blocks must be resident at once: the grid is at most the SMs times the
+// blocks that fit on one (checked on the host), and each barrier gives up
+// after spin_limit polls, reporting a timeout in *status.
+
+struct OrthoArgs {
+  const float *src;    // the split-K partials of Y [nsrc][rows][n]
+  int nsrc;
+  int64_t rows;
+  int nblk;            // row blocks of kGramRows rows
+  float *x;            // X = the sum of the partials [rows][n]
+  float *q;            // Q [rows][n]
+  double *gpart;       // partial Gram matrices [nblk][n][n]
+  double *L;           // reduced Gram matrix (row-major), then the packed factor L^-1
+  double *Gp;          // the reduced Gram matrix in packed tiles
+  int *dead, *skip2;
+  int nlive;           // the rank (columns nlive .. n-1 are padding)
+  double near_id;      // the second pass's first-order bound (lr_qr2_tol)
+  double kappa2_max;   // the skip test's bound on kappa^2 (0: never skip)
+  __nv_bfloat16 *qthi, *qtlo;
+  int r;
+  unsigned *amax;      // the INT4 column maxima of Q (nullptr: not the last sweep)
+  unsigned *gbar;      // this sweep's barrier counter, zero at launch
+  int *status;
+  uint32_t spin_limit;
+};
+
+template <int TT>
+struct OrthoShared {
+  int dead_s[16 * TT];
+  double gdiag[16 * TT];
+  double red[8];
+  double part[8][32];
+  unsigned cmax[16 * TT];
+  int ok;
+};
+
+// Grid-wide barrier number k (1, 2, ...) of the launch: every block adds one
+// to the counter and waits until it reaches k gridDim.x.  The block's writes
+// are ordered before its arrival by the block barrier and the release of the
+// add, and the other blocks' writes before everything after the wait by the
+// acquiring poll and the block barrier after it; data written by other blocks
+// is still read through L2 (ld.cg).  False (uniform over the block, after
+// the status is set) when the wait ran out.
+__device__ __forceinline__ bool ortho_sync(const OrthoArgs &A, unsigned k, int *ok) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(A.gbar) : "memory");
+    const unsigned target = k * gridDim.x;
+    int good = 0;
+    for (uint32_t it = 0; it < A.spin_limit; it++) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(A.gbar) : "memory");
+      if (v >= target) {
+        good = 1;
+        break;
+      }
+    }
+    if (!good) atomicOr(A.status, kStatusTimeout);
+    *ok = good;
   }
   __syncthreads();
-  gram_tiles<TT>(gs, gpart + (int64_t)blockIdx.x * n * n, warp, lane);
+  return *ok != 0;
+}
+
+template <int TT>
+__global__ void __launch_bounds__(256, 1) lr_ortho_kernel(const OrthoArgs A) {
+  pdl_enter();
+  constexpr int n = 16 * TT;
+  extern __shared__ __align__(16) uint8_t osm[];
+  __shared__ OrthoShared<TT> sh;
+  const int ngroups = (n * n + 31) / 32;
+  unsigned nb = 0;
+  // first pass: the Gram rows of X = sum of the partials
+  for (int rb = blockIdx.x; rb < A.nblk; rb += gridDim.x)
+    gram_rows<TT>(A.src, A.nsrc, A.rows, rb, A.x, A.gpart, reinterpret_cast<float *>(osm));
+  if (!ortho_sync(A, ++nb, &sh.ok)) return;
+  for (int g = blockIdx.x; g < ngroups; g += gridDim.x) reduce_group(A.gpart, A.nblk, n, A.L, A.Gp, g, sh.part);
+  if (!ortho_sync(A, ++nb, &sh.ok)) return;
+  if (blockIdx.x == 0)
+    chol_factor<TT>(A.L, A.Gp, A.L, A.dead, 0.0, A.nlive, A.skip2, 1, A.kappa2_max, osm, sh.dead_s, sh.gdiag, sh.red);
+  if (!ortho_sync(A, ++nb, &sh.ok)) return;
+  const bool final_q = __ldcg(A.skip2) != 0;  // uniform over the grid
+  apply_phase<TT>(A.x, A.L, A.rows, A.nblk, A.q, A.gpart, final_q, A.qthi, A.qtlo, A.r, A.amax, osm, sh.cmax);
+  if (final_q) return;
+  // second pass on Q1
+  if (!ortho_sync(A, ++nb, &sh.ok)) return;
+  for (int g = blockIdx.x; g < ngroups; g += gridDim.x) reduce_group(A.gpart, A.nblk, n, A.L, A.Gp, g, sh.part);
+  if (!ortho_sync(A, ++nb, &sh.ok)) return;
+  if (blockIdx.x == 0)
+    chol_factor<TT>(A.L, A.Gp, A.L, A.dead, A.near_id, A.nlive, A.skip2, 0, 0.0, osm, sh.dead_s, sh.gdiag, sh.red);
+  if (!ortho_sync(A, ++nb, &sh.ok)) return;
+  apply_phase<TT>(A.q, A.L, A.rows, A.nblk, A.q, nullptr, true, A.qthi, A.qtlo, A.r, A.amax, osm, sh.cmax);
 }
 
 // V = sum of the partial slabs (fixed order) [cols][n]; V_prev (state,
@@ -1545,13 +1646,17 @@ cudaError_t set_shared_smem_limits() {
   if (e != cudaSuccess) return e;
   return set_recon_smem((int)recon_smem(kMaxRank / kTileK, 1));
 }
-size_t apply_smem(int n) {  // n = 16 TT: apply_mld = apply_xld = n + 4
-  const size_t xt = (size_t)kApplyRows * (n + 4) * 4, qt = (size_t)n * (kApplyRows + 1) * 4;
-  return (size_t)n * (n + 4) * 8 + (xt > qt ? xt : qt);
-}
-size_t apply_gram_smem(int n) {  // gram_ld = n + 8
+size_t apply_gram_smem(int n) {  // n = 16 TT: apply_mld = apply_xld = n + 4, gram_ld = n + 8
   return (size_t)n * (n + 4) * 8 + (size_t)kGramRows * (n + 4) * 4 + (size_t)kGramRows * (n + 8) * 4;
 }
+// Dynamic shared memory of the orthonormalisation kernel: its phases use the
+// same buffer (the Gram tile, the Cholesky tiles, the apply operands).
+size_t ortho_smem(int n) {
+  const size_t a = apply_gram_smem(n), c = chol_smem_tt(n / 16), g = (size_t)kGramRows * (n + 8) * 4;
+  return a > c ? (a > g ? a : g) : (c > g ? c : g);
+}
+// Polls of a grid barrier of the orthonormalisation kernel before it gives up.
+constexpr uint32_t kOrthoSpinLimit = 1u << 20;
 
 }  // namespace
 
@@ -1604,6 +1709,7 @@ void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *p
   enc += pad256(mx * rp * 4) * 2 + pad256(C * rp * 4);        // xbuf, q, v
   enc += pad256((size_t)plan->nblk_gram * rp * rp * 8);       // gpart
   enc += pad256(rp * rp * 8) + pad256(rp * 4) + pad256(4);    // L, dead, skip flag
+  enc += pad256(2 * 4);                                       // barrier counters of the two sweeps
   enc += pad256(gpk_bytes(rp));                                // G in packed tiles
   enc += pad256(2 * rp * 4);                                  // amax
   plan->enc_scratch_bytes = enc;
@@ -1612,27 +1718,32 @@ void lowrank_plan(int64_t rows, int64_t cols, const cf_params &p, LowrankPlan *p
 
 namespace {
 
+// The orthonormalisation kernel's shared-memory limit (one value per TT, so
+// states of different ranks do not interfere) and the largest grid whose
+// blocks are all resident at once.
 template <int TT>
-cudaError_t set_apply_smem_tt() {
-  cudaError_t e = cudaFuncSetAttribute(lr_apply_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)apply_smem(16 * TT));
+cudaError_t set_ortho_tt(int *resident) {
+  const int sm = (int)ortho_smem(16 * TT);
+  cudaError_t e = cudaFuncSetAttribute(lr_ortho_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(lr_apply_gram_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)apply_gram_smem(16 * TT));
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(lr_chol_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)chol_smem_tt(TT));
+  int occ = 0, nsm = 0, dev = 0;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, lr_ortho_kernel<TT>, 256, sm)) != cudaSuccess) return e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  *resident = occ * nsm;
+  return occ > 0 ? cudaSuccess : cudaErrorInvalidConfiguration;
 }
 
-cudaError_t set_apply_smem(int n) {
+cudaError_t set_ortho(int n, int *resident) {
   switch (n / 16) {
-    case 1: return set_apply_smem_tt<1>();
-    case 2: return set_apply_smem_tt<2>();
-    case 3: return set_apply_smem_tt<3>();
-    case 4: return set_apply_smem_tt<4>();
-    case 5: return set_apply_smem_tt<5>();
-    case 6: return set_apply_smem_tt<6>();
-    case 7: return set_apply_smem_tt<7>();
-    case 8: return set_apply_smem_tt<8>();
+    case 1: return set_ortho_tt<1>(resident);
+    case 2: return set_ortho_tt<2>(resident);
+    case 3: return set_ortho_tt<3>(resident);
+    case 4: return set_ortho_tt<4>(resident);
+    case 5: return set_ortho_tt<5>(resident);
+    case 6: return set_ortho_tt<6>(resident);
+    case 7: return set_ortho_tt<7>(resident);
+    case 8: return set_ortho_tt<8>(resident);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1671,6 +1782,7 @@ int lowrank_bind(LowrankPlan *plan, void *scratch) {
     b.L = reinterpret_cast<double *>(take(rp * rp * 8));
     b.dead = reinterpret_cast<int *>(take(rp * 4));
     b.skip2 = reinterpret_cast<int *>(take(4));
+    b.gbar = reinterpret_cast<unsigned *>(take(2 * 4));
     b.gpk = reinterpret_cast<double *>(take(gpk_bytes(rp)));
     b.amax = reinterpret_cast<unsigned *>(take(2 * rp * 4));
     ok = ok && make_map(&plan->tm_dhi, b.dhi, C, R, kTileM) && make_map(&plan->tm_dlo, b.dlo, C, R, kTileM) &&
@@ -1680,11 +1792,13 @@ int lowrank_bind(LowrankPlan *plan, void *scratch) {
   }
   if (!ok) return CF_ERR_CUDA;
   // kernels that need more than 48 KiB of dynamic shared memory
-  const int rpi = plan->rp;
-  if (set_shared_smem_limits() != cudaSuccess || set_apply_smem(rpi) != cudaSuccess) {
+  int resident = 0;
+  if (set_shared_smem_limits() != cudaSuccess || set_ortho(plan->rp, &resident) != cudaSuccess) {
     (void)cudaGetLastError();
     return CF_ERR_CUDA;
   }
+  const int nblk = (int)(plan->rows / kGramRows);
+  plan->ortho_grid = nblk < resident ? nblk : resident;
   return CF_OK;
 }
 
@@ -1708,96 +1822,49 @@ cudaError_t launch_thin(const LowrankPlan &P, const CUtensorMap &ah, const CUten
   return cudaGetLastError();
 }
 
-cudaError_t launch_gram(int n, int nblk, const float *src, int nsrc, int64_t rows, float *x, double *gpart,
-                        cudaStream_t st) {
-  switch (n / 16) {
-    case 1: launch_pdl(lr_gram_kernel<1>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
-    case 2: launch_pdl(lr_gram_kernel<2>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
-    case 3: launch_pdl(lr_gram_kernel<3>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
-    case 4: launch_pdl(lr_gram_kernel<4>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
-    case 5: launch_pdl(lr_gram_kernel<5>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
-    case 6: launch_pdl(lr_gram_kernel<6>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
-    case 7: launch_pdl(lr_gram_kernel<7>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
-    case 8: launch_pdl(lr_gram_kernel<8>, dim3(nblk), dim3(256), 0, st, src, nsrc, rows, x, gpart); break;
-    default: return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_chol(int n, double *L, const double *Gp, int *dead, double near_id, int nlive, int *skip2,
-                        int first_pass, double kappa2_max, cudaStream_t st) {
-  switch (n / 16) {
-    case 1: launch_pdl(lr_chol_kernel<1>, dim3(1), dim3(256), chol_smem_tt(1), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 2: launch_pdl(lr_chol_kernel<2>, dim3(1), dim3(256), chol_smem_tt(2), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 3: launch_pdl(lr_chol_kernel<3>, dim3(1), dim3(256), chol_smem_tt(3), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 4: launch_pdl(lr_chol_kernel<4>, dim3(1), dim3(256), chol_smem_tt(4), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 5: launch_pdl(lr_chol_kernel<5>, dim3(1), dim3(256), chol_smem_tt(5), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 6: launch_pdl(lr_chol_kernel<6>, dim3(1), dim3(256), chol_smem_tt(6), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 7: launch_pdl(lr_chol_kernel<7>, dim3(1), dim3(256), chol_smem_tt(7), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    case 8: launch_pdl(lr_chol_kernel<8>, dim3(1), dim3(256), chol_smem_tt(8), st, L, Gp, L, dead, near_id, nlive, skip2, first_pass, kappa2_max); break;
-    default: return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_apply(int n, const float *x, const double *M, int64_t rows, float *q, __nv_bfloat16 *qthi,
-                         __nv_bfloat16 *qtlo, int r, unsigned *amax, const int *skip2, cudaStream_t st) {
-  const unsigned grid = (unsigned)((rows + kApplyRows - 1) / kApplyRows);
-  const size_t sm = apply_smem(n);
-  switch (n / 16) {
-    case 1: launch_pdl(lr_apply_kernel<1>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
-    case 2: launch_pdl(lr_apply_kernel<2>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
-    case 3: launch_pdl(lr_apply_kernel<3>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
-    case 4: launch_pdl(lr_apply_kernel<4>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
-    case 5: launch_pdl(lr_apply_kernel<5>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
-    case 6: launch_pdl(lr_apply_kernel<6>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
-    case 7: launch_pdl(lr_apply_kernel<7>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
-    case 8: launch_pdl(lr_apply_kernel<8>, dim3(grid), dim3(256), sm, st, x, M, rows, q, qthi, qtlo, r, amax, skip2); break;
-    default: return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_apply_gram(int n, const float *x, const double *M, int64_t rows, float *q, double *gpart,
-                              const int *skip2, __nv_bfloat16 *qthi, __nv_bfloat16 *qtlo, int r, unsigned *amax,
-                              cudaStream_t st) {
-  const unsigned grid = (unsigned)(rows / kGramRows);
-  const size_t sm = apply_gram_smem(n);
-  switch (n / 16) {
-    case 1: launch_pdl(lr_apply_gram_kernel<1>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
-    case 2: launch_pdl(lr_apply_gram_kernel<2>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
-    case 3: launch_pdl(lr_apply_gram_kernel<3>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
-    case 4: launch_pdl(lr_apply_gram_kernel<4>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
-    case 5: launch_pdl(lr_apply_gram_kernel<5>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
-    case 6: launch_pdl(lr_apply_gram_kernel<6>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
-    case 7: launch_pdl(lr_apply_gram_kernel<7>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
-    case 8: launch_pdl(lr_apply_gram_kernel<8>, dim3(grid), dim3(256), sm, st, x, M, rows, q, gpart, skip2, qthi, qtlo, r, amax); break;
-    default: return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
-}
-
-cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int64_t rows, bool final_pass,
-                           unsigned *amax, cudaStream_t st) {
+// One sweep's CholeskyQR2 of Y (its split-K partials src) into Q: one
+// launch of the persistent orthonormalisation kernel, whose first pass
+// decides whether the second one runs (lr_qr2_tol = 0: always, the full
+// CholeskyQR2).
+cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int sweep, unsigned *amax, int *status,
+                           cudaStream_t st) {
   const LowrankBufs &b = P.b;
-  const int n = P.rp;
-  const int nblk = (int)(rows / kGramRows);
-  cudaError_t e = cudaSuccess;
-  // the first pass's partial Gram matrices come from the Gram kernel (over the
-  // split-K partials of Y), the second pass's from the first pass's apply
-  if (!final_pass && (e = launch_gram(n, nblk, src, nsrc, rows, b.xbuf, b.gpart, st)) != cudaSuccess) return e;
-  // the reduced Gram matrix goes to L (row-major) and gpk (packed tiles);
-  // the Cholesky kernel then overwrites L with X = L^-1 in packed tiles; the
-  // first pass decides whether the second one runs (lr_qr2_tol = 0: always,
-  // the full CholeskyQR2)
-  launch_pdl(lr_gram_reduce_kernel, dim3((unsigned)((n * n + 31) / 32)), dim3(256), 0, st, b.gpart, nblk, n, b.L,
-             b.gpk, final_pass ? b.skip2 : nullptr);
-  const double kappa2_max = P.qr2_tol > 0.0 ? kSkipKappa * kSkipKappa : 0.0;
-  e = launch_chol(n, b.L, b.gpk, b.dead, final_pass ? P.qr2_tol : 0.0, P.rank, b.skip2, final_pass ? 0 : 1,
-                  kappa2_max, st);
-  if (e != cudaSuccess) return e;
-  if (!final_pass) return launch_apply_gram(n, b.xbuf, b.L, rows, b.q, b.gpart, b.skip2, b.qthi, b.qtlo, P.rank, amax, st);
-  return launch_apply(n, b.q, b.L, rows, b.q, b.qthi, b.qtlo, P.rank, amax, b.skip2, st);
+  OrthoArgs A{};
+  A.src = src;
+  A.nsrc = nsrc;
+  A.rows = P.rows;
+  A.nblk = (int)(P.rows / kGramRows);
+  A.x = b.xbuf;
+  A.q = b.q;
+  A.gpart = b.gpart;
+  A.L = b.L;
+  A.Gp = b.gpk;
+  A.dead = b.dead;
+  A.skip2 = b.skip2;
+  A.nlive = P.rank;
+  A.near_id = P.qr2_tol;
+  A.kappa2_max = P.qr2_tol > 0.0 ? kSkipKappa * kSkipKappa : 0.0;
+  A.qthi = b.qthi;
+  A.qtlo = b.qtlo;
+  A.r = P.rank;
+  A.amax = amax;
+  A.gbar = b.gbar + sweep;
+  A.status = status;
+  A.spin_limit = kOrthoSpinLimit;
+  const dim3 grid((unsigned)P.ortho_grid);
+  const size_t sm = ortho_smem(P.rp);
+  switch (P.rp / 16) {
+    case 1: launch_pdl(lr_ortho_kernel<1>, grid, dim3(256), sm, st, A); break;
+    case 2: launch_pdl(lr_ortho_kernel<2>, grid, dim3(256), sm, st, A); break;
+    case 3: launch_pdl(lr_ortho_kernel<3>, grid, dim3(256), sm, st, A); break;
+    case 4: launch_pdl(lr_ortho_kernel<4>, grid, dim3(256), sm, st, A); break;
+    case 5: launch_pdl(lr_ortho_kernel<5>, grid, dim3(256), sm, st, A); break;
+    case 6: launch_pdl(lr_ortho_kernel<6>, grid, dim3(256), sm, st, A); break;
+    case 7: launch_pdl(lr_ortho_kernel<7>, grid, dim3(256), sm, st, A); break;
+    case 8: launch_pdl(lr_ortho_kernel<8>, grid, dim3(256), sm, st, A); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
 }
 
 PackArgs pack_args(const LowrankPlan &P, uint8_t *payload, const Header &hdr) {
@@ -1893,6 +1960,7 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
   V.vthi = b.vthi;
   V.vtlo = b.vtlo;
   V.amax = b.amax;
+  V.gbar = b.gbar;
   const dim3 dg((unsigned)(P.rp + (C / 64) * (R / 64)));
   if (P.dtype == CF_BF16)
     launch_pdl(lr_delta_kernel<__nv_bfloat16>, dim3(dg), dim3(256), 0, st, static_cast<const __nv_bfloat16 *>(args.a),
@@ -1914,8 +1982,7 @@ cudaError_t lowrank_encode(const LowrankPlan &P, const EncArgs &args, const PtrT
     unsigned *amax_q = (P.int4 && !more) ? b.amax : nullptr;
     unsigned *amax_v = (P.int4 && !more) ? b.amax + P.rp : nullptr;
     // Q = orth(Y): CholeskyQR2
-    if ((e = orthonormalise(P, b.ypart, P.sy, R, false, amax_q, st)) != cudaSuccess) return e;
-    if ((e = orthonormalise(P, b.q, 1, R, true, amax_q, st)) != cudaSuccess) return e;
+    if ((e = orthonormalise(P, b.ypart, P.sy, it, amax_q, args.status, st)) != cudaSuccess) return e;
     // V = D^T Q
     if ((e = launch_thin(P, P.tm_dmhi, P.tm_dmlo, P.tm_qthi, P.tm_qtlo, b.vpart, C, R, P.sv, args.status, st, true,
                          2)) !=

@@ -25,6 +25,7 @@ struct LowrankBufs {
   double *L = nullptr;                             // Cholesky factor [rp][rp]
   int *dead = nullptr;                             // rank-deficient column flags [rp]
   int *skip2 = nullptr;                            // the sweep's first CholeskyQR pass suffices (set on the device)
+  unsigned *gbar = nullptr;                        // grid-barrier counters of the two sweeps' orthonormalisation
   double *gpk = nullptr;                           // G in the Cholesky kernel's packed 8 x 8 tile layout
   unsigned *amax = nullptr;                        // column absmax bit patterns of Q [rp] and V [rp]
   // both roles: reconstruction operands dequantised from the payload
@@ -40,6 +41,7 @@ struct LowrankPlan {
   uint32_t test_wait_polls = 0;  // test hook: > 0 makes the reconstruction's operand wait run out
   int sy = 1, sv = 1;            // split-K factors of the two thin GEMMs
   int nblk_gram = 1;             // row blocks of the partial Gram matrices
+  int ortho_grid = 1;            // blocks of the orthonormalisation kernel (all resident at once)
   size_t enc_scratch_bytes = 0;
   size_t dec_scratch_bytes = 0;
   bool supported = false;
