@@ -1076,6 +1076,7 @@ struct OrthoArgs {
   unsigned *gbar;      // this sweep's barrier counter, zero at launch
   int *status;
   uint32_t spin_limit;
+  int withhold_arrival;  // test hook: block 0 does not arrive at the first barrier, so every block's wait runs out
 };
 
 template <int TT>
@@ -1098,7 +1099,8 @@ struct OrthoShared {
 __device__ __forceinline__ bool ortho_sync(const OrthoArgs &A, unsigned k, int *ok) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(A.gbar) : "memory");
+    if (!(A.withhold_arrival && k == 1 && blockIdx.x == 0))
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(A.gbar) : "memory");
     const unsigned target = k * gridDim.x;
     int good = 0;
     for (uint32_t it = 0; it < A.spin_limit; it++) {
@@ -1850,7 +1852,8 @@ cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int
   A.amax = amax;
   A.gbar = b.gbar + sweep;
   A.status = status;
-  A.spin_limit = kOrthoSpinLimit;
+  A.spin_limit = P.test_wait_polls ? P.test_wait_polls : kOrthoSpinLimit;
+  A.withhold_arrival = P.test_wait_polls != 0;
   const dim3 grid((unsigned)P.ortho_grid);
   const size_t sm = ortho_smem(P.rp);
   switch (P.rp / 16) {

@@ -247,7 +247,11 @@ CF_API int cf_reset(cf_state *s);
  * wait gives up: the kernel records the timeout in the state's status word
  * (cf_status then returns CF_ERR_TIMEOUT), frees its tensor memory and
  * returns without writing ahat, e or recon.  No copy or MMA is left in
- * flight.  polls = 0 restores normal operation; cf_reset clears the status.
+ * flight.  In a sender's encode the orthonormalisation kernel's first
+ * grid-wide barrier is made to run out as well (one block withholds its
+ * arrival; every block waits at most `polls` polls, records the timeout and
+ * returns before Q is formed, so the payload's U scales stay zero).
+ * polls = 0 restores normal operation; cf_reset clears the status.
  * Returns CF_ERR_UNSUPPORTED for the other modes. */
 CF_API int cf_test_wait_timeout(cf_state *s, uint32_t polls);
 

@@ -63,8 +63,12 @@ def test_lowrank_bounded_wait_runs_out(role):
     made to run out by the test hook (no copy is issued, so nothing is in flight;
     a limit of 256 polls): the kernel returns, cf_status reports CF_ERR_TIMEOUT
     for that state only, and the state it would have updated (receiver: ahat and
-    recon; sender: ahat and e) is unchanged.  With the hook off and both states
-    reset, a clean request runs and reports no error."""
+    recon; sender: ahat and e) is unchanged.  In the sender's encode the
+    orthonormalisation kernel's first grid barrier runs out as well (one block
+    withholds its arrival): every block leaves before Q is formed, so the U
+    scales of the payload stay zero (the column maxima are zeroed at the start
+    of each encode).  With the hook off and both states reset, a clean request
+    runs and reports no error."""
     rows, cols = 256, 256
     pair = GpuPair(rows, cols, "lowrank", dtype="bf16", rank=16, iters=1, lr_int4=1, seed=3)
     s = inputs.ar1("cuda", rows=rows, cols=cols)
@@ -83,6 +87,11 @@ def test_lowrank_bounded_wait_runs_out(role):
             cf.cf_decode(pair.R, pair.payload, pair.recon)
         assert cf.cf_status(hooked) == cf.CF_ERR_TIMEOUT
         assert cf.cf_status(other) == cf.CF_OK
+        u_scales = to_np(pair.payload[64:64 + 4 * 16]).view(np.float32)  # header, then the r U scales
+        if role == "sender":
+            assert np.all(u_scales == 0.0), u_scales
+        else:
+            assert np.all(u_scales > 0.0), u_scales
         after = pair.state(which)
         assert np.array_equal(before[0].view(np.uint32), after[0].view(np.uint32))
         if role == "sender":
