@@ -40,8 +40,8 @@ def _teacher_force(orc, pair, a_np, step):
     return orc.encode(a_np)
 
 
-def _lr_pair(rows, cols, rank, iters, int4, dtype="bf16", seed=7):
-    return GpuPair(rows, cols, "lowrank", dtype=dtype, rank=rank, iters=iters, lr_int4=int4, seed=seed)
+def _lr_pair(rows, cols, rank, iters, int4, dtype="bf16", seed=7, **extra):
+    return GpuPair(rows, cols, "lowrank", dtype=dtype, rank=rank, iters=iters, lr_int4=int4, seed=seed, **extra)
 
 
 @pytest.mark.parametrize("rows,cols", [(256, 128), (384, 128)])
@@ -95,7 +95,23 @@ def test_exact_rank_r_residual_is_recovered():
     # fp32 activations
     (512, 384, 40, 1, "f32")])
 def test_teacher_forced_matches_oracle(rows, cols, rank, iters, dtype):
-    pair = _lr_pair(rows, cols, rank, iters, 1, dtype=dtype)
+    _teacher_forced_run(rows, cols, rank, iters, dtype)
+
+
+@pytest.mark.parametrize("iters,qr2_tol", [(1, None), (2, None), (1, 0.0)])
+def test_teacher_forced_more_row_blocks_than_blocks(iters, qr2_tol):
+    """6144 rows make 192 row blocks of 32 for the orthonormalisation kernel,
+    more than its grid (one block per SM, all resident), so its blocks loop
+    over two row blocks in the Gram and apply phases (the factor staged once,
+    the rows of X restaged per row block); with lr_qr2_tol = 0 the second
+    CholeskyQR pass (reduction, elimination, apply over the same loops) runs
+    at every step.  Same gates as the teacher-forced test above."""
+    extra = {} if qr2_tol is None else {"lr_qr2_tol": qr2_tol}
+    _teacher_forced_run(6144, 256, 40, iters, "bf16", **extra)
+
+
+def _teacher_forced_run(rows, cols, rank, iters, dtype, **extra):
+    pair = _lr_pair(rows, cols, rank, iters, 1, dtype=dtype, **extra)
     orc = oracle.Oracle(rows, cols, "lowrank", dtype=dtype, rank=rank, iters=iters, lr_int4=1, seed=7)
     s = inputs.ar1("cuda", rows=rows, cols=cols)
     if dtype == "f32":
