@@ -1857,14 +1857,14 @@ cudaError_t orthonormalise(const LowrankPlan &P, const float *src, int nsrc, int
   const dim3 grid((unsigned)P.ortho_grid);
   const size_t sm = ortho_smem(P.rp);
   switch (P.rp / 16) {
-    case 1: launch_pdl(lr_ortho_kernel<1>, grid, dim3(256), sm, st, A); break;
-    case 2: launch_pdl(lr_ortho_kernel<2>, grid, dim3(256), sm, st, A); break;
-    case 3: launch_pdl(lr_ortho_kernel<3>, grid, dim3(256), sm, st, A); break;
-    case 4: launch_pdl(lr_ortho_kernel<4>, grid, dim3(256), sm, st, A); break;
-    case 5: launch_pdl(lr_ortho_kernel<5>, grid, dim3(256), sm, st, A); break;
-    case 6: launch_pdl(lr_ortho_kernel<6>, grid, dim3(256), sm, st, A); break;
-    case 7: launch_pdl(lr_ortho_kernel<7>, grid, dim3(256), sm, st, A); break;
-    case 8: launch_pdl(lr_ortho_kernel<8>, grid, dim3(256), sm, st, A); break;
+    case 1: launch_pdl_coop(lr_ortho_kernel<1>, grid, dim3(256), sm, st, A); break;
+    case 2: launch_pdl_coop(lr_ortho_kernel<2>, grid, dim3(256), sm, st, A); break;
+    case 3: launch_pdl_coop(lr_ortho_kernel<3>, grid, dim3(256), sm, st, A); break;
+    case 4: launch_pdl_coop(lr_ortho_kernel<4>, grid, dim3(256), sm, st, A); break;
+    case 5: launch_pdl_coop(lr_ortho_kernel<5>, grid, dim3(256), sm, st, A); break;
+    case 6: launch_pdl_coop(lr_ortho_kernel<6>, grid, dim3(256), sm, st, A); break;
+    case 7: launch_pdl_coop(lr_ortho_kernel<7>, grid, dim3(256), sm, st, A); break;
+    case 8: launch_pdl_coop(lr_ortho_kernel<8>, grid, dim3(256), sm, st, A); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

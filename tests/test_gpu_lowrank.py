@@ -505,3 +505,50 @@ def test_encode_captured_into_a_caller_graph():
     finally:
         direct.close()
         captured.close()
+
+
+def test_concurrent_encodes_on_two_streams():
+    """Two low-rank pairs stepping at once on two streams.  The orthonormalisation
+    kernel's blocks wait for one another at grid-wide barriers, and at 4096 rows
+    its grid takes 128 SMs, so two such grids cannot be resident together: each
+    is launched cooperatively (it starts only when all its blocks fit), so
+    neither waits for blocks the other holds.  Both pairs report no error, and
+    each pair's payloads and states equal those of the same stream run alone."""
+    rows, cols = 4096, 256
+    steps = 5
+
+    def stream_of(seed):
+        s = inputs.ar1("cuda", rows=rows, cols=cols, seed=seed)
+        return [s.next() for _ in range(steps)]
+
+    acts = [stream_of(11), stream_of(12)]
+    # reference: each pair alone, one after the other
+    ref = []
+    for i in range(2):
+        pair = _lr_pair(rows, cols, 40, 1, 1, seed=5 + i)
+        try:
+            pays = []
+            for t in range(steps):
+                pair.step(acts[i][t])
+                torch.cuda.synchronize()
+                pays.append(pair.payload_np(t == 0).copy())
+            ref.append((pays, pair.state("S")[0].copy()))
+        finally:
+            pair.close()
+    # the same two streams, interleaved on two CUDA streams without waiting
+    pairs = [_lr_pair(rows, cols, 40, 1, 1, seed=5 + i) for i in range(2)]
+    cs = [torch.cuda.Stream(), torch.cuda.Stream()]
+    try:
+        for t in range(steps):
+            for i in range(2):
+                with torch.cuda.stream(cs[i]):
+                    pairs[i].step(acts[i][t], cs[i])
+            torch.cuda.synchronize()
+            for i in range(2):
+                assert np.array_equal(pairs[i].payload_np(t == 0), ref[i][0][t]), (i, t)
+        for i in range(2):
+            assert cf.cf_status(pairs[i].S) == cf.CF_OK and cf.cf_status(pairs[i].R) == cf.CF_OK
+            assert np.array_equal(pairs[i].state("S")[0].view(np.uint32), ref[i][1].view(np.uint32))
+    finally:
+        for p in pairs:
+            p.close()
