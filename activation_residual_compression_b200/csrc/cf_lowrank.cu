@@ -443,7 +443,7 @@ __device__ __forceinline__ void gram_rows(const float *src, int nsrc, int64_t ro
   gram_tiles<TT>(tile, gpart + (int64_t)rb * n * n, threadIdx.x >> 5, threadIdx.x & 31);
 }
 
-// Offset of entry (i, j), j <= i, in the Cholesky kernel's packed array of
+// Offset of entry (i, j), j <= i, in the Cholesky factor's packed array of
 // 8 x 8 tiles (tile (I, J), J <= I, at I (I + 1) / 2 + J; rows of kCholTld
 // doubles).
 constexpr int kCholTld = 9;  // tile row stride (doubles): a half-warp's 4 x 4 fragment in distinct banks
@@ -530,9 +530,9 @@ __device__ __forceinline__ void reduce_group(const double *gpart, int nblk, int 
 // of X) are zero and the column updates nothing; the other columns are the
 // Cholesky factor of G restricted to them.
 //
-// The factor leaves the kernel as X in the same packed tile layout (all
+// The factor leaves shared memory as X in the same packed tile layout (all
 // chol_ntiles tiles, those past the live ones zero): a flat copy here, and
-// the apply kernels stage M = X^T from it.
+// the apply phase stages M = X^T from it.
 
 template <int TT>
 __host__ __device__ constexpr int chol_ntiles() {
@@ -1609,7 +1609,7 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, 
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-// Bytes of G in the Cholesky kernel's packed layout: the lower 8 x 8 tiles of
+// Bytes of G in the Cholesky factor's packed layout: the lower 8 x 8 tiles of
 // an rp x rp matrix, rows of kCholTld doubles.
 size_t gpk_bytes(size_t rp) { return (rp / 8) * (rp / 8 + 1) / 2 * 8 * kCholTld * 8; }
 

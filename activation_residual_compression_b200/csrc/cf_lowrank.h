@@ -26,7 +26,7 @@ struct LowrankBufs {
   int *dead = nullptr;                             // rank-deficient column flags [rp]
   int *skip2 = nullptr;                            // the sweep's first CholeskyQR pass suffices (set on the device)
   unsigned *gbar = nullptr;                        // grid-barrier counters of the two sweeps' orthonormalisation
-  double *gpk = nullptr;                           // G in the Cholesky kernel's packed 8 x 8 tile layout
+  double *gpk = nullptr;                           // G in the Cholesky factor's packed 8 x 8 tile layout
   unsigned *amax = nullptr;                        // column absmax bit patterns of Q [rp] and V [rp]
   // both roles: reconstruction operands dequantised from the payload
   __nv_bfloat16 *uahi = nullptr, *ualo = nullptr;  // [rows][kp]
