@@ -401,12 +401,7 @@ __device__ __forceinline__ void gram_rows(const float *src, int nsrc, int64_t ro
   const float4 *s4 = reinterpret_cast<const float4 *>(src) + r0 * n4;
   const int64_t slab4 = rows * n4;
   float4 acc4[NV];
-#pragma unroll
-  for (int v = 0; v < NV; v++) {
-    const int e = threadIdx.x + 256 * v;
-    acc4[v] = e < kGramRows * n4 ? __ldcg(s4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int p0 = 1; p0 < nsrc; p0 += 4) {  // four slabs' loads in flight, added in slab order
+  for (int p0 = 0; p0 < nsrc; p0 += 4) {  // four slabs' loads in flight, added in slab order
     float4 t[4][NV];
 #pragma unroll
     for (int u = 0; u < 4; u++)
@@ -421,10 +416,14 @@ __device__ __forceinline__ void gram_rows(const float *src, int nsrc, int64_t ro
       if (p0 + u >= nsrc) break;
 #pragma unroll
       for (int v = 0; v < NV; v++) {
-        acc4[v].x = __fadd_rn(acc4[v].x, t[u][v].x);
-        acc4[v].y = __fadd_rn(acc4[v].y, t[u][v].y);
-        acc4[v].z = __fadd_rn(acc4[v].z, t[u][v].z);
-        acc4[v].w = __fadd_rn(acc4[v].w, t[u][v].w);
+        if (p0 + u == 0) {
+          acc4[v] = t[0][v];
+        } else {
+          acc4[v].x = __fadd_rn(acc4[v].x, t[u][v].x);
+          acc4[v].y = __fadd_rn(acc4[v].y, t[u][v].y);
+          acc4[v].z = __fadd_rn(acc4[v].z, t[u][v].z);
+          acc4[v].w = __fadd_rn(acc4[v].w, t[u][v].w);
+        }
       }
     }
   }
@@ -944,6 +943,7 @@ __device__ __forceinline__ void apply_store(const double (&acc)[apply_rounds<TT>
 #pragma unroll
   for (int jt = 0; jt < JR; jt++) {
     const int J = apply_ctile<TT>(warp, jt);
+    uint32_t m0 = 0u, m1 = 0u;  // this lane's column maxima over its rows (bit patterns of |Q| >= 0)
 #pragma unroll
     for (int i = 0; i < RT; i++) {
       res[jt][i][0] = (float)acc[jt][i][0];
@@ -952,10 +952,21 @@ __device__ __forceinline__ void apply_store(const double (&acc)[apply_rounds<TT>
       if (J >= 0 && row < rows) {
         const int c = 8 * J + 2 * t4;
         *reinterpret_cast<float2 *>(q + row * n + c) = make_float2(res[jt][i][0], res[jt][i][1]);
-        if (amax != nullptr) {  // the INT4 column maxima of Q (non-negative bit patterns)
-          atomicMax(&cmax[c], __float_as_uint(fabsf(res[jt][i][0])));
-          atomicMax(&cmax[c + 1], __float_as_uint(fabsf(res[jt][i][1])));
-        }
+        m0 = max(m0, __float_as_uint(fabsf(res[jt][i][0])));
+        m1 = max(m1, __float_as_uint(fabsf(res[jt][i][1])));
+      }
+    }
+    if (amax != nullptr && J >= 0) {  // uniform over the warp: the INT4 column maxima of Q
+      // the 8 lanes of a column pair (lane bits 2-4) first, then one shared atomic per column and warp
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        m0 = max(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+        m1 = max(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+      }
+      if (gq == 0) {
+        const int c = 8 * J + 2 * t4;
+        atomicMax(&cmax[c], m0);
+        atomicMax(&cmax[c + 1], m1);
       }
     }
   }
@@ -1164,14 +1175,14 @@ __global__ void __launch_bounds__(256) lr_vsum_kernel(const float *vpart, int ns
   }
   const int64_t total = cols * n;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
-    float acc = vpart[idx];
-    for (int p0 = 1; p0 < nsrc; p0 += 4) {  // four slabs' loads in flight, added in slab order
-      float t[4];
+    float acc = 0.0f;
+    for (int p0 = 0; p0 < nsrc; p0 += 8) {  // eight slabs' loads in flight, added in slab order
+      float t[8];
 #pragma unroll
-      for (int u = 0; u < 4; u++) t[u] = p0 + u < nsrc ? vpart[(int64_t)(p0 + u) * total + idx] : 0.0f;
+      for (int u = 0; u < 8; u++) t[u] = p0 + u < nsrc ? vpart[(int64_t)(p0 + u) * total + idx] : 0.0f;
 #pragma unroll
-      for (int u = 0; u < 4; u++)
-        if (p0 + u < nsrc) acc = __fadd_rn(acc, t[u]);
+      for (int u = 0; u < 8; u++)
+        if (p0 + u < nsrc) acc = p0 + u == 0 ? t[0] : __fadd_rn(acc, t[u]);
     }
     const uint32_t j = (uint32_t)idx / (uint32_t)n;
     const int k = (int)((uint32_t)idx - j * (uint32_t)n);
