@@ -265,8 +265,9 @@ def launches_per_call(mode, kw, encode):
         return 1
     if not encode:
         return 2                                   # dequantise, reconstruction
-    return 1 + 10 * kw["iters"] + 2                # residual with the V preparation; per sweep: 2 GEMMs, Gram,
-                                                   # 2 x (reduce, Cholesky, apply), V sum; pack, reconstruction
+    return 1 + 4 * kw["iters"] + 2                 # residual with the V preparation; per sweep: 2 GEMMs, the
+                                                   # orthonormalisation (one persistent kernel), V sum; pack,
+                                                   # reconstruction
 
 
 def run_cf(args, rank, world, device):
