@@ -75,7 +75,20 @@ cudaError_t launch(const void *fn, int grid, size_t smem, const Args &args, cons
   if (grid < 1) grid = 1;
   NoTable none;
   void *params[2] = {const_cast<Args *>(&args), tab ? const_cast<PtrTable *>(tab) : static_cast<void *>(&none)};
-  return cudaLaunchKernel(fn, dim3(grid), dim3(kBlock), params, smem, st);
+  // programmatic dependent launch: the kernel may be scheduled while the
+  // previous kernel of the stream drains (it waits for it before any memory
+  // access, pdl_enter), which hides the launch gap between back-to-back calls
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kBlock);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, params);
 }
 
 int occupancy(const void *fn, size_t smem) {

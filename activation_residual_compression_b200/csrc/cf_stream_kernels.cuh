@@ -32,6 +32,7 @@
 #include <cstdint>
 
 #include "cf_internal.h"
+#include "cf_launch.cuh"
 
 // Resident blocks per SM the compiler must allow (register budget), measured
 // on B200: the decode kernels take 4 for N:M with two kept values per block
@@ -644,6 +645,7 @@ __global__ void __launch_bounds__(kBlock, EncMinBlocks<MODE, VPT>::value) encode
   const int64_t nrows = (int64_t)A.batch * A.rows;
   const int64_t n_rg = (nrows + tpb - 1) / tpb;
 
+  pdl_enter();  // every global access below follows the previous kernel of the stream
   if (blockIdx.x == 0 && threadIdx.x < 16) reinterpret_cast<uint32_t *>(A.payload)[threadIdx.x] = A.hdr.w[threadIdx.x];
   zero_padding(A);
 
@@ -835,6 +837,7 @@ struct DecMinBlocks {
 
 template <int MODE, typename T, int VPT, int NM_M, int NM_N, typename Tab, typename S = float>
 __global__ void __launch_bounds__(kBlock, DecMinBlocks<MODE, NM_N>::value) decode_kernel(const DecArgs A, const __grid_constant__ Tab tab) {
+  pdl_enter();
   if (!header_ok(A)) return;
   const int tlog = A.team_log2;
   const int TEAM = 1 << tlog;
@@ -880,6 +883,7 @@ __global__ void __launch_bounds__(kBlock, DecMinBlocks<MODE, NM_N>::value) decod
 // Step 0: payload body = raw a; ahat = fp32(a); e = 0.
 template <typename T, int VPT, typename Tab, typename S = float>
 __global__ void __launch_bounds__(kBlock) warm_encode_kernel(const EncArgs A, const __grid_constant__ Tab tab) {
+  pdl_enter();
   const int tlog = A.team_log2;
   const int TEAM = 1 << tlog;
   const int t = threadIdx.x & (TEAM - 1);
@@ -916,6 +920,7 @@ __global__ void __launch_bounds__(kBlock) warm_encode_kernel(const EncArgs A, co
 // Step 0 receiver: ahat = fp32(body); recon = body.
 template <typename T, int VPT, typename Tab, typename S = float>
 __global__ void __launch_bounds__(kBlock) warm_decode_kernel(const DecArgs A, const __grid_constant__ Tab tab) {
+  pdl_enter();
   if (!header_ok(A)) return;
   const int tlog = A.team_log2;
   const int TEAM = 1 << tlog;
