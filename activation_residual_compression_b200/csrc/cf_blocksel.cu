@@ -367,6 +367,7 @@ __global__ void __launch_bounds__(kBsThreads) bs_pack_kernel(const T *a, const u
 template <typename T>
 __global__ void __launch_bounds__(kBsThreads) bs_warm_encode_kernel(const T *a, T *prev, uint8_t *payload, int64_t E,
                                                                      const Header hdr) {
+  pdl_enter();
   if (blockIdx.x == 0 && threadIdx.x < 16) reinterpret_cast<uint32_t *>(payload)[threadIdx.x] = hdr.w[threadIdx.x];
   T *body = reinterpret_cast<T *>(payload + kHdrBytes);
   const int64_t n8 = E / 8;
@@ -380,6 +381,7 @@ __global__ void __launch_bounds__(kBsThreads) bs_warm_encode_kernel(const T *a, 
 template <typename T>
 __global__ void __launch_bounds__(kBsThreads) bs_warm_decode_kernel(const uint8_t *payload, T *ahat, T *recon,
                                                                      int64_t E, const Header expect, int *status) {
+  pdl_enter();
   int bad = 0;
   if (threadIdx.x < 16) bad = reinterpret_cast<const uint32_t *>(payload)[threadIdx.x] != expect.w[threadIdx.x];
   if (__syncthreads_or(bad)) {
@@ -401,6 +403,7 @@ template <typename T>
 __global__ void __launch_bounds__(kBsThreads) bs_decode_kernel(const uint8_t *payload, T *ahat, T *recon, int W,
                                                                 int b, int64_t cols, int k, int K,
                                                                 const Header expect, int *status) {
+  pdl_enter();
   __shared__ int slot;
   const int i = blockIdx.x / b, y = blockIdx.x - (blockIdx.x / b) * b;
   int bad = 0;
@@ -537,7 +540,7 @@ cudaError_t blocksel_encode(const BlockselPlan &P, const void *a, void *prev, ui
     const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a);
     __nv_bfloat16 *pv = static_cast<__nv_bfloat16 *>(prev);
     if (warm) {
-      bs_warm_encode_kernel<__nv_bfloat16><<<warm_grid(E), kBsThreads, 0, st>>>(x, pv, payload, E, hdr);
+      launch_pdl(bs_warm_encode_kernel<__nv_bfloat16>, dim3(warm_grid(E)), dim3(kBsThreads), 0, st, x, pv, payload, E, hdr);
       return cudaGetLastError();
     }
     return encode_t(P, x, pv, payload, hdr, st);
@@ -545,7 +548,7 @@ cudaError_t blocksel_encode(const BlockselPlan &P, const void *a, void *prev, ui
   const float *x = static_cast<const float *>(a);
   float *pv = static_cast<float *>(prev);
   if (warm) {
-    bs_warm_encode_kernel<float><<<warm_grid(E), kBsThreads, 0, st>>>(x, pv, payload, E, hdr);
+    launch_pdl(bs_warm_encode_kernel<float>, dim3(warm_grid(E)), dim3(kBsThreads), 0, st, x, pv, payload, E, hdr);
     return cudaGetLastError();
   }
   return encode_t(P, x, pv, payload, hdr, st);
@@ -558,17 +561,20 @@ cudaError_t blocksel_decode(const BlockselPlan &P, const uint8_t *payload, void 
   if (P.dtype == CF_BF16) {
     __nv_bfloat16 *h = static_cast<__nv_bfloat16 *>(ahat), *r = static_cast<__nv_bfloat16 *>(recon);
     if (warm)
-      bs_warm_decode_kernel<__nv_bfloat16><<<warm_grid(E), kBsThreads, 0, st>>>(payload, h, r, E, expect, status);
+      launch_pdl(bs_warm_decode_kernel<__nv_bfloat16>, dim3(warm_grid(E)), dim3(kBsThreads), 0, st, payload, h, r, E,
+                 expect, status);
     else
-      bs_decode_kernel<__nv_bfloat16><<<grid, kBsThreads, 0, st>>>(payload, h, r, P.W, P.b, P.cols, P.k, P.K, expect,
-                                                                   status);
+      launch_pdl(bs_decode_kernel<__nv_bfloat16>, dim3(grid), dim3(kBsThreads), 0, st, payload, h, r, P.W, P.b, P.cols,
+                 P.k, P.K, expect, status);
     return cudaGetLastError();
   }
   float *h = static_cast<float *>(ahat), *r = static_cast<float *>(recon);
   if (warm)
-    bs_warm_decode_kernel<float><<<warm_grid(E), kBsThreads, 0, st>>>(payload, h, r, E, expect, status);
+    launch_pdl(bs_warm_decode_kernel<float>, dim3(warm_grid(E)), dim3(kBsThreads), 0, st, payload, h, r, E, expect,
+               status);
   else
-    bs_decode_kernel<float><<<grid, kBsThreads, 0, st>>>(payload, h, r, P.W, P.b, P.cols, P.k, P.K, expect, status);
+    launch_pdl(bs_decode_kernel<float>, dim3(grid), dim3(kBsThreads), 0, st, payload, h, r, P.W, P.b, P.cols, P.k, P.K,
+               expect, status);
   return cudaGetLastError();
 }
 
