@@ -270,6 +270,41 @@ def launches_per_call(mode, kw, encode):
                                                    # reconstruction
 
 
+def grouped_times(enc_j, dec_j, pay, n, stream, slot_bytes=4 << 30):
+    """Mean device time per encode and per decode over n calls, with no event
+    between two kernels: the encodes of a group run back to back, each into
+    its own payload slot, between two events; then the decodes of those
+    payloads in the same order between two more.  enc_j(j, p) encodes call j
+    into slot p, dec_j(j, p) decodes it.  Groups hold as many slots as fit
+    in slot_bytes; their times are summed."""
+    import torch
+
+    g = max(1, min(n, slot_bytes // max(1, pay.numel())))
+    slots = [torch.empty_like(pay) for _ in range(g)]
+    t_enc = t_dec = 0.0
+    j = 0
+    with torch.cuda.stream(stream):
+        while j < n:
+            m = min(g, n - j)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            # a device-side spin first, so the group's first call does not
+            # time the host's launch latency into an empty queue
+            torch.cuda._sleep(1_000_000)
+            ev[0].record(stream)
+            for u in range(m):
+                enc_j(j + u, slots[u])
+            ev[1].record(stream)
+            for u in range(m):
+                dec_j(j + u, slots[u])
+            ev[2].record(stream)
+            torch.cuda.synchronize()
+            t_enc += ev[0].elapsed_time(ev[1])
+            t_dec += ev[1].elapsed_time(ev[2])
+            j += m
+    del slots
+    return t_enc / n, t_dec / n
+
+
 def run_cf(args, rank, world, device):
     import torch
 
@@ -302,18 +337,20 @@ def run_cf(args, rank, world, device):
     torch.cuda.empty_cache()
     torch.cuda.synchronize()
 
-    def enc(c, a):
+    def enc(c, a, pay=None):
+        pay = c["pay"] if pay is None else pay
         if batched:
-            cf.cf_encode_batched(c["S"], [a[b] for b in range(B_)], c["pay"], stream)
+            cf.cf_encode_batched(c["S"], [a[b] for b in range(B_)], pay, stream)
         else:
-            cf.cf_encode(c["S"], a, c["pay"], stream)
+            cf.cf_encode(c["S"], a, pay, stream)
 
-    def dec(c, out=None):
+    def dec(c, out=None, pay=None):
         out = c["rec"] if out is None else out
+        pay = c["pay"] if pay is None else pay
         if batched:
-            cf.cf_decode_batched(c["R"], c["pay"], [out[b] for b in range(B_)], stream)
+            cf.cf_decode_batched(c["R"], pay, [out[b] for b in range(B_)], stream)
         else:
-            cf.cf_decode(c["R"], c["pay"], out, stream)
+            cf.cf_decode(c["R"], pay, out, stream)
 
     def step(i, evs=None):
         for c in codecs:
@@ -394,6 +431,21 @@ def run_cf(args, rank, world, device):
     for c in codecs:
         if cf.cf_status(c["R"], stream) != cf.CF_OK or cf.cf_status(c["S"], stream) != cf.CF_OK:
             raise RuntimeError(f"codec {c['name']} reported an error status")
+
+    # Per-kernel times without events between kernels: per codec, K encodes
+    # back to back (each into its own payload slot) between two events, then
+    # the K decodes of those payloads between two more.  Both states advance
+    # exactly as in the interleaved loops; each call still streams a state
+    # larger than L2.
+    grouped = {}
+    i0 = W_run + 2 * K
+    for c in codecs:
+        ms_e, ms_d = grouped_times(
+            lambda j, p, c=c: enc(c, c["acts"][(i0 + j) % n_inputs], p),
+            lambda j, p, c=c: dec(c, None, p), c["pay"], K, stream)
+        grouped[c["name"]] = {"enc": ms_e, "dec": ms_d}
+        if cf.cf_status(c["R"], stream) != cf.CF_OK or cf.cf_status(c["S"], stream) != cf.CF_OK:
+            raise RuntimeError(f"codec {c['name']} reported an error status in the grouped loop")
 
     # full sequences: each a new request (both states reset, the warm-up step
     # untimed) of SEQ_STEPS compressed steps, every encode and decode bracketed
@@ -493,7 +545,7 @@ def run_cf(args, rank, world, device):
     torch.cuda.empty_cache()
 
     ms_step = total_ms / K
-    stats = dict(ms_step=ms_step, ms_step_instr=instr_ms / K,
+    stats = dict(ms_step=ms_step, ms_step_instr=instr_ms / K, grouped=grouped,
                  per={m: {k: statistics.mean(v) for k, v in d.items()} for m, d in per.items()},
                  per_steps=per, e2e=e2e, clocks=clk, codecs=info, seq=seq)
     return stats
@@ -510,8 +562,9 @@ def _lr_alg_bytes(rows, cols, iters, payload, ef="explicit"):
 
 
 def run_suite(args, device):
-    """The other workloads, timed the same way (CUDA events around each
-    encode and decode on the launching stream, inputs resident)."""
+    """The other workloads, timed the same way (inputs resident; per workload
+    K encodes back to back then their K decodes, between CUDA events on the
+    launching stream, beside a loop with an event around every call)."""
     import torch
 
     import activation_residual_compression_b200 as cf
@@ -547,9 +600,24 @@ def run_suite(args, device):
         torch.cuda.synchronize()
         enc = [evs[3 * k].elapsed_time(evs[3 * k + 1]) for k in range(steps)]
         dec = [evs[3 * k + 1].elapsed_time(evs[3 * k + 2]) for k in range(steps)]
+
+        # the same number of calls grouped: encodes back to back, then their decodes
+        def genc(j, p):
+            a = acts[(warm + steps + j) % len(acts)]
+            if batched:
+                cf.cf_encode_batched(S, [a[b] for b in range(a.shape[0])], p, stream)
+            else:
+                cf.cf_encode(S, a, p, stream)
+
+        def gdec(j, p):
+            if batched:
+                cf.cf_decode_batched(R, p, recs, stream)
+            else:
+                cf.cf_decode(R, p, recs, stream)
+        g_enc, g_dec = grouped_times(genc, gdec, pay, steps, stream)
         if cf.cf_status(R, stream) != cf.CF_OK or cf.cf_status(S, stream) != cf.CF_OK:
             raise RuntimeError("suite: a codec reported an error status")
-        return statistics.mean(enc), statistics.mean(dec)
+        return g_enc, g_dec, statistics.mean(enc), statistics.mean(dec)
 
     def make(rows, cols, mode, kw, batch=1):
         base = dict(dtype=cf.CF_BF16, batch=batch, **kw)
@@ -559,11 +627,14 @@ def run_suite(args, device):
                           device="cuda")
         return S, R, pay
 
-    def entry(e_ms, d_ms, alg, act_bytes, P, **extra):
+    def entry(times, alg, act_bytes, P, **extra):
+        e_ms, d_ms, ee_ms, de_ms = times
         t = (e_ms + d_ms) / 1e3
         return {"ms_per_step": round(e_ms + d_ms, 5), "encode_ms": round(e_ms, 5), "decode_ms": round(d_ms, 5),
                 "activation_gbs": round(act_bytes / t / 1e9, 2), "roofline_frac": round(alg / t / 1e9 / peak, 4),
                 "roofline_frac_datasheet": round(alg / t / 1e9 / DATASHEET_GBS, 4),
+                "encode_ms_evented": round(ee_ms, 5), "decode_ms_evented": round(de_ms, 5),
+                "roofline_frac_evented": round(alg / ((ee_ms + de_ms) / 1e3) / 1e9 / peak, 4),
                 "payload_bytes": P, "ratio_vs_bf16": round(act_bytes / P, 2), **extra}
 
     # implicit error feedback on the FLUX-shaped stream: the form that settles to a
@@ -573,9 +644,9 @@ def run_suite(args, device):
         acts = [s.next() for _ in range(24)]
         S, R, pay = make(ROWS, COLS, mode, dict(kw, ef=EF_CODES["implicit"]))
         rec = torch.empty(ROWS, COLS, dtype=torch.bfloat16, device="cuda")
-        e_ms, d_ms = timed(S, R, pay, rec, acts, 20, 4, False)
+        tt = timed(S, R, pay, rec, acts, 20, 4, False)
         alg = encode_bytes(mode, ROWS, COLS, kw, ef="implicit") + decode_bytes(mode, ROWS, COLS, kw)
-        out[f"{_codec_name(mode, kw)}_flux_implicit"] = entry(e_ms, d_ms, alg, ROWS * COLS * 2,
+        out[f"{_codec_name(mode, kw)}_flux_implicit"] = entry(tt, alg, ROWS * COLS * 2,
                                                               cf.cf_payload_bytes(S, False))
         cf.cf_destroy(S); cf.cf_destroy(R)
         del acts
@@ -585,9 +656,9 @@ def run_suite(args, device):
     acts = [s.next() for _ in range(28)]
     S, R, pay = make(4096, 3072, "blocksel", bkw)
     rec = torch.empty(4096, 3072, dtype=torch.bfloat16, device="cuda")
-    e_ms, d_ms = timed(S, R, pay, rec, acts, 20, bkw["bs_warm"] + 2, False)
+    tt = timed(S, R, pay, rec, acts, 20, bkw["bs_warm"] + 2, False)
     alg = encode_bytes("blocksel", 4096, 3072, bkw) + decode_bytes("blocksel", 4096, 3072, bkw)
-    out["blocksel_grid64x64_3072_b8_k16"] = entry(e_ms, d_ms, alg, 4096 * 3072 * 2, cf.cf_payload_bytes(S, False),
+    out["blocksel_grid64x64_3072_b8_k16"] = entry(tt, alg, 4096 * 3072 * 2, cf.cf_payload_bytes(S, False),
                                                   launches_per_step=3)
     cf.cf_destroy(S); cf.cf_destroy(R)
     del acts
@@ -599,10 +670,10 @@ def run_suite(args, device):
         acts = [s.next() for _ in range(24)]
         S, R, pay = make(ROWS, COLS, "nm", kw)
         rec = torch.empty(ROWS, COLS, dtype=torch.bfloat16, device="cuda")
-        e_ms, d_ms = timed(S, R, pay, rec, acts, 20, 4, False)
+        tt = timed(S, R, pay, rec, acts, 20, 4, False)
         alg = encode_bytes("nm", ROWS, COLS, kw) + decode_bytes("nm", ROWS, COLS, kw)
         P = 64 + _payload_body("nm", ROWS, COLS, kw)
-        out[f"nm{n}_16_flux"] = entry(e_ms, d_ms, alg, ROWS * COLS * 2, P)
+        out[f"nm{n}_16_flux"] = entry(tt, alg, ROWS * COLS * 2, P)
         cf.cf_destroy(S); cf.cf_destroy(R)
         del acts
     # low-rank ~100x on 4096 x 3072, rank 70, INT4, 1 and 2 iterations (explicit
@@ -614,11 +685,11 @@ def run_suite(args, device):
         S, R, pay = make(lr_rows, lr_cols, "lowrank", {"rank": 70, "iters": it, "lr_int4": 1, "seed": 7,
                                                        "ef": EF_CODES[ef]})
         rec = torch.empty(lr_rows, lr_cols, dtype=torch.bfloat16, device="cuda")
-        e_ms, d_ms = timed(S, R, pay, rec, acts, 20, 5, False)
+        tt = timed(S, R, pay, rec, acts, 20, 5, False)
         P = cf.cf_payload_bytes(S, False)
         alg = _lr_alg_bytes(lr_rows, lr_cols, it, P, ef=ef)
         name = f"lowrank_r70_k{it}" + ("" if ef == "explicit" else "_implicit")
-        out[name] = entry(e_ms, d_ms, alg, lr_rows * lr_cols * 2, P,
+        out[name] = entry(tt, alg, lr_rows * lr_cols * 2, P,
                           launches_per_step=launches_per_call("lowrank", {"iters": it}, True) + 2,
                           budget_note="pages quote a ~1 ms compression budget")
         cf.cf_destroy(S); cf.cf_destroy(R)
@@ -632,10 +703,10 @@ def run_suite(args, device):
         torch.cuda.empty_cache()
         S, R, pay = make(cr, cc, "q2", {}, batch=B)
         recs = [torch.empty(cr, cc, dtype=torch.bfloat16, device="cuda") for _ in range(B)]
-        e_ms, d_ms = timed(S, R, pay, recs, acts, 6, 2, True)
+        tt = timed(S, R, pay, recs, acts, 6, 2, True)
         E = B * cr * cc
         alg = B * (encode_bytes("q2", cr, cc, {}) + decode_bytes("q2", cr, cc, {}))
-        out["cogvideox_q2_60x17550x1920"] = entry(e_ms, d_ms, alg, E * 2, cf.cf_payload_bytes(S, False),
+        out["cogvideox_q2_60x17550x1920"] = entry(tt, alg, E * 2, cf.cf_payload_bytes(S, False),
                                                   launches_per_step=2)
         cf.cf_destroy(S); cf.cf_destroy(R)
         del acts, recs
@@ -1097,7 +1168,7 @@ def main():
     value = act_bytes / (ms / 1e3) / 1e9
     peak, peak_kind = _peaks()
     c0 = st["codecs"][0]
-    enc_ms = st["per"][c0["name"]]["enc"]
+    enc_ms = st["grouped"][c0["name"]]["enc"]
     if c0["mode"] == "lowrank":
         E = R_ * C_
         enc_alg = E * (2 + 16 + 4 * c0["kw"]["iters"]) + c0["P"]
@@ -1115,12 +1186,15 @@ def main():
     achieved = enc_alg / (enc_ms / 1e3) / 1e9
     per_mode = {}
     for c in st["codecs"]:
-        pm = st["per"][c["name"]]
+        pm = st["grouped"][c["name"]]
+        pe = st["per"][c["name"]]
         step_ms = pm["enc"] + pm["dec"]
         alg = B_ * step_bytes(c["mode"], R_, C_, c["kw"], c["P"], ef=args.ef,
                               state_size=2 if args.state == "bf16" else 4)
         per_mode[c["name"]] = {"ms_per_step": round(step_ms, 5), "encode_ms": round(pm["enc"], 5),
                                "decode_ms": round(pm["dec"], 5),
+                               "encode_ms_evented": round(pe["enc"], 5), "decode_ms_evented": round(pe["dec"], 5),
+                               "roofline_frac_evented": round(alg / ((pe["enc"] + pe["dec"]) / 1e3) / 1e9 / peak, 4),
                                "activation_gbs": round(B_ * R_ * C_ * 2 / (step_ms / 1e3) / 1e9, 2),
                                "hbm_gbs": round(alg / (step_ms / 1e3) / 1e9, 1),
                                "roofline_frac": round(alg / (step_ms / 1e3) / 1e9 / peak, 4),
@@ -1133,8 +1207,11 @@ def main():
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "ms_per_step_instrumented": round(ms_instr, 5),
-        "timing": "value and ms_per_step: K steps between two CUDA events; per_mode and roofline: a second "
-                  "loop of K steps with an event around every encode and decode (ms_per_step_instrumented)",
+        "timing": "value and ms_per_step: K steps between two CUDA events; per_mode and roofline: per codec K "
+                  "encodes back to back (one payload slot each) between two events, then their K decodes between "
+                  "two more, so no event sits between two kernels; *_evented and ms_per_step_instrumented: a loop "
+                  "of K steps with an event around every encode and decode (each such event adds ~2.7 us of device "
+                  "time between two kernels)",
         "config": {**workload_config(args, wl, world),
                    "l2": f"inputs larger than L2: a fresh {in_mb:.0f} MB input per codec per step, state "
                          f"{B_ * R_ * C_ * state_bytes_per_elem(args) / 1e6:.0f} MB per codec",
