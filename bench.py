@@ -36,6 +36,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -270,17 +271,31 @@ def launches_per_call(mode, kw, encode):
                                                    # reconstruction
 
 
-def grouped_times(enc_j, dec_j, pay, n, stream, slot_bytes=4 << 30):
-    """Mean device time per encode and per decode over n calls, with no event
-    between two kernels: the encodes of a group run back to back, each into
-    its own payload slot, between two events; then the decodes of those
-    payloads in the same order between two more.  enc_j(j, p) encodes call j
-    into slot p, dec_j(j, p) decodes it.  Groups hold as many slots as fit
-    in slot_bytes; their times are summed."""
+L2_BYTES = 126e6  # B200 L2
+
+
+def n_replicas(dec_bytes):
+    """Sender/receiver pairs a grouped loop cycles through so that between two
+    calls of one pair the others move more than twice the L2: a decode's
+    state is smaller than the L2 on some workloads, and back-to-back decodes
+    of one receiver would find part of it there."""
+    return int(min(6, max(1, math.ceil(3 * L2_BYTES / max(1, dec_bytes)))))
+
+
+def grouped_times(reps, n, stream, slot_bytes=4 << 30):
+    """Mean device time per encode and per decode with no event between two
+    kernels.  reps: one (enc_j, dec_j, pay) per sender/receiver pair of the
+    same configuration; enc_j(j, p) makes the pair's call j into payload slot
+    p, dec_j(j, p) decodes it, pay is a payload buffer to copy the slot size
+    from.  Per group: the encodes (call j of every pair, then call j + 1 ...)
+    back to back between two events, each into its own slot, then the decodes
+    of those slots in the same order between two more.  Groups hold as many
+    slots as fit in slot_bytes; the mean is over n calls of every pair."""
     import torch
 
-    g = max(1, min(n, slot_bytes // max(1, pay.numel())))
-    slots = [torch.empty_like(pay) for _ in range(g)]
+    per_call = sum(p.numel() for _, _, p in reps)
+    g = max(1, min(n, slot_bytes // max(1, per_call)))
+    slots = [[torch.empty_like(p) for _ in range(g)] for _, _, p in reps]
     t_enc = t_dec = 0.0
     j = 0
     with torch.cuda.stream(stream):
@@ -292,17 +307,19 @@ def grouped_times(enc_j, dec_j, pay, n, stream, slot_bytes=4 << 30):
             torch.cuda._sleep(1_000_000)
             ev[0].record(stream)
             for u in range(m):
-                enc_j(j + u, slots[u])
+                for r, (enc_j, _, _) in enumerate(reps):
+                    enc_j(j + u, slots[r][u])
             ev[1].record(stream)
             for u in range(m):
-                dec_j(j + u, slots[u])
+                for r, (_, dec_j, _) in enumerate(reps):
+                    dec_j(j + u, slots[r][u])
             ev[2].record(stream)
             torch.cuda.synchronize()
             t_enc += ev[0].elapsed_time(ev[1])
             t_dec += ev[1].elapsed_time(ev[2])
             j += m
     del slots
-    return t_enc / n, t_dec / n
+    return t_enc / (n * len(reps)), t_dec / (n * len(reps))
 
 
 def run_cf(args, rank, world, device):
@@ -333,7 +350,7 @@ def run_cf(args, rank, world, device):
                           device="cuda")
         rec = torch.empty(B_, R_, C_, dtype=torch.bfloat16, device="cuda")
         codecs.append(dict(mode=mode, kw=kw, name=_codec_name(mode, kw), S=S, R=R, pay=pay, rec=rec, acts=acts,
-                           P=cf.cf_payload_bytes(S, False)))
+                           P=cf.cf_payload_bytes(S, False), params=base))
     torch.cuda.empty_cache()
     torch.cuda.synchronize()
 
@@ -435,17 +452,39 @@ def run_cf(args, rank, world, device):
     # Per-kernel times without events between kernels: per codec, K encodes
     # back to back (each into its own payload slot) between two events, then
     # the K decodes of those payloads between two more.  Both states advance
-    # exactly as in the interleaved loops; each call still streams a state
-    # larger than L2.
+    # exactly as in the interleaved loops.  Where a decode's state is not much
+    # larger than the L2, the loop cycles through several sender/receiver
+    # pairs of the same configuration (each warmed up like the first), so that
+    # no call finds its state left in the L2 by its own previous call.
     grouped = {}
     i0 = W_run + 2 * K
     for c in codecs:
+        zs = 2 if (args.state == "bf16" or c["mode"] == "blocksel") else 4
+        nrep = n_replicas(B_ * R_ * C_ * (2 * zs + 2))
+        reps = [c]
+        for _ in range(nrep - 1):
+            x = dict(c, S=cf.cf_create(R_, C_, cf.MODE_NAMES[c["mode"]],
+                                       cf.cf_params_init(role=cf.CF_SENDER, **c["params"])),
+                     R=cf.cf_create(R_, C_, cf.MODE_NAMES[c["mode"]],
+                                    cf.cf_params_init(role=cf.CF_RECEIVER, **c["params"])),
+                     pay=torch.empty_like(c["pay"]), rec=torch.empty_like(c["rec"]))
+            with torch.cuda.stream(stream):
+                for i in range(W_run):
+                    enc(x, x["acts"][i % n_inputs])
+                    dec(x)
+            reps.append(x)
+        torch.cuda.synchronize()
         ms_e, ms_d = grouped_times(
-            lambda j, p, c=c: enc(c, c["acts"][(i0 + j) % n_inputs], p),
-            lambda j, p, c=c: dec(c, None, p), c["pay"], K, stream)
-        grouped[c["name"]] = {"enc": ms_e, "dec": ms_d}
-        if cf.cf_status(c["R"], stream) != cf.CF_OK or cf.cf_status(c["S"], stream) != cf.CF_OK:
-            raise RuntimeError(f"codec {c['name']} reported an error status in the grouped loop")
+            [(lambda j, p, x=x: enc(x, x["acts"][(i0 + j) % n_inputs], p),
+              lambda j, p, x=x: dec(x, None, p), x["pay"]) for x in reps], K, stream)
+        grouped[c["name"]] = {"enc": ms_e, "dec": ms_d, "pairs": nrep}
+        for x in reps:
+            if cf.cf_status(x["R"], stream) != cf.CF_OK or cf.cf_status(x["S"], stream) != cf.CF_OK:
+                raise RuntimeError(f"codec {c['name']} reported an error status in the grouped loop")
+        for x in reps[1:]:
+            cf.cf_destroy(x["S"]); cf.cf_destroy(x["R"])
+        del reps
+        torch.cuda.empty_cache()
 
     # full sequences: each a new request (both states reset, the warm-up step
     # untimed) of SEQ_STEPS compressed steps, every encode and decode bracketed
@@ -574,49 +613,70 @@ def run_suite(args, device):
     stream = torch.cuda.Stream()
     out = {}
 
-    def timed(S, R, pay, recs, acts, steps, warm, batched):
-        def one(i, evs=None):
+    def timed(S, R, pay, recs, acts, steps, warm, batched, mk=None, dec_ws=0):
+        """Evented loop on (S, R), then the grouped loop over (S, R) and, when
+        mk is given, the extra pairs n_replicas(dec_ws) asks for: mk() makes
+        one (S, R, pay, recs), warmed up here and destroyed after."""
+        def one(S, R, pay, recs, i, evs=None, p=None):
             a = acts[i % len(acts)]
+            p = pay if p is None else p
             if evs is not None:
                 evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
             if batched:
-                cf.cf_encode_batched(S, [a[b] for b in range(a.shape[0])], pay, stream)
+                cf.cf_encode_batched(S, [a[b] for b in range(a.shape[0])], p, stream)
             else:
-                cf.cf_encode(S, a, pay, stream)
+                cf.cf_encode(S, a, p, stream)
             if evs is not None:
                 evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
             if batched:
-                cf.cf_decode_batched(R, pay, recs, stream)
+                cf.cf_decode_batched(R, p, recs, stream)
             else:
-                cf.cf_decode(R, pay, recs, stream)
+                cf.cf_decode(R, p, recs, stream)
             if evs is not None:
                 evs.append(torch.cuda.Event(enable_timing=True)); evs[-1].record(stream)
         with torch.cuda.stream(stream):
             for i in range(warm):
-                one(i)
+                one(S, R, pay, recs, i)
             evs = []
             for i in range(warm, warm + steps):
-                one(i, evs)
+                one(S, R, pay, recs, i, evs)
         torch.cuda.synchronize()
         enc = [evs[3 * k].elapsed_time(evs[3 * k + 1]) for k in range(steps)]
         dec = [evs[3 * k + 1].elapsed_time(evs[3 * k + 2]) for k in range(steps)]
 
         # the same number of calls grouped: encodes back to back, then their decodes
-        def genc(j, p):
-            a = acts[(warm + steps + j) % len(acts)]
-            if batched:
-                cf.cf_encode_batched(S, [a[b] for b in range(a.shape[0])], p, stream)
-            else:
-                cf.cf_encode(S, a, p, stream)
+        pairs = [(S, R, pay, recs)]
+        if mk is not None:
+            for _ in range(n_replicas(dec_ws) - 1):
+                x = mk()
+                with torch.cuda.stream(stream):
+                    for i in range(warm + steps):
+                        one(*x, i)
+                pairs.append(x)
+            torch.cuda.synchronize()
+        j0 = warm + steps
+        reps = []
+        for (S_, R_, pay_, recs_) in pairs:
+            def genc(j, p, S_=S_):
+                a = acts[(j0 + j) % len(acts)]
+                if batched:
+                    cf.cf_encode_batched(S_, [a[b] for b in range(a.shape[0])], p, stream)
+                else:
+                    cf.cf_encode(S_, a, p, stream)
 
-        def gdec(j, p):
-            if batched:
-                cf.cf_decode_batched(R, p, recs, stream)
-            else:
-                cf.cf_decode(R, p, recs, stream)
-        g_enc, g_dec = grouped_times(genc, gdec, pay, steps, stream)
-        if cf.cf_status(R, stream) != cf.CF_OK or cf.cf_status(S, stream) != cf.CF_OK:
-            raise RuntimeError("suite: a codec reported an error status")
+            def gdec(j, p, R_=R_, recs_=recs_):
+                if batched:
+                    cf.cf_decode_batched(R_, p, recs_, stream)
+                else:
+                    cf.cf_decode(R_, p, recs_, stream)
+            reps.append((genc, gdec, pay_))
+        g_enc, g_dec = grouped_times(reps, steps, stream)
+        for (S_, R_, _, _) in pairs:
+            if cf.cf_status(R_, stream) != cf.CF_OK or cf.cf_status(S_, stream) != cf.CF_OK:
+                raise RuntimeError("suite: a codec reported an error status")
+        for (S_, R_, _, _) in pairs[1:]:
+            cf.cf_destroy(S_); cf.cf_destroy(R_)
+        del pairs, reps
         return g_enc, g_dec, statistics.mean(enc), statistics.mean(dec)
 
     def make(rows, cols, mode, kw, batch=1):
@@ -644,7 +704,10 @@ def run_suite(args, device):
         acts = [s.next() for _ in range(24)]
         S, R, pay = make(ROWS, COLS, mode, dict(kw, ef=EF_CODES["implicit"]))
         rec = torch.empty(ROWS, COLS, dtype=torch.bfloat16, device="cuda")
-        tt = timed(S, R, pay, rec, acts, 20, 4, False)
+        tt = timed(S, R, pay, rec, acts, 20, 4, False,
+                   mk=lambda mode=mode, kw=kw: (*make(ROWS, COLS, mode, dict(kw, ef=EF_CODES["implicit"])),
+                                                torch.empty_like(rec)),
+                   dec_ws=ROWS * COLS * 10)
         alg = encode_bytes(mode, ROWS, COLS, kw, ef="implicit") + decode_bytes(mode, ROWS, COLS, kw)
         out[f"{_codec_name(mode, kw)}_flux_implicit"] = entry(tt, alg, ROWS * COLS * 2,
                                                               cf.cf_payload_bytes(S, False))
@@ -656,7 +719,8 @@ def run_suite(args, device):
     acts = [s.next() for _ in range(28)]
     S, R, pay = make(4096, 3072, "blocksel", bkw)
     rec = torch.empty(4096, 3072, dtype=torch.bfloat16, device="cuda")
-    tt = timed(S, R, pay, rec, acts, 20, bkw["bs_warm"] + 2, False)
+    tt = timed(S, R, pay, rec, acts, 20, bkw["bs_warm"] + 2, False,
+               mk=lambda: (*make(4096, 3072, "blocksel", bkw), torch.empty_like(rec)), dec_ws=4096 * 3072 * 6)
     alg = encode_bytes("blocksel", 4096, 3072, bkw) + decode_bytes("blocksel", 4096, 3072, bkw)
     out["blocksel_grid64x64_3072_b8_k16"] = entry(tt, alg, 4096 * 3072 * 2, cf.cf_payload_bytes(S, False),
                                                   launches_per_step=3)
@@ -670,7 +734,8 @@ def run_suite(args, device):
         acts = [s.next() for _ in range(24)]
         S, R, pay = make(ROWS, COLS, "nm", kw)
         rec = torch.empty(ROWS, COLS, dtype=torch.bfloat16, device="cuda")
-        tt = timed(S, R, pay, rec, acts, 20, 4, False)
+        tt = timed(S, R, pay, rec, acts, 20, 4, False,
+                   mk=lambda kw=kw: (*make(ROWS, COLS, "nm", kw), torch.empty_like(rec)), dec_ws=ROWS * COLS * 10)
         alg = encode_bytes("nm", ROWS, COLS, kw) + decode_bytes("nm", ROWS, COLS, kw)
         P = 64 + _payload_body("nm", ROWS, COLS, kw)
         out[f"nm{n}_16_flux"] = entry(tt, alg, ROWS * COLS * 2, P)
@@ -682,10 +747,12 @@ def run_suite(args, device):
     for it, ef in ((1, "explicit"), (2, "explicit"), (1, "implicit")):
         s = inputs.ar1("cuda", rows=lr_rows, cols=lr_cols)
         acts = [s.next() for _ in range(28)]
-        S, R, pay = make(lr_rows, lr_cols, "lowrank", {"rank": 70, "iters": it, "lr_int4": 1, "seed": 7,
-                                                       "ef": EF_CODES[ef]})
+        lkw = {"rank": 70, "iters": it, "lr_int4": 1, "seed": 7, "ef": EF_CODES[ef]}
+        S, R, pay = make(lr_rows, lr_cols, "lowrank", lkw)
         rec = torch.empty(lr_rows, lr_cols, dtype=torch.bfloat16, device="cuda")
-        tt = timed(S, R, pay, rec, acts, 20, 5, False)
+        tt = timed(S, R, pay, rec, acts, 20, 5, False,
+                   mk=lambda lkw=lkw: (*make(lr_rows, lr_cols, "lowrank", lkw), torch.empty_like(rec)),
+                   dec_ws=lr_rows * lr_cols * 10)
         P = cf.cf_payload_bytes(S, False)
         alg = _lr_alg_bytes(lr_rows, lr_cols, it, P, ef=ef)
         name = f"lowrank_r70_k{it}" + ("" if ef == "explicit" else "_implicit")
