@@ -1474,6 +1474,21 @@ __global__ void __launch_bounds__(kReconThreads, 2)
   const uint32_t tmem = tmem_base;
   ReconRows<T, SENDER> L;
   L.load(R, m0, n0, warp, lane, 0);
+  {
+    // the rows of the later update batches go to L2 meanwhile (a bulk
+    // prefetch holds no register): lane l < (NB - 1) B of warp w takes row
+    // w + 8 (B b + u) of the tile, b = 1 + l / B, u = l % B
+    constexpr int Bq = ReconRows<T, SENDER>::B, NBq = ReconRows<T, SENDER>::NB;
+    if (lane < (NBq - 1) * Bq) {
+      const int rr = warp + 8 * (Bq * (1 + lane / Bq) + lane % Bq);
+      const int64_t off = (m0 + rr) * R.cols + n0;
+      umma::prefetch_l2(R.ahat + off, kReconN * 4);
+      if constexpr (SENDER) {
+        if (R.ef_explicit) umma::prefetch_l2(R.err + off, kReconN * 4);
+        umma::prefetch_l2(static_cast<const T *>(R.a) + off, kReconN * (uint32_t)sizeof(T));
+      }
+    }
+  }
   int ok = 1;
   if (warp == 0 && lane == 0) {
     umma::mbar_arrive_expect_tx(&full, total);
