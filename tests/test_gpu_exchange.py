@@ -9,7 +9,9 @@
 * A world of one rank on NCCL, all-gather on a communication stream (the
   collective degenerates to a copy).
 The multi-rank host logic is also covered on the CPU by test_exchange.py."""
+import datetime
 import os
+import queue
 import socket
 
 import numpy as np
@@ -71,7 +73,7 @@ def _gpu_worker(rank, world, port, mode, kw, q):
         torch.cuda.set_device(0)
         os.environ["MASTER_ADDR"] = "127.0.0.1"
         os.environ["MASTER_PORT"] = str(port)
-        dist.init_process_group("gloo", rank=rank, world_size=world)
+        dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
         from activation_residual_compression_b200.exchange import SPExchange
         from test_exchange import OracleCodec
         ex = SPExchange(ROWS, COLS, mode, n_tensors=2, device="cuda:0", **kw)   # libcf codecs
@@ -114,11 +116,22 @@ def test_two_ranks_on_one_gpu_decode_peers_bit_exactly(mode, kw):
     procs = [ctx.Process(target=_gpu_worker, args=(r, 2, port, mode, kw, q)) for r in range(2)]
     for p in procs:
         p.start()
+    results = {}
     try:
-        results = dict(q.get(timeout=300) for _ in procs)
+        # the first rank that fails reports at once; its peer may then wait in
+        # a collective until its group timeout, so stop collecting there
+        while len(results) < len(procs):
+            try:
+                r, msg = q.get(timeout=300)
+            except queue.Empty:
+                pytest.fail(f"no report from a rank within 300 s; reports so far: {results}")
+            results[r] = msg
+            if msg != "ok":
+                break
     finally:
+        ok = len(results) == len(procs) and all(v == "ok" for v in results.values())
         for p in procs:
-            p.join(timeout=60)
+            p.join(timeout=60 if ok else 5)
             if p.is_alive():
                 p.kill()
     assert results == {0: "ok", 1: "ok"}, results
